@@ -1,0 +1,681 @@
+// C ABI of the DFlash hot path: argument checks, model prepacking, workspace
+// layout and the launch sequences of inject / draft / verify.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace dflash;
+
+// ============================================================== timing
+namespace dflash {
+namespace timing_detail {
+struct Pending {
+  int cls;
+  cudaEvent_t a, b;
+};
+std::mutex g_tmu;
+bool g_timing = false;
+std::vector<Pending> g_pending;
+std::vector<cudaEvent_t> g_pool;
+std::vector<std::pair<int, cudaEvent_t>> g_open;  // begin events waiting for their end
+double g_ms[TC_N];
+int64_t g_cnt[TC_N];
+
+cudaEvent_t take_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e;
+  cudaEventCreate(&e);
+  return e;
+}
+}  // namespace timing_detail
+using namespace timing_detail;
+
+void timing_begin(cudaStream_t s, int cls) {
+  if (!g_timing) return;
+  std::lock_guard<std::mutex> lk(g_tmu);
+  cudaEvent_t e = take_event();
+  cudaEventRecord(e, s);
+  g_open.push_back({cls, e});
+}
+void timing_end(cudaStream_t s, int cls) {
+  if (!g_timing) return;
+  std::lock_guard<std::mutex> lk(g_tmu);
+  if (g_open.empty()) return;
+  auto p = g_open.back();
+  g_open.pop_back();
+  cudaEvent_t e = take_event();
+  cudaEventRecord(e, s);
+  g_pending.push_back({cls, p.second, e});
+}
+}  // namespace dflash
+using namespace dflash::timing_detail;
+
+extern "C" int dflash_timing_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  g_timing = on != 0;
+  return DFLASH_OK;
+}
+
+extern "C" int dflash_timing_read(double* ms, int64_t* cnt, int n) {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  for (auto& p : g_pending) {
+    float t = 0.f;
+    if (cudaEventSynchronize(p.b) != cudaSuccess) return DFLASH_ECUDA;
+    cudaEventElapsedTime(&t, p.a, p.b);
+    g_ms[p.cls] += t;
+    g_cnt[p.cls] += 1;
+    g_pool.push_back(p.a);
+    g_pool.push_back(p.b);
+  }
+  g_pending.clear();
+  for (int i = 0; i < n && i < TC_N; ++i) {
+    if (ms) ms[i] = g_ms[i];
+    if (cnt) cnt[i] = g_cnt[i];
+    g_ms[i] = 0.0;
+    g_cnt[i] = 0;
+  }
+  return DFLASH_OK;
+}
+
+// ============================================================== model
+struct LayerPack {
+  void* Wqkv = nullptr;  // [qkv_out, d]
+  void* Wo = nullptr;    // [d, nq*hd]
+  void* Wgu = nullptr;   // [2I, d]
+  void* Wd = nullptr;    // [d, I]
+  float* g_in = nullptr;
+  float* g_post = nullptr;
+  WeightMap mqkv, mo, mgu, md;
+};
+
+struct dflash_model {
+  dflash_config cfg;
+  int device = 0;
+  size_t esz = 2;
+  void* emb = nullptr;
+  void* W_fc = nullptr;
+  void* W_kv = nullptr;  // [L*2*nkv*hd, d]: for each layer [Wk; Wv]
+  void* W_lm = nullptr;
+  float* g_ctx = nullptr;
+  float* g_final = nullptr;
+  float* rope_cos = nullptr;
+  float* rope_sin = nullptr;
+  std::vector<LayerPack> layers;
+  WeightMap mfc, mkv, mlm;
+  std::vector<void*> allocs;
+};
+
+namespace {
+
+template <typename T>
+__global__ void gain_to_f32_kernel(const T* __restrict__ g, float* __restrict__ out, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = to_f(g[i]);
+}
+
+// cos/sin of p * base^(-2i/hd), evaluated in double precision, stored fp32.
+__global__ void rope_table_kernel(float* __restrict__ cs, float* __restrict__ sn, int max_pos,
+                                  int half, double base) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)max_pos * half) return;
+  const int p = (int)(idx / half), i = (int)(idx % half);
+  const double theta = pow(base, -2.0 * (double)i / (2.0 * half));
+  const double ang = (double)p * theta;
+  cs[idx] = (float)cos(ang);
+  sn[idx] = (float)sin(ang);
+}
+
+void* dmalloc(dflash_model* m, size_t bytes) {
+  void* p = nullptr;
+  if (cudaMalloc(&p, bytes) != cudaSuccess) return nullptr;
+  m->allocs.push_back(p);
+  return p;
+}
+
+void free_model(dflash_model* m) {
+  for (void* p : m->allocs) cudaFree(p);
+  m->allocs.clear();
+}
+
+bool copy_rows(void* dst, const void* src, size_t bytes) {
+  return src != nullptr && cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToDevice) == cudaSuccess;
+}
+
+float* gain_copy(dflash_model* m, const void* g) {
+  const int d = m->cfg.d;
+  float* out = static_cast<float*>(dmalloc(m, sizeof(float) * d));
+  if (!out || !g) return nullptr;
+  if (m->cfg.dtype == DFLASH_BF16)
+    gain_to_f32_kernel<<<(d + 255) / 256, 256>>>(static_cast<const __nv_bfloat16*>(g), out, d);
+  else
+    gain_to_f32_kernel<<<(d + 255) / 256, 256>>>(static_cast<const float*>(g), out, d);
+  return out;
+}
+
+bool config_ok(const dflash_config& c) {
+  if (c.dtype != DFLASH_F32 && c.dtype != DFLASH_BF16) return false;
+  if (c.H_t <= 0 || c.n_tap < 1 || c.n_tap > kMaxSeg || c.n_layers < 1 || c.d <= 0) return false;
+  if (c.n_q <= 0 || c.n_kv <= 0 || c.n_q % c.n_kv) return false;
+  if (c.head_dim <= 0 || c.head_dim % 2 || c.head_dim > 256 || c.inter <= 0) return false;
+  if (c.vocab < 2 || c.mask_id < 0 || c.mask_id >= c.vocab || c.max_pos < 1) return false;
+  if (!(c.eps >= 0.f) || !(c.rope_base > 0.0)) return false;
+  if (c.d > 4096) return false;  // row kernels hold a row in registers (16 per thread)
+  return true;
+}
+
+bool config_supported(const dflash_config& c) {
+  if (c.head_dim != 64 && c.head_dim != 128) return false;
+  if (c.dtype == DFLASH_BF16) {
+    if (c.d % 64 || c.H_t % 64 || c.inter % 64 || (c.n_q * c.head_dim) % 64) return false;
+  } else {
+    const int kmax = std::max(std::max(c.n_tap * c.H_t, c.d), std::max(c.inter, c.n_q * c.head_dim));
+    if (kmax > 12288) return false;  // SIMT GEMM keeps one token row in shared memory
+  }
+  return true;
+}
+
+int qkv_out(const dflash_config& c) { return (c.n_q + 2 * c.n_kv) * c.head_dim; }
+
+// ---------------------------------------------------------------- workspace layout
+constexpr size_t kHeader = 256;
+constexpr int kMaxChunks = 64;
+constexpr int kAttnRows = 64;
+constexpr int kInjectChunkRows = 16384;
+constexpr int kMaxSplits = 16;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct DraftLayout {
+  size_t tokens, zrow, lm_rows, cstep, req_valid, lm_tok, lm_conf, x, h, q, kb, vb, o, act, part,
+      attn_o, attn_ml, stats, logits, end;
+  size_t part_elems;
+};
+
+struct InjectLayout {
+  size_t c, part, end;
+  size_t part_elems;
+  int chunk_rows;
+};
+
+int draft_part_cols(const dflash_config& c) {
+  return std::max(std::max(qkv_out(c), c.d), 2 * c.inter);
+}
+
+DraftLayout draft_layout(const dflash_config& c, int batch, int B) {
+  DraftLayout L{};
+  const size_t M = (size_t)batch * B;
+  const size_t esz = c.dtype == DFLASH_BF16 ? 2 : 4;
+  const int n_vt = (c.vocab + kTileN - 1) / kTileN;
+  size_t off = kHeader;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.tokens = take(4 * M);
+  L.zrow = take(4 * M);
+  L.lm_rows = take(4 * M);
+  L.cstep = take(4 * M);
+  L.req_valid = take(4 * (size_t)batch);
+  L.lm_tok = take(4 * M);
+  L.lm_conf = take(4 * M);
+  L.x = take(4 * M * c.d);
+  L.h = take(esz * M * std::max(c.d, c.n_q * c.head_dim));
+  L.q = take(esz * M * c.n_q * c.head_dim);
+  L.kb = take(esz * M * c.n_kv * c.head_dim);
+  L.vb = take(esz * M * c.n_kv * c.head_dim);
+  L.o = take(esz * M * c.n_q * c.head_dim);
+  L.act = take(esz * M * c.inter);
+  // split-K partials: room for 4 splits of the widest projection
+  L.part_elems = 4 * M * (size_t)draft_part_cols(c);
+  L.part = take(4 * L.part_elems);
+  const size_t arows = (size_t)batch * c.n_kv * kMaxChunks * kAttnRows;
+  L.attn_o = take(4 * arows * c.head_dim);
+  L.attn_ml = take(8 * arows);
+  L.stats = take(sizeof(LmStat) * M * n_vt);
+  L.logits = c.dtype == DFLASH_F32 ? take(4 * M * (size_t)c.vocab) : off;
+  L.end = off;
+  return L;
+}
+
+InjectLayout inject_layout(const dflash_config& c, int max_rows) {
+  InjectLayout L{};
+  const size_t esz = c.dtype == DFLASH_BF16 ? 2 : 4;
+  L.chunk_rows = std::min(std::max(max_rows, 1), kInjectChunkRows);
+  const size_t n = L.chunk_rows;
+  const size_t ncol = std::max((size_t)c.d, (size_t)c.n_layers * 2 * c.n_kv * c.head_dim);
+  size_t off = kHeader;
+  L.c = off;
+  off = align256(off + esz * n * c.d);
+  // small row counts may split K up to kMaxSplits ways
+  L.part_elems = (n <= 256 ? (size_t)kMaxSplits : 1) * n * ncol;
+  L.part = off;
+  off = align256(off + 4 * L.part_elems);
+  L.end = off;
+  return L;
+}
+
+size_t verify_bytes(int batch, int B, int V) {
+  const int rows = batch * B;
+  return kHeader + align256((size_t)rows * verify_chunks(rows, V) * 8);
+}
+
+int32_t* err_word(void* ws) { return static_cast<int32_t*>(ws); }
+
+template <typename P>
+P* at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int cuda_status() { return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA; }
+
+// Split count for a draft/inject GEMM: the picker's choice, lowered until the
+// partials fit the workspace; always a count gemm_tc runs unchanged.
+int splits_for(int M, int N, int K, size_t cap_elems) {
+  int s = gemm_pick_splits(M, N, K, kMaxSplits);
+  const size_t fit = std::max<size_t>(1, cap_elems / ((size_t)M * N));
+  while ((size_t)s > fit) s = gemm_effective_splits(K, s - 1);
+  return s;
+}
+
+}  // namespace
+
+extern "C" const char* dflash_status_str(int st) {
+  switch (st) {
+    case DFLASH_OK: return "ok";
+    case DFLASH_EINVAL: return "invalid argument";
+    case DFLASH_EUNSUPPORTED: return "unsupported shape or dtype";
+    case DFLASH_ECUDA: return "CUDA error";
+    case DFLASH_ENOMEM: return "out of device memory";
+    case DFLASH_EWORKSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weights* w,
+                                   dflash_model** out) {
+  if (!cfg || !w || !out || !w->layers) return DFLASH_EINVAL;
+  *out = nullptr;
+  if (!config_ok(*cfg)) return DFLASH_EINVAL;
+  if (!config_supported(*cfg)) return DFLASH_EUNSUPPORTED;
+  const dflash_config& c = *cfg;
+  dflash_model* m = new dflash_model();
+  m->cfg = c;
+  cudaGetDevice(&m->device);
+  m->esz = c.dtype == DFLASH_BF16 ? 2 : 4;
+  const size_t e = m->esz;
+  const size_t d = c.d, hd = c.head_dim, nq = c.n_q, nkv = c.n_kv, I = c.inter, V = c.vocab;
+  auto fail = [&](int code) {
+    free_model(m);
+    delete m;
+    return code;
+  };
+  m->emb = dmalloc(m, e * V * d);
+  m->W_fc = dmalloc(m, e * d * c.n_tap * c.H_t);
+  m->W_lm = dmalloc(m, e * V * d);
+  m->W_kv = dmalloc(m, e * c.n_layers * 2 * nkv * hd * d);
+  if (!m->emb || !m->W_fc || !m->W_lm || !m->W_kv) return fail(DFLASH_ENOMEM);
+  if (!copy_rows(m->emb, w->emb, e * V * d) ||
+      !copy_rows(m->W_fc, w->W_fc, e * d * c.n_tap * c.H_t) ||
+      !copy_rows(m->W_lm, w->W_lm, e * V * d))
+    return fail(DFLASH_EINVAL);
+  m->g_ctx = gain_copy(m, w->g_ctx);
+  m->g_final = gain_copy(m, w->g_final);
+  if (!m->g_ctx || !m->g_final) return fail(w->g_ctx && w->g_final ? DFLASH_ENOMEM : DFLASH_EINVAL);
+  m->layers.resize(c.n_layers);
+  const size_t kvrows = nkv * hd;
+  for (int l = 0; l < c.n_layers; ++l) {
+    const dflash_layer_weights& lw = w->layers[l];
+    LayerPack& P = m->layers[l];
+    P.Wqkv = dmalloc(m, e * qkv_out(c) * d);
+    P.Wo = dmalloc(m, e * d * nq * hd);
+    P.Wgu = dmalloc(m, e * 2 * I * d);
+    P.Wd = dmalloc(m, e * d * I);
+    if (!P.Wqkv || !P.Wo || !P.Wgu || !P.Wd) return fail(DFLASH_ENOMEM);
+    uint8_t* qkv = static_cast<uint8_t*>(P.Wqkv);
+    uint8_t* gu = static_cast<uint8_t*>(P.Wgu);
+    uint8_t* kv = static_cast<uint8_t*>(m->W_kv) + (size_t)l * 2 * kvrows * d * e;
+    if (!copy_rows(qkv, lw.Wq, e * nq * hd * d) ||
+        !copy_rows(qkv + e * nq * hd * d, lw.Wk, e * kvrows * d) ||
+        !copy_rows(qkv + e * (nq * hd + kvrows) * d, lw.Wv, e * kvrows * d) ||
+        !copy_rows(P.Wo, lw.Wo, e * d * nq * hd) || !copy_rows(gu, lw.Wg, e * I * d) ||
+        !copy_rows(gu + e * I * d, lw.Wu, e * I * d) || !copy_rows(P.Wd, lw.Wd, e * d * I) ||
+        !copy_rows(kv, lw.Wk, e * kvrows * d) || !copy_rows(kv + e * kvrows * d, lw.Wv, e * kvrows * d))
+      return fail(DFLASH_EINVAL);
+    P.g_in = gain_copy(m, lw.g_in);
+    P.g_post = gain_copy(m, lw.g_post);
+    if (!P.g_in || !P.g_post) return fail(DFLASH_EINVAL);
+  }
+  const int half = c.head_dim / 2;
+  m->rope_cos = static_cast<float*>(dmalloc(m, sizeof(float) * (size_t)c.max_pos * half));
+  m->rope_sin = static_cast<float*>(dmalloc(m, sizeof(float) * (size_t)c.max_pos * half));
+  if (!m->rope_cos || !m->rope_sin) return fail(DFLASH_ENOMEM);
+  {
+    const int64_t n = (int64_t)c.max_pos * half;
+    rope_table_kernel<<<(unsigned)((n + 255) / 256), 256>>>(m->rope_cos, m->rope_sin, c.max_pos,
+                                                             half, c.rope_base);
+  }
+  if (c.dtype == DFLASH_BF16) {
+    bool ok = encode_weight_map(m->mfc, m->W_fc, c.d, c.n_tap * c.H_t) &&
+              encode_weight_map(m->mkv, m->W_kv, c.n_layers * 2 * kvrows, c.d) &&
+              encode_weight_map(m->mlm, m->W_lm, c.vocab, c.d);
+    for (int l = 0; l < c.n_layers && ok; ++l) {
+      LayerPack& P = m->layers[l];
+      ok = encode_weight_map(P.mqkv, P.Wqkv, qkv_out(c), c.d) &&
+           encode_weight_map(P.mo, P.Wo, c.d, c.n_q * c.head_dim) &&
+           encode_weight_map(P.mgu, P.Wgu, 2 * c.inter, c.d) &&
+           encode_weight_map(P.md, P.Wd, c.d, c.inter);
+    }
+    if (!ok) return fail(DFLASH_ECUDA);
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess || cudaGetLastError() != cudaSuccess)
+    return fail(DFLASH_ECUDA);
+  *out = m;
+  return DFLASH_OK;
+}
+
+extern "C" int dflash_model_destroy(dflash_model* m) {
+  if (!m) return DFLASH_OK;
+  cudaDeviceSynchronize();
+  free_model(m);
+  delete m;
+  return DFLASH_OK;
+}
+
+extern "C" size_t dflash_workspace_size(const dflash_model* m, int max_batch, int B,
+                                        int max_inject_rows) {
+  if (!m || max_batch < 0 || B < 0 || max_inject_rows < 0) return 0;
+  size_t s = kHeader;
+  if (max_batch > 0 && B > 0) {
+    s = std::max(s, draft_layout(m->cfg, max_batch, B).end);
+    s = std::max(s, verify_bytes(max_batch, B, m->cfg.vocab));
+  }
+  if (max_inject_rows > 0) s = std::max(s, inject_layout(m->cfg, max_inject_rows).end);
+  return s;
+}
+
+extern "C" size_t dflash_verify_workspace_size(int batch, int B, int V) {
+  if (batch < 0 || B < 0 || V < 1) return 0;
+  if (batch == 0 || B == 0) return kHeader;
+  return verify_bytes(batch, B, V);
+}
+
+extern "C" int dflash_workspace_init(void* ws, size_t bytes, void* stream) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return DFLASH_EINVAL;
+  return cudaMemsetAsync(ws, 0, bytes, (cudaStream_t)stream) == cudaSuccess ? DFLASH_OK
+                                                                           : DFLASH_ECUDA;
+}
+
+extern "C" int dflash_get_error(void* ws, void* stream, int32_t* bits) {
+  if (!ws || !bits) return DFLASH_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return DFLASH_ECUDA;
+  if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return DFLASH_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DFLASH_ECUDA;
+  *bits = h;
+  return DFLASH_OK;
+}
+
+// ============================================================== inject
+extern "C" int dflash_inject_kv(const dflash_model* m, const void* const* taps,
+                                const int32_t* cu_rows, const int32_t* start_pos, int batch,
+                                int n_rows, void* k_cache, void* v_cache, int cache_cap, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (!m || batch < 1 || n_rows < 0 || cache_cap < 1) return DFLASH_EINVAL;
+  if (n_rows == 0) return DFLASH_OK;
+  const dflash_config& c = m->cfg;
+  if (!taps || !cu_rows || !start_pos || !k_cache || !v_cache || !ws) return DFLASH_EINVAL;
+  for (int t = 0; t < c.n_tap; ++t)
+    if (!taps[t] || !aligned16(taps[t])) return DFLASH_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return DFLASH_EINVAL;
+  const InjectLayout L = inject_layout(c, n_rows);
+  if (ws_bytes < L.end) return DFLASH_EWORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t* err = err_word(ws);
+  const int kvN = c.n_layers * 2 * c.n_kv * c.head_dim;
+  const size_t e = m->esz;
+  for (int r0 = 0; r0 < n_rows; r0 += L.chunk_rows) {
+    const int n = std::min(L.chunk_rows, n_rows - r0);
+    const void* seg[kMaxSeg];
+    for (int t = 0; t < c.n_tap; ++t)
+      seg[t] = static_cast<const uint8_t*>(taps[t]) + (size_t)r0 * c.H_t * e;
+    float* part = at<float>(ws, L.part);
+    void* cbuf = at<void>(ws, L.c);
+    int st;
+    if (c.dtype == DFLASH_BF16) {
+      const int s1 = splits_for(n, c.d, c.n_tap * c.H_t, L.part_elems);
+      GemmOut o;
+      o.part = part;
+      st = gemm_tc(m->mfc, seg, c.n_tap, c.H_t, c.H_t, n, s1, EPI_PARTIAL, o, err, s);
+      if (st) return st;
+      launch_ctx_norm<__nv_bfloat16>(part, s1, n, c.d, m->g_ctx,
+                                     static_cast<__nv_bfloat16*>(cbuf), c.eps, s);
+      const int s2 = splits_for(n, kvN, c.d, L.part_elems);
+      const void* cseg[1] = {cbuf};
+      st = gemm_tc(m->mkv, cseg, 1, c.d, c.d, n, s2, EPI_PARTIAL, o, err, s);
+      if (st) return st;
+      launch_kv_scatter<__nv_bfloat16>(part, s2, n, r0, c.n_layers, c.n_kv, c.head_dim, cu_rows,
+                                       start_pos, batch, cache_cap, m->rope_cos, m->rope_sin,
+                                       c.max_pos, static_cast<__nv_bfloat16*>(k_cache),
+                                       static_cast<__nv_bfloat16*>(v_cache), err, s);
+    } else {
+      const float* fseg[kMaxSeg];
+      for (int t = 0; t < c.n_tap; ++t) fseg[t] = static_cast<const float*>(seg[t]);
+      gemm_simt_f32(static_cast<const float*>(m->W_fc), c.d, c.n_tap * c.H_t, fseg, c.n_tap,
+                    c.H_t, n, part, s);
+      launch_ctx_norm<float>(part, 1, n, c.d, m->g_ctx, static_cast<float*>(cbuf), c.eps, s);
+      const float* cseg[1] = {static_cast<const float*>(cbuf)};
+      gemm_simt_f32(static_cast<const float*>(m->W_kv), kvN, c.d, cseg, 1, c.d, n, part, s);
+      launch_kv_scatter<float>(part, 1, n, r0, c.n_layers, c.n_kv, c.head_dim, cu_rows,
+                               start_pos, batch, cache_cap, m->rope_cos, m->rope_sin, c.max_pos,
+                               static_cast<float*>(k_cache), static_cast<float*>(v_cache), err, s);
+    }
+    if ((st = cuda_status())) return st;
+  }
+  return DFLASH_OK;
+}
+
+// ============================================================== draft
+namespace {
+
+template <typename T>
+int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_len,
+               const void* k_cache, const void* v_cache, int cap, int batch, int B, int n_steps,
+               int32_t* draft_tokens, int32_t* commit_step, float* logits_dbg, void* ws,
+               cudaStream_t s) {
+  const dflash_config& c = m->cfg;
+  const DraftLayout L = draft_layout(c, batch, B);
+  const int M = batch * B;
+  const int hd = c.head_dim, nq = c.n_q, nkv = c.n_kv;
+  int32_t* err = err_word(ws);
+  int32_t* tokens = at<int32_t>(ws, L.tokens);
+  int32_t* zrow = at<int32_t>(ws, L.zrow);
+  int32_t* lm_rows = at<int32_t>(ws, L.lm_rows);
+  int32_t* cstep = at<int32_t>(ws, L.cstep);
+  int32_t* valid = at<int32_t>(ws, L.req_valid);
+  int32_t* lm_tok = at<int32_t>(ws, L.lm_tok);
+  float* lm_conf = at<float>(ws, L.lm_conf);
+  float* x = at<float>(ws, L.x);
+  T* h = at<T>(ws, L.h);
+  T* q = at<T>(ws, L.q);
+  T* kb = at<T>(ws, L.kb);
+  T* vb = at<T>(ws, L.vb);
+  T* o = at<T>(ws, L.o);
+  T* act = at<T>(ws, L.act);
+  float* part = at<float>(ws, L.part);
+  float* attn_o = at<float>(ws, L.attn_o);
+  float* attn_ml = at<float>(ws, L.attn_ml);
+  LmStat* stats = at<LmStat>(ws, L.stats);
+  const T* kc = static_cast<const T*>(k_cache);
+  const T* vc = static_cast<const T*>(v_cache);
+  const int n_vt = (c.vocab + kTileN - 1) / kTileN;
+  const bool bf16 = c.dtype == DFLASH_BF16;
+
+  int chunk = (cap + B + kMaxChunks - 1) / kMaxChunks;
+  chunk = std::max(256, (chunk + 31) / 32 * 32);
+  const int n_chunks = (cap + B + chunk - 1) / chunk;
+
+  launch_draft_init(anchor, ctx_len, batch, B, c.vocab, c.mask_id, cap, tokens, zrow, lm_rows,
+                    cstep, valid, err, s);
+  auto gemm = [&](const WeightMap& W, const void* wptr, int N, int K, const T* X, float* out,
+                  size_t cap_elems, int* splits_out) -> int {
+    if (bf16) {
+      const int sp = splits_for(M, N, K, cap_elems);
+      *splits_out = sp;
+      GemmOut go;
+      go.part = out;
+      const void* seg[1] = {X};
+      return gemm_tc(W, seg, 1, K, K, M, sp, EPI_PARTIAL, go, err, s);
+    }
+    *splits_out = 1;
+    const float* seg[1] = {reinterpret_cast<const float*>(X)};
+    gemm_simt_f32(static_cast<const float*>(wptr), N, K, seg, 1, K, M, out, s);
+    return DFLASH_OK;
+  };
+
+  int rem = B - 1;
+  int st = DFLASH_OK;
+  for (int t = 0; t < n_steps; ++t) {
+    const int k = (rem + (n_steps - t) - 1) / (n_steps - t);
+    launch_embed_norm<T>(tokens, static_cast<const T*>(m->emb), m->layers[0].g_in, x, h, M, c.d,
+                         c.eps, s);
+    for (int l = 0; l < c.n_layers; ++l) {
+      const LayerPack& P = m->layers[l];
+      int sp = 1;
+      if ((st = gemm(P.mqkv, P.Wqkv, qkv_out(c), c.d, h, part, L.part_elems, &sp))) return st;
+      launch_qkv_post<T>(part, sp, M, B, ctx_len, valid, nq, nkv, hd, m->rope_cos, m->rope_sin,
+                         q, kb, vb, s);
+      if ((st = launch_block_attention<T>(q, kb, vb, kc, vc, l, batch, cap, ctx_len, valid, B, nq,
+                                          nkv, hd, attn_o, attn_ml, n_chunks, chunk, o, s)))
+        return st;
+      if ((st = gemm(P.mo, P.Wo, c.d, nq * hd, o, part, L.part_elems, &sp))) return st;
+      launch_residual_norm<T>(part, sp, M, c.d, x, P.g_post, h, nullptr, c.eps, s);
+      if ((st = gemm(P.mgu, P.Wgu, 2 * c.inter, c.d, h, part, L.part_elems, &sp))) return st;
+      launch_swiglu<T>(part, sp, M, c.inter, act, s);
+      if ((st = gemm(P.md, P.Wd, c.d, c.inter, act, part, L.part_elems, &sp))) return st;
+      if (l + 1 < c.n_layers)
+        launch_residual_norm<T>(part, sp, M, c.d, x, m->layers[l + 1].g_in, h, nullptr, c.eps, s);
+      else
+        launch_residual_norm<T>(part, sp, M, c.d, x, m->g_final, h, zrow, c.eps, s);
+    }
+    // LM head over the still-masked rows (compact, request-major)
+    const int rows = batch * rem;
+    float* dbg = logits_dbg ? logits_dbg + (size_t)t * M * c.vocab : nullptr;
+    if (bf16) {
+      GemmOut go;
+      go.stats = stats;
+      go.dbg = dbg;
+      go.dbg_rows = lm_rows;
+      go.dbg_ld = c.vocab;
+      const void* seg[1] = {h};
+      if ((st = gemm_tc(m->mlm, seg, 1, c.d, c.d, rows, 1, EPI_LMHEAD, go, err, s))) return st;
+    } else {
+      float* logits = at<float>(ws, L.logits);
+      const float* seg[1] = {reinterpret_cast<const float*>(h)};
+      gemm_simt_f32(static_cast<const float*>(m->W_lm), c.vocab, c.d, seg, 1, c.d, rows, logits,
+                    s);
+      launch_lm_stats_from_logits(logits, rows, c.vocab, stats, dbg, lm_rows, c.vocab, s);
+    }
+    launch_lm_reduce(stats, n_vt, rows, lm_tok, lm_conf, s);
+    launch_commit(lm_tok, lm_conf, batch, B, rem, k, t, tokens, zrow, lm_rows, cstep, s);
+    rem -= k;
+  }
+  launch_draft_finish(tokens, cstep, valid, batch, B, draft_tokens, commit_step, s);
+  return cuda_status();
+}
+
+}  // namespace
+
+extern "C" int dflash_draft_block(const dflash_model* m, const int32_t* anchor,
+                                  const int32_t* ctx_len, const void* k_cache, const void* v_cache,
+                                  int cache_cap, int batch, int B, int n_steps,
+                                  int32_t* draft_tokens, int32_t* commit_step, float* logits_dbg,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  if (!m || batch < 0 || B < 2 || B > 16 || n_steps < 1 || n_steps > B - 1 || cache_cap < 1)
+    return DFLASH_EINVAL;
+  if (batch == 0) return DFLASH_OK;
+  const dflash_config& c = m->cfg;
+  if (!anchor || !ctx_len || !k_cache || !v_cache || !draft_tokens || !ws) return DFLASH_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return DFLASH_EINVAL;
+  if (cache_cap > c.max_pos) return DFLASH_EINVAL;
+  if (B * (c.n_q / c.n_kv) > kAttnRows) return DFLASH_EUNSUPPORTED;
+  if ((size_t)batch * B > 65535) return DFLASH_EUNSUPPORTED;
+  if (ws_bytes < draft_layout(c, batch, B).end) return DFLASH_EWORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (c.dtype == DFLASH_BF16)
+    return draft_impl<__nv_bfloat16>(m, anchor, ctx_len, k_cache, v_cache, cache_cap, batch, B,
+                                     n_steps, draft_tokens, commit_step, logits_dbg, ws, s);
+  return draft_impl<float>(m, anchor, ctx_len, k_cache, v_cache, cache_cap, batch, B, n_steps,
+                           draft_tokens, commit_step, logits_dbg, ws, s);
+}
+
+// ============================================================== verify
+extern "C" int dflash_verify(const void* target_logits, int logits_dtype,
+                             const int32_t* draft_tokens, int batch, int B, int V,
+                             int32_t* out_tokens, int32_t* out_len, int out_cap, int32_t* seq_lens,
+                             int32_t* accept_len, int32_t* next_anchor, void* ws, size_t ws_bytes,
+                             void* stream) {
+  if (batch < 0 || B < 2 || B > 32 || V < 1 || out_cap < 1) return DFLASH_EINVAL;
+  if (logits_dtype != DFLASH_BF16 && logits_dtype != DFLASH_F32) return DFLASH_EINVAL;
+  if (batch == 0) return DFLASH_OK;
+  if (!target_logits || !draft_tokens || !out_tokens || !out_len || !seq_lens || !accept_len ||
+      !next_anchor || !ws)
+    return DFLASH_EINVAL;
+  if (!aligned16(target_logits) || (reinterpret_cast<uintptr_t>(ws) & 255)) return DFLASH_EINVAL;
+  if ((int64_t)batch * B > 65535) return DFLASH_EUNSUPPORTED;
+  if (ws_bytes < verify_bytes(batch, B, V)) return DFLASH_EWORKSPACE;
+  const int chunks = verify_chunks(batch * B, V);
+  return launch_verify(target_logits, logits_dtype, draft_tokens, batch, B, V, out_tokens,
+                       out_len, out_cap, seq_lens, accept_len, next_anchor,
+                       at<void>(ws, kHeader), chunks, err_word(ws), (cudaStream_t)stream);
+}
+
+// ============================================================== test hooks (dflash_debug.h)
+#include "../../include/dflash_debug.h"
+
+extern "C" int dflash_debug_gemm_bf16(const void* W, int N, int K, const void* X, int M,
+                                      int splits, float* out, int* splits_used, void* err_ws,
+                                      void* stream) {
+  if (!W || !X || !out || !err_ws || N < 1 || K < 64 || K % 64 || M < 1) return DFLASH_EINVAL;
+  if (!aligned16(W) || !aligned16(X)) return DFLASH_EINVAL;
+  WeightMap wm;
+  if (!encode_weight_map(wm, W, N, K)) return DFLASH_ECUDA;
+  splits = gemm_effective_splits(K, splits);
+  if (splits_used) *splits_used = splits;
+  GemmOut o;
+  o.part = out;
+  const void* seg[1] = {X};
+  return gemm_tc(wm, seg, 1, K, K, M, splits, EPI_PARTIAL, o, err_word(err_ws),
+                 (cudaStream_t)stream);
+}
+
+extern "C" int dflash_debug_lmhead_bf16(const void* W, int N, int K, const void* X, int M,
+                                        void* stats, float* logits, void* err_ws, void* stream) {
+  if (!W || !X || !stats || !err_ws || N < 1 || K < 64 || K % 64 || M < 1) return DFLASH_EINVAL;
+  if (!aligned16(W) || !aligned16(X)) return DFLASH_EINVAL;
+  WeightMap wm;
+  if (!encode_weight_map(wm, W, N, K)) return DFLASH_ECUDA;
+  GemmOut o;
+  o.stats = static_cast<LmStat*>(stats);
+  o.dbg = logits;
+  o.dbg_rows = nullptr;
+  o.dbg_ld = N;
+  const void* seg[1] = {X};
+  return gemm_tc(wm, seg, 1, K, K, M, 1, EPI_LMHEAD, o, err_word(err_ws), (cudaStream_t)stream);
+}

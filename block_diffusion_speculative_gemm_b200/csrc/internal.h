@@ -1,0 +1,127 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/dflash.h"
+
+namespace dflash {
+
+// ---------------------------------------------------------------- timing
+enum TimingClass { TC_GEMM = 0, TC_ATTN = 1, TC_ROW = 2, TC_VERIFY = 3, TC_LMHEAD = 4, TC_N = 5 };
+void timing_begin(cudaStream_t s, int cls);
+void timing_end(cudaStream_t s, int cls);
+struct TimedScope {
+  cudaStream_t s;
+  int cls;
+  TimedScope(cudaStream_t s_, int c) : s(s_), cls(c) { timing_begin(s, cls); }
+  ~TimedScope() { timing_end(s, cls); }
+};
+
+// ---------------------------------------------------------------- tcgen05 GEMM
+constexpr int kTileN = 128;    // weight rows per CTA tile (UMMA M)
+constexpr int kTileK = 64;     // K elements per pipeline stage
+constexpr int kMaxSeg = 8;     // K segments of the activation operand
+constexpr int kMaxBN = 256;    // largest token tile (UMMA N)
+
+struct LmStat {                // per (token row, 128-wide vocab tile)
+  float max;                   // largest logit in the tile
+  int32_t idx;                 // its vocabulary id (lowest on ties)
+  float sumexp;                // sum over the tile of exp(logit - max)
+  float pad;
+};
+
+enum GemmEpi { EPI_PARTIAL = 0, EPI_LMHEAD = 1 };
+
+struct GemmOut {
+  float* part = nullptr;          // EPI_PARTIAL: [splits][M][N] fp32
+  LmStat* stats = nullptr;        // EPI_LMHEAD: [M][ceil(N/128)]
+  float* dbg = nullptr;           // EPI_LMHEAD, optional: logits rows
+  const int32_t* dbg_rows = nullptr;  // token row -> dbg row
+  int64_t dbg_ld = 0;             // dbg row stride (elements)
+};
+
+// A weight operand prepared once: tensor map over [N, K] bf16 rows.
+struct WeightMap {
+  CUtensorMap map;
+  const void* ptr = nullptr;
+  int N = 0, K = 0;
+};
+
+bool encode_weight_map(WeightMap& w, const void* ptr, int N, int K);
+
+// Y = X * W^T for bf16 X [M, K] (given as n_seg K-segments of seg_k columns,
+// each [M, seg_k] with row stride ld_seg elements) and W [N, K].
+int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, int ld_seg, int M,
+            int splits, int epi, const GemmOut& out, int32_t* err, cudaStream_t s);
+
+// Number of K splits for an M x N x K weight-streaming GEMM; always a count
+// that gemm_tc uses unchanged (see gemm_effective_splits).
+int gemm_pick_splits(int M, int N, int K, int max_splits);
+// The split count gemm_tc actually runs for a requested count: every split
+// gets ceil(k-blocks / splits) k-blocks, the last one possibly fewer.
+int gemm_effective_splits(int K, int splits);
+
+// ---------------------------------------------------------------- fp32 SIMT GEMM
+void gemm_simt_f32(const float* W, int N, int K, const float* const* xseg, int n_seg, int seg_k,
+                   int M, float* out, cudaStream_t s);
+
+// ---------------------------------------------------------------- row kernels
+template <typename T>
+void launch_embed_norm(const int32_t* tokens, const T* emb, const float* g, float* x, T* h, int M,
+                       int d, float eps, cudaStream_t s);
+template <typename T>
+void launch_residual_norm(const float* part, int splits, int M, int d, float* x, const float* g,
+                          T* h, const int32_t* out_row, float eps, cudaStream_t s);
+template <typename T>
+void launch_ctx_norm(const float* part, int splits, int n, int d, const float* g, T* c, float eps,
+                     cudaStream_t s);
+template <typename T>
+void launch_qkv_post(const float* part, int splits, int M, int B, const int32_t* ctx_len,
+                     const int32_t* req_valid, int nq, int nkv, int hd, const float* cos_t,
+                     const float* sin_t, T* q, T* kb, T* vb, cudaStream_t s);
+template <typename T>
+void launch_swiglu(const float* part, int splits, int M, int I, T* act, cudaStream_t s);
+template <typename T>
+void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int L, int nkv, int hd,
+                       const int32_t* cu_rows, const int32_t* start_pos, int batch, int cap,
+                       const float* cos_t, const float* sin_t, int max_pos, T* kc, T* vc,
+                       int32_t* err, cudaStream_t s);
+
+// ---------------------------------------------------------------- attention
+template <typename T>
+int launch_block_attention(const T* q, const T* kb, const T* vb, const T* kc, const T* vc,
+                           int layer, int batch, int cap, const int32_t* ctx_len,
+                           const int32_t* req_valid, int B, int nq, int nkv, int hd,
+                           float* part_o, float* part_ml, int n_chunks, int chunk, T* o,
+                           cudaStream_t s);
+
+// ---------------------------------------------------------------- draft bookkeeping
+void launch_draft_init(const int32_t* anchor, const int32_t* ctx_len, int batch, int B, int V,
+                       int mask_id, int cap, int32_t* tokens, int32_t* zrow, int32_t* lm_rows,
+                       int32_t* cstep, int32_t* req_valid, int32_t* err, cudaStream_t s);
+void launch_lm_reduce(const LmStat* stats, int n_vtiles, int rows, int32_t* tok, float* conf,
+                      cudaStream_t s);
+void launch_lm_stats_from_logits(const float* logits, int rows, int V, LmStat* stats,
+                                 float* dbg, const int32_t* dbg_rows, int64_t dbg_ld,
+                                 cudaStream_t s);
+void launch_commit(const int32_t* tok, const float* conf, int batch, int B, int rem, int k,
+                   int step, int32_t* tokens, int32_t* zrow, int32_t* lm_rows, int32_t* cstep,
+                   cudaStream_t s);
+void launch_draft_finish(const int32_t* tokens, const int32_t* cstep, const int32_t* req_valid,
+                         int batch, int B, int32_t* draft_out, int32_t* cstep_out,
+                         cudaStream_t s);
+
+// ---------------------------------------------------------------- verify
+int launch_verify(const void* logits, int dtype, const int32_t* draft, int batch, int B, int V,
+                  int32_t* out_tokens, int32_t* out_len, int out_cap, int32_t* seq_lens,
+                  int32_t* accept_len, int32_t* next_anchor, void* part, int chunks,
+                  int32_t* err, cudaStream_t s);
+int verify_chunks(int rows, int V);
+
+}  // namespace dflash

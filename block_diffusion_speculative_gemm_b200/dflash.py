@@ -1,0 +1,327 @@
+"""ctypes binding of libdflash.so (see include/dflash.h).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity and passed as raw pointers; every step of the hot path runs in the
+library's CUDA kernels.  PyTorch provides device memory and streams.  There
+is no fallback: if the library is missing, importing the binding fails.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Dict, Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdflash.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "dflash.h")
+HEADERS = [HEADER, os.path.join(os.path.dirname(_HERE), "include", "dflash_debug.h")]
+
+OK, EINVAL, EUNSUPPORTED, ECUDA, ENOMEM, EWORKSPACE = 0, -1, -2, -3, -4, -5
+DEV_CTX_CAP, DEV_OUT_CAP, DEV_TOKEN_RANGE, DEV_TIMEOUT, DEV_ROWS = 1, 2, 4, 8, 16
+F32, BF16 = 0, 1
+TIMING_CLASSES = ("gemm", "attention", "row", "verify", "lm_head")
+
+
+class DFlashError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        super().__init__(f"{call} failed: {status} ({status_str(status)})")
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "dtype", "H_t", "n_tap", "n_layers", "d", "n_q", "n_kv", "head_dim", "inter", "vocab",
+        "mask_id", "max_pos")] + [("eps", ctypes.c_float), ("rope_base", ctypes.c_double)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("g_in", "Wq", "Wk", "Wv", "Wo", "g_post", "Wg", "Wu", "Wd")]
+
+
+class Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("emb", "W_fc", "g_ctx", "g_final", "W_lm")] + [
+        ("layers", ctypes.POINTER(LayerWeights))]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m block_diffusion_speculative_gemm_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.dflash_model_create.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Weights),
+                                          ctypes.POINTER(vp)]
+        L.dflash_model_destroy.argtypes = [vp]
+        L.dflash_workspace_size.argtypes = [vp, i32, i32, i32]
+        L.dflash_workspace_size.restype = sz
+        L.dflash_verify_workspace_size.argtypes = [i32, i32, i32]
+        L.dflash_verify_workspace_size.restype = sz
+        L.dflash_workspace_init.argtypes = [vp, sz, vp]
+        L.dflash_inject_kv.argtypes = [vp, ctypes.POINTER(vp), vp, vp, i32, i32, vp, vp, i32, vp,
+                                       sz, vp]
+        L.dflash_draft_block.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp,
+                                         sz, vp]
+        L.dflash_verify.argtypes = [vp, i32, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp, sz,
+                                    vp]
+        L.dflash_get_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+        L.dflash_status_str.argtypes = [i32]
+        L.dflash_status_str.restype = ctypes.c_char_p
+        L.dflash_timing_enable.argtypes = [i32]
+        L.dflash_timing_read.argtypes = [ctypes.POINTER(ctypes.c_double),
+                                         ctypes.POINTER(ctypes.c_int64), i32]
+        L.dflash_debug_gemm_bf16.argtypes = [vp, i32, i32, vp, i32, i32, vp,
+                                             ctypes.POINTER(ctypes.c_int), vp, vp]
+        L.dflash_debug_lmhead_bf16.argtypes = [vp, i32, i32, vp, i32, vp, vp, vp, vp]
+        _lib = L
+    return _lib
+
+
+def header_symbols() -> list:
+    """Function names declared in the headers under include/."""
+    txt = ""
+    for h in HEADERS:
+        with open(h) as f:
+            txt += f.read()
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(dflash_\w+)\s*\(", txt,
+                                 flags=re.M)))
+
+
+def status_str(status: int) -> str:
+    return lib().dflash_status_str(int(status)).decode()
+
+
+def _check(call: str, st: int):
+    if st != OK:
+        raise DFlashError(call, st)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(int(stream.cuda_stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+_TORCH_DT = {F32: torch.float32, BF16: torch.bfloat16}
+
+
+class Model:
+    """A draft model prepacked on the current CUDA device.
+
+    ``shape`` is any object with attributes dtype ("f32"/"bf16"), H_t, n_tap,
+    L, d, nq, nkv, hd, I, V, mask_id, eps, rope_base.  ``weights`` is a dict
+    of CUDA tensors laid out as in include/dflash.h (keys emb, W_fc, g_ctx,
+    g_final, W_lm, layers[l] with g_in, Wq, Wk, Wv, Wo, g_post, Wg, Wu, Wd).
+    """
+
+    def __init__(self, shape, weights: Dict, max_pos: int):
+        self.shape = shape
+        self.dtype = BF16 if shape.dtype == "bf16" else F32
+        self.tdtype = _TORCH_DT[self.dtype]
+        cfg = Config(dtype=self.dtype, H_t=shape.H_t, n_tap=shape.n_tap, n_layers=shape.L,
+                     d=shape.d, n_q=shape.nq, n_kv=shape.nkv, head_dim=shape.hd, inter=shape.I,
+                     vocab=shape.V, mask_id=shape.mask_id, max_pos=int(max_pos),
+                     eps=float(shape.eps), rope_base=float(shape.rope_base))
+        keep = []
+
+        def p(t, name):
+            _need(t, name, self.tdtype)
+            keep.append(t)
+            return t.data_ptr()
+
+        layers = (LayerWeights * shape.L)()
+        for l, lw in enumerate(weights["layers"]):
+            for k in LayerWeights._fields_:
+                setattr(layers[l], k[0], p(lw[k[0]], f"layers[{l}].{k[0]}"))
+        w = Weights(emb=p(weights["emb"], "emb"), W_fc=p(weights["W_fc"], "W_fc"),
+                    g_ctx=p(weights["g_ctx"], "g_ctx"), g_final=p(weights["g_final"], "g_final"),
+                    W_lm=p(weights["W_lm"], "W_lm"), layers=layers)
+        handle = ctypes.c_void_p()
+        _check("dflash_model_create", lib().dflash_model_create(ctypes.byref(cfg), ctypes.byref(w),
+                                                                ctypes.byref(handle)))
+        self.handle = handle
+        self.max_pos = int(max_pos)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().dflash_model_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_size(self, max_batch: int, B: int, max_inject_rows: int) -> int:
+        return int(lib().dflash_workspace_size(self.handle, max_batch, B, max_inject_rows))
+
+    def workspace(self, max_batch: int, B: int, max_inject_rows: int, device=None) -> torch.Tensor:
+        return new_workspace(self.workspace_size(max_batch, B, max_inject_rows), device)
+
+
+def new_workspace(nbytes: int, device=None, stream=None) -> torch.Tensor:
+    """A zero-filled, 256-byte aligned device workspace of ``nbytes`` bytes."""
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+    assert ws.data_ptr() % 256 == 0
+    _check("dflash_workspace_init", lib().dflash_workspace_init(_ptr(ws), ws.numel(),
+                                                                _stream(stream)))
+    return ws
+
+
+def verify_workspace_size(batch: int, B: int, V: int) -> int:
+    return int(lib().dflash_verify_workspace_size(batch, B, V))
+
+
+def inject_kv(model: Model, taps: Sequence[torch.Tensor], cu_rows: torch.Tensor,
+              start_pos: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              ws: torch.Tensor, stream=None):
+    s = model.shape
+    batch = start_pos.numel()
+    n_rows = taps[0].shape[0]
+    if len(taps) != s.n_tap:
+        raise ValueError(f"expected {s.n_tap} taps")
+    for i, t in enumerate(taps):
+        _need(t, f"taps[{i}]", model.tdtype, (n_rows, s.H_t))
+    _need(cu_rows, "cu_rows", torch.int32, (batch + 1,))
+    _need(start_pos, "start_pos", torch.int32)
+    _need(k_cache, "k_cache", model.tdtype)
+    _need(v_cache, "v_cache", model.tdtype, k_cache.shape)
+    if k_cache.dim() != 5 or tuple(k_cache.shape[:3]) != (s.L, batch, s.nkv) or k_cache.shape[4] != s.hd:
+        raise ValueError("k_cache must be [L, batch, n_kv, cap, head_dim]")
+    _need(ws, "ws", torch.uint8)
+    arr = (ctypes.c_void_p * s.n_tap)(*[t.data_ptr() for t in taps])
+    _check("dflash_inject_kv", lib().dflash_inject_kv(
+        model.handle, arr, _ptr(cu_rows), _ptr(start_pos), batch, n_rows, _ptr(k_cache),
+        _ptr(v_cache), k_cache.shape[3], _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def draft_block(model: Model, anchor: torch.Tensor, ctx_len: torch.Tensor, k_cache: torch.Tensor,
+                v_cache: torch.Tensor, B: int, n_steps: int, draft_tokens: torch.Tensor,
+                ws: torch.Tensor, commit_step: Optional[torch.Tensor] = None,
+                logits_dbg: Optional[torch.Tensor] = None, stream=None):
+    s = model.shape
+    batch = anchor.numel()
+    _need(anchor, "anchor", torch.int32)
+    _need(ctx_len, "ctx_len", torch.int32, (batch,))
+    _need(k_cache, "k_cache", model.tdtype)
+    _need(v_cache, "v_cache", model.tdtype, k_cache.shape)
+    if k_cache.dim() != 5 or tuple(k_cache.shape[:3]) != (s.L, batch, s.nkv) or k_cache.shape[4] != s.hd:
+        raise ValueError("k_cache must be [L, batch, n_kv, cap, head_dim]")
+    _need(draft_tokens, "draft_tokens", torch.int32, (batch, B))
+    if commit_step is not None:
+        _need(commit_step, "commit_step", torch.int32, (batch, B))
+    if logits_dbg is not None:
+        _need(logits_dbg, "logits_dbg", torch.float32, (n_steps, batch, B, s.V))
+    _need(ws, "ws", torch.uint8)
+    _check("dflash_draft_block", lib().dflash_draft_block(
+        model.handle, _ptr(anchor), _ptr(ctx_len), _ptr(k_cache), _ptr(v_cache), k_cache.shape[3],
+        batch, B, n_steps, _ptr(draft_tokens), _ptr(commit_step), _ptr(logits_dbg), _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def verify(target_logits: torch.Tensor, draft_tokens: torch.Tensor, out_tokens: torch.Tensor,
+           out_len: torch.Tensor, seq_lens: torch.Tensor, accept_len: torch.Tensor,
+           next_anchor: torch.Tensor, ws: torch.Tensor, stream=None):
+    if target_logits.dim() != 3:
+        raise ValueError("target_logits must be [batch, B, V]")
+    batch, B, V = target_logits.shape
+    dt = {torch.bfloat16: BF16, torch.float32: F32}.get(target_logits.dtype)
+    if dt is None:
+        raise TypeError("target_logits must be bfloat16 or float32")
+    _need(target_logits, "target_logits")
+    _need(draft_tokens, "draft_tokens", torch.int32, (batch, B))
+    _need(out_tokens, "out_tokens", torch.int32)
+    if out_tokens.dim() != 2 or out_tokens.shape[0] != batch:
+        raise ValueError("out_tokens must be [batch, out_cap]")
+    for n, t in (("out_len", out_len), ("seq_lens", seq_lens), ("accept_len", accept_len),
+                 ("next_anchor", next_anchor)):
+        _need(t, n, torch.int32, (batch,))
+    _need(ws, "ws", torch.uint8)
+    _check("dflash_verify", lib().dflash_verify(
+        _ptr(target_logits), dt, _ptr(draft_tokens), batch, B, V, _ptr(out_tokens), _ptr(out_len),
+        out_tokens.shape[1], _ptr(seq_lens), _ptr(accept_len), _ptr(next_anchor), _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def get_error(ws: torch.Tensor, stream=None) -> int:
+    """Reads and clears the device error word (synchronises the stream)."""
+    bits = ctypes.c_int32(0)
+    _check("dflash_get_error", lib().dflash_get_error(_ptr(ws), _stream(stream), ctypes.byref(bits)))
+    return int(bits.value)
+
+
+def timing_enable(on: bool = True):
+    lib().dflash_timing_enable(1 if on else 0)
+
+
+def timing_read() -> Dict[str, Dict[str, float]]:
+    """Per kernel class: total device ms and launch count since the last read."""
+    n = len(TIMING_CLASSES)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    _check("dflash_timing_read", lib().dflash_timing_read(ms, cnt, n))
+    return {TIMING_CLASSES[i]: {"ms": ms[i], "launches": int(cnt[i])} for i in range(n)}
+
+
+# ---------------------------------------------------------------- test hooks (dflash_debug.h)
+
+def debug_gemm(W: torch.Tensor, X: torch.Tensor, splits: int, err_ws: torch.Tensor, stream=None):
+    """fp32 split-K partials [splits_used, M, N] of X @ W^T from the tcgen05 core."""
+    _need(W, "W", torch.bfloat16)
+    _need(X, "X", torch.bfloat16)
+    N, K = W.shape
+    M = X.shape[0]
+    nkb = K // 64
+    s_req = max(1, min(splits, nkb))
+    per = -(-nkb // s_req)
+    s_used = -(-nkb // per)
+    out = torch.empty((s_used, M, N), dtype=torch.float32, device=W.device)
+    used = ctypes.c_int(0)
+    _check("dflash_debug_gemm_bf16", lib().dflash_debug_gemm_bf16(
+        _ptr(W), N, K, _ptr(X), M, s_req, _ptr(out), ctypes.byref(used), _ptr(err_ws),
+        _stream(stream)))
+    assert used.value == s_used
+    return out
+
+
+def debug_lmhead(W: torch.Tensor, X: torch.Tensor, err_ws: torch.Tensor, want_logits=True,
+                 stream=None):
+    """(stats [M, tiles, 4] as (max, idx, sumexp, 0), logits [M, N] or None)."""
+    _need(W, "W", torch.bfloat16)
+    _need(X, "X", torch.bfloat16)
+    N, K = W.shape
+    M = X.shape[0]
+    tiles = -(-N // 128)
+    stats = torch.empty((M, tiles, 4), dtype=torch.float32, device=W.device)
+    logits = torch.empty((M, N), dtype=torch.float32, device=W.device) if want_logits else None
+    _check("dflash_debug_lmhead_bf16", lib().dflash_debug_lmhead_bf16(
+        _ptr(W), N, K, _ptr(X), M, _ptr(stats), _ptr(logits), _ptr(err_ws), _stream(stream)))
+    return stats, logits

@@ -1,0 +1,218 @@
+/*
+ * dflash.h - C ABI of the DFlash block-diffusion speculative-decoding hot path
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The three hot calls follow the problem statement of the DFlash pages:
+ *
+ *   dflash_inject_kv    "DFlash: Block Diffusion for Flash Speculative Decoding",
+ *                       §1 上下文特征提取 and §2 KV 注入; "DFlash + Spec V2 深度解析",
+ *                       §2.2 KV 注入: hidden states of tapped target layers are
+ *                       fused into context features and written into every draft
+ *                       layer's K/V cache (§Immediate Materialization: one
+ *                       layer-batched projection).
+ *   dflash_draft_block  "DFlash + Spec V2 深度解析", §2.3 块扩散: a block of
+ *                       [anchor, MASK, ..., MASK] is predicted in one forward per
+ *                       denoising step, most confident positions first.
+ *                       Blog "DFlash：用“块扩散”魔法", §核心创新:
+ *                       generate_block(context, block_size).
+ *   dflash_verify       Blog "DFlash：用“块扩散”魔法", §2 Flash Verification:
+ *                       decide_acceptance(logits, draft_block), read greedily.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Pointers marked "device" are CUDA device pointers in the caller's current
+ *   device; "host" pointers are read during the call only.  Every device buffer
+ *   is owned by the caller, except the model's prepacked weight copies, which
+ *   dflash_model_create allocates and dflash_model_destroy frees.  The hot calls
+ *   (inject, draft, verify) allocate nothing.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   The hot calls only enqueue work on it: none synchronises with the host.
+ * - Matrices are row-major.  Weight matrices are [out_features, in_features].
+ * - Return value: DFLASH_OK (0) or a negative DFLASH_E* code.  Host-side
+ *   argument checks happen before anything is enqueued; a failing call leaves
+ *   every buffer untouched.
+ * - Errors that only the device can see (a context too long for the cache, an
+ *   output buffer that would overflow, a token id outside [0, V), an expired
+ *   bounded wait) set bits in a sticky device error word inside the workspace;
+ *   the affected request writes nothing and the kernel never traps.
+ *   dflash_get_error reads and clears that word.
+ * - Workspace: a caller-allocated device buffer of at least the size the
+ *   matching *_workspace_size call returns, 256-byte aligned, zero-filled once
+ *   (dflash_workspace_init) before its first use.  Calls leave its counters at
+ *   zero.  Two calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef DFLASH_H
+#define DFLASH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------- */
+#define DFLASH_OK            0
+#define DFLASH_EINVAL       -1  /* null/misaligned pointer, bad size or shape */
+#define DFLASH_EUNSUPPORTED -2  /* dtype or shape the library was not built for */
+#define DFLASH_ECUDA        -3  /* a CUDA call or kernel launch failed */
+#define DFLASH_ENOMEM       -4  /* model creation could not allocate device memory */
+#define DFLASH_EWORKSPACE   -5  /* workspace smaller than the size query returned */
+
+/* ---- device error word bits (dflash_get_error) ------------------------ */
+#define DFLASH_DEV_CTX_CAP     1  /* position outside the K/V cache capacity */
+#define DFLASH_DEV_OUT_CAP     2  /* verify output would pass out_cap */
+#define DFLASH_DEV_TOKEN_RANGE 4  /* token id outside [0, V) */
+#define DFLASH_DEV_TIMEOUT     8  /* a bounded device wait expired */
+#define DFLASH_DEV_ROWS        16 /* cu_rows not monotone or not ending at n_rows */
+
+/* ---- element types ---------------------------------------------------- */
+#define DFLASH_F32  0
+#define DFLASH_BF16 1
+
+typedef struct dflash_model dflash_model; /* opaque */
+
+/* Draft model shape.  Constraints: n_q % n_kv == 0; head_dim even and <= 256.
+ * For DFLASH_BF16: d, H_t, inter, n_q*head_dim multiples of 64, head_dim 64 or
+ * 128.  For DFLASH_F32 (SIMT path, for small correctness models) no further
+ * constraint.  vocab >= 2; mask_id in [0, vocab). */
+typedef struct {
+  int32_t dtype;     /* DFLASH_F32 or DFLASH_BF16: weights, activations, K/V cache */
+  int32_t H_t;       /* target hidden size of one tapped layer */
+  int32_t n_tap;     /* tapped target layers (1..8) */
+  int32_t n_layers;  /* draft layers L */
+  int32_t d;         /* draft hidden size */
+  int32_t n_q;       /* query heads */
+  int32_t n_kv;      /* key/value heads */
+  int32_t head_dim;  /* per-head size */
+  int32_t inter;     /* SwiGLU intermediate size */
+  int32_t vocab;     /* V */
+  int32_t mask_id;   /* the [MASK] token id */
+  int32_t max_pos;   /* positions 0..max_pos-1 get a RoPE table entry */
+  float eps;         /* RMSNorm epsilon */
+  double rope_base;  /* RoPE base; angle of pair i at position p = p*base^(-2i/head_dim) */
+} dflash_config;
+
+/* One draft layer, device pointers in the config's dtype, borrowed during
+ * dflash_model_create only. */
+typedef struct {
+  const void* g_in;   /* [d]              input RMSNorm gain */
+  const void* Wq;     /* [n_q*hd, d] */
+  const void* Wk;     /* [n_kv*hd, d]     also projects the injected context */
+  const void* Wv;     /* [n_kv*hd, d]     also projects the injected context */
+  const void* Wo;     /* [d, n_q*hd] */
+  const void* g_post; /* [d]              post-attention RMSNorm gain */
+  const void* Wg;     /* [inter, d]       SwiGLU gate */
+  const void* Wu;     /* [inter, d]       SwiGLU up */
+  const void* Wd;     /* [d, inter]       SwiGLU down */
+} dflash_layer_weights;
+
+typedef struct {
+  const void* emb;      /* [V, d]           token embedding */
+  const void* W_fc;     /* [d, n_tap*H_t]   context-feature fc (taps concatenated in order) */
+  const void* g_ctx;    /* [d]              context-feature RMSNorm gain */
+  const void* g_final;  /* [d]              final RMSNorm gain */
+  const void* W_lm;     /* [V, d]           LM head */
+  const dflash_layer_weights* layers; /* host array of n_layers entries */
+} dflash_weights;
+
+/* Creates a model on the current device: checks the shape, prepacks the
+ * weights into library-owned device buffers (layer-batched [Wk;Wv] of every
+ * layer for injection, [Wq;Wk;Wv] and [Wg;Wu] per layer) and builds the RoPE
+ * cos/sin table in fp64 (stored fp32).  Synchronises the device once.
+ * Returns DFLASH_EINVAL / DFLASH_EUNSUPPORTED / DFLASH_ENOMEM / DFLASH_ECUDA. */
+int dflash_model_create(const dflash_config* cfg, const dflash_weights* w, dflash_model** out);
+
+/* Frees the model's device buffers (synchronises the device).  NULL is a no-op. */
+int dflash_model_destroy(dflash_model* m);
+
+/* Bytes of workspace that inject (up to max_inject_rows rows), draft (up to
+ * max_batch requests of block size B) and verify (max_batch x B rows) need. */
+size_t dflash_workspace_size(const dflash_model* m, int max_batch, int B, int max_inject_rows);
+
+/* Bytes of workspace that dflash_verify needs without a model. */
+size_t dflash_verify_workspace_size(int batch, int B, int V);
+
+/* Zero-fills a workspace (asynchronous on `stream`). */
+int dflash_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * KV injection.
+ *   taps[t]    host array of n_tap device pointers; taps[t] is [n_rows, H_t]
+ *              (hidden states of tapped layer t, ascending tap order), 16-byte aligned.
+ *   cu_rows    device int32 [batch+1]: rows cu_rows[r]..cu_rows[r+1]-1 belong to
+ *              request r; cu_rows[0] = 0, cu_rows[batch] = n_rows.
+ *   start_pos  device int32 [batch]: absolute position of request r's first row.
+ *   k_cache, v_cache  device [n_layers][batch][n_kv][cache_cap][head_dim] in the
+ *              model dtype; K is stored after RoPE.
+ * Computes c = RMSNorm(concat_t(taps[t]) W_fc^T; g_ctx) and, for every layer l,
+ * K_l[p] = RoPE(c Wk_l^T, p), V_l[p] = c Wv_l^T at p = start_pos[r] + i.
+ * Rows whose position falls outside [0, cache_cap) are skipped and set
+ * DFLASH_DEV_CTX_CAP.  n_rows == 0 is a no-op.
+ */
+int dflash_inject_kv(const dflash_model* m, const void* const* taps, const int32_t* cu_rows,
+                     const int32_t* start_pos, int batch, int n_rows, void* k_cache, void* v_cache,
+                     int cache_cap, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Masked-block draft forward with n_steps denoising steps.
+ *   anchor     device int32 [batch]: token at block position 0 (position ctx_len[r]).
+ *   ctx_len    device int32 [batch]: injected context length T_r; the block sits at
+ *              positions T_r..T_r+B-1 and attends to cache positions 0..T_r-1 plus
+ *              the whole block (no mask inside the block).
+ *   draft_tokens  device int32 [batch, B] out: anchor then the B-1 drafted tokens.
+ *   commit_step   device int32 [batch, B] out or NULL: denoising step at which each
+ *              position was committed (-1 at position 0).
+ *   logits_dbg    device fp32 [n_steps, batch, B, V] out or NULL: the LM-head logits
+ *              of every still-masked position at each step (other rows untouched).
+ * Step t commits the ceil(remaining / (n_steps - t)) masked positions with the
+ * highest softmax max-probability (ties to the lower position) to their argmax
+ * token (ties to the lower token id).  B in [2, 16], n_steps in [1, B-1].
+ * A request with ctx_len + B > cache_cap or an anchor outside [0, V) sets a
+ * device error bit and writes nothing.
+ */
+int dflash_draft_block(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_len,
+                       const void* k_cache, const void* v_cache, int cache_cap, int batch, int B,
+                       int n_steps, int32_t* draft_tokens, int32_t* commit_step, float* logits_dbg,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Greedy verify.
+ *   target_logits  device [batch, B, V] of logits_dtype (DFLASH_BF16 or DFLASH_F32),
+ *                  16-byte aligned; row i of request r scores the token after block
+ *                  position i.
+ *   draft_tokens   device int32 [batch, B] (position 0 = anchor).
+ *   out_tokens     device int32 [batch, out_cap]; out_len device int32 [batch] in/out.
+ *   seq_lens       device int32 [batch] in/out; accept_len, next_anchor device int32
+ *                  [batch] out.
+ * g_i = argmax_v logits[r, i] (lowest v on ties); a = longest prefix with
+ * g_i == draft[r, i+1], a <= B-1; emits draft[r, 1..a] then g_a at
+ * out_tokens[r, out_len[r]...]; out_len += a+1; seq_lens += a+1;
+ * accept_len = a; next_anchor = g_a.  A request whose draft holds an id outside
+ * [0, V) or whose emission would pass out_cap writes nothing and sets a device
+ * error bit.  B in [2, 32]; batch == 0 is a no-op.
+ */
+int dflash_verify(const void* target_logits, int logits_dtype, const int32_t* draft_tokens,
+                  int batch, int B, int V, int32_t* out_tokens, int32_t* out_len, int out_cap,
+                  int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor, void* ws,
+                  size_t ws_bytes, void* stream);
+
+/* Waits for `stream`, copies the workspace's device error word to *bits and
+ * clears it.  The only call that synchronises with the host. */
+int dflash_get_error(void* ws, void* stream, int32_t* bits);
+
+/* Static description of a status code. */
+const char* dflash_status_str(int status);
+
+/* Per-kernel-class device timing (CUDA events on the launching stream).  While
+ * enabled, every hot call records an event pair around each kernel it launches
+ * and adds the elapsed time to the class's total when dflash_timing_read is
+ * called.  Classes: 0 GEMM (tcgen05), 1 attention, 2 row/elementwise,
+ * 3 verify, 4 LM head.  read() synchronises on the recorded events. */
+int dflash_timing_enable(int on);
+int dflash_timing_read(double* ms_per_class, int64_t* launches_per_class, int n_classes);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DFLASH_H */

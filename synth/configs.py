@@ -93,8 +93,8 @@ VERIFY_SWEEP = {
 }
 
 
-def get_config(name: str, **overrides) -> DraftConfig:
-    cfg = CONFIGS[name]
+def get_config(key: str, **overrides) -> DraftConfig:
+    cfg = CONFIGS[key]
     return cfg.replace(**overrides) if overrides else cfg
 
 

@@ -1,0 +1,127 @@
+"""Masked-block draft forward on the GPU against the oracle.
+
+The K/V cache is filled with seeded synthetic values (the injection path has
+its own tests), so the oracle can recompute any request from the same cache.
+Draft tokens must equal the oracle's argmax except at near-ties (top-2 margin
+< 0.05); LM-head logits of every masked row agree within 1e-2 of max |oracle|;
+commit sets must be admitted by the oracle (see tests/gpu_common.py).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from synth.configs import shrink
+from tests.gpu_common import DraftReport, built, check_draft_request, oracle_caches_from
+from block_diffusion_speculative_gemm_b200 import dflash as D
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_draft(b, cfg, steps=None, dbg=True, ctx=None, anchors=None):
+    steps = cfg.steps if steps is None else steps
+    ctx = synth.make_ctx_lens(cfg) if ctx is None else ctx
+    anchors = synth.make_anchors(cfg) if anchors is None else anchors
+    kc, vc = synth.make_kv_cache(cfg, b.cap)
+    dk, dv = kc.cuda(), vc.cuda()
+    out = torch.full((cfg.batch, cfg.B), -5, dtype=torch.int32, device="cuda")
+    cst = torch.full((cfg.batch, cfg.B), -5, dtype=torch.int32, device="cuda")
+    lg = (torch.full((steps, cfg.batch, cfg.B, cfg.V), float("nan"), device="cuda")
+          if dbg else None)
+    ws = b.model.workspace(cfg.batch, cfg.B, 0)
+    D.draft_block(b.model, anchors.cuda(), ctx.cuda(), dk, dv, cfg.B, steps, out, ws,
+                  commit_step=cst, logits_dbg=lg)
+    torch.cuda.synchronize()
+    return dict(ctx=ctx, anchors=anchors, kc=kc, vc=vc, out=out.cpu(), cst=cst.cpu(),
+                lg=lg, err=D.get_error(ws))
+
+
+def _check(b, cfg, res, steps, requests):
+    rep = DraftReport()
+    for r in requests:
+        T = int(res["ctx"][r])
+        caches = oracle_caches_from(res["kc"], res["vc"], cfg.L, r, T)
+        glog = None
+        if res["lg"] is not None:
+            glog = [{p: res["lg"][t, r, p].cpu().numpy() for p in range(1, cfg.B)}
+                    for t in range(steps)]
+        check_draft_request(b, r, int(res["anchors"][r]), T, caches, res["out"][r],
+                            res["cst"][r], glog, steps, rep)
+        assert int(res["cst"][r][0]) == -1
+    return rep
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_draft_tiny(dtype):
+    cfg = synth.get_config("tiny_f32", dtype=dtype, name=f"tiny_{dtype}")
+    b = built(cfg)
+    res = _run_draft(b, cfg)
+    assert res["err"] == 0
+    rep = _check(b, cfg, res, cfg.steps, range(cfg.batch))
+    if dtype == "f32":
+        assert rep.max_logit_rel < 1e-5 and rep.token_near_ties == 0
+    print(rep)
+
+
+@pytest.mark.parametrize("steps", [1, 2, 3])
+def test_draft_tiny_bf16_denoising_steps(steps):
+    cfg = synth.get_config("tiny_f32", dtype="bf16", name="tiny_bf16", batch=3)
+    b = built(cfg)
+    res = _run_draft(b, cfg, steps=steps)
+    assert res["err"] == 0
+    print(_check(b, cfg, res, steps, range(cfg.batch)))
+
+
+@pytest.mark.parametrize("B,steps", [(8, 2), (16, 1), (4, 3)])
+def test_draft_small_8b_geometry(B, steps):
+    base = synth.get_config("qwen3_8b_bs32")
+    cfg = shrink(base, L=2, V=4096, batch=5, ctx=("uniform", 30, 700), I=1024, d=1024,
+                 H_t=512).replace(B=B, steps=steps, name=f"small8b_B{B}")
+    b = built(cfg)
+    res = _run_draft(b, cfg)
+    assert res["err"] == 0
+    print(_check(b, cfg, res, steps, range(cfg.batch)))
+
+
+def test_draft_context_lengths_edge_cases():
+    base = synth.get_config("qwen3_8b_bs32")
+    cfg = shrink(base, L=1, V=2048, batch=4, ctx=("fixed", 600), I=512, d=512, H_t=512).replace(
+        name="edge8b")
+    b = built(cfg)
+    # empty context, one position, a full chunk boundary, the longest context the cache holds
+    ctx = torch.tensor([0, 1, 256, b.cap - cfg.B], dtype=torch.int32)
+    res = _run_draft(b, cfg, ctx=ctx)
+    assert res["err"] == 0
+    print(_check(b, cfg, res, cfg.steps, range(cfg.batch)))
+
+
+def test_draft_rejects_bad_requests_without_writing():
+    base = synth.get_config("qwen3_8b_bs32")
+    cfg = shrink(base, L=1, V=2048, batch=3, ctx=("fixed", 16), I=512, d=512, H_t=512).replace(
+        name="bad8b")
+    b = built(cfg)
+    ctx = torch.tensor([16, b.cap - cfg.B + 1, 16], dtype=torch.int32)  # request 1 overflows
+    anchors = torch.tensor([5, 6, cfg.V], dtype=torch.int32)            # request 2 out of range
+    res = _run_draft(b, cfg, ctx=ctx, anchors=anchors, dbg=False)
+    assert res["err"] == D.DEV_CTX_CAP | D.DEV_TOKEN_RANGE
+    assert (res["out"][1] == -5).all() and (res["out"][2] == -5).all()
+    assert int(res["out"][0][0]) == 5 and (res["out"][0] >= 0).all()
+
+
+@pytest.mark.parametrize("name,requests", [
+    ("qwen3_4b_bs1", [0]),
+    ("qwen3_8b_bs32", [0, 13, 31]),
+    ("qwen3_8b_ctx32k", [2]),
+])
+def test_draft_full_size_sampled_requests(name, requests):
+    cfg = synth.get_config(name)
+    b = built(cfg)
+    res = _run_draft(b, cfg)
+    assert res["err"] == 0
+    # every request produced a complete block
+    out = res["out"]
+    assert (out[:, 1:] >= 0).all() and (out[:, 1:] < cfg.V).all()
+    assert (res["cst"][:, 1:] >= 0).all() and (res["cst"][:, 1:] < cfg.steps).all()
+    print(name, _check(b, cfg, res, cfg.steps, requests))

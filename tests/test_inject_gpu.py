@@ -1,0 +1,133 @@
+"""KV injection on the GPU against the oracle: K (after RoPE) and V of every
+draft layer at every injected position, within 1e-2 of max |oracle| per layer."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from synth.configs import shrink
+from tests.gpu_common import built, rel_err, REL_TOL
+from block_diffusion_speculative_gemm_b200 import dflash as D
+
+pytestmark = pytest.mark.gpu
+
+
+def _inject(b, cfg, mode, rows_check=None, cap=None):
+    cap = b.cap if cap is None else cap
+    ctx = synth.make_ctx_lens(cfg)
+    cu, st, n = synth.make_inject_layout(cfg, ctx, mode)
+    taps = synth.make_tap_hiddens(cfg, n, label=f"taps_{mode}")
+    kc = torch.zeros((cfg.L, cfg.batch, cfg.nkv, cap, cfg.hd), dtype=b.tdtype(), device="cuda")
+    vc = torch.zeros_like(kc)
+    ws = b.model.workspace(cfg.batch, cfg.B, n)
+    D.inject_kv(b.model, [t.cuda() for t in taps], cu.cuda(), st.cuda(), kc, vc, ws)
+    torch.cuda.synchronize()
+    return ctx, cu, st, n, taps, kc, vc, ws
+
+
+def _check_rows(b, cfg, cu, st, taps, kc, vc, rows):
+    """Oracle K/V for the given packed rows, compared per layer."""
+    cu_np = cu.numpy()
+    sub_taps = [t[rows] for t in taps]
+    c = O.context_features(sub_taps, b.W.mat("W_fc"), b.W.mat("g_ctx"), cfg.eps)
+    req = np.searchsorted(cu_np, rows, side="right") - 1
+    pos = st.numpy()[req] + rows - cu_np[req]
+    worst = 0.0
+    for l in range(cfg.L):
+        K, V = O.inject_kv(c, pos, b.W.layer(l, "Wk"), b.W.layer(l, "Wv"), cfg.nkv, cfg.hd,
+                           cfg.rope_base)
+        gk = kc[l][torch.as_tensor(req), :, torch.as_tensor(pos), :].float().cpu().numpy()
+        gv = vc[l][torch.as_tensor(req), :, torch.as_tensor(pos), :].float().cpu().numpy()
+        ek, ev = rel_err(gk, K), rel_err(gv, V)
+        worst = max(worst, ek, ev)
+        assert ek <= REL_TOL and ev <= REL_TOL, (l, ek, ev)
+    return worst
+
+
+@pytest.mark.parametrize("name,dtype", [("tiny_f32", "f32"), ("tiny_f32", "bf16")])
+def test_inject_tiny_prefill(name, dtype):
+    cfg = synth.get_config(name, dtype=dtype, name=f"{name}_{dtype}")
+    b = built(cfg)
+    ctx, cu, st, n, taps, kc, vc, ws = _inject(b, cfg, "prefill")
+    assert D.get_error(ws) == 0
+    worst = _check_rows(b, cfg, cu, st, taps, kc, vc, np.arange(n))
+    if dtype == "f32":
+        assert worst < 1e-5
+    # positions past the injected rows stay untouched
+    assert kc[:, :, :, n:, :].abs().max().item() == 0.0
+
+
+def test_inject_small_batched_steady_and_prefill():
+    base = synth.get_config("qwen3_8b_bs32")
+    cfg = shrink(base, L=2, V=4096, batch=6, ctx=("uniform", 40, 300), I=1024, d=1024, H_t=512)
+    b = built(cfg)
+    for mode in ("prefill", "steady"):
+        ctx, cu, st, n, taps, kc, vc, ws = _inject(b, cfg, mode)
+        assert D.get_error(ws) == 0
+        _check_rows(b, cfg, cu, st, taps, kc, vc, np.arange(n))
+
+
+def test_inject_qwen3_8b_steady_state_full_size():
+    cfg = synth.get_config("qwen3_8b_bs32")
+    b = built(cfg)
+    ctx, cu, st, n, taps, kc, vc, ws = _inject(b, cfg, "steady")
+    assert 32 <= n <= 32 * cfg.B
+    assert D.get_error(ws) == 0
+    _check_rows(b, cfg, cu, st, taps, kc, vc, np.arange(n))
+
+
+def test_inject_qwen3_4b_prefill_sampled_rows():
+    cfg = synth.get_config("qwen3_4b_bs1")
+    b = built(cfg)
+    ctx, cu, st, n, taps, kc, vc, ws = _inject(b, cfg, "prefill")
+    assert D.get_error(ws) == 0
+    rows = np.unique(np.concatenate([np.arange(0, n, 97), [n - 1]]))
+    _check_rows(b, cfg, cu, st, taps, kc, vc, rows)
+
+
+def test_inject_chunks_equal_one_call():
+    base = synth.get_config("qwen3_8b_bs32")
+    cfg = shrink(base, L=2, V=4096, batch=2, ctx=("fixed", 64), I=1024, d=1024, H_t=512)
+    b = built(cfg)
+    taps = synth.make_tap_hiddens(cfg, 128, label="chunks")
+    cap = b.cap
+    kc1 = torch.zeros((cfg.L, 2, cfg.nkv, cap, cfg.hd), dtype=torch.bfloat16, device="cuda")
+    vc1 = torch.zeros_like(kc1)
+    kc2, vc2 = torch.zeros_like(kc1), torch.zeros_like(kc1)
+    ws = b.model.workspace(2, cfg.B, 128)
+    dt = [t.cuda() for t in taps]
+    one_cu = torch.tensor([0, 64, 128], dtype=torch.int32).cuda()
+    D.inject_kv(b.model, dt, one_cu, torch.tensor([0, 0], dtype=torch.int32).cuda(), kc1, vc1, ws)
+    # same rows in two calls of 32 rows per request
+    for half in range(2):
+        rows = torch.cat([torch.arange(half * 32, half * 32 + 32),
+                          torch.arange(64 + half * 32, 64 + half * 32 + 32)])
+        sub = [t[rows].contiguous() for t in dt]
+        D.inject_kv(b.model, sub, torch.tensor([0, 32, 64], dtype=torch.int32).cuda(),
+                    torch.tensor([32 * half, 32 * half], dtype=torch.int32).cuda(), kc2, vc2, ws)
+    torch.cuda.synchronize()
+    assert D.get_error(ws) == 0
+    scale = kc1.float().abs().max().item()
+    assert (kc1.float() - kc2.float()).abs().max().item() <= 1e-2 * scale
+    assert (vc1.float() - vc2.float()).abs().max().item() <= 1e-2 * vc1.float().abs().max().item()
+
+
+def test_inject_past_capacity_sets_error_and_skips():
+    base = synth.get_config("qwen3_8b_bs32")
+    cfg = shrink(base, L=2, V=4096, batch=2, ctx=("fixed", 64), I=1024, d=1024, H_t=512)
+    b = built(cfg)
+    cap = 48
+    taps = [t.cuda() for t in synth.make_tap_hiddens(cfg, 8, label="cap")]
+    kc = torch.zeros((cfg.L, 2, cfg.nkv, cap, cfg.hd), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    ws = b.model.workspace(2, cfg.B, 8)
+    cu = torch.tensor([0, 4, 8], dtype=torch.int32).cuda()
+    st = torch.tensor([10, 46], dtype=torch.int32).cuda()  # request 1 rows at 46..49: two past cap
+    D.inject_kv(b.model, taps, cu, st, kc, vc, ws)
+    torch.cuda.synchronize()
+    assert D.get_error(ws) == D.DEV_CTX_CAP
+    assert kc[:, 0, :, 10:14].abs().max().item() > 0
+    assert kc[:, 1, :, 46:48].abs().max().item() > 0
+    assert kc[:, 0, :, :10].abs().max().item() == 0 and kc[:, 0, :, 14:].abs().max().item() == 0
