@@ -1,0 +1,496 @@
+"""Benchmark of the DFlash draft hot path on B200.
+
+One step = one whole cycle of the hot path over the Qwen3-8B-shaped workload
+with 32 requests (contexts uniform in [512, 4096], block 8, two denoising
+steps): KV injection of the rows accepted in the previous cycle, the masked
+block draft (both denoising steps) and greedy verify of the block against
+given target logits.  Metric: block tokens per second of that cycle
+(32 * 8 tokens drafted and verified per step); the JSON line also carries the
+draft-only and verify-only rates, the per-kernel-class device times and the
+roofline of the dominant kernel class.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dflash|reference]
+
+Multi-GPU: one process per GPU (torchrun), every rank runs its own 32
+requests (requests are independent: no data-path collective), max time over
+ranks, value = all ranks' tokens / that time.  `--impl reference` times the
+fp64 CPU oracle on a bounded sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from synth.device import to_device  # noqa: E402
+
+WORKLOAD = "qwen3_8b_bs32"
+METRIC = "draft-block tokens/s + verify rows/s at 8B-shape bs32, % of HBM/TC roofline"
+UNIT = "block tok/s"
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, period_ms: int = 50):
+        self.idx = device_index
+        self.period = period_ms
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 f"-lms={self.period}"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        # samples under load: the upper half of the observed clocks
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gemm_bytes(N, K, M, out_bytes_per_row):
+    """Algorithmic bytes of one weight-streaming GEMM: weights + inputs + outputs."""
+    return N * K * 2 + M * K * 2 + M * out_bytes_per_row
+
+
+def step_algorithmic(cfg, n_inject, ctx_lens):
+    """Algorithmic bytes / flops of one cycle, per kernel class."""
+    b, B, L, d = cfg.batch, cfg.B, cfg.L, cfg.d
+    M = b * B
+    q = cfg.nq * cfg.hd
+    kv = cfg.nkv * cfg.hd
+    qkv = q + 2 * kv
+    out = {"gemm": {"bytes": 0, "flops": 0, "launches": 0}, "lm_head": {"bytes": 0, "flops": 0},
+           "attention": {"bytes": 0}, "verify": {"bytes": 0}}
+    g = out["gemm"]
+    # injection: fc over the concatenated taps, then the layer-batched K/V projection
+    for N, K in ((d, cfg.n_tap * cfg.H_t), (L * 2 * kv, d)):
+        g["bytes"] += gemm_bytes(N, K, n_inject, N * 2)
+        g["flops"] += 2 * N * K * n_inject
+    rem = B - 1
+    for t in range(cfg.steps):
+        k = -(-rem // (cfg.steps - t))
+        for N, K in ((qkv, d), (d, q), (2 * cfg.I, d), (d, cfg.I)):
+            g["bytes"] += L * gemm_bytes(N, K, M, N * 2)
+            g["flops"] += L * 2 * N * K * M
+        rows = b * rem
+        n_vt = -(-cfg.V // 128)
+        out["lm_head"]["bytes"] += gemm_bytes(cfg.V, d, rows, n_vt * 16)
+        out["lm_head"]["flops"] += 2 * cfg.V * d * rows
+        # attention: context K and V of every layer, plus the block's q/k/v/o rows
+        T = int(ctx_lens.sum())
+        out["attention"]["bytes"] += L * (T * kv * 2 * 2 + M * (2 * q + 2 * kv) * 2)
+        rem -= k
+    out["verify"]["bytes"] = M * cfg.V * 2 + M * 4 * 2
+    return out
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_dflash(args, rank, world, local_rank):
+    from block_diffusion_speculative_gemm_b200 import dflash as D
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = synth.get_config(WORKLOAD)
+    b, B, V = cfg.batch, cfg.B, cfg.V
+    cap = cfg.cache_cap
+    w = synth.make_weights(cfg)
+    model = D.Model(cfg, to_device(w, dev), cap + 2 * B + 16)
+    ctx = synth.make_ctx_lens(cfg)
+    anchors = synth.make_anchors(cfg)
+    kc = torch.zeros((cfg.L, b, cfg.nkv, cap, cfg.hd), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+
+    # prefix: inject every context position once (tapped hiddens drawn on the device)
+    cu_p, st_p, n_p = synth.make_inject_layout(cfg, ctx, "prefill")
+    cu_s, st_s, n_s = synth.make_inject_layout(cfg, ctx, "steady")
+    ws = model.workspace(b, B, max(n_s, 16384))
+    gen = torch.Generator(device=dev).manual_seed(synth.sub_seed(0x5EED, WORKLOAD, "prefix"))
+    cu_p_d = cu_p.to(dev)
+    taps_p = [(torch.randn((n_p, cfg.H_t), generator=gen, device=dev) * cfg.h_std).to(torch.bfloat16)
+              for _ in range(cfg.n_tap)]
+    D.inject_kv(model, taps_p, cu_p_d, st_p.to(dev), kc, vc, ws)
+    del taps_p
+    torch.cuda.synchronize()
+    assert D.get_error(ws) == 0
+
+    taps_s = [t.to(dev) for t in synth.make_tap_hiddens(cfg, n_s, label="taps_steady")]
+    cu_s_d, st_s_d = cu_s.to(dev), st_s.to(dev)
+    anchors_d, ctx_d = anchors.to(dev), ctx.to(dev)
+    draft = torch.zeros((b, B), dtype=torch.int32, device=dev)
+    D.draft_block(model, anchors_d, ctx_d, kc, vc, B, cfg.steps, draft, ws)
+    torch.cuda.synchronize()
+    # target logits whose greedy argmax agrees with the drafted block on a planted prefix
+    case = synth.make_verify_case(b, B, V, "bench", plant=cfg.plant, draft=draft.cpu())
+    logits = case["logits"].to(dev)
+    steps_total = args.warmup + args.steps + 4
+    out_cap = steps_total * B
+    out_tok = torch.zeros((b, out_cap), dtype=torch.int32, device=dev)
+    out_len = torch.zeros(b, dtype=torch.int32, device=dev)
+    seq = ctx.clone().to(dev)
+    acc = torch.zeros(b, dtype=torch.int32, device=dev)
+    nxt = torch.zeros(b, dtype=torch.int32, device=dev)
+
+    def step():
+        D.inject_kv(model, taps_s, cu_s_d, st_s_d, kc, vc, ws)
+        D.draft_block(model, anchors_d, ctx_d, kc, vc, B, cfg.steps, draft, ws)
+        D.verify(logits, draft, out_tok, out_len, seq, acc, nxt, ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.timing_read()  # discard
+    D.timing_enable(True)
+    with ClockSampler(local_rank) as clk:
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+    D.timing_enable(False)
+    per_class = D.timing_read()
+    ms = e0.elapsed_time(e1)
+    err = D.get_error(ws)
+    if err:
+        raise RuntimeError(f"device error word {err}")
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+    ms_step = ms_max / args.steps
+    tokens = b * B * world
+    value = tokens / (ms_step / 1e3)
+
+    # ---- per-class device times (this rank) and the roofline of the dominant class
+    peaks = load_peaks()
+    alg = step_algorithmic(cfg, n_s, ctx)
+    classes = {}
+    for name, key in (("gemm", "gemm"), ("attention", "attention"), ("lm_head", "lm_head"),
+                      ("verify", "verify"), ("row", "row")):
+        c = per_class.get(key, {"ms": 0.0, "launches": 0})
+        classes[name] = {"ms_per_step": c["ms"] / args.steps,
+                         "launches_per_step": c["launches"] / args.steps}
+    for name in ("gemm", "attention", "lm_head", "verify"):
+        t = classes[name]["ms_per_step"] / 1e3
+        if t > 0:
+            classes[name]["algorithmic_GBps"] = alg[name]["bytes"] / t / 1e9
+            classes[name]["frac_hbm"] = classes[name]["algorithmic_GBps"] / peaks["hbm_gbs"]
+    dom = max(("gemm", "attention", "lm_head", "verify"), key=lambda n: classes[n]["ms_per_step"])
+    launches = sum(int(c["launches"]) for c in per_class.values())
+    n_dom = per_class[dom]["launches"] / args.steps
+    traffic = load_traffic(dom)
+    achieved = classes[dom]["algorithmic_GBps"]
+    roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "peak_source": peaks["source"],
+            "algorithmic_bytes_per_launch": alg[dom]["bytes"] / max(n_dom, 1),
+            "avg_launch_ms": classes[dom]["ms_per_step"] / max(n_dom, 1),
+            "traffic": traffic}
+    # whole-cycle roofline: every class at HBM speed (all are bandwidth-bound at M <= 256)
+    roof_ms = sum(alg[n]["bytes"] for n in ("gemm", "attention", "lm_head", "verify")) / (
+        peaks["hbm_gbs"] * 1e9) * 1e3
+    draft_ms = sum(classes[n]["ms_per_step"] for n in ("gemm", "attention", "lm_head", "row"))
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded random-init weights and inputs)",
+        "config": {"workload": WORKLOAD, "model": "Qwen3-8B-shaped DFlash draft (5 layers)",
+                   "global_batch": b * world, "block": B, "denoise_steps": cfg.steps,
+                   "ctx": "uniform[512,4096]", "inject_rows": n_s, "parallelism": f"dp{world}",
+                   "l2": "no flush: every step streams ~7.4 GB of weights and K/V (> 126 MB L2)"},
+        "roofline": roof,
+        "cycle_roofline_ms": round(roof_ms, 4),
+        "cycle_frac_of_roofline": round(roof_ms / ms_step, 4),
+        "classes": classes,
+        "gpu_launches": launches,
+        "verify_rows_s": round(b * B / (classes["verify"]["ms_per_step"] / 1e3), 1)
+        if classes["verify"]["ms_per_step"] > 0 else None,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_e2e:
+        res["e2e"] = run_e2e(args, D, model, cfg, taps_s, cu_s, st_s, anchors, ctx, case, kc, vc, ws,
+                             dev, world)
+    elif world > 1 and not args.no_e2e:
+        run_e2e(args, D, model, cfg, taps_s, cu_s, st_s, anchors, ctx, case, kc, vc, ws, dev, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, cfg, ctx, anchors, cu_s, st_s, n_s, case)
+    model.close()
+    return res
+
+
+def run_e2e(args, D, model, cfg, taps_s, cu_s, st_s, anchors, ctx, case, kc, vc, ws, dev, world):
+    """Same cycle through the public API with host inputs/outputs: every step copies its
+    inputs from pinned host memory and reads its results back."""
+    b, B = cfg.batch, cfg.B
+    h_taps = [t.cpu().pin_memory() for t in taps_s]
+    h_small = {k: v.pin_memory() for k, v in dict(cu=cu_s, st=st_s, anchor=anchors, ctx=ctx).items()}
+    h_logits = case["logits"].pin_memory()
+    d_taps = [torch.empty_like(t) for t in taps_s]
+    d_small = {k: torch.empty_like(v, device=dev) for k, v in h_small.items()}
+    d_logits = torch.empty_like(h_logits, device=dev)
+    draft = torch.zeros((b, B), dtype=torch.int32, device=dev)
+    steps = max(3, args.steps // 4)
+    out_cap = (steps + 8) * B
+    out_tok = torch.zeros((b, out_cap), dtype=torch.int32, device=dev)
+    out_len = torch.zeros(b, dtype=torch.int32, device=dev)
+    seq = torch.zeros(b, dtype=torch.int32, device=dev)
+    acc = torch.zeros(b, dtype=torch.int32, device=dev)
+    nxt = torch.zeros(b, dtype=torch.int32, device=dev)
+    h_res = {k: torch.empty(v.shape, dtype=torch.int32).pin_memory() for k, v in
+             dict(draft=draft, acc=acc, nxt=nxt, out_len=out_len).items()}
+    h2d = sum(t.numel() * t.element_size() for t in h_taps) + sum(
+        v.numel() * 4 for v in h_small.values()) + h_logits.numel() * 2
+    d2h = sum(v.numel() * 4 for v in h_res.values())
+
+    def step():
+        for h, d in zip(h_taps, d_taps):
+            d.copy_(h, non_blocking=True)
+        for k in h_small:
+            d_small[k].copy_(h_small[k], non_blocking=True)
+        d_logits.copy_(h_logits, non_blocking=True)
+        seq.copy_(d_small["ctx"])
+        D.inject_kv(model, d_taps, d_small["cu"], d_small["st"], kc, vc, ws)
+        D.draft_block(model, d_small["anchor"], d_small["ctx"], kc, vc, B, cfg.steps, draft, ws)
+        D.verify(d_logits, draft, out_tok, out_len, seq, acc, nxt, ws)
+        for k, d in (("draft", draft), ("acc", acc), ("nxt", nxt), ("out_len", out_len)):
+            h_res[k].copy_(d, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    out_len.zero_()
+    for _ in range(2):
+        step()
+    out_len.zero_()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(b * B * world / (ms / steps / 1e3), 1), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+def load_traffic(kernel_class):
+    """DRAM traffic per launch of a kernel class from the committed ncu summary, if it was
+    captured from the current source of that kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        ent = d.get(kernel_class)
+        if not ent:
+            return None
+        import hashlib
+        src = os.path.join(ROOT, ent["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        return ent["bytes_per_launch"] if h == ent["source_sha256"] else None
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ oracle (CPU) legs
+
+def oracle_cycle(O, W, cfg, ctx, anchors, cu_s, st_s, taps_h, case, r, caches_by_req):
+    """One request's cycle in the oracle: inject its new rows, draft its block, verify it."""
+    lo, hi = int(cu_s[r]), int(cu_s[r + 1])
+    T = int(ctx[r])
+    c = O.context_features([t[lo:hi] for t in taps_h], W.mat("W_fc"), W.mat("g_ctx"), cfg.eps)
+    pos = int(st_s[r]) + (torch.arange(hi - lo)).numpy()
+    caches = caches_by_req[r]
+    for l in range(cfg.L):
+        K, V = O.inject_kv(c, pos, W.layer(l, "Wk"), W.layer(l, "Wv"), cfg.nkv, cfg.hd,
+                           cfg.rope_base)
+        caches[l][0][pos] = K
+        caches[l][1][pos] = V
+    toks, _ = O.draft_block(int(anchors[r]), T, [(k[:T], v[:T]) for k, v in caches], W, cfg)
+    return O.verify_request(case["logits"][r], case["draft"][r])
+
+
+def _oracle_caches(cfg, T, seed):
+    import numpy as np
+
+    rng = np.random.default_rng(seed)
+    s = synth.gen.kv_std(cfg)
+    return [(rng.normal(0, s, size=(T, cfg.nkv, cfg.hd)), rng.normal(0, s, size=(T, cfg.nkv, cfg.hd)))
+            for _ in range(cfg.L)]
+
+
+def cpu_baseline(w, cfg, ctx, anchors, cu_s, st_s, n_s, case, n_req=1):
+    """The oracle, as it stands, on a bounded sample: the first request's full cycle."""
+    import oracle as O
+
+    taps_h = synth.make_tap_hiddens(cfg, n_s, label="taps_steady")
+    caches = {r: _oracle_caches(cfg, int(ctx[r]), r) for r in range(n_req)}
+    threads = torch.get_num_threads()
+    t0 = time.perf_counter()
+    W = O.Weights64(w, cfg)
+    for r in range(n_req):
+        oracle_cycle(O, W, cfg, ctx, anchors, cu_s, st_s, taps_h, case, r, caches)
+    dt = time.perf_counter() - t0
+    return {"value": round(n_req * cfg.B / dt, 4), "unit": UNIT, "cores": os.cpu_count(),
+            "threads": threads, "kind": "oracle",
+            "sample": f"{n_req} of {cfg.batch} requests: inject its rows, 2-step draft, verify; "
+                      f"fp64 NumPy, weights converted once per sample ({dt:.1f} s)"}
+
+
+def run_reference(args):
+    """The oracle timed as the reference arm: each step is one request's cycle."""
+    import oracle as O
+
+    cfg = synth.get_config(WORKLOAD)
+    w = synth.make_weights(cfg)
+    ctx = synth.make_ctx_lens(cfg)
+    anchors = synth.make_anchors(cfg)
+    cu_s, st_s, n_s = synth.make_inject_layout(cfg, ctx, "steady")
+    case = synth.make_verify_case(cfg.batch, cfg.B, cfg.V, "bench_ref", plant=cfg.plant)
+    taps_h = synth.make_tap_hiddens(cfg, n_s, label="taps_steady")
+    W = O.Weights64(w, cfg)
+    caches = {r: _oracle_caches(cfg, int(ctx[r]), r) for r in range(cfg.batch)}
+    times = []
+    for i in range(args.warmup + args.steps):
+        r = i % cfg.batch
+        t0 = time.perf_counter()
+        oracle_cycle(O, W, cfg, ctx, anchors, cu_s, st_s, taps_h, case, r, caches)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = cfg.B / sec
+    cores = os.cpu_count()
+    return {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded random-init weights and inputs)", "impl": "reference",
+            "config": {"workload": WORKLOAD, "sample": "one request's cycle per step"},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores,
+                             "kind": "oracle",
+                             "sample": "one of 32 requests per step: inject, 2-step draft, verify"},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="dflash", choices=["dflash", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            requested = args.steps
+            args.steps = min(args.steps, 8)  # each step is seconds of fp64 CPU work
+            line = run_reference(args)
+            line["steps_requested"] = requested
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        res = run_dflash(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

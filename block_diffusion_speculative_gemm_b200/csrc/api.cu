@@ -152,6 +152,28 @@ bool copy_rows(void* dst, const void* src, size_t bytes) {
   return src != nullptr && cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToDevice) == cudaSuccess;
 }
 
+__global__ void bf16_to_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
+                                   size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = __float2half_rn(__bfloat162float(src[i]));
+}
+
+// Copies `elems` weight elements into a prepacked buffer.  For the bf16 model
+// type the GEMM weights are stored as fp16: every bf16 value of magnitude in
+// [2^-14, 65504] is exactly representable in fp16 (10 vs 7 mantissa bits);
+// smaller values land on fp16 subnormals (absolute error <= 2^-25).  fp16
+// operands let the activations that feed the tensor cores be stored with 3
+// more mantissa bits at the same tcgen05 rate.
+bool pack_weights(const dflash_model* m, void* dst, const void* src, size_t elems) {
+  if (!src) return false;
+  if (m->cfg.dtype != DFLASH_BF16) return copy_rows(dst, src, elems * sizeof(float));
+  const unsigned blocks = (unsigned)std::min<size_t>((elems + 255) / 256, 148 * 32);
+  bf16_to_f16_kernel<<<blocks, 256>>>(static_cast<const __nv_bfloat16*>(src),
+                                      static_cast<__half*>(dst), elems);
+  return cudaGetLastError() == cudaSuccess;
+}
+
 float* gain_copy(dflash_model* m, const void* g) {
   const int d = m->cfg.d;
   float* out = static_cast<float*>(dmalloc(m, sizeof(float) * d));
@@ -328,9 +350,11 @@ extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weight
   m->W_lm = dmalloc(m, e * V * d);
   m->W_kv = dmalloc(m, e * c.n_layers * 2 * nkv * hd * d);
   if (!m->emb || !m->W_fc || !m->W_lm || !m->W_kv) return fail(DFLASH_ENOMEM);
+  // embedding and fc stay in the model dtype (their inputs are exact in it);
+  // every other GEMM weight goes through pack_weights
   if (!copy_rows(m->emb, w->emb, e * V * d) ||
       !copy_rows(m->W_fc, w->W_fc, e * d * c.n_tap * c.H_t) ||
-      !copy_rows(m->W_lm, w->W_lm, e * V * d))
+      !pack_weights(m, m->W_lm, w->W_lm, V * d))
     return fail(DFLASH_EINVAL);
   m->g_ctx = gain_copy(m, w->g_ctx);
   m->g_final = gain_copy(m, w->g_final);
@@ -348,12 +372,12 @@ extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weight
     uint8_t* qkv = static_cast<uint8_t*>(P.Wqkv);
     uint8_t* gu = static_cast<uint8_t*>(P.Wgu);
     uint8_t* kv = static_cast<uint8_t*>(m->W_kv) + (size_t)l * 2 * kvrows * d * e;
-    if (!copy_rows(qkv, lw.Wq, e * nq * hd * d) ||
-        !copy_rows(qkv + e * nq * hd * d, lw.Wk, e * kvrows * d) ||
-        !copy_rows(qkv + e * (nq * hd + kvrows) * d, lw.Wv, e * kvrows * d) ||
-        !copy_rows(P.Wo, lw.Wo, e * d * nq * hd) || !copy_rows(gu, lw.Wg, e * I * d) ||
-        !copy_rows(gu + e * I * d, lw.Wu, e * I * d) || !copy_rows(P.Wd, lw.Wd, e * d * I) ||
-        !copy_rows(kv, lw.Wk, e * kvrows * d) || !copy_rows(kv + e * kvrows * d, lw.Wv, e * kvrows * d))
+    if (!pack_weights(m, qkv, lw.Wq, nq * hd * d) ||
+        !pack_weights(m, qkv + e * nq * hd * d, lw.Wk, kvrows * d) ||
+        !pack_weights(m, qkv + e * (nq * hd + kvrows) * d, lw.Wv, kvrows * d) ||
+        !pack_weights(m, P.Wo, lw.Wo, d * nq * hd) || !pack_weights(m, gu, lw.Wg, I * d) ||
+        !pack_weights(m, gu + e * I * d, lw.Wu, I * d) || !pack_weights(m, P.Wd, lw.Wd, d * I) ||
+        !pack_weights(m, kv, lw.Wk, kvrows * d) || !pack_weights(m, kv + e * kvrows * d, lw.Wv, kvrows * d))
       return fail(DFLASH_EINVAL);
     P.g_in = gain_copy(m, lw.g_in);
     P.g_post = gain_copy(m, lw.g_post);
@@ -369,15 +393,16 @@ extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weight
                                                              half, c.rope_base);
   }
   if (c.dtype == DFLASH_BF16) {
-    bool ok = encode_weight_map(m->mfc, m->W_fc, c.d, c.n_tap * c.H_t) &&
-              encode_weight_map(m->mkv, m->W_kv, c.n_layers * 2 * kvrows, c.d) &&
-              encode_weight_map(m->mlm, m->W_lm, c.vocab, c.d);
+    const int H = DFLASH_F16;
+    bool ok = encode_weight_map(m->mfc, m->W_fc, c.d, c.n_tap * c.H_t, DFLASH_BF16) &&
+              encode_weight_map(m->mkv, m->W_kv, c.n_layers * 2 * kvrows, c.d, H) &&
+              encode_weight_map(m->mlm, m->W_lm, c.vocab, c.d, H);
     for (int l = 0; l < c.n_layers && ok; ++l) {
       LayerPack& P = m->layers[l];
-      ok = encode_weight_map(P.mqkv, P.Wqkv, qkv_out(c), c.d) &&
-           encode_weight_map(P.mo, P.Wo, c.d, c.n_q * c.head_dim) &&
-           encode_weight_map(P.mgu, P.Wgu, 2 * c.inter, c.d) &&
-           encode_weight_map(P.md, P.Wd, c.d, c.inter);
+      ok = encode_weight_map(P.mqkv, P.Wqkv, qkv_out(c), c.d, H) &&
+           encode_weight_map(P.mo, P.Wo, c.d, c.n_q * c.head_dim, H) &&
+           encode_weight_map(P.mgu, P.Wgu, 2 * c.inter, c.d, H) &&
+           encode_weight_map(P.md, P.Wd, c.d, c.inter, H);
     }
     if (!ok) return fail(DFLASH_ECUDA);
   }
@@ -463,8 +488,7 @@ extern "C" int dflash_inject_kv(const dflash_model* m, const void* const* taps,
       o.part = part;
       st = gemm_tc(m->mfc, seg, c.n_tap, c.H_t, c.H_t, n, s1, EPI_PARTIAL, o, err, s);
       if (st) return st;
-      launch_ctx_norm<__nv_bfloat16>(part, s1, n, c.d, m->g_ctx,
-                                     static_cast<__nv_bfloat16*>(cbuf), c.eps, s);
+      launch_ctx_norm<__half>(part, s1, n, c.d, m->g_ctx, static_cast<__half*>(cbuf), c.eps, s);
       const int s2 = splits_for(n, kvN, c.d, L.part_elems);
       const void* cseg[1] = {cbuf};
       st = gemm_tc(m->mkv, cseg, 1, c.d, c.d, n, s2, EPI_PARTIAL, o, err, s);
@@ -493,7 +517,8 @@ extern "C" int dflash_inject_kv(const dflash_model* m, const void* const* taps,
 // ============================================================== draft
 namespace {
 
-template <typename T>
+// T: activation / GEMM operand type; TC: K/V cache type; TE: embedding type.
+template <typename T, typename TC, typename TE>
 int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_len,
                const void* k_cache, const void* v_cache, int cap, int batch, int B, int n_steps,
                int32_t* draft_tokens, int32_t* commit_step, float* logits_dbg, void* ws,
@@ -521,13 +546,14 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
   float* attn_o = at<float>(ws, L.attn_o);
   float* attn_ml = at<float>(ws, L.attn_ml);
   LmStat* stats = at<LmStat>(ws, L.stats);
-  const T* kc = static_cast<const T*>(k_cache);
-  const T* vc = static_cast<const T*>(v_cache);
+  const TC* kc = static_cast<const TC*>(k_cache);
+  const TC* vc = static_cast<const TC*>(v_cache);
   const int n_vt = (c.vocab + kTileN - 1) / kTileN;
   const bool bf16 = c.dtype == DFLASH_BF16;
 
+  // split-KV chunk: a multiple of the attention tile (64 keys), at least 512 keys
   int chunk = (cap + B + kMaxChunks - 1) / kMaxChunks;
-  chunk = std::max(256, (chunk + 31) / 32 * 32);
+  chunk = std::max(512, (chunk + 63) / 64 * 64);
   const int n_chunks = (cap + B + chunk - 1) / chunk;
 
   launch_draft_init(anchor, ctx_len, batch, B, c.vocab, c.mask_id, cap, tokens, zrow, lm_rows,
@@ -552,7 +578,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
   int st = DFLASH_OK;
   for (int t = 0; t < n_steps; ++t) {
     const int k = (rem + (n_steps - t) - 1) / (n_steps - t);
-    launch_embed_norm<T>(tokens, static_cast<const T*>(m->emb), m->layers[0].g_in, x, h, M, c.d,
+    launch_embed_norm<TE, T>(tokens, static_cast<const TE*>(m->emb), m->layers[0].g_in, x, h, M, c.d,
                          c.eps, s);
     for (int l = 0; l < c.n_layers; ++l) {
       const LayerPack& P = m->layers[l];
@@ -560,7 +586,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
       if ((st = gemm(P.mqkv, P.Wqkv, qkv_out(c), c.d, h, part, L.part_elems, &sp))) return st;
       launch_qkv_post<T>(part, sp, M, B, ctx_len, valid, nq, nkv, hd, m->rope_cos, m->rope_sin,
                          q, kb, vb, s);
-      if ((st = launch_block_attention<T>(q, kb, vb, kc, vc, l, batch, cap, ctx_len, valid, B, nq,
+      if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, l, batch, cap, ctx_len, valid, B, nq,
                                           nkv, hd, attn_o, attn_ml, n_chunks, chunk, o, s)))
         return st;
       if ((st = gemm(P.mo, P.Wo, c.d, nq * hd, o, part, L.part_elems, &sp))) return st;
@@ -619,9 +645,9 @@ extern "C" int dflash_draft_block(const dflash_model* m, const int32_t* anchor,
   if (ws_bytes < draft_layout(c, batch, B).end) return DFLASH_EWORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   if (c.dtype == DFLASH_BF16)
-    return draft_impl<__nv_bfloat16>(m, anchor, ctx_len, k_cache, v_cache, cache_cap, batch, B,
+    return draft_impl<__half, __nv_bfloat16, __nv_bfloat16>(m, anchor, ctx_len, k_cache, v_cache, cache_cap, batch, B,
                                      n_steps, draft_tokens, commit_step, logits_dbg, ws, s);
-  return draft_impl<float>(m, anchor, ctx_len, k_cache, v_cache, cache_cap, batch, B, n_steps,
+  return draft_impl<float, float, float>(m, anchor, ctx_len, k_cache, v_cache, cache_cap, batch, B, n_steps,
                            draft_tokens, commit_step, logits_dbg, ws, s);
 }
 
@@ -649,13 +675,14 @@ extern "C" int dflash_verify(const void* target_logits, int logits_dtype,
 // ============================================================== test hooks (dflash_debug.h)
 #include "../../include/dflash_debug.h"
 
-extern "C" int dflash_debug_gemm_bf16(const void* W, int N, int K, const void* X, int M,
-                                      int splits, float* out, int* splits_used, void* err_ws,
-                                      void* stream) {
+extern "C" int dflash_debug_gemm(const void* W, int N, int K, const void* X, int M, int elem,
+                                 int splits, float* out, int* splits_used, void* err_ws,
+                                 void* stream) {
   if (!W || !X || !out || !err_ws || N < 1 || K < 64 || K % 64 || M < 1) return DFLASH_EINVAL;
   if (!aligned16(W) || !aligned16(X)) return DFLASH_EINVAL;
   WeightMap wm;
-  if (!encode_weight_map(wm, W, N, K)) return DFLASH_ECUDA;
+  if (elem != DFLASH_BF16 && elem != DFLASH_F16) return DFLASH_EINVAL;
+  if (!encode_weight_map(wm, W, N, K, elem)) return DFLASH_ECUDA;
   splits = gemm_effective_splits(K, splits);
   if (splits_used) *splits_used = splits;
   GemmOut o;
@@ -665,12 +692,13 @@ extern "C" int dflash_debug_gemm_bf16(const void* W, int N, int K, const void* X
                  (cudaStream_t)stream);
 }
 
-extern "C" int dflash_debug_lmhead_bf16(const void* W, int N, int K, const void* X, int M,
-                                        void* stats, float* logits, void* err_ws, void* stream) {
+extern "C" int dflash_debug_lmhead(const void* W, int N, int K, const void* X, int M, int elem,
+                                   void* stats, float* logits, void* err_ws, void* stream) {
   if (!W || !X || !stats || !err_ws || N < 1 || K < 64 || K % 64 || M < 1) return DFLASH_EINVAL;
   if (!aligned16(W) || !aligned16(X)) return DFLASH_EINVAL;
   WeightMap wm;
-  if (!encode_weight_map(wm, W, N, K)) return DFLASH_ECUDA;
+  if (elem != DFLASH_BF16 && elem != DFLASH_F16) return DFLASH_EINVAL;
+  if (!encode_weight_map(wm, W, N, K, elem)) return DFLASH_ECUDA;
   GemmOut o;
   o.stats = static_cast<LmStat*>(stats);
   o.dbg = logits;

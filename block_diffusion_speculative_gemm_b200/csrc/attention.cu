@@ -7,6 +7,8 @@
 // forward).  The key axis is cut into chunks; each CTA (request, kv head,
 // chunk) produces an online-softmax partial (row max m, row sum l, unnormalised
 // o), and a combine kernel merges the chunks in ascending order.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -14,13 +16,13 @@ namespace dflash {
 
 constexpr int kAttnThreads = 128;
 constexpr int kKeyTile = 32;
-constexpr int kMaxRows = 64;  // B * G
+constexpr int kMaxRows = kAttnMaxRows;
 
-template <typename T, int HD>
+template <typename T, typename TC, int HD>
 __global__ void __launch_bounds__(kAttnThreads)
     attn_partial_kernel(const T* __restrict__ q, const T* __restrict__ kb,
-                        const T* __restrict__ vb, const T* __restrict__ kc,
-                        const T* __restrict__ vc, int layer, int batch, int cap,
+                        const T* __restrict__ vb, const TC* __restrict__ kc,
+                        const TC* __restrict__ vc, int layer, int batch, int cap,
                         const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ req_valid,
                         int B, int nq, int nkv, int chunk, int n_chunks,
                         float* __restrict__ part_o, float* __restrict__ part_ml) {
@@ -152,26 +154,30 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o,
   }
 }
 
-template <typename T>
-int launch_block_attention(const T* q, const T* kb, const T* vb, const T* kc, const T* vc,
+template <typename T, typename TC>
+int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, const TC* vc,
                            int layer, int batch, int cap, const int32_t* ctx_len,
                            const int32_t* req_valid, int B, int nq, int nkv, int hd,
                            float* part_o, float* part_ml, int n_chunks, int chunk, T* o,
                            cudaStream_t s) {
   if (B * (nq / nkv) > kMaxRows) return DFLASH_EUNSUPPORTED;
   dim3 grid(n_chunks, nkv, batch);
-  {
+  if constexpr (std::is_same<T, __half>::value) {
+    const int st = launch_attn_partial_tc(q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid,
+                                          B, nq, nkv, hd, chunk, n_chunks, part_o, part_ml, s);
+    if (st != DFLASH_OK) return st;
+  } else {
     TimedScope ts(s, TC_ATTN);
     if (hd == 128) {
       const size_t sm = (kMaxRows * 128 + kKeyTile * 129 + kKeyTile * 128) * sizeof(float);
-      cudaFuncSetAttribute(attn_partial_kernel<T, 128>,
+      cudaFuncSetAttribute(attn_partial_kernel<T, TC, 128>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-      attn_partial_kernel<T, 128><<<grid, kAttnThreads, sm, s>>>(
+      attn_partial_kernel<T, TC, 128><<<grid, kAttnThreads, sm, s>>>(
           q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks,
           part_o, part_ml);
     } else if (hd == 64) {
       const size_t sm = (kMaxRows * 64 + kKeyTile * 65 + kKeyTile * 64) * sizeof(float);
-      attn_partial_kernel<T, 64><<<grid, kAttnThreads, sm, s>>>(
+      attn_partial_kernel<T, TC, 64><<<grid, kAttnThreads, sm, s>>>(
           q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks,
           part_o, part_ml);
     } else {
@@ -191,15 +197,14 @@ int launch_block_attention(const T* q, const T* kb, const T* vb, const T* kc, co
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 
-template int launch_block_attention<float>(const float*, const float*, const float*, const float*,
-                                           const float*, int, int, int, const int32_t*,
-                                           const int32_t*, int, int, int, int, float*, float*, int,
-                                           int, float*, cudaStream_t);
-template int launch_block_attention<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
-                                                   const __nv_bfloat16*, const __nv_bfloat16*,
-                                                   const __nv_bfloat16*, int, int, int,
-                                                   const int32_t*, const int32_t*, int, int, int,
-                                                   int, float*, float*, int, int, __nv_bfloat16*,
-                                                   cudaStream_t);
+template int launch_block_attention<float, float>(const float*, const float*, const float*,
+                                                  const float*, const float*, int, int, int,
+                                                  const int32_t*, const int32_t*, int, int, int,
+                                                  int, float*, float*, int, int, float*,
+                                                  cudaStream_t);
+template int launch_block_attention<__half, __nv_bfloat16>(
+    const __half*, const __half*, const __half*, const __nv_bfloat16*, const __nv_bfloat16*, int,
+    int, int, const int32_t*, const int32_t*, int, int, int, int, float*, float*, int, int,
+    __half*, cudaStream_t);
 
 }  // namespace dflash

@@ -41,6 +41,7 @@ struct GemmArgs {
   int kb_per_split;   // 64-wide k-blocks per split
   int n_kb;           // total k-blocks
   int n_vtiles;       // LM head: number of 128-row vocabulary tiles
+  uint32_t idesc;     // tcgen05 instruction descriptor (operand type, 128 x BN)
   GemmOut out;
   int32_t* err;
 };
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(128, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kTileN, a.BN);
+      const uint32_t idesc = a.idesc;
       for (int i = 0; i < nk; ++i) {
         const int s = i % a.stages;
         const uint32_t ph = (i / a.stages) & 1;
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(128, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kTileK / 16; ++kk) {
-          umma_bf16(tmem, smem_desc_sw128(sA(s) + kk * 32), smem_desc_sw128(sB(s) + kk * 32),
+          umma_f16(tmem, smem_desc_sw128(sA(s) + kk * 32), smem_desc_sw128(sB(s) + kk * 32),
                     idesc, (i | kk) != 0 ? 1u : 0u);
         }
         umma_commit(empty(s));
@@ -226,26 +227,32 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// 2D bf16 tensor map: `rows` rows of `cols` elements, row stride `ld` elements,
-// box = 64 columns x box_rows rows, 128-byte swizzle, zero fill outside.
-static bool encode_2d(CUtensorMap* m, const void* ptr, int rows, int cols, int ld, int box_rows) {
+// 2D 16-bit tensor map (bf16 or fp16): `rows` rows of `cols` elements, row
+// stride `ld` elements, box = 64 columns x box_rows rows, 128-byte swizzle,
+// zero fill outside.
+static bool encode_2d(CUtensorMap* m, const void* ptr, int rows, int cols, int ld, int box_rows,
+                      int elem) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
   cuuint32_t box[2] = {(cuuint32_t)kTileK, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+  const CUtensorMapDataType dt =
+      elem == DFLASH_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = enc(m, dt, 2, const_cast<void*>(ptr), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-bool encode_weight_map(WeightMap& w, const void* ptr, int N, int K) {
+bool encode_weight_map(WeightMap& w, const void* ptr, int N, int K, int elem) {
+  if (elem != DFLASH_BF16 && elem != DFLASH_F16) return false;
   w.ptr = ptr;
   w.N = N;
   w.K = K;
-  return encode_2d(&w.map, ptr, N, K, K, kTileN);
+  w.elem = elem;
+  return encode_2d(&w.map, ptr, N, K, K, kTileN, elem);
 }
 
 int gemm_effective_splits(int K, int splits) {
@@ -294,7 +301,7 @@ int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, i
   BMaps maps;
   memset(&maps, 0, sizeof(maps));
   for (int i = 0; i < n_seg; ++i)
-    if (!encode_2d(&maps.m[i], xseg[i], M, seg_k, ld_seg, BN)) return DFLASH_ECUDA;
+    if (!encode_2d(&maps.m[i], xseg[i], M, seg_k, ld_seg, BN, W.elem)) return DFLASH_ECUDA;
 
   GemmArgs a;
   a.N = W.N;
@@ -310,6 +317,7 @@ int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, i
   splits = gemm_effective_splits(W.K, splits);
   a.kb_per_split = (a.n_kb + splits - 1) / splits;
   a.n_vtiles = (W.N + kTileN - 1) / kTileN;
+  a.idesc = idesc_f16kind(kTileN, BN, W.elem == DFLASH_BF16);
   a.out = out;
   a.err = err;
 

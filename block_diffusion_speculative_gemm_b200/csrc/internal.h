@@ -46,17 +46,20 @@ struct GemmOut {
   int64_t dbg_ld = 0;             // dbg row stride (elements)
 };
 
-// A weight operand prepared once: tensor map over [N, K] bf16 rows.
+// A weight operand prepared once: tensor map over [N, K] rows of 16-bit
+// elements (elem = DFLASH_BF16 or DFLASH_F16).  The activation operand of a
+// GEMM against it must have the same element type.
 struct WeightMap {
   CUtensorMap map;
   const void* ptr = nullptr;
   int N = 0, K = 0;
+  int elem = DFLASH_BF16;
 };
 
-bool encode_weight_map(WeightMap& w, const void* ptr, int N, int K);
+bool encode_weight_map(WeightMap& w, const void* ptr, int N, int K, int elem);
 
-// Y = X * W^T for bf16 X [M, K] (given as n_seg K-segments of seg_k columns,
-// each [M, seg_k] with row stride ld_seg elements) and W [N, K].
+// Y = X * W^T for X [M, K] of W's element type (given as n_seg K-segments of
+// seg_k columns, each [M, seg_k] with row stride ld_seg elements) and W [N, K].
 int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, int ld_seg, int M,
             int splits, int epi, const GemmOut& out, int32_t* err, cudaStream_t s);
 
@@ -72,8 +75,8 @@ void gemm_simt_f32(const float* W, int N, int K, const float* const* xseg, int n
                    int M, float* out, cudaStream_t s);
 
 // ---------------------------------------------------------------- row kernels
-template <typename T>
-void launch_embed_norm(const int32_t* tokens, const T* emb, const float* g, float* x, T* h, int M,
+template <typename TE, typename T>
+void launch_embed_norm(const int32_t* tokens, const TE* emb, const float* g, float* x, T* h, int M,
                        int d, float eps, cudaStream_t s);
 template <typename T>
 void launch_residual_norm(const float* part, int splits, int M, int d, float* x, const float* g,
@@ -94,8 +97,18 @@ void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int 
                        int32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- attention
-template <typename T>
-int launch_block_attention(const T* q, const T* kb, const T* vb, const T* kc, const T* vc,
+constexpr int kAttnMaxRows = 64;  // B * (n_q / n_kv) query rows per (request, kv head)
+
+// Split-KV partials of the tensor-core attention (fp16 block rows, bf16 cache):
+// part_o [batch][nkv][n_chunks][kAttnMaxRows][hd] fp32, part_ml [...][2] (max, sum).
+int launch_attn_partial_tc(const __half* q, const __half* kb, const __half* vb,
+                           const __nv_bfloat16* kc, const __nv_bfloat16* vc, int layer, int batch,
+                           int cap, const int32_t* ctx_len, const int32_t* req_valid, int B,
+                           int nq, int nkv, int hd, int chunk, int n_chunks, float* part_o,
+                           float* part_ml, cudaStream_t s);
+// T: type of q, the block's k/v and the output o; TC: K/V cache type.
+template <typename T, typename TC>
+int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, const TC* vc,
                            int layer, int batch, int cap, const int32_t* ctx_len,
                            const int32_t* req_valid, int B, int nq, int nkv, int hd,
                            float* part_o, float* part_ml, int n_chunks, int chunk, T* o,

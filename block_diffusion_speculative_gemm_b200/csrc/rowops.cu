@@ -20,15 +20,15 @@ __device__ __forceinline__ float sum_splits(const float* part, int splits, size_
 
 // ---------------------------------------------------------------- embedding + RMSNorm
 // x[m] = emb[tokens[m]] (fp32 residual stream); h[m] = RMSNorm(x[m]; g).
-template <typename T>
+template <typename TE, typename T>
 __global__ void __launch_bounds__(kRowThreads)
-    embed_norm_kernel(const int32_t* __restrict__ tokens, const T* __restrict__ emb,
+    embed_norm_kernel(const int32_t* __restrict__ tokens, const TE* __restrict__ emb,
                       const float* __restrict__ g, float* __restrict__ x, T* __restrict__ h, int d,
                       float eps) {
   __shared__ float red[32];
   const int m = blockIdx.x;
   const int tok = tokens[m];
-  const T* e = emb + (size_t)tok * d;
+  const TE* e = emb + (size_t)tok * d;
   float v[kMaxRowElems];
   float ss = 0.f;
 #pragma unroll
@@ -48,12 +48,12 @@ __global__ void __launch_bounds__(kRowThreads)
   }
 }
 
-template <typename T>
-void launch_embed_norm(const int32_t* tokens, const T* emb, const float* g, float* x, T* h, int M,
+template <typename TE, typename T>
+void launch_embed_norm(const int32_t* tokens, const TE* emb, const float* g, float* x, T* h, int M,
                        int d, float eps, cudaStream_t s) {
   if (M <= 0) return;
   TimedScope ts(s, TC_ROW);
-  embed_norm_kernel<T><<<M, kRowThreads, 0, s>>>(tokens, emb, g, x, h, d, eps);
+  embed_norm_kernel<TE, T><<<M, kRowThreads, 0, s>>>(tokens, emb, g, x, h, d, eps);
 }
 
 // ---------------------------------------------------------------- residual + RMSNorm
@@ -269,9 +269,8 @@ void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int 
                                             batch, cap, cos_t, sin_t, max_pos, kc, vc, err);
 }
 
-#define DFLASH_INST(T)                                                                           \
-  template void launch_embed_norm<T>(const int32_t*, const T*, const float*, float*, T*, int, int, \
-                                     float, cudaStream_t);                                       \
+// T: activation type (GEMM operand); TC: K/V cache type; TE: embedding type.
+#define DFLASH_INST_A(T)                                                                         \
   template void launch_residual_norm<T>(const float*, int, int, int, float*, const float*, T*,   \
                                         const int32_t*, float, cudaStream_t);                    \
   template void launch_ctx_norm<T>(const float*, int, int, int, const float*, T*, float,         \
@@ -279,12 +278,20 @@ void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int 
   template void launch_qkv_post<T>(const float*, int, int, int, const int32_t*, const int32_t*,  \
                                    int, int, int, const float*, const float*, T*, T*, T*,        \
                                    cudaStream_t);                                                \
-  template void launch_swiglu<T>(const float*, int, int, int, T*, cudaStream_t);                 \
-  template void launch_kv_scatter<T>(const float*, int, int, int, int, int, int, const int32_t*, \
-                                     const int32_t*, int, int, const float*, const float*, int,  \
-                                     T*, T*, int32_t*, cudaStream_t);
+  template void launch_swiglu<T>(const float*, int, int, int, T*, cudaStream_t);
+#define DFLASH_INST_C(TC)                                                                        \
+  template void launch_kv_scatter<TC>(const float*, int, int, int, int, int, int,                \
+                                      const int32_t*, const int32_t*, int, int, const float*,    \
+                                      const float*, int, TC*, TC*, int32_t*, cudaStream_t);
 
-DFLASH_INST(float)
-DFLASH_INST(__nv_bfloat16)
+DFLASH_INST_A(float)
+DFLASH_INST_A(__half)
+DFLASH_INST_C(float)
+DFLASH_INST_C(__nv_bfloat16)
+template void launch_embed_norm<float, float>(const int32_t*, const float*, const float*, float*,
+                                              float*, int, int, float, cudaStream_t);
+template void launch_embed_norm<__nv_bfloat16, __half>(const int32_t*, const __nv_bfloat16*,
+                                                       const float*, float*, __half*, int, int,
+                                                       float, cudaStream_t);
 
 }  // namespace dflash

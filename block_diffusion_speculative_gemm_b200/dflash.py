@@ -22,7 +22,7 @@ HEADERS = [HEADER, os.path.join(os.path.dirname(_HERE), "include", "dflash_debug
 
 OK, EINVAL, EUNSUPPORTED, ECUDA, ENOMEM, EWORKSPACE = 0, -1, -2, -3, -4, -5
 DEV_CTX_CAP, DEV_OUT_CAP, DEV_TOKEN_RANGE, DEV_TIMEOUT, DEV_ROWS = 1, 2, 4, 8, 16
-F32, BF16 = 0, 1
+F32, BF16, F16 = 0, 1, 2
 TIMING_CLASSES = ("gemm", "attention", "row", "verify", "lm_head")
 
 
@@ -80,9 +80,9 @@ def lib() -> ctypes.CDLL:
         L.dflash_timing_enable.argtypes = [i32]
         L.dflash_timing_read.argtypes = [ctypes.POINTER(ctypes.c_double),
                                          ctypes.POINTER(ctypes.c_int64), i32]
-        L.dflash_debug_gemm_bf16.argtypes = [vp, i32, i32, vp, i32, i32, vp,
-                                             ctypes.POINTER(ctypes.c_int), vp, vp]
-        L.dflash_debug_lmhead_bf16.argtypes = [vp, i32, i32, vp, i32, vp, vp, vp, vp]
+        L.dflash_debug_gemm.argtypes = [vp, i32, i32, vp, i32, i32, i32, vp,
+                                        ctypes.POINTER(ctypes.c_int), vp, vp]
+        L.dflash_debug_lmhead.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp, vp, vp]
         _lib = L
     return _lib
 
@@ -293,10 +293,15 @@ def timing_read() -> Dict[str, Dict[str, float]]:
 
 # ---------------------------------------------------------------- test hooks (dflash_debug.h)
 
+_ELEM = {torch.bfloat16: BF16, torch.float16: F16}
+
+
 def debug_gemm(W: torch.Tensor, X: torch.Tensor, splits: int, err_ws: torch.Tensor, stream=None):
-    """fp32 split-K partials [splits_used, M, N] of X @ W^T from the tcgen05 core."""
-    _need(W, "W", torch.bfloat16)
-    _need(X, "X", torch.bfloat16)
+    """fp32 split-K partials [splits_used, M, N] of X @ W^T from the tcgen05 core
+    (W and X both bf16 or both fp16)."""
+    _need(W, "W")
+    _need(X, "X", W.dtype)
+    elem = _ELEM[W.dtype]
     N, K = W.shape
     M = X.shape[0]
     nkb = K // 64
@@ -305,8 +310,8 @@ def debug_gemm(W: torch.Tensor, X: torch.Tensor, splits: int, err_ws: torch.Tens
     s_used = -(-nkb // per)
     out = torch.empty((s_used, M, N), dtype=torch.float32, device=W.device)
     used = ctypes.c_int(0)
-    _check("dflash_debug_gemm_bf16", lib().dflash_debug_gemm_bf16(
-        _ptr(W), N, K, _ptr(X), M, s_req, _ptr(out), ctypes.byref(used), _ptr(err_ws),
+    _check("dflash_debug_gemm", lib().dflash_debug_gemm(
+        _ptr(W), N, K, _ptr(X), M, elem, s_req, _ptr(out), ctypes.byref(used), _ptr(err_ws),
         _stream(stream)))
     assert used.value == s_used
     return out
@@ -315,13 +320,14 @@ def debug_gemm(W: torch.Tensor, X: torch.Tensor, splits: int, err_ws: torch.Tens
 def debug_lmhead(W: torch.Tensor, X: torch.Tensor, err_ws: torch.Tensor, want_logits=True,
                  stream=None):
     """(stats [M, tiles, 4] as (max, idx, sumexp, 0), logits [M, N] or None)."""
-    _need(W, "W", torch.bfloat16)
-    _need(X, "X", torch.bfloat16)
+    _need(W, "W")
+    _need(X, "X", W.dtype)
+    elem = _ELEM[W.dtype]
     N, K = W.shape
     M = X.shape[0]
     tiles = -(-N // 128)
     stats = torch.empty((M, tiles, 4), dtype=torch.float32, device=W.device)
     logits = torch.empty((M, N), dtype=torch.float32, device=W.device) if want_logits else None
-    _check("dflash_debug_lmhead_bf16", lib().dflash_debug_lmhead_bf16(
-        _ptr(W), N, K, _ptr(X), M, _ptr(stats), _ptr(logits), _ptr(err_ws), _stream(stream)))
+    _check("dflash_debug_lmhead", lib().dflash_debug_lmhead(
+        _ptr(W), N, K, _ptr(X), M, elem, _ptr(stats), _ptr(logits), _ptr(err_ws), _stream(stream)))
     return stats, logits

@@ -69,6 +69,7 @@ extern "C" {
 /* ---- element types ---------------------------------------------------- */
 #define DFLASH_F32  0
 #define DFLASH_BF16 1
+#define DFLASH_F16  2  /* operand type of the test hooks in dflash_debug.h only */
 
 typedef struct dflash_model dflash_model; /* opaque */
 

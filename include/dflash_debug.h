@@ -16,19 +16,21 @@ extern "C" {
 #endif
 
 /* out[s][m][n] = sum over split s's K range of X[m][k] * W[n][k].
- * W: device bf16 [N, K]; X: device bf16 [M, K]; K % 64 == 0; 16-byte aligned
- * rows (K % 8 == 0).  out: device fp32 [splits][M][N].  The split count is
- * clamped to [1, K/64]; the count used is written to *splits_used.
- * err_ws: a zero-filled 256-byte device block that receives device error bits. */
-int dflash_debug_gemm_bf16(const void* W, int N, int K, const void* X, int M, int splits,
-                           float* out, int* splits_used, void* err_ws, void* stream);
+ * W: device [N, K]; X: device [M, K]; both of element type elem (DFLASH_BF16 or
+ * DFLASH_F16); K % 64 == 0; 16-byte aligned.  out: device fp32
+ * [splits][M][N].  The split count is clamped to [1, K/64] and rounded so that
+ * every split but the last has the same number of 64-wide K blocks; the count
+ * used is written to *splits_used.  err_ws: a zero-filled 256-byte device
+ * block that receives device error bits. */
+int dflash_debug_gemm(const void* W, int N, int K, const void* X, int M, int elem, int splits,
+                      float* out, int* splits_used, void* err_ws, void* stream);
 
 /* LM-head epilogue: for every token row m and 128-row weight tile t,
  * stats[m][t] = {max_n logit, argmax n (lowest), sum exp(logit - max), 0}
  * (16 bytes per entry); logits (device fp32 [M, N]) receives the raw products
  * when not NULL. */
-int dflash_debug_lmhead_bf16(const void* W, int N, int K, const void* X, int M, void* stats,
-                             float* logits, void* err_ws, void* stream);
+int dflash_debug_lmhead(const void* W, int N, int K, const void* X, int M, int elem, void* stats,
+                        float* logits, void* err_ws, void* stream);
 
 #ifdef __cplusplus
 }

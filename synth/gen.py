@@ -170,10 +170,12 @@ def _bf16_step(x: torch.Tensor, up: bool) -> torch.Tensor:
 
 
 def make_verify_case(b: int, B: int, V: int, label: str, plant=("uniform",), dtype: str = "bf16",
-                     adversarial: bool = False, raise_by: float = 8.0, master: int = MASTER_SEED):
+                     adversarial: bool = False, raise_by: float = 8.0, master: int = MASTER_SEED,
+                     draft: Optional[torch.Tensor] = None):
     """Target logits [b, B, V] ~ N(0,1) with planted accept prefixes.
 
-    Draft tokens are uniform over the vocabulary.  For rows i < a_r the draft
+    Draft tokens are uniform over the vocabulary unless ``draft`` supplies
+    them (e.g. a drafted block the logits should partly agree with).  For rows i < a_r the draft
     token d[i+1] gets its logit raised by ``raise_by``; at row a_r (if a_r < B-1)
     d[a_r+1] is lowered to the row minimum.  With ``adversarial`` some planted
     rows instead put d[i+1] one bf16 ulp above or below the row maximum, or
@@ -185,7 +187,8 @@ def make_verify_case(b: int, B: int, V: int, label: str, plant=("uniform",), dty
     g = _gen(seed)
     dt = _dtype(dtype)
     logits = torch.randn((b, B, V), generator=g).to(dt)
-    draft = torch.randint(0, V, (b, B), generator=g, dtype=torch.int64).to(torch.int32)
+    rnd = torch.randint(0, V, (b, B), generator=g, dtype=torch.int64).to(torch.int32)
+    draft = rnd if draft is None else draft.to(torch.int32).cpu().clone()
     plants = sample_plants(plant, b, B, sub_seed(seed, "plant"))
     modes = torch.randint(0, 5, (b, B), generator=g)
     others = torch.randint(0, V, (b, B), generator=g)

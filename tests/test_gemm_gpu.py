@@ -8,10 +8,10 @@ from block_diffusion_speculative_gemm_b200 import dflash as D
 pytestmark = pytest.mark.gpu
 
 
-def _inputs(N, K, M, seed):
+def _inputs(N, K, M, seed, dtype=torch.bfloat16):
     g = torch.Generator().manual_seed(seed)
-    W = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
-    X = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g) * 0.05).to(dtype)
+    X = torch.randn(M, K, generator=g).to(dtype)
     return W, X
 
 
@@ -24,8 +24,9 @@ def _inputs(N, K, M, seed):
     (128, 192, 1, 5),        # one token row, more splits than fit evenly
     (6144, 4096, 256, 3),    # QKV projection of the 8B-shaped draft
 ])
-def test_gemm_matches_float64(N, K, M, splits):
-    W, X = _inputs(N, K, M, N * 7 + K + M)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_gemm_matches_float64(N, K, M, splits, dtype):
+    W, X = _inputs(N, K, M, N * 7 + K + M, dtype)
     err = D.new_workspace(256)
     out = D.debug_gemm(W.cuda(), X.cuda(), splits, err)
     torch.cuda.synchronize()
@@ -43,8 +44,9 @@ def test_gemm_matches_float64(N, K, M, splits):
 
 
 @pytest.mark.parametrize("N,K,M", [(1024, 256, 40), (151936 // 16, 512, 224), (2000, 128, 96)])
-def test_lmhead_epilogue_stats(N, K, M):
-    W, X = _inputs(N, K, M, N + K + M)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_lmhead_epilogue_stats(N, K, M, dtype):
+    W, X = _inputs(N, K, M, N + K + M, dtype)
     err = D.new_workspace(256)
     stats, logits = D.debug_lmhead(W.cuda(), X.cuda(), err)
     torch.cuda.synchronize()
