@@ -155,13 +155,16 @@ def run_dflash(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     cfg = synth.get_config(WORKLOAD)
+    if args.layers:
+        # profiling variant: the same per-layer shapes with fewer layers (smaller footprint)
+        cfg = cfg.replace(L=args.layers, name=f"{WORKLOAD}_L{args.layers}")
     b, B, V = cfg.batch, cfg.B, cfg.V
     cap = cfg.cache_cap
     w = synth.make_weights(cfg)
     model = D.Model(cfg, to_device(w, dev), cap + 2 * B + 16)
     ctx = synth.make_ctx_lens(cfg)
     anchors = synth.make_anchors(cfg)
-    kc = torch.zeros((cfg.L, b, cfg.nkv, cap, cfg.hd), dtype=torch.bfloat16, device=dev)
+    kc = torch.zeros((cfg.L, b, cfg.nkv, cap, cfg.hd), dtype=model.cache_dtype, device=dev)
     vc = torch.zeros_like(kc)
 
     # prefix: inject every context position once (tapped hiddens drawn on the device)
@@ -269,7 +272,7 @@ def run_dflash(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded random-init weights and inputs)",
-        "config": {"workload": WORKLOAD, "model": "Qwen3-8B-shaped DFlash draft (5 layers)",
+        "config": {"workload": cfg.name, "model": f"Qwen3-8B-shaped DFlash draft ({cfg.L} layers)",
                    "global_batch": b * world, "block": B, "denoise_steps": cfg.steps,
                    "ctx": "uniform[512,4096]", "inject_rows": n_s, "parallelism": f"dp{world}",
                    "l2": "no flush: every step streams ~7.4 GB of weights and K/V (> 126 MB L2)"},
@@ -464,6 +467,8 @@ def main():
     ap.add_argument("--impl", default="dflash", choices=["dflash", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling only: override the draft layer count")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

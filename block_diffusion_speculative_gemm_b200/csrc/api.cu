@@ -493,10 +493,10 @@ extern "C" int dflash_inject_kv(const dflash_model* m, const void* const* taps,
       const void* cseg[1] = {cbuf};
       st = gemm_tc(m->mkv, cseg, 1, c.d, c.d, n, s2, EPI_PARTIAL, o, err, s);
       if (st) return st;
-      launch_kv_scatter<__nv_bfloat16>(part, s2, n, r0, c.n_layers, c.n_kv, c.head_dim, cu_rows,
+      launch_kv_scatter<__half>(part, s2, n, r0, c.n_layers, c.n_kv, c.head_dim, cu_rows,
                                        start_pos, batch, cache_cap, m->rope_cos, m->rope_sin,
-                                       c.max_pos, static_cast<__nv_bfloat16*>(k_cache),
-                                       static_cast<__nv_bfloat16*>(v_cache), err, s);
+                                       c.max_pos, static_cast<__half*>(k_cache),
+                                       static_cast<__half*>(v_cache), err, s);
     } else {
       const float* fseg[kMaxSeg];
       for (int t = 0; t < c.n_tap; ++t) fseg[t] = static_cast<const float*>(seg[t]);
@@ -586,8 +586,9 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
       if ((st = gemm(P.mqkv, P.Wqkv, qkv_out(c), c.d, h, part, L.part_elems, &sp))) return st;
       launch_qkv_post<T>(part, sp, M, B, ctx_len, valid, nq, nkv, hd, m->rope_cos, m->rope_sin,
                          q, kb, vb, s);
-      if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, l, batch, cap, ctx_len, valid, B, nq,
-                                          nkv, hd, attn_o, attn_ml, n_chunks, chunk, o, s)))
+      if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, l, c.n_layers, batch, cap, ctx_len,
+                                              valid, B, nq, nkv, hd, attn_o, attn_ml, n_chunks,
+                                              chunk, o, err, s)))
         return st;
       if ((st = gemm(P.mo, P.Wo, c.d, nq * hd, o, part, L.part_elems, &sp))) return st;
       launch_residual_norm<T>(part, sp, M, c.d, x, P.g_post, h, nullptr, c.eps, s);
@@ -645,7 +646,7 @@ extern "C" int dflash_draft_block(const dflash_model* m, const int32_t* anchor,
   if (ws_bytes < draft_layout(c, batch, B).end) return DFLASH_EWORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   if (c.dtype == DFLASH_BF16)
-    return draft_impl<__half, __nv_bfloat16, __nv_bfloat16>(m, anchor, ctx_len, k_cache, v_cache, cache_cap, batch, B,
+    return draft_impl<__half, __half, __nv_bfloat16>(m, anchor, ctx_len, k_cache, v_cache, cache_cap, batch, B,
                                      n_steps, draft_tokens, commit_step, logits_dbg, ws, s);
   return draft_impl<float, float, float>(m, anchor, ctx_len, k_cache, v_cache, cache_cap, batch, B, n_steps,
                            draft_tokens, commit_step, logits_dbg, ws, s);

@@ -1,21 +1,19 @@
-// Tensor-core block-vs-context attention (split-KV partials) for fp16 block
-// activations over a bf16 K/V cache.
+// Tensor-core block-vs-context attention (split-KV partials), fp16 rows over
+// an fp16 K/V cache.
 //
-// A CTA handles (key chunk, kv head, request) with 4 warps.  The chunk's keys
-// -- cache positions below T_r, then the block's own B keys -- are streamed in
-// 64-key tiles through a 3-stage cp.async ring of 16-byte copies, each key row
-// XOR-swizzled in 16-byte units so that ldmatrix reads are conflict-free.
-// Cache rows arrive as bf16 and are rewritten as fp16 in shared memory by the
-// thread that copied them (exact for the cache's value range), so every
-// product is an fp16 x fp16 -> fp32 mma.sync.m16n8k16.  Warp (mt, kg) owns
-// query rows [16 mt, 16 mt + 16) and key group kg of every tile; it keeps the
-// online-softmax state (row max m, row sum l, unnormalised O) in registers.
-// The key groups of a row tile are merged through shared memory and one
-// (m, l, O) partial per query row is written; a combine kernel merges chunks.
+// A CTA handles (key chunk, kv head, request) with 4 warps.  Context keys of
+// the chunk (cache positions below T_r) arrive in 64-key tiles by TMA: per
+// tile two 64-column boxes of K and of V (128-byte swizzled), completing on a
+// per-stage mbarrier, issued one thread ahead of the consumers through a
+// 3-stage ring.  The block's own keys (at most 16) come last, as a small tile
+// copied with cp.async into the query area once the query fragments are in
+// registers.  Warp (mt, kg) owns query rows [16 mt, 16 mt + 16) and key group
+// kg of every tile: S = Q K^T and O += P V run as fp16 mma.sync.m16n8k16 with
+// fp32 accumulation; the online softmax (row max m, row sum l) is updated once
+// per tile.  Key groups are merged through shared memory and one (m, l, O)
+// partial per query row and chunk is written; a combine kernel merges chunks.
 //
-// Memory-bound at 2 * 4 * B * G flop per cache byte: the cache is read once,
-// in 512-byte rows per key per matrix, and every stage is in flight while the
-// previous tiles are multiplied.
+// Memory-bound: 4 * B * G flop per cache byte read, every cache byte read once.
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,7 +22,8 @@ namespace dflash {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kKeys = 64;    // keys per tile
+constexpr int kKeys = 64;    // keys per context tile
+constexpr int kBlkKeys = 16; // rows of the block tile
 constexpr int kStages = 3;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
@@ -35,9 +34,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int sr
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
@@ -65,107 +66,176 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int HD>
-struct Layout {
-  static constexpr int kRowBytes = HD * 2;
-  static constexpr int kChunks = kRowBytes / 16;      // 16-byte chunks per key row
-  static constexpr int kTileBytes = kKeys * kRowBytes;  // K or V of one tile
-  static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kQBytes = kAttnMaxRows * kRowBytes;
-  static constexpr int kSmem = kStages * kStageBytes + kQBytes;
-  __device__ static __forceinline__ uint32_t off(int row, int ch) {
-    return (uint32_t)(row * kRowBytes + ((ch ^ (row & 7)) << 4));
-  }
-};
+// A tile of `rows` key rows of HD fp16 is stored as HD/64 column halves; each
+// half is [rows][128 bytes] with 16-byte chunk j of row r at chunk j ^ (r & 7)
+// (the 128-byte TMA swizzle).  Chunk c of a row (8 elements) is in half c / 8.
+__device__ __forceinline__ uint32_t toff(int rows, int row, int c) {
+  return (uint32_t)((c >> 3) * rows * 128 + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+}
 
 template <int HD>
+struct Layout {
+  static constexpr int kTile = kKeys * HD * 2;       // K or V of one context tile
+  static constexpr int kStage = 2 * kTile;
+  static constexpr int kQ = kAttnMaxRows * HD * 2;   // query rows, later the block tile
+  static constexpr int kBars = kStages * 8;
+  static constexpr int kSmem = kStages * kStage + kQ + kBars + 1024;  // + alignment slack
+  static_assert(2 * kBlkKeys * HD * 2 <= kQ, "block tile fits the query area");
+};
+
+template <int HD, int MT>
+struct Warp {
+  static constexpr int KG = MT == 1 ? 4 : (MT == 2 ? 2 : 1);  // key groups
+  static constexpr int KPW = kKeys / KG;                      // keys per warp per tile
+  static constexpr int NT = HD / 8;
+  static constexpr int KS = HD / 16;
+};
+
+// One tile's worth of keys for one warp: keys [kbeg, kbeg + NKEYS) of a tile
+// stored with `rows` rows; keys at tile-local index >= nvalid are masked.
+template <int HD, int NKEYS>
+__device__ __forceinline__ void attend(uint32_t sK, uint32_t sV, int rows, int kbeg, int nvalid,
+                                       const uint32_t (&qa)[HD / 16][4], float (&o)[HD / 8][4],
+                                       float& m0, float& m1, float& l0, float& l1, float scale,
+                                       int lane) {
+  constexpr int NS = NKEYS / 8;
+  const int tq = lane & 3, mi = lane >> 3, li = lane & 7;
+  float s[NS][4];
+#pragma unroll
+  for (int n = 0; n < NS; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < HD / 16; ++ks) {
+#pragma unroll
+    for (int np = 0; np < NKEYS / 16; ++np) {
+      uint32_t b0, b1, b2, b3;
+      const int row = kbeg + np * 16 + (mi >> 1) * 8 + li;
+      ldsm_x4(sK + toff(rows, row, ks * 2 + (mi & 1)), b0, b1, b2, b3);
+      mma16816(s[2 * np], qa[ks], b0, b1);
+      mma16816(s[2 * np + 1], qa[ks], b2, b3);
+    }
+  }
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+  for (int n = 0; n < NS; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int k = kbeg + n * 8 + 2 * tq + (e & 1);
+      s[n][e] = k < nvalid ? s[n][e] * scale : -INFINITY;
+      if (e < 2) mx0 = fmaxf(mx0, s[n][e]); else mx1 = fmaxf(mx1, s[n][e]);
+    }
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+  const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+  // every key masked (the same for all rows): nothing to add
+  if (__all_sync(0xffffffffu, n0 == -INFINITY && n1 == -INFINITY)) return;
+  const float c0 = (m0 == -INFINITY) ? 0.f : expf(m0 - n0);
+  const float c1 = (m1 == -INFINITY) ? 0.f : expf(m1 - n1);
+  float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+  for (int n = 0; n < NS; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float mref = e < 2 ? n0 : n1;
+      s[n][e] = s[n][e] == -INFINITY ? 0.f : expf(s[n][e] - mref);
+      if (e < 2) ps0 += s[n][e]; else ps1 += s[n][e];
+    }
+  l0 = l0 * c0 + ps0;
+  l1 = l1 * c1 + ps1;
+  m0 = n0;
+  m1 = n1;
+#pragma unroll
+  for (int n = 0; n < HD / 8; ++n) {
+    o[n][0] *= c0;
+    o[n][1] *= c0;
+    o[n][2] *= c1;
+    o[n][3] *= c1;
+  }
+#pragma unroll
+  for (int kb = 0; kb < NKEYS / 16; ++kb) {
+    const uint32_t pa[4] = {pack_h2(s[2 * kb][0], s[2 * kb][1]),
+                            pack_h2(s[2 * kb][2], s[2 * kb][3]),
+                            pack_h2(s[2 * kb + 1][0], s[2 * kb + 1][1]),
+                            pack_h2(s[2 * kb + 1][2], s[2 * kb + 1][3])};
+#pragma unroll
+    for (int nd = 0; nd < HD / 8; nd += 2) {
+      uint32_t b0, b1, b2, b3;
+      const int row = kbeg + kb * 16 + (mi & 1) * 8 + li;
+      ldsm_x4_t(sV + toff(rows, row, nd + (mi >> 1)), b0, b1, b2, b3);
+      mma16816(o[nd], pa, b0, b1);
+      mma16816(o[nd + 1], pa, b2, b3);
+    }
+  }
+}
+
+template <int HD, int MT>
 __global__ void __launch_bounds__(kThreads)
-    attn_tc_kernel(const __half* __restrict__ q, const __half* __restrict__ kb,
-                   const __half* __restrict__ vb, const __nv_bfloat16* __restrict__ kc,
-                   const __nv_bfloat16* __restrict__ vc, int layer, int batch, int cap,
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   const __half* __restrict__ q, const __half* __restrict__ kb,
+                   const __half* __restrict__ vb, int layer, int batch, int cap,
                    const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ req_valid,
                    int B, int nq, int nkv, int chunk, int n_chunks, float* __restrict__ part_o,
-                   float* __restrict__ part_ml) {
+                   float* __restrict__ part_ml, int32_t* err) {
   using LY = Layout<HD>;
-  constexpr int NT = HD / 8;   // n8 tiles of the output row
-  constexpr int KS = HD / 16;  // k16 steps of q.k
-  extern __shared__ __align__(128) uint8_t smem[];
+  using WP = Warp<HD, MT>;
+  constexpr int NT = WP::NT, KS = WP::KS, KG = WP::KG, KPW = WP::KPW;
+  constexpr int HALVES = HD / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
-  const uint32_t s_q = s_base + kStages * LY::kStageBytes;
+  const uint32_t s_q = s_base + kStages * LY::kStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * LY::kStage + LY::kQ);
 
   const int c = blockIdx.x, g = blockIdx.y, r = blockIdx.z;
   const int G = nq / nkv;
   const int R = B * G;
   const int Tc = req_valid[r] ? ctx_len[r] : 0;
-  const int total = Tc + B;
   const int k0 = c * chunk;
-  if (k0 >= total) return;
-  const int k1 = min(total, k0 + chunk);
-  const int ntiles = (k1 - k0 + kKeys - 1) / kKeys;
-  const int MT = (R + 15) / 16;
-  const int KG = (MT == 1) ? 4 : (MT == 2 ? 2 : 1);
-  const int keys_per_warp = kKeys / KG;
+  if (k0 >= Tc + B) return;
+  const int k1 = min(Tc + B, k0 + chunk);
+  const int kc_end = min(k1, Tc);                       // context keys [k0, kc_end)
+  const int nt = kc_end > k0 ? (kc_end - k0 + kKeys - 1) / kKeys : 0;
+  const int kb_lo = max(k0, Tc), kb_hi = min(k1, Tc + B);  // block keys [kb_lo, kb_hi)
+  const int row_base = ((layer * batch + r) * nkv + g) * cap;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mt = warp % MT, kg = warp / MT;
   const bool computes = warp < MT * KG;
-  const size_t cache_base = (((size_t)layer * batch + r) * nkv + g) * (size_t)cap * HD;
 
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(bars + s), 1);
+    fence_barrier_init();
+  }
   // query rows of this kv head: row i = (block position i / G, head g*G + i % G)
-  for (int idx = tid; idx < MT * 16 * LY::kChunks; idx += kThreads) {
-    const int row = idx / LY::kChunks, ch = idx % LY::kChunks;
+  for (int idx = tid; idx < MT * 16 * (HD / 8); idx += kThreads) {
+    const int row = idx / (HD / 8), ch = idx % (HD / 8);
     const void* src = q;
     int bytes = 0;
     if (row < R) {
       src = q + ((size_t)(r * B + row / G) * nq + g * G + row % G) * HD + ch * 8;
       bytes = 16;
     }
-    cp_async16(s_q + LY::off(row, ch), src, bytes);
+    cp_async16(s_q + toff(kAttnMaxRows, row, ch), src, bytes);
   }
+  cp_async_commit();
+  __syncthreads();  // barrier init visible before any wait
 
-  auto load_tile = [&](int t, int st) {
-    const uint32_t sb = s_base + st * LY::kStageBytes;
-    for (int idx = tid; idx < 2 * kKeys * LY::kChunks; idx += kThreads) {
-      const int mat = idx / (kKeys * LY::kChunks);
-      const int rem = idx % (kKeys * LY::kChunks);
-      const int row = rem / LY::kChunks, ch = rem % LY::kChunks;
-      const int key = k0 + t * kKeys + row;
-      const void* src = kc;
-      int bytes = 0;
-      if (key < Tc) {
-        src = (mat ? vc : kc) + cache_base + (size_t)key * HD + ch * 8;
-        bytes = 16;
-      } else if (key < k1) {
-        src = (mat ? vb : kb) + ((size_t)(r * B + key - Tc) * nkv + g) * HD + ch * 8;
-        bytes = 16;
-      }
-      cp_async16(sb + mat * LY::kTileBytes + LY::off(row, ch), src, bytes);
+  auto issue = [&](int t) {  // one thread: TMA of context tile t into its stage
+    const int st = t % kStages;
+    const uint32_t sK = s_base + st * LY::kStage, sV = sK + LY::kTile;
+    const uint32_t bar = smem_u32(bars + st);
+    mbar_arrive_expect_tx(bar, 2 * LY::kTile);
+    const int y = row_base + k0 + t * kKeys;
+#pragma unroll
+    for (int h = 0; h < HALVES; ++h) {
+      tma_load_2d(sK + h * kKeys * 128, &tmK, bar, h * 64, y, policy_evict_first());
+      tma_load_2d(sV + h * kKeys * 128, &tmV, bar, h * 64, y, policy_evict_first());
     }
   };
-  // cache rows were copied as bf16: the copying thread rewrites its chunks as fp16
-  auto convert_tile = [&](int t, int st) {
-    uint8_t* sb = smem + st * LY::kStageBytes;
-    for (int idx = tid; idx < 2 * kKeys * LY::kChunks; idx += kThreads) {
-      const int mat = idx / (kKeys * LY::kChunks);
-      const int rem = idx % (kKeys * LY::kChunks);
-      const int row = rem / LY::kChunks, ch = rem % LY::kChunks;
-      if (k0 + t * kKeys + row >= Tc) continue;
-      uint4* p = reinterpret_cast<uint4*>(sb + mat * LY::kTileBytes + LY::off(row, ch));
-      uint4 u = *p;
-      uint32_t* w = reinterpret_cast<uint32_t*>(&u);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float lo = __uint_as_float(w[k] << 16);
-        const float hi = __uint_as_float(w[k] & 0xffff0000u);
-        w[k] = pack_h2(lo, hi);
-      }
-      *p = u;
-    }
-  };
-
-#pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
-    if (s < ntiles) load_tile(s, s);
-    cp_async_commit();
+  if (tid == 0) {
+    fence_proxy_async();
+    for (int t = 0; t < kStages - 1 && t < nt; ++t) issue(t);
   }
 
   uint32_t qa[KS][4];
@@ -174,100 +244,80 @@ __global__ void __launch_bounds__(kThreads)
   for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   const float scale = rsqrtf((float)HD);
-  const int tq = lane & 3;                  // thread inside an mma row group
-  const int mi = lane >> 3, li = lane & 7;  // ldmatrix: matrix index, row inside it
+  const int mi = lane >> 3, li = lane & 7;
 
-  for (int t = 0; t < ntiles; ++t) {
-    const int st = t % kStages;
-    if (t + kStages - 1 < ntiles) load_tile(t + kStages - 1, (t + kStages - 1) % kStages);
+  cp_async_wait_all();
+  __syncthreads();
+  if (computes) {
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int row = mt * 16 + (mi & 1) * 8 + li;
+      ldsm_x4(s_q + toff(kAttnMaxRows, row, ks * 2 + (mi >> 1)), qa[ks][0], qa[ks][1], qa[ks][2],
+              qa[ks][3]);
+    }
+  }
+  __syncthreads();  // the query area now holds the block tile
+  const bool has_blk = kb_hi > kb_lo;
+  if (has_blk) {
+    for (int idx = tid; idx < 2 * kBlkKeys * (HD / 8); idx += kThreads) {
+      const int mat = idx / (kBlkKeys * (HD / 8));
+      const int rem = idx % (kBlkKeys * (HD / 8));
+      const int row = rem / (HD / 8), ch = rem % (HD / 8);
+      const int key = kb_lo + row;
+      const void* src = kb;
+      int bytes = 0;
+      if (key < kb_hi) {
+        src = (mat ? vb : kb) + ((size_t)(r * B + key - Tc) * nkv + g) * HD + ch * 8;
+        bytes = 16;
+      }
+      cp_async16(s_q + mat * (kBlkKeys * HD * 2) + toff(kBlkKeys, row, ch), src, bytes);
+    }
     cp_async_commit();
-    cp_async_wait<kStages - 1>();
-    convert_tile(t, st);
-    __syncthreads();
-    if (t == 0 && computes) {
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        const int row = mt * 16 + (mi & 1) * 8 + li;
-        ldsm_x4(s_q + LY::off(row, ks * 2 + (mi >> 1)), qa[ks][0], qa[ks][1], qa[ks][2],
-                qa[ks][3]);
-      }
+  }
+
+  bool ok = true;
+  for (int t = 0; t < nt; ++t) {
+    const int st = t % kStages;
+    if (tid == 0 && t + kStages - 1 < nt) {
+      fence_proxy_async();
+      issue(t + kStages - 1);
     }
-    if (computes) {
-      const uint32_t sK = s_base + st * LY::kStageBytes;
-      const uint32_t sV = sK + LY::kTileBytes;
-      for (int kb16 = 0; kb16 < keys_per_warp / 16; ++kb16) {
-        const int key0 = kg * keys_per_warp + kb16 * 16;  // tile-local
-        if (k0 + t * kKeys + key0 >= k1) break;           // all 16 keys past the chunk
-        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          uint32_t b0, b1, b2, b3;
-          const int row = key0 + (mi >> 1) * 8 + li;
-          ldsm_x4(sK + LY::off(row, ks * 2 + (mi & 1)), b0, b1, b2, b3);
-          mma16816(s[0], qa[ks], b0, b1);
-          mma16816(s[1], qa[ks], b2, b3);
-        }
-        // scale, mask keys past the chunk, online softmax for rows gq and gq + 8
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int key = k0 + t * kKeys + key0 + n * 8 + 2 * tq + (e & 1);
-            s[n][e] = key < k1 ? s[n][e] * scale : -INFINITY;
-            if (e < 2) mx0 = fmaxf(mx0, s[n][e]); else mx1 = fmaxf(mx1, s[n][e]);
-          }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-        const float c0 = (m0 == -INFINITY) ? 0.f : expf(m0 - n0);
-        const float c1 = (m1 == -INFINITY) ? 0.f : expf(m1 - n1);
-        float p[2][4];
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float mref = e < 2 ? n0 : n1;
-            p[n][e] = s[n][e] == -INFINITY ? 0.f : expf(s[n][e] - mref);
-          }
-        l0 = l0 * c0 + p[0][0] + p[0][1] + p[1][0] + p[1][1];
-        l1 = l1 * c1 + p[0][2] + p[0][3] + p[1][2] + p[1][3];
-        m0 = n0;
-        m1 = n1;
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          o[n][0] *= c0;
-          o[n][1] *= c0;
-          o[n][2] *= c1;
-          o[n][3] *= c1;
-        }
-        const uint32_t pa[4] = {pack_h2(p[0][0], p[0][1]), pack_h2(p[0][2], p[0][3]),
-                                pack_h2(p[1][0], p[1][1]), pack_h2(p[1][2], p[1][3])};
-#pragma unroll
-        for (int nd = 0; nd < NT; nd += 2) {
-          uint32_t b0, b1, b2, b3;
-          const int row = key0 + (mi & 1) * 8 + li;
-          ldsm_x4_t(sV + LY::off(row, nd + (mi >> 1)), b0, b1, b2, b3);
-          mma16816(o[nd], pa, b0, b1);
-          mma16816(o[nd + 1], pa, b2, b3);
-        }
+    if (!mbar_wait(smem_u32(bars + st), (t / kStages) & 1)) ok = false;
+    const int nvalid = min(kKeys, kc_end - (k0 + t * kKeys));
+    const uint32_t sK = s_base + st * LY::kStage, sV = sK + LY::kTile;
+    if (nvalid < kKeys) {
+      // rows past the context hold other cache positions: zero V so that
+      // masked keys contribute exactly nothing
+      uint8_t* v = smem + st * LY::kStage + LY::kTile;
+      for (int idx = tid; idx < (kKeys - nvalid) * (HD / 8); idx += kThreads) {
+        const int row = nvalid + idx / (HD / 8), ch = idx % (HD / 8);
+        *reinterpret_cast<uint4*>(v + toff(kKeys, row, ch)) = make_uint4(0, 0, 0, 0);
       }
+      __syncthreads();
     }
+    if (computes)
+      attend<HD, KPW>(sK, sV, kKeys, kg * KPW, nvalid, qa, o, m0, m1, l0, l1, scale, lane);
     __syncthreads();
   }
-  cp_async_wait<0>();
+  if (!ok && tid == 0) set_error(err, DFLASH_DEV_TIMEOUT);
+  if (has_blk) {
+    cp_async_wait_all();
+    __syncthreads();
+    if (computes && kg == 0)
+      attend<HD, kBlkKeys>(s_q, s_q + kBlkKeys * HD * 2, kBlkKeys, 0, kb_hi - kb_lo, qa, o, m0, m1,
+                           l0, l1, scale, lane);
+  }
 
   // row sums over the quad, then merge the key groups of each row tile
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  float* scratch = reinterpret_cast<float*>(smem);  // stage buffers are idle now
   constexpr int kSlot = NT * 4 + 4;
-  static_assert(4 * 32 * kSlot * 4 <= kStages * Layout<HD>::kStageBytes, "merge scratch");
-  if (computes && kg > 0) {
+  static_assert(4 * 32 * kSlot * 4 <= kStages * Layout<HD>::kStage, "merge scratch");
+  float* scratch = reinterpret_cast<float*>(smem);
+  __syncthreads();
+  if (KG > 1 && computes && kg > 0) {
     float* sl = scratch + ((size_t)warp * 32 + lane) * kSlot;
 #pragma unroll
     for (int n = 0; n < NT; ++n)
@@ -280,6 +330,7 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
   if (!computes || kg > 0) return;
+#pragma unroll
   for (int k = 1; k < KG; ++k) {
     const float* sl = scratch + ((size_t)(k * MT + mt) * 32 + lane) * kSlot;
     const float pm0 = sl[NT * 4 + 0], pm1 = sl[NT * 4 + 1];
@@ -301,6 +352,7 @@ __global__ void __launch_bounds__(kThreads)
     m1 = nm1;
   }
   const size_t pbase = (((size_t)r * nkv + g) * n_chunks + c) * kAttnMaxRows;
+  const int tq = lane & 3;
   const int row0 = mt * 16 + (lane >> 2), row1 = row0 + 8;
 #pragma unroll
   for (int n = 0; n < NT; ++n) {
@@ -318,37 +370,60 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-template <int HD>
-int launch_hd(const __half* q, const __half* kb, const __half* vb, const __nv_bfloat16* kc,
-              const __nv_bfloat16* vc, int layer, int batch, int cap, const int32_t* ctx_len,
-              const int32_t* req_valid, int B, int nq, int nkv, int chunk, int n_chunks,
-              float* part_o, float* part_ml, cudaStream_t s) {
+template <int HD, int MT>
+int launch_cfg(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q, const __half* kb,
+               const __half* vb, int layer, int batch, int cap, const int32_t* ctx_len,
+               const int32_t* req_valid, int B, int nq, int nkv, int chunk, int n_chunks,
+               float* part_o, float* part_ml, int32_t* err, cudaStream_t s) {
   const int smem = Layout<HD>::kSmem;
-  if (cudaFuncSetAttribute(attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
+  if (cudaFuncSetAttribute(attn_tc_kernel<HD, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
     return DFLASH_ECUDA;
   dim3 grid(n_chunks, nkv, batch);
-  attn_tc_kernel<HD><<<grid, kThreads, smem, s>>>(q, kb, vb, kc, vc, layer, batch, cap, ctx_len,
-                                                  req_valid, B, nq, nkv, chunk, n_chunks, part_o,
-                                                  part_ml);
+  attn_tc_kernel<HD, MT><<<grid, kThreads, smem, s>>>(tk, tv, q, kb, vb, layer, batch, cap,
+                                                      ctx_len, req_valid, B, nq, nkv, chunk,
+                                                      n_chunks, part_o, part_ml, err);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
+}
+
+template <int HD>
+int launch_hd(const __half* q, const __half* kb, const __half* vb, const __half* kc,
+              const __half* vc, int layer, int batch, int cap, const int32_t* ctx_len,
+              const int32_t* req_valid, int B, int nq, int nkv, int L, int chunk, int n_chunks,
+              float* part_o, float* part_ml, int32_t* err, cudaStream_t s) {
+  CUtensorMap tk, tv;
+  const int64_t rows = (int64_t)L * batch * nkv * cap;
+  if (!encode_2d(&tk, kc, rows, HD, HD, kKeys, DFLASH_F16) ||
+      !encode_2d(&tv, vc, rows, HD, HD, kKeys, DFLASH_F16))
+    return DFLASH_ECUDA;
+  const int R = B * (nq / nkv);
+  if (R <= 16)
+    return launch_cfg<HD, 1>(tk, tv, q, kb, vb, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
+                             chunk, n_chunks, part_o, part_ml, err, s);
+  if (R <= 32)
+    return launch_cfg<HD, 2>(tk, tv, q, kb, vb, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
+                             chunk, n_chunks, part_o, part_ml, err, s);
+  return launch_cfg<HD, 4>(tk, tv, q, kb, vb, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
+                           chunk, n_chunks, part_o, part_ml, err, s);
 }
 
 }  // namespace
 
-int launch_attn_partial_tc(const __half* q, const __half* kb, const __half* vb,
-                           const __nv_bfloat16* kc, const __nv_bfloat16* vc, int layer, int batch,
-                           int cap, const int32_t* ctx_len, const int32_t* req_valid, int B,
-                           int nq, int nkv, int hd, int chunk, int n_chunks, float* part_o,
-                           float* part_ml, cudaStream_t s) {
-  if (B * (nq / nkv) > kAttnMaxRows || chunk % kKeys != 0) return DFLASH_EUNSUPPORTED;
+int launch_attn_partial_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
+                           const __half* vc, int layer, int batch, int cap, const int32_t* ctx_len,
+                           const int32_t* req_valid, int B, int nq, int nkv, int hd, int L,
+                           int chunk, int n_chunks, float* part_o, float* part_ml, int32_t* err,
+                           cudaStream_t s) {
+  if (B * (nq / nkv) > kAttnMaxRows || chunk % kKeys != 0 || B > kBlkKeys)
+    return DFLASH_EUNSUPPORTED;
+  if ((int64_t)L * batch * nkv * cap > 0x7fffffffLL) return DFLASH_EUNSUPPORTED;
   TimedScope ts(s, TC_ATTN);
   if (hd == 128)
-    return launch_hd<128>(q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
-                          chunk, n_chunks, part_o, part_ml, s);
+    return launch_hd<128>(q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, L,
+                          chunk, n_chunks, part_o, part_ml, err, s);
   if (hd == 64)
-    return launch_hd<64>(q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
-                         chunk, n_chunks, part_o, part_ml, s);
+    return launch_hd<64>(q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, L,
+                         chunk, n_chunks, part_o, part_ml, err, s);
   return DFLASH_EUNSUPPORTED;
 }
 

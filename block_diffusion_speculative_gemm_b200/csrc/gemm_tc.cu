@@ -53,7 +53,7 @@ __host__ __device__ inline int tmem_cols_for(int bn) {
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128, 2)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps tmB,
                    const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -230,8 +230,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 // 2D 16-bit tensor map (bf16 or fp16): `rows` rows of `cols` elements, row
 // stride `ld` elements, box = 64 columns x box_rows rows, 128-byte swizzle,
 // zero fill outside.
-static bool encode_2d(CUtensorMap* m, const void* ptr, int rows, int cols, int ld, int box_rows,
-                      int elem) {
+bool encode_2d(CUtensorMap* m, const void* ptr, int64_t rows, int cols, int ld, int box_rows,
+               int elem) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -309,12 +309,22 @@ int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, i
   a.seg_k = seg_k;
   a.BN = BN;
   const int stage_bytes = kTileN * 128 + BN * 128;
-  const int budget = 200 * 1024;
-  a.stages = budget / stage_bytes;
-  if (a.stages > 8) a.stages = 8;
   a.n_kb = W.K / kTileK;
   if (epi == EPI_LMHEAD) splits = 1;
   splits = gemm_effective_splits(W.K, splits);
+  const long ctas = (long)((W.N + kTileN - 1) / kTileN) * ((M + BN - 1) / BN) * splits;
+  // More than one wave: ~100 KB per CTA so that two CTAs share an SM and one's
+  // prologue/epilogue overlaps the other's weight stream; otherwise one deep
+  // pipeline per SM.
+  int budget = ctas > 148 ? 100 * 1024 : 200 * 1024;
+  // the LM-head epilogue stages the BN x 128 fp32 tile (padded rows) in the stage buffers
+  const int lm_tile = BN * (kTileN + 1) * 4;
+  if (epi == EPI_LMHEAD && budget < lm_tile) budget = lm_tile;
+  a.stages = (budget + stage_bytes - 1) / stage_bytes;
+  if (a.stages > 8) a.stages = 8;
+  if (a.stages < 2) a.stages = 2;
+  if (epi == EPI_LMHEAD && a.stages * stage_bytes < lm_tile) return DFLASH_EUNSUPPORTED;
+  if (a.stages * stage_bytes > 210 * 1024) a.stages = 210 * 1024 / stage_bytes;
   a.kb_per_split = (a.n_kb + splits - 1) / splits;
   a.n_vtiles = (W.N + kTileN - 1) / kTileN;
   a.idesc = idesc_f16kind(kTileN, BN, W.elem == DFLASH_BF16);

@@ -58,6 +58,12 @@ struct WeightMap {
 
 bool encode_weight_map(WeightMap& w, const void* ptr, int N, int K, int elem);
 
+// 2D tensor map over `rows` rows of `cols` 16-bit elements (row stride `ld`
+// elements) with a box of 64 columns x box_rows rows, 128-byte swizzle, zero
+// fill outside the tensor.
+bool encode_2d(CUtensorMap* m, const void* ptr, int64_t rows, int cols, int ld, int box_rows,
+               int elem);
+
 // Y = X * W^T for X [M, K] of W's element type (given as n_seg K-segments of
 // seg_k columns, each [M, seg_k] with row stride ld_seg elements) and W [N, K].
 int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, int ld_seg, int M,
@@ -99,20 +105,22 @@ void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int 
 // ---------------------------------------------------------------- attention
 constexpr int kAttnMaxRows = 64;  // B * (n_q / n_kv) query rows per (request, kv head)
 
-// Split-KV partials of the tensor-core attention (fp16 block rows, bf16 cache):
+// Split-KV partials of the tensor-core attention (fp16 rows and fp16 cache):
 // part_o [batch][nkv][n_chunks][kAttnMaxRows][hd] fp32, part_ml [...][2] (max, sum).
-int launch_attn_partial_tc(const __half* q, const __half* kb, const __half* vb,
-                           const __nv_bfloat16* kc, const __nv_bfloat16* vc, int layer, int batch,
-                           int cap, const int32_t* ctx_len, const int32_t* req_valid, int B,
-                           int nq, int nkv, int hd, int chunk, int n_chunks, float* part_o,
-                           float* part_ml, cudaStream_t s);
+// The cache is [L][batch][nkv][cap][hd]; `layer` selects the layer.
+int launch_attn_partial_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
+                           const __half* vc, int layer, int batch, int cap, const int32_t* ctx_len,
+                           const int32_t* req_valid, int B, int nq, int nkv, int hd, int L,
+                           int chunk, int n_chunks, float* part_o, float* part_ml, int32_t* err,
+                           cudaStream_t s);
+
 // T: type of q, the block's k/v and the output o; TC: K/V cache type.
 template <typename T, typename TC>
 int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, const TC* vc,
-                           int layer, int batch, int cap, const int32_t* ctx_len,
+                           int layer, int L, int batch, int cap, const int32_t* ctx_len,
                            const int32_t* req_valid, int B, int nq, int nkv, int hd,
                            float* part_o, float* part_ml, int n_chunks, int chunk, T* o,
-                           cudaStream_t s);
+                           int32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- draft bookkeeping
 void launch_draft_init(const int32_t* anchor, const int32_t* ctx_len, int batch, int B, int V,

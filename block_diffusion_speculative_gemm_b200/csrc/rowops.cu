@@ -287,7 +287,7 @@ void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int 
 DFLASH_INST_A(float)
 DFLASH_INST_A(__half)
 DFLASH_INST_C(float)
-DFLASH_INST_C(__nv_bfloat16)
+DFLASH_INST_C(__half)
 template void launch_embed_norm<float, float>(const int32_t*, const float*, const float*, float*,
                                               float*, int, int, float, cudaStream_t);
 template void launch_embed_norm<__nv_bfloat16, __half>(const int32_t*, const __nv_bfloat16*,

@@ -145,6 +145,8 @@ class Model:
         self.shape = shape
         self.dtype = BF16 if shape.dtype == "bf16" else F32
         self.tdtype = _TORCH_DT[self.dtype]
+        # K/V cache element type: fp16 for bf16 models (see include/dflash.h), fp32 for fp32
+        self.cache_dtype = torch.float16 if self.dtype == BF16 else torch.float32
         cfg = Config(dtype=self.dtype, H_t=shape.H_t, n_tap=shape.n_tap, n_layers=shape.L,
                      d=shape.d, n_q=shape.nq, n_kv=shape.nkv, head_dim=shape.hd, inter=shape.I,
                      vocab=shape.V, mask_id=shape.mask_id, max_pos=int(max_pos),
@@ -212,8 +214,8 @@ def inject_kv(model: Model, taps: Sequence[torch.Tensor], cu_rows: torch.Tensor,
         _need(t, f"taps[{i}]", model.tdtype, (n_rows, s.H_t))
     _need(cu_rows, "cu_rows", torch.int32, (batch + 1,))
     _need(start_pos, "start_pos", torch.int32)
-    _need(k_cache, "k_cache", model.tdtype)
-    _need(v_cache, "v_cache", model.tdtype, k_cache.shape)
+    _need(k_cache, "k_cache", model.cache_dtype)
+    _need(v_cache, "v_cache", model.cache_dtype, k_cache.shape)
     if k_cache.dim() != 5 or tuple(k_cache.shape[:3]) != (s.L, batch, s.nkv) or k_cache.shape[4] != s.hd:
         raise ValueError("k_cache must be [L, batch, n_kv, cap, head_dim]")
     _need(ws, "ws", torch.uint8)
@@ -231,8 +233,8 @@ def draft_block(model: Model, anchor: torch.Tensor, ctx_len: torch.Tensor, k_cac
     batch = anchor.numel()
     _need(anchor, "anchor", torch.int32)
     _need(ctx_len, "ctx_len", torch.int32, (batch,))
-    _need(k_cache, "k_cache", model.tdtype)
-    _need(v_cache, "v_cache", model.tdtype, k_cache.shape)
+    _need(k_cache, "k_cache", model.cache_dtype)
+    _need(v_cache, "v_cache", model.cache_dtype, k_cache.shape)
     if k_cache.dim() != 5 or tuple(k_cache.shape[:3]) != (s.L, batch, s.nkv) or k_cache.shape[4] != s.hd:
         raise ValueError("k_cache must be [L, batch, n_kv, cap, head_dim]")
     _need(draft_tokens, "draft_tokens", torch.int32, (batch, B))

@@ -73,12 +73,19 @@ extern "C" {
 
 typedef struct dflash_model dflash_model; /* opaque */
 
-/* Draft model shape.  Constraints: n_q % n_kv == 0; head_dim even and <= 256.
+/* Element types inside a model.  DFLASH_F32 models compute and store in fp32.
+ * DFLASH_BF16 models take bf16 weights and bf16 tapped hidden states; the
+ * library keeps its GEMM weight copies and GEMM activations in fp16 (every
+ * bf16 weight in fp16's normal range converts exactly) and multiplies
+ * fp16 x fp16 -> fp32 on the tensor cores, and the K/V cache holds fp16.
+ * Same bytes as bf16, three more mantissa bits.
+ *
+ * Draft model shape.  Constraints: n_q % n_kv == 0; head_dim even and <= 256.
  * For DFLASH_BF16: d, H_t, inter, n_q*head_dim multiples of 64, head_dim 64 or
  * 128.  For DFLASH_F32 (SIMT path, for small correctness models) no further
  * constraint.  vocab >= 2; mask_id in [0, vocab). */
 typedef struct {
-  int32_t dtype;     /* DFLASH_F32 or DFLASH_BF16: weights, activations, K/V cache */
+  int32_t dtype;     /* DFLASH_F32 or DFLASH_BF16: type of the weights and tapped states */
   int32_t H_t;       /* target hidden size of one tapped layer */
   int32_t n_tap;     /* tapped target layers (1..8) */
   int32_t n_layers;  /* draft layers L */
@@ -144,8 +151,9 @@ int dflash_workspace_init(void* ws, size_t ws_bytes, void* stream);
  *   cu_rows    device int32 [batch+1]: rows cu_rows[r]..cu_rows[r+1]-1 belong to
  *              request r; cu_rows[0] = 0, cu_rows[batch] = n_rows.
  *   start_pos  device int32 [batch]: absolute position of request r's first row.
- *   k_cache, v_cache  device [n_layers][batch][n_kv][cache_cap][head_dim] in the
- *              model dtype; K is stored after RoPE.
+ *   k_cache, v_cache  device [n_layers][batch][n_kv][cache_cap][head_dim] of the
+ *              model's cache type (fp16 for DFLASH_BF16 models, fp32 for
+ *              DFLASH_F32), 16-byte aligned; K is stored after RoPE.
  * Computes c = RMSNorm(concat_t(taps[t]) W_fc^T; g_ctx) and, for every layer l,
  * K_l[p] = RoPE(c Wk_l^T, p), V_l[p] = c Wv_l^T at p = start_pos[r] + i.
  * Rows whose position falls outside [0, cache_cap) are skipped and set
@@ -158,6 +166,7 @@ int dflash_inject_kv(const dflash_model* m, const void* const* taps, const int32
 /*
  * Masked-block draft forward with n_steps denoising steps.
  *   anchor     device int32 [batch]: token at block position 0 (position ctx_len[r]).
+ *   k_cache, v_cache  the caches dflash_inject_kv fills (same layout and type).
  *   ctx_len    device int32 [batch]: injected context length T_r; the block sits at
  *              positions T_r..T_r+B-1 and attends to cache positions 0..T_r-1 plus
  *              the whole block (no mask inside the block).

@@ -115,10 +115,11 @@ def kv_std(cfg: DraftConfig) -> float:
 
 
 def make_kv_cache(cfg: DraftConfig, cap: Optional[int] = None, label: str = "kv",
-                  master: int = MASTER_SEED):
-    """Synthetic K/V cache contents [L, batch, nkv, cap, hd] (every slot filled)."""
+                  master: int = MASTER_SEED, dtype: Optional[torch.dtype] = None):
+    """Synthetic K/V cache contents [L, batch, nkv, cap, hd] (every slot filled),
+    rounded to ``dtype`` (default: the workload's dtype)."""
     cap = cfg.cache_cap if cap is None else cap
-    dt = _dtype(cfg)
+    dt = _dtype(cfg) if dtype is None else dtype
     shp = (cfg.L, cfg.batch, cfg.nkv, cap, cfg.hd)
     k = _randn(shp, kv_std(cfg), sub_seed(master, cfg.name, label, "k"), dt)
     v = _randn(shp, kv_std(cfg), sub_seed(master, cfg.name, label, "v"), dt)

@@ -24,7 +24,7 @@ def _run_draft(b, cfg, steps=None, dbg=True, ctx=None, anchors=None):
     steps = cfg.steps if steps is None else steps
     ctx = synth.make_ctx_lens(cfg) if ctx is None else ctx
     anchors = synth.make_anchors(cfg) if anchors is None else anchors
-    kc, vc = synth.make_kv_cache(cfg, b.cap)
+    kc, vc = synth.make_kv_cache(cfg, b.cap, dtype=b.model.cache_dtype)
     dk, dv = kc.cuda(), vc.cuda()
     out = torch.full((cfg.batch, cfg.B), -5, dtype=torch.int32, device="cuda")
     cst = torch.full((cfg.batch, cfg.B), -5, dtype=torch.int32, device="cuda")

@@ -19,7 +19,8 @@ def _inject(b, cfg, mode, rows_check=None, cap=None):
     ctx = synth.make_ctx_lens(cfg)
     cu, st, n = synth.make_inject_layout(cfg, ctx, mode)
     taps = synth.make_tap_hiddens(cfg, n, label=f"taps_{mode}")
-    kc = torch.zeros((cfg.L, cfg.batch, cfg.nkv, cap, cfg.hd), dtype=b.tdtype(), device="cuda")
+    kc = torch.zeros((cfg.L, cfg.batch, cfg.nkv, cap, cfg.hd), dtype=b.model.cache_dtype,
+                     device="cuda")
     vc = torch.zeros_like(kc)
     ws = b.model.workspace(cfg.batch, cfg.B, n)
     D.inject_kv(b.model, [t.cuda() for t in taps], cu.cuda(), st.cuda(), kc, vc, ws)
@@ -93,7 +94,7 @@ def test_inject_chunks_equal_one_call():
     b = built(cfg)
     taps = synth.make_tap_hiddens(cfg, 128, label="chunks")
     cap = b.cap
-    kc1 = torch.zeros((cfg.L, 2, cfg.nkv, cap, cfg.hd), dtype=torch.bfloat16, device="cuda")
+    kc1 = torch.zeros((cfg.L, 2, cfg.nkv, cap, cfg.hd), dtype=b.model.cache_dtype, device="cuda")
     vc1 = torch.zeros_like(kc1)
     kc2, vc2 = torch.zeros_like(kc1), torch.zeros_like(kc1)
     ws = b.model.workspace(2, cfg.B, 128)
@@ -120,7 +121,7 @@ def test_inject_past_capacity_sets_error_and_skips():
     b = built(cfg)
     cap = 48
     taps = [t.cuda() for t in synth.make_tap_hiddens(cfg, 8, label="cap")]
-    kc = torch.zeros((cfg.L, 2, cfg.nkv, cap, cfg.hd), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((cfg.L, 2, cfg.nkv, cap, cfg.hd), dtype=b.model.cache_dtype, device="cuda")
     vc = torch.zeros_like(kc)
     ws = b.model.workspace(2, cfg.B, 8)
     cu = torch.tensor([0, 4, 8], dtype=torch.int32).cuda()
