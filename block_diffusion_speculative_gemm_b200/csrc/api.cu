@@ -323,6 +323,7 @@ extern "C" const char* dflash_status_str(int st) {
     case DFLASH_ECUDA: return "CUDA error";
     case DFLASH_ENOMEM: return "out of device memory";
     case DFLASH_EWORKSPACE: return "workspace too small";
+    case DFLASH_ESCRATCH: return "request exceeds the fixed scratch of dflash_verify_noalloc";
     default: return "unknown status";
   }
 }

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libdflash.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "dflash.h")
 HEADERS = [HEADER, os.path.join(os.path.dirname(_HERE), "include", "dflash_debug.h")]
 
-OK, EINVAL, EUNSUPPORTED, ECUDA, ENOMEM, EWORKSPACE = 0, -1, -2, -3, -4, -5
+OK, EINVAL, EUNSUPPORTED, ECUDA, ENOMEM, EWORKSPACE, ESCRATCH = 0, -1, -2, -3, -4, -5, -6
 DEV_CTX_CAP, DEV_OUT_CAP, DEV_TOKEN_RANGE, DEV_TIMEOUT, DEV_ROWS = 1, 2, 4, 8, 16
 F32, BF16, F16 = 0, 1, 2
 TIMING_CLASSES = ("gemm", "attention", "row", "verify", "lm_head")
@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.dflash_verify.argtypes = [vp, i32, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp, sz,
                                     vp]
         L.dflash_get_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+        L.dflash_verify_noalloc.argtypes = [vp, i32, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp,
+                                            vp, vp]
         L.dflash_status_str.argtypes = [i32]
         L.dflash_status_str.restype = ctypes.c_char_p
         L.dflash_timing_enable.argtypes = [i32]
@@ -271,6 +273,37 @@ def verify(target_logits: torch.Tensor, draft_tokens: torch.Tensor, out_tokens: 
         _ptr(target_logits), dt, _ptr(draft_tokens), batch, B, V, _ptr(out_tokens), _ptr(out_len),
         out_tokens.shape[1], _ptr(seq_lens), _ptr(accept_len), _ptr(next_anchor), _ptr(ws),
         ws.numel(), _stream(stream)))
+
+
+def verify_noalloc(target_logits: torch.Tensor, draft_tokens: torch.Tensor,
+                   out_tokens: torch.Tensor, out_len: torch.Tensor, seq_lens: torch.Tensor,
+                   accept_len: torch.Tensor, next_anchor: torch.Tensor,
+                   error_bits: Optional[torch.Tensor] = None, stream=None):
+    """Greedy verify without a workspace, for callers that cannot allocate device
+    memory: the library keeps the scratch in a fixed array of its own.  Same
+    results as ``verify``; ``error_bits`` (int32 [1] on the device, optional)
+    receives the call's device error bits.  Calls that overlap on the GPU race
+    on the shared scratch."""
+    if target_logits.dim() != 3:
+        raise ValueError("target_logits must be [batch, B, V]")
+    batch, B, V = target_logits.shape
+    dt = {torch.bfloat16: BF16, torch.float32: F32}.get(target_logits.dtype)
+    if dt is None:
+        raise TypeError("target_logits must be bfloat16 or float32")
+    _need(target_logits, "target_logits")
+    _need(draft_tokens, "draft_tokens", torch.int32, (batch, B))
+    _need(out_tokens, "out_tokens", torch.int32)
+    if out_tokens.dim() != 2 or out_tokens.shape[0] != batch:
+        raise ValueError("out_tokens must be [batch, out_cap]")
+    for n, t in (("out_len", out_len), ("seq_lens", seq_lens), ("accept_len", accept_len),
+                 ("next_anchor", next_anchor)):
+        _need(t, n, torch.int32, (batch,))
+    if error_bits is not None:
+        _need(error_bits, "error_bits", torch.int32, (1,))
+    _check("dflash_verify_noalloc", lib().dflash_verify_noalloc(
+        _ptr(target_logits), dt, _ptr(draft_tokens), batch, B, V, _ptr(out_tokens), _ptr(out_len),
+        out_tokens.shape[1], _ptr(seq_lens), _ptr(accept_len), _ptr(next_anchor),
+        _ptr(error_bits), _stream(stream)))
 
 
 def get_error(ws: torch.Tensor, stream=None) -> int:

@@ -58,6 +58,7 @@ extern "C" {
 #define DFLASH_ECUDA        -3  /* a CUDA call or kernel launch failed */
 #define DFLASH_ENOMEM       -4  /* model creation could not allocate device memory */
 #define DFLASH_EWORKSPACE   -5  /* workspace smaller than the size query returned */
+#define DFLASH_ESCRATCH     -6  /* request larger than dflash_verify_noalloc's fixed scratch */
 
 /* ---- device error word bits (dflash_get_error) ------------------------ */
 #define DFLASH_DEV_CTX_CAP     1  /* position outside the K/V cache capacity */
@@ -206,6 +207,35 @@ int dflash_verify(const void* target_logits, int logits_dtype, const int32_t* dr
                   int batch, int B, int V, int32_t* out_tokens, int32_t* out_len, int out_cap,
                   int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor, void* ws,
                   size_t ws_bytes, void* stream);
+
+/*
+ * Greedy verify without any workspace or allocation.  The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory -- an inference server that reserves all of its device memory
+ * in its own pool at start-up and allows no allocation afterwards, a plugin
+ * that runs inside another framework's allocator, or a latency-critical loop
+ * that avoids cudaMalloc because it may synchronise the device.
+ *
+ * Same arguments, semantics and results as dflash_verify, without ws /
+ * ws_bytes.  Its scratch (argmax partials and the device error word) is a
+ * fixed array of 256 KiB + 256 bytes in the library's device memory, present on
+ * every GPU that loads the library until the process exits.  That bounds a call
+ * to batch * B <= 32768 rows (8 bytes of partials per row chunk; rows are split
+ * into chunks only while batch * B < ~600); larger calls return DFLASH_ESCRATCH
+ * before anything is enqueued.
+ *   error_bits  device int32 out or NULL: the call's device error bits
+ *               (DFLASH_DEV_*), written on `stream` at the end of the call.
+ * The first call on a device looks up the scratch array's device address and
+ * caches it; make that first call before any stream capture.  Every call
+ * shares the array and clears its error word at the start: calls that overlap
+ * on the GPU (different streams, or different host threads) race on it.
+ * Allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ */
+int dflash_verify_noalloc(const void* target_logits, int logits_dtype,
+                          const int32_t* draft_tokens, int batch, int B, int V,
+                          int32_t* out_tokens, int32_t* out_len, int out_cap, int32_t* seq_lens,
+                          int32_t* accept_len, int32_t* next_anchor, int32_t* error_bits,
+                          void* stream);
 
 /* Waits for `stream`, copies the workspace's device error word to *bits and
  * clears it.  The only call that synchronises with the host. */
