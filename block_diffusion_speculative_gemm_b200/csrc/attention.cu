@@ -124,33 +124,57 @@ __global__ void __launch_bounds__(kAttnThreads)
   }
 }
 
-// o[m][head*HD + e] = sum_c exp(m_c - M) o_c[e] / sum_c exp(m_c - M) l_c
+// Merge of the split-KV partials of one (kv head, request): for query row i,
+// o_i = sum_c exp(m_ci - M_i) o_ci / sum_c exp(m_ci - M_i) l_ci with
+// M_i = max_c m_ci, chunks in ascending order.  The per-(chunk, row) weights
+// are computed once into shared memory, then the CTA streams the [R][HD]
+// partial blocks with 16-byte loads.
+constexpr int kCombineThreads = 256;
+constexpr int kMaxChunksC = 64;
+
 template <typename T, int HD>
-__global__ void attn_combine_kernel(const float* __restrict__ part_o,
-                                    const float* __restrict__ part_ml,
-                                    const int32_t* __restrict__ ctx_len,
-                                    const int32_t* __restrict__ req_valid, int B, int nq, int nkv,
-                                    int chunk, int n_chunks, T* __restrict__ o) {
-  const int m = blockIdx.x, head = blockIdx.y;
-  const int r = m / B, j = m % B;
-  const int G = nq / nkv, g = head / G;
-  const int row = j * G + head % G;
+__global__ void __launch_bounds__(kCombineThreads)
+    attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
+                        const int32_t* __restrict__ ctx_len,
+                        const int32_t* __restrict__ req_valid, int B, int nq, int nkv, int chunk,
+                        int n_chunks, T* __restrict__ o) {
+  __shared__ float wgt[kMaxChunksC * kMaxRows];
+  const int g = blockIdx.x, r = blockIdx.y;
+  const int G = nq / nkv, R = B * G;
   const int T_r = req_valid[r] ? ctx_len[r] : 0;
-  const int nc = (T_r + B + chunk - 1) / chunk;
+  const int nc = min(n_chunks, (T_r + B + chunk - 1) / chunk);
   const size_t base = ((size_t)r * nkv + g) * n_chunks * kMaxRows;
-  float M = -INFINITY;
-  for (int c = 0; c < nc; ++c) M = fmaxf(M, part_ml[(base + (size_t)c * kMaxRows + row) * 2]);
-  float L = 0.f;
-  for (int e = threadIdx.x; e < HD; e += blockDim.x) {
-    float acc = 0.f;
-    L = 0.f;
+  for (int row = threadIdx.x; row < R; row += blockDim.x) {
+    float M = -INFINITY;
+    for (int c = 0; c < nc; ++c) M = fmaxf(M, part_ml[(base + (size_t)c * kMaxRows + row) * 2]);
+    float L = 0.f;
     for (int c = 0; c < nc; ++c) {
       const size_t pr = base + (size_t)c * kMaxRows + row;
       const float w = expf(part_ml[pr * 2] - M);
+      wgt[c * kMaxRows + row] = w;
       L += w * part_ml[pr * 2 + 1];
-      acc += w * part_o[pr * HD + e];
     }
-    o[((size_t)m * nq + head) * HD + e] = from_f<T>(acc / L);
+    const float inv = 1.f / L;
+    for (int c = 0; c < nc; ++c) wgt[c * kMaxRows + row] *= inv;
+  }
+  __syncthreads();
+  for (int i4 = threadIdx.x; i4 < R * HD / 4; i4 += blockDim.x) {
+    const int row = (i4 * 4) / HD, col = (i4 * 4) % HD;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < nc; ++c) {
+      const float w = wgt[c * kMaxRows + row];
+      const float4 v = *reinterpret_cast<const float4*>(
+          part_o + (base + (size_t)c * kMaxRows + row) * HD + col);
+      acc.x += w * v.x;
+      acc.y += w * v.y;
+      acc.z += w * v.z;
+      acc.w += w * v.w;
+    }
+    T* dst = o + ((size_t)(r * B + row / G) * nq + g * G + row % G) * HD + col;
+    dst[0] = from_f<T>(acc.x);
+    dst[1] = from_f<T>(acc.y);
+    dst[2] = from_f<T>(acc.z);
+    dst[3] = from_f<T>(acc.w);
   }
 }
 
@@ -187,13 +211,16 @@ int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, c
   }
   {
     TimedScope ts(s, TC_ATTN);
-    dim3 g2(batch * B, nq);
+    if (n_chunks > kMaxChunksC) return DFLASH_EUNSUPPORTED;
+    dim3 g2(nkv, batch);
     if (hd == 128)
-      attn_combine_kernel<T, 128><<<g2, 128, 0, s>>>(part_o, part_ml, ctx_len, req_valid, B, nq,
-                                                     nkv, chunk, n_chunks, o);
+      attn_combine_kernel<T, 128><<<g2, kCombineThreads, 0, s>>>(part_o, part_ml, ctx_len,
+                                                                 req_valid, B, nq, nkv, chunk,
+                                                                 n_chunks, o);
     else
-      attn_combine_kernel<T, 64><<<g2, 64, 0, s>>>(part_o, part_ml, ctx_len, req_valid, B, nq, nkv,
-                                                   chunk, n_chunks, o);
+      attn_combine_kernel<T, 64><<<g2, kCombineThreads, 0, s>>>(part_o, part_ml, ctx_len,
+                                                                req_valid, B, nq, nkv, chunk,
+                                                                n_chunks, o);
   }
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }

@@ -24,7 +24,6 @@ namespace {
 constexpr int kThreads = 128;
 constexpr int kKeys = 64;    // keys per context tile
 constexpr int kBlkKeys = 16; // rows of the block tile
-constexpr int kStages = 3;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
@@ -73,11 +72,16 @@ __device__ __forceinline__ uint32_t toff(int rows, int row, int c) {
   return (uint32_t)((c >> 3) * rows * 128 + row * 128 + (((c & 7) ^ (row & 7)) << 4));
 }
 
-template <int HD>
+// Shared memory of one CTA: the TMA stage ring, then the query rows (later
+// reused for the block tile), then the stage barriers.  Sized so that two
+// CTAs fit on an SM: 3 stages for up to 32 query rows, 2 stages for 64.
+template <int HD, int MT>
 struct Layout {
+  static constexpr int kStages = MT <= 2 ? 3 : 2;
   static constexpr int kTile = kKeys * HD * 2;       // K or V of one context tile
   static constexpr int kStage = 2 * kTile;
-  static constexpr int kQ = kAttnMaxRows * HD * 2;   // query rows, later the block tile
+  static constexpr int kQRows = MT * 16;
+  static constexpr int kQ = (kQRows > 2 * kBlkKeys ? kQRows : 2 * kBlkKeys) * HD * 2;
   static constexpr int kBars = kStages * 8;
   static constexpr int kSmem = kStages * kStage + kQ + kBars + 1024;  // + alignment slack
   static_assert(2 * kBlkKeys * HD * 2 <= kQ, "block tile fits the query area");
@@ -177,8 +181,9 @@ __global__ void __launch_bounds__(kThreads)
                    const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ req_valid,
                    int B, int nq, int nkv, int chunk, int n_chunks, float* __restrict__ part_o,
                    float* __restrict__ part_ml, int32_t* err) {
-  using LY = Layout<HD>;
+  using LY = Layout<HD, MT>;
   using WP = Warp<HD, MT>;
+  constexpr int kStages = LY::kStages;
   constexpr int NT = WP::NT, KS = WP::KS, KG = WP::KG, KPW = WP::KPW;
   constexpr int HALVES = HD / 64;
   extern __shared__ uint8_t smem_raw[];
@@ -216,7 +221,7 @@ __global__ void __launch_bounds__(kThreads)
       src = q + ((size_t)(r * B + row / G) * nq + g * G + row % G) * HD + ch * 8;
       bytes = 16;
     }
-    cp_async16(s_q + toff(kAttnMaxRows, row, ch), src, bytes);
+    cp_async16(s_q + toff(LY::kQRows, row, ch), src, bytes);
   }
   cp_async_commit();
   __syncthreads();  // barrier init visible before any wait
@@ -252,7 +257,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       const int row = mt * 16 + (mi & 1) * 8 + li;
-      ldsm_x4(s_q + toff(kAttnMaxRows, row, ks * 2 + (mi >> 1)), qa[ks][0], qa[ks][1], qa[ks][2],
+      ldsm_x4(s_q + toff(LY::kQRows, row, ks * 2 + (mi >> 1)), qa[ks][0], qa[ks][1], qa[ks][2],
               qa[ks][3]);
     }
   }
@@ -314,7 +319,7 @@ __global__ void __launch_bounds__(kThreads)
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
   constexpr int kSlot = NT * 4 + 4;
-  static_assert(4 * 32 * kSlot * 4 <= kStages * Layout<HD>::kStage, "merge scratch");
+  static_assert(4 * 32 * kSlot * 4 <= kStages * LY::kStage, "merge scratch");
   float* scratch = reinterpret_cast<float*>(smem);
   __syncthreads();
   if (KG > 1 && computes && kg > 0) {
@@ -375,7 +380,7 @@ int launch_cfg(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q, co
                const __half* vb, int layer, int batch, int cap, const int32_t* ctx_len,
                const int32_t* req_valid, int B, int nq, int nkv, int chunk, int n_chunks,
                float* part_o, float* part_ml, int32_t* err, cudaStream_t s) {
-  const int smem = Layout<HD>::kSmem;
+  const int smem = Layout<HD, MT>::kSmem;
   if (cudaFuncSetAttribute(attn_tc_kernel<HD, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess)
     return DFLASH_ECUDA;

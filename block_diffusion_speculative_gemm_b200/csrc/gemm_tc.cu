@@ -1,23 +1,30 @@
-// tcgen05 weight-streaming GEMM for sm_100a.
+// Persistent tcgen05 weight-streaming GEMM for sm_100a.
 //
 // Every dense contraction of the draft hot path multiplies a small set of
 // token rows X [M, K] (M <= 256 per tile) by a large weight W [N, K]:
 // context-feature fc, the layer-batched K/V injection projection, the QKV,
-// output and SwiGLU projections, and the LM head.  The CTA tile therefore puts
-// 128 weight rows on the UMMA M axis and the token rows on the UMMA N axis
-// ("swap-AB"): one weight tile is streamed from HBM exactly once, the token
-// tile is re-read from L2.
+// output and SwiGLU projections, and the LM head.  A tile therefore puts 128
+// weight rows on the UMMA M axis and up to 256 token rows on the UMMA N axis
+// ("swap-AB"): each weight tile streams from HBM once, the token tile is
+// re-read from L2.
 //
-// Structure of one CTA (128 threads, one output tile, one K range):
-//   warp 0 lane 0  TMA producer: weight tile [128 x 64] + token tile [BN x 64]
-//                  per stage, 128-byte swizzled, completion on a full barrier.
-//   warp 1 lane 0  MMA issuer: 4 x tcgen05.mma (K = 16 each) per stage into a
-//                  TMEM accumulator of 128 lanes x BN fp32 columns; a
-//                  tcgen05.commit per stage releases the stage to the producer.
-//   warp 2         allocates and frees the TMEM columns.
-//   all warps      epilogue: tcgen05.ld of the accumulator (lane = weight row)
-//                  and either a coalesced fp32 partial store (split-K) or the
-//                  LM-head reduction (per token: max, argmax, sum of exp).
+// Work units are (token tile, weight tile, K split), ordered split-major so
+// that CTAs running at the same time share the K range of X.  One CTA per SM
+// walks units u = blockIdx.x, + gridDim.x, ... with warp-specialised roles:
+//   warp 0 (one lane)  TMA producer: per 64-wide k-block, the weight tile
+//                      [128 x 64] and the token tile [BN x 64], 128-byte
+//                      swizzled, through a ring of `stages` smem stages that
+//                      runs on across unit boundaries.
+//   warp 1 (one lane)  MMA issuer: 4 x tcgen05.mma (K = 16) per stage into one
+//                      of two TMEM accumulators (128 lanes x BN fp32 columns),
+//                      alternating per unit; tcgen05.commit releases the stage.
+//   warps 2..5         epilogue: drain the accumulator of unit j while the
+//                      MMA warp fills the other one for unit j + 1, then give it
+//                      back.  PARTIAL: coalesced fp32 store of the split's
+//                      partial product.  LMHEAD: per token and 128-row
+//                      vocabulary tile, the maximum, its lowest index and the
+//                      sum of exp(logit - max), through per-warp 32 x 33 shared
+//                      transposes (no fp32 logits leave the SM).
 // Every mbarrier wait is bounded (1 s) and reports DFLASH_DEV_TIMEOUT.
 #include <cudaTypedefs.h>
 
@@ -40,11 +47,18 @@ struct GemmArgs {
   int stages;
   int kb_per_split;   // 64-wide k-blocks per split
   int n_kb;           // total k-blocks
-  int n_vtiles;       // LM head: number of 128-row vocabulary tiles
+  int tiles_n;        // weight tiles
+  int tiles_m;        // token tiles
+  int units;          // tiles_n * tiles_m * splits
+  int n_vtiles;       // LM head: number of 128-row vocabulary tiles (= tiles_n)
   uint32_t idesc;     // tcgen05 instruction descriptor (operand type, 128 x BN)
   GemmOut out;
   int32_t* err;
 };
+
+constexpr int kGemmThreads = 192;
+constexpr int kEpiWarp0 = 2;  // first epilogue warp
+constexpr int kLmTr = 32 * 33;  // floats of one warp's transpose buffer
 
 __host__ __device__ inline int tmem_cols_for(int bn) {
   int c = 32;
@@ -52,30 +66,62 @@ __host__ __device__ inline int tmem_cols_for(int bn) {
   return c;
 }
 
+struct Unit {
+  int n0, m0, split, kb0, nk;
+};
+
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
+  Unit w;
+  const int per = a.tiles_n * a.tiles_m;
+  w.split = u / per;
+  const int rem = u % per;
+  w.m0 = (rem / a.tiles_n) * a.BN;
+  w.n0 = (rem % a.tiles_n) * kTileN;
+  w.kb0 = w.split * a.kb_per_split;
+  w.nk = min(a.n_kb, w.kb0 + a.kb_per_split) - w.kb0;
+  return w;
+}
+
+__device__ __forceinline__ void epi_bar_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kGemmThreads - kEpiWarp0 * 32) : "memory");
+}
+// AND of `v` over the epilogue warps (named barrier 1)
+__device__ __forceinline__ bool epi_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kGemmThreads - kEpiWarp0 * 32)
+      : "memory");
+  return r != 0;
+}
+
 template <int EPI>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps tmB,
                    const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int stage_bytes = kTileN * 128 + a.BN * 128;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.stages * stage_bytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * a.stages + 1);
+  // [stages][A | B] | LM-head transposes + partials | barriers
+  float* lm_tr = reinterpret_cast<float*>(smem + a.stages * stage_bytes);
+  LmStat* lm_part = reinterpret_cast<LmStat*>(lm_tr + (EPI == EPI_LMHEAD ? 4 * kLmTr : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      reinterpret_cast<uint8_t*>(lm_part) + (EPI == EPI_LMHEAD ? 4 * kMaxBN * sizeof(LmStat) : 0));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * a.stages + 4);
   const uint32_t smem0 = smem_u32(smem);
   auto sA = [&](int s) { return smem0 + s * stage_bytes; };
   auto sB = [&](int s) { return smem0 + s * stage_bytes + kTileN * 128; };
   auto full = [&](int s) { return smem_u32(bars + s); };
   auto empty = [&](int s) { return smem_u32(bars + a.stages + s); };
-  const uint32_t accum = smem_u32(bars + 2 * a.stages);
+  auto acc_full = [&](int b) { return smem_u32(bars + 2 * a.stages + b); };
+  auto acc_empty = [&](int b) { return smem_u32(bars + 2 * a.stages + 2 + b); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kTileN;
-  const int m0 = blockIdx.y * a.BN;
-  const int split = blockIdx.z;
-  const int kb0 = split * a.kb_per_split;
-  const int kb1 = min(a.n_kb, kb0 + a.kb_per_split);
-  const int nk = kb1 - kb0;
   const uint32_t ncols = tmem_cols_for(a.BN);
 
   if (threadIdx.x == 0) {
@@ -83,14 +129,15 @@ __global__ void __launch_bounds__(128, 2)
       mbar_init(full(s), 1);
       mbar_init(empty(s), 1);
     }
-    mbar_init(accum, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full(b), 1);
+      mbar_init(acc_empty(b), 4);  // one elected lane per epilogue warp
+    }
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-  }
-  if (warp == 2) {
-    tmem_alloc(smem_u32(tmem_slot), ncols);
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmA);
+  if (warp == kEpiWarp0) {
+    tmem_alloc(smem_u32(tmem_slot), 2 * ncols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -100,115 +147,149 @@ __global__ void __launch_bounds__(128, 2)
 
   bool ok = true;
   if (warp == 0) {
-    if (lane == 0 && nk > 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
-      for (int i = 0; i < nk; ++i) {
-        const int s = i % a.stages;
-        const uint32_t ph = (i / a.stages) & 1;
-        if (!mbar_wait(empty(s), ph ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(full(s), stage_bytes);
-        const int kx = (kb0 + i) * kTileK;
-        tma_load_2d(sA(s), &tmA, full(s), kx, n0, pol_w);
-        const int seg = kx / a.seg_k;
-        tma_load_2d(sB(s), &tmB.m[seg], full(s), kx - seg * a.seg_k, m0, pol_x);
+      uint32_t it = 0;
+      for (int u = blockIdx.x; u < a.units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(a, u);
+        for (int i = 0; i < w.nk; ++i, ++it) {
+          const int s = it % a.stages;
+          const uint32_t ph = (it / a.stages) & 1;
+          if (!mbar_wait(empty(s), ph ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(full(s), stage_bytes);
+          const int kx = (w.kb0 + i) * kTileK;
+          tma_load_2d(sA(s), &tmA, full(s), kx, w.n0, pol_w);
+          const int seg = kx / a.seg_k;
+          tma_load_2d(sB(s), &tmB.m[seg], full(s), kx - seg * a.seg_k, w.m0, pol_x);
+        }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = a.idesc;
-      for (int i = 0; i < nk; ++i) {
-        const int s = i % a.stages;
-        const uint32_t ph = (i / a.stages) & 1;
-        if (!mbar_wait(full(s), ph)) { ok = false; break; }
+      uint32_t it = 0;
+      int j = 0;
+      for (int u = blockIdx.x; u < a.units && ok; u += gridDim.x, ++j) {
+        const Unit w = decode_unit(a, u);
+        const int b = j & 1;
+        if (!mbar_wait(acc_empty(b), ((j >> 1) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t d = tmem + b * ncols;
+        for (int i = 0; i < w.nk; ++i, ++it) {
+          const int s = it % a.stages;
+          const uint32_t ph = (it / a.stages) & 1;
+          if (!mbar_wait(full(s), ph)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kTileK / 16; ++kk) {
-          umma_f16(tmem, smem_desc_sw128(sA(s) + kk * 32), smem_desc_sw128(sB(s) + kk * 32),
-                    idesc, (i | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < kTileK / 16; ++kk)
+            umma_f16(d, smem_desc_sw128(sA(s) + kk * 32), smem_desc_sw128(sB(s) + kk * 32),
+                     a.idesc, (i | kk) != 0 ? 1u : 0u);
+          umma_commit(empty(s));
         }
-        umma_commit(empty(s));
+        umma_commit(acc_full(b));
       }
-      umma_commit(accum);
     }
     __syncwarp();
-  }
-
-  // ---------------------------------------------------------------- epilogue
-  const bool acc_ok = (nk > 0) ? mbar_wait(accum, 0) : true;
-  __syncwarp();
-  tc_fence_after();
-  if ((!ok || !acc_ok) && lane == 0) set_error(a.err, DFLASH_DEV_TIMEOUT);
-
-  const int row = warp * 32 + lane;  // TMEM lane = weight row inside the tile
-  const int n = n0 + row;
-  const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16);
-  const int nchunk = a.BN / 32;
-
-  if (EPI == EPI_PARTIAL) {
-    float* out = a.out.part + (size_t)split * a.M * a.N;
-    for (int c = 0; c < nchunk; ++c) {
-      if (m0 + c * 32 >= a.M) break;  // uniform across the CTA
-      float v[32];
-      if (nk > 0) {
-        tmem_ld32(tbase + c * 32, v);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = 0.f;
-      }
-      if (n < a.N) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int m = m0 + c * 32 + j;
-          if (m < a.M) out[(size_t)m * a.N + n] = v[j];
-        }
-      }
-    }
   } else {
-    // LM head: stage the tile as [token][weight row] in shared memory, then one
-    // thread per token reduces its 128 logits (max, lowest argmax, sum exp).
-    float* tile = reinterpret_cast<float*>(smem);  // stages are idle once accum completed
-    const int ld = kTileN + 1;
-    for (int c = 0; c < nchunk; ++c) {
-      float v[32];
-      tmem_ld32(tbase + c * 32, v);
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;              // TMEM lane group of this warp
+    const int row = q * 32 + lane;       // weight row inside the tile
+    const int nchunk = a.BN / 32;
+    int j = 0;
+    for (int u = blockIdx.x; u < a.units; u += gridDim.x, ++j) {
+      const Unit w = decode_unit(a, u);
+      const int b = j & 1;
+      bool got = mbar_wait(acc_full(b), (j >> 1) & 1);
+      if (EPI == EPI_LMHEAD) got = epi_bar_and(got);  // the epilogue warps leave together
+      __syncwarp();
+      if (!got) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tb = tmem + b * ncols + ((uint32_t)(q * 32) << 16);
+      const int n = w.n0 + row;
+      if (EPI == EPI_PARTIAL) {
+        float* out = a.out.part + (size_t)w.split * a.M * a.N;
+        for (int c = 0; c < nchunk; ++c) {
+          if (w.m0 + c * 32 >= a.M) break;  // uniform across the warp
+          float v[32];
+          tmem_ld32(tb + c * 32, v);
+          if (n < a.N) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) tile[(c * 32 + j) * ld + row] = (n < a.N) ? v[j] : -INFINITY;
-      if (a.out.dbg != nullptr && n < a.N) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int m = m0 + c * 32 + j;
-          if (m < a.M)
-            a.out.dbg[(a.out.dbg_rows ? (int64_t)a.out.dbg_rows[m] : (int64_t)m) * a.out.dbg_ld + n] = v[j];
+            for (int jj = 0; jj < 32; ++jj) {
+              const int m = w.m0 + c * 32 + jj;
+              if (m < a.M) out[(size_t)m * a.N + n] = v[jj];
+            }
+          }
         }
+      } else {
+        float* tr = lm_tr + q * kLmTr;
+        for (int c = 0; c < nchunk; ++c) {
+          float v[32];
+          tmem_ld32(tb + c * 32, v);
+          if (a.out.dbg != nullptr && n < a.N) {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+              const int m = w.m0 + c * 32 + jj;
+              if (m < a.M)
+                a.out.dbg[(a.out.dbg_rows ? (int64_t)a.out.dbg_rows[m] : (int64_t)m) *
+                              a.out.dbg_ld + n] = v[jj];
+            }
+          }
+          // transpose through shared memory: lane jj then owns token column jj
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) tr[jj * 33 + lane] = (n < a.N) ? v[jj] : -INFINITY;
+          __syncwarp();
+          const float* col = tr + lane * 33;
+          float mx = col[0];
+          int bi = 0;
+#pragma unroll 8
+          for (int i = 1; i < 32; ++i)
+            if (col[i] > mx) { mx = col[i]; bi = i; }
+          float se = 0.f;
+          if (mx != -INFINITY) {
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) se += expf(col[i] - mx);
+          }
+          LmStat st;
+          st.max = mx;
+          st.idx = w.n0 + q * 32 + bi;
+          st.sumexp = se;
+          st.pad = 0.f;
+          lm_part[q * kMaxBN + c * 32 + lane] = st;
+          __syncwarp();
+        }
+        epi_bar_sync();
+        // merge the four row groups (ascending vocabulary order) per token column
+        for (int col = threadIdx.x - kEpiWarp0 * 32; col < a.BN; col += 128) {
+          const int m = w.m0 + col;
+          if (m >= a.M) continue;
+          LmStat r = lm_part[col];
+          for (int g = 1; g < 4; ++g) {
+            const LmStat p = lm_part[g * kMaxBN + col];
+            if (p.max > r.max) {
+              r.sumexp = r.sumexp * expf(r.max - p.max) + p.sumexp;
+              r.max = p.max;
+              r.idx = p.idx;
+            } else {
+              r.sumexp += (p.max == -INFINITY) ? 0.f : p.sumexp * expf(p.max - r.max);
+            }
+          }
+          a.out.stats[(size_t)m * a.n_vtiles + w.n0 / kTileN] = r;
+        }
+        epi_bar_sync();
       }
-    }
-    __syncthreads();
-    for (int col = threadIdx.x; col < a.BN; col += blockDim.x) {
-      const int m = m0 + col;
-      if (m >= a.M) continue;
-      const float* t = tile + col * ld;
-      float mx = t[0];
-      int bi = 0;
-      for (int i = 1; i < kTileN; ++i) {
-        const float x = t[i];
-        if (x > mx) { mx = x; bi = i; }
-      }
-      float se = 0.f;
-      for (int i = 0; i < kTileN; ++i) se += expf(t[i] - mx);
-      LmStat st;
-      st.max = mx;
-      st.idx = n0 + bi;
-      st.sumexp = se;
-      st.pad = 0.f;
-      a.out.stats[(size_t)m * a.n_vtiles + blockIdx.x] = st;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty(b))
+                                  : "memory");
     }
   }
-
+  if (!ok) set_error(a.err, DFLASH_DEV_TIMEOUT);
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) tmem_dealloc(tmem, ncols);
+  if (warp == kEpiWarp0) tmem_dealloc(tmem, 2 * ncols);
 }
 
 // ---------------------------------------------------------------- host side
@@ -240,8 +321,8 @@ bool encode_2d(CUtensorMap* m, const void* ptr, int64_t rows, int cols, int ld, 
   cuuint32_t estr[2] = {1, 1};
   const CUtensorMapDataType dt =
       elem == DFLASH_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  CUresult r = enc(m, dt, 2, const_cast<void*>(ptr), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -263,19 +344,33 @@ int gemm_effective_splits(int K, int splits) {
   return (nkb + per - 1) / per;
 }
 
+static int num_sms() {
+  static int sms[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (sms[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    sms[dev] = v > 0 ? v : 148;
+  }
+  return sms[dev];
+}
+
 int gemm_pick_splits(int M, int N, int K, int max_splits) {
   const int tiles = ((N + kTileN - 1) / kTileN) * ((M + kMaxBN - 1) / kMaxBN);
   const int nkb = K / kTileK;
-  const int sms = 148;
+  const int sms = num_sms();
   int best = 1;
   double best_score = -1.0;
   // at least 4 k-blocks (256 of K) per split keeps the TMA pipeline busy
   const int smax = std::max(1, std::min(max_splits, nkb / 4));
   for (int s = 1; s <= smax; ++s) {
     const int se = gemm_effective_splits(K, s);
-    const int ctas = tiles * se;
-    const int waves = (ctas + sms - 1) / sms;
-    const double eff = (double)ctas / (waves * sms);
+    const int units = tiles * se;
+    // persistent CTAs: the busiest SM runs ceil(units / sms) units
+    const int per_sm = (units + sms - 1) / sms;
+    const double eff = (double)units / ((double)per_sm * sms);
     // each split writes (and its consumer reads) one fp32 partial of the
     // output: M*N*4*2 bytes next to the N*K*2 bytes of weights
     const double score = eff / (1.0 + 4.0 * se * (double)M / K);
@@ -312,36 +407,32 @@ int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, i
   a.n_kb = W.K / kTileK;
   if (epi == EPI_LMHEAD) splits = 1;
   splits = gemm_effective_splits(W.K, splits);
-  const long ctas = (long)((W.N + kTileN - 1) / kTileN) * ((M + BN - 1) / BN) * splits;
-  // More than one wave: ~100 KB per CTA so that two CTAs share an SM and one's
-  // prologue/epilogue overlaps the other's weight stream; otherwise one deep
-  // pipeline per SM.
-  int budget = ctas > 148 ? 100 * 1024 : 200 * 1024;
-  // the LM-head epilogue stages the BN x 128 fp32 tile (padded rows) in the stage buffers
-  const int lm_tile = BN * (kTileN + 1) * 4;
-  if (epi == EPI_LMHEAD && budget < lm_tile) budget = lm_tile;
-  a.stages = (budget + stage_bytes - 1) / stage_bytes;
-  if (a.stages > 8) a.stages = 8;
-  if (a.stages < 2) a.stages = 2;
-  if (epi == EPI_LMHEAD && a.stages * stage_bytes < lm_tile) return DFLASH_EUNSUPPORTED;
-  if (a.stages * stage_bytes > 210 * 1024) a.stages = 210 * 1024 / stage_bytes;
   a.kb_per_split = (a.n_kb + splits - 1) / splits;
-  a.n_vtiles = (W.N + kTileN - 1) / kTileN;
+  a.tiles_n = (W.N + kTileN - 1) / kTileN;
+  a.tiles_m = (M + BN - 1) / BN;
+  a.units = a.tiles_n * a.tiles_m * splits;
+  a.n_vtiles = a.tiles_n;
   a.idesc = idesc_f16kind(kTileN, BN, W.elem == DFLASH_BF16);
   a.out = out;
   a.err = err;
 
-  const size_t smem = (size_t)a.stages * stage_bytes + 1024 + 8 * (2 * a.stages + 2) + 64;
-  dim3 grid((W.N + kTileN - 1) / kTileN, (M + BN - 1) / BN, splits);
+  const size_t epi_bytes =
+      epi == EPI_LMHEAD ? 4 * kLmTr * sizeof(float) + 4 * kMaxBN * sizeof(LmStat) : 0;
+  const size_t fixed = 1024 + epi_bytes + 8 * (2 * 8 + 4) + 16;
+  const size_t cap = 227 * 1024;
+  a.stages = (int)std::min<size_t>(8, (cap - fixed) / stage_bytes);
+  if (a.stages < 2) return DFLASH_EUNSUPPORTED;
+  const size_t smem = fixed + (size_t)a.stages * stage_bytes;
+  const int grid = std::min(a.units, num_sms());
   TimedScope ts(s, epi == EPI_LMHEAD ? TC_LMHEAD : TC_GEMM);
   if (epi == EPI_PARTIAL) {
     cudaFuncSetAttribute(gemm_tc_kernel<EPI_PARTIAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    gemm_tc_kernel<EPI_PARTIAL><<<grid, 128, smem, s>>>(W.map, maps, a);
+    gemm_tc_kernel<EPI_PARTIAL><<<grid, kGemmThreads, smem, s>>>(W.map, maps, a);
   } else {
     cudaFuncSetAttribute(gemm_tc_kernel<EPI_LMHEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    gemm_tc_kernel<EPI_LMHEAD><<<grid, 128, smem, s>>>(W.map, maps, a);
+    gemm_tc_kernel<EPI_LMHEAD><<<grid, kGemmThreads, smem, s>>>(W.map, maps, a);
   }
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
