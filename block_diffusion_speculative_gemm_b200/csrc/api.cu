@@ -198,8 +198,12 @@ bool config_ok(const dflash_config& c) {
 
 bool config_supported(const dflash_config& c) {
   if (c.head_dim != 64 && c.head_dim != 128) return false;
+  if (c.inter % 64) return false;  // gate/up rows are packed in 64-row blocks
+  if (c.d % 64) return false;      // row kernels move 16-byte vectors
   if (c.dtype == DFLASH_BF16) {
-    if (c.d % 64 || c.H_t % 64 || c.inter % 64 || (c.n_q * c.head_dim) % 64) return false;
+    if (c.d % 64 || c.H_t % 64 || (c.n_q * c.head_dim) % 128) return false;
+    // fused epilogues need every 128-row weight tile to hold whole heads
+    if ((c.n_kv * c.head_dim) % 128) return false;
   } else {
     const int kmax = std::max(std::max(c.n_tap * c.H_t, c.d), std::max(c.inter, c.n_q * c.head_dim));
     if (kmax > 12288) return false;  // SIMT GEMM keeps one token row in shared memory
@@ -210,6 +214,7 @@ bool config_supported(const dflash_config& c) {
 int qkv_out(const dflash_config& c) { return (c.n_q + 2 * c.n_kv) * c.head_dim; }
 
 // ---------------------------------------------------------------- workspace layout
+// Workspace header: word 0 = device error bits.
 constexpr size_t kHeader = 256;
 constexpr int kMaxChunks = 64;
 constexpr int kAttnRows = 64;
@@ -221,11 +226,11 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct DraftLayout {
   size_t tokens, zrow, lm_rows, cstep, req_valid, lm_tok, lm_conf, x, h, q, kb, vb, o, act, part,
       attn_o, attn_ml, stats, logits, end;
-  size_t part_elems;
+  size_t part_elems;  // fp32 elements of split-K partials
 };
 
 struct InjectLayout {
-  size_t c, part, end;
+  size_t c, u, part, end;
   size_t part_elems;
   int chunk_rows;
 };
@@ -280,6 +285,8 @@ InjectLayout inject_layout(const dflash_config& c, int max_rows) {
   size_t off = kHeader;
   L.c = off;
   off = align256(off + esz * n * c.d);
+  L.u = off;  // fc output before its RMSNorm (fp32)
+  off = align256(off + 4 * n * c.d);
   // small row counts may split K up to kMaxSplits ways
   L.part_elems = (n <= 256 ? (size_t)kMaxSplits : 1) * n * ncol;
   L.part = off;
@@ -305,12 +312,28 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 int cuda_status() { return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA; }
 
 // Split count for a draft/inject GEMM: the picker's choice, lowered until the
-// partials fit the workspace; always a count gemm_tc runs unchanged.
+// split partials fit the workspace; always a count gemm_tc runs unchanged.
+// One split means the GEMM applies the following step itself (fused op).
 int splits_for(int M, int N, int K, size_t cap_elems) {
   int s = gemm_pick_splits(M, N, K, kMaxSplits);
   const size_t fit = std::max<size_t>(1, cap_elems / ((size_t)M * N));
-  while ((size_t)s > fit) s = gemm_effective_splits(K, s - 1);
+  while (s > 1 && (size_t)s > fit) s = gemm_effective_splits(K, s - 1);
   return s;
+}
+
+// Gate and up projections packed for the fused SwiGLU epilogue: 128-row blocks
+// holding 64 gate rows, then the 64 up rows of the same features.
+template <typename Tin, typename Tout>
+__global__ void pack_gu_kernel(const Tin* __restrict__ wg, const Tin* __restrict__ wu,
+                               Tout* __restrict__ out, int I, int d) {
+  const size_t total = (size_t)2 * I * d;
+  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int n = (int)(idx / d), k = (int)(idx % d);
+    const int blk = n >> 7, w = n & 127;
+    const Tin* src = (w < 64 ? wg : wu) + ((size_t)(blk * 64 + (w & 63))) * d + k;
+    out[idx] = from_f<Tout>(to_f(*src));
+  }
 }
 
 }  // namespace
@@ -376,10 +399,22 @@ extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weight
     if (!pack_weights(m, qkv, lw.Wq, nq * hd * d) ||
         !pack_weights(m, qkv + e * nq * hd * d, lw.Wk, kvrows * d) ||
         !pack_weights(m, qkv + e * (nq * hd + kvrows) * d, lw.Wv, kvrows * d) ||
-        !pack_weights(m, P.Wo, lw.Wo, d * nq * hd) || !pack_weights(m, gu, lw.Wg, I * d) ||
-        !pack_weights(m, gu + e * I * d, lw.Wu, I * d) || !pack_weights(m, P.Wd, lw.Wd, d * I) ||
+        !pack_weights(m, P.Wo, lw.Wo, d * nq * hd) || !lw.Wg || !lw.Wu ||
+        !pack_weights(m, P.Wd, lw.Wd, d * I) ||
         !pack_weights(m, kv, lw.Wk, kvrows * d) || !pack_weights(m, kv + e * kvrows * d, lw.Wv, kvrows * d))
       return fail(DFLASH_EINVAL);
+    {
+      const unsigned blocks = (unsigned)std::min<size_t>((2 * I * d + 255) / 256, 148 * 32);
+      if (c.dtype == DFLASH_BF16)
+        pack_gu_kernel<__nv_bfloat16, __half><<<blocks, 256>>>(
+            static_cast<const __nv_bfloat16*>(lw.Wg), static_cast<const __nv_bfloat16*>(lw.Wu),
+            static_cast<__half*>((void*)gu), (int)I, (int)d);
+      else
+        pack_gu_kernel<float, float><<<blocks, 256>>>(static_cast<const float*>(lw.Wg),
+                                                     static_cast<const float*>(lw.Wu),
+                                                     static_cast<float*>((void*)gu), (int)I,
+                                                     (int)d);
+    }
     P.g_in = gain_copy(m, lw.g_in);
     P.g_post = gain_copy(m, lw.g_post);
     if (!P.g_in || !P.g_post) return fail(DFLASH_EINVAL);
@@ -484,20 +519,47 @@ extern "C" int dflash_inject_kv(const dflash_model* m, const void* const* taps,
     void* cbuf = at<void>(ws, L.c);
     int st;
     if (c.dtype == DFLASH_BF16) {
+      // u = concat(taps) W_fc^T, c = RMSNorm(u; g_ctx)
       const int s1 = splits_for(n, c.d, c.n_tap * c.H_t, L.part_elems);
-      GemmOut o;
-      o.part = part;
-      st = gemm_tc(m->mfc, seg, c.n_tap, c.H_t, c.H_t, n, s1, EPI_PARTIAL, o, err, s);
+      GemmOut o1;
+      if (s1 == 1) {
+        o1.op = OP_STORE;
+        o1.f32 = at<float>(ws, L.u);
+      } else {
+        o1.part = part;
+      }
+      st = gemm_tc(m->mfc, seg, c.n_tap, c.H_t, c.H_t, n, s1, EPI_PARTIAL, o1, err, s);
       if (st) return st;
-      launch_ctx_norm<__half>(part, s1, n, c.d, m->g_ctx, static_cast<__half*>(cbuf), c.eps, s);
+      launch_ctx_norm<__half>(s1 == 1 ? o1.f32 : part, s1, n, c.d, m->g_ctx,
+                              static_cast<__half*>(cbuf), c.eps, s);
+      // every layer's K (RoPE) and V into the cache
       const int s2 = splits_for(n, kvN, c.d, L.part_elems);
       const void* cseg[1] = {cbuf};
-      st = gemm_tc(m->mkv, cseg, 1, c.d, c.d, n, s2, EPI_PARTIAL, o, err, s);
+      GemmOut o2;
+      if (s2 == 1) {
+        o2.op = OP_KV;
+        o2.h1 = static_cast<__half*>(k_cache);
+        o2.h2 = static_cast<__half*>(v_cache);
+        o2.cos_t = m->rope_cos;
+        o2.sin_t = m->rope_sin;
+        o2.cu_rows = cu_rows;
+        o2.start_pos = start_pos;
+        o2.nkv = c.n_kv;
+        o2.hd = c.head_dim;
+        o2.row0 = r0;
+        o2.batch = batch;
+        o2.cap = cache_cap;
+        o2.max_pos = c.max_pos;
+      } else {
+        o2.part = part;
+      }
+      st = gemm_tc(m->mkv, cseg, 1, c.d, c.d, n, s2, EPI_PARTIAL, o2, err, s);
       if (st) return st;
-      launch_kv_scatter<__half>(part, s2, n, r0, c.n_layers, c.n_kv, c.head_dim, cu_rows,
-                                       start_pos, batch, cache_cap, m->rope_cos, m->rope_sin,
-                                       c.max_pos, static_cast<__half*>(k_cache),
-                                       static_cast<__half*>(v_cache), err, s);
+      if (s2 > 1)
+        launch_kv_scatter<__half>(part, s2, n, r0, c.n_layers, c.n_kv, c.head_dim, cu_rows,
+                                  start_pos, batch, cache_cap, m->rope_cos, m->rope_sin,
+                                  c.max_pos, static_cast<__half*>(k_cache),
+                                  static_cast<__half*>(v_cache), err, s);
     } else {
       const float* fseg[kMaxSeg];
       for (int t = 0; t < c.n_tap; ++t) fseg[t] = static_cast<const float*>(seg[t]);
@@ -583,6 +645,53 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
                          c.eps, s);
     for (int l = 0; l < c.n_layers; ++l) {
       const LayerPack& P = m->layers[l];
+      const float* g_next = l + 1 < c.n_layers ? m->layers[l + 1].g_in : m->g_final;
+      const int32_t* next_rows = l + 1 < c.n_layers ? nullptr : zrow;
+      if (bf16) {
+        // an unsplit GEMM applies the next step in its epilogue; a split one
+        // leaves partials (in L2) for the reduction kernel of that step
+        GemmOut go;
+        go.part = part;
+        go.cos_t = m->rope_cos;
+        go.sin_t = m->rope_sin;
+        go.ctx_len = ctx_len;
+        go.req_valid = valid;
+        go.B = B;
+        go.nq = nq;
+        go.nkv = nkv;
+        go.hd = hd;
+        go.I = c.inter;
+        int sp = 1;
+        auto run = [&](const WeightMap& W, int N, int K, const void* X, int op) {
+          sp = splits_for(M, N, K, L.part_elems);
+          GemmOut g2 = go;
+          g2.op = sp == 1 ? op : OP_PARTIAL;
+          const void* seg[1] = {X};
+          return gemm_tc(W, seg, 1, K, K, M, sp, EPI_PARTIAL, g2, err, s);
+        };
+        go.h1 = reinterpret_cast<__half*>(q);
+        go.h2 = reinterpret_cast<__half*>(kb);
+        go.h3 = reinterpret_cast<__half*>(vb);
+        if ((st = run(P.mqkv, qkv_out(c), c.d, h, OP_QKV))) return st;
+        if (sp > 1)
+          launch_qkv_post<T>(part, sp, M, B, ctx_len, valid, nq, nkv, hd, m->rope_cos,
+                             m->rope_sin, q, kb, vb, s);
+        if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, l, c.n_layers, batch, cap,
+                                                ctx_len, valid, B, nq, nkv, hd, attn_o, attn_ml,
+                                                n_chunks, chunk, o, err, s)))
+          return st;
+        go.f32 = x;
+        if ((st = run(P.mo, c.d, nq * hd, o, OP_RESID))) return st;
+        launch_residual_norm<T>(sp > 1 ? part : nullptr, sp, M, c.d, x, P.g_post, h, nullptr,
+                                c.eps, s);
+        go.h1 = reinterpret_cast<__half*>(act);
+        if ((st = run(P.mgu, 2 * c.inter, c.d, h, OP_SWIGLU))) return st;
+        if (sp > 1) launch_swiglu<T>(part, sp, M, c.inter, act, s);
+        if ((st = run(P.md, c.d, c.inter, act, OP_RESID))) return st;
+        launch_residual_norm<T>(sp > 1 ? part : nullptr, sp, M, c.d, x, g_next, h, next_rows,
+                                c.eps, s);
+        continue;
+      }
       int sp = 1;
       if ((st = gemm(P.mqkv, P.Wqkv, qkv_out(c), c.d, h, part, L.part_elems, &sp))) return st;
       launch_qkv_post<T>(part, sp, M, B, ctx_len, valid, nq, nkv, hd, m->rope_cos, m->rope_sin,
@@ -596,10 +705,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
       if ((st = gemm(P.mgu, P.Wgu, 2 * c.inter, c.d, h, part, L.part_elems, &sp))) return st;
       launch_swiglu<T>(part, sp, M, c.inter, act, s);
       if ((st = gemm(P.md, P.Wd, c.d, c.inter, act, part, L.part_elems, &sp))) return st;
-      if (l + 1 < c.n_layers)
-        launch_residual_norm<T>(part, sp, M, c.d, x, m->layers[l + 1].g_in, h, nullptr, c.eps, s);
-      else
-        launch_residual_norm<T>(part, sp, M, c.d, x, m->g_final, h, zrow, c.eps, s);
+      launch_residual_norm<T>(part, sp, M, c.d, x, g_next, h, next_rows, c.eps, s);
     }
     // LM head over the still-masked rows (compact, request-major)
     const int rows = batch * rem;

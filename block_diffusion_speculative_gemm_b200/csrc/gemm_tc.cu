@@ -21,7 +21,9 @@
 //   warps 2..5         epilogue: drain the accumulator of unit j while the
 //                      MMA warp fills the other one for unit j + 1, then give it
 //                      back.  PARTIAL: coalesced fp32 store of the split's
-//                      partial product.  LMHEAD: per token and 128-row
+//                      partial product (kept in L2 for the reduction kernel),
+//                      or, for an unsplit GEMM, a fused step (residual add,
+//                      RoPE + q/k/v split, SwiGLU, K/V cache scatter).  LMHEAD: per token and 128-row
 //                      vocabulary tile, the maximum, its lowest index and the
 //                      sum of exp(logit - max), through per-warp 32 x 33 shared
 //                      transposes (no fp32 logits leave the SM).
@@ -50,6 +52,7 @@ struct GemmArgs {
   int tiles_n;        // weight tiles
   int tiles_m;        // token tiles
   int units;          // tiles_n * tiles_m * splits
+  int splits;
   int n_vtiles;       // LM head: number of 128-row vocabulary tiles (= tiles_n)
   uint32_t idesc;     // tcgen05 instruction descriptor (operand type, 128 x BN)
   GemmOut out;
@@ -59,6 +62,99 @@ struct GemmArgs {
 constexpr int kGemmThreads = 192;
 constexpr int kEpiWarp0 = 2;  // first epilogue warp
 constexpr int kLmTr = 32 * 33;  // floats of one warp's transpose buffer
+constexpr int kStLd = kTileN + 1; // row stride of the fused-op staging tile [32 tokens][128 rows]
+constexpr int kFusedSmem = 32 * kStLd * 4 + 64 * 4 + 16;  // staging tile + token maps + flag
+constexpr int kLmSmem = 4 * kLmTr * 4 + 4 * kMaxBN * (int)sizeof(LmStat);
+
+// Applies the fused op to one 32-token chunk of a finished output tile.
+// st[j * kStLd + r] = Y[m_base + j][n0 + r]; t = epilogue thread (0..127).
+// For OP_KV, tok_req/tok_pos hold each token's request and cache position
+// (request -1: skip).
+__device__ __forceinline__ void apply_op(const GemmOut& o, int M, int N, const float* st,
+                                         const int* tok_req, const int* tok_pos, int m_base,
+                                         int n0, int t) {
+  switch (o.op) {
+    case OP_STORE:
+    case OP_RESID: {
+      const int n = n0 + t;
+      if (n >= N) break;
+      for (int j = 0; j < 32; ++j) {
+        const int m = m_base + j;
+        if (m >= M) break;
+        float* d = o.f32 + (size_t)m * N + n;
+        *d = (o.op == OP_RESID ? *d : 0.f) + st[j * kStLd + t];
+      }
+    } break;
+    case OP_SWIGLU: {
+      const int p = t & 63, par = t >> 6;
+      const int i = (n0 >> 1) + p;
+      for (int j = par; j < 32; j += 2) {
+        const int m = m_base + j;
+        if (m >= M) break;
+        const float g = st[j * kStLd + p], u = st[j * kStLd + p + 64];
+        o.h1[(size_t)m * o.I + i] = __float2half_rn(g / (1.f + expf(-g)) * u);
+      }
+    } break;
+    case OP_QKV: {
+      const int hd = o.hd, half = hd >> 1;
+      const int p = t & 63, par = t >> 6;
+      const int hl = p / half, i = p % half;
+      const int ra = hl * hd + i;
+      const int head = (n0 + hl * hd) / hd;
+      for (int j = par; j < 32; j += 2) {
+        const int m = m_base + j;
+        if (m >= M) break;
+        float x1 = st[j * kStLd + ra], x2 = st[j * kStLd + ra + half];
+        __half* dst;
+        if (head < o.nq + o.nkv) {
+          const int r = m / o.B;
+          const int pos = (o.req_valid[r] ? o.ctx_len[r] : 0) + m % o.B;
+          const float c = o.cos_t[(size_t)pos * half + i], sn = o.sin_t[(size_t)pos * half + i];
+          const float y1 = x1 * c - x2 * sn, y2 = x2 * c + x1 * sn;
+          x1 = y1;
+          x2 = y2;
+          dst = head < o.nq ? o.h1 + ((size_t)m * o.nq + head) * hd
+                            : o.h2 + ((size_t)m * o.nkv + head - o.nq) * hd;
+        } else {
+          dst = o.h3 + ((size_t)m * o.nkv + head - o.nq - o.nkv) * hd;
+        }
+        dst[i] = __float2half_rn(x1);
+        dst[i + half] = __float2half_rn(x2);
+      }
+    } break;
+    case OP_KV: {
+      const int hd = o.hd, half = hd >> 1;
+      const int p = t & 63, par = t >> 6;
+      const int hl = p / half, i = p % half;
+      const int ra = hl * hd + i;
+      const int per_layer = 2 * o.nkv * hd;
+      const int nl = n0 + hl * hd;
+      const int layer = nl / per_layer, wl = nl % per_layer;
+      const bool is_v = wl >= o.nkv * hd;
+      const int head = (wl % (o.nkv * hd)) / hd;
+      for (int j = par; j < 32; j += 2) {
+        const int m = m_base + j;
+        if (m >= M) break;
+        const int req = tok_req[j];
+        if (req < 0) continue;
+        const int pos = tok_pos[j];
+        float x1 = st[j * kStLd + ra], x2 = st[j * kStLd + ra + half];
+        if (!is_v) {
+          const float c = o.cos_t[(size_t)pos * half + i], sn = o.sin_t[(size_t)pos * half + i];
+          const float y1 = x1 * c - x2 * sn, y2 = x2 * c + x1 * sn;
+          x1 = y1;
+          x2 = y2;
+        }
+        __half* dst = (is_v ? o.h2 : o.h1) +
+                      ((((size_t)layer * o.batch + req) * o.nkv + head) * o.cap + pos) * hd;
+        dst[i] = __float2half_rn(x1);
+        dst[i + half] = __float2half_rn(x2);
+      }
+    } break;
+    default:
+      break;
+  }
+}
 
 __host__ __device__ inline int tmem_cols_for(int bn) {
   int c = 32;
@@ -67,7 +163,7 @@ __host__ __device__ inline int tmem_cols_for(int bn) {
 }
 
 struct Unit {
-  int n0, m0, split, kb0, nk;
+  int n0, m0, split, kb0, nk, tile;
 };
 
 __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
@@ -75,11 +171,16 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
   const int per = a.tiles_n * a.tiles_m;
   w.split = u / per;
   const int rem = u % per;
+  w.tile = rem;
   w.m0 = (rem / a.tiles_n) * a.BN;
   w.n0 = (rem % a.tiles_n) * kTileN;
   w.kb0 = w.split * a.kb_per_split;
   w.nk = min(a.n_kb, w.kb0 + a.kb_per_split) - w.kb0;
   return w;
+}
+
+__device__ __forceinline__ void st_keep(float* p, float v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
 }
 
 __device__ __forceinline__ void epi_bar_sync() {
@@ -107,11 +208,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int stage_bytes = kTileN * 128 + a.BN * 128;
-  // [stages][A | B] | LM-head transposes + partials | barriers
-  float* lm_tr = reinterpret_cast<float*>(smem + a.stages * stage_bytes);
-  LmStat* lm_part = reinterpret_cast<LmStat*>(lm_tr + (EPI == EPI_LMHEAD ? 4 * kLmTr : 0));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(
-      reinterpret_cast<uint8_t*>(lm_part) + (EPI == EPI_LMHEAD ? 4 * kMaxBN * sizeof(LmStat) : 0));
+  // [stages][A | B] | epilogue region (LM-head transposes + partials, or the
+  // fused-op staging tile + token maps + flag) | barriers
+  uint8_t* epi_smem = smem + a.stages * stage_bytes;
+  float* lm_tr = reinterpret_cast<float*>(epi_smem);
+  LmStat* lm_part = reinterpret_cast<LmStat*>(lm_tr + 4 * kLmTr);
+  float* st = reinterpret_cast<float*>(epi_smem);
+  int* tok_req = reinterpret_cast<int*>(st + 32 * kStLd);
+  int* tok_pos = tok_req + 32;
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(epi_smem + (EPI == EPI_LMHEAD ? kLmSmem : kFusedSmem));
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * a.stages + 4);
   const uint32_t smem0 = smem_u32(smem);
   auto sA = [&](int s) { return smem0 + s * stage_bytes; };
@@ -154,12 +260,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t it = 0;
       for (int u = blockIdx.x; u < a.units && ok; u += gridDim.x) {
         const Unit w = decode_unit(a, u);
+        // each CTA starts its K walk at its own offset so that the SMs do not
+        // all request the same activation rows of L2 at the same moment
+        const int rot = (int)((blockIdx.x * 7u) % (unsigned)w.nk);
         for (int i = 0; i < w.nk; ++i, ++it) {
           const int s = it % a.stages;
           const uint32_t ph = (it / a.stages) & 1;
           if (!mbar_wait(empty(s), ph ^ 1)) { ok = false; break; }
           mbar_arrive_expect_tx(full(s), stage_bytes);
-          const int kx = (w.kb0 + i) * kTileK;
+          int ki = i + rot;
+          if (ki >= w.nk) ki -= w.nk;
+          const int kx = (w.kb0 + ki) * kTileK;
           tma_load_2d(sA(s), &tmA, full(s), kx, w.n0, pol_w);
           const int seg = kx / a.seg_k;
           tma_load_2d(sB(s), &tmB.m[seg], full(s), kx - seg * a.seg_k, w.m0, pol_x);
@@ -203,26 +314,75 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const Unit w = decode_unit(a, u);
       const int b = j & 1;
       bool got = mbar_wait(acc_full(b), (j >> 1) & 1);
-      if (EPI == EPI_LMHEAD) got = epi_bar_and(got);  // the epilogue warps leave together
+      got = epi_bar_and(got);  // the epilogue warps leave together
       __syncwarp();
       if (!got) { ok = false; break; }
       tc_fence_after();
       const uint32_t tb = tmem + b * ncols + ((uint32_t)(q * 32) << 16);
       const int n = w.n0 + row;
-      if (EPI == EPI_PARTIAL) {
+      const int et = threadIdx.x - kEpiWarp0 * 32;
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty(b)) : "memory");
+      };
+      // token -> (request, cache position) for OP_KV, one thread per token of the chunk
+      auto token_maps = [&](int m_base) {
+        if (a.out.op != OP_KV || et >= 32) return;
+        const int m = m_base + et;
+        int req = -1, pos = 0;
+        if (m < a.M) {
+          const int nrow = a.out.row0 + m;
+          int lo = 0, hi = a.out.batch - 1;
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (a.out.cu_rows[mid] <= nrow) lo = mid; else hi = mid - 1;
+          }
+          if (nrow < a.out.cu_rows[lo] || nrow >= a.out.cu_rows[lo + 1]) {
+            set_error(a.err, DFLASH_DEV_ROWS);
+          } else {
+            pos = a.out.start_pos[lo] + (nrow - a.out.cu_rows[lo]);
+            if (pos < 0 || pos >= a.out.cap || pos >= a.out.max_pos)
+              set_error(a.err, DFLASH_DEV_CTX_CAP);
+            else
+              req = lo;
+          }
+        }
+        tok_req[et] = req;
+        tok_pos[et] = pos;
+      };
+      if (EPI == EPI_PARTIAL && a.out.op == OP_PARTIAL) {
+        // partials are read back right away by the reduction kernel: keep them in L2
+        const uint64_t keep = policy_evict_last();
         float* out = a.out.part + (size_t)w.split * a.M * a.N;
         for (int c = 0; c < nchunk; ++c) {
-          if (w.m0 + c * 32 >= a.M) break;  // uniform across the warp
+          if (w.m0 + c * 32 >= a.M) break;  // uniform across the CTA
           float v[32];
           tmem_ld32(tb + c * 32, v);
           if (n < a.N) {
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
               const int m = w.m0 + c * 32 + jj;
-              if (m < a.M) out[(size_t)m * a.N + n] = v[jj];
+              if (m < a.M) st_keep(out + (size_t)m * a.N + n, v[jj], keep);
             }
           }
         }
+        release();
+      } else if (EPI == EPI_PARTIAL && a.splits == 1) {
+        // the whole K range is in TMEM: apply the op chunk by chunk
+        for (int c = 0; c < nchunk; ++c) {
+          if (w.m0 + c * 32 >= a.M) break;
+          float v[32];
+          tmem_ld32(tb + c * 32, v);
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) st[jj * kStLd + row] = v[jj];
+          token_maps(w.m0 + c * 32);
+          epi_bar_sync();
+          apply_op(a.out, a.M, a.N, st, tok_req, tok_pos, w.m0 + c * 32, w.n0, et);
+          epi_bar_sync();
+        }
+        release();
       } else {
         float* tr = lm_tr + q * kLmTr;
         for (int c = 0; c < nchunk; ++c) {
@@ -280,10 +440,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         epi_bar_sync();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty(b))
-                                  : "memory");
+      if (EPI == EPI_LMHEAD) release();
     }
   }
   if (!ok) set_error(a.err, DFLASH_DEV_TIMEOUT);
@@ -411,13 +568,15 @@ int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, i
   a.tiles_n = (W.N + kTileN - 1) / kTileN;
   a.tiles_m = (M + BN - 1) / BN;
   a.units = a.tiles_n * a.tiles_m * splits;
+  a.splits = splits;
+  // fused ops need the whole K range in one unit
+  if (epi == EPI_PARTIAL && out.op != OP_PARTIAL && splits > 1) return DFLASH_EINVAL;
   a.n_vtiles = a.tiles_n;
   a.idesc = idesc_f16kind(kTileN, BN, W.elem == DFLASH_BF16);
   a.out = out;
   a.err = err;
 
-  const size_t epi_bytes =
-      epi == EPI_LMHEAD ? 4 * kLmTr * sizeof(float) + 4 * kMaxBN * sizeof(LmStat) : 0;
+  const size_t epi_bytes = epi == EPI_LMHEAD ? kLmSmem : kFusedSmem;
   const size_t fixed = 1024 + epi_bytes + 8 * (2 * 8 + 4) + 16;
   const size_t cap = 227 * 1024;
   a.stages = (int)std::min<size_t>(8, (cap - fixed) / stage_bytes);

@@ -38,13 +38,46 @@ struct LmStat {                // per (token row, 128-wide vocab tile)
 
 enum GemmEpi { EPI_PARTIAL = 0, EPI_LMHEAD = 1 };
 
+// What the EPI_PARTIAL kernel does with the product Y[m][n] = sum_k X[m][k] W[n][k].
+// OP_PARTIAL writes each K split's share (fp32, for a reduction kernel); the
+// other ops need an unsplit GEMM and apply the step that follows the
+// projection on the hot path straight from the accumulator.
+enum GemmOp {
+  OP_PARTIAL = 0,  // part[split][m][n] = split's share                         (fp32)
+  OP_STORE = 1,    // f32[m][n] = Y                                             (fp32)
+  OP_RESID = 2,    // f32[m][n] += Y   (the residual stream)                    (fp32)
+  OP_QKV = 3,      // Y = [q heads | k heads | v heads]: RoPE on q and k at position
+                   // ctx_len[m / B] + m % B; h1 = q [M][nq][hd], h2 = k [M][nkv][hd],
+                   // h3 = v [M][nkv][hd]                                       (fp16)
+  OP_SWIGLU = 4,   // weight rows interleaved in 64-row blocks (64 gate rows, then the
+                   // 64 up rows of the same features): h1 = act [M][I] = silu(g) * u
+  OP_KV = 5,       // Y = per layer [K heads | V heads] of injected rows row0 + m:
+                   // RoPE on K at start_pos[r] + row - cu_rows[r]; h1/h2 = K/V cache
+                   // [L][batch][nkv][cap][hd] (fp16); bad positions set err, skip
+};
+
 struct GemmOut {
-  float* part = nullptr;          // EPI_PARTIAL: [splits][M][N] fp32
+  int op = OP_PARTIAL;
+  float* part = nullptr;          // OP_PARTIAL: [splits][M][N] fp32
   LmStat* stats = nullptr;        // EPI_LMHEAD: [M][ceil(N/128)]
   float* dbg = nullptr;           // EPI_LMHEAD, optional: logits rows
   const int32_t* dbg_rows = nullptr;  // token row -> dbg row
   int64_t dbg_ld = 0;             // dbg row stride (elements)
+  // fused ops
+  float* f32 = nullptr;           // OP_STORE / OP_RESID: [M][N]
+  __half* h1 = nullptr;
+  __half* h2 = nullptr;
+  __half* h3 = nullptr;
+  const float* cos_t = nullptr;   // RoPE tables [max_pos][hd/2]
+  const float* sin_t = nullptr;
+  const int32_t* ctx_len = nullptr;    // OP_QKV
+  const int32_t* req_valid = nullptr;  // OP_QKV
+  const int32_t* cu_rows = nullptr;    // OP_KV
+  const int32_t* start_pos = nullptr;  // OP_KV
+  int B = 0, nq = 0, nkv = 0, hd = 0, I = 0;
+  int row0 = 0, batch = 0, cap = 0, max_pos = 0;
 };
+
 
 // A weight operand prepared once: tensor map over [N, K] rows of 16-bit
 // elements (elem = DFLASH_BF16 or DFLASH_F16).  The activation operand of a

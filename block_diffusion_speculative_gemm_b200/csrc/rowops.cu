@@ -18,6 +18,41 @@ __device__ __forceinline__ float sum_splits(const float* part, int splits, size_
   return v;
 }
 
+// Sum of the K-split partials of 4 consecutive fp32 elements (16-byte aligned
+// index), in ascending split order.  Partials are dead after this read.
+__device__ __forceinline__ float4 sum_splits4(const float* part, int splits, size_t stride,
+                                              size_t idx) {
+  float4 v = __ldcs(reinterpret_cast<const float4*>(part + idx));
+  for (int s = 1; s < splits; ++s) {
+    const float4 w = __ldcs(reinterpret_cast<const float4*>(part + (size_t)s * stride + idx));
+    v.x += w.x;
+    v.y += w.y;
+    v.z += w.z;
+    v.w += w.w;
+  }
+  return v;
+}
+
+template <typename T>
+__device__ __forceinline__ void store4(T* dst, float a, float b, float c, float d) {
+  dst[0] = from_f<T>(a);
+  dst[1] = from_f<T>(b);
+  dst[2] = from_f<T>(c);
+  dst[3] = from_f<T>(d);
+}
+template <>
+__device__ __forceinline__ void store4<__half>(__half* dst, float a, float b, float c, float d) {
+  __half2 lo = __floats2half2_rn(a, b), hi = __floats2half2_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&lo);
+  u.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(dst) = u;
+}
+template <>
+__device__ __forceinline__ void store4<float>(float* dst, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(dst) = make_float4(a, b, c, d);
+}
+
 // ---------------------------------------------------------------- embedding + RMSNorm
 // x[m] = emb[tokens[m]] (fp32 residual stream); h[m] = RMSNorm(x[m]; g).
 template <typename TE, typename T>
@@ -57,8 +92,9 @@ void launch_embed_norm(const int32_t* tokens, const TE* emb, const float* g, flo
 }
 
 // ---------------------------------------------------------------- residual + RMSNorm
-// x[m] += sum_s part[s][m]; h[out_row[m]] = RMSNorm(x[m]; g) (all rows when
-// out_row is null; rows with out_row < 0 are not written).
+// x[m] += sum_s part[s][m] (skipped when part is null); h[out_row[m]] =
+// RMSNorm(x[m]; g) (all rows when out_row is null; rows with out_row < 0 are
+// not written).
 template <typename T>
 __global__ void __launch_bounds__(kRowThreads)
     residual_norm_kernel(const float* __restrict__ part, int splits, int M, int d,
@@ -67,27 +103,39 @@ __global__ void __launch_bounds__(kRowThreads)
   __shared__ float red[32];
   const int m = blockIdx.x;
   const size_t stride = (size_t)M * d;
-  float v[kMaxRowElems];
+  constexpr int kV = kMaxRowElems / 4;  // float4 per thread
+  float4 v[kV];
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxRowElems; ++i) {
-    const int c = threadIdx.x + i * kRowThreads;
+  for (int i = 0; i < kV; ++i) {
+    const int c = (threadIdx.x + i * kRowThreads) * 4;
     if (c < d) {
       const size_t idx = (size_t)m * d + c;
-      v[i] = x[idx] + sum_splits(part, splits, stride, idx);
-      x[idx] = v[i];
+      v[i] = *reinterpret_cast<const float4*>(x + idx);
+      if (part != nullptr) {
+        const float4 p = sum_splits4(part, splits, stride, idx);
+        v[i].x += p.x;
+        v[i].y += p.y;
+        v[i].z += p.z;
+        v[i].w += p.w;
+        *reinterpret_cast<float4*>(x + idx) = v[i];
+      }
     } else {
-      v[i] = 0.f;
+      v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    ss += v[i] * v[i];
+    ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
   }
   const float inv = rsqrtf(block_sum(ss, red) / d + eps);
   const int orow = out_row ? out_row[m] : m;
   if (orow < 0) return;
 #pragma unroll
-  for (int i = 0; i < kMaxRowElems; ++i) {
-    const int c = threadIdx.x + i * kRowThreads;
-    if (c < d) h[(size_t)orow * d + c] = from_f<T>(v[i] * inv * g[c]);
+  for (int i = 0; i < kV; ++i) {
+    const int c = (threadIdx.x + i * kRowThreads) * 4;
+    if (c < d) {
+      const float4 gg = *reinterpret_cast<const float4*>(g + c);
+      store4<T>(h + (size_t)orow * d + c, v[i].x * inv * gg.x, v[i].y * inv * gg.y,
+                v[i].z * inv * gg.z, v[i].w * inv * gg.w);
+    }
   }
 }
 
@@ -96,7 +144,8 @@ void launch_residual_norm(const float* part, int splits, int M, int d, float* x,
                           T* h, const int32_t* out_row, float eps, cudaStream_t s) {
   if (M <= 0) return;
   TimedScope ts(s, TC_ROW);
-  residual_norm_kernel<T><<<M, kRowThreads, 0, s>>>(part, splits, M, d, x, g, h, out_row, eps);
+  residual_norm_kernel<T><<<M, kRowThreads, 0, s>>>(part, splits, M, d, x, g, h, out_row,
+                                                         eps);
 }
 
 // ---------------------------------------------------------------- context-feature RMSNorm
@@ -108,19 +157,25 @@ __global__ void __launch_bounds__(kRowThreads)
   __shared__ float red[32];
   const int n = blockIdx.x;
   const size_t stride = (size_t)n_rows * d;
-  float v[kMaxRowElems];
+  constexpr int kV = kMaxRowElems / 4;
+  float4 v[kV];
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxRowElems; ++i) {
-    const int col = threadIdx.x + i * kRowThreads;
-    v[i] = col < d ? sum_splits(part, splits, stride, (size_t)n * d + col) : 0.f;
-    ss += v[i] * v[i];
+  for (int i = 0; i < kV; ++i) {
+    const int col = (threadIdx.x + i * kRowThreads) * 4;
+    v[i] = col < d ? sum_splits4(part, splits, stride, (size_t)n * d + col)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
   }
   const float inv = rsqrtf(block_sum(ss, red) / d + eps);
 #pragma unroll
-  for (int i = 0; i < kMaxRowElems; ++i) {
-    const int col = threadIdx.x + i * kRowThreads;
-    if (col < d) c[(size_t)n * d + col] = from_f<T>(v[i] * inv * g[col]);
+  for (int i = 0; i < kV; ++i) {
+    const int col = (threadIdx.x + i * kRowThreads) * 4;
+    if (col < d) {
+      const float4 gg = *reinterpret_cast<const float4*>(g + col);
+      store4<T>(c + (size_t)n * d + col, v[i].x * inv * gg.x, v[i].y * inv * gg.y,
+                v[i].z * inv * gg.z, v[i].w * inv * gg.w);
+    }
   }
 }
 
@@ -146,26 +201,31 @@ __global__ void qkv_post_kernel(const float* __restrict__ part, int splits, int 
   const int half = hd / 2;
   const int nh = nq + 2 * nkv;
   const int N = nh * hd;
-  const int p = blockIdx.x * blockDim.x + threadIdx.x;
-  if (p >= nh * half) return;
-  const int head = p / half, i = p % half;
+  const int p4 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;  // first of 4 pairs
+  if (p4 >= nh * half) return;
+  const int head = p4 / half, i = p4 % half;
   const int r = m / B, j = m % B;
   const int pos = (req_valid[r] ? ctx_len[r] : 0) + j;
   const size_t stride = (size_t)M * N;
   const size_t c0 = (size_t)m * N + head * hd + i;
-  const float x1 = sum_splits(part, splits, stride, c0);
-  const float x2 = sum_splits(part, splits, stride, c0 + half);
+  float4 x1 = sum_splits4(part, splits, stride, c0);
+  float4 x2 = sum_splits4(part, splits, stride, c0 + half);
+  T* dst;
   if (head < nq + nkv) {
-    const float c = cos_t[(size_t)pos * half + i], s = sin_t[(size_t)pos * half + i];
-    const float y1 = x1 * c - x2 * s, y2 = x2 * c + x1 * s;
-    T* dst = head < nq ? q + ((size_t)m * nq + head) * hd : kb + ((size_t)m * nkv + head - nq) * hd;
-    dst[i] = from_f<T>(y1);
-    dst[i + half] = from_f<T>(y2);
+    const float4 c = *reinterpret_cast<const float4*>(cos_t + (size_t)pos * half + i);
+    const float4 sn = *reinterpret_cast<const float4*>(sin_t + (size_t)pos * half + i);
+    const float4 y1 = make_float4(x1.x * c.x - x2.x * sn.x, x1.y * c.y - x2.y * sn.y,
+                                  x1.z * c.z - x2.z * sn.z, x1.w * c.w - x2.w * sn.w);
+    const float4 y2 = make_float4(x2.x * c.x + x1.x * sn.x, x2.y * c.y + x1.y * sn.y,
+                                  x2.z * c.z + x1.z * sn.z, x2.w * c.w + x1.w * sn.w);
+    x1 = y1;
+    x2 = y2;
+    dst = head < nq ? q + ((size_t)m * nq + head) * hd : kb + ((size_t)m * nkv + head - nq) * hd;
   } else {
-    T* dst = vb + ((size_t)m * nkv + head - nq - nkv) * hd;
-    dst[i] = from_f<T>(x1);
-    dst[i + half] = from_f<T>(x2);
+    dst = vb + ((size_t)m * nkv + head - nq - nkv) * hd;
   }
+  store4<T>(dst + i, x1.x, x1.y, x1.z, x1.w);
+  store4<T>(dst + i + half, x2.x, x2.y, x2.z, x2.w);
 }
 
 template <typename T>
@@ -174,30 +234,34 @@ void launch_qkv_post(const float* part, int splits, int M, int B, const int32_t*
                      const float* sin_t, T* q, T* kb, T* vb, cudaStream_t s) {
   if (M <= 0) return;
   const int pairs = (nq + 2 * nkv) * hd / 2;
-  dim3 grid((pairs + 255) / 256, M);
+  dim3 grid((pairs / 4 + 255) / 256, M);
   TimedScope ts(s, TC_ROW);
   qkv_post_kernel<T><<<grid, 256, 0, s>>>(part, splits, M, B, ctx_len, req_valid, nq, nkv, hd,
                                           cos_t, sin_t, q, kb, vb);
 }
 
 // ---------------------------------------------------------------- SwiGLU
-// part columns: [gate (I) | up (I)]; act = silu(gate) * up.
+// part columns: 128-column blocks of 64 gate outputs then the 64 up outputs
+// of the same features; act = silu(gate) * up.
 template <typename T>
 __global__ void swiglu_kernel(const float* __restrict__ part, int splits, int M, int I,
                               T* __restrict__ act) {
   const int m = blockIdx.y;
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int i = (blockIdx.x * blockDim.x + threadIdx.x) * 4;  // 4 features in one 64-block
   if (i >= I) return;
   const size_t stride = (size_t)M * 2 * I;
-  const float g = sum_splits(part, splits, stride, (size_t)m * 2 * I + i);
-  const float u = sum_splits(part, splits, stride, (size_t)m * 2 * I + I + i);
-  act[(size_t)m * I + i] = from_f<T>(g / (1.f + expf(-g)) * u);
+  const size_t gc = (size_t)m * 2 * I + (size_t)(i >> 6) * 128 + (i & 63);
+  const float4 g = sum_splits4(part, splits, stride, gc);
+  const float4 u = sum_splits4(part, splits, stride, gc + 64);
+  store4<T>(act + (size_t)m * I + i, g.x / (1.f + expf(-g.x)) * u.x,
+            g.y / (1.f + expf(-g.y)) * u.y, g.z / (1.f + expf(-g.z)) * u.z,
+            g.w / (1.f + expf(-g.w)) * u.w);
 }
 
 template <typename T>
 void launch_swiglu(const float* part, int splits, int M, int I, T* act, cudaStream_t s) {
   if (M <= 0) return;
-  dim3 grid((I + 255) / 256, M);
+  dim3 grid((I / 4 + 255) / 256, M);
   TimedScope ts(s, TC_ROW);
   swiglu_kernel<T><<<grid, 256, 0, s>>>(part, splits, M, I, act);
 }
@@ -217,7 +281,7 @@ __global__ void kv_scatter_kernel(const float* __restrict__ part, int splits, in
   const int n = row0 + nl;         // row of the whole call (cu_rows)
   const int half = hd / 2;
   const int per_layer = 2 * nkv * half;  // pairs per layer (K and V)
-  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  const int p = (blockIdx.x * blockDim.x + threadIdx.x) * 4;  // first of 4 pairs
   if (p >= L * per_layer) return;
   // request of row n: last r with cu_rows[r] <= n
   int lo = 0, hi = batch - 1;
@@ -243,17 +307,21 @@ __global__ void kv_scatter_kernel(const float* __restrict__ part, int splits, in
   const int N = L * 2 * nkv * hd;
   const size_t stride = (size_t)n_rows * N;
   const size_t c0 = (size_t)nl * N + (size_t)l * 2 * nkv * hd + (is_v ? nkv * hd : 0) + head * hd + i;
-  float x1 = sum_splits(part, splits, stride, c0);
-  float x2 = sum_splits(part, splits, stride, c0 + half);
+  float4 x1 = sum_splits4(part, splits, stride, c0);
+  float4 x2 = sum_splits4(part, splits, stride, c0 + half);
   if (!is_v) {
-    const float c = cos_t[(size_t)pos * half + i], s = sin_t[(size_t)pos * half + i];
-    const float y1 = x1 * c - x2 * s, y2 = x2 * c + x1 * s;
+    const float4 c = *reinterpret_cast<const float4*>(cos_t + (size_t)pos * half + i);
+    const float4 sn = *reinterpret_cast<const float4*>(sin_t + (size_t)pos * half + i);
+    const float4 y1 = make_float4(x1.x * c.x - x2.x * sn.x, x1.y * c.y - x2.y * sn.y,
+                                  x1.z * c.z - x2.z * sn.z, x1.w * c.w - x2.w * sn.w);
+    const float4 y2 = make_float4(x2.x * c.x + x1.x * sn.x, x2.y * c.y + x1.y * sn.y,
+                                  x2.z * c.z + x1.z * sn.z, x2.w * c.w + x1.w * sn.w);
     x1 = y1;
     x2 = y2;
   }
   T* dst = (is_v ? vc : kc) + ((((size_t)l * batch + r) * nkv + head) * cap + pos) * hd;
-  dst[i] = from_f<T>(x1);
-  dst[i + half] = from_f<T>(x2);
+  store4<T>(dst + i, x1.x, x1.y, x1.z, x1.w);
+  store4<T>(dst + i + half, x2.x, x2.y, x2.z, x2.w);
 }
 
 template <typename T>
@@ -263,7 +331,7 @@ void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int 
                        int32_t* err, cudaStream_t s) {
   if (n_rows <= 0) return;
   const int pairs = L * 2 * nkv * hd / 2;
-  dim3 grid((pairs + 255) / 256, n_rows);
+  dim3 grid((pairs / 4 + 255) / 256, n_rows);
   TimedScope ts(s, TC_ROW);
   kv_scatter_kernel<T><<<grid, 256, 0, s>>>(part, splits, n_rows, row0, L, nkv, hd, cu_rows, start_pos,
                                             batch, cap, cos_t, sin_t, max_pos, kc, vc, err);
