@@ -441,6 +441,37 @@ extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weight
            encode_weight_map(P.md, P.Wd, c.d, c.inter, H);
     }
     if (!ok) return fail(DFLASH_ECUDA);
+    // pre-tile every GEMM weight for bulk streaming, then drop the row-major copies
+    std::vector<void*> row_major;
+    auto tile_into = [&](WeightMap& wm, void* rm, int N, int K) -> bool {
+      void* t = dmalloc(m, tiled_bytes(N, K));
+      if (!t) return false;
+      tile_weights(rm, t, N, K, 0);
+      wm.tiled = t;
+      row_major.push_back(rm);
+      return true;
+    };
+    ok = tile_into(m->mfc, m->W_fc, c.d, c.n_tap * c.H_t) &&
+         tile_into(m->mkv, m->W_kv, c.n_layers * 2 * kvrows, c.d) &&
+         tile_into(m->mlm, m->W_lm, c.vocab, c.d);
+    for (int l = 0; l < c.n_layers && ok; ++l) {
+      LayerPack& P = m->layers[l];
+      ok = tile_into(P.mqkv, P.Wqkv, qkv_out(c), c.d) &&
+           tile_into(P.mo, P.Wo, c.d, c.n_q * c.head_dim) &&
+           tile_into(P.mgu, P.Wgu, 2 * c.inter, c.d) &&
+           tile_into(P.md, P.Wd, c.d, c.inter);
+    }
+    if (!ok) return fail(DFLASH_ENOMEM);
+    if (cudaDeviceSynchronize() != cudaSuccess) return fail(DFLASH_ECUDA);
+    for (void* rm : row_major) {
+      cudaFree(rm);
+      m->allocs.erase(std::find(m->allocs.begin(), m->allocs.end(), rm));
+    }
+    m->W_fc = m->W_kv = m->W_lm = nullptr;
+    for (auto& P : m->layers) P.Wqkv = P.Wo = P.Wgu = P.Wd = nullptr;
+    // the tensor maps stay valid as descriptors only; the GEMMs read `tiled`
+    m->mfc.ptr = m->mkv.ptr = m->mlm.ptr = nullptr;
+    for (auto& P : m->layers) P.mqkv.ptr = P.mo.ptr = P.mgu.ptr = P.md.ptr = nullptr;
   }
   if (cudaDeviceSynchronize() != cudaSuccess || cudaGetLastError() != cudaSuccess)
     return fail(DFLASH_ECUDA);
@@ -798,6 +829,39 @@ extern "C" int dflash_debug_gemm(const void* W, int N, int K, const void* X, int
   const void* seg[1] = {X};
   return gemm_tc(wm, seg, 1, K, K, M, splits, EPI_PARTIAL, o, err_word(err_ws),
                  (cudaStream_t)stream);
+}
+
+extern "C" int dflash_debug_gemm_tiled(const void* Wt, int N, int K, const void* X, int M,
+                                       int elem, int splits, float* out, int* splits_used,
+                                       void* err_ws, void* stream) {
+  if (!Wt || !X || !out || !err_ws || N < 1 || K < 64 || K % 64 || M < 1) return DFLASH_EINVAL;
+  if (!aligned16(Wt) || !aligned16(X)) return DFLASH_EINVAL;
+  if (elem != DFLASH_BF16 && elem != DFLASH_F16) return DFLASH_EINVAL;
+  WeightMap wm;
+  memset(&wm.map, 0, sizeof(wm.map));
+  wm.N = N;
+  wm.K = K;
+  wm.elem = elem;
+  wm.tiled = Wt;
+  splits = gemm_effective_splits(K, splits);
+  if (splits_used) *splits_used = splits;
+  GemmOut o;
+  o.part = out;
+  const void* seg[1] = {X};
+  return gemm_tc(wm, seg, 1, K, K, M, splits, EPI_PARTIAL, o, err_word(err_ws),
+                 (cudaStream_t)stream);
+}
+
+extern "C" size_t dflash_debug_tiled_bytes(int N, int K) {
+  if (N < 1 || K < 64 || K % 64) return 0;
+  return tiled_bytes(N, K);
+}
+
+extern "C" int dflash_debug_tile_weights(const void* W, void* Wt, int N, int K, void* stream) {
+  if (!W || !Wt || N < 1 || K < 64 || K % 64 || !aligned16(W) || !aligned16(Wt))
+    return DFLASH_EINVAL;
+  tile_weights(W, Wt, N, K, (cudaStream_t)stream);
+  return cuda_status();
 }
 
 extern "C" int dflash_debug_lmhead(const void* W, int N, int K, const void* X, int M, int elem,

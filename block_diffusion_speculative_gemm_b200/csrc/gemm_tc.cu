@@ -55,6 +55,7 @@ struct GemmArgs {
   int splits;
   int n_vtiles;       // LM head: number of 128-row vocabulary tiles (= tiles_n)
   uint32_t idesc;     // tcgen05 instruction descriptor (operand type, 128 x BN)
+  const uint8_t* a_tiled;  // pre-tiled weights (bulk copies) or null (tensor map)
   GemmOut out;
   int32_t* err;
 };
@@ -179,6 +180,16 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
   return w;
 }
 
+// Contiguous global -> shared bulk copy completing on an mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void st_keep(float* p, float v, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
 }
@@ -271,7 +282,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           int ki = i + rot;
           if (ki >= w.nk) ki -= w.nk;
           const int kx = (w.kb0 + ki) * kTileK;
-          tma_load_2d(sA(s), &tmA, full(s), kx, w.n0, pol_w);
+          if (a.a_tiled != nullptr)
+            bulk_load(sA(s), a.a_tiled + ((size_t)(w.n0 / kTileN) * a.n_kb + kx / kTileK) * 16384,
+                      16384, full(s), pol_w);
+          else
+            tma_load_2d(sA(s), &tmA, full(s), kx, w.n0, pol_w);
           const int seg = kx / a.seg_k;
           tma_load_2d(sB(s), &tmB.m[seg], full(s), kx - seg * a.seg_k, w.m0, pol_x);
         }
@@ -539,6 +554,38 @@ int gemm_pick_splits(int M, int N, int K, int max_splits) {
   return best;
 }
 
+// ---------------------------------------------------------------- weight tiling
+
+__global__ void tile_weights_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int N,
+                                    int K) {
+  // one 16-byte chunk (8 elements) per thread: tile (t, kb), row r, chunk j
+  const int nkb = K / kTileK;
+  const size_t total = (size_t)((N + kTileN - 1) / kTileN) * nkb * kTileN * 8;
+  for (size_t c = (size_t)blockIdx.x * blockDim.x + threadIdx.x; c < total;
+       c += (size_t)gridDim.x * blockDim.x) {
+    const int j = (int)(c & 7);
+    const int r = (int)((c >> 3) & (kTileN - 1));
+    const size_t tk = c >> 10;  // tile index t * nkb + kb
+    const int kb = (int)(tk % nkb);
+    const int t = (int)(tk / nkb);
+    const int n = t * kTileN + r;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (n < N) v = src[((size_t)n * K + (size_t)kb * kTileK) / 8 + j];
+    dst[tk * 1024 + (size_t)r * 8 + (j ^ (r & 7))] = v;
+  }
+}
+
+size_t tiled_bytes(int N, int K) {
+  return (size_t)((N + kTileN - 1) / kTileN) * (K / kTileK) * 16384;
+}
+
+void tile_weights(const void* src, void* dst, int N, int K, cudaStream_t s) {
+  const size_t chunks = tiled_bytes(N, K) / 16;
+  const unsigned blocks = (unsigned)std::min<size_t>((chunks + 255) / 256, 148 * 32);
+  tile_weights_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(src),
+                                             static_cast<uint4*>(dst), N, K);
+}
+
 static int token_tile(int M) {
   if (M >= kMaxBN) return kMaxBN;
   return (M + 31) / 32 * 32;
@@ -573,6 +620,7 @@ int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, i
   if (epi == EPI_PARTIAL && out.op != OP_PARTIAL && splits > 1) return DFLASH_EINVAL;
   a.n_vtiles = a.tiles_n;
   a.idesc = idesc_f16kind(kTileN, BN, W.elem == DFLASH_BF16);
+  a.a_tiled = static_cast<const uint8_t*>(W.tiled);
   a.out = out;
   a.err = err;
 

@@ -82,14 +82,25 @@ struct GemmOut {
 // A weight operand prepared once: tensor map over [N, K] rows of 16-bit
 // elements (elem = DFLASH_BF16 or DFLASH_F16).  The activation operand of a
 // GEMM against it must have the same element type.
+//
+// `tiled`, when set, holds the same weights pre-tiled for streaming: tile
+// (n-tile t, k-block kb) is 16 KB at ((t * K/64) + kb) * 16384, already in the
+// 128-byte-swizzled shared-memory image of a [128 x 64] K-major tile, so the
+// GEMM fetches it with one bulk copy instead of a 128-row tensor box.
 struct WeightMap {
   CUtensorMap map;
   const void* ptr = nullptr;
+  const void* tiled = nullptr;
   int N = 0, K = 0;
   int elem = DFLASH_BF16;
 };
 
 bool encode_weight_map(WeightMap& w, const void* ptr, int N, int K, int elem);
+
+// Writes the pre-tiled streaming image of a row-major 16-bit W [N, K] (K % 64
+// == 0) into dst (ceil(N/128) * K/64 * 16384 bytes; rows past N are zero).
+void tile_weights(const void* src, void* dst, int N, int K, cudaStream_t s);
+size_t tiled_bytes(int N, int K);
 
 // 2D tensor map over `rows` rows of `cols` 16-bit elements (row stride `ld`
 // elements) with a box of 64 columns x box_rows rows, 128-byte swizzle, zero

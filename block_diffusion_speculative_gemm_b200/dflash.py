@@ -85,6 +85,11 @@ def lib() -> ctypes.CDLL:
         L.dflash_debug_gemm.argtypes = [vp, i32, i32, vp, i32, i32, i32, vp,
                                         ctypes.POINTER(ctypes.c_int), vp, vp]
         L.dflash_debug_lmhead.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp, vp, vp]
+        L.dflash_debug_gemm_tiled.argtypes = [vp, i32, i32, vp, i32, i32, i32, vp,
+                                              ctypes.POINTER(ctypes.c_int), vp, vp]
+        L.dflash_debug_tiled_bytes.argtypes = [i32, i32]
+        L.dflash_debug_tiled_bytes.restype = sz
+        L.dflash_debug_tile_weights.argtypes = [vp, vp, i32, i32, vp]
         _lib = L
     return _lib
 
@@ -331,9 +336,10 @@ def timing_read() -> Dict[str, Dict[str, float]]:
 _ELEM = {torch.bfloat16: BF16, torch.float16: F16}
 
 
-def debug_gemm(W: torch.Tensor, X: torch.Tensor, splits: int, err_ws: torch.Tensor, stream=None):
+def debug_gemm(W: torch.Tensor, X: torch.Tensor, splits: int, err_ws: torch.Tensor, stream=None,
+               tiled: bool = False):
     """fp32 split-K partials [splits_used, M, N] of X @ W^T from the tcgen05 core
-    (W and X both bf16 or both fp16)."""
+    (W and X both bf16 or both fp16); ``tiled`` streams W from its pre-tiled image."""
     _need(W, "W")
     _need(X, "X", W.dtype)
     elem = _ELEM[W.dtype]
@@ -345,9 +351,17 @@ def debug_gemm(W: torch.Tensor, X: torch.Tensor, splits: int, err_ws: torch.Tens
     s_used = -(-nkb // per)
     out = torch.empty((s_used, M, N), dtype=torch.float32, device=W.device)
     used = ctypes.c_int(0)
-    _check("dflash_debug_gemm", lib().dflash_debug_gemm(
-        _ptr(W), N, K, _ptr(X), M, elem, s_req, _ptr(out), ctypes.byref(used), _ptr(err_ws),
-        _stream(stream)))
+    if tiled:
+        Wt = torch.empty(lib().dflash_debug_tiled_bytes(N, K), dtype=torch.uint8, device=W.device)
+        _check("dflash_debug_tile_weights", lib().dflash_debug_tile_weights(
+            _ptr(W), _ptr(Wt), N, K, _stream(stream)))
+        _check("dflash_debug_gemm_tiled", lib().dflash_debug_gemm_tiled(
+            _ptr(Wt), N, K, _ptr(X), M, elem, s_req, _ptr(out), ctypes.byref(used),
+            _ptr(err_ws), _stream(stream)))
+    else:
+        _check("dflash_debug_gemm", lib().dflash_debug_gemm(
+            _ptr(W), N, K, _ptr(X), M, elem, s_req, _ptr(out), ctypes.byref(used),
+            _ptr(err_ws), _stream(stream)))
     assert used.value == s_used
     return out
 

@@ -25,6 +25,17 @@ extern "C" {
 int dflash_debug_gemm(const void* W, int N, int K, const void* X, int M, int elem, int splits,
                       float* out, int* splits_used, void* err_ws, void* stream);
 
+/* Same product with the weights read from their pre-tiled streaming image
+ * (written by dflash_debug_tile_weights) instead of a tensor map over W. */
+int dflash_debug_gemm_tiled(const void* W_tiled, int N, int K, const void* X, int M, int elem,
+                            int splits, float* out, int* splits_used, void* err_ws, void* stream);
+
+/* Bytes of the pre-tiled streaming image of a [N, K] 16-bit weight, and the
+ * call that writes it (128-row x 64-column tiles, each the 128-byte-swizzled
+ * shared-memory image of the tile, rows past N zero). */
+size_t dflash_debug_tiled_bytes(int N, int K);
+int dflash_debug_tile_weights(const void* W, void* W_tiled, int N, int K, void* stream);
+
 /* LM-head epilogue: for every token row m and 128-row weight tile t,
  * stats[m][t] = {max_n logit, argmax n (lowest), sum exp(logit - max), 0}
  * (16 bytes per entry); logits (device fp32 [M, N]) receives the raw products

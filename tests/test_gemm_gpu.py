@@ -25,10 +25,11 @@ def _inputs(N, K, M, seed, dtype=torch.bfloat16):
     (6144, 4096, 256, 3),    # QKV projection of the 8B-shaped draft
 ])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
-def test_gemm_matches_float64(N, K, M, splits, dtype):
+@pytest.mark.parametrize("tiled", [False, True])
+def test_gemm_matches_float64(N, K, M, splits, dtype, tiled):
     W, X = _inputs(N, K, M, N * 7 + K + M, dtype)
     err = D.new_workspace(256)
-    out = D.debug_gemm(W.cuda(), X.cuda(), splits, err)
+    out = D.debug_gemm(W.cuda(), X.cuda(), splits, err, tiled=tiled)
     torch.cuda.synchronize()
     assert D.get_error(err) == 0
     got = out.double().sum(0).cpu()
