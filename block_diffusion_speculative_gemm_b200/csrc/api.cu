@@ -447,7 +447,7 @@ extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weight
       void* t = dmalloc(m, tiled_bytes(N, K));
       if (!t) return false;
       tile_weights(rm, t, N, K, 0);
-      wm.tiled = t;
+      if (!set_tiled_weights(wm, t)) return false;
       row_major.push_back(rm);
       return true;
     };
@@ -842,7 +842,7 @@ extern "C" int dflash_debug_gemm_tiled(const void* Wt, int N, int K, const void*
   wm.N = N;
   wm.K = K;
   wm.elem = elem;
-  wm.tiled = Wt;
+  if (!set_tiled_weights(wm, Wt)) return DFLASH_ECUDA;
   splits = gemm_effective_splits(K, splits);
   if (splits_used) *splits_used = splits;
   GemmOut o;
@@ -862,6 +862,33 @@ extern "C" int dflash_debug_tile_weights(const void* W, void* Wt, int N, int K, 
     return DFLASH_EINVAL;
   tile_weights(W, Wt, N, K, (cudaStream_t)stream);
   return cuda_status();
+}
+
+extern "C" int dflash_debug_gemm_mode(int mode) {
+  if (mode < 0 || mode > 2) return DFLASH_EINVAL;
+  gemm_set_mode(mode);
+  return DFLASH_OK;
+}
+
+extern "C" int dflash_debug_lmhead_tiled(const void* Wt, int N, int K, const void* X, int M,
+                                         int elem, void* stats, float* logits, void* err_ws,
+                                         void* stream) {
+  if (!Wt || !X || !stats || !err_ws || N < 1 || K < 64 || K % 64 || M < 1) return DFLASH_EINVAL;
+  if (!aligned16(Wt) || !aligned16(X)) return DFLASH_EINVAL;
+  if (elem != DFLASH_BF16 && elem != DFLASH_F16) return DFLASH_EINVAL;
+  WeightMap wm;
+  memset(&wm.map, 0, sizeof(wm.map));
+  wm.N = N;
+  wm.K = K;
+  wm.elem = elem;
+  if (!set_tiled_weights(wm, Wt)) return DFLASH_ECUDA;
+  GemmOut o;
+  o.stats = static_cast<LmStat*>(stats);
+  o.dbg = logits;
+  o.dbg_rows = nullptr;
+  o.dbg_ld = N;
+  const void* seg[1] = {X};
+  return gemm_tc(wm, seg, 1, K, K, M, 1, EPI_LMHEAD, o, err_word(err_ws), (cudaStream_t)stream);
 }
 
 extern "C" int dflash_debug_lmhead(const void* W, int N, int K, const void* X, int M, int elem,

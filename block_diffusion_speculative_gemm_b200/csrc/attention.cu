@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(kAttnThreads)
                         const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ req_valid,
                         int B, int nq, int nkv, int chunk, int n_chunks,
                         float* __restrict__ part_o, float* __restrict__ part_ml) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int EPL = HD / 32;  // output elements per lane
   extern __shared__ float sm[];
   const int c = blockIdx.x, g = blockIdx.y, r = blockIdx.z;
@@ -138,6 +140,8 @@ __global__ void __launch_bounds__(kCombineThreads)
                         const int32_t* __restrict__ ctx_len,
                         const int32_t* __restrict__ req_valid, int B, int nq, int nkv, int chunk,
                         int n_chunks, T* __restrict__ o) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float wgt[kMaxChunksC * kMaxRows];
   const int g = blockIdx.x, r = blockIdx.y;
   const int G = nq / nkv, R = B * G;
@@ -197,14 +201,14 @@ int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, c
       const size_t sm = (kMaxRows * 128 + kKeyTile * 129 + kKeyTile * 128) * sizeof(float);
       cudaFuncSetAttribute(attn_partial_kernel<T, TC, 128>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-      attn_partial_kernel<T, TC, 128><<<grid, kAttnThreads, sm, s>>>(
-          q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks,
-          part_o, part_ml);
+      launch_pdl(attn_partial_kernel<T, TC, 128>, dim3(grid), dim3(kAttnThreads), sm, s, 1, q, kb,
+          vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, part_o,
+          part_ml);
     } else if (hd == 64) {
       const size_t sm = (kMaxRows * 64 + kKeyTile * 65 + kKeyTile * 64) * sizeof(float);
-      attn_partial_kernel<T, TC, 64><<<grid, kAttnThreads, sm, s>>>(
-          q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks,
-          part_o, part_ml);
+      launch_pdl(attn_partial_kernel<T, TC, 64>, dim3(grid), dim3(kAttnThreads), sm, s, 1, q, kb,
+          vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, part_o,
+          part_ml);
     } else {
       return DFLASH_EUNSUPPORTED;
     }
@@ -214,13 +218,11 @@ int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, c
     if (n_chunks > kMaxChunksC) return DFLASH_EUNSUPPORTED;
     dim3 g2(nkv, batch);
     if (hd == 128)
-      attn_combine_kernel<T, 128><<<g2, kCombineThreads, 0, s>>>(part_o, part_ml, ctx_len,
-                                                                 req_valid, B, nq, nkv, chunk,
-                                                                 n_chunks, o);
+      launch_pdl(attn_combine_kernel<T, 128>, dim3(g2), dim3(kCombineThreads), 0, s, 1, part_o,
+          part_ml, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, o);
     else
-      attn_combine_kernel<T, 64><<<g2, kCombineThreads, 0, s>>>(part_o, part_ml, ctx_len,
-                                                                req_valid, B, nq, nkv, chunk,
-                                                                n_chunks, o);
+      launch_pdl(attn_combine_kernel<T, 64>, dim3(g2), dim3(kCombineThreads), 0, s, 1, part_o,
+          part_ml, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, o);
   }
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }

@@ -181,6 +181,8 @@ __global__ void __launch_bounds__(kThreads)
                    const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ req_valid,
                    int B, int nq, int nkv, int chunk, int n_chunks, float* __restrict__ part_o,
                    float* __restrict__ part_ml, int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   using LY = Layout<HD, MT>;
   using WP = Warp<HD, MT>;
   constexpr int kStages = LY::kStages;
@@ -385,9 +387,8 @@ int launch_cfg(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q, co
                            smem) != cudaSuccess)
     return DFLASH_ECUDA;
   dim3 grid(n_chunks, nkv, batch);
-  attn_tc_kernel<HD, MT><<<grid, kThreads, smem, s>>>(tk, tv, q, kb, vb, layer, batch, cap,
-                                                      ctx_len, req_valid, B, nq, nkv, chunk,
-                                                      n_chunks, part_o, part_ml, err);
+  launch_pdl(attn_tc_kernel<HD, MT>, dim3(grid), dim3(kThreads), smem, s, 1, tk, tv, q, kb, vb,
+      layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, part_o, part_ml, err);
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 

@@ -22,6 +22,8 @@ __global__ void draft_init_kernel(const int32_t* __restrict__ anchor,
                                   int mask_id, int cap, int32_t* tokens, int32_t* zrow,
                                   int32_t* lm_rows, int32_t* cstep, int32_t* req_valid,
                                   int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x * blockDim.y + threadIdx.y;
   const int j = threadIdx.x;
   if (r >= batch || j >= B) return;
@@ -51,9 +53,8 @@ void launch_draft_init(const int32_t* anchor, const int32_t* ctx_len, int batch,
                        int32_t* cstep, int32_t* req_valid, int32_t* err, cudaStream_t s) {
   dim3 block(32, 8);
   TimedScope ts(s, TC_ROW);
-  draft_init_kernel<<<(batch + 7) / 8, block, 0, s>>>(anchor, ctx_len, batch, B, V, mask_id, cap,
-                                                      tokens, zrow, lm_rows, cstep, req_valid,
-                                                      err);
+  launch_pdl(draft_init_kernel, dim3((batch + 7) / 8), dim3(block), 0, s, 1, anchor, ctx_len, batch,
+      B, V, mask_id, cap, tokens, zrow, lm_rows, cstep, req_valid, err);
 }
 
 // Merge of two tile statistics: the larger maximum wins (lower id on equal
@@ -71,6 +72,8 @@ __device__ __forceinline__ void stat_merge(float& mx, int& id, float& se, float 
 
 __global__ void lm_reduce_kernel(const LmStat* __restrict__ stats, int n_vtiles,
                                  int32_t* __restrict__ tok, float* __restrict__ conf) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float s_m[32], s_s[32];
   __shared__ int s_i[32];
   const int q = blockIdx.x;
@@ -111,13 +114,15 @@ void launch_lm_reduce(const LmStat* stats, int n_vtiles, int rows, int32_t* tok,
                       cudaStream_t s) {
   if (rows <= 0) return;
   TimedScope ts(s, TC_ROW);
-  lm_reduce_kernel<<<rows, 256, 0, s>>>(stats, n_vtiles, tok, conf);
+  launch_pdl(lm_reduce_kernel, dim3(rows), dim3(256), 0, s, 1, stats, n_vtiles, tok, conf);
 }
 
 // fp32 model type: tile statistics from a full logits matrix [rows, V].
 __global__ void lm_stats_from_logits_kernel(const float* __restrict__ logits, int V,
                                             LmStat* __restrict__ stats, float* dbg,
                                             const int32_t* dbg_rows, int64_t dbg_ld) {
+  pdl_trigger();
+  pdl_wait();
   const int q = blockIdx.y, t = blockIdx.x;
   const int n_vtiles = gridDim.x;
   const int v = t * kTileN + threadIdx.x;
@@ -148,7 +153,8 @@ void launch_lm_stats_from_logits(const float* logits, int rows, int V, LmStat* s
   if (rows <= 0) return;
   dim3 grid((V + kTileN - 1) / kTileN, rows);
   TimedScope ts(s, TC_LMHEAD);
-  lm_stats_from_logits_kernel<<<grid, kTileN, 0, s>>>(logits, V, stats, dbg, dbg_rows, dbg_ld);
+  launch_pdl(lm_stats_from_logits_kernel, dim3(grid), dim3(kTileN), 0, s, 1, logits, V, stats, dbg,
+      dbg_rows, dbg_ld);
 }
 
 // One warp per request, lane j = block position j.  The k most confident
@@ -158,6 +164,8 @@ void launch_lm_stats_from_logits(const float* logits, int rows, int V, LmStat* s
 __global__ void commit_kernel(const int32_t* __restrict__ tok, const float* __restrict__ conf,
                               int batch, int B, int rem, int k, int step, int32_t* tokens,
                               int32_t* zrow, int32_t* lm_rows, int32_t* cstep) {
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= batch) return;
@@ -198,14 +206,16 @@ void launch_commit(const int32_t* tok, const float* conf, int batch, int B, int 
                    cudaStream_t s) {
   TimedScope ts(s, TC_ROW);
   const int wpb = 4;
-  commit_kernel<<<(batch + wpb - 1) / wpb, 32 * wpb, 0, s>>>(tok, conf, batch, B, rem, k, step,
-                                                             tokens, zrow, lm_rows, cstep);
+  launch_pdl(commit_kernel, dim3((batch + wpb - 1) / wpb), dim3(32 * wpb), 0, s, 1, tok, conf,
+      batch, B, rem, k, step, tokens, zrow, lm_rows, cstep);
 }
 
 __global__ void draft_finish_kernel(const int32_t* __restrict__ tokens,
                                     const int32_t* __restrict__ cstep,
                                     const int32_t* __restrict__ req_valid, int batch, int B,
                                     int32_t* draft_out, int32_t* cstep_out) {
+  pdl_trigger();
+  pdl_wait();
   const int m = blockIdx.x * blockDim.x + threadIdx.x;
   if (m >= batch * B) return;
   if (!req_valid[m / B]) return;
@@ -218,8 +228,8 @@ void launch_draft_finish(const int32_t* tokens, const int32_t* cstep, const int3
                          cudaStream_t s) {
   TimedScope ts(s, TC_ROW);
   const int n = batch * B;
-  draft_finish_kernel<<<(n + 255) / 256, 256, 0, s>>>(tokens, cstep, req_valid, batch, B,
-                                                      draft_out, cstep_out);
+  launch_pdl(draft_finish_kernel, dim3((n + 255) / 256), dim3(256), 0, s, 1, tokens, cstep,
+      req_valid, batch, B, draft_out, cstep_out);
 }
 
 }  // namespace dflash

@@ -12,6 +12,8 @@ struct SegPtrs {
 
 __global__ void gemm_simt_f32_kernel(const float* __restrict__ W, int N, int K, SegPtrs xs,
                                      int seg_k, int M, float* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float xrow[];  // one token row of X (K floats)
   const int m = blockIdx.y;
   for (int k = threadIdx.x; k < K; k += blockDim.x) {
@@ -34,7 +36,8 @@ void gemm_simt_f32(const float* W, int N, int K, const float* const* xseg, int n
   for (int i = 0; i < kMaxSeg; ++i) xs.p[i] = i < n_seg ? xseg[i] : nullptr;
   dim3 grid((N + 127) / 128, M);
   TimedScope ts(s, TC_GEMM);
-  gemm_simt_f32_kernel<<<grid, 128, (size_t)K * sizeof(float), s>>>(W, N, K, xs, seg_k, M, out);
+  launch_pdl(gemm_simt_f32_kernel, dim3(grid), dim3(128), (size_t)K * sizeof(float), s, 1, W, N, K,
+      xs, seg_k, M, out);
 }
 
 }  // namespace dflash

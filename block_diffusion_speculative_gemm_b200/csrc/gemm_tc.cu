@@ -53,14 +53,17 @@ struct GemmArgs {
   int tiles_m;        // token tiles
   int units;          // tiles_n * tiles_m * splits
   int splits;
-  int n_vtiles;       // LM head: number of 128-row vocabulary tiles (= tiles_n)
-  uint32_t idesc;     // tcgen05 instruction descriptor (operand type, 128 x BN)
+  int tile_rows;      // weight rows per unit: 128, or 256 for a CTA pair
+  int n_vtiles;       // LM head: number of 128-row vocabulary tiles
+  int epi_bytes;      // shared bytes of the epilogue region
+  uint32_t idesc;     // tcgen05 instruction descriptor (operand type, tile_rows x BN)
   const uint8_t* a_tiled;  // pre-tiled weights (bulk copies) or null (tensor map)
   GemmOut out;
   int32_t* err;
 };
 
 constexpr int kGemmThreads = 192;
+constexpr int kMaxStages = 8;   // smem ring depth cap
 constexpr int kEpiWarp0 = 2;  // first epilogue warp
 constexpr int kLmTr = 32 * 33;  // floats of one warp's transpose buffer
 constexpr int kStLd = kTileN + 1; // row stride of the fused-op staging tile [32 tokens][128 rows]
@@ -167,14 +170,16 @@ struct Unit {
   int n0, m0, split, kb0, nk, tile;
 };
 
-__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
+// Unit u of the CTA with pair rank `rank` (0 outside pairs): its 128 weight
+// rows start at n0.
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int rank) {
   Unit w;
   const int per = a.tiles_n * a.tiles_m;
   w.split = u / per;
   const int rem = u % per;
   w.tile = rem;
   w.m0 = (rem / a.tiles_n) * a.BN;
-  w.n0 = (rem % a.tiles_n) * kTileN;
+  w.n0 = (rem % a.tiles_n) * a.tile_rows + rank * kTileN;
   w.kb0 = w.split * a.kb_per_split;
   w.nk = min(a.n_kb, w.kb0 + a.kb_per_split) - w.kb0;
   return w;
@@ -211,14 +216,22 @@ __device__ __forceinline__ bool epi_bar_and(bool v) {
   return r != 0;
 }
 
-template <int EPI>
+// PAIR: launched as clusters of two CTAs sharing each 256-row weight tile
+// (see the CTA-pair notes in common.cuh).  Both CTAs stream their own weight
+// rows and half of the token tile; their loads complete on rank 0's `full`
+// barriers, rank 0 issues the M = 256 MMAs and its commits release the stages
+// and accumulators of both CTAs; both CTAs' epilogue warps hand the
+// accumulator back to rank 0.  tmA is then the pre-tiled weight map.
+template <int EPI, bool PAIR>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps tmB,
                    const GemmArgs a) {
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const int stage_bytes = kTileN * 128 + a.BN * 128;
+  const int bn_cta = PAIR ? a.BN / 2 : a.BN;  // token rows this CTA stages per k-block
+  const int stage_bytes = kTileN * 128 + bn_cta * 128;
   // [stages][A | B] | epilogue region (LM-head transposes + partials, or the
   // fused-op staging tile + token maps + flag) | barriers
   uint8_t* epi_smem = smem + a.stages * stage_bytes;
@@ -227,8 +240,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   float* st = reinterpret_cast<float*>(epi_smem);
   int* tok_req = reinterpret_cast<int*>(st + 32 * kStLd);
   int* tok_pos = tok_req + 32;
-  uint64_t* bars =
-      reinterpret_cast<uint64_t*>(epi_smem + (EPI == EPI_LMHEAD ? kLmSmem : kFusedSmem));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_smem + a.epi_bytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * a.stages + 4);
   const uint32_t smem0 = smem_u32(smem);
   auto sA = [&](int s) { return smem0 + s * stage_bytes; };
@@ -240,6 +252,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ncols = tmem_cols_for(a.BN);
+  // pair rank, and the index / count of the CTAs (or pairs) walking the units
+  const int rank = PAIR ? (int)cluster_rank() : 0;
+  const int cid = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int ncl = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
@@ -248,17 +264,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(acc_full(b), 1);
-      mbar_init(acc_empty(b), 4);  // one elected lane per epilogue warp
+      // one elected lane per epilogue warp (of both CTAs for a pair)
+      mbar_init(acc_empty(b), PAIR ? 8 : 4);
     }
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) tma_prefetch_desc(&tmA);
   if (warp == kEpiWarp0) {
-    tmem_alloc(smem_u32(tmem_slot), 2 * ncols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_slot), 2 * ncols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), 2 * ncols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR)
+    cluster_sync_all();  // the peer's barriers are initialised before any remote use
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -268,38 +293,78 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
+      // k-block i of unit w: the rotated index (each CTA or pair starts its K
+      // walk at its own offset so that the SMs do not all request the same
+      // activation rows of L2 at the same moment)
+      auto kx_of = [&](const Unit& w, int i) {
+        int ki = i + (int)((cid * 7u) % (unsigned)w.nk);
+        if (ki >= w.nk) ki -= w.nk;
+        return (w.kb0 + ki) * kTileK;
+      };
+      auto expect = [&](int s) {
+        if (!PAIR)
+          mbar_arrive_expect_tx(full(s), stage_bytes);
+        else if (rank == 0)  // rank 0 expects both CTAs' bytes; the peer's may land first
+          mbar_arrive_expect_tx(full(s), 2 * stage_bytes);
+      };
+      auto load_w = [&](int s, const Unit& w, int kx) {
+        if (PAIR)  // weight tile n0/128, k-block kx/64 of the tiled image; rows past
+                   // the last tile read as zeros
+          tma_load_2d_pair(sA(s), &tmA, mapa_shared(full(s), 0), 0,
+                           ((w.n0 / kTileN) * a.n_kb + kx / kTileK) * kTileN, pol_w);
+        else if (a.a_tiled != nullptr)
+          bulk_load(sA(s), a.a_tiled + ((size_t)(w.n0 / kTileN) * a.n_kb + kx / kTileK) * 16384,
+                    16384, full(s), pol_w);
+        else
+          tma_load_2d(sA(s), &tmA, full(s), kx, w.n0, pol_w);
+      };
+      auto load_x = [&](int s, const Unit& w, int kx) {
+        const int seg = kx / a.seg_k;
+        if (PAIR)
+          tma_load_2d_pair(sB(s), &tmB.m[seg], mapa_shared(full(s), 0), kx - seg * a.seg_k,
+                           w.m0 + rank * bn_cta, pol_x);
+        else
+          tma_load_2d(sB(s), &tmB.m[seg], full(s), kx - seg * a.seg_k, w.m0, pol_x);
+      };
+      // The weights are never written by another kernel: the first stages of
+      // the first unit are requested before the predecessor kernel has
+      // finished (their empty barriers are fresh), the activations after it.
+      int pre = 0;
+      if (cid < a.units) {
+        const Unit w = decode_unit(a, cid, rank);
+        pre = min(a.stages, w.nk);
+        for (int i = 0; i < pre; ++i) {
+          expect(i);
+          load_w(i, w, kx_of(w, i));
+        }
+      }
+      pdl_wait();
       uint32_t it = 0;
-      for (int u = blockIdx.x; u < a.units && ok; u += gridDim.x) {
-        const Unit w = decode_unit(a, u);
-        // each CTA starts its K walk at its own offset so that the SMs do not
-        // all request the same activation rows of L2 at the same moment
-        const int rot = (int)((blockIdx.x * 7u) % (unsigned)w.nk);
+      for (int u = cid; u < a.units && ok; u += ncl) {
+        const Unit w = decode_unit(a, u, rank);
         for (int i = 0; i < w.nk; ++i, ++it) {
           const int s = it % a.stages;
           const uint32_t ph = (it / a.stages) & 1;
+          const int kx = kx_of(w, i);
+          if ((int)it < pre) {  // weights already requested
+            load_x(s, w, kx);
+            continue;
+          }
           if (!mbar_wait(empty(s), ph ^ 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(full(s), stage_bytes);
-          int ki = i + rot;
-          if (ki >= w.nk) ki -= w.nk;
-          const int kx = (w.kb0 + ki) * kTileK;
-          if (a.a_tiled != nullptr)
-            bulk_load(sA(s), a.a_tiled + ((size_t)(w.n0 / kTileN) * a.n_kb + kx / kTileK) * 16384,
-                      16384, full(s), pol_w);
-          else
-            tma_load_2d(sA(s), &tmA, full(s), kx, w.n0, pol_w);
-          const int seg = kx / a.seg_k;
-          tma_load_2d(sB(s), &tmB.m[seg], full(s), kx - seg * a.seg_k, w.m0, pol_x);
+          expect(s);
+          load_w(s, w, kx);
+          load_x(s, w, kx);
         }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       uint32_t it = 0;
       int j = 0;
-      for (int u = blockIdx.x; u < a.units && ok; u += gridDim.x, ++j) {
-        const Unit w = decode_unit(a, u);
+      for (int u = cid; u < a.units && ok; u += ncl, ++j) {
+        const Unit w = decode_unit(a, u, 0);
         const int b = j & 1;
         if (!mbar_wait(acc_empty(b), ((j >> 1) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
@@ -309,13 +374,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t ph = (it / a.stages) & 1;
           if (!mbar_wait(full(s), ph)) { ok = false; break; }
           tc_fence_after();
+          if (PAIR) {
 #pragma unroll
-          for (int kk = 0; kk < kTileK / 16; ++kk)
-            umma_f16(d, smem_desc_sw128(sA(s) + kk * 32), smem_desc_sw128(sB(s) + kk * 32),
-                     a.idesc, (i | kk) != 0 ? 1u : 0u);
-          umma_commit(empty(s));
+            for (int kk = 0; kk < kTileK / 16; ++kk)
+              umma_f16_pair(d, smem_desc_sw128(sA(s) + kk * 32), smem_desc_sw128(sB(s) + kk * 32),
+                            a.idesc, (i | kk) != 0 ? 1u : 0u);
+            umma_commit_pair(empty(s));
+            umma_commit_pair(mapa_shared(empty(s), 1));
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kTileK / 16; ++kk)
+              umma_f16(d, smem_desc_sw128(sA(s) + kk * 32), smem_desc_sw128(sB(s) + kk * 32),
+                       a.idesc, (i | kk) != 0 ? 1u : 0u);
+            umma_commit(empty(s));
+          }
         }
-        umma_commit(acc_full(b));
+        if (PAIR) {
+          umma_commit_pair(acc_full(b));
+          umma_commit_pair(mapa_shared(acc_full(b), 1));
+        } else {
+          umma_commit(acc_full(b));
+        }
       }
     }
     __syncwarp();
@@ -324,10 +403,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;              // TMEM lane group of this warp
     const int row = q * 32 + lane;       // weight row inside the tile
     const int nchunk = a.BN / 32;
+    pdl_wait();  // the epilogue reads and writes other kernels' buffers
     int j = 0;
-    for (int u = blockIdx.x; u < a.units; u += gridDim.x, ++j) {
-      const Unit w = decode_unit(a, u);
+    for (int u = cid; u < a.units; u += ncl, ++j) {
+      const Unit w = decode_unit(a, u, rank);
       const int b = j & 1;
+      // the second half of a pair's last tile can lie past the weights
+      const bool live = w.n0 < a.N;
       bool got = mbar_wait(acc_full(b), (j >> 1) & 1);
       got = epi_bar_and(got);  // the epilogue warps leave together
       __syncwarp();
@@ -339,9 +421,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       auto release = [&]() {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0)
-          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty(b)) : "memory");
+        if (lane == 0) {
+          if (PAIR)
+            mbar_arrive_cluster(mapa_shared(acc_empty(b), 0));
+          else
+            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty(b)) : "memory");
+        }
       };
+      if (!live) {
+        release();
+        continue;
+      }
       // token -> (request, cache position) for OP_KV, one thread per token of the chunk
       auto token_maps = [&](int m_base) {
         if (a.out.op != OP_KV || et >= 32) return;
@@ -460,8 +550,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   if (!ok) set_error(a.err, DFLASH_DEV_TIMEOUT);
   tc_fence_before();
-  __syncthreads();
-  if (warp == kEpiWarp0) tmem_dealloc(tmem, 2 * ncols);
+  if (PAIR) {
+    // neither CTA leaves while the other may still touch its barriers, shared
+    // memory or TMEM
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == kEpiWarp0) tmem_dealloc_pair(tmem, 2 * ncols);
+  } else {
+    __syncthreads();
+    if (warp == kEpiWarp0) tmem_dealloc(tmem, 2 * ncols);
+  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -499,6 +597,27 @@ bool encode_2d(CUtensorMap* m, const void* ptr, int64_t rows, int cols, int ld, 
   return r == CUDA_SUCCESS;
 }
 
+bool set_tiled_weights(WeightMap& w, const void* tiled) {
+  auto enc = get_encode();
+  if (!enc || !tiled || (reinterpret_cast<uintptr_t>(tiled) & 15) != 0) return false;
+  if (w.elem != DFLASH_BF16 && w.elem != DFLASH_F16) return false;
+  // the tiled image viewed as rows of 64 elements (128 bytes): tile t, k-block
+  // kb is rows [(t * K/64 + kb) * 128, + 128), already in the swizzled order
+  const cuuint64_t rows = (cuuint64_t)((w.N + kTileN - 1) / kTileN) * (w.K / kTileK) * kTileN;
+  cuuint64_t dims[2] = {(cuuint64_t)kTileK, rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kTileK * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kTileK, (cuuint32_t)kTileN};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt =
+      w.elem == DFLASH_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = enc(&w.tmap, dt, 2, const_cast<void*>(tiled), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  w.tiled = tiled;
+  return true;
+}
+
 bool encode_weight_map(WeightMap& w, const void* ptr, int N, int K, int elem) {
   if (elem != DFLASH_BF16 && elem != DFLASH_F16) return false;
   w.ptr = ptr;
@@ -529,10 +648,26 @@ static int num_sms() {
   return sms[dev];
 }
 
+static int g_gemm_mode = 0;
+
+void gemm_set_mode(int mode) { g_gemm_mode = mode; }
+
+bool gemm_use_pair(int M, int N) {
+  if (g_gemm_mode == 1) return false;
+  if (g_gemm_mode == 2) return true;
+  // a pair halves the token bytes each SM stages and reads per weight byte;
+  // measured on B200 it pays only for a large token tile against a wide weight
+  // (SwiGLU gate/up and LM head at 224-256 tokens), where the coarser 256-row
+  // work units still balance across the SM pairs
+  return M > 160 && N >= 16384;
+}
+
 int gemm_pick_splits(int M, int N, int K, int max_splits) {
-  const int tiles = ((N + kTileN - 1) / kTileN) * ((M + kMaxBN - 1) / kMaxBN);
+  const bool pair = gemm_use_pair(M, N);
+  const int rows = pair ? 2 * kTileN : kTileN;
+  const int tiles = ((N + rows - 1) / rows) * ((M + kMaxBN - 1) / kMaxBN);
   const int nkb = K / kTileK;
-  const int sms = num_sms();
+  const int sms = pair ? num_sms() / 2 : num_sms();
   int best = 1;
   double best_score = -1.0;
   // at least 4 k-blocks (256 of K) per split keeps the TMA pipeline busy
@@ -540,7 +675,7 @@ int gemm_pick_splits(int M, int N, int K, int max_splits) {
   for (int s = 1; s <= smax; ++s) {
     const int se = gemm_effective_splits(K, s);
     const int units = tiles * se;
-    // persistent CTAs: the busiest SM runs ceil(units / sms) units
+    // persistent CTAs (pairs): the busiest one runs ceil(units / sms) units
     const int per_sm = (units + sms - 1) / sms;
     const double eff = (double)units / ((double)per_sm * sms);
     // each split writes (and its consumer reads) one fp32 partial of the
@@ -597,51 +732,60 @@ int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, i
   if (n_seg < 1 || n_seg > kMaxSeg || seg_k % kTileK != 0 || W.K != n_seg * seg_k)
     return DFLASH_EINVAL;
   const int BN = token_tile(M);
+  const bool pair = W.tiled != nullptr && gemm_use_pair(M, W.N);
+  const int bn_cta = pair ? BN / 2 : BN;
   BMaps maps;
   memset(&maps, 0, sizeof(maps));
   for (int i = 0; i < n_seg; ++i)
-    if (!encode_2d(&maps.m[i], xseg[i], M, seg_k, ld_seg, BN, W.elem)) return DFLASH_ECUDA;
+    if (!encode_2d(&maps.m[i], xseg[i], M, seg_k, ld_seg, bn_cta, W.elem)) return DFLASH_ECUDA;
 
   GemmArgs a;
   a.N = W.N;
   a.M = M;
   a.seg_k = seg_k;
   a.BN = BN;
-  const int stage_bytes = kTileN * 128 + BN * 128;
+  const int stage_bytes = kTileN * 128 + bn_cta * 128;
   a.n_kb = W.K / kTileK;
   if (epi == EPI_LMHEAD) splits = 1;
   splits = gemm_effective_splits(W.K, splits);
   a.kb_per_split = (a.n_kb + splits - 1) / splits;
-  a.tiles_n = (W.N + kTileN - 1) / kTileN;
+  a.tile_rows = pair ? 2 * kTileN : kTileN;
+  a.tiles_n = (W.N + a.tile_rows - 1) / a.tile_rows;
   a.tiles_m = (M + BN - 1) / BN;
   a.units = a.tiles_n * a.tiles_m * splits;
   a.splits = splits;
   // fused ops need the whole K range in one unit
   if (epi == EPI_PARTIAL && out.op != OP_PARTIAL && splits > 1) return DFLASH_EINVAL;
-  a.n_vtiles = a.tiles_n;
-  a.idesc = idesc_f16kind(kTileN, BN, W.elem == DFLASH_BF16);
+  a.n_vtiles = (W.N + kTileN - 1) / kTileN;
+  a.idesc = idesc_f16kind(a.tile_rows, BN, W.elem == DFLASH_BF16);
   a.a_tiled = static_cast<const uint8_t*>(W.tiled);
   a.out = out;
   a.err = err;
 
-  const size_t epi_bytes = epi == EPI_LMHEAD ? kLmSmem : kFusedSmem;
-  const size_t fixed = 1024 + epi_bytes + 8 * (2 * 8 + 4) + 16;
+  // plain partial stores need no epilogue staging: the space goes to stages
+  a.epi_bytes = epi == EPI_LMHEAD ? kLmSmem : (out.op == OP_PARTIAL ? 0 : kFusedSmem);
+  const size_t fixed = 1024 + a.epi_bytes + 8 * (2 * kMaxStages + 4) + 16;
   const size_t cap = 227 * 1024;
-  a.stages = (int)std::min<size_t>(8, (cap - fixed) / stage_bytes);
+  a.stages = (int)std::min<size_t>(kMaxStages, (cap - fixed) / stage_bytes);
   if (a.stages < 2) return DFLASH_EUNSUPPORTED;
   const size_t smem = fixed + (size_t)a.stages * stage_bytes;
-  const int grid = std::min(a.units, num_sms());
+  const int sms = num_sms();
   TimedScope ts(s, epi == EPI_LMHEAD ? TC_LMHEAD : TC_GEMM);
-  if (epi == EPI_PARTIAL) {
-    cudaFuncSetAttribute(gemm_tc_kernel<EPI_PARTIAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    gemm_tc_kernel<EPI_PARTIAL><<<grid, kGemmThreads, smem, s>>>(W.map, maps, a);
-  } else {
-    cudaFuncSetAttribute(gemm_tc_kernel<EPI_LMHEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    gemm_tc_kernel<EPI_LMHEAD><<<grid, kGemmThreads, smem, s>>>(W.map, maps, a);
+  if (!pair) {
+    const int grid = std::min(a.units, sms);
+    auto k = epi == EPI_PARTIAL ? gemm_tc_kernel<EPI_PARTIAL, false>
+                                : gemm_tc_kernel<EPI_LMHEAD, false>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const cudaError_t e =
+        launch_pdl(k, dim3(grid), dim3(kGemmThreads), smem, s, 1, W.map, maps, a);
+    return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
   }
-  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
+  auto k =
+      epi == EPI_PARTIAL ? gemm_tc_kernel<EPI_PARTIAL, true> : gemm_tc_kernel<EPI_LMHEAD, true>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const cudaError_t e = launch_pdl(k, dim3(2 * std::min(a.units, sms / 2)), dim3(kGemmThreads),
+                                   smem, s, 2, W.tmap, maps, a);
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 
 }  // namespace dflash

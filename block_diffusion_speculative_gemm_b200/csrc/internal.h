@@ -6,11 +6,41 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
 #include <vector>
 
 #include "../../include/dflash.h"
 
 namespace dflash {
+
+// ---------------------------------------------------------------- launches
+// Hot-path launch with programmatic stream serialization (the kernel starts
+// while its predecessor finishes; it must begin with pdl_trigger/pdl_wait as
+// common.cuh describes).  `cluster` > 1 also groups CTAs into clusters of
+// that many along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, int cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------------- timing
 enum TimingClass { TC_GEMM = 0, TC_ATTN = 1, TC_ROW = 2, TC_VERIFY = 3, TC_LMHEAD = 4, TC_N = 5 };
@@ -88,7 +118,8 @@ struct GemmOut {
 // 128-byte-swizzled shared-memory image of a [128 x 64] K-major tile, so the
 // GEMM fetches it with one bulk copy instead of a 128-row tensor box.
 struct WeightMap {
-  CUtensorMap map;
+  CUtensorMap map;         // row-major weights, 128-byte swizzle (when ptr is set)
+  CUtensorMap tmap;        // pre-tiled weights as rows of 128 bytes, no swizzle
   const void* ptr = nullptr;
   const void* tiled = nullptr;
   int N = 0, K = 0;
@@ -96,6 +127,13 @@ struct WeightMap {
 };
 
 bool encode_weight_map(WeightMap& w, const void* ptr, int N, int K, int elem);
+// Sets w.tiled and the tensor map the CTA-pair GEMM streams it through.
+bool set_tiled_weights(WeightMap& w, const void* tiled);
+
+// CTA-pair GEMM choice for M token rows and N weight rows; a debug override
+// (0 automatic, 1 single CTAs, 2 pairs) replaces the rule when non-zero.
+bool gemm_use_pair(int M, int N);
+void gemm_set_mode(int mode);
 
 // Writes the pre-tiled streaming image of a row-major 16-bit W [N, K] (K % 64
 // == 0) into dst (ceil(N/128) * K/64 * 16384 bytes; rows past N are zero).

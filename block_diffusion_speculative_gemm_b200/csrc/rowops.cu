@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(kRowThreads)
     embed_norm_kernel(const int32_t* __restrict__ tokens, const TE* __restrict__ emb,
                       const float* __restrict__ g, float* __restrict__ x, T* __restrict__ h, int d,
                       float eps) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[32];
   const int m = blockIdx.x;
   const int tok = tokens[m];
@@ -88,7 +90,8 @@ void launch_embed_norm(const int32_t* tokens, const TE* emb, const float* g, flo
                        int d, float eps, cudaStream_t s) {
   if (M <= 0) return;
   TimedScope ts(s, TC_ROW);
-  embed_norm_kernel<TE, T><<<M, kRowThreads, 0, s>>>(tokens, emb, g, x, h, d, eps);
+  launch_pdl(embed_norm_kernel<TE, T>, dim3(M), dim3(kRowThreads), 0, s, 1, tokens, emb, g, x, h, d,
+      eps);
 }
 
 // ---------------------------------------------------------------- residual + RMSNorm
@@ -100,6 +103,8 @@ __global__ void __launch_bounds__(kRowThreads)
     residual_norm_kernel(const float* __restrict__ part, int splits, int M, int d,
                          float* __restrict__ x, const float* __restrict__ g, T* __restrict__ h,
                          const int32_t* __restrict__ out_row, float eps) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[32];
   const int m = blockIdx.x;
   const size_t stride = (size_t)M * d;
@@ -144,8 +149,8 @@ void launch_residual_norm(const float* part, int splits, int M, int d, float* x,
                           T* h, const int32_t* out_row, float eps, cudaStream_t s) {
   if (M <= 0) return;
   TimedScope ts(s, TC_ROW);
-  residual_norm_kernel<T><<<M, kRowThreads, 0, s>>>(part, splits, M, d, x, g, h, out_row,
-                                                         eps);
+  launch_pdl(residual_norm_kernel<T>, dim3(M), dim3(kRowThreads), 0, s, 1, part, splits, M, d, x, g,
+      h, out_row, eps);
 }
 
 // ---------------------------------------------------------------- context-feature RMSNorm
@@ -154,6 +159,8 @@ template <typename T>
 __global__ void __launch_bounds__(kRowThreads)
     ctx_norm_kernel(const float* __restrict__ part, int splits, int n_rows, int d,
                     const float* __restrict__ g, T* __restrict__ c, float eps) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[32];
   const int n = blockIdx.x;
   const size_t stride = (size_t)n_rows * d;
@@ -184,7 +191,7 @@ void launch_ctx_norm(const float* part, int splits, int n, int d, const float* g
                      cudaStream_t s) {
   if (n <= 0) return;
   TimedScope ts(s, TC_ROW);
-  ctx_norm_kernel<T><<<n, kRowThreads, 0, s>>>(part, splits, n, d, g, c, eps);
+  launch_pdl(ctx_norm_kernel<T>, dim3(n), dim3(kRowThreads), 0, s, 1, part, splits, n, d, g, c, eps);
 }
 
 // ---------------------------------------------------------------- QKV epilogue
@@ -197,6 +204,8 @@ __global__ void qkv_post_kernel(const float* __restrict__ part, int splits, int 
                                 const int32_t* __restrict__ req_valid, int nq, int nkv, int hd,
                                 const float* __restrict__ cos_t, const float* __restrict__ sin_t,
                                 T* __restrict__ q, T* __restrict__ kb, T* __restrict__ vb) {
+  pdl_trigger();
+  pdl_wait();
   const int m = blockIdx.y;
   const int half = hd / 2;
   const int nh = nq + 2 * nkv;
@@ -236,8 +245,8 @@ void launch_qkv_post(const float* part, int splits, int M, int B, const int32_t*
   const int pairs = (nq + 2 * nkv) * hd / 2;
   dim3 grid((pairs / 4 + 255) / 256, M);
   TimedScope ts(s, TC_ROW);
-  qkv_post_kernel<T><<<grid, 256, 0, s>>>(part, splits, M, B, ctx_len, req_valid, nq, nkv, hd,
-                                          cos_t, sin_t, q, kb, vb);
+  launch_pdl(qkv_post_kernel<T>, dim3(grid), dim3(256), 0, s, 1, part, splits, M, B, ctx_len,
+      req_valid, nq, nkv, hd, cos_t, sin_t, q, kb, vb);
 }
 
 // ---------------------------------------------------------------- SwiGLU
@@ -246,6 +255,8 @@ void launch_qkv_post(const float* part, int splits, int M, int B, const int32_t*
 template <typename T>
 __global__ void swiglu_kernel(const float* __restrict__ part, int splits, int M, int I,
                               T* __restrict__ act) {
+  pdl_trigger();
+  pdl_wait();
   const int m = blockIdx.y;
   const int i = (blockIdx.x * blockDim.x + threadIdx.x) * 4;  // 4 features in one 64-block
   if (i >= I) return;
@@ -263,7 +274,7 @@ void launch_swiglu(const float* part, int splits, int M, int I, T* act, cudaStre
   if (M <= 0) return;
   dim3 grid((I / 4 + 255) / 256, M);
   TimedScope ts(s, TC_ROW);
-  swiglu_kernel<T><<<grid, 256, 0, s>>>(part, splits, M, I, act);
+  launch_pdl(swiglu_kernel<T>, dim3(grid), dim3(256), 0, s, 1, part, splits, M, I, act);
 }
 
 // ---------------------------------------------------------------- K/V cache scatter
@@ -277,6 +288,8 @@ __global__ void kv_scatter_kernel(const float* __restrict__ part, int splits, in
                                   const float* __restrict__ cos_t,
                                   const float* __restrict__ sin_t, int max_pos,
                                   T* __restrict__ kc, T* __restrict__ vc, int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   const int nl = blockIdx.y;       // row inside this chunk (partials)
   const int n = row0 + nl;         // row of the whole call (cu_rows)
   const int half = hd / 2;
@@ -333,8 +346,8 @@ void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int 
   const int pairs = L * 2 * nkv * hd / 2;
   dim3 grid((pairs / 4 + 255) / 256, n_rows);
   TimedScope ts(s, TC_ROW);
-  kv_scatter_kernel<T><<<grid, 256, 0, s>>>(part, splits, n_rows, row0, L, nkv, hd, cu_rows, start_pos,
-                                            batch, cap, cos_t, sin_t, max_pos, kc, vc, err);
+  launch_pdl(kv_scatter_kernel<T>, dim3(grid), dim3(256), 0, s, 1, part, splits, n_rows, row0, L,
+      nkv, hd, cu_rows, start_pos, batch, cap, cos_t, sin_t, max_pos, kc, vc, err);
 }
 
 // T: activation type (GEMM operand); TC: K/V cache type; TE: embedding type.

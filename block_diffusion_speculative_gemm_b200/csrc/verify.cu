@@ -23,6 +23,8 @@ struct ArgPart {
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kVerifyThreads)
     verify_argmax_kernel(const T* __restrict__ logits, int V, int chunk, ArgPart* __restrict__ part) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float s_v[kVerifyThreads / 32];
   __shared__ int s_i[kVerifyThreads / 32];
   const int row = blockIdx.y, c = blockIdx.x;
@@ -72,6 +74,8 @@ __global__ void verify_accept_kernel(const ArgPart* __restrict__ part, int chunk
                                      int32_t* out_tokens, int32_t* out_len, int out_cap,
                                      int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
                                      int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= batch) return;
@@ -133,20 +137,24 @@ int launch_verify(const void* logits, int dtype, const int32_t* draft, int batch
     TimedScope ts(s, TC_VERIFY);
     if (dtype == DFLASH_BF16) {
       const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(logits);
-      if (vec) verify_argmax_kernel<__nv_bfloat16, true><<<grid, kVerifyThreads, 0, s>>>(x, V, chunk, part);
-      else verify_argmax_kernel<__nv_bfloat16, false><<<grid, kVerifyThreads, 0, s>>>(x, V, chunk, part);
+      if (vec) launch_pdl(verify_argmax_kernel<__nv_bfloat16, true>, dim3(grid),
+          dim3(kVerifyThreads), 0, s, 1, x, V, chunk, part);
+      else launch_pdl(verify_argmax_kernel<__nv_bfloat16, false>, dim3(grid), dim3(kVerifyThreads),
+          0, s, 1, x, V, chunk, part);
     } else {
       const float* x = static_cast<const float*>(logits);
-      if (vec) verify_argmax_kernel<float, true><<<grid, kVerifyThreads, 0, s>>>(x, V, chunk, part);
-      else verify_argmax_kernel<float, false><<<grid, kVerifyThreads, 0, s>>>(x, V, chunk, part);
+      if (vec) launch_pdl(verify_argmax_kernel<float, true>, dim3(grid), dim3(kVerifyThreads), 0, s,
+          1, x, V, chunk, part);
+      else launch_pdl(verify_argmax_kernel<float, false>, dim3(grid), dim3(kVerifyThreads), 0, s, 1,
+          x, V, chunk, part);
     }
   }
   {
     TimedScope ts(s, TC_VERIFY);
     const int wpb = 4;
-    verify_accept_kernel<<<(batch + wpb - 1) / wpb, 32 * wpb, 0, s>>>(
-        part, chunks, draft, batch, B, V, out_tokens, out_len, out_cap, seq_lens, accept_len,
-        next_anchor, err);
+    launch_pdl(verify_accept_kernel, dim3((batch + wpb - 1) / wpb), dim3(32 * wpb), 0, s, 1, part,
+        chunks, draft, batch, B, V, out_tokens, out_len, out_cap, seq_lens, accept_len, next_anchor,
+        err);
   }
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }

@@ -45,6 +45,8 @@ int scratch_address(void** out) {
 }
 
 __global__ void copy_error_word(const int32_t* __restrict__ src, int32_t* __restrict__ dst) {
+  pdl_trigger();
+  pdl_wait();
   *dst = *src;
 }
 
@@ -81,7 +83,7 @@ extern "C" int dflash_verify_noalloc(const void* target_logits, int logits_dtype
                      static_cast<unsigned char*>(scratch) + kNoAllocHeader, chunks, err, s);
   if (st != DFLASH_OK) return st;
   if (error_bits) {
-    copy_error_word<<<1, 1, 0, s>>>(err, error_bits);
+    launch_pdl(copy_error_word, dim3(1), dim3(1), 0, s, 1, err, error_bits);
     if (cudaGetLastError() != cudaSuccess) return DFLASH_ECUDA;
   }
   return DFLASH_OK;

@@ -90,6 +90,8 @@ def lib() -> ctypes.CDLL:
         L.dflash_debug_tiled_bytes.argtypes = [i32, i32]
         L.dflash_debug_tiled_bytes.restype = sz
         L.dflash_debug_tile_weights.argtypes = [vp, vp, i32, i32, vp]
+        L.dflash_debug_lmhead_tiled.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp, vp, vp]
+        L.dflash_debug_gemm_mode.argtypes = [i32]
         _lib = L
     return _lib
 
@@ -336,6 +338,16 @@ def timing_read() -> Dict[str, Dict[str, float]]:
 _ELEM = {torch.bfloat16: BF16, torch.float16: F16}
 
 
+def debug_tile_weights(W: torch.Tensor, stream=None) -> torch.Tensor:
+    """The pre-tiled streaming image (uint8) of a 16-bit weight W [N, K]."""
+    _need(W, "W")
+    N, K = W.shape
+    Wt = torch.empty(lib().dflash_debug_tiled_bytes(N, K), dtype=torch.uint8, device=W.device)
+    _check("dflash_debug_tile_weights", lib().dflash_debug_tile_weights(
+        _ptr(W), _ptr(Wt), N, K, _stream(stream)))
+    return Wt
+
+
 def debug_gemm(W: torch.Tensor, X: torch.Tensor, splits: int, err_ws: torch.Tensor, stream=None,
                tiled: bool = False):
     """fp32 split-K partials [splits_used, M, N] of X @ W^T from the tcgen05 core
@@ -352,9 +364,7 @@ def debug_gemm(W: torch.Tensor, X: torch.Tensor, splits: int, err_ws: torch.Tens
     out = torch.empty((s_used, M, N), dtype=torch.float32, device=W.device)
     used = ctypes.c_int(0)
     if tiled:
-        Wt = torch.empty(lib().dflash_debug_tiled_bytes(N, K), dtype=torch.uint8, device=W.device)
-        _check("dflash_debug_tile_weights", lib().dflash_debug_tile_weights(
-            _ptr(W), _ptr(Wt), N, K, _stream(stream)))
+        Wt = debug_tile_weights(W, stream)
         _check("dflash_debug_gemm_tiled", lib().dflash_debug_gemm_tiled(
             _ptr(Wt), N, K, _ptr(X), M, elem, s_req, _ptr(out), ctypes.byref(used),
             _ptr(err_ws), _stream(stream)))
@@ -367,8 +377,9 @@ def debug_gemm(W: torch.Tensor, X: torch.Tensor, splits: int, err_ws: torch.Tens
 
 
 def debug_lmhead(W: torch.Tensor, X: torch.Tensor, err_ws: torch.Tensor, want_logits=True,
-                 stream=None):
-    """(stats [M, tiles, 4] as (max, idx, sumexp, 0), logits [M, N] or None)."""
+                 stream=None, tiled: bool = False):
+    """(stats [M, tiles, 4] as (max, idx, sumexp, 0), logits [M, N] or None);
+    ``tiled`` streams W from its pre-tiled image."""
     _need(W, "W")
     _need(X, "X", W.dtype)
     elem = _ELEM[W.dtype]
@@ -377,6 +388,19 @@ def debug_lmhead(W: torch.Tensor, X: torch.Tensor, err_ws: torch.Tensor, want_lo
     tiles = -(-N // 128)
     stats = torch.empty((M, tiles, 4), dtype=torch.float32, device=W.device)
     logits = torch.empty((M, N), dtype=torch.float32, device=W.device) if want_logits else None
-    _check("dflash_debug_lmhead", lib().dflash_debug_lmhead(
-        _ptr(W), N, K, _ptr(X), M, elem, _ptr(stats), _ptr(logits), _ptr(err_ws), _stream(stream)))
+    if tiled:
+        Wt = debug_tile_weights(W, stream)
+        _check("dflash_debug_lmhead_tiled", lib().dflash_debug_lmhead_tiled(
+            _ptr(Wt), N, K, _ptr(X), M, elem, _ptr(stats), _ptr(logits), _ptr(err_ws),
+            _stream(stream)))
+    else:
+        _check("dflash_debug_lmhead", lib().dflash_debug_lmhead(
+            _ptr(W), N, K, _ptr(X), M, elem, _ptr(stats), _ptr(logits), _ptr(err_ws),
+            _stream(stream)))
     return stats, logits
+
+
+def debug_gemm_mode(mode: int) -> None:
+    """Process-wide GEMM launch mode for tiled weights: 0 the library's rule,
+    1 single CTAs, 2 CTA pairs (tests only)."""
+    _check("dflash_debug_gemm_mode", lib().dflash_debug_gemm_mode(int(mode)))

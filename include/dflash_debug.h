@@ -43,6 +43,18 @@ int dflash_debug_tile_weights(const void* W, void* W_tiled, int N, int K, void* 
 int dflash_debug_lmhead(const void* W, int N, int K, const void* X, int M, int elem, void* stats,
                         float* logits, void* err_ws, void* stream);
 
+/* Same as dflash_debug_lmhead with the weights read from their pre-tiled
+ * image (the layout the model's LM head uses). */
+int dflash_debug_lmhead_tiled(const void* W_tiled, int N, int K, const void* X, int M, int elem,
+                              void* stats, float* logits, void* err_ws, void* stream);
+
+/* How the tiled GEMMs are launched from now on, process-wide: 0 = the
+ * library's rule, 1 = one CTA per 128-row weight tile, 2 = CTA pairs (cluster
+ * of two CTAs on one TPC sharing a 256-row weight tile, M = 256 tcgen05.mma
+ * with cta_group::2).  Non-tiled weights always use single CTAs.  Returns
+ * DFLASH_EINVAL for any other value.  Not thread-safe; tests only. */
+int dflash_debug_gemm_mode(int mode);
+
 #ifdef __cplusplus
 }
 #endif

@@ -7,6 +7,16 @@ from block_diffusion_speculative_gemm_b200 import dflash as D
 
 pytestmark = pytest.mark.gpu
 
+# weight layout and launch shape: row-major weights through a tensor map (single
+# CTAs), or the pre-tiled image with single CTAs or CTA pairs (cta_group::2)
+MODES = {"rowmajor": (False, 0), "single": (True, 1), "pair": (True, 2)}
+
+
+@pytest.fixture(autouse=True)
+def _reset_mode():
+    yield
+    D.debug_gemm_mode(0)
+
 
 def _inputs(N, K, M, seed, dtype=torch.bfloat16):
     g = torch.Generator().manual_seed(seed)
@@ -23,10 +33,14 @@ def _inputs(N, K, M, seed, dtype=torch.bfloat16):
     (512, 1024, 300, 2),     # two token tiles, ragged second one
     (128, 192, 1, 5),        # one token row, more splits than fit evenly
     (6144, 4096, 256, 3),    # QKV projection of the 8B-shaped draft
+    (640, 320, 64, 2),       # five weight tiles: the last pair has one live half
+    (130, 128, 48, 1),       # two weight tiles, the second with 2 live rows
 ])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
-@pytest.mark.parametrize("tiled", [False, True])
-def test_gemm_matches_float64(N, K, M, splits, dtype, tiled):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_gemm_matches_float64(N, K, M, splits, dtype, mode):
+    tiled, launch = MODES[mode]
+    D.debug_gemm_mode(launch)
     W, X = _inputs(N, K, M, N * 7 + K + M, dtype)
     err = D.new_workspace(256)
     out = D.debug_gemm(W.cuda(), X.cuda(), splits, err, tiled=tiled)
@@ -46,10 +60,13 @@ def test_gemm_matches_float64(N, K, M, splits, dtype, tiled):
 
 @pytest.mark.parametrize("N,K,M", [(1024, 256, 40), (151936 // 16, 512, 224), (2000, 128, 96)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
-def test_lmhead_epilogue_stats(N, K, M, dtype):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_lmhead_epilogue_stats(N, K, M, dtype, mode):
+    tiled, launch = MODES[mode]
+    D.debug_gemm_mode(launch)
     W, X = _inputs(N, K, M, N + K + M, dtype)
     err = D.new_workspace(256)
-    stats, logits = D.debug_lmhead(W.cuda(), X.cuda(), err)
+    stats, logits = D.debug_lmhead(W.cuda(), X.cuda(), err, tiled=tiled)
     torch.cuda.synchronize()
     assert D.get_error(err) == 0
     ref = (X.double() @ W.double().T)
