@@ -217,6 +217,7 @@ int qkv_out(const dflash_config& c) { return (c.n_q + 2 * c.n_kv) * c.head_dim; 
 // Workspace header: word 0 = device error bits.
 constexpr size_t kHeader = 256;
 constexpr int kMaxChunks = 64;
+int g_attn_chunk = 0;  // split-KV chunk override in keys (tests and tuning; 0 = rule)
 constexpr int kAttnRows = 64;
 constexpr int kInjectChunkRows = 16384;
 constexpr int kMaxSplits = 16;
@@ -648,6 +649,8 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
   // split-KV chunk: a multiple of the attention tile (64 keys), at least 512 keys
   int chunk = (cap + B + kMaxChunks - 1) / kMaxChunks;
   chunk = std::max(512, (chunk + 63) / 64 * 64);
+  if (g_attn_chunk > 0 && (cap + B + g_attn_chunk - 1) / g_attn_chunk <= kMaxChunks)
+    chunk = g_attn_chunk;
   const int n_chunks = (cap + B + chunk - 1) / chunk;
 
   launch_draft_init(anchor, ctx_len, batch, B, c.vocab, c.mask_id, cap, tokens, zrow, lm_rows,
@@ -862,6 +865,12 @@ extern "C" int dflash_debug_tile_weights(const void* W, void* Wt, int N, int K, 
     return DFLASH_EINVAL;
   tile_weights(W, Wt, N, K, (cudaStream_t)stream);
   return cuda_status();
+}
+
+extern "C" int dflash_debug_attn_chunk(int keys) {
+  if (keys < 0 || keys % 64 != 0) return DFLASH_EINVAL;
+  g_attn_chunk = keys;
+  return DFLASH_OK;
 }
 
 extern "C" int dflash_debug_gemm_mode(int mode) {

@@ -21,7 +21,8 @@ namespace dflash {
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kComputeWarps = 4;
+constexpr int kThreads = 32 * kComputeWarps + 32;  // + one producer warp
 constexpr int kKeys = 64;    // keys per context tile
 constexpr int kBlkKeys = 16; // rows of the block tile
 
@@ -73,8 +74,9 @@ __device__ __forceinline__ uint32_t toff(int rows, int row, int c) {
 }
 
 // Shared memory of one CTA: the TMA stage ring, then the query rows (later
-// reused for the block tile), then the stage barriers.  Sized so that two
-// CTAs fit on an SM: 3 stages for up to 32 query rows, 2 stages for 64.
+// reused for the block tile), then the stage barriers (full, then empty).
+// Sized so that two CTAs fit on an SM: 3 stages for up to 32 query rows, 2
+// stages for 64.
 template <int HD, int MT>
 struct Layout {
   static constexpr int kStages = MT <= 2 ? 3 : 2;
@@ -82,7 +84,7 @@ struct Layout {
   static constexpr int kStage = 2 * kTile;
   static constexpr int kQRows = MT * 16;
   static constexpr int kQ = (kQRows > 2 * kBlkKeys ? kQRows : 2 * kBlkKeys) * HD * 2;
-  static constexpr int kBars = kStages * 8;
+  static constexpr int kBars = 2 * kStages * 8;
   static constexpr int kSmem = kStages * kStage + kQ + kBars + 1024;  // + alignment slack
   static_assert(2 * kBlkKeys * HD * 2 <= kQ, "block tile fits the query area");
 };
@@ -95,15 +97,40 @@ struct Warp {
   static constexpr int KS = HD / 16;
 };
 
+// Byte offsets of this lane's ldmatrix rows inside a swizzled tile: every row
+// a lane addresses has row & 7 == lane & 7, so the swizzle term of 16-byte
+// chunk j is (j ^ (lane & 7)) << 4.  K fragments (non-transposed) take chunk
+// 2 q + (mi & 1) of column half q / 4; V fragments (transposed) take chunk
+// 2 q + (mi >> 1).
+struct LdsmOff {
+  uint32_t rk, rv;        // row offset of the lane's K / V row inside a 16-row group
+  uint32_t xk[4], xv[4];  // swizzled chunk offsets for q = 0..3
+};
+__device__ __forceinline__ LdsmOff ldsm_offsets(int lane) {
+  const int mi = lane >> 3, li = lane & 7;
+  LdsmOff o;
+  o.rk = (uint32_t)(((mi >> 1) * 8 + li) * 128);
+  o.rv = (uint32_t)(((mi & 1) * 8 + li) * 128);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    o.xk[q] = (uint32_t)(((2 * q + (mi & 1)) ^ li) << 4);
+    o.xv[q] = (uint32_t)(((2 * q + (mi >> 1)) ^ li) << 4);
+  }
+  return o;
+}
+
 // One tile's worth of keys for one warp: keys [kbeg, kbeg + NKEYS) of a tile
 // stored with `rows` rows; keys at tile-local index >= nvalid are masked.
+// The running row maxima m0/m1 are kept in log2 units of the scaled score
+// (score * sl2, sl2 = log2(e) / sqrt(hd)), so that every exponential is one
+// FMA and one exp2.
 template <int HD, int NKEYS>
 __device__ __forceinline__ void attend(uint32_t sK, uint32_t sV, int rows, int kbeg, int nvalid,
                                        const uint32_t (&qa)[HD / 16][4], float (&o)[HD / 8][4],
-                                       float& m0, float& m1, float& l0, float& l1, float scale,
-                                       int lane) {
+                                       float& m0, float& m1, float& l0, float& l1, float sl2,
+                                       const LdsmOff& lo, int lane) {
   constexpr int NS = NKEYS / 8;
-  const int tq = lane & 3, mi = lane >> 3, li = lane & 7;
+  const int tq = lane & 3;
   float s[NS][4];
 #pragma unroll
   for (int n = 0; n < NS; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
@@ -112,50 +139,60 @@ __device__ __forceinline__ void attend(uint32_t sK, uint32_t sV, int rows, int k
 #pragma unroll
     for (int np = 0; np < NKEYS / 16; ++np) {
       uint32_t b0, b1, b2, b3;
-      const int row = kbeg + np * 16 + (mi >> 1) * 8 + li;
-      ldsm_x4(sK + toff(rows, row, ks * 2 + (mi & 1)), b0, b1, b2, b3);
+      ldsm_x4(sK + (ks >> 2) * rows * 128 + (kbeg + np * 16) * 128 + lo.rk + lo.xk[ks & 3], b0,
+              b1, b2, b3);
       mma16816(s[2 * np], qa[ks], b0, b1);
       mma16816(s[2 * np + 1], qa[ks], b2, b3);
     }
   }
+  if (kbeg + NKEYS > nvalid) {  // keys past the context in this warp's range
+#pragma unroll
+    for (int n = 0; n < NS; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (kbeg + n * 8 + 2 * tq + (e & 1) >= nvalid) s[n][e] = -INFINITY;
+  }
   float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-  for (int n = 0; n < NS; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int k = kbeg + n * 8 + 2 * tq + (e & 1);
-      s[n][e] = k < nvalid ? s[n][e] * scale : -INFINITY;
-      if (e < 2) mx0 = fmaxf(mx0, s[n][e]); else mx1 = fmaxf(mx1, s[n][e]);
-    }
+  for (int n = 0; n < NS; ++n) {
+    mx0 = fmaxf(mx0, fmaxf(s[n][0], s[n][1]));
+    mx1 = fmaxf(mx1, fmaxf(s[n][2], s[n][3]));
+  }
   mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
   mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
   mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
   mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-  const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+  const float n0 = fmaxf(m0, mx0 * sl2), n1 = fmaxf(m1, mx1 * sl2);
   // every key masked (the same for all rows): nothing to add
-  if (__all_sync(0xffffffffu, n0 == -INFINITY && n1 == -INFINITY)) return;
-  const float c0 = (m0 == -INFINITY) ? 0.f : expf(m0 - n0);
-  const float c1 = (m1 == -INFINITY) ? 0.f : expf(m1 - n1);
+  if (kbeg + NKEYS > nvalid && __all_sync(0xffffffffu, n0 == -INFINITY && n1 == -INFINITY))
+    return;
+  const float c0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - n0);
+  const float c1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - n1);
   float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-  for (int n = 0; n < NS; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float mref = e < 2 ? n0 : n1;
-      s[n][e] = s[n][e] == -INFINITY ? 0.f : expf(s[n][e] - mref);
-      if (e < 2) ps0 += s[n][e]; else ps1 += s[n][e];
-    }
+  for (int n = 0; n < NS; ++n) {
+    // a masked score is -inf and gives exp2(-inf) = 0 (n0, n1 are finite here)
+    s[n][0] = exp2f(fmaf(s[n][0], sl2, -n0));
+    s[n][1] = exp2f(fmaf(s[n][1], sl2, -n0));
+    s[n][2] = exp2f(fmaf(s[n][2], sl2, -n1));
+    s[n][3] = exp2f(fmaf(s[n][3], sl2, -n1));
+    ps0 += s[n][0] + s[n][1];
+    ps1 += s[n][2] + s[n][3];
+  }
   l0 = l0 * c0 + ps0;
   l1 = l1 * c1 + ps1;
+  // the output only needs rescaling when some row's maximum moved
+  if (__any_sync(0xffffffffu, n0 != m0 || n1 != m1)) {
+#pragma unroll
+    for (int n = 0; n < HD / 8; ++n) {
+      o[n][0] *= c0;
+      o[n][1] *= c0;
+      o[n][2] *= c1;
+      o[n][3] *= c1;
+    }
+  }
   m0 = n0;
   m1 = n1;
-#pragma unroll
-  for (int n = 0; n < HD / 8; ++n) {
-    o[n][0] *= c0;
-    o[n][1] *= c0;
-    o[n][2] *= c1;
-    o[n][3] *= c1;
-  }
 #pragma unroll
   for (int kb = 0; kb < NKEYS / 16; ++kb) {
     const uint32_t pa[4] = {pack_h2(s[2 * kb][0], s[2 * kb][1]),
@@ -165,14 +202,19 @@ __device__ __forceinline__ void attend(uint32_t sK, uint32_t sV, int rows, int k
 #pragma unroll
     for (int nd = 0; nd < HD / 8; nd += 2) {
       uint32_t b0, b1, b2, b3;
-      const int row = kbeg + kb * 16 + (mi & 1) * 8 + li;
-      ldsm_x4_t(sV + toff(rows, row, nd + (mi >> 1)), b0, b1, b2, b3);
+      ldsm_x4_t(sV + (nd >> 3) * rows * 128 + (kbeg + kb * 16) * 128 + lo.rv +
+                    lo.xv[(nd & 7) >> 1],
+                b0, b1, b2, b3);
       mma16816(o[nd], pa, b0, b1);
       mma16816(o[nd + 1], pa, b2, b3);
     }
   }
 }
 
+// Warps 0-3 compute (warp (mt, kg) = (warp % MT, warp / MT)); warp 4 lane 0
+// streams the context tiles: it refills a stage once the four compute warps
+// have released it on the stage's `empty` barrier, so the warps never wait
+// for one another inside the tile loop.
 template <int HD, int MT>
 __global__ void __launch_bounds__(kThreads)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -194,6 +236,8 @@ __global__ void __launch_bounds__(kThreads)
   const uint32_t s_base = smem_u32(smem);
   const uint32_t s_q = s_base + kStages * LY::kStage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * LY::kStage + LY::kQ);
+  auto full = [&](int st) { return smem_u32(bars + st); };
+  auto empty = [&](int st) { return smem_u32(bars + kStages + st); };
 
   const int c = blockIdx.x, g = blockIdx.y, r = blockIdx.z;
   const int G = nq / nkv;
@@ -208,10 +252,13 @@ __global__ void __launch_bounds__(kThreads)
   const int row_base = ((layer * batch + r) * nkv + g) * cap;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mt = warp % MT, kg = warp / MT;
-  const bool computes = warp < MT * KG;
+  const bool computes = warp < kComputeWarps;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(bars + s), 1);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(full(st), 1);
+      mbar_init(empty(st), kComputeWarps);
+    }
     fence_barrier_init();
   }
   // query rows of this kv head: row i = (block position i / G, head g*G + i % G)
@@ -231,27 +278,26 @@ __global__ void __launch_bounds__(kThreads)
   auto issue = [&](int t) {  // one thread: TMA of context tile t into its stage
     const int st = t % kStages;
     const uint32_t sK = s_base + st * LY::kStage, sV = sK + LY::kTile;
-    const uint32_t bar = smem_u32(bars + st);
-    mbar_arrive_expect_tx(bar, 2 * LY::kTile);
+    mbar_arrive_expect_tx(full(st), 2 * LY::kTile);
     const int y = row_base + k0 + t * kKeys;
 #pragma unroll
     for (int h = 0; h < HALVES; ++h) {
-      tma_load_2d(sK + h * kKeys * 128, &tmK, bar, h * 64, y, policy_evict_first());
-      tma_load_2d(sV + h * kKeys * 128, &tmV, bar, h * 64, y, policy_evict_first());
+      tma_load_2d(sK + h * kKeys * 128, &tmK, full(st), h * 64, y, policy_evict_first());
+      tma_load_2d(sV + h * kKeys * 128, &tmV, full(st), h * 64, y, policy_evict_first());
     }
   };
-  if (tid == 0) {
-    fence_proxy_async();
-    for (int t = 0; t < kStages - 1 && t < nt; ++t) issue(t);
-  }
+  const bool producer = warp == kComputeWarps && lane == 0;
+  if (producer)
+    for (int t = 0; t < kStages && t < nt; ++t) issue(t);  // fresh stages
 
   uint32_t qa[KS][4];
   float o[NT][4];
 #pragma unroll
   for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  const float scale = rsqrtf((float)HD);
+  const float sl2 = rsqrtf((float)HD) * 1.4426950408889634f;  // log2(e) / sqrt(hd)
   const int mi = lane >> 3, li = lane & 7;
+  const LdsmOff lo = ldsm_offsets(lane);
 
   cp_async_wait_all();
   __syncthreads();
@@ -283,36 +329,45 @@ __global__ void __launch_bounds__(kThreads)
   }
 
   bool ok = true;
-  for (int t = 0; t < nt; ++t) {
-    const int st = t % kStages;
-    if (tid == 0 && t + kStages - 1 < nt) {
-      fence_proxy_async();
-      issue(t + kStages - 1);
+  if (producer) {
+    for (int t = kStages; t < nt; ++t) {
+      const int st = t % kStages;
+      if (!mbar_wait(empty(st), ((t / kStages) + 1) & 1)) { ok = false; break; }
+      issue(t);
     }
-    if (!mbar_wait(smem_u32(bars + st), (t / kStages) & 1)) ok = false;
-    const int nvalid = min(kKeys, kc_end - (k0 + t * kKeys));
-    const uint32_t sK = s_base + st * LY::kStage, sV = sK + LY::kTile;
-    if (nvalid < kKeys) {
-      // rows past the context hold other cache positions: zero V so that
-      // masked keys contribute exactly nothing
-      uint8_t* v = smem + st * LY::kStage + LY::kTile;
-      for (int idx = tid; idx < (kKeys - nvalid) * (HD / 8); idx += kThreads) {
-        const int row = nvalid + idx / (HD / 8), ch = idx % (HD / 8);
-        *reinterpret_cast<uint4*>(v + toff(kKeys, row, ch)) = make_uint4(0, 0, 0, 0);
+  } else if (computes) {
+    for (int t = 0; t < nt; ++t) {
+      const int st = t % kStages;
+      if (!mbar_wait(full(st), (t / kStages) & 1)) ok = false;
+      const int nvalid = min(kKeys, kc_end - (k0 + t * kKeys));
+      const uint32_t sK = s_base + st * LY::kStage, sV = sK + LY::kTile;
+      const int kbeg = kg * KPW;
+      if (nvalid < kbeg + KPW) {
+        // rows past the context hold other cache positions: zero this warp's V
+        // rows there so that masked keys contribute exactly nothing (the other
+        // warp of the same key group writes the same zeros)
+        uint8_t* v = smem + st * LY::kStage + LY::kTile;
+        const int z0 = max(nvalid, kbeg);
+        for (int idx = lane; idx < (kbeg + KPW - z0) * (HD / 8); idx += 32) {
+          const int row = z0 + idx / (HD / 8), ch = idx % (HD / 8);
+          *reinterpret_cast<uint4*>(v + toff(kKeys, row, ch)) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async();  // before the stage goes back to the TMA
+        __syncwarp();
       }
-      __syncthreads();
+      attend<HD, KPW>(sK, sV, kKeys, kbeg, nvalid, qa, o, m0, m1, l0, l1, sl2, lo, lane);
+      __syncwarp();
+      if (lane == 0)
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty(st)) : "memory");
     }
-    if (computes)
-      attend<HD, KPW>(sK, sV, kKeys, kg * KPW, nvalid, qa, o, m0, m1, l0, l1, scale, lane);
-    __syncthreads();
   }
-  if (!ok && tid == 0) set_error(err, DFLASH_DEV_TIMEOUT);
+  if (!ok) set_error(err, DFLASH_DEV_TIMEOUT);
   if (has_blk) {
     cp_async_wait_all();
     __syncthreads();
     if (computes && kg == 0)
       attend<HD, kBlkKeys>(s_q, s_q + kBlkKeys * HD * 2, kBlkKeys, 0, kb_hi - kb_lo, qa, o, m0, m1,
-                           l0, l1, scale, lane);
+                           l0, l1, sl2, lo, lane);
   }
 
   // row sums over the quad, then merge the key groups of each row tile
@@ -323,7 +378,7 @@ __global__ void __launch_bounds__(kThreads)
   constexpr int kSlot = NT * 4 + 4;
   static_assert(4 * 32 * kSlot * 4 <= kStages * LY::kStage, "merge scratch");
   float* scratch = reinterpret_cast<float*>(smem);
-  __syncthreads();
+  __syncthreads();  // every tile consumed: the stage ring becomes merge scratch
   if (KG > 1 && computes && kg > 0) {
     float* sl = scratch + ((size_t)warp * 32 + lane) * kSlot;
 #pragma unroll
@@ -342,10 +397,10 @@ __global__ void __launch_bounds__(kThreads)
     const float* sl = scratch + ((size_t)(k * MT + mt) * 32 + lane) * kSlot;
     const float pm0 = sl[NT * 4 + 0], pm1 = sl[NT * 4 + 1];
     const float nm0 = fmaxf(m0, pm0), nm1 = fmaxf(m1, pm1);
-    const float a0 = m0 == -INFINITY ? 0.f : expf(m0 - nm0);
-    const float a1 = m1 == -INFINITY ? 0.f : expf(m1 - nm1);
-    const float b0 = pm0 == -INFINITY ? 0.f : expf(pm0 - nm0);
-    const float b1 = pm1 == -INFINITY ? 0.f : expf(pm1 - nm1);
+    const float a0 = m0 == -INFINITY ? 0.f : exp2f(m0 - nm0);
+    const float a1 = m1 == -INFINITY ? 0.f : exp2f(m1 - nm1);
+    const float b0 = pm0 == -INFINITY ? 0.f : exp2f(pm0 - nm0);
+    const float b1 = pm1 == -INFINITY ? 0.f : exp2f(pm1 - nm1);
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       o[n][0] = o[n][0] * a0 + sl[n * 4 + 0] * b0;
@@ -358,6 +413,10 @@ __global__ void __launch_bounds__(kThreads)
     m0 = nm0;
     m1 = nm1;
   }
+  // partial maxima leave in natural-log units of the scaled score
+  const float ln2 = 0.6931471805599453f;
+  m0 *= ln2;
+  m1 *= ln2;
   const size_t pbase = (((size_t)r * nkv + g) * n_chunks + c) * kAttnMaxRows;
   const int tq = lane & 3;
   const int row0 = mt * 16 + (lane >> 2), row1 = row0 + 8;

@@ -92,6 +92,7 @@ def lib() -> ctypes.CDLL:
         L.dflash_debug_tile_weights.argtypes = [vp, vp, i32, i32, vp]
         L.dflash_debug_lmhead_tiled.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp, vp, vp]
         L.dflash_debug_gemm_mode.argtypes = [i32]
+        L.dflash_debug_attn_chunk.argtypes = [i32]
         _lib = L
     return _lib
 
@@ -398,6 +399,12 @@ def debug_lmhead(W: torch.Tensor, X: torch.Tensor, err_ws: torch.Tensor, want_lo
             _ptr(W), N, K, _ptr(X), M, elem, _ptr(stats), _ptr(logits), _ptr(err_ws),
             _stream(stream)))
     return stats, logits
+
+
+def debug_attn_chunk(keys: int) -> None:
+    """Process-wide split-KV chunk (keys, multiple of 64) of the draft attention;
+    0 restores the library's rule (tests and tuning only)."""
+    _check("dflash_debug_attn_chunk", lib().dflash_debug_attn_chunk(int(keys)))
 
 
 def debug_gemm_mode(mode: int) -> None:

@@ -55,6 +55,13 @@ int dflash_debug_lmhead_tiled(const void* W_tiled, int N, int K, const void* X, 
  * DFLASH_EINVAL for any other value.  Not thread-safe; tests only. */
 int dflash_debug_gemm_mode(int mode);
 
+/* Split-KV chunk of the draft attention, in keys, for every later
+ * dflash_draft_block call, process-wide: 0 = the library's rule (at least 512
+ * keys, at most 64 chunks per request), else a multiple of 64 that is used
+ * whenever it gives at most 64 chunks.  Returns DFLASH_EINVAL for a negative
+ * value or one that is not a multiple of 64.  Not thread-safe; tests only. */
+int dflash_debug_attn_chunk(int keys);
+
 #ifdef __cplusplus
 }
 #endif

@@ -97,6 +97,24 @@ def test_draft_context_lengths_edge_cases():
     print(_check(b, cfg, res, cfg.steps, range(cfg.batch)))
 
 
+@pytest.mark.parametrize("chunk", [64, 192, 4096])
+def test_draft_attention_chunk_sizes(chunk):
+    """The same requests with the split-KV chunk forced from one tile per chunk to one
+    chunk per request: every split and the chunk combine give the oracle's result."""
+    base = synth.get_config("qwen3_8b_bs32")
+    cfg = shrink(base, L=1, V=2048, batch=4, ctx=("uniform", 1, 900), I=512, d=512,
+                 H_t=512).replace(name="chunk8b")
+    b = built(cfg)
+    ctx = torch.tensor([0, 63, 64, 900], dtype=torch.int32)
+    D.debug_attn_chunk(chunk)
+    try:
+        res = _run_draft(b, cfg, ctx=ctx)
+    finally:
+        D.debug_attn_chunk(0)
+    assert res["err"] == 0
+    print(chunk, _check(b, cfg, res, cfg.steps, range(cfg.batch)))
+
+
 def test_draft_rejects_bad_requests_without_writing():
     base = synth.get_config("qwen3_8b_bs32")
     cfg = shrink(base, L=1, V=2048, batch=3, ctx=("fixed", 16), I=512, d=512, H_t=512).replace(
