@@ -215,7 +215,12 @@ int qkv_out(const dflash_config& c) { return (c.n_q + 2 * c.n_kv) * c.head_dim; 
 
 // ---------------------------------------------------------------- workspace layout
 // Workspace header: word 0 = device error bits.
-constexpr size_t kHeader = 256;
+// Workspace header: the device error word (byte 0), then one verify
+// completion counter per request (at most 65535 / 2 requests).  No call writes
+// the header except through those words, and every call leaves the counters
+// at zero; each call's own buffers start after it.
+constexpr size_t kCntOff = 256;
+constexpr size_t kHeader = kCntOff + (size_t(128) << 10);
 constexpr int kMaxChunks = 64;
 int g_attn_chunk = 0;  // split-KV chunk override in keys (tests and tuning; 0 = rule)
 constexpr int kAttnRows = 64;
@@ -296,6 +301,8 @@ InjectLayout inject_layout(const dflash_config& c, int max_rows) {
   return L;
 }
 
+// verify workspace: header (error word, completion counters) | argmax
+// partials (8 bytes per row and chunk)
 size_t verify_bytes(int batch, int B, int V) {
   const int rows = batch * B;
   return kHeader + align256((size_t)rows * verify_chunks(rows, V) * 8);
@@ -811,7 +818,8 @@ extern "C" int dflash_verify(const void* target_logits, int logits_dtype,
   const int chunks = verify_chunks(batch * B, V);
   return launch_verify(target_logits, logits_dtype, draft_tokens, batch, B, V, out_tokens,
                        out_len, out_cap, seq_lens, accept_len, next_anchor,
-                       at<void>(ws, kHeader), chunks, err_word(ws), (cudaStream_t)stream);
+                       at<void>(ws, kHeader), chunks, at<unsigned>(ws, kCntOff), err_word(ws),
+                       (cudaStream_t)stream);
 }
 
 // ============================================================== test hooks (dflash_debug.h)

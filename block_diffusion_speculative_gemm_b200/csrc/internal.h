@@ -224,7 +224,7 @@ void launch_draft_finish(const int32_t* tokens, const int32_t* cstep, const int3
 int launch_verify(const void* logits, int dtype, const int32_t* draft, int batch, int B, int V,
                   int32_t* out_tokens, int32_t* out_len, int out_cap, int32_t* seq_lens,
                   int32_t* accept_len, int32_t* next_anchor, void* part, int chunks,
-                  int32_t* err, cudaStream_t s);
+                  unsigned* cnt, int32_t* err, cudaStream_t s);
 int verify_chunks(int rows, int V);
 
 }  // namespace dflash

@@ -1,91 +1,54 @@
 // Greedy verify ("DFlash：用“块扩散”魔法", §2 Flash Verification:
 // decide_acceptance(logits, draft_block), read greedily).
 //
-// Kernel 1 (bandwidth-bound): every target-logit row is cut into chunks; a CTA
-// scans one chunk with 16-byte loads and keeps (max, lowest index).  Kernel 2:
-// one warp per request merges the chunk partials of its B rows (lane i = row
-// i), finds the accept length with one ballot and writes the accepted tokens
-// plus the bonus token behind out_len, then advances out_len and seq_lens.
-// Comparisons are exact on the stored logit values, so the result does not
-// depend on the chunking.
+// One bandwidth-bound kernel.  Every target-logit row is cut into chunks; a
+// CTA scans one chunk with 16-byte streaming loads (four in flight per
+// thread) and keeps (max, lowest index).  It publishes that partial and counts
+// itself in its request's counter; the CTA that completes a request's count
+// merges the request's partials with one warp (lane i = row i, chunks in
+// order), finds the accept length with one ballot and writes the accepted
+// tokens plus the bonus token behind out_len, advances out_len and seq_lens,
+// and sets the counter back to zero.  Comparisons are exact on the stored
+// logit values, so the result does not depend on the chunking or on which
+// CTA finishes last.
 #include "common.cuh"
 #include "internal.h"
 
 namespace dflash {
 
 constexpr int kVerifyThreads = 256;
+constexpr int kVerifyUnroll = 4;
 
 struct ArgPart {
   float v;
   int32_t i;
 };
 
-template <typename T, bool VEC>
-__global__ void __launch_bounds__(kVerifyThreads)
-    verify_argmax_kernel(const T* __restrict__ logits, int V, int chunk, ArgPart* __restrict__ part) {
-  pdl_trigger();
-  pdl_wait();
-  __shared__ float s_v[kVerifyThreads / 32];
-  __shared__ int s_i[kVerifyThreads / 32];
-  const int row = blockIdx.y, c = blockIdx.x;
-  const int v0 = c * chunk;
-  const int v1 = min(V, v0 + chunk);
-  const T* x = logits + (size_t)row * V;
-  float best = -INFINITY;
-  int bi = 0x7fffffff;
-  if (VEC) {
-    constexpr int W = 16 / sizeof(T);  // elements per 16-byte load (chunk is a multiple)
-    const int nvec = (v1 - v0) / W;
-    const uint4* p = reinterpret_cast<const uint4*>(x + v0);
-    for (int t = threadIdx.x; t < nvec; t += kVerifyThreads) {
-      uint4 u = __ldg(p + t);
-      const T* e = reinterpret_cast<const T*>(&u);
-      const int base = v0 + t * W;
+template <typename T>
+__device__ __forceinline__ void scan16(const uint4& u, int base, float& best, int& bi) {
+  constexpr int W = 16 / sizeof(T);
+  const T* e = reinterpret_cast<const T*>(&u);
 #pragma unroll
-      for (int k = 0; k < W; ++k) {
-        const float f = to_f(e[k]);
-        if (f > best) { best = f; bi = base + k; }
-      }
-    }
-    for (int v = v0 + nvec * W + threadIdx.x; v < v1; v += kVerifyThreads) {
-      const float f = to_f(x[v]);
-      if (f > best || (f == best && v < bi)) { best = f; bi = v; }
-    }
-  } else {
-    for (int v = v0 + threadIdx.x; v < v1; v += kVerifyThreads) {
-      const float f = to_f(x[v]);
-      if (f > best) { best = f; bi = v; }
-    }
-  }
-  warp_argmax(best, bi);
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  if (lane == 0) { s_v[w] = best; s_i[w] = bi; }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    best = s_v[0];
-    bi = s_i[0];
-    for (int k = 1; k < kVerifyThreads / 32; ++k) argmax_merge(best, bi, s_v[k], s_i[k]);
-    part[(size_t)row * gridDim.x + c] = ArgPart{best, bi};
+  for (int k = 0; k < W; ++k) {
+    const float f = to_f(e[k]);
+    if (f > best) { best = f; bi = base + k; }
   }
 }
 
-__global__ void verify_accept_kernel(const ArgPart* __restrict__ part, int chunks,
-                                     const int32_t* __restrict__ draft, int batch, int B, int V,
-                                     int32_t* out_tokens, int32_t* out_len, int out_cap,
-                                     int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
-                                     int32_t* err) {
-  pdl_trigger();
-  pdl_wait();
-  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+// Accept step of request r from its B x chunks partials (one warp).
+__device__ void verify_accept(const ArgPart* part, int chunks, int r, const int32_t* draft, int B,
+                              int V, int32_t* out_tokens, int32_t* out_len, int out_cap,
+                              int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
+                              int32_t* err) {
   const int lane = threadIdx.x & 31;
-  if (r >= batch) return;
   int g = 0;
   int d = 0;
   if (lane < B) {
+    // written by other CTAs of this grid: read from L2
     const ArgPart* p = part + (size_t)(r * B + lane) * chunks;
-    float best = p[0].v;
-    int bi = p[0].i;
-    for (int c = 1; c < chunks; ++c) argmax_merge(best, bi, p[c].v, p[c].i);
+    float best = __ldcg(&p[0].v);
+    int bi = __ldcg(&p[0].i);
+    for (int c = 1; c < chunks; ++c) argmax_merge(best, bi, __ldcg(&p[c].v), __ldcg(&p[c].i));
     g = bi;
     d = draft[(size_t)r * B + lane];
   }
@@ -114,6 +77,71 @@ __global__ void verify_accept_kernel(const ArgPart* __restrict__ part, int chunk
   }
 }
 
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kVerifyThreads)
+    verify_kernel(const T* __restrict__ logits, int V, int chunk, int chunks,
+                  ArgPart* __restrict__ part, unsigned* __restrict__ cnt,
+                  const int32_t* __restrict__ draft, int B, int32_t* out_tokens, int32_t* out_len,
+                  int out_cap, int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
+                  int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float s_v[kVerifyThreads / 32];
+  __shared__ int s_i[kVerifyThreads / 32];
+  __shared__ int s_last;
+  const int row = blockIdx.y, c = blockIdx.x;
+  const int v0 = c * chunk;
+  const int v1 = min(V, v0 + chunk);
+  const T* x = logits + (size_t)row * V;
+  float best = -INFINITY;
+  int bi = 0x7fffffff;
+  if (VEC) {
+    constexpr int W = 16 / sizeof(T);  // elements per 16-byte load (chunk is a multiple)
+    const int nvec = (v1 - v0) / W;
+    const uint4* p = reinterpret_cast<const uint4*>(x + v0);
+    int t = threadIdx.x;
+    // each thread visits its elements in increasing index order, so a strict
+    // '>' keeps the lowest index among equal maxima
+    for (; t + (kVerifyUnroll - 1) * kVerifyThreads < nvec; t += kVerifyUnroll * kVerifyThreads) {
+      uint4 u[kVerifyUnroll];
+#pragma unroll
+      for (int j = 0; j < kVerifyUnroll; ++j) u[j] = __ldcs(p + t + j * kVerifyThreads);
+#pragma unroll
+      for (int j = 0; j < kVerifyUnroll; ++j)
+        scan16<T>(u[j], v0 + (t + j * kVerifyThreads) * W, best, bi);
+    }
+    for (; t < nvec; t += kVerifyThreads) scan16<T>(__ldcs(p + t), v0 + t * W, best, bi);
+    for (int v = v0 + nvec * W + threadIdx.x; v < v1; v += kVerifyThreads) {
+      const float f = to_f(x[v]);
+      if (f > best || (f == best && v < bi)) { best = f; bi = v; }
+    }
+  } else {
+    for (int v = v0 + threadIdx.x; v < v1; v += kVerifyThreads) {
+      const float f = to_f(x[v]);
+      if (f > best) { best = f; bi = v; }
+    }
+  }
+  warp_argmax(best, bi);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if (lane == 0) { s_v[w] = best; s_i[w] = bi; }
+  __syncthreads();
+  const int r = row / B;
+  if (threadIdx.x == 0) {
+    best = s_v[0];
+    bi = s_i[0];
+    for (int k = 1; k < kVerifyThreads / 32; ++k) argmax_merge(best, bi, s_v[k], s_i[k]);
+    part[(size_t)row * chunks + c] = ArgPart{best, bi};
+    __threadfence();  // the partial is visible before this CTA is counted
+    s_last = atomicAdd(&cnt[r], 1u) == (unsigned)(B * chunks - 1);
+  }
+  __syncthreads();
+  if (!s_last || threadIdx.x >= 32) return;
+  __threadfence();  // every partial of request r counted before this CTA's reads
+  verify_accept(part, chunks, r, draft, B, V, out_tokens, out_len, out_cap, seq_lens, accept_len,
+                next_anchor, err);
+  if (lane == 0) cnt[r] = 0;  // ready for the next call
+}
+
 int verify_chunks(int rows, int V) {
   // enough CTAs for ~4 per SM, chunks of at least 4096 elements, multiple of 64
   int target = (4 * 148 + rows - 1) / rows;
@@ -125,38 +153,28 @@ int verify_chunks(int rows, int V) {
 int launch_verify(const void* logits, int dtype, const int32_t* draft, int batch, int B, int V,
                   int32_t* out_tokens, int32_t* out_len, int out_cap, int32_t* seq_lens,
                   int32_t* accept_len, int32_t* next_anchor, void* part_v, int chunks,
-                  int32_t* err, cudaStream_t s) {
+                  unsigned* cnt, int32_t* err, cudaStream_t s) {
   const int rows = batch * B;
   ArgPart* part = reinterpret_cast<ArgPart*>(part_v);
   int chunk = (V + chunks - 1) / chunks;
   chunk = (chunk + 63) / 64 * 64;
   const int esz = dtype == DFLASH_BF16 ? 2 : 4;
   const bool vec = ((size_t)V * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(logits) % 16) == 0;
-  dim3 grid(chunks, rows);
-  {
-    TimedScope ts(s, TC_VERIFY);
-    if (dtype == DFLASH_BF16) {
-      const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(logits);
-      if (vec) launch_pdl(verify_argmax_kernel<__nv_bfloat16, true>, dim3(grid),
-          dim3(kVerifyThreads), 0, s, 1, x, V, chunk, part);
-      else launch_pdl(verify_argmax_kernel<__nv_bfloat16, false>, dim3(grid), dim3(kVerifyThreads),
-          0, s, 1, x, V, chunk, part);
-    } else {
-      const float* x = static_cast<const float*>(logits);
-      if (vec) launch_pdl(verify_argmax_kernel<float, true>, dim3(grid), dim3(kVerifyThreads), 0, s,
-          1, x, V, chunk, part);
-      else launch_pdl(verify_argmax_kernel<float, false>, dim3(grid), dim3(kVerifyThreads), 0, s, 1,
-          x, V, chunk, part);
-    }
+  const dim3 grid(chunks, rows), block(kVerifyThreads);
+  TimedScope ts(s, TC_VERIFY);
+  cudaError_t e;
+  if (dtype == DFLASH_BF16) {
+    const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(logits);
+    auto k = vec ? verify_kernel<__nv_bfloat16, true> : verify_kernel<__nv_bfloat16, false>;
+    e = launch_pdl(k, grid, block, 0, s, 1, x, V, chunk, chunks, part, cnt, draft, B, out_tokens,
+                   out_len, out_cap, seq_lens, accept_len, next_anchor, err);
+  } else {
+    const float* x = static_cast<const float*>(logits);
+    auto k = vec ? verify_kernel<float, true> : verify_kernel<float, false>;
+    e = launch_pdl(k, grid, block, 0, s, 1, x, V, chunk, chunks, part, cnt, draft, B, out_tokens,
+                   out_len, out_cap, seq_lens, accept_len, next_anchor, err);
   }
-  {
-    TimedScope ts(s, TC_VERIFY);
-    const int wpb = 4;
-    launch_pdl(verify_accept_kernel, dim3((batch + wpb - 1) / wpb), dim3(32 * wpb), 0, s, 1, part,
-        chunks, draft, batch, B, V, out_tokens, out_len, out_cap, seq_lens, accept_len, next_anchor,
-        err);
-  }
-  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 
 }  // namespace dflash

@@ -5,9 +5,9 @@
 // allocation, or a plugin running inside another framework's allocator), and
 // latency-critical loops avoid cudaMalloc because it may synchronise the
 // device.  Such callers cannot provide the workspace dflash_verify needs.
-// dflash_verify_noalloc runs the same two kernels with their scratch (the
-// per-chunk argmax partials and the device error word) in a fixed array in
-// the library's own device memory.
+// dflash_verify_noalloc runs the same kernel with its scratch (the per-chunk
+// argmax partials, the per-request completion counters and the device error
+// word) in a fixed array in the library's own device memory.
 #include <mutex>
 
 #include "common.cuh"
@@ -17,10 +17,14 @@ namespace dflash {
 namespace {
 
 // Scratch of the no-alloc verify: a 256-byte header (word 0 = device error
-// bits) followed by the argmax partials, 8 bytes each.  Every GPU that loads
-// the library holds this array until the process exits.
+// bits), the argmax partials (8 bytes each), then one completion counter per
+// request.  The counters start at zero (device globals are zero-initialised)
+// and every call leaves them at zero.  Every GPU that loads the library holds
+// this array until the process exits.
 constexpr size_t kNoAllocHeader = 256;
-constexpr size_t kNoAllocBytes = kNoAllocHeader + (size_t(256) << 10);  // 256 KiB of partials
+constexpr size_t kNoAllocPart = size_t(256) << 10;  // 256 KiB of partials: <= 32768 rows
+constexpr size_t kNoAllocCnt = size_t(64) << 10;    // 16384 requests (B >= 2 with <= 32768 rows)
+constexpr size_t kNoAllocBytes = kNoAllocHeader + kNoAllocPart + kNoAllocCnt;
 static __device__ __align__(256) unsigned char g_verify_scratch[kNoAllocBytes];
 
 constexpr int kMaxDevices = 64;
@@ -70,7 +74,8 @@ extern "C" int dflash_verify_noalloc(const void* target_logits, int logits_dtype
   if ((int64_t)batch * B > 65535) return DFLASH_EUNSUPPORTED;
   const int rows = batch * B;
   const int chunks = verify_chunks(rows, V);
-  if ((size_t)rows * chunks * 8 > kNoAllocBytes - kNoAllocHeader) return DFLASH_ESCRATCH;
+  if ((size_t)rows * chunks * 8 > kNoAllocPart || (size_t)batch * 4 > kNoAllocCnt)
+    return DFLASH_ESCRATCH;
   void* scratch = nullptr;
   int st = scratch_address(&scratch);
   if (st != DFLASH_OK) return st;
@@ -78,9 +83,10 @@ extern "C" int dflash_verify_noalloc(const void* target_logits, int logits_dtype
   int32_t* err = static_cast<int32_t*>(scratch);
   // the array keeps the previous call's contents: the error word must start at zero
   if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess) return DFLASH_ECUDA;
+  unsigned char* base = static_cast<unsigned char*>(scratch);
   st = launch_verify(target_logits, logits_dtype, draft_tokens, batch, B, V, out_tokens, out_len,
-                     out_cap, seq_lens, accept_len, next_anchor,
-                     static_cast<unsigned char*>(scratch) + kNoAllocHeader, chunks, err, s);
+                     out_cap, seq_lens, accept_len, next_anchor, base + kNoAllocHeader, chunks,
+                     reinterpret_cast<unsigned*>(base + kNoAllocHeader + kNoAllocPart), err, s);
   if (st != DFLASH_OK) return st;
   if (error_bits) {
     launch_pdl(copy_error_word, dim3(1), dim3(1), 0, s, 1, err, error_bits);

@@ -217,9 +217,10 @@ int dflash_verify(const void* target_logits, int logits_dtype, const int32_t* dr
  * that avoids cudaMalloc because it may synchronise the device.
  *
  * Same arguments, semantics and results as dflash_verify, without ws /
- * ws_bytes.  Its scratch (argmax partials and the device error word) is a
- * fixed array of 256 KiB + 256 bytes in the library's device memory, present on
- * every GPU that loads the library until the process exits.  That bounds a call
+ * ws_bytes.  Its scratch (argmax partials, per-request completion counters
+ * and the device error word) is a fixed array of 320 KiB + 256 bytes in the
+ * library's device memory, present on every GPU that loads the library until
+ * the process exits.  That bounds a call
  * to batch * B <= 32768 rows (8 bytes of partials per row chunk; rows are split
  * into chunks only while batch * B < ~600); larger calls return DFLASH_ESCRATCH
  * before anything is enqueued.

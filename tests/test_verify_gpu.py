@@ -75,6 +75,39 @@ def test_verify_chained_calls_append():
         out, ol, seq = res["out_tokens"], res["out_len"], res["seq_lens"]
 
 
+def test_verify_workspace_reuse_across_batches_and_calls():
+    """One workspace serves verify calls of different batch sizes (each request's
+    chunk CTAs count themselves in a per-request counter that the last of them
+    sets back to zero), with a draft call on the same workspace in between."""
+    V = 151936
+    cfg = synth.get_config("qwen3_8b_bs32")
+    from synth.configs import shrink
+    from tests.gpu_common import built
+    small = shrink(cfg, L=1, V=2048, batch=4, ctx=("fixed", 40), I=512, d=512, H_t=512).replace(
+        name="verify_ws_reuse")
+    bm = built(small)
+    ws = D.new_workspace(max(bm.model.workspace_size(40, 8, 0), D.verify_workspace_size(40, 8, V)))
+    kc, vc = synth.make_kv_cache(small, bm.cap, dtype=bm.model.cache_dtype)
+    kc, vc = kc.cuda(), vc.cuda()
+    for it, (b, B) in enumerate([(40, 8), (3, 8), (40, 4), (1, 8), (40, 8)]):
+        case = synth.make_verify_case(b, B, V, f"reuse{it}", plant=("uniform",), adversarial=True)
+        cap = 2 * B
+        out0 = torch.full((b, cap), -1, dtype=torch.int32)
+        ol0 = torch.zeros(b, dtype=torch.int32)
+        seq0 = torch.full((b,), 77, dtype=torch.int32)
+        res = _run(case["logits"], case["draft"], out0, ol0, seq0, ws=ws)
+        want = O.verify_batch(case["logits"], case["draft"], out0, ol0, cap, seq0)
+        assert res["err"] == 0
+        _compare(res, want)
+        # a draft call between verifies writes its own buffers in the same workspace
+        anchors = torch.arange(small.batch, dtype=torch.int32).cuda()
+        ctx = torch.full((small.batch,), 40, dtype=torch.int32).cuda()
+        out = torch.zeros((small.batch, 8), dtype=torch.int32, device="cuda")
+        D.draft_block(bm.model, anchors, ctx, kc, vc, 8, 1, out, ws)
+        torch.cuda.synchronize()
+        assert D.get_error(ws) == 0
+
+
 @pytest.mark.parametrize("V", [1024, 1001, 7])
 def test_verify_fp32_and_ragged_vocab(V):
     b, B = 3, 4
