@@ -215,10 +215,11 @@ int qkv_out(const dflash_config& c) { return (c.n_q + 2 * c.n_kv) * c.head_dim; 
 
 // ---------------------------------------------------------------- workspace layout
 // Workspace header: word 0 = device error bits.
-// Workspace header: the device error word (byte 0), then one verify
-// completion counter per request (at most 65535 / 2 requests).  No call writes
-// the header except through those words, and every call leaves the counters
-// at zero; each call's own buffers start after it.
+// Workspace header: the device error word (byte 0), then 32768 completion
+// counters: verify uses one per request, the draft attention one per
+// (request, kv head).  No call writes the header except through those words,
+// every call leaves the counters it used at zero (calls sharing a workspace
+// never overlap), and each call's own buffers start after the header.
 constexpr size_t kCntOff = 256;
 constexpr size_t kHeader = kCntOff + (size_t(128) << 10);
 constexpr int kMaxChunks = 64;
@@ -647,15 +648,21 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
   float* part = at<float>(ws, L.part);
   float* attn_o = at<float>(ws, L.attn_o);
   float* attn_ml = at<float>(ws, L.attn_ml);
+  unsigned* attn_cnt = at<unsigned>(ws, kCntOff);  // per (request, kv head), zero between calls
   LmStat* stats = at<LmStat>(ws, L.stats);
   const TC* kc = static_cast<const TC*>(k_cache);
   const TC* vc = static_cast<const TC*>(v_cache);
   const int n_vt = (c.vocab + kTileN - 1) / kTileN;
   const bool bf16 = c.dtype == DFLASH_BF16;
 
-  // split-KV chunk: a multiple of the attention tile (64 keys), at least 512 keys
-  int chunk = (cap + B + kMaxChunks - 1) / kMaxChunks;
-  chunk = std::max(512, (chunk + 63) / 64 * 64);
+  // split-KV chunk: a multiple of the attention tile (64 keys) sized for
+  // about four CTAs per SM over the whole (request, kv head, chunk) grid, at
+  // most 768 keys (each chunk's partial is merged by the last CTA of its
+  // request and head) and at most kMaxChunks chunks per request
+  int chunk = (int)std::min<int64_t>(768, (int64_t)(cap + B) * batch * c.n_kv / (4 * num_sms()));
+  chunk = std::max(64, (chunk + 63) / 64 * 64);
+  chunk = std::max(chunk, (cap + B + kMaxChunks - 1) / kMaxChunks);
+  chunk = (chunk + 63) / 64 * 64;
   if (g_attn_chunk > 0 && (cap + B + g_attn_chunk - 1) / g_attn_chunk <= kMaxChunks)
     chunk = g_attn_chunk;
   const int n_chunks = (cap + B + chunk - 1) / chunk;
@@ -719,7 +726,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
                              m->rope_sin, q, kb, vb, s);
         if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, l, c.n_layers, batch, cap,
                                                 ctx_len, valid, B, nq, nkv, hd, attn_o, attn_ml,
-                                                n_chunks, chunk, o, err, s)))
+                                                n_chunks, chunk, o, attn_cnt, err, s)))
           return st;
         go.f32 = x;
         if ((st = run(P.mo, c.d, nq * hd, o, OP_RESID))) return st;
@@ -739,7 +746,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
                          q, kb, vb, s);
       if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, l, c.n_layers, batch, cap, ctx_len,
                                               valid, B, nq, nkv, hd, attn_o, attn_ml, n_chunks,
-                                              chunk, o, err, s)))
+                                              chunk, o, attn_cnt, err, s)))
         return st;
       if ((st = gemm(P.mo, P.Wo, c.d, nq * hd, o, part, L.part_elems, &sp))) return st;
       launch_residual_norm<T>(part, sp, M, c.d, x, P.g_post, h, nullptr, c.eps, s);
@@ -791,6 +798,7 @@ extern "C" int dflash_draft_block(const dflash_model* m, const int32_t* anchor,
   if (cache_cap > c.max_pos) return DFLASH_EINVAL;
   if (B * (c.n_q / c.n_kv) > kAttnRows) return DFLASH_EUNSUPPORTED;
   if ((size_t)batch * B > 65535) return DFLASH_EUNSUPPORTED;
+  if ((size_t)batch * c.n_kv * 4 > kHeader - kCntOff) return DFLASH_EUNSUPPORTED;
   if (ws_bytes < draft_layout(c, batch, B).end) return DFLASH_EWORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   if (c.dtype == DFLASH_BF16)

@@ -187,14 +187,13 @@ int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, c
                            int layer, int L, int batch, int cap, const int32_t* ctx_len,
                            const int32_t* req_valid, int B, int nq, int nkv, int hd,
                            float* part_o, float* part_ml, int n_chunks, int chunk, T* o,
-                           int32_t* err, cudaStream_t s) {
+                           unsigned* cnt, int32_t* err, cudaStream_t s) {
   if (B * (nq / nkv) > kMaxRows) return DFLASH_EUNSUPPORTED;
   dim3 grid(n_chunks, nkv, batch);
   if constexpr (std::is_same<T, __half>::value) {
-    const int st = launch_attn_partial_tc(q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid,
-                                          B, nq, nkv, hd, L, chunk, n_chunks, part_o, part_ml, err,
-                                          s);
-    if (st != DFLASH_OK) return st;
+    // the tensor-core kernel merges its chunks itself
+    return launch_attn_tc(q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
+                          hd, L, chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
   } else {
     TimedScope ts(s, TC_ATTN);
     if (hd == 128) {
@@ -230,12 +229,12 @@ int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, c
 template int launch_block_attention<float, float>(const float*, const float*, const float*,
                                                   const float*, const float*, int, int, int, int,
                                                   const int32_t*, const int32_t*, int, int, int,
-                                                  int, float*, float*, int, int, float*, int32_t*,
-                                                  cudaStream_t);
+                                                  int, float*, float*, int, int, float*, unsigned*,
+                                                  int32_t*, cudaStream_t);
 template int launch_block_attention<__half, __half>(const __half*, const __half*, const __half*,
                                                     const __half*, const __half*, int, int, int,
                                                     int, const int32_t*, const int32_t*, int, int,
                                                     int, int, float*, float*, int, int, __half*,
-                                                    int32_t*, cudaStream_t);
+                                                    unsigned*, int32_t*, cudaStream_t);
 
 }  // namespace dflash

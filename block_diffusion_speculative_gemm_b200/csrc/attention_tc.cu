@@ -11,7 +11,9 @@
 // kg of every tile: S = Q K^T and O += P V run as fp16 mma.sync.m16n8k16 with
 // fp32 accumulation; the online softmax (row max m, row sum l) is updated once
 // per tile.  Key groups are merged through shared memory and one (m, l, O)
-// partial per query row and chunk is written; a combine kernel merges chunks.
+// partial per query row and chunk is written; the last chunk CTA of each
+// (request, kv head) -- counted on a per-(request, head) counter that it sets
+// back to zero -- merges the chunks into the output rows.
 //
 // Memory-bound: 4 * B * G flop per cache byte read, every cache byte read once.
 #include "common.cuh"
@@ -24,6 +26,7 @@ namespace {
 constexpr int kComputeWarps = 4;
 constexpr int kThreads = 32 * kComputeWarps + 32;  // + one producer warp
 constexpr int kKeys = 64;    // keys per context tile
+constexpr int kMaxChunksTc = 64;  // split-KV chunks per request
 constexpr int kBlkKeys = 16; // rows of the block tile
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
@@ -222,7 +225,8 @@ __global__ void __launch_bounds__(kThreads)
                    const __half* __restrict__ vb, int layer, int batch, int cap,
                    const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ req_valid,
                    int B, int nq, int nkv, int chunk, int n_chunks, float* __restrict__ part_o,
-                   float* __restrict__ part_ml, int32_t* err) {
+                   float* __restrict__ part_ml, unsigned* __restrict__ cnt,
+                   __half* __restrict__ out, int32_t* err) {
   pdl_trigger();
   pdl_wait();
   using LY = Layout<HD, MT>;
@@ -391,71 +395,147 @@ __global__ void __launch_bounds__(kThreads)
     sl[NT * 4 + 3] = l1;
   }
   __syncthreads();
-  if (!computes || kg > 0) return;
+  const size_t pbase = (((size_t)r * nkv + g) * n_chunks + c) * kAttnMaxRows;
+  if (computes && kg == 0) {
 #pragma unroll
-  for (int k = 1; k < KG; ++k) {
-    const float* sl = scratch + ((size_t)(k * MT + mt) * 32 + lane) * kSlot;
-    const float pm0 = sl[NT * 4 + 0], pm1 = sl[NT * 4 + 1];
-    const float nm0 = fmaxf(m0, pm0), nm1 = fmaxf(m1, pm1);
-    const float a0 = m0 == -INFINITY ? 0.f : exp2f(m0 - nm0);
-    const float a1 = m1 == -INFINITY ? 0.f : exp2f(m1 - nm1);
-    const float b0 = pm0 == -INFINITY ? 0.f : exp2f(pm0 - nm0);
-    const float b1 = pm1 == -INFINITY ? 0.f : exp2f(pm1 - nm1);
+    for (int k = 1; k < KG; ++k) {
+      const float* sl = scratch + ((size_t)(k * MT + mt) * 32 + lane) * kSlot;
+      const float pm0 = sl[NT * 4 + 0], pm1 = sl[NT * 4 + 1];
+      const float nm0 = fmaxf(m0, pm0), nm1 = fmaxf(m1, pm1);
+      const float a0 = m0 == -INFINITY ? 0.f : exp2f(m0 - nm0);
+      const float a1 = m1 == -INFINITY ? 0.f : exp2f(m1 - nm1);
+      const float b0 = pm0 == -INFINITY ? 0.f : exp2f(pm0 - nm0);
+      const float b1 = pm1 == -INFINITY ? 0.f : exp2f(pm1 - nm1);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        o[n][0] = o[n][0] * a0 + sl[n * 4 + 0] * b0;
+        o[n][1] = o[n][1] * a0 + sl[n * 4 + 1] * b0;
+        o[n][2] = o[n][2] * a1 + sl[n * 4 + 2] * b1;
+        o[n][3] = o[n][3] * a1 + sl[n * 4 + 3] * b1;
+      }
+      l0 = l0 * a0 + sl[NT * 4 + 2] * b0;
+      l1 = l1 * a1 + sl[NT * 4 + 3] * b1;
+      m0 = nm0;
+      m1 = nm1;
+    }
+    // partial maxima leave in natural-log units of the scaled score
+    const float ln2 = 0.6931471805599453f;
+    m0 *= ln2;
+    m1 *= ln2;
+    const int tq = lane & 3;
+    const int row0 = mt * 16 + (lane >> 2), row1 = row0 + 8;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-      o[n][0] = o[n][0] * a0 + sl[n * 4 + 0] * b0;
-      o[n][1] = o[n][1] * a0 + sl[n * 4 + 1] * b0;
-      o[n][2] = o[n][2] * a1 + sl[n * 4 + 2] * b1;
-      o[n][3] = o[n][3] * a1 + sl[n * 4 + 3] * b1;
+      const int col = n * 8 + 2 * tq;
+      if (row0 < R)
+        *reinterpret_cast<float2*>(part_o + (pbase + row0) * HD + col) =
+            make_float2(o[n][0], o[n][1]);
+      if (row1 < R)
+        *reinterpret_cast<float2*>(part_o + (pbase + row1) * HD + col) =
+            make_float2(o[n][2], o[n][3]);
     }
-    l0 = l0 * a0 + sl[NT * 4 + 2] * b0;
-    l1 = l1 * a1 + sl[NT * 4 + 3] * b1;
-    m0 = nm0;
-    m1 = nm1;
+    if (tq == 0) {
+      if (row0 < R) *reinterpret_cast<float2*>(part_ml + (pbase + row0) * 2) = make_float2(m0, l0);
+      if (row1 < R) *reinterpret_cast<float2*>(part_ml + (pbase + row1) * 2) = make_float2(m1, l1);
+    }
+    __threadfence();  // this chunk's partial is visible before the chunk is counted
   }
-  // partial maxima leave in natural-log units of the scaled score
-  const float ln2 = 0.6931471805599453f;
-  m0 *= ln2;
-  m1 *= ln2;
-  const size_t pbase = (((size_t)r * nkv + g) * n_chunks + c) * kAttnMaxRows;
-  const int tq = lane & 3;
-  const int row0 = mt * 16 + (lane >> 2), row1 = row0 + 8;
+
+  // ---- chunk combine: the last chunk CTA of (request, kv head) merges every
+  // chunk's (m, l, O) into the output rows (o = sum_c w_c O_c, w_c =
+  // exp(m_c - M) / sum_c' exp(m_c' - M) l_c', chunks in order)
+  __shared__ int s_last;
+  const int nvc = min(n_chunks, (Tc + B + chunk - 1) / chunk);  // chunks with keys
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&cnt[r * nkv + g], 1u) == (unsigned)(nvc - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();  // every counted chunk's partial is visible to the reads below
+  const size_t base = ((size_t)r * nkv + g) * n_chunks * kAttnMaxRows;
+  // every chunk's (m, l) of every row, fetched by all threads at once; the
+  // chunk weights then replace the m values in place
+  float* sml = scratch;  // [nvc][kAttnMaxRows][2]
+  static_assert(2 * kMaxChunksTc * kAttnMaxRows * 4 <= kStages * LY::kStage, "combine scratch");
+  for (int idx = tid; idx < nvc * R; idx += kThreads) {
+    const int cc = idx / R, row = idx % R;
+    const float2 ml =
+        __ldcg(reinterpret_cast<const float2*>(part_ml + (base + (size_t)cc * kAttnMaxRows + row) * 2));
+    sml[(cc * kAttnMaxRows + row) * 2] = ml.x;
+    sml[(cc * kAttnMaxRows + row) * 2 + 1] = ml.y;
+  }
+  __syncthreads();
+  for (int row = tid; row < R; row += kThreads) {
+    float M = -INFINITY;
+    for (int cc = 0; cc < nvc; ++cc) M = fmaxf(M, sml[(cc * kAttnMaxRows + row) * 2]);
+    float Lsum = 0.f;
+    for (int cc = 0; cc < nvc; ++cc) {
+      float* e = sml + (cc * kAttnMaxRows + row) * 2;
+      const float w = expf(e[0] - M);
+      e[0] = w;
+      Lsum += w * e[1];
+    }
+    const float inv = 1.f / Lsum;
+    for (int cc = 0; cc < nvc; ++cc) sml[(cc * kAttnMaxRows + row) * 2] *= inv;
+  }
+  __syncthreads();
+  for (int i4 = tid; i4 < R * HD / 4; i4 += kThreads) {
+    const int row = (i4 * 4) / HD, col = (i4 * 4) % HD;
+    const float4* src = reinterpret_cast<const float4*>(part_o + (base + row) * HD + col);
+    const size_t cstride = (size_t)kAttnMaxRows * HD / 4;  // float4s from chunk to chunk
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int cc = 0;
+    for (; cc + 4 <= nvc; cc += 4) {  // four chunk loads in flight, summed in chunk order
+      float4 v[4];
 #pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    const int col = n * 8 + 2 * tq;
-    if (row0 < R)
-      *reinterpret_cast<float2*>(part_o + (pbase + row0) * HD + col) =
-          make_float2(o[n][0], o[n][1]);
-    if (row1 < R)
-      *reinterpret_cast<float2*>(part_o + (pbase + row1) * HD + col) =
-          make_float2(o[n][2], o[n][3]);
+      for (int u = 0; u < 4; ++u) v[u] = __ldcg(src + (size_t)(cc + u) * cstride);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float w = sml[((cc + u) * kAttnMaxRows + row) * 2];
+        acc.x += w * v[u].x;
+        acc.y += w * v[u].y;
+        acc.z += w * v[u].z;
+        acc.w += w * v[u].w;
+      }
+    }
+    for (; cc < nvc; ++cc) {
+      const float4 v = __ldcg(src + (size_t)cc * cstride);
+      const float w = sml[(cc * kAttnMaxRows + row) * 2];
+      acc.x += w * v.x;
+      acc.y += w * v.y;
+      acc.z += w * v.z;
+      acc.w += w * v.w;
+    }
+    __half* dst = out + ((size_t)(r * B + row / G) * nq + g * G + row % G) * HD + col;
+    *reinterpret_cast<__half2*>(dst) = __floats2half2_rn(acc.x, acc.y);
+    *reinterpret_cast<__half2*>(dst + 2) = __floats2half2_rn(acc.z, acc.w);
   }
-  if (tq == 0) {
-    if (row0 < R) *reinterpret_cast<float2*>(part_ml + (pbase + row0) * 2) = make_float2(m0, l0);
-    if (row1 < R) *reinterpret_cast<float2*>(part_ml + (pbase + row1) * 2) = make_float2(m1, l1);
-  }
+  if (tid == 0) cnt[r * nkv + g] = 0;  // ready for the next launch
 }
 
 template <int HD, int MT>
 int launch_cfg(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q, const __half* kb,
                const __half* vb, int layer, int batch, int cap, const int32_t* ctx_len,
                const int32_t* req_valid, int B, int nq, int nkv, int chunk, int n_chunks,
-               float* part_o, float* part_ml, int32_t* err, cudaStream_t s) {
+               float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
+               cudaStream_t s) {
   const int smem = Layout<HD, MT>::kSmem;
   if (cudaFuncSetAttribute(attn_tc_kernel<HD, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess)
     return DFLASH_ECUDA;
   dim3 grid(n_chunks, nkv, batch);
-  launch_pdl(attn_tc_kernel<HD, MT>, dim3(grid), dim3(kThreads), smem, s, 1, tk, tv, q, kb, vb,
-      layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, part_o, part_ml, err);
-  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
+  const cudaError_t e =
+      launch_pdl(attn_tc_kernel<HD, MT>, grid, dim3(kThreads), smem, s, 1, tk, tv, q, kb, vb,
+                 layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, part_o,
+                 part_ml, cnt, o, err);
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 
 template <int HD>
 int launch_hd(const __half* q, const __half* kb, const __half* vb, const __half* kc,
               const __half* vc, int layer, int batch, int cap, const int32_t* ctx_len,
               const int32_t* req_valid, int B, int nq, int nkv, int L, int chunk, int n_chunks,
-              float* part_o, float* part_ml, int32_t* err, cudaStream_t s) {
+              float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
+              cudaStream_t s) {
   CUtensorMap tk, tv;
   const int64_t rows = (int64_t)L * batch * nkv * cap;
   if (!encode_2d(&tk, kc, rows, HD, HD, kKeys, DFLASH_F16) ||
@@ -464,31 +544,32 @@ int launch_hd(const __half* q, const __half* kb, const __half* vb, const __half*
   const int R = B * (nq / nkv);
   if (R <= 16)
     return launch_cfg<HD, 1>(tk, tv, q, kb, vb, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
-                             chunk, n_chunks, part_o, part_ml, err, s);
+                             chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
   if (R <= 32)
     return launch_cfg<HD, 2>(tk, tv, q, kb, vb, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
-                             chunk, n_chunks, part_o, part_ml, err, s);
+                             chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
   return launch_cfg<HD, 4>(tk, tv, q, kb, vb, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
-                           chunk, n_chunks, part_o, part_ml, err, s);
+                           chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
 }
 
 }  // namespace
 
-int launch_attn_partial_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
-                           const __half* vc, int layer, int batch, int cap, const int32_t* ctx_len,
-                           const int32_t* req_valid, int B, int nq, int nkv, int hd, int L,
-                           int chunk, int n_chunks, float* part_o, float* part_ml, int32_t* err,
-                           cudaStream_t s) {
-  if (B * (nq / nkv) > kAttnMaxRows || chunk % kKeys != 0 || B > kBlkKeys)
+int launch_attn_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
+                   const __half* vc, int layer, int batch, int cap, const int32_t* ctx_len,
+                   const int32_t* req_valid, int B, int nq, int nkv, int hd, int L, int chunk,
+                   int n_chunks, float* part_o, float* part_ml, unsigned* cnt, __half* o,
+                   int32_t* err, cudaStream_t s) {
+  if (B * (nq / nkv) > kAttnMaxRows || chunk % kKeys != 0 || B > kBlkKeys ||
+      n_chunks > kMaxChunksTc)
     return DFLASH_EUNSUPPORTED;
   if ((int64_t)L * batch * nkv * cap > 0x7fffffffLL) return DFLASH_EUNSUPPORTED;
   TimedScope ts(s, TC_ATTN);
   if (hd == 128)
     return launch_hd<128>(q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, L,
-                          chunk, n_chunks, part_o, part_ml, err, s);
+                          chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
   if (hd == 64)
     return launch_hd<64>(q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, L,
-                         chunk, n_chunks, part_o, part_ml, err, s);
+                         chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
   return DFLASH_EUNSUPPORTED;
 }
 

@@ -635,7 +635,7 @@ int gemm_effective_splits(int K, int splits) {
   return (nkb + per - 1) / per;
 }
 
-static int num_sms() {
+int num_sms() {
   static int sms[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);

@@ -42,6 +42,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Streaming multiprocessors of the current device (cached per device).
+int num_sms();
+
 // ---------------------------------------------------------------- timing
 enum TimingClass { TC_GEMM = 0, TC_ATTN = 1, TC_ROW = 2, TC_VERIFY = 3, TC_LMHEAD = 4, TC_N = 5 };
 void timing_begin(cudaStream_t s, int cls);
@@ -187,14 +190,17 @@ void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int 
 // ---------------------------------------------------------------- attention
 constexpr int kAttnMaxRows = 64;  // B * (n_q / n_kv) query rows per (request, kv head)
 
-// Split-KV partials of the tensor-core attention (fp16 rows and fp16 cache):
-// part_o [batch][nkv][n_chunks][kAttnMaxRows][hd] fp32, part_ml [...][2] (max, sum).
-// The cache is [L][batch][nkv][cap][hd]; `layer` selects the layer.
-int launch_attn_partial_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
-                           const __half* vc, int layer, int batch, int cap, const int32_t* ctx_len,
-                           const int32_t* req_valid, int B, int nq, int nkv, int hd, int L,
-                           int chunk, int n_chunks, float* part_o, float* part_ml, int32_t* err,
-                           cudaStream_t s);
+// Tensor-core block attention (fp16 rows and fp16 cache) with its chunk
+// combine: split-KV partials part_o [batch][nkv][n_chunks][kAttnMaxRows][hd]
+// fp32 and part_ml [...][2] (max, sum); the last chunk CTA of each (request,
+// kv head), found with cnt[request * nkv + head] (zero before and after the
+// call), merges them into o [batch * B][nq][hd].  The cache is
+// [L][batch][nkv][cap][hd]; `layer` selects the layer.
+int launch_attn_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
+                   const __half* vc, int layer, int batch, int cap, const int32_t* ctx_len,
+                   const int32_t* req_valid, int B, int nq, int nkv, int hd, int L, int chunk,
+                   int n_chunks, float* part_o, float* part_ml, unsigned* cnt, __half* o,
+                   int32_t* err, cudaStream_t s);
 
 // T: type of q, the block's k/v and the output o; TC: K/V cache type.
 template <typename T, typename TC>
@@ -202,7 +208,7 @@ int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, c
                            int layer, int L, int batch, int cap, const int32_t* ctx_len,
                            const int32_t* req_valid, int B, int nq, int nkv, int hd,
                            float* part_o, float* part_ml, int n_chunks, int chunk, T* o,
-                           int32_t* err, cudaStream_t s);
+                           unsigned* cnt, int32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- draft bookkeeping
 void launch_draft_init(const int32_t* anchor, const int32_t* ctx_len, int batch, int B, int V,
