@@ -115,35 +115,47 @@ def gemm_bytes(N, K, M, out_bytes_per_row):
     return N * K * 2 + M * K * 2 + M * out_bytes_per_row
 
 
-def step_algorithmic(cfg, n_inject, ctx_lens):
-    """Algorithmic bytes / flops of one cycle, per kernel class."""
+def step_algorithmic(cfg, n_inject, ctx_lens, peaks):
+    """Algorithmic bytes / flops of one cycle per kernel class, and each class's
+    roofline time `roof_s`: every GEMM takes the longer of its flops at the sustained
+    bf16 tensor peak and its bytes at the HBM peak; attention and verify are bytes at
+    the HBM peak."""
     b, B, L, d = cfg.batch, cfg.B, cfg.L, cfg.d
     M = b * B
     q = cfg.nq * cfg.hd
     kv = cfg.nkv * cfg.hd
     qkv = q + 2 * kv
-    out = {"gemm": {"bytes": 0, "flops": 0, "launches": 0}, "lm_head": {"bytes": 0, "flops": 0},
-           "attention": {"bytes": 0}, "verify": {"bytes": 0}}
-    g = out["gemm"]
+    hbm = peaks["hbm_gbs"] * 1e9
+    tc = (peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]) * 1e12
+    out = {k: {"bytes": 0, "flops": 0, "roof_s": 0.0, "roof_tensor_s": 0.0}
+           for k in ("gemm", "lm_head", "attention", "verify")}
+
+    def gemm(cls, N, K, rows, out_bytes_per_row, times=1):
+        by = gemm_bytes(N, K, rows, out_bytes_per_row)
+        fl = 2 * N * K * rows
+        c = out[cls]
+        c["bytes"] += times * by
+        c["flops"] += times * fl
+        c["roof_s"] += times * max(fl / tc, by / hbm)
+        c["roof_tensor_s"] += times * (fl / tc if fl / tc >= by / hbm else 0.0)
+
     # injection: fc over the concatenated taps, then the layer-batched K/V projection
     for N, K in ((d, cfg.n_tap * cfg.H_t), (L * 2 * kv, d)):
-        g["bytes"] += gemm_bytes(N, K, n_inject, N * 2)
-        g["flops"] += 2 * N * K * n_inject
+        gemm("gemm", N, K, n_inject, N * 2)
     rem = B - 1
+    T = int(ctx_lens.sum())
     for t in range(cfg.steps):
         k = -(-rem // (cfg.steps - t))
         for N, K in ((qkv, d), (d, q), (2 * cfg.I, d), (d, cfg.I)):
-            g["bytes"] += L * gemm_bytes(N, K, M, N * 2)
-            g["flops"] += L * 2 * N * K * M
-        rows = b * rem
+            gemm("gemm", N, K, M, N * 2, times=L)
         n_vt = -(-cfg.V // 128)
-        out["lm_head"]["bytes"] += gemm_bytes(cfg.V, d, rows, n_vt * 16)
-        out["lm_head"]["flops"] += 2 * cfg.V * d * rows
+        gemm("lm_head", cfg.V, d, b * rem, n_vt * 16)
         # attention: context K and V of every layer, plus the block's q/k/v/o rows
-        T = int(ctx_lens.sum())
         out["attention"]["bytes"] += L * (T * kv * 2 * 2 + M * (2 * q + 2 * kv) * 2)
         rem -= k
     out["verify"]["bytes"] = M * cfg.V * 2 + M * 4 * 2
+    for k in ("attention", "verify"):
+        out[k]["roof_s"] = out[k]["bytes"] / hbm
     return out
 
 
@@ -246,33 +258,45 @@ def run_dflash(args, rank, world, local_rank):
 
     # ---- per-class device times (this rank) and the roofline of the dominant class
     peaks = load_peaks()
-    alg = step_algorithmic(cfg, n_s, ctx)
+    alg = step_algorithmic(cfg, n_s, ctx, peaks)
     classes = {}
     for name, key in (("gemm", "gemm"), ("attention", "attention"), ("lm_head", "lm_head"),
                       ("verify", "verify"), ("row", "row")):
         c = per_class.get(key, {"ms": 0.0, "launches": 0})
         classes[name] = {"ms_per_step": c["ms"] / n_cls,
                          "launches_per_step": c["launches"] / n_cls}
+    tc_peak = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
     for name in ("gemm", "attention", "lm_head", "verify"):
         t = classes[name]["ms_per_step"] / 1e3
         if t > 0:
-            classes[name]["algorithmic_GBps"] = alg[name]["bytes"] / t / 1e9
-            classes[name]["frac_hbm"] = classes[name]["algorithmic_GBps"] / peaks["hbm_gbs"]
+            c = classes[name]
+            c["algorithmic_GBps"] = alg[name]["bytes"] / t / 1e9
+            c["frac_hbm"] = c["algorithmic_GBps"] / peaks["hbm_gbs"]
+            if alg[name]["flops"]:
+                c["TFLOPs"] = alg[name]["flops"] / t / 1e12
+                c["frac_tensor_sustained"] = c["TFLOPs"] / tc_peak
+            c["frac_roofline"] = alg[name]["roof_s"] / t
     dom = max(("gemm", "attention", "lm_head", "verify"), key=lambda n: classes[n]["ms_per_step"])
     # kernels launched inside the timed region: every step launches the same list
     launches = sum(int(c["launches"]) for c in per_class.values()) * args.steps // n_cls
     n_dom = per_class[dom]["launches"] / n_cls
     traffic = load_traffic(dom)
-    achieved = classes[dom]["algorithmic_GBps"]
-    roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
-            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "peak_source": peaks["source"],
-            "algorithmic_bytes_per_launch": alg[dom]["bytes"] / max(n_dom, 1),
-            "avg_launch_ms": classes[dom]["ms_per_step"] / max(n_dom, 1),
-            "traffic": traffic}
-    # whole-cycle roofline: every class at HBM speed (all are bandwidth-bound at M <= 256)
-    roof_ms = sum(alg[n]["bytes"] for n in ("gemm", "attention", "lm_head", "verify")) / (
-        peaks["hbm_gbs"] * 1e9) * 1e3
+    common = {"kernel": dom, "peak_source": peaks["source"],
+              "algorithmic_bytes_per_launch": alg[dom]["bytes"] / max(n_dom, 1),
+              "algorithmic_flops_per_launch": alg[dom]["flops"] / max(n_dom, 1),
+              "avg_launch_ms": classes[dom]["ms_per_step"] / max(n_dom, 1), "traffic": traffic}
+    if alg[dom]["roof_tensor_s"] * 2 > alg[dom]["roof_s"]:
+        # mostly compute-bound at the sustained peak (a kernel inside a long step)
+        achieved = classes[dom]["TFLOPs"]
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak,
+                "peak_kind": "bf16 sustained", "unit": "TFLOP/s",
+                "frac": round(achieved / tc_peak, 4), **common}
+    else:
+        achieved = classes[dom]["algorithmic_GBps"]
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), **common}
+    # whole-cycle roofline: the sum of the classes' roofline times
+    roof_ms = sum(alg[n]["roof_s"] for n in ("gemm", "attention", "lm_head", "verify")) * 1e3
     draft_ms = sum(classes[n]["ms_per_step"] for n in ("gemm", "attention", "lm_head", "row"))
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
