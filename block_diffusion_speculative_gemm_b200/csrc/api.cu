@@ -889,6 +889,12 @@ extern "C" int dflash_debug_attn_chunk(int keys) {
   return DFLASH_OK;
 }
 
+extern "C" int dflash_debug_split_weight(float w) {
+  if (!(w >= 0.f && w <= 64.f)) return DFLASH_EINVAL;
+  gemm_set_split_weight(w);
+  return DFLASH_OK;
+}
+
 extern "C" int dflash_debug_gemm_mode(int mode) {
   if (mode < 0 || mode > 2) return DFLASH_EINVAL;
   gemm_set_mode(mode);

@@ -649,8 +649,10 @@ int num_sms() {
 }
 
 static int g_gemm_mode = 0;
+static float g_split_weight = 4.0f;
 
 void gemm_set_mode(int mode) { g_gemm_mode = mode; }
+void gemm_set_split_weight(float w) { g_split_weight = w; }
 
 bool gemm_use_pair(int M, int N) {
   if (g_gemm_mode == 1) return false;
@@ -680,7 +682,7 @@ int gemm_pick_splits(int M, int N, int K, int max_splits) {
     const double eff = (double)units / ((double)per_sm * sms);
     // each split writes (and its consumer reads) one fp32 partial of the
     // output: M*N*4*2 bytes next to the N*K*2 bytes of weights
-    const double score = eff / (1.0 + 4.0 * se * (double)M / K);
+    const double score = eff / (1.0 + g_split_weight * se * (double)M / K);
     if (score > best_score + 1e-9) {
       best_score = score;
       best = se;

@@ -137,6 +137,8 @@ bool set_tiled_weights(WeightMap& w, const void* tiled);
 // (0 automatic, 1 single CTAs, 2 pairs) replaces the rule when non-zero.
 bool gemm_use_pair(int M, int N);
 void gemm_set_mode(int mode);
+// Weight of the split partials' traffic in the split picker (default 4).
+void gemm_set_split_weight(float w);
 
 // Writes the pre-tiled streaming image of a row-major 16-bit W [N, K] (K % 64
 // == 0) into dst (ceil(N/128) * K/64 * 16384 bytes; rows past N are zero).

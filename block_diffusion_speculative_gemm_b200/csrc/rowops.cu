@@ -19,12 +19,32 @@ __device__ __forceinline__ float sum_splits(const float* part, int splits, size_
 }
 
 // Sum of the K-split partials of 4 consecutive fp32 elements (16-byte aligned
-// index), in ascending split order.  Partials are dead after this read.
+// index), in ascending split order.  Partials are dead after this read.  Up to
+// four splits, every load is issued before the first add, so a thread waits
+// for one memory round trip instead of one per split.
 __device__ __forceinline__ float4 sum_splits4(const float* part, int splits, size_t stride,
                                               size_t idx) {
-  float4 v = __ldcs(reinterpret_cast<const float4*>(part + idx));
+  const float4* p = reinterpret_cast<const float4*>(part + idx);
+  const size_t st4 = stride / 4;
+  if (splits <= 4) {
+    float4 w[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+      if (s < splits) w[s] = __ldcs(p + s * st4);
+    float4 v = w[0];
+#pragma unroll
+    for (int s = 1; s < 4; ++s)
+      if (s < splits) {
+        v.x += w[s].x;
+        v.y += w[s].y;
+        v.z += w[s].z;
+        v.w += w[s].w;
+      }
+    return v;
+  }
+  float4 v = __ldcs(p);
   for (int s = 1; s < splits; ++s) {
-    const float4 w = __ldcs(reinterpret_cast<const float4*>(part + (size_t)s * stride + idx));
+    const float4 w = __ldcs(p + s * st4);
     v.x += w.x;
     v.y += w.y;
     v.z += w.z;

@@ -93,6 +93,7 @@ def lib() -> ctypes.CDLL:
         L.dflash_debug_lmhead_tiled.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp, vp, vp]
         L.dflash_debug_gemm_mode.argtypes = [i32]
         L.dflash_debug_attn_chunk.argtypes = [i32]
+        L.dflash_debug_split_weight.argtypes = [ctypes.c_float]
         _lib = L
     return _lib
 

@@ -55,6 +55,12 @@ int dflash_debug_lmhead_tiled(const void* W_tiled, int N, int K, const void* X, 
  * DFLASH_EINVAL for any other value.  Not thread-safe; tests only. */
 int dflash_debug_gemm_mode(int mode);
 
+/* Weight w of the split partials' traffic in the K-split picker of the draft
+ * and injection GEMMs, process-wide (default 4): a split count s scores
+ * balance / (1 + w * s * M / K).  Returns DFLASH_EINVAL outside [0, 64].  Not
+ * thread-safe; tests and tuning only. */
+int dflash_debug_split_weight(float w);
+
 /* Split-KV chunk of the draft attention, in keys, for every later
  * dflash_draft_block call, process-wide: 0 = the library's rule (at least 512
  * keys, at most 64 chunks per request), else a multiple of 64 that is used
