@@ -65,28 +65,48 @@ class ClockSampler:
         self.idx = device_index
         self.period = period_ms
         self.proc = None
+        self.samples = []  # (arrival time, csv line)
         self.lines = []
+        self.thread = None
+        self.t0 = self.t1 = 0.0
+
+    def _read(self):
+        for line in self.proc.stdout:
+            if line.strip():
+                self.samples.append((time.monotonic(), line))
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
                  f"-lms={self.period}"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            # the timed region starts once the sampler is producing samples
+            deadline = time.monotonic() + 3.0
+            while not self.samples and time.monotonic() < deadline:
+                time.sleep(0.01)
         except OSError:
             self.proc = None
-        time.sleep(0.3)
+        self.t0 = time.monotonic()
         return self
 
     def __exit__(self, *a):
+        self.t1 = time.monotonic()
         if self.proc is not None:
-            time.sleep(0.1)
+            time.sleep(self.period / 1000.0 + 0.05)
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+                self.proc.wait()
+            if self.thread is not None:
+                self.thread.join(timeout=5)
+            # samples taken while the timed region ran
+            self.lines = [l for t, l in self.samples
+                          if self.t0 <= t <= self.t1 + self.period / 1000.0]
 
     def summary(self):
         sm, mx, reasons = [], None, set()
@@ -105,7 +125,6 @@ class ClockSampler:
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        # samples under load: the upper half of the observed clocks
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
 
@@ -201,7 +220,9 @@ def run_dflash(args, rank, world, local_rank):
     # target logits whose greedy argmax agrees with the drafted block on a planted prefix
     case = synth.make_verify_case(b, B, V, "bench", plant=cfg.plant, draft=draft.cpu())
     logits = case["logits"].to(dev)
-    steps_total = args.warmup + args.steps + 4
+    # every verify call appends up to B tokens per request: warm-up, timed and
+    # per-class timing steps
+    steps_total = args.warmup + args.steps + min(args.steps, 20) + 4
     out_cap = steps_total * B
     out_tok = torch.zeros((b, out_cap), dtype=torch.int32, device=dev)
     out_len = torch.zeros(b, dtype=torch.int32, device=dev)
@@ -351,18 +372,52 @@ def run_e2e(args, D, model, cfg, taps_s, cu_s, st_s, anchors, ctx, case, kc, vc,
         v.numel() * 4 for v in h_small.values()) + h_logits.numel() * 2
     d2h = sum(v.numel() * 4 for v in h_res.values())
 
-    def step():
+    # The target logits are needed only by verify: they cross PCIe on a side stream
+    # while injection and drafting run.  Host-to-device copies share one copy
+    # engine, so the inputs that injection needs first go before them; the logits
+    # copy is ordered after those on the main stream, inside the timed region.
+    copy_stream = torch.cuda.Stream(device=dev)
+    ev_start, ev_logits = torch.cuda.Event(), torch.cuda.Event()
+
+    def body():
+        main = torch.cuda.current_stream()
         for h, d in zip(h_taps, d_taps):
             d.copy_(h, non_blocking=True)
         for k in h_small:
             d_small[k].copy_(h_small[k], non_blocking=True)
-        d_logits.copy_(h_logits, non_blocking=True)
+        ev_start.record(main)
+        copy_stream.wait_event(ev_start)
+        with torch.cuda.stream(copy_stream):
+            d_logits.copy_(h_logits, non_blocking=True)
+            ev_logits.record(copy_stream)
         seq.copy_(d_small["ctx"])
         D.inject_kv(model, d_taps, d_small["cu"], d_small["st"], kc, vc, ws)
         D.draft_block(model, d_small["anchor"], d_small["ctx"], kc, vc, B, cfg.steps, draft, ws)
+        main.wait_event(ev_logits)
         D.verify(d_logits, draft, out_tok, out_len, seq, acc, nxt, ws)
         for k, d in (("draft", draft), ("acc", acc), ("nxt", nxt), ("out_len", out_len)):
             h_res[k].copy_(d, non_blocking=True)
+
+    # One step's API calls (copies in, inject, draft, verify, read-back) are captured
+    # once into a CUDA graph and replayed every step, as a serving loop would; each
+    # step still waits for its results on the host.
+    graph = None
+    try:
+        body()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            body()
+        graph = g
+    except Exception as e:  # capture unsupported here: launch eagerly
+        print(f"[bench] e2e graph capture failed ({e}); launching eagerly", file=sys.stderr)
+        torch.cuda.synchronize()
+
+    def step():
+        if graph is not None:
+            graph.replay()
+        else:
+            body()
         torch.cuda.current_stream().synchronize()
 
     out_len.zero_()
@@ -385,7 +440,8 @@ def run_e2e(args, D, model, cfg, taps_s, cu_s, st_s, anchors, ctx, case, kc, vc,
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
     return {"value": round(b * B * world / (ms / steps / 1e3), 1), "unit": UNIT,
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "launch": "cuda graph replay" if graph is not None else "eager"}
 
 
 def load_traffic(kernel_class):
