@@ -548,6 +548,68 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ main
 
+def gemm_report():
+    """Context for the projection GEMMs: the library's tcgen05 GEMM (through its test
+    hook, with the split count and launch mode the draft path picks) next to
+    torch.matmul (cuBLAS, not on the hot path) on the same fp16 shapes, one JSON line
+    per shape. Each call runs on a freshly flushed L2; median of 15 calls."""
+    import ctypes
+    from block_diffusion_speculative_gemm_b200 import dflash as D
+
+    dev = torch.device("cuda")
+    cfg = synth.get_config(WORKLOAD)
+    d, I, kv = cfg.d, cfg.I, cfg.nkv * cfg.hd
+    qkv = cfg.nq * cfg.hd + 2 * kv
+    M, n_inj = cfg.batch * cfg.B, 154
+    shapes = [("qkv", qkv, d, M), ("o", d, cfg.nq * cfg.hd, M), ("gate_up", 2 * I, d, M),
+              ("down", d, I, M), ("inject_fc", d, cfg.n_tap * cfg.H_t, n_inj),
+              ("inject_kv", cfg.L * 2 * kv, d, n_inj)]
+    L = D.lib()
+    err = D.new_workspace(256)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream().cuda_stream
+
+    def median_ms(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(15):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    for name, N, K, Mr in shapes:
+        W = (torch.randn(N, K, device=dev) * 0.02).half()
+        X = torch.randn(Mr, K, device=dev).half()
+        Wt = D.debug_tile_weights(W)
+        splits = L.dflash_debug_pick_splits(Mr, N, K)
+        out = torch.empty(splits * Mr * N, device=dev)
+        used = ctypes.c_int(0)
+
+        def ours():
+            r = L.dflash_debug_gemm_tiled(ctypes.c_void_p(Wt.data_ptr()), N, K,
+                                          ctypes.c_void_p(X.data_ptr()), Mr, D.F16, splits,
+                                          ctypes.c_void_p(out.data_ptr()), ctypes.byref(used),
+                                          ctypes.c_void_p(err.data_ptr()), ctypes.c_void_p(st))
+            assert r == 0, r
+
+        t_ours = median_ms(ours)
+        t_cublas = median_ms(lambda: torch.matmul(X, W.t()))
+        print(json.dumps({"gemm": name, "N": N, "K": K, "M": Mr, "splits": splits,
+                          "tcgen05_us": round(t_ours * 1e3, 1),
+                          "cublas_us": round(t_cublas * 1e3, 1),
+                          "tcgen05_TFLOPs": round(2 * Mr * N * K / t_ours / 1e9, 1),
+                          "tcgen05_weight_GBps": round(N * K * 2 / t_ours / 1e6)}), flush=True)
+        del W, Wt, X, out
+    assert D.get_error(err) == 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -558,7 +620,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling only: override the draft layer count")
+    ap.add_argument("--gemm-report", action="store_true",
+                    help="context only: time the projection GEMMs against torch.matmul")
     args = ap.parse_args()
+    if args.gemm_report:
+        gemm_report()
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -883,6 +883,11 @@ extern "C" int dflash_debug_tile_weights(const void* W, void* Wt, int N, int K, 
   return cuda_status();
 }
 
+extern "C" int dflash_debug_pick_splits(int M, int N, int K) {
+  if (M < 1 || N < 1 || K < 64 || K % 64) return DFLASH_EINVAL;
+  return gemm_pick_splits(M, N, K, kMaxSplits);
+}
+
 extern "C" int dflash_debug_attn_chunk(int keys) {
   if (keys < 0 || keys % 64 != 0) return DFLASH_EINVAL;
   g_attn_chunk = keys;

@@ -54,11 +54,14 @@ _lib = None
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
+        # DFLASH_LIB names another build of the same library (e.g. one built out
+        # of tree); there is no fallback when the file is missing
+        path = os.environ.get("DFLASH_LIB") or LIB_PATH
+        if not os.path.exists(path):
             raise RuntimeError(
-                f"{LIB_PATH} is missing: build it with "
+                f"{path} is missing: build it with "
                 "`python -m block_diffusion_speculative_gemm_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
+        L = ctypes.CDLL(path)
         vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         L.dflash_model_create.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Weights),
                                           ctypes.POINTER(vp)]
@@ -93,6 +96,7 @@ def lib() -> ctypes.CDLL:
         L.dflash_debug_lmhead_tiled.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp, vp, vp]
         L.dflash_debug_gemm_mode.argtypes = [i32]
         L.dflash_debug_attn_chunk.argtypes = [i32]
+        L.dflash_debug_pick_splits.argtypes = [i32, i32, i32]
         L.dflash_debug_split_weight.argtypes = [ctypes.c_float]
         _lib = L
     return _lib

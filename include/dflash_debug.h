@@ -55,6 +55,10 @@ int dflash_debug_lmhead_tiled(const void* W_tiled, int N, int K, const void* X, 
  * DFLASH_EINVAL for any other value.  Not thread-safe; tests only. */
 int dflash_debug_gemm_mode(int mode);
 
+/* The K split count the draft and injection paths pick for an M x N x K
+ * weight-streaming GEMM (before any workspace limit), or DFLASH_EINVAL. */
+int dflash_debug_pick_splits(int M, int N, int K);
+
 /* Weight w of the split partials' traffic in the K-split picker of the draft
  * and injection GEMMs, process-wide (default 4): a split count s scores
  * balance / (1 + w * s * M / K).  Returns DFLASH_EINVAL outside [0, 64].  Not
