@@ -206,9 +206,18 @@ def run_dflash(args, rank, world, local_rank):
     cu_p_d = cu_p.to(dev)
     taps_p = [(torch.randn((n_p, cfg.H_t), generator=gen, device=dev) * cfg.h_std).to(torch.bfloat16)
               for _ in range(cfg.n_tap)]
-    D.inject_kv(model, taps_p, cu_p_d, st_p.to(dev), kc, vc, ws)
-    del taps_p
+    st_p_d = st_p.to(dev)
+    D.inject_kv(model, taps_p, cu_p_d, st_p_d, kc, vc, ws)
     torch.cuda.synchronize()
+    # the prefill injection once more, timed: it rewrites the same cache rows, and at
+    # tens of thousands of rows its GEMMs are the tensor-bound part of the path
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record()
+    D.inject_kv(model, taps_p, cu_p_d, st_p_d, kc, vc, ws)
+    p1.record()
+    torch.cuda.synchronize()
+    prefill_ms = p0.elapsed_time(p1)
+    del taps_p
     assert D.get_error(ws) == 0
 
     taps_s = [t.to(dev) for t in synth.make_tap_hiddens(cfg, n_s, label="taps_steady")]
@@ -255,6 +264,17 @@ def run_dflash(args, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
     ms = e0.elapsed_time(e1)
+    # dflash_draft_block alone (all denoising steps), back to back
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_draft = args.steps
+    for _ in range(3):  # the clocks settle after the sampler's pause
+        D.draft_block(model, anchors_d, ctx_d, kc, vc, B, cfg.steps, draft, ws)
+    d0.record(stream)
+    for _ in range(n_draft):
+        D.draft_block(model, anchors_d, ctx_d, kc, vc, B, cfg.steps, draft, ws)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    draft_ms = d0.elapsed_time(d1) / n_draft
     # per-class device times from separate steps: the events recorded around each
     # class serialise the kernels they bracket, so they stay out of the timed region
     n_cls = min(args.steps, 20)
@@ -335,6 +355,11 @@ def run_dflash(args, rank, world, local_rank):
         "gpu_launches": launches,
         "verify_rows_s": round(b * B / (classes["verify"]["ms_per_step"] / 1e3), 1)
         if classes["verify"]["ms_per_step"] > 0 else None,
+        # dflash_draft_block alone: block positions and drafted (masked) positions per s
+        "draft_block": {"ms": round(draft_ms, 4),
+                        "block_tok_s": round(b * world * B / (draft_ms / 1e3), 1),
+                        "drafted_tok_s": round(b * world * (B - 1) / (draft_ms / 1e3), 1)},
+        "prefill_inject": prefill_report(cfg, n_p, prefill_ms, peaks),
         "clocks": clk.summary(),
     }
     if rank == 0 and not args.no_e2e:
@@ -547,6 +572,18 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ main
+
+def prefill_report(cfg, n_rows, ms, peaks):
+    """The timed prefill injection (every context position of every request): its two
+    GEMMs (fc over the concatenated taps, the layer-batched K/V projection) dominate
+    and are tensor-bound at this many rows."""
+    kv = cfg.nkv * cfg.hd
+    flops = 2 * n_rows * (cfg.d * cfg.n_tap * cfg.H_t + cfg.L * 2 * kv * cfg.d)
+    tf = flops / (ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
+    return {"rows": int(n_rows), "ms": round(ms, 3), "TFLOPs": round(tf, 1),
+            "frac_tensor_sustained": round(tf / peak, 4)}
+
 
 def gemm_report():
     """Context for the projection GEMMs: the library's tcgen05 GEMM (through its test

@@ -658,10 +658,12 @@ bool gemm_use_pair(int M, int N) {
   if (g_gemm_mode == 1) return false;
   if (g_gemm_mode == 2) return true;
   // a pair halves the token bytes each SM stages and reads per weight byte;
-  // measured on B200 it pays only for a large token tile against a wide weight
+  // measured on B200 it pays for a large token tile against a wide weight
   // (SwiGLU gate/up and LM head at 224-256 tokens), where the coarser 256-row
-  // work units still balance across the SM pairs
-  return M > 160 && N >= 16384;
+  // work units still balance across the SM pairs, and for the tensor-bound
+  // GEMMs of thousands of token rows (prefill injection: 66% of the sustained
+  // bf16 peak with pairs, 63% without)
+  return (M > 160 && N >= 16384) || M >= 1024;
 }
 
 int gemm_pick_splits(int M, int N, int K, int max_splits) {
