@@ -6,7 +6,9 @@
 // ("DFlash + Spec V2 深度解析", §2.3: the whole block is predicted in one
 // forward).  The key axis is cut into chunks; each CTA (request, kv head,
 // chunk) produces an online-softmax partial (row max m, row sum l, unnormalised
-// o), and a combine kernel merges the chunks in ascending order.
+// o), merged over the chunks in ascending order.  fp16 models run the
+// tensor-core kernel of attention_tc.cu, which merges its chunks itself; fp32
+// models run the SIMT kernel below and the combine kernel after it.
 #include <type_traits>
 
 #include "common.cuh"
@@ -195,24 +197,24 @@ int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, c
     return launch_attn_tc(q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
                           hd, L, chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
   } else {
-    TimedScope ts(s, TC_ATTN);
-    if (hd == 128) {
-      const size_t sm = (kMaxRows * 128 + kKeyTile * 129 + kKeyTile * 128) * sizeof(float);
-      cudaFuncSetAttribute(attn_partial_kernel<T, TC, 128>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-      launch_pdl(attn_partial_kernel<T, TC, 128>, dim3(grid), dim3(kAttnThreads), sm, s, 1, q, kb,
-          vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, part_o,
-          part_ml);
-    } else if (hd == 64) {
-      const size_t sm = (kMaxRows * 64 + kKeyTile * 65 + kKeyTile * 64) * sizeof(float);
-      launch_pdl(attn_partial_kernel<T, TC, 64>, dim3(grid), dim3(kAttnThreads), sm, s, 1, q, kb,
-          vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, part_o,
-          part_ml);
-    } else {
-      return DFLASH_EUNSUPPORTED;
+    {
+      TimedScope ts(s, TC_ATTN);
+      if (hd == 128) {
+        const size_t sm = (kMaxRows * 128 + kKeyTile * 129 + kKeyTile * 128) * sizeof(float);
+        cudaFuncSetAttribute(attn_partial_kernel<T, TC, 128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        launch_pdl(attn_partial_kernel<T, TC, 128>, dim3(grid), dim3(kAttnThreads), sm, s, 1, q,
+            kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks,
+            part_o, part_ml);
+      } else if (hd == 64) {
+        const size_t sm = (kMaxRows * 64 + kKeyTile * 65 + kKeyTile * 64) * sizeof(float);
+        launch_pdl(attn_partial_kernel<T, TC, 64>, dim3(grid), dim3(kAttnThreads), sm, s, 1, q,
+            kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks,
+            part_o, part_ml);
+      } else {
+        return DFLASH_EUNSUPPORTED;
+      }
     }
-  }
-  {
     TimedScope ts(s, TC_ATTN);
     if (n_chunks > kMaxChunksC) return DFLASH_EUNSUPPORTED;
     dim3 g2(nkv, batch);
@@ -222,8 +224,8 @@ int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, c
     else
       launch_pdl(attn_combine_kernel<T, 64>, dim3(g2), dim3(kCombineThreads), 0, s, 1, part_o,
           part_ml, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, o);
+    return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
   }
-  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 
 template int launch_block_attention<float, float>(const float*, const float*, const float*,
