@@ -43,6 +43,21 @@ UNIT = "block tok/s"
 
 # ------------------------------------------------------------------ helpers
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of every rank's value (a device time): the job is as slow as its
+    slowest replica."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(per_rank_units: int, world: int, ms_per_step: float) -> float:
+    """Whole-job units per second: every rank processes its own units each step."""
+    return per_rank_units * world / (ms_per_step / 1e3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -288,14 +303,8 @@ def run_dflash(args, rank, world, local_rank):
     err = D.get_error(ws)
     if err:
         raise RuntimeError(f"device error word {err}")
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t.item())
-    ms_step = ms_max / args.steps
-    tokens = b * B * world
-    value = tokens / (ms_step / 1e3)
+    ms_step = max_over_ranks(ms, world, dev) / args.steps
+    value = job_throughput(b * B, world, ms_step)
 
     # ---- per-class device times (this rank) and the roofline of the dominant class
     peaks = load_peaks()
@@ -459,12 +468,8 @@ def run_e2e(args, D, model, cfg, taps_s, cu_s, st_s, anchors, ctx, case, kc, vc,
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": round(b * B * world / (ms / steps / 1e3), 1), "unit": UNIT,
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return {"value": round(job_throughput(b * B, world, ms / steps), 1), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "launch": "cuda graph replay" if graph is not None else "eager"}
 
