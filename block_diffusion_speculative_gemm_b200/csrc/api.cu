@@ -883,6 +883,26 @@ extern "C" int dflash_debug_tile_weights(const void* W, void* Wt, int N, int K, 
   return cuda_status();
 }
 
+namespace {
+// One thread waits, through the library's bounded mbarrier wait, for a phase
+// that no arrival ever completes: after the wait limit it gives up and sets
+// DFLASH_DEV_TIMEOUT, as every pipeline wait of the library does.
+__global__ void debug_timeout_kernel(int32_t* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+    if (!mbar_wait(smem_u32(&bar), 0)) set_error(err, DFLASH_DEV_TIMEOUT);
+  }
+}
+}  // namespace
+
+extern "C" int dflash_debug_wait_timeout(void* err_ws, void* stream) {
+  if (!err_ws || (reinterpret_cast<uintptr_t>(err_ws) & 255)) return DFLASH_EINVAL;
+  debug_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(err_word(err_ws));
+  return cuda_status();
+}
+
 extern "C" int dflash_debug_pick_splits(int M, int N, int K) {
   if (M < 1 || N < 1 || K < 64 || K % 64) return DFLASH_EINVAL;
   return gemm_pick_splits(M, N, K, kMaxSplits);

@@ -97,6 +97,7 @@ def lib() -> ctypes.CDLL:
         L.dflash_debug_gemm_mode.argtypes = [i32]
         L.dflash_debug_attn_chunk.argtypes = [i32]
         L.dflash_debug_pick_splits.argtypes = [i32, i32, i32]
+        L.dflash_debug_wait_timeout.argtypes = [vp, vp]
         L.dflash_debug_split_weight.argtypes = [ctypes.c_float]
         _lib = L
     return _lib

@@ -55,6 +55,13 @@ int dflash_debug_lmhead_tiled(const void* W_tiled, int N, int K, const void* X, 
  * DFLASH_EINVAL for any other value.  Not thread-safe; tests only. */
 int dflash_debug_gemm_mode(int mode);
 
+/* Failure-detection check: launches one thread that waits, with the
+ * library's bounded pipeline wait, on an mbarrier phase nothing completes.
+ * After the wait limit (1 s) the kernel sets DFLASH_DEV_TIMEOUT in the error
+ * word of err_ws (a 256-byte aligned workspace) and returns; the context stays
+ * usable.  No fault and no trap. */
+int dflash_debug_wait_timeout(void* err_ws, void* stream);
+
 /* The K split count the draft and injection paths pick for an M x N x K
  * weight-streaming GEMM (before any workspace limit), or DFLASH_EINVAL. */
 int dflash_debug_pick_splits(int M, int N, int K);
