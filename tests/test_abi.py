@@ -39,6 +39,9 @@ def test_model_create_rejects_null_and_bad_config():
     assert L.dflash_model_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)) == D.EINVAL
     cfg.n_q, cfg.n_kv, cfg.head_dim = 2, 1, 96  # head_dim 96 not built
     assert L.dflash_model_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)) == D.EUNSUPPORTED
+    cfg.head_dim, cfg.d = 64, 4160  # rows wider than the row kernels hold (d <= 4096)
+    assert L.dflash_model_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)) == D.EINVAL
+    cfg.d = 64
     assert h.value is None
     assert L.dflash_model_destroy(None) == D.OK
 
