@@ -11,13 +11,6 @@ namespace dflash {
 constexpr int kRowThreads = 256;
 constexpr int kMaxRowElems = 16;  // d <= 4096 per 256 threads
 
-__device__ __forceinline__ float sum_splits(const float* part, int splits, size_t stride,
-                                            size_t idx) {
-  float v = part[idx];
-  for (int s = 1; s < splits; ++s) v += part[(size_t)s * stride + idx];
-  return v;
-}
-
 // Sum of the K-split partials of 4 consecutive fp32 elements (16-byte aligned
 // index), in ascending split order.  Partials are dead after this read.  Up to
 // four splits, every load is issued before the first add, so a thread waits
