@@ -13,7 +13,6 @@ Tolerances (the draft-path rules for bf16 storage with fp32 accumulation):
   * verify: bit-exact.
 """
 
-import math
 
 import numpy as np
 import torch

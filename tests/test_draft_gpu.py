@@ -7,7 +7,6 @@ Draft tokens must equal the oracle's argmax except at near-ties (top-2 margin
 commit sets must be admitted by the oracle (see tests/gpu_common.py).
 """
 
-import numpy as np
 import pytest
 import torch
 

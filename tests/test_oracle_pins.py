@@ -5,7 +5,6 @@ a closed-form value, a mathematical invariant, an independent library routine
 (scipy's softmax) or the loop-based restatement in ``tests/bruteforce.py``.
 """
 
-import itertools
 import math
 
 import numpy as np
