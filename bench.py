@@ -652,6 +652,76 @@ def gemm_report():
     assert D.get_error(err) == 0
 
 
+def graph_report():
+    """One cycle (steady-state injection, the 2-step draft, verify) launched call by
+    call versus replayed from a CUDA graph captured once, every cycle followed by a
+    host wait for its results (as a serving loop reading its accepted tokens would),
+    at batch 1, 8 and 32 of the 8B-shaped workload. One JSON line per batch."""
+    from block_diffusion_speculative_gemm_b200 import dflash as D
+
+    dev = torch.device("cuda")
+    base = synth.get_config(WORKLOAD)
+    B, V = base.B, base.V
+    model = D.Model(base, to_device(synth.make_weights(base), dev),
+                    base.cache_cap + 2 * B + 16)
+    n = 50
+    stream = torch.cuda.current_stream()
+    for batch in (1, 8, 32):
+        cfg = base.replace(batch=batch)
+        ctx = synth.make_ctx_lens(cfg)
+        anchors = synth.make_anchors(cfg).to(dev)
+        cap = cfg.cache_cap
+        kc = torch.zeros((cfg.L, batch, cfg.nkv, cap, cfg.hd), dtype=model.cache_dtype,
+                         device=dev)
+        vc = torch.zeros_like(kc)
+        cu, st, n_rows = synth.make_inject_layout(cfg, ctx, "steady")
+        taps = [t.to(dev) for t in synth.make_tap_hiddens(cfg, n_rows, label="graph_taps")]
+        logits = synth.make_verify_case(batch, B, V, "graph", plant=cfg.plant)["logits"].to(dev)
+        ws = D.new_workspace(max(model.workspace_size(batch, B, n_rows),
+                                 D.verify_workspace_size(batch, B, V)))
+        cu_d, st_d, ctx_d = cu.to(dev), st.to(dev), ctx.to(dev)
+        draft = torch.zeros((batch, B), dtype=torch.int32, device=dev)
+        out_tok = torch.zeros((batch, (2 * n + 16) * B), dtype=torch.int32, device=dev)
+        out_len = torch.zeros(batch, dtype=torch.int32, device=dev)
+        seq = torch.zeros(batch, dtype=torch.int32, device=dev)
+        acc = torch.zeros(batch, dtype=torch.int32, device=dev)
+        nxt = torch.zeros(batch, dtype=torch.int32, device=dev)
+
+        def cycle():
+            D.inject_kv(model, taps, cu_d, st_d, kc, vc, ws)
+            D.draft_block(model, anchors, ctx_d, kc, vc, B, cfg.steps, draft, ws)
+            D.verify(logits, draft, out_tok, out_len, seq, acc, nxt, ws)
+
+        def timed(fn):
+            for _ in range(3):
+                fn()
+                stream.synchronize()
+            out_len.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                fn()
+                stream.synchronize()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            out_len.zero_()
+            return e0.elapsed_time(e1) / n
+
+        eager_ms = timed(cycle)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            cycle()
+        graph_ms = timed(g.replay)
+        assert D.get_error(ws) == 0
+        print(json.dumps({"batch": batch, "block": B, "cycles": n,
+                          "eager_ms_per_cycle": round(eager_ms, 4),
+                          "graph_ms_per_cycle": round(graph_ms, 4),
+                          "saving_ms": round(eager_ms - graph_ms, 4),
+                          "graph_block_tok_s": round(batch * B / (graph_ms / 1e3), 1)}), flush=True)
+        del kc, vc, ws, g
+    model.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -664,9 +734,14 @@ def main():
                     help="profiling only: override the draft layer count")
     ap.add_argument("--gemm-report", action="store_true",
                     help="context only: time the projection GEMMs against torch.matmul")
+    ap.add_argument("--graph-report", action="store_true",
+                    help="cycles launched call by call versus replayed from a CUDA graph")
     args = ap.parse_args()
     if args.gemm_report:
         gemm_report()
+        return
+    if args.graph_report:
+        graph_report()
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
