@@ -19,6 +19,7 @@ from .gen import (
     make_anchors,
     make_kv_cache,
     make_verify_case,
+    make_sampled_verify_case,
     make_inject_layout,
 )
 
@@ -34,5 +35,6 @@ __all__ = [
     "make_anchors",
     "make_kv_cache",
     "make_verify_case",
+    "make_sampled_verify_case",
     "make_inject_layout",
 ]

@@ -212,3 +212,32 @@ def make_verify_case(b: int, B: int, V: int, label: str, plant=("uniform",), dty
             elif i == a:
                 row[t] = row.min()
     return {"logits": logits, "draft": draft, "planted": plants.to(torch.int32)}
+
+
+def make_sampled_verify_case(b: int, B: int, V: int, label: str, plant=("uniform",),
+                             dtype: str = "bf16", raise_target: float = 6.0,
+                             raise_draft: float = 6.0, master: int = MASTER_SEED):
+    """Target logits Z and draft logits Y, both [b, B, V] ~ N(0,1), with draft tokens.
+
+    Draft tokens are uniform over the vocabulary (column 0 is the anchor).  For
+    every block position j >= 1 the draft's own logit Y[r, j, d_j] is raised by
+    ``raise_draft`` (the draft favours what it proposed); for target rows
+    i < a_r the target logit Z[r, i, d_{i+1}] is raised by ``raise_target``
+    (planted agreement).  Row 0 of Y is drawn but unused.  What sampled
+    verification accepts is decided by the oracle, not by this generator.
+    """
+    seed = sub_seed(master, "sampled_verify", label, b, B, V)
+    g = _gen(seed)
+    dt = _dtype(dtype)
+    Z = torch.randn((b, B, V), generator=g)
+    Y = torch.randn((b, B, V), generator=g)
+    draft = torch.randint(0, V, (b, B), generator=g, dtype=torch.int64)
+    plants = sample_plants(plant, b, B, sub_seed(seed, "plant"))
+    rows = torch.arange(b)
+    for j in range(1, B):
+        Y[rows, j, draft[:, j]] += raise_draft
+    for i in range(B - 1):
+        sel = plants > i
+        Z[rows[sel], i, draft[sel, i + 1]] += raise_target
+    return {"target": Z.to(dt), "draft_logits": Y.to(dt), "draft": draft.to(torch.int32),
+            "planted": plants.to(torch.int32)}
