@@ -722,6 +722,76 @@ def graph_report():
     model.close()
 
 
+def sampled_verify_report():
+    """Sampled (temperature) verify at the 8B-shaped batch (32 requests, block 8,
+    vocabulary 151936, bf16 target and draft logits) against its HBM roofline, with
+    greedy verify on the same target logits for context.  The algorithmic bytes
+    are one read of the target rows (b*B*V*2) and of the draft rows 1..B-1
+    (b*(B-1)*V*2); the draw's second read of one row pair per request is not
+    counted.  Every iteration reads fresh logit buffers (two sets alternate, each
+    larger than L2 together with the flush), and the L2 is flushed in between.
+    One JSON line."""
+    from block_diffusion_speculative_gemm_b200 import dflash as D
+
+    peaks = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    dev = torch.device("cuda")
+    b, B, V, tau = 32, 8, 151936, 1.0
+    sets = []
+    for k in range(2):
+        c = synth.make_sampled_verify_case(b, B, V, f"bench_sv{k}", plant=("geometric", 4.0))
+        sets.append((c["target"].to(dev), c["draft_logits"].to(dev), c["draft"].to(dev)))
+    out = torch.zeros((b, 4096), dtype=torch.int32, device=dev)
+    out_len = torch.zeros(b, dtype=torch.int32, device=dev)
+    seq = torch.zeros(b, dtype=torch.int32, device=dev)
+    acc = torch.zeros(b, dtype=torch.int32, device=dev)
+    nxt = torch.zeros(b, dtype=torch.int32, device=dev)
+    ws = D.new_workspace(max(D.verify_sampled_workspace_size(b, B, V),
+                             D.verify_workspace_size(b, B, V)))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n=50):
+        for k in range(5):
+            fn(k)
+        torch.cuda.synchronize()
+        ts = []
+        for k in range(n):
+            out_len.zero_()
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn(k)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    def sampled(k):
+        Z, Y, d = sets[k % 2]
+        D.verify_sampled(Z, Y, d, tau, 0x5EED, k, out, out_len, seq, acc, nxt, ws)
+
+    def greedy(k):
+        Z, _, d = sets[k % 2]
+        D.verify(Z, d, out, out_len, seq, acc, nxt, ws)
+
+    ms_s = timed(sampled)
+    ms_g = timed(greedy)
+    assert D.get_error(ws) == 0
+    bytes_s = b * (2 * B - 1) * V * 2
+    bytes_g = b * B * V * 2
+    print(json.dumps({
+        "report": "sampled_verify", "workload": "qwen3_8b_bs32 verify (32 x 8 x 151936, bf16)",
+        "temperature": tau, "sampled_us": round(ms_s * 1e3, 2),
+        "sampled_algorithmic_GBps": round(bytes_s / ms_s / 1e6, 1),
+        "sampled_frac_hbm": round(bytes_s / ms_s / 1e6 / hbm, 4),
+        "greedy_us": round(ms_g * 1e3, 2),
+        "greedy_frac_hbm": round(bytes_g / ms_g / 1e6 / hbm, 4),
+        "rows_per_s_sampled": round(b * B / (ms_s / 1e3), 1),
+        "hbm_peak_GBps": hbm, "peak_source": peaks["source"]}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -736,12 +806,17 @@ def main():
                     help="context only: time the projection GEMMs against torch.matmul")
     ap.add_argument("--graph-report", action="store_true",
                     help="cycles launched call by call versus replayed from a CUDA graph")
+    ap.add_argument("--sampled-verify-report", action="store_true",
+                    help="sampled (temperature) verify against its HBM roofline")
     args = ap.parse_args()
     if args.gemm_report:
         gemm_report()
         return
     if args.graph_report:
         graph_report()
+        return
+    if args.sampled_verify_report:
+        sampled_verify_report()
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

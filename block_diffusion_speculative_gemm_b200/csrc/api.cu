@@ -214,7 +214,6 @@ bool config_supported(const dflash_config& c) {
 int qkv_out(const dflash_config& c) { return (c.n_q + 2 * c.n_kv) * c.head_dim; }
 
 // ---------------------------------------------------------------- workspace layout
-// Workspace header: word 0 = device error bits.
 // Workspace header: the device error word (byte 0), then 32768 completion
 // counters: verify uses one per request, the draft attention one per
 // (request, kv head).  No call writes the header except through those words,
@@ -828,6 +827,39 @@ extern "C" int dflash_verify(const void* target_logits, int logits_dtype,
                        out_len, out_cap, seq_lens, accept_len, next_anchor,
                        at<void>(ws, kHeader), chunks, at<unsigned>(ws, kCntOff), err_word(ws),
                        (cudaStream_t)stream);
+}
+
+// ============================================================== sampled verify
+extern "C" size_t dflash_verify_sampled_workspace_size(int batch, int B, int V) {
+  if (batch < 0 || B < 0 || V < 1) return 0;
+  if (batch == 0 || B == 0) return kHeader;
+  return kHeader + sampled_verify_bytes(batch, B, V);
+}
+
+extern "C" int dflash_verify_sampled(const void* target_logits, const void* draft_logits,
+                                     int logits_dtype, const int32_t* draft_tokens, int batch,
+                                     int B, int V, float temperature, uint64_t seed,
+                                     uint64_t offset, int32_t* out_tokens, int32_t* out_len,
+                                     int out_cap, int32_t* seq_lens, int32_t* accept_len,
+                                     int32_t* next_anchor, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  if (batch < 0 || B < 2 || B > 32 || V < 1 || out_cap < 1) return DFLASH_EINVAL;
+  if (logits_dtype != DFLASH_BF16 && logits_dtype != DFLASH_F32) return DFLASH_EINVAL;
+  if (!(temperature >= 1e-4f && temperature <= 1e4f)) return DFLASH_EINVAL;
+  if (batch == 0) return DFLASH_OK;
+  if (!target_logits || !draft_logits || !draft_tokens || !out_tokens || !out_len || !seq_lens ||
+      !accept_len || !next_anchor || !ws)
+    return DFLASH_EINVAL;
+  if (!aligned16(target_logits) || !aligned16(draft_logits) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255))
+    return DFLASH_EINVAL;
+  // target and draft rows share one grid dimension
+  if ((int64_t)2 * batch * B > 65535) return DFLASH_EUNSUPPORTED;
+  if (ws_bytes < kHeader + sampled_verify_bytes(batch, B, V)) return DFLASH_EWORKSPACE;
+  return launch_sampled_verify(target_logits, draft_logits, logits_dtype, draft_tokens, batch, B,
+                               V, temperature, seed, offset, out_tokens, out_len, out_cap,
+                               seq_lens, accept_len, next_anchor, at<void>(ws, kHeader),
+                               at<unsigned>(ws, kCntOff), err_word(ws), (cudaStream_t)stream);
 }
 
 // ============================================================== test hooks (dflash_debug.h)

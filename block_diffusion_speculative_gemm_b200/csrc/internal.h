@@ -235,4 +235,13 @@ int launch_verify(const void* logits, int dtype, const int32_t* draft, int batch
                   unsigned* cnt, int32_t* err, cudaStream_t s);
 int verify_chunks(int rows, int V);
 
+// ---------------------------------------------------------------- sampled verify
+// Scratch bytes of one sampled-verify call (placed after the workspace header).
+size_t sampled_verify_bytes(int batch, int B, int V);
+int launch_sampled_verify(const void* target, const void* drafted, int dtype, const int32_t* draft,
+                          int batch, int B, int V, float tau, uint64_t seed, uint64_t offset,
+                          int32_t* out_tokens, int32_t* out_len, int out_cap, int32_t* seq_lens,
+                          int32_t* accept_len, int32_t* next_anchor, void* scratch,
+                          unsigned* cnt, int32_t* err, cudaStream_t s);
+
 }  // namespace dflash

@@ -1,0 +1,466 @@
+// Sampled (temperature) verify of a drafted block.
+//
+// Sources: "DFlash: Block Diffusion for Flash Speculative Decoding" (study
+// notes), §消融实验结论 (drafting holds up under high-temperature sampling) and
+// §与 Speculative Decoding 系列的关系 (the speculative-decoding line of Leviathan
+// et al., 2023); blog "DFlash：用“块扩散”魔法", §2 Flash Verification (the
+// target's probabilities are compared with the draft's).  The pages give no
+// acceptance rule; this is standard speculative sampling:
+//
+//   p_i = softmax(Z_i / tau) (target row i: the token after block position i),
+//   q_j = softmax(Y_j / tau) (draft distribution at block position j);
+//   for i = 0..B-2 in order, d_{i+1} is accepted while
+//     log U_i < log p_i(d_{i+1}) - log q_{i+1}(d_{i+1});
+//   the first rejection at i draws the last token from max(0, p_i - q_{i+1}),
+//   no rejection draws it from p_{B-1}; emit d_1..d_a and the drawn token.
+//
+// Draws are Gumbel-max, argmax_v (log w_v - log(-log U'_v)), ties to the lower
+// index.  Uniforms come from Philox4x64-10 (Salmon, Moraes, Dror and Shaw,
+// "Parallel random numbers: as easy as 1, 2, 3", SC 2011) under key (seed, 0)
+// with counter (offset, request, stream, n / 4), word n % 4: stream 0 gives
+// U_i (n = i), stream 1 gives U'_v (n = v).  A word w gives
+// U = (w >> 11) 2^-53 in [0, 1) and U' = ((w >> 11) + 1/2) 2^-53 in (0, 1).
+//
+// Two bandwidth-bound kernels chained by programmatic dependent launch:
+//   sv_stats_kernel  one CTA per (row chunk, row) of the target and the draft
+//                    logits: (max, sum of 2^(x log2e / tau - max)) per chunk.
+//                    The last CTA of a request merges its rows (one warp,
+//                    lane i = row i), takes the accept decisions in the log
+//                    domain and records the accept length and the normalisers
+//                    of the row(s) the draw needs.
+//   sv_draw_kernel   one CTA per (vocabulary chunk, request) reads target row a
+//                    (and draft row a+1) once more, forms the Gumbel-perturbed
+//                    log-weights and keeps the best; the last CTA of a request
+//                    merges the chunks in order, writes d_1..d_a and the drawn
+//                    token behind out_len and advances the lengths.
+// Counters count arrivals per request and are set back to zero by the CTA
+// that completes them, so the workspace stays reusable.
+#include "common.cuh"
+#include "internal.h"
+
+namespace dflash {
+
+namespace {
+
+constexpr int kSvThreads = 256;
+constexpr float kLn2 = 0.69314718055994531f;
+constexpr float kLog2e = 1.44269504088896341f;
+constexpr float kTwoM53 = 1.1102230246251565e-16f;  // 2^-53
+
+enum SvMode : int { SV_SKIP = 0, SV_RESIDUAL = 1, SV_BONUS = 2 };
+
+struct SvPart {  // per (tensor row, chunk): max and sum of 2^(x c - max), c = log2e / tau
+  float m, s;
+};
+
+struct SvRec {  // per request, written by the stats kernel for the draw kernel
+  int a, mode;
+  float mt, lst;  // target row a: max and log of the sum, natural units (x / tau)
+  float md, lsd;  // draft row a+1 (residual mode)
+  int pad[2];
+};
+
+struct SvDraw {  // per (request, chunk): best residual and best target-only draw
+  float sr;
+  int ir;
+  float sp;
+  int ip;
+};
+
+// Philox4x64-10 block function: counter (c0..c3), key (k0, k1).
+__device__ __forceinline__ void philox4x64_10(uint64_t (&c)[4], uint64_t k0, uint64_t k1) {
+  constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+  constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += W0;
+      k1 += W1;
+    }
+    const uint64_t hi0 = __umul64hi(M0, c[0]), lo0 = M0 * c[0];
+    const uint64_t hi1 = __umul64hi(M1, c[2]), lo1 = M1 * c[2];
+    const uint64_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+    c[0] = n0;
+    c[1] = lo1;
+    c[2] = n2;
+    c[3] = lo0;
+  }
+}
+
+__device__ __forceinline__ void philox_block(uint64_t seed, uint64_t offset, int request,
+                                             int stream, uint64_t n4, uint64_t (&w)[4]) {
+  w[0] = offset;
+  w[1] = (uint64_t)request;
+  w[2] = (uint64_t)stream;
+  w[3] = n4;
+  philox4x64_10(w, seed, 0ull);
+}
+
+// log U for U = (w >> 11) 2^-53 in [0, 1) (-inf at 0); the upper half goes
+// through log1p(-(1 - U)) with 1 - U formed exactly from the integer.
+__device__ __forceinline__ float log_u_closed_open(uint64_t w) {
+  const uint64_t k = w >> 11;
+  if (k < (1ull << 52)) return k == 0 ? -INFINITY : logf(__ull2float_rn(k) * kTwoM53);
+  const uint64_t m = (1ull << 53) - k;  // 1 - U = m 2^-53
+  return log1pf(-__ull2float_rn(m) * kTwoM53);
+}
+
+// Gumbel variate -log(-log U') for U' = ((w >> 11) + 1/2) 2^-53 in (0, 1).
+__device__ __forceinline__ float gumbel_of(uint64_t w) {
+  const uint64_t k = w >> 11;
+  float e;  // -log U' > 0
+  if (k < (1ull << 52)) {
+    e = -logf((__ull2float_rn(k) + 0.5f) * kTwoM53);
+  } else {
+    const uint64_t m = (1ull << 53) - 1 - k;  // 1 - U' = (m + 1/2) 2^-53
+    e = -log1pf(-(__ull2float_rn(m) + 0.5f) * kTwoM53);
+  }
+  return -logf(e);
+}
+
+__device__ __forceinline__ void stat_merge(float& m, float& s, float m2, float s2) {
+  if (m2 == -INFINITY) return;
+  if (m == -INFINITY) {
+    m = m2;
+    s = s2;
+    return;
+  }
+  const float M = fmaxf(m, m2);
+  s = s * exp2f(m - M) + s2 * exp2f(m2 - M);
+  m = M;
+}
+
+template <typename T>
+__device__ __forceinline__ void stat_add16(const uint4& u, float c, float& m, float& s) {
+  constexpr int W = 16 / sizeof(T);
+  const T* e = reinterpret_cast<const T*>(&u);
+  float x[W];
+  float mb = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < W; ++k) {
+    x[k] = to_f(e[k]) * c;
+    mb = fmaxf(mb, x[k]);
+  }
+  if (mb > m) {
+    s = (m == -INFINITY) ? 0.f : s * exp2f(m - mb);
+    m = mb;
+  }
+  if (m == -INFINITY) return;  // nothing finite yet: every x is -inf
+#pragma unroll
+  for (int k = 0; k < W; ++k) s += exp2f(x[k] - m);
+}
+
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kSvThreads)
+    sv_stats_kernel(const T* __restrict__ target, const T* __restrict__ drafted, int rows, int B,
+                    int V, float c2, float inv_tau, int chunk, int chunks, SvPart* __restrict__ part,
+                    unsigned* __restrict__ cnt, const int32_t* __restrict__ draft,
+                    const int32_t* __restrict__ out_len, int out_cap, uint64_t seed,
+                    uint64_t offset, SvRec* __restrict__ rec, int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float s_m[kSvThreads / 32], s_s[kSvThreads / 32];
+  __shared__ int s_last;
+  const int y = blockIdx.y, c = blockIdx.x;
+  const bool is_draft = y >= rows;
+  const int row = is_draft ? y - rows : y;  // r * B + i
+  const int r = row / B;
+  float m = -INFINITY, s = 0.f;
+  if (!(is_draft && row % B == 0)) {  // draft row 0 (the anchor) has no distribution
+    const T* x = (is_draft ? drafted : target) + (size_t)row * V;
+    const int v0 = c * chunk, v1 = min(V, v0 + chunk);
+    if (VEC) {
+      constexpr int W = 16 / sizeof(T);
+      const int nvec = max(0, v1 - v0) / W;
+      const uint4* p = reinterpret_cast<const uint4*>(x + v0);
+      int t = threadIdx.x;
+      for (; t + 3 * kSvThreads < nvec; t += 4 * kSvThreads) {
+        uint4 u[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) u[j] = __ldcs(p + t + j * kSvThreads);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) stat_add16<T>(u[j], c2, m, s);
+      }
+      for (; t < nvec; t += kSvThreads) stat_add16<T>(__ldcs(p + t), c2, m, s);
+      for (int v = v0 + nvec * W + threadIdx.x; v < v1; v += kSvThreads)
+        stat_merge(m, s, to_f(x[v]) * c2, 1.f);
+    } else {
+      for (int v = v0 + threadIdx.x; v < v1; v += kSvThreads) stat_merge(m, s, to_f(x[v]) * c2, 1.f);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float sv2 = __shfl_xor_sync(0xffffffffu, s, o);
+    stat_merge(m, s, m2, sv2);
+  }
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if (lane == 0) {
+    s_m[w] = m;
+    s_s[w] = s;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    m = s_m[0];
+    s = s_s[0];
+    for (int k = 1; k < kSvThreads / 32; ++k) stat_merge(m, s, s_m[k], s_s[k]);
+    part[(size_t)y * chunks + c] = SvPart{m, s};
+    __threadfence();  // the partial is visible before this CTA is counted
+    s_last = atomicAdd(&cnt[r], 1u) == (unsigned)(2 * B * chunks - 1);
+  }
+  __syncthreads();
+  if (!s_last || threadIdx.x >= 32) return;
+  __threadfence();  // every partial of request r counted before the reads below
+
+  // ---- accept decisions of request r: lane i = block row i
+  auto merged = [&](int yy) {
+    const SvPart* p = part + (size_t)yy * chunks;
+    float mm = __ldcg(&p[0].m), ss = __ldcg(&p[0].s);
+    for (int k = 1; k < chunks; ++k) stat_merge(mm, ss, __ldcg(&p[k].m), __ldcg(&p[k].s));
+    return SvPart{mm, ss};
+  };
+  SvPart st{-INFINITY, 0.f}, sd{-INFINITY, 0.f};
+  int d = 0;
+  if (lane < B) {
+    st = merged(r * B + lane);
+    if (lane > 0) sd = merged(rows + r * B + lane);
+    d = draft[(size_t)r * B + lane];
+  }
+  const unsigned bad = __ballot_sync(0xffffffffu, lane < B && (d < 0 || d >= V));
+  const int d_next = __shfl_down_sync(0xffffffffu, d, 1);
+  const float md_next = __shfl_down_sync(0xffffffffu, sd.m, 1);
+  const float sd_next = __shfl_down_sync(0xffffffffu, sd.s, 1);
+  bool reject = false;
+  if (!bad && lane < B - 1) {
+    const float z = to_f(target[((size_t)r * B + lane) * V + d_next]) * c2;
+    const float yv = to_f(drafted[((size_t)r * B + lane + 1) * V + d_next]) * c2;
+    // log2 p_i(x) - log2 q_{i+1}(x), then natural units
+    const float l2rho = (z - st.m - log2f(st.s)) - (yv - md_next - log2f(sd_next));
+    uint64_t wds[4];
+    philox_block(seed, offset, r, 0, (uint64_t)(lane >> 2), wds);
+    const int q = lane & 3;
+    const uint64_t wsel = q == 0 ? wds[0] : q == 1 ? wds[1] : q == 2 ? wds[2] : wds[3];
+    const float lu = log_u_closed_open(wsel);
+    reject = !(lu < l2rho * kLn2);
+  }
+  const unsigned rej = __ballot_sync(0xffffffffu, reject);
+  const int a = rej ? (__ffs(rej) - 1) : (B - 1);
+  int mode = SV_SKIP;
+  if (bad) {
+    if (lane == 0) set_error(err, DFLASH_DEV_TOKEN_RANGE);
+  } else {
+    const int ol = out_len[r];
+    if (ol < 0 || (long long)ol + a + 1 > out_cap) {
+      if (lane == 0) set_error(err, DFLASH_DEV_OUT_CAP);
+    } else {
+      mode = a < B - 1 ? SV_RESIDUAL : SV_BONUS;
+    }
+  }
+  if (lane == a) {
+    SvRec q;
+    q.a = a;
+    q.mode = mode;
+    q.mt = st.m * kLn2;
+    q.lst = logf(st.s);
+    q.md = md_next * kLn2;
+    q.lsd = mode == SV_RESIDUAL ? logf(sd_next) : 0.f;
+    q.pad[0] = q.pad[1] = 0;
+    rec[r] = q;
+  }
+  if (lane == 0) cnt[r] = 0;  // ready for the draw kernel and the next call
+}
+
+__device__ __forceinline__ void draw_merge(float& s, int& i, float s2, int i2) {
+  if (s2 > s || (s2 == s && i2 < i)) {
+    s = s2;
+    i = i2;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void load4(const T* p, bool vec, float (&x)[4], int n) {
+  if (vec && n == 4) {
+    if (sizeof(T) == 2) {
+      const uint2 u = *reinterpret_cast<const uint2*>(p);
+      const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) x[k] = to_f(e[k]);
+    } else {
+      const float4 u = *reinterpret_cast<const float4*>(p);
+      x[0] = u.x;
+      x[1] = u.y;
+      x[2] = u.z;
+      x[3] = u.w;
+    }
+    return;
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) x[k] = k < n ? to_f(p[k]) : 0.f;
+}
+
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kSvThreads)
+    sv_draw_kernel(const T* __restrict__ target, const T* __restrict__ drafted, int B, int V,
+                   float inv_tau, int chunk, int chunks, const SvRec* __restrict__ rec,
+                   SvDraw* __restrict__ part, unsigned* __restrict__ cnt,
+                   const int32_t* __restrict__ draft, int32_t* out_tokens, int32_t* out_len,
+                   int out_cap, int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
+                   uint64_t seed, uint64_t offset) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ SvDraw s_d[kSvThreads / 32];
+  __shared__ int s_last;
+  const int r = blockIdx.y, c = blockIdx.x;
+  const SvRec q = rec[r];
+  float sr = -INFINITY, sp = -INFINITY;
+  int ir = 0x7fffffff, ip = 0x7fffffff;
+  if (q.mode != SV_SKIP) {
+    const bool residual = q.mode == SV_RESIDUAL;
+    const T* zr = target + ((size_t)r * B + q.a) * V;
+    const T* yr = residual ? drafted + ((size_t)r * B + q.a + 1) * V : zr;  // draft row a+1
+    const int v0 = c * chunk, v1 = min(V, v0 + chunk);  // chunk is a multiple of 4
+    // groups of 4 consecutive entries share one Philox block; each thread
+    // visits its groups in increasing order, so '>' keeps the lowest index
+    for (int g = v0 / 4 + threadIdx.x; g * 4 < v1; g += kSvThreads) {
+      const int vb = g * 4, n = min(4, v1 - vb);
+      float z[4], yv[4];
+      load4<T>(zr + vb, VEC, z, n);
+      if (residual) load4<T>(yr + vb, VEC, yv, n);
+      uint64_t wds[4];
+      philox_block(seed, offset, r, 1, (uint64_t)g, wds);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (k >= n) break;
+        const float gum = gumbel_of(wds[k]);
+        const float lp = z[k] * inv_tau - q.mt - q.lst;
+        const float scp = lp + gum;
+        if (scp > sp) { sp = scp; ip = vb + k; }
+        if (residual) {
+          const float lq = yv[k] * inv_tau - q.md - q.lsd;
+          if (lp > lq) {
+            const float scr = lp + logf(-expm1f(lq - lp)) + gum;
+            if (scr > sr) { sr = scr; ir = vb + k; }
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    draw_merge(sr, ir, __shfl_xor_sync(0xffffffffu, sr, o), __shfl_xor_sync(0xffffffffu, ir, o));
+    draw_merge(sp, ip, __shfl_xor_sync(0xffffffffu, sp, o), __shfl_xor_sync(0xffffffffu, ip, o));
+  }
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if (lane == 0) s_d[w] = SvDraw{sr, ir, sp, ip};
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    SvDraw b = s_d[0];
+    for (int k = 1; k < kSvThreads / 32; ++k) {
+      draw_merge(b.sr, b.ir, s_d[k].sr, s_d[k].ir);
+      draw_merge(b.sp, b.ip, s_d[k].sp, s_d[k].ip);
+    }
+    part[(size_t)r * chunks + c] = b;
+    __threadfence();
+    s_last = atomicAdd(&cnt[r], 1u) == (unsigned)(chunks - 1);
+  }
+  __syncthreads();
+  if (!s_last || threadIdx.x >= 32) return;
+  __threadfence();
+  if (q.mode != SV_SKIP) {
+    // chunks in order; the residual draw unless fp32 left it empty
+    float br = -INFINITY, bp = -INFINITY;
+    int jr = 0x7fffffff, jp = 0x7fffffff;
+    for (int k = lane; k < chunks; k += 32) {
+      const SvDraw* p = part + (size_t)r * chunks + k;
+      draw_merge(br, jr, __ldcg(&p->sr), __ldcg(&p->ir));
+      draw_merge(bp, jp, __ldcg(&p->sp), __ldcg(&p->ip));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      draw_merge(br, jr, __shfl_xor_sync(0xffffffffu, br, o), __shfl_xor_sync(0xffffffffu, jr, o));
+      draw_merge(bp, jp, __shfl_xor_sync(0xffffffffu, bp, o), __shfl_xor_sync(0xffffffffu, jp, o));
+    }
+    const int tok = (q.mode == SV_RESIDUAL && br != -INFINITY) ? jr : jp;
+    const int a = q.a, ol = out_len[r];
+    int32_t* o = out_tokens + (size_t)r * out_cap + ol;
+    if (lane < a) o[lane] = draft[(size_t)r * B + lane + 1];
+    if (lane == a) o[a] = tok;
+    if (lane == 0) {
+      out_len[r] = ol + a + 1;
+      seq_lens[r] += a + 1;
+      accept_len[r] = a;
+      next_anchor[r] = tok;
+    }
+  }
+  if (lane == 0) cnt[r] = 0;
+}
+
+int sv_chunks(int rows, int V, int min_chunk) {
+  int target = (4 * 148 + rows - 1) / rows;
+  int max_c = (V + min_chunk - 1) / min_chunk;
+  int c = target < max_c ? target : max_c;
+  return c < 1 ? 1 : c;
+}
+
+int chunk_len(int V, int chunks) {
+  int chunk = (V + chunks - 1) / chunks;
+  return (chunk + 63) / 64 * 64;
+}
+
+}  // namespace
+
+size_t sampled_verify_bytes(int batch, int B, int V) {
+  const int c1 = sv_chunks(2 * batch * B, V, 4096), c2 = sv_chunks(batch, V, 2048);
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  return al((size_t)2 * batch * B * c1 * sizeof(SvPart)) + al((size_t)batch * sizeof(SvRec)) +
+         al((size_t)batch * c2 * sizeof(SvDraw));
+}
+
+int launch_sampled_verify(const void* target, const void* drafted, int dtype, const int32_t* draft,
+                          int batch, int B, int V, float tau, uint64_t seed, uint64_t offset,
+                          int32_t* out_tokens, int32_t* out_len, int out_cap, int32_t* seq_lens,
+                          int32_t* accept_len, int32_t* next_anchor, void* scratch,
+                          unsigned* cnt, int32_t* err, cudaStream_t s) {
+  const int rows = batch * B;
+  const int c1 = sv_chunks(2 * rows, V, 4096), c2 = sv_chunks(batch, V, 2048);
+  const int k1 = chunk_len(V, c1), k2 = chunk_len(V, c2);
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  SvPart* part1 = reinterpret_cast<SvPart*>(base);
+  SvRec* rec = reinterpret_cast<SvRec*>(base + al((size_t)2 * rows * c1 * sizeof(SvPart)));
+  SvDraw* part2 = reinterpret_cast<SvDraw*>(reinterpret_cast<uint8_t*>(rec) +
+                                            al((size_t)batch * sizeof(SvRec)));
+  const int esz = dtype == DFLASH_BF16 ? 2 : 4;
+  const bool vec = ((size_t)V * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(target) % 16) == 0 &&
+                   (reinterpret_cast<uintptr_t>(drafted) % 16) == 0;
+  const float inv_tau = 1.f / tau, c2f = kLog2e / tau;
+  TimedScope ts(s, TC_VERIFY);
+  cudaError_t e;
+  const dim3 g1(c1, 2 * rows), g2(c2, batch), blk(kSvThreads);
+  if (dtype == DFLASH_BF16) {
+    const __nv_bfloat16* zt = static_cast<const __nv_bfloat16*>(target);
+    const __nv_bfloat16* yd = static_cast<const __nv_bfloat16*>(drafted);
+    auto ka = vec ? sv_stats_kernel<__nv_bfloat16, true> : sv_stats_kernel<__nv_bfloat16, false>;
+    auto kb = vec ? sv_draw_kernel<__nv_bfloat16, true> : sv_draw_kernel<__nv_bfloat16, false>;
+    e = launch_pdl(ka, g1, blk, 0, s, 1, zt, yd, rows, B, V, c2f, inv_tau, k1, c1, part1, cnt,
+                   draft, (const int32_t*)out_len, out_cap, seed, offset, rec, err);
+    if (e == cudaSuccess)
+      e = launch_pdl(kb, g2, blk, 0, s, 1, zt, yd, B, V, inv_tau, k2, c2, (const SvRec*)rec, part2,
+                     cnt, draft, out_tokens, out_len, out_cap, seq_lens, accept_len, next_anchor,
+                     seed, offset);
+  } else {
+    const float* zt = static_cast<const float*>(target);
+    const float* yd = static_cast<const float*>(drafted);
+    auto ka = vec ? sv_stats_kernel<float, true> : sv_stats_kernel<float, false>;
+    auto kb = vec ? sv_draw_kernel<float, true> : sv_draw_kernel<float, false>;
+    e = launch_pdl(ka, g1, blk, 0, s, 1, zt, yd, rows, B, V, c2f, inv_tau, k1, c1, part1, cnt,
+                   draft, (const int32_t*)out_len, out_cap, seed, offset, rec, err);
+    if (e == cudaSuccess)
+      e = launch_pdl(kb, g2, blk, 0, s, 1, zt, yd, B, V, inv_tau, k2, c2, (const SvRec*)rec, part2,
+                     cnt, draft, out_tokens, out_len, out_cap, seq_lens, accept_len, next_anchor,
+                     seed, offset);
+  }
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
+}
+
+}  // namespace dflash

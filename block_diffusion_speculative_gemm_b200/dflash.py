@@ -80,6 +80,11 @@ def lib() -> ctypes.CDLL:
         L.dflash_get_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
         L.dflash_verify_noalloc.argtypes = [vp, i32, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp,
                                             vp, vp]
+        u64 = ctypes.c_uint64
+        L.dflash_verify_sampled_workspace_size.argtypes = [i32, i32, i32]
+        L.dflash_verify_sampled_workspace_size.restype = sz
+        L.dflash_verify_sampled.argtypes = [vp, vp, i32, vp, i32, i32, i32, ctypes.c_float, u64,
+                                            u64, vp, vp, i32, vp, vp, vp, vp, sz, vp]
         L.dflash_status_str.argtypes = [i32]
         L.dflash_status_str.restype = ctypes.c_char_p
         L.dflash_timing_enable.argtypes = [i32]
@@ -318,6 +323,41 @@ def verify_noalloc(target_logits: torch.Tensor, draft_tokens: torch.Tensor,
         _ptr(target_logits), dt, _ptr(draft_tokens), batch, B, V, _ptr(out_tokens), _ptr(out_len),
         out_tokens.shape[1], _ptr(seq_lens), _ptr(accept_len), _ptr(next_anchor),
         _ptr(error_bits), _stream(stream)))
+
+
+def verify_sampled_workspace_size(batch: int, B: int, V: int) -> int:
+    return int(lib().dflash_verify_sampled_workspace_size(batch, B, V))
+
+
+def verify_sampled(target_logits: torch.Tensor, draft_logits: torch.Tensor,
+                   draft_tokens: torch.Tensor, temperature: float, seed: int, offset: int,
+                   out_tokens: torch.Tensor, out_len: torch.Tensor, seq_lens: torch.Tensor,
+                   accept_len: torch.Tensor, next_anchor: torch.Tensor, ws: torch.Tensor,
+                   stream=None):
+    """Sampled (temperature) verify: speculative sampling of the drafted block
+    against the target, draws from Philox4x64-10 under (seed, offset); see
+    dflash_verify_sampled in include/dflash.h."""
+    if target_logits.dim() != 3:
+        raise ValueError("target_logits must be [batch, B, V]")
+    batch, B, V = target_logits.shape
+    dt = {torch.bfloat16: BF16, torch.float32: F32}.get(target_logits.dtype)
+    if dt is None:
+        raise TypeError("target_logits must be bfloat16 or float32")
+    _need(target_logits, "target_logits")
+    _need(draft_logits, "draft_logits", target_logits.dtype, (batch, B, V))
+    _need(draft_tokens, "draft_tokens", torch.int32, (batch, B))
+    _need(out_tokens, "out_tokens", torch.int32)
+    if out_tokens.dim() != 2 or out_tokens.shape[0] != batch:
+        raise ValueError("out_tokens must be [batch, out_cap]")
+    for n, t in (("out_len", out_len), ("seq_lens", seq_lens), ("accept_len", accept_len),
+                 ("next_anchor", next_anchor)):
+        _need(t, n, torch.int32, (batch,))
+    _need(ws, "ws", torch.uint8)
+    _check("dflash_verify_sampled", lib().dflash_verify_sampled(
+        _ptr(target_logits), _ptr(draft_logits), dt, _ptr(draft_tokens), batch, B, V,
+        float(temperature), int(seed) & (2**64 - 1), int(offset) & (2**64 - 1), _ptr(out_tokens),
+        _ptr(out_len), out_tokens.shape[1], _ptr(seq_lens), _ptr(accept_len), _ptr(next_anchor),
+        _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def get_error(ws: torch.Tensor, stream=None) -> int:

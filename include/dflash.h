@@ -17,6 +17,8 @@
  *                       generate_block(context, block_size).
  *   dflash_verify       Blog "DFlash：用“块扩散”魔法", §2 Flash Verification:
  *                       decide_acceptance(logits, draft_block), read greedily.
+ *   dflash_verify_sampled  the same step under temperature sampling
+ *                       (speculative sampling; see its declaration).
  *
  * Conventions shared by every call
  * --------------------------------
@@ -207,6 +209,45 @@ int dflash_verify(const void* target_logits, int logits_dtype, const int32_t* dr
                   int batch, int B, int V, int32_t* out_tokens, int32_t* out_len, int out_cap,
                   int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor, void* ws,
                   size_t ws_bytes, void* stream);
+
+/*
+ * Sampled (temperature) verify.  The pages fix no acceptance rule for sampling
+ * ("DFlash: Block Diffusion for Flash Speculative Decoding", §消融实验结论: drafting
+ * holds up under high-temperature sampling; §与 Speculative Decoding 系列的关系:
+ * the speculative-decoding line of Leviathan et al., 2023; blog "DFlash：用“块
+ * 扩散”魔法", §2 Flash Verification: the target's probabilities are compared
+ * with the draft's).  The rule is standard speculative sampling:
+ *   p_i = softmax(target_logits[r, i] / temperature)  (token after position i),
+ *   q_j = softmax(draft_logits[r, j] / temperature)   (draft at position j);
+ *   for i = 0..B-2 in order d_{i+1} is accepted while
+ *   log U_i < log p_i(d_{i+1}) - log q_{i+1}(d_{i+1}); at the first rejection
+ *   (a = i) the last token is drawn from max(0, p_i - q_{i+1}); with none
+ *   (a = B-1) it is drawn from p_{B-1}.  Emits d_1..d_a and the drawn token as
+ *   dflash_verify does; next_anchor = the drawn token.
+ * Draws are Gumbel-max, argmax_v (log w_v - log(-log U'_v)), ties to the lower
+ * id; if fp32 rounding leaves max(0, p_i - q_{i+1}) empty, the draw uses p_i.
+ * Uniforms: Philox4x64-10 (Salmon et al., SC 2011) under key (seed, 0),
+ * counter (offset, r, stream, n / 4), 64-bit word n % 4; stream 0 gives U_i
+ * (n = i) as (w >> 11) 2^-53, stream 1 gives U'_v (n = v) as
+ * ((w >> 11) + 1/2) 2^-53.  Equal (seed, offset) repeat the call's draws;
+ * advance offset between calls.  Arithmetic is fp32.
+ *   target_logits, draft_logits  device [batch, B, V] of logits_dtype
+ *                  (DFLASH_BF16 or DFLASH_F32), 16-byte aligned; row 0 of
+ *                  draft_logits is not read.
+ *   draft_tokens   device int32 [batch, B] (position 0 = anchor).
+ *   temperature    in [1e-4, 1e4].
+ *   out_tokens .. next_anchor  as in dflash_verify.
+ *   ws             workspace of at least
+ *                  dflash_verify_sampled_workspace_size(batch, B, V) bytes.
+ * Errors as in dflash_verify; B in [2, 32]; 2 * batch * B <= 65535
+ * (DFLASH_EUNSUPPORTED beyond); batch == 0 is a no-op.
+ */
+size_t dflash_verify_sampled_workspace_size(int batch, int B, int V);
+int dflash_verify_sampled(const void* target_logits, const void* draft_logits, int logits_dtype,
+                          const int32_t* draft_tokens, int batch, int B, int V, float temperature,
+                          uint64_t seed, uint64_t offset, int32_t* out_tokens, int32_t* out_len,
+                          int out_cap, int32_t* seq_lens, int32_t* accept_len,
+                          int32_t* next_anchor, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Greedy verify without any workspace or allocation.  The pages have no

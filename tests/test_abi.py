@@ -86,3 +86,45 @@ def test_draft_and_inject_reject_null_model_and_bad_block():
     assert L.dflash_inject_kv(None, None, p, p, 1, 4, p, p, 64, p, 1 << 20, None) == D.EINVAL
     assert L.dflash_workspace_init(ctypes.c_void_p(4100), 256, None) == D.EINVAL
     assert L.dflash_get_error(None, None, None) == D.EINVAL
+
+
+def test_sampled_verify_size_query():
+    L = D.lib()
+    hdr = L.dflash_verify_sampled_workspace_size(0, 8, 100)
+    assert hdr == L.dflash_verify_workspace_size(0, 8, 100)  # the shared header alone
+    big = L.dflash_verify_sampled_workspace_size(32, 8, 151936)
+    assert big > hdr and big % 256 == 0
+    assert L.dflash_verify_sampled_workspace_size(-1, 8, 100) == 0
+    assert L.dflash_verify_sampled_workspace_size(4, 8, 0) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=1), D.EINVAL),
+    (dict(B=33), D.EINVAL),
+    (dict(V=0), D.EINVAL),
+    (dict(out_cap=0), D.EINVAL),
+    (dict(dtype=5), D.EINVAL),
+    (dict(tau=0.0), D.EINVAL),            # greedy is dflash_verify
+    (dict(tau=-1.0), D.EINVAL),
+    (dict(tau=float("nan")), D.EINVAL),
+    (dict(tau=1e5), D.EINVAL),
+    (dict(logits=None), D.EINVAL),
+    (dict(dlogits=None), D.EINVAL),
+    (dict(dlogits=4104), D.EINVAL),       # misaligned draft logits
+    (dict(ws=64), D.EINVAL),
+    (dict(batch=20000, B=2), D.EUNSUPPORTED),  # 2 * batch * B rows > 65535
+    (dict(ws_bytes=8), D.EWORKSPACE),
+    (dict(batch=0), D.OK),
+])
+def test_sampled_verify_host_checks(kw, code):
+    L = D.lib()
+    a = dict(logits=4096, dlogits=8192, dtype=D.BF16, draft=4096, batch=2, B=4, V=1000, tau=0.7,
+             out=4096, out_len=4096, out_cap=16, seq=4096, acc=4096, nxt=4096, ws=4096,
+             ws_bytes=1 << 20)
+    a.update(kw)
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    st = L.dflash_verify_sampled(vp(a["logits"]), vp(a["dlogits"]), a["dtype"], vp(a["draft"]),
+                                 a["batch"], a["B"], a["V"], a["tau"], 1, 0, vp(a["out"]),
+                                 vp(a["out_len"]), a["out_cap"], vp(a["seq"]), vp(a["acc"]),
+                                 vp(a["nxt"]), vp(a["ws"]), a["ws_bytes"], None)
+    assert st == code
