@@ -8,3 +8,4 @@ library and its Python binding never call it, and it shares no code with them.
 from .dflash_oracle import *  # noqa: F401,F403
 from .dflash_oracle import __all__  # noqa: F401
 from . import sampled_verify  # noqa: F401
+from . import sampled_draft  # noqa: F401
