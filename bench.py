@@ -294,11 +294,15 @@ def run_dflash(args, rank, world, local_rank):
     n_draft = args.steps
     for _ in range(3):
         D.draft_block(model, anchors_d, ctx_d, kc, vc, B, cfg.steps, draft, ws)
-    d0.record(stream)
-    for _ in range(n_draft):
-        D.draft_block(model, anchors_d, ctx_d, kc, vc, B, cfg.steps, draft, ws)
-    d1.record(stream)
     torch.cuda.synchronize()
+    # sampled like the timed region: the draft-only loop runs after seconds of load,
+    # where the power cap may have lowered the SM clock
+    with ClockSampler(local_rank) as dclk:
+        d0.record(stream)
+        for _ in range(n_draft):
+            D.draft_block(model, anchors_d, ctx_d, kc, vc, B, cfg.steps, draft, ws)
+        d1.record(stream)
+        torch.cuda.synchronize()
     draft_ms = d0.elapsed_time(d1) / n_draft
     err = D.get_error(ws)
     if err:
@@ -367,7 +371,8 @@ def run_dflash(args, rank, world, local_rank):
         # dflash_draft_block alone: block positions and drafted (masked) positions per s
         "draft_block": {"ms": round(draft_ms, 4),
                         "block_tok_s": round(b * world * B / (draft_ms / 1e3), 1),
-                        "drafted_tok_s": round(b * world * (B - 1) / (draft_ms / 1e3), 1)},
+                        "drafted_tok_s": round(b * world * (B - 1) / (draft_ms / 1e3), 1),
+                        "clocks": dclk.summary()},
         "prefill_inject": prefill_report(cfg, n_p, prefill_ms, peaks),
         "clocks": clk.summary(),
     }
