@@ -9,3 +9,4 @@ from .dflash_oracle import *  # noqa: F401,F403
 from .dflash_oracle import __all__  # noqa: F401
 from . import sampled_verify  # noqa: F401
 from . import sampled_draft  # noqa: F401
+from . import paged_kv  # noqa: F401
