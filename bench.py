@@ -569,8 +569,11 @@ def run_reference(args):
     sec = sum(times) / len(times)
     value = cfg.B / sec
     cores = os.cpu_count()
-    return {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": 0,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 2),
+    # n_gpus is the launch's N (the line pairs with our arm's line at that N); the
+    # oracle itself runs on rank 0's host cores
+    return {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
+            "device": "cpu", "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(sec * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded random-init weights and inputs)", "impl": "reference",
             "config": {"workload": WORKLOAD, "sample": "one request's cycle per step"},
