@@ -1,4 +1,4 @@
-"""Writes tests/golden/tiny_f32_oracle.json from the oracle alone.
+"""Writes tests/golden/tiny_f32_oracle.json and sampled_oracle.json from the oracle alone.
 
 Run from the repository root: ``python tests/golden/make_golden.py``.  It
 imports only ``oracle`` and the seeded input generators in ``synth``; the
@@ -44,8 +44,38 @@ def tiny_case():
     }
 
 
+def sampled_case():
+    """Sampled verify on a small batch and sampled drafting on the tiny model."""
+    b, B, V, tau, seed, offset = 4, 6, 300, 0.8, 0x5EED, 3
+    c = synth.make_sampled_verify_case(b, B, V, "golden_sv", plant=("geometric", 4.0),
+                                       dtype="f32")
+    res = O.sampled_verify.sampled_verify_batch(c["target"], c["draft_logits"], c["draft"], tau,
+                                                seed, offset, np.zeros((b, 3 * B)),
+                                                np.zeros(b), 3 * B, np.zeros(b))
+    cfg = synth.get_config("tiny_f32")
+    W = O.Weights64(synth.make_weights(cfg), cfg)
+    T = cfg.ctx[1]
+    taps = synth.make_tap_hiddens(cfg, T)
+    inj = O.inject_kv_requests(taps, np.array([0, T]), np.array([0]), W, cfg)
+    caches = [(inj[(l, 0)][1], inj[(l, 0)][2]) for l in range(cfg.L)]
+    toks, q, rec = O.sampled_draft.sampled_draft_block(5, T, caches, W, cfg, 0.9, seed, offset, 0,
+                                                       steps=2)
+    return {
+        "verify_accept": [int(a) for a in res["accept"]],
+        "verify_next_anchor": [int(t) for t in res["next_anchor"]],
+        "verify_log_rho_first": [float(d["log_rho"][0]) for d in res["detail"]],
+        "draft_tokens": [int(t) for t in toks],
+        "draft_commit": [r["commit"] for r in rec],
+        "draft_conf_step0": [float(x) for x in rec[0]["conf"]],
+    }
+
+
 if __name__ == "__main__":
     out = tiny_case()
     with open(os.path.join(HERE, "tiny_f32_oracle.json"), "w") as f:
+        json.dump(out, f, indent=1)
+    print(json.dumps(out))
+    out = sampled_case()
+    with open(os.path.join(HERE, "sampled_oracle.json"), "w") as f:
         json.dump(out, f, indent=1)
     print(json.dumps(out))

@@ -6,7 +6,7 @@ import os
 import pytest
 
 import synth
-from tests.golden.make_golden import tiny_case
+from tests.golden.make_golden import sampled_case, tiny_case
 
 G = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
@@ -44,3 +44,12 @@ def test_oracle_regression_record():
     assert got["verify_emitted"] == want["verify_emitted"]
     assert got["draft_margins"] == pytest.approx(want["draft_margins"], rel=1e-12)
     assert got["k_cache_l0_pos5_head0"] == pytest.approx(want["k_cache_l0_pos5_head0"], rel=1e-12)
+
+
+def test_sampled_oracle_regression_record():
+    want = _load("sampled_oracle.json")
+    got = sampled_case()
+    for k in ("verify_accept", "verify_next_anchor", "draft_tokens", "draft_commit"):
+        assert got[k] == want[k], k
+    assert got["verify_log_rho_first"] == pytest.approx(want["verify_log_rho_first"], rel=1e-12)
+    assert got["draft_conf_step0"] == pytest.approx(want["draft_conf_step0"], rel=1e-12)
