@@ -306,7 +306,13 @@ def test_draft_block_one_commit_per_step_when_steps_is_block_minus_one():
     toks, rec = O.draft_block(7, 3, caches, W, cfg, steps=3)
     assert [len(r["commit"]) for r in rec] == [1, 1, 1]
     committed = sorted(p for r in rec for p in r["commit"])
-    assert committed == [1, 2, 3] and cfg.mask_id not in list(toks[1:]) or True
+    assert committed == [1, 2, 3]
+    # each position holds the argmax that its committing step computed for it (the
+    # argmax is not restricted, so [MASK] itself may legitimately be drafted)
+    for r in rec:
+        idx = {p: i for i, p in enumerate(r["stats"]["pos"])}
+        for p in r["commit"]:
+            assert int(toks[p]) == int(r["stats"]["tok"][idx[p]])
     # the first commit is the most confident position of the all-mask forward
     st0 = rec[0]["stats"]
     best = st0["pos"][int(np.argmax(st0["conf"]))]
@@ -389,3 +395,61 @@ def test_verify_capacity_and_range_errors_write_nothing():
         assert r["status"][1] == O.VERIFY_OUT_CAP
         assert list(r["out_tokens"][1]) == [-7] * 4 and r["seq_lens"][1] == 10
     assert r["status"][0] == O.VERIFY_OK and r["out_len"][0] == r["accept"][0] + 1
+
+
+# ---------------------------------------------------------------- multi-step drafting, brute force
+
+def _bf_weights(w):
+    return {"emb": nested(w["emb"]), "g_final": nested(w["g_final"]), "W_lm": nested(w["W_lm"]),
+            "layers": [{k: nested(v) for k, v in lw.items()} for lw in w["layers"]]}
+
+
+def _bf_draft(anchor, T, bf_caches, wn, cfg, steps):
+    """Denoising by hand on the loop-based forward: every step reruns the whole block
+    with the tokens committed so far, scores each still-masked position by its
+    softmax max-probability, and commits the ceil(remaining / steps left) best
+    (ties to the lower position) to their argmax.  Returns the tokens and, per
+    step, (committed positions, {position: argmax of that step})."""
+    B = cfg.B
+    toks = [anchor] + [cfg.mask_id] * (B - 1)
+    masked = list(range(1, B))
+    steps_log = []
+    for t in range(steps):
+        logits = BF.forward_logits(toks, T, bf_caches, wn, cfg)
+        score = {}
+        for p in masked:
+            row = logits[p]
+            mx = max(row)
+            score[p] = (1.0 / sum(math.exp(v - mx) for v in row), BF.argmax_first(row))
+        left = steps - t
+        k = (len(masked) + left - 1) // left
+        ranked = sorted(masked, key=lambda p: (-score[p][0], p))
+        commit = sorted(ranked[:k])
+        for p in commit:
+            toks[p] = score[p][1]
+        steps_log.append((commit, {p: score[p][1] for p in masked}))
+        masked = [p for p in masked if p not in commit]
+    return toks, steps_log
+
+
+@pytest.mark.parametrize("steps", [2, 3])
+def test_multi_step_draft_matches_bruteforce(steps):
+    cfg = MICRO.replace(B=4)
+    w = micro_weights(cfg)
+    W = O.Weights64(w, cfg)
+    wn = _bf_weights(w)
+    T = 3
+    saw_changed_argmax = False
+    for anchor, seed in ((7, 11), (3, 12), (12, 13), (0, 14)):
+        caches = _micro_caches(cfg, T, seed=seed)
+        bf_caches = [(K.tolist(), V.tolist()) for K, V in caches]
+        want, log = _bf_draft(anchor, T, bf_caches, wn, cfg, steps)
+        got, rec = O.draft_block(anchor, T, caches, W, cfg, steps=steps)
+        assert [int(v) for v in got] == want
+        assert [r["commit"] for r in rec] == [c for c, _ in log]
+        # a later step re-predicts the positions still masked: somewhere its argmax
+        # differs from the first step's, so committing a stale argmax would fail here
+        for t in range(1, steps):
+            for p, tok in log[t][1].items():
+                saw_changed_argmax |= tok != log[0][1][p]
+    assert saw_changed_argmax
