@@ -85,3 +85,14 @@ def test_roofline_times_are_the_slower_resource(cyc):
     assert out["gemm"]["flops"] == fl
     total_ms = sum(c["roof_s"] for c in out.values()) * 1e3
     assert 1.4 < total_ms < 1.8  # the cycle roofline quoted with the bench (1.595 ms)
+
+
+def test_tensor_peak_follows_the_sampled_clock():
+    # near max clock: the burst figure; a clock lowered by the power cap: sustained
+    assert bench.tensor_peak(PEAKS, {"sm_mhz": 1897.5, "sm_max_mhz": 1965.0}) == (1644.9, "burst")
+    assert bench.tensor_peak(PEAKS, {"sm_mhz": 1350.0, "sm_max_mhz": 1965.0}) == (
+        1403.3, "sustained")
+    # no clock samples: the conservative sustained figure
+    assert bench.tensor_peak(PEAKS, {"sm_mhz": None, "sm_max_mhz": None})[1] == "sustained"
+    # no sustained figure measured: burst
+    assert bench.tensor_peak({"bf16_tflops": 1590.0}, {})[1] == "burst"
