@@ -25,3 +25,20 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """Writes the parity figures the GPU tests collected (near-tie counts, largest
+    relative errors per test) to the JSON file DFLASH_PARITY_RECORD names."""
+    path = os.environ.get("DFLASH_PARITY_RECORD")
+    if not path:
+        return
+    mod = sys.modules.get("tests.gpu_common")
+    rec = getattr(mod, "RECORD", None) if mod else None
+    if not rec:
+        return
+    import json
+
+    with open(path, "w") as f:
+        json.dump({"exitstatus": int(exitstatus), "tests": rec}, f, indent=1, sort_keys=True)
+        f.write("\n")

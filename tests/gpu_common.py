@@ -65,12 +65,36 @@ def rel_err(gpu, ref) -> float:
     return float(np.abs(gpu - ref).max() / (den if den > 0 else 1.0))
 
 
+# Per-test parity figures (near-tie counts, largest relative errors) collected
+# during a run; tests/conftest.py writes them as JSON at the end of the session
+# when DFLASH_PARITY_RECORD names a file.
+RECORD = {}
+
+
+def record(test: str, **fields):
+    ent = RECORD.setdefault(test, {})
+    for k, v in fields.items():
+        if isinstance(v, (int, float)) and k.startswith("max_") and k in ent:
+            ent[k] = max(ent[k], v)
+        elif isinstance(v, int) and k in ent and not k.startswith("max_"):
+            ent[k] += v
+        else:
+            ent[k] = v
+
+
 class DraftReport:
     def __init__(self):
         self.token_near_ties = 0
         self.commit_near_ties = 0
         self.positions = 0
         self.max_logit_rel = 0.0
+
+    def save(self, test: str, **extra):
+        """Adds this report's counts to the session's parity record under `test`."""
+        record(test, positions=self.positions, token_near_ties=self.token_near_ties,
+               commit_near_ties=self.commit_near_ties, max_logit_rel=self.max_logit_rel,
+               **extra)
+        return self
 
     def __repr__(self):
         return (f"positions={self.positions} token_near_ties={self.token_near_ties} "

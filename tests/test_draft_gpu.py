@@ -37,7 +37,7 @@ def _run_draft(b, cfg, steps=None, dbg=True, ctx=None, anchors=None):
                 lg=lg, err=D.get_error(ws))
 
 
-def _check(b, cfg, res, steps, requests):
+def _check(b, cfg, res, steps, requests, test=None):
     rep = DraftReport()
     for r in requests:
         T = int(res["ctx"][r])
@@ -49,6 +49,8 @@ def _check(b, cfg, res, steps, requests):
         check_draft_request(b, r, int(res["anchors"][r]), T, caches, res["out"][r],
                             res["cst"][r], glog, steps, rep)
         assert int(res["cst"][r][0]) == -1
+    if test:
+        rep.save(test, config=cfg.name, requests=len(list(requests)))
     return rep
 
 
@@ -58,7 +60,7 @@ def test_draft_tiny(dtype):
     b = built(cfg)
     res = _run_draft(b, cfg)
     assert res["err"] == 0
-    rep = _check(b, cfg, res, cfg.steps, range(cfg.batch))
+    rep = _check(b, cfg, res, cfg.steps, range(cfg.batch), test=f"draft_tiny[{dtype}]")
     if dtype == "f32":
         assert rep.max_logit_rel < 1e-5 and rep.token_near_ties == 0
     print(rep)
@@ -70,7 +72,7 @@ def test_draft_tiny_bf16_denoising_steps(steps):
     b = built(cfg)
     res = _run_draft(b, cfg, steps=steps)
     assert res["err"] == 0
-    print(_check(b, cfg, res, steps, range(cfg.batch)))
+    print(_check(b, cfg, res, steps, range(cfg.batch), test=f"draft_tiny_bf16_steps[{steps}]"))
 
 
 @pytest.mark.parametrize("B,steps", [(8, 2), (16, 1), (4, 3)])
@@ -81,7 +83,7 @@ def test_draft_small_8b_geometry(B, steps):
     b = built(cfg)
     res = _run_draft(b, cfg)
     assert res["err"] == 0
-    print(_check(b, cfg, res, steps, range(cfg.batch)))
+    print(_check(b, cfg, res, steps, range(cfg.batch), test=f"draft_small_8b[B{B},s{steps}]"))
 
 
 def test_draft_context_lengths_edge_cases():
@@ -93,7 +95,7 @@ def test_draft_context_lengths_edge_cases():
     ctx = torch.tensor([0, 1, 256, b.cap - cfg.B], dtype=torch.int32)
     res = _run_draft(b, cfg, ctx=ctx)
     assert res["err"] == 0
-    print(_check(b, cfg, res, cfg.steps, range(cfg.batch)))
+    print(_check(b, cfg, res, cfg.steps, range(cfg.batch), test="draft_context_edge_cases"))
 
 
 @pytest.mark.parametrize("chunk", [64, 192, 4096])
@@ -111,7 +113,8 @@ def test_draft_attention_chunk_sizes(chunk):
     finally:
         D.debug_attn_chunk(0)
     assert res["err"] == 0
-    print(chunk, _check(b, cfg, res, cfg.steps, range(cfg.batch)))
+    print(chunk, _check(b, cfg, res, cfg.steps, range(cfg.batch),
+                        test=f"draft_attention_chunk[{chunk}]"))
 
 
 def test_draft_rejects_bad_requests_without_writing():
@@ -141,4 +144,4 @@ def test_draft_full_size_sampled_requests(name, requests):
     out = res["out"]
     assert (out[:, 1:] >= 0).all() and (out[:, 1:] < cfg.V).all()
     assert (res["cst"][:, 1:] >= 0).all() and (res["cst"][:, 1:] < cfg.steps).all()
-    print(name, _check(b, cfg, res, cfg.steps, requests))
+    print(name, _check(b, cfg, res, cfg.steps, requests, test=f"draft_full_size[{name}]"))

@@ -8,7 +8,8 @@ import torch
 import oracle as O
 import synth
 from synth.configs import shrink
-from tests.gpu_common import built, rel_err, REL_TOL
+from tests.gpu_common import (DraftReport, built, check_draft_request, oracle_caches_from,
+                              record, rel_err, REL_TOL)
 from block_diffusion_speculative_gemm_b200 import dflash as D
 
 pytestmark = pytest.mark.gpu
@@ -28,7 +29,7 @@ def _inject(b, cfg, mode, rows_check=None, cap=None):
     return ctx, cu, st, n, taps, kc, vc, ws
 
 
-def _check_rows(b, cfg, cu, st, taps, kc, vc, rows):
+def _check_rows(b, cfg, cu, st, taps, kc, vc, rows, test=None):
     """Oracle K/V for the given packed rows, compared per layer."""
     cu_np = cu.numpy()
     sub_taps = [t[rows] for t in taps]
@@ -44,6 +45,8 @@ def _check_rows(b, cfg, cu, st, taps, kc, vc, rows):
         ek, ev = rel_err(gk, K), rel_err(gv, V)
         worst = max(worst, ek, ev)
         assert ek <= REL_TOL and ev <= REL_TOL, (l, ek, ev)
+    if test:
+        record(test, config=cfg.name, rows_checked=len(rows), max_kv_rel=worst)
     return worst
 
 
@@ -53,7 +56,8 @@ def test_inject_tiny_prefill(name, dtype):
     b = built(cfg)
     ctx, cu, st, n, taps, kc, vc, ws = _inject(b, cfg, "prefill")
     assert D.get_error(ws) == 0
-    worst = _check_rows(b, cfg, cu, st, taps, kc, vc, np.arange(n))
+    worst = _check_rows(b, cfg, cu, st, taps, kc, vc, np.arange(n),
+                        test=f"inject_tiny_prefill[{dtype}]")
     if dtype == "f32":
         assert worst < 1e-5
     # positions past the injected rows stay untouched
@@ -76,7 +80,7 @@ def test_inject_qwen3_8b_steady_state_full_size():
     ctx, cu, st, n, taps, kc, vc, ws = _inject(b, cfg, "steady")
     assert 32 <= n <= 32 * cfg.B
     assert D.get_error(ws) == 0
-    _check_rows(b, cfg, cu, st, taps, kc, vc, np.arange(n))
+    _check_rows(b, cfg, cu, st, taps, kc, vc, np.arange(n), test="inject_qwen3_8b_steady")
 
 
 def test_inject_qwen3_4b_prefill_sampled_rows():
@@ -85,7 +89,7 @@ def test_inject_qwen3_4b_prefill_sampled_rows():
     ctx, cu, st, n, taps, kc, vc, ws = _inject(b, cfg, "prefill")
     assert D.get_error(ws) == 0
     rows = np.unique(np.concatenate([np.arange(0, n, 97), [n - 1]]))
-    _check_rows(b, cfg, cu, st, taps, kc, vc, rows)
+    _check_rows(b, cfg, cu, st, taps, kc, vc, rows, test="inject_qwen3_4b_prefill_sampled")
 
 
 def test_inject_chunks_equal_one_call():
@@ -110,9 +114,20 @@ def test_inject_chunks_equal_one_call():
                     torch.tensor([32 * half, 32 * half], dtype=torch.int32).cuda(), kc2, vc2, ws)
     torch.cuda.synchronize()
     assert D.get_error(ws) == 0
-    scale = kc1.float().abs().max().item()
-    assert (kc1.float() - kc2.float()).abs().max().item() <= 1e-2 * scale
-    assert (vc1.float() - vc2.float()).abs().max().item() <= 1e-2 * vc1.float().abs().max().item()
+    # Not bit-identical by design: the GEMM picks its K split count from the row
+    # count and starts each CTA's K walk at a CTA-dependent offset (to spread the
+    # SMs' L2 requests), so the fp32 accumulation order depends on how the rows are
+    # batched.  What remains is fp32 reassociation plus at most a unit or two in the
+    # last place of the fp16 features and cache entries: far inside the 1e-2
+    # tolerance, and asserted at 2e-3 of the largest entry.
+    worst = 0.0
+    for a, c in ((kc1, kc2), (vc1, vc2)):
+        diff = (a.float() - c.float()).abs().max().item()
+        worst = max(worst, diff / a.float().abs().max().item())
+    record("inject_chunks_vs_one_call", max_rel_diff=worst,
+           identical_fraction=float(((kc1 == kc2).float().mean().item() +
+                                     (vc1 == vc2).float().mean().item()) / 2))
+    assert worst <= 2e-3, worst
 
 
 def test_inject_past_capacity_sets_error_and_skips():
@@ -132,3 +147,78 @@ def test_inject_past_capacity_sets_error_and_skips():
     assert kc[:, 0, :, 10:14].abs().max().item() > 0
     assert kc[:, 1, :, 46:48].abs().max().item() > 0
     assert kc[:, 0, :, :10].abs().max().item() == 0 and kc[:, 0, :, 14:].abs().max().item() == 0
+
+
+def test_inject_qwen3_8b_ctx32k_full_prefix_then_draft():
+    """The long-context workload as it runs: 4 requests x 32768 positions injected in
+    one call (131072 rows, the tensor-bound GEMMs at full length, processed in
+    16384-row chunks), then one block forward over that injected cache.
+
+    Injection: 512 seeded random positions per request plus the first and the last,
+    every layer, K and V, against the oracle's injection of the same tapped rows.
+    Draft: requests 0 and 3 over the cache as injected (the oracle reads the same
+    fp16 values), with the draft tolerances."""
+    cfg = synth.get_config("qwen3_8b_ctx32k")
+    b = built(cfg)
+    dev = torch.device("cuda")
+    ctx = synth.make_ctx_lens(cfg)
+    cu, st, n = synth.make_inject_layout(cfg, ctx, "prefill")
+    assert n == 4 * 32768
+    # 5.4 GB of tapped states: drawn on the device from a seeded generator; the
+    # oracle reads the sampled rows of the same buffers
+    gen = torch.Generator(device=dev).manual_seed(synth.sub_seed(0x5EED, cfg.name, "prefix"))
+    taps = [(torch.randn((n, cfg.H_t), generator=gen, device=dev) * cfg.h_std).to(torch.bfloat16)
+            for _ in range(cfg.n_tap)]
+    kc = torch.zeros((cfg.L, cfg.batch, cfg.nkv, b.cap, cfg.hd), dtype=b.model.cache_dtype,
+                     device=dev)
+    vc = torch.zeros_like(kc)
+    ws = b.model.workspace(cfg.batch, cfg.B, n)
+    D.inject_kv(b.model, taps, cu.to(dev), st.to(dev), kc, vc, ws)
+    torch.cuda.synchronize()
+    assert D.get_error(ws) == 0
+    rng = np.random.default_rng(synth.sub_seed(0x5EED, cfg.name, "sample_rows"))
+    rows = []
+    for r in range(cfg.batch):
+        lo, hi = int(cu[r]), int(cu[r + 1])
+        pick = rng.choice(np.arange(lo + 1, hi - 1), size=512, replace=False)
+        rows.append(np.concatenate([[lo], np.sort(pick), [hi - 1]]))
+    rows = np.concatenate(rows)
+    idx = torch.as_tensor(rows, device=dev)
+    host_taps = [t.index_select(0, idx).cpu() for t in taps]
+    del taps
+    # _check_rows indexes the taps by packed row: hand it a sparse view
+    sparse = [_RowsView(rows, h) for h in host_taps]
+    _check_rows(b, cfg, cu, st, sparse, kc, vc, rows, test="inject_qwen3_8b_ctx32k_prefill")
+    # positions past the contexts stay untouched
+    assert kc[:, :, :, 32768:, :].abs().max().item() == 0.0
+
+    # one block forward over the injected cache
+    anchors = synth.make_anchors(cfg)
+    out = torch.full((cfg.batch, cfg.B), -5, dtype=torch.int32, device=dev)
+    cst = torch.full((cfg.batch, cfg.B), -5, dtype=torch.int32, device=dev)
+    lg = torch.full((1, cfg.batch, cfg.B, cfg.V), float("nan"), device=dev)
+    wsd = b.model.workspace(cfg.batch, cfg.B, 0)
+    D.draft_block(b.model, anchors.to(dev), ctx.to(dev), kc, vc, cfg.B, 1, out, wsd,
+                  commit_step=cst, logits_dbg=lg)
+    torch.cuda.synchronize()
+    assert D.get_error(wsd) == 0
+    rep = DraftReport()
+    for r in (0, 3):
+        caches = oracle_caches_from(kc, vc, cfg.L, r, int(ctx[r]))
+        glog = [{p: lg[0, r, p].cpu().numpy() for p in range(1, cfg.B)}]
+        check_draft_request(b, r, int(anchors[r]), int(ctx[r]), caches, out[r].cpu(),
+                            cst[r].cpu(), glog, 1, rep)
+    rep.save("draft_over_injected_ctx32k", config=cfg.name, requests=2)
+    print(rep)
+
+
+class _RowsView:
+    """Rows `rows` of a packed [n_rows, H] tensor, held sparsely: indexing with
+    those packed row numbers returns the matching host rows."""
+
+    def __init__(self, rows, data):
+        self.pos = {int(r): i for i, r in enumerate(rows)}
+        self.data = data
+
+    def __getitem__(self, rows):
+        return self.data[[self.pos[int(r)] for r in rows]]

@@ -86,3 +86,24 @@ def test_noalloc_reports_device_errors_and_rejects_oversize():
     p = ctypes.c_void_p(case["logits"].cuda().data_ptr())
     st = L.dflash_verify_noalloc(p, D.BF16, p, 2100, 16, V, p, p, 8, p, p, p, None, None)
     assert st == D.ESCRATCH  # 33600 rows > 32768
+
+
+def test_noalloc_allocates_nothing():
+    """After a first call (which may load the module that holds the fixed array),
+    further calls at the largest parametrised shape leave the device's free memory
+    unchanged: no call allocates device memory."""
+    b, B, V = 128, 16, 151936
+    n_calls = 5
+    case = synth.make_verify_case(b, B, V, "noalloc_mem", plant=("geometric", 4.0))
+    logits, draft = case["logits"].cuda(), case["draft"].cuda()
+    o = _buffers(b, B, (n_calls + 1) * B, torch.full((b,), 11, dtype=torch.int32))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _noalloc_abi(logits, draft, o, err)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(n_calls):
+        _noalloc_abi(logits, draft, o, err)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert int(err.item()) == 0
+    assert (o["out_len"].cpu() > n_calls).all()
