@@ -231,12 +231,12 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct DraftLayout {
   size_t tokens, zrow, lm_rows, cstep, req_valid, lm_tok, lm_conf, x, h, q, kb, vb, o, act, part,
-      attn_o, attn_ml, stats, logits, end;
+      attn_o, attn_ml, stats, draw, logits, end;
   size_t part_elems;  // fp32 elements of split-K partials
 };
 
 struct InjectLayout {
-  size_t c, u, part, end;
+  size_t c, u, part, req_ok, end;
   size_t part_elems;
   int chunk_rows;
 };
@@ -277,12 +277,17 @@ DraftLayout draft_layout(const dflash_config& c, int batch, int B) {
   L.attn_o = take(4 * arows * c.head_dim);
   L.attn_ml = take(8 * arows);
   L.stats = take(sizeof(LmStat) * M * n_vt);
+  // sampled drafting's draw partials: rows x chunks never exceeds M + 600 (the
+  // chunk count falls as the row count grows)
+  L.draw = take(std::max(sampled_draw_part_bytes((int)M, sampled_draw_chunks((int)M, c.vocab)),
+                         sampled_draw_part_bytes((int)M + 600, 1)));
   L.logits = c.dtype == DFLASH_F32 ? take(4 * M * (size_t)c.vocab) : off;
   L.end = off;
   return L;
 }
 
-InjectLayout inject_layout(const dflash_config& c, int max_rows) {
+// batch: requests of a paged injection (one page-check flag each), 0 otherwise.
+InjectLayout inject_layout(const dflash_config& c, int max_rows, int batch = 0) {
   InjectLayout L{};
   const size_t esz = c.dtype == DFLASH_BF16 ? 2 : 4;
   L.chunk_rows = std::min(std::max(max_rows, 1), kInjectChunkRows);
@@ -297,6 +302,8 @@ InjectLayout inject_layout(const dflash_config& c, int max_rows) {
   L.part_elems = (n <= 256 ? (size_t)kMaxSplits : 1) * n * ncol;
   L.part = off;
   off = align256(off + 4 * L.part_elems);
+  L.req_ok = off;
+  off = align256(off + 4 * (size_t)std::max(batch, 0));
   L.end = off;
   return L;
 }
@@ -503,7 +510,8 @@ extern "C" size_t dflash_workspace_size(const dflash_model* m, int max_batch, in
     s = std::max(s, draft_layout(m->cfg, max_batch, B).end);
     s = std::max(s, verify_bytes(max_batch, B, m->cfg.vocab));
   }
-  if (max_inject_rows > 0) s = std::max(s, inject_layout(m->cfg, max_inject_rows).end);
+  if (max_inject_rows > 0)
+    s = std::max(s, inject_layout(m->cfg, max_inject_rows, std::max(max_batch, 0)).end);
   return s;
 }
 
@@ -531,24 +539,25 @@ extern "C" int dflash_get_error(void* ws, void* stream, int32_t* bits) {
 }
 
 // ============================================================== inject
-extern "C" int dflash_inject_kv(const dflash_model* m, const void* const* taps,
-                                const int32_t* cu_rows, const int32_t* start_pos, int batch,
-                                int n_rows, void* k_cache, void* v_cache, int cache_cap, void* ws,
-                                size_t ws_bytes, void* stream) {
-  if (!m || batch < 1 || n_rows < 0 || cache_cap < 1) return DFLASH_EINVAL;
-  if (n_rows == 0) return DFLASH_OK;
+namespace {
+
+// Injection into the contiguous cache (pg.table == nullptr) or into paged
+// pools; `cap` is the positions a request can hold.
+int inject_impl(const dflash_model* m, const void* const* taps, const int32_t* cu_rows,
+                const int32_t* start_pos, int batch, int n_rows, void* k_cache, void* v_cache,
+                int cache_cap, KvPages pg, void* ws, cudaStream_t s) {
   const dflash_config& c = m->cfg;
-  if (!taps || !cu_rows || !start_pos || !k_cache || !v_cache || !ws) return DFLASH_EINVAL;
-  for (int t = 0; t < c.n_tap; ++t)
-    if (!taps[t] || !aligned16(taps[t])) return DFLASH_EINVAL;
-  if (!aligned16(k_cache) || !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(ws) & 255))
-    return DFLASH_EINVAL;
-  const InjectLayout L = inject_layout(c, n_rows);
-  if (ws_bytes < L.end) return DFLASH_EWORKSPACE;
-  cudaStream_t s = (cudaStream_t)stream;
+  const InjectLayout L = inject_layout(c, n_rows, pg.table ? batch : 0);
   int32_t* err = err_word(ws);
   const int kvN = c.n_layers * 2 * c.n_kv * c.head_dim;
   const size_t e = m->esz;
+  if (pg.table != nullptr) {
+    pg.req_ok = at<int32_t>(ws, L.req_ok);
+    launch_inject_page_check(cu_rows, start_pos, batch, pg, at<int32_t>(ws, L.req_ok), err, s);
+  }
+  const int64_t kv_ls = pg.table ? (int64_t)pg.n_pages * c.n_kv * pg.page
+                                 : (int64_t)batch * c.n_kv * cache_cap;
+  const int64_t kv_hs = pg.table ? pg.page : cache_cap;
   for (int r0 = 0; r0 < n_rows; r0 += L.chunk_rows) {
     const int n = std::min(L.chunk_rows, n_rows - r0);
     const void* seg[kMaxSeg];
@@ -589,6 +598,9 @@ extern "C" int dflash_inject_kv(const dflash_model* m, const void* const* taps,
         o2.batch = batch;
         o2.cap = cache_cap;
         o2.max_pos = c.max_pos;
+        o2.pages = pg;
+        o2.kv_ls = kv_ls;
+        o2.kv_hs = kv_hs;
       } else {
         o2.part = part;
       }
@@ -596,7 +608,7 @@ extern "C" int dflash_inject_kv(const dflash_model* m, const void* const* taps,
       if (st) return st;
       if (s2 > 1)
         launch_kv_scatter<__half>(part, s2, n, r0, c.n_layers, c.n_kv, c.head_dim, cu_rows,
-                                  start_pos, batch, cache_cap, m->rope_cos, m->rope_sin,
+                                  start_pos, batch, cache_cap, pg, m->rope_cos, m->rope_sin,
                                   c.max_pos, static_cast<__half*>(k_cache),
                                   static_cast<__half*>(v_cache), err, s);
     } else {
@@ -608,23 +620,94 @@ extern "C" int dflash_inject_kv(const dflash_model* m, const void* const* taps,
       const float* cseg[1] = {static_cast<const float*>(cbuf)};
       gemm_simt_f32(static_cast<const float*>(m->W_kv), kvN, c.d, cseg, 1, c.d, n, part, s);
       launch_kv_scatter<float>(part, 1, n, r0, c.n_layers, c.n_kv, c.head_dim, cu_rows,
-                               start_pos, batch, cache_cap, m->rope_cos, m->rope_sin, c.max_pos,
-                               static_cast<float*>(k_cache), static_cast<float*>(v_cache), err, s);
+                               start_pos, batch, cache_cap, pg, m->rope_cos, m->rope_sin,
+                               c.max_pos, static_cast<float*>(k_cache),
+                               static_cast<float*>(v_cache), err, s);
     }
     if ((st = cuda_status())) return st;
   }
   return DFLASH_OK;
 }
 
+// Host checks of a paged K/V description shared by the paged calls.
+int check_pages(const dflash_model* m, const void* k_pool, const void* v_pool, int n_pages,
+                int page_size, const int32_t* page_table, int max_pages) {
+  const dflash_config& c = m->cfg;
+  if (!k_pool || !v_pool || !page_table || n_pages < 1 || max_pages < 1 || page_size < 1)
+    return DFLASH_EINVAL;
+  if (!aligned16(k_pool) || !aligned16(v_pool)) return DFLASH_EINVAL;
+  if (c.dtype != DFLASH_BF16) return DFLASH_EUNSUPPORTED;  // the tensor-core attention only
+  if (page_size % 64 != 0) return DFLASH_EUNSUPPORTED;     // whole 64-key attention tiles
+  if ((int64_t)c.n_layers * n_pages * c.n_kv * page_size > 0x7fffffffLL)
+    return DFLASH_EUNSUPPORTED;
+  if ((int64_t)max_pages * page_size > 0x7fffffffLL) return DFLASH_EUNSUPPORTED;
+  return DFLASH_OK;
+}
+
+}  // namespace
+
+extern "C" int dflash_inject_kv(const dflash_model* m, const void* const* taps,
+                                const int32_t* cu_rows, const int32_t* start_pos, int batch,
+                                int n_rows, void* k_cache, void* v_cache, int cache_cap, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (!m || batch < 1 || n_rows < 0 || cache_cap < 1) return DFLASH_EINVAL;
+  if (n_rows == 0) return DFLASH_OK;
+  const dflash_config& c = m->cfg;
+  if (!taps || !cu_rows || !start_pos || !k_cache || !v_cache || !ws) return DFLASH_EINVAL;
+  for (int t = 0; t < c.n_tap; ++t)
+    if (!taps[t] || !aligned16(taps[t])) return DFLASH_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return DFLASH_EINVAL;
+  if (ws_bytes < inject_layout(c, n_rows).end) return DFLASH_EWORKSPACE;
+  return inject_impl(m, taps, cu_rows, start_pos, batch, n_rows, k_cache, v_cache, cache_cap,
+                     KvPages{}, ws, (cudaStream_t)stream);
+}
+
+extern "C" int dflash_inject_kv_paged(const dflash_model* m, const void* const* taps,
+                                      const int32_t* cu_rows, const int32_t* start_pos,
+                                      int batch, int n_rows, void* k_pool, void* v_pool,
+                                      int n_pages, int page_size, const int32_t* page_table,
+                                      int max_pages, void* ws, size_t ws_bytes, void* stream) {
+  if (!m || batch < 1 || n_rows < 0) return DFLASH_EINVAL;
+  if (n_rows == 0) return DFLASH_OK;
+  const dflash_config& c = m->cfg;
+  if (!taps || !cu_rows || !start_pos || !ws) return DFLASH_EINVAL;
+  for (int t = 0; t < c.n_tap; ++t)
+    if (!taps[t] || !aligned16(taps[t])) return DFLASH_EINVAL;
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return DFLASH_EINVAL;
+  int st = check_pages(m, k_pool, v_pool, n_pages, page_size, page_table, max_pages);
+  if (st) return st;
+  if (ws_bytes < inject_layout(c, n_rows, batch).end) return DFLASH_EWORKSPACE;
+  KvPages pg;
+  pg.table = page_table;
+  pg.max_pages = max_pages;
+  pg.page = page_size;
+  pg.n_pages = n_pages;
+  return inject_impl(m, taps, cu_rows, start_pos, batch, n_rows, k_pool, v_pool,
+                     max_pages * page_size, pg, ws, (cudaStream_t)stream);
+}
+
 // ============================================================== draft
 namespace {
 
+// Sampled drafting: temperature, Philox key and offset, and the caller's
+// draft-logits output (fp32 or bf16 [batch, B, V]).
+struct SampleArgs {
+  float tau;
+  uint64_t seed, offset;
+  void* q;
+  int q_bf16;
+};
+
 // T: activation / GEMM operand type; TC: K/V cache type; TE: embedding type.
+// samp == nullptr: greedy drafting (argmax, max-probability confidence).
+// pg.table set: the context is read from paged pools, cap = positions per
+// request (the RoPE bound on ctx_len + B).
 template <typename T, typename TC, typename TE>
 int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_len,
-               const void* k_cache, const void* v_cache, int cap, int batch, int B, int n_steps,
-               int32_t* draft_tokens, int32_t* commit_step, float* logits_dbg, void* ws,
-               cudaStream_t s) {
+               const void* k_cache, const void* v_cache, int cap, const KvPages& pg, int batch,
+               int B, int n_steps, int32_t* draft_tokens, int32_t* commit_step, float* logits_dbg,
+               const SampleArgs* samp, void* ws, cudaStream_t s) {
   const dflash_config& c = m->cfg;
   const DraftLayout L = draft_layout(c, batch, B);
   const int M = batch * B;
@@ -666,7 +749,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
     chunk = g_attn_chunk;
   const int n_chunks = (cap + B + chunk - 1) / chunk;
 
-  launch_draft_init(anchor, ctx_len, batch, B, c.vocab, c.mask_id, cap, tokens, zrow, lm_rows,
+  launch_draft_init(anchor, ctx_len, batch, B, c.vocab, c.mask_id, cap, pg, tokens, zrow, lm_rows,
                     cstep, valid, err, s);
   auto gemm = [&](const WeightMap& W, const void* wptr, int N, int K, const T* X, float* out,
                   size_t cap_elems, int* splits_out) -> int {
@@ -723,7 +806,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
         if (sp > 1)
           launch_qkv_post<T>(part, sp, M, B, ctx_len, valid, nq, nkv, hd, m->rope_cos,
                              m->rope_sin, q, kb, vb, s);
-        if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, l, c.n_layers, batch, cap,
+        if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, pg, l, c.n_layers, batch, cap,
                                                 ctx_len, valid, B, nq, nkv, hd, attn_o, attn_ml,
                                                 n_chunks, chunk, o, attn_cnt, err, s)))
           return st;
@@ -743,9 +826,9 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
       if ((st = gemm(P.mqkv, P.Wqkv, qkv_out(c), c.d, h, part, L.part_elems, &sp))) return st;
       launch_qkv_post<T>(part, sp, M, B, ctx_len, valid, nq, nkv, hd, m->rope_cos, m->rope_sin,
                          q, kb, vb, s);
-      if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, l, c.n_layers, batch, cap, ctx_len,
-                                              valid, B, nq, nkv, hd, attn_o, attn_ml, n_chunks,
-                                              chunk, o, attn_cnt, err, s)))
+      if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, pg, l, c.n_layers, batch, cap,
+                                              ctx_len, valid, B, nq, nkv, hd, attn_o, attn_ml,
+                                              n_chunks, chunk, o, attn_cnt, err, s)))
         return st;
       if ((st = gemm(P.mo, P.Wo, c.d, nq * hd, o, part, L.part_elems, &sp))) return st;
       launch_residual_norm<T>(part, sp, M, c.d, x, P.g_post, h, nullptr, c.eps, s);
@@ -754,15 +837,28 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
       if ((st = gemm(P.md, P.Wd, c.d, c.inter, act, part, L.part_elems, &sp))) return st;
       launch_residual_norm<T>(part, sp, M, c.d, x, g_next, h, next_rows, c.eps, s);
     }
-    // LM head over the still-masked rows (compact, request-major)
+    // LM head over the still-masked rows (compact, request-major).  Sampled
+    // drafting writes every masked row's logits into the caller's draft-logits
+    // rows (a position's row is last written at the step that commits it) and
+    // draws from them; greedy drafting reduces the tile statistics.
     const int rows = batch * rem;
-    float* dbg = logits_dbg ? logits_dbg + (size_t)t * M * c.vocab : nullptr;
+    void* dbg = logits_dbg ? logits_dbg + (size_t)t * M * c.vocab : nullptr;
+    int dbg_bf16 = 0;
+    const int32_t* dbg_valid = nullptr;
+    if (samp) {
+      dbg = samp->q;
+      dbg_bf16 = samp->q_bf16;
+      dbg_valid = valid;  // a request that writes nothing leaves its rows untouched
+    }
     if (bf16) {
       GemmOut go;
       go.stats = stats;
       go.dbg = dbg;
       go.dbg_rows = lm_rows;
       go.dbg_ld = c.vocab;
+      go.dbg_bf16 = dbg_bf16;
+      go.dbg_valid = dbg_valid;
+      go.B = B;
       const void* seg[1] = {h};
       if ((st = gemm_tc(m->mlm, seg, 1, c.d, c.d, rows, 1, EPI_LMHEAD, go, err, s))) return st;
     } else {
@@ -770,9 +866,18 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
       const float* seg[1] = {reinterpret_cast<const float*>(h)};
       gemm_simt_f32(static_cast<const float*>(m->W_lm), c.vocab, c.d, seg, 1, c.d, rows, logits,
                     s);
-      launch_lm_stats_from_logits(logits, rows, c.vocab, stats, dbg, lm_rows, c.vocab, s);
+      launch_lm_stats_from_logits(logits, rows, c.vocab, stats, dbg, lm_rows, c.vocab, dbg_bf16,
+                                  dbg_valid, B, s);
     }
-    launch_lm_reduce(stats, n_vt, rows, lm_tok, lm_conf, s);
+    if (samp) {
+      if ((st = launch_sampled_draw(samp->q, samp->q_bf16, lm_rows, valid, rows, B, c.vocab, t,
+                                    samp->tau, samp->seed, samp->offset, lm_tok, lm_conf,
+                                    at<void>(ws, L.draw), sampled_draw_chunks(rows, c.vocab),
+                                    attn_cnt, s)))
+        return st;
+    } else {
+      launch_lm_reduce(stats, n_vt, rows, lm_tok, lm_conf, s);
+    }
     launch_commit(lm_tok, lm_conf, batch, B, rem, k, t, tokens, zrow, lm_rows, cstep, s);
     rem -= k;
   }
@@ -801,10 +906,80 @@ extern "C" int dflash_draft_block(const dflash_model* m, const int32_t* anchor,
   if (ws_bytes < draft_layout(c, batch, B).end) return DFLASH_EWORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   if (c.dtype == DFLASH_BF16)
-    return draft_impl<__half, __half, __nv_bfloat16>(m, anchor, ctx_len, k_cache, v_cache, cache_cap, batch, B,
-                                     n_steps, draft_tokens, commit_step, logits_dbg, ws, s);
-  return draft_impl<float, float, float>(m, anchor, ctx_len, k_cache, v_cache, cache_cap, batch, B, n_steps,
-                           draft_tokens, commit_step, logits_dbg, ws, s);
+    return draft_impl<__half, __half, __nv_bfloat16>(m, anchor, ctx_len, k_cache, v_cache,
+                                                     cache_cap, KvPages{}, batch, B, n_steps,
+                                                     draft_tokens, commit_step, logits_dbg,
+                                                     nullptr, ws, s);
+  return draft_impl<float, float, float>(m, anchor, ctx_len, k_cache, v_cache, cache_cap,
+                                         KvPages{}, batch, B, n_steps, draft_tokens, commit_step,
+                                         logits_dbg, nullptr, ws, s);
+}
+
+extern "C" int dflash_draft_block_paged(const dflash_model* m, const int32_t* anchor,
+                                        const int32_t* ctx_len, const void* k_pool,
+                                        const void* v_pool, int n_pages, int page_size,
+                                        const int32_t* page_table, int max_pages, int batch, int B,
+                                        int n_steps, int32_t* draft_tokens, int32_t* commit_step,
+                                        float* logits_dbg, void* ws, size_t ws_bytes,
+                                        void* stream) {
+  if (!m || batch < 0 || B < 2 || B > 16 || n_steps < 1 || n_steps > B - 1) return DFLASH_EINVAL;
+  if (batch == 0) return DFLASH_OK;
+  const dflash_config& c = m->cfg;
+  if (!anchor || !ctx_len || !draft_tokens || !ws) return DFLASH_EINVAL;
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return DFLASH_EINVAL;
+  int st = check_pages(m, k_pool, v_pool, n_pages, page_size, page_table, max_pages);
+  if (st) return st;
+  if (B * (c.n_q / c.n_kv) > kAttnRows) return DFLASH_EUNSUPPORTED;
+  if ((size_t)batch * B > 65535) return DFLASH_EUNSUPPORTED;
+  if ((size_t)batch * c.n_kv * 4 > kHeader - kCntOff) return DFLASH_EUNSUPPORTED;
+  if (ws_bytes < draft_layout(c, batch, B).end) return DFLASH_EWORKSPACE;
+  KvPages pg;
+  pg.table = page_table;
+  pg.max_pages = max_pages;
+  pg.page = page_size;
+  pg.n_pages = n_pages;
+  // positions a request can reach: its table row, and the RoPE table for the block
+  const int cap = (int)std::min<int64_t>((int64_t)max_pages * page_size + B, c.max_pos);
+  return draft_impl<__half, __half, __nv_bfloat16>(m, anchor, ctx_len, k_pool, v_pool, cap, pg,
+                                                   batch, B, n_steps, draft_tokens, commit_step,
+                                                   logits_dbg, nullptr, ws, (cudaStream_t)stream);
+}
+
+extern "C" int dflash_draft_block_sampled(const dflash_model* m, const int32_t* anchor,
+                                          const int32_t* ctx_len, const void* k_cache,
+                                          const void* v_cache, int cache_cap, int batch, int B,
+                                          int n_steps, float temperature, uint64_t seed,
+                                          uint64_t offset, int32_t* draft_tokens,
+                                          int32_t* commit_step, void* draft_logits,
+                                          int draft_logits_dtype, void* ws, size_t ws_bytes,
+                                          void* stream) {
+  if (!m || batch < 0 || B < 2 || B > 16 || n_steps < 1 || n_steps > B - 1 || cache_cap < 1)
+    return DFLASH_EINVAL;
+  if (!(temperature >= 1e-4f && temperature <= 1e4f)) return DFLASH_EINVAL;
+  if (draft_logits_dtype != DFLASH_F32 && draft_logits_dtype != DFLASH_BF16) return DFLASH_EINVAL;
+  if (batch == 0) return DFLASH_OK;
+  const dflash_config& c = m->cfg;
+  if (!anchor || !ctx_len || !k_cache || !v_cache || !draft_tokens || !draft_logits || !ws)
+    return DFLASH_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(draft_logits) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255))
+    return DFLASH_EINVAL;
+  if (cache_cap > c.max_pos) return DFLASH_EINVAL;
+  if (B * (c.n_q / c.n_kv) > kAttnRows) return DFLASH_EUNSUPPORTED;
+  // one completion counter per masked row of the draw
+  if ((size_t)batch * B * 4 > kHeader - kCntOff) return DFLASH_EUNSUPPORTED;
+  if ((size_t)batch * c.n_kv * 4 > kHeader - kCntOff) return DFLASH_EUNSUPPORTED;
+  if (ws_bytes < draft_layout(c, batch, B).end) return DFLASH_EWORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  SampleArgs sa{temperature, seed, offset, draft_logits, draft_logits_dtype == DFLASH_BF16};
+  if (c.dtype == DFLASH_BF16)
+    return draft_impl<__half, __half, __nv_bfloat16>(m, anchor, ctx_len, k_cache, v_cache,
+                                                     cache_cap, KvPages{}, batch, B, n_steps,
+                                                     draft_tokens, commit_step, nullptr, &sa, ws,
+                                                     s);
+  return draft_impl<float, float, float>(m, anchor, ctx_len, k_cache, v_cache, cache_cap,
+                                         KvPages{}, batch, B, n_steps, draft_tokens, commit_step,
+                                         nullptr, &sa, ws, s);
 }
 
 // ============================================================== verify

@@ -222,7 +222,7 @@ template <int HD, int MT>
 __global__ void __launch_bounds__(kThreads)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __half* __restrict__ q, const __half* __restrict__ kb,
-                   const __half* __restrict__ vb, int layer, int batch, int cap,
+                   const __half* __restrict__ vb, const KvPages pg, int layer, int batch, int cap,
                    const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ req_valid,
                    int B, int nq, int nkv, int chunk, int n_chunks, float* __restrict__ part_o,
                    float* __restrict__ part_ml, unsigned* __restrict__ cnt,
@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kThreads)
   const int kc_end = min(k1, Tc);                       // context keys [k0, kc_end)
   const int nt = kc_end > k0 ? (kc_end - k0 + kKeys - 1) / kKeys : 0;
   const int kb_lo = max(k0, Tc), kb_hi = min(k1, Tc + B);  // block keys [kb_lo, kb_hi)
-  const int row_base = ((layer * batch + r) * nkv + g) * cap;
+  const int row_base = pg.table == nullptr ? ((layer * batch + r) * nkv + g) * cap : 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mt = warp % MT, kg = warp / MT;
   const bool computes = warp < kComputeWarps;
@@ -283,7 +283,11 @@ __global__ void __launch_bounds__(kThreads)
     const int st = t % kStages;
     const uint32_t sK = s_base + st * LY::kStage, sV = sK + LY::kTile;
     mbar_arrive_expect_tx(full(st), 2 * LY::kTile);
-    const int y = row_base + k0 + t * kKeys;
+    // the tile's first key position; a paged store finds its row through the
+    // request's page table (a tile never crosses a page)
+    const int p0 = k0 + t * kKeys;
+    const int y = pg.table == nullptr ? row_base + p0
+                                      : (int)kv_row(pg, layer, batch, r, nkv, g, cap, p0);
 #pragma unroll
     for (int h = 0; h < HALVES; ++h) {
       tma_load_2d(sK + h * kKeys * 128, &tmK, full(st), h * 64, y, policy_evict_first());
@@ -514,7 +518,8 @@ __global__ void __launch_bounds__(kThreads)
 
 template <int HD, int MT>
 int launch_cfg(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q, const __half* kb,
-               const __half* vb, int layer, int batch, int cap, const int32_t* ctx_len,
+               const __half* vb, const KvPages& pg, int layer, int batch, int cap,
+               const int32_t* ctx_len,
                const int32_t* req_valid, int B, int nq, int nkv, int chunk, int n_chunks,
                float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
                cudaStream_t s) {
@@ -524,7 +529,7 @@ int launch_cfg(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q, co
     return DFLASH_ECUDA;
   dim3 grid(n_chunks, nkv, batch);
   const cudaError_t e =
-      launch_pdl(attn_tc_kernel<HD, MT>, grid, dim3(kThreads), smem, s, 1, tk, tv, q, kb, vb,
+      launch_pdl(attn_tc_kernel<HD, MT>, grid, dim3(kThreads), smem, s, 1, tk, tv, q, kb, vb, pg,
                  layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, part_o,
                  part_ml, cnt, o, err);
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
@@ -532,43 +537,50 @@ int launch_cfg(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q, co
 
 template <int HD>
 int launch_hd(const __half* q, const __half* kb, const __half* vb, const __half* kc,
-              const __half* vc, int layer, int batch, int cap, const int32_t* ctx_len,
+              const __half* vc, const KvPages& pg, int layer, int batch, int cap,
+              const int32_t* ctx_len,
               const int32_t* req_valid, int B, int nq, int nkv, int L, int chunk, int n_chunks,
               float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
               cudaStream_t s) {
   CUtensorMap tk, tv;
-  const int64_t rows = (int64_t)L * batch * nkv * cap;
+  const int64_t rows = pg.table == nullptr ? (int64_t)L * batch * nkv * cap
+                                           : (int64_t)L * pg.n_pages * nkv * pg.page;
   if (!encode_2d(&tk, kc, rows, HD, HD, kKeys, DFLASH_F16) ||
       !encode_2d(&tv, vc, rows, HD, HD, kKeys, DFLASH_F16))
     return DFLASH_ECUDA;
   const int R = B * (nq / nkv);
   if (R <= 16)
-    return launch_cfg<HD, 1>(tk, tv, q, kb, vb, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
+    return launch_cfg<HD, 1>(tk, tv, q, kb, vb, pg, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
                              chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
   if (R <= 32)
-    return launch_cfg<HD, 2>(tk, tv, q, kb, vb, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
+    return launch_cfg<HD, 2>(tk, tv, q, kb, vb, pg, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
                              chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
-  return launch_cfg<HD, 4>(tk, tv, q, kb, vb, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
+  return launch_cfg<HD, 4>(tk, tv, q, kb, vb, pg, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
                            chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
 }
 
 }  // namespace
 
 int launch_attn_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
-                   const __half* vc, int layer, int batch, int cap, const int32_t* ctx_len,
+                   const __half* vc, const KvPages& pg, int layer, int batch, int cap,
+                   const int32_t* ctx_len,
                    const int32_t* req_valid, int B, int nq, int nkv, int hd, int L, int chunk,
                    int n_chunks, float* part_o, float* part_ml, unsigned* cnt, __half* o,
                    int32_t* err, cudaStream_t s) {
   if (B * (nq / nkv) > kAttnMaxRows || chunk % kKeys != 0 || B > kBlkKeys ||
       n_chunks > kMaxChunksTc)
     return DFLASH_EUNSUPPORTED;
-  if ((int64_t)L * batch * nkv * cap > 0x7fffffffLL) return DFLASH_EUNSUPPORTED;
+  if (pg.table == nullptr && (int64_t)L * batch * nkv * cap > 0x7fffffffLL)
+    return DFLASH_EUNSUPPORTED;
+  if (pg.table != nullptr &&
+      (pg.page % kKeys != 0 || (int64_t)L * pg.n_pages * nkv * pg.page > 0x7fffffffLL))
+    return DFLASH_EUNSUPPORTED;
   TimedScope ts(s, TC_ATTN);
   if (hd == 128)
-    return launch_hd<128>(q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, L,
+    return launch_hd<128>(q, kb, vb, kc, vc, pg, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, L,
                           chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
   if (hd == 64)
-    return launch_hd<64>(q, kb, vb, kc, vc, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, L,
+    return launch_hd<64>(q, kb, vb, kc, vc, pg, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, L,
                          chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
   return DFLASH_EUNSUPPORTED;
 }

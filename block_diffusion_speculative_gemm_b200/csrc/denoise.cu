@@ -17,24 +17,39 @@
 
 namespace dflash {
 
+// One warp per request (lane j = block position j; blockDim.x == 32).  With
+// paged K/V the warp also checks that every page holding a context position
+// is mapped; a request with an unmapped one is invalid (DFLASH_DEV_PAGE).
 __global__ void draft_init_kernel(const int32_t* __restrict__ anchor,
                                   const int32_t* __restrict__ ctx_len, int batch, int B, int V,
-                                  int mask_id, int cap, int32_t* tokens, int32_t* zrow,
-                                  int32_t* lm_rows, int32_t* cstep, int32_t* req_valid,
-                                  int32_t* err) {
+                                  int mask_id, int cap, const KvPages pg, int32_t* tokens,
+                                  int32_t* zrow, int32_t* lm_rows, int32_t* cstep,
+                                  int32_t* req_valid, int32_t* err) {
   pdl_trigger();
   pdl_wait();
   const int r = blockIdx.x * blockDim.y + threadIdx.y;
   const int j = threadIdx.x;
-  if (r >= batch || j >= B) return;
+  if (r >= batch) return;  // the whole warp
   const int a = anchor[r];
   const int T = ctx_len[r];
   const bool ok_tok = a >= 0 && a < V;
   const bool ok_ctx = T >= 0 && (long long)T + B <= cap;
+  bool ok_page = true;
+  if (pg.table != nullptr && ok_ctx) {
+    bool bad = false;
+    const int n_pg = (T + pg.page - 1) / pg.page;
+    for (int k = j; k < n_pg; k += 32) {
+      const int e = k < pg.max_pages ? pg.table[(long long)r * pg.max_pages + k] : -1;
+      bad |= e < 0 || e >= pg.n_pages;
+    }
+    ok_page = !__any_sync(0xffffffffu, bad);
+  }
+  if (j >= B) return;
   if (j == 0) {
-    req_valid[r] = (ok_tok && ok_ctx) ? 1 : 0;
+    req_valid[r] = (ok_tok && ok_ctx && ok_page) ? 1 : 0;
     if (!ok_tok) set_error(err, DFLASH_DEV_TOKEN_RANGE);
     if (!ok_ctx) set_error(err, DFLASH_DEV_CTX_CAP);
+    if (!ok_page) set_error(err, DFLASH_DEV_PAGE);
   }
   const int m = r * B + j;
   tokens[m] = j == 0 ? (ok_tok ? a : 0) : mask_id;
@@ -49,12 +64,13 @@ __global__ void draft_init_kernel(const int32_t* __restrict__ anchor,
 }
 
 void launch_draft_init(const int32_t* anchor, const int32_t* ctx_len, int batch, int B, int V,
-                       int mask_id, int cap, int32_t* tokens, int32_t* zrow, int32_t* lm_rows,
-                       int32_t* cstep, int32_t* req_valid, int32_t* err, cudaStream_t s) {
+                       int mask_id, int cap, const KvPages& pages, int32_t* tokens, int32_t* zrow,
+                       int32_t* lm_rows, int32_t* cstep, int32_t* req_valid, int32_t* err,
+                       cudaStream_t s) {
   dim3 block(32, 8);
   TimedScope ts(s, TC_ROW);
   launch_pdl(draft_init_kernel, dim3((batch + 7) / 8), dim3(block), 0, s, 1, anchor, ctx_len, batch,
-      B, V, mask_id, cap, tokens, zrow, lm_rows, cstep, req_valid, err);
+      B, V, mask_id, cap, pages, tokens, zrow, lm_rows, cstep, req_valid, err);
 }
 
 // Merge of two tile statistics: the larger maximum wins (lower id on equal
@@ -119,15 +135,24 @@ void launch_lm_reduce(const LmStat* stats, int n_vtiles, int rows, int32_t* tok,
 
 // fp32 model type: tile statistics from a full logits matrix [rows, V].
 __global__ void lm_stats_from_logits_kernel(const float* __restrict__ logits, int V,
-                                            LmStat* __restrict__ stats, float* dbg,
-                                            const int32_t* dbg_rows, int64_t dbg_ld) {
+                                            LmStat* __restrict__ stats, void* dbg,
+                                            const int32_t* dbg_rows, int64_t dbg_ld,
+                                            int dbg_bf16, const int32_t* dbg_valid, int B) {
   pdl_trigger();
   pdl_wait();
   const int q = blockIdx.y, t = blockIdx.x;
   const int n_vtiles = gridDim.x;
   const int v = t * kTileN + threadIdx.x;
   const float x = v < V ? logits[(size_t)q * V + v] : -INFINITY;
-  if (dbg && v < V) dbg[(int64_t)dbg_rows[q] * dbg_ld + v] = x;
+  if (dbg && v < V) {
+    const int64_t d = dbg_rows[q];
+    if (!dbg_valid || dbg_valid[d / B]) {
+      if (dbg_bf16)
+        static_cast<__nv_bfloat16*>(dbg)[d * dbg_ld + v] = __float2bfloat16_rn(x);
+      else
+        static_cast<float*>(dbg)[d * dbg_ld + v] = x;
+    }
+  }
   __shared__ float xs[kTileN];
   xs[threadIdx.x] = x;
   __syncthreads();
@@ -148,13 +173,13 @@ __global__ void lm_stats_from_logits_kernel(const float* __restrict__ logits, in
 }
 
 void launch_lm_stats_from_logits(const float* logits, int rows, int V, LmStat* stats,
-                                 float* dbg, const int32_t* dbg_rows, int64_t dbg_ld,
-                                 cudaStream_t s) {
+                                 void* dbg, const int32_t* dbg_rows, int64_t dbg_ld,
+                                 int dbg_bf16, const int32_t* dbg_valid, int B, cudaStream_t s) {
   if (rows <= 0) return;
   dim3 grid((V + kTileN - 1) / kTileN, rows);
   TimedScope ts(s, TC_LMHEAD);
   launch_pdl(lm_stats_from_logits_kernel, dim3(grid), dim3(kTileN), 0, s, 1, logits, V, stats, dbg,
-      dbg_rows, dbg_ld);
+      dbg_rows, dbg_ld, dbg_bf16, dbg_valid, B);
 }
 
 // One warp per request, lane j = block position j.  The k most confident

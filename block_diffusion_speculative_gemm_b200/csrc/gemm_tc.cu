@@ -67,16 +67,17 @@ constexpr int kMaxStages = 8;   // smem ring depth cap
 constexpr int kEpiWarp0 = 2;  // first epilogue warp
 constexpr int kLmTr = 32 * 33;  // floats of one warp's transpose buffer
 constexpr int kStLd = kTileN + 1; // row stride of the fused-op staging tile [32 tokens][128 rows]
-constexpr int kFusedSmem = 32 * kStLd * 4 + 64 * 4 + 16;  // staging tile + token maps + flag
+// staging tile + token maps (request, position: int; row base: int64) + flag
+constexpr int kFusedSmem = 32 * kStLd * 4 + 64 * 4 + 32 * 8 + 16;
 constexpr int kLmSmem = 4 * kLmTr * 4 + 4 * kMaxBN * (int)sizeof(LmStat);
 
 // Applies the fused op to one 32-token chunk of a finished output tile.
 // st[j * kStLd + r] = Y[m_base + j][n0 + r]; t = epilogue thread (0..127).
-// For OP_KV, tok_req/tok_pos hold each token's request and cache position
-// (request -1: skip).
+// For OP_KV, tok_req/tok_pos hold each token's request and position (request
+// -1: skip) and tok_base the token's row in the K/V store at layer 0, head 0.
 __device__ __forceinline__ void apply_op(const GemmOut& o, int M, int N, const float* st,
-                                         const int* tok_req, const int* tok_pos, int m_base,
-                                         int n0, int t) {
+                                         const int* tok_req, const int* tok_pos,
+                                         const long long* tok_base, int m_base, int n0, int t) {
   switch (o.op) {
     case OP_STORE:
     case OP_RESID: {
@@ -150,7 +151,7 @@ __device__ __forceinline__ void apply_op(const GemmOut& o, int M, int N, const f
           x2 = y2;
         }
         __half* dst = (is_v ? o.h2 : o.h1) +
-                      ((((size_t)layer * o.batch + req) * o.nkv + head) * o.cap + pos) * hd;
+                      (size_t)(layer * o.kv_ls + tok_base[j] + head * o.kv_hs) * hd;
         dst[i] = __float2half_rn(x1);
         dst[i + half] = __float2half_rn(x2);
       }
@@ -240,6 +241,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   float* st = reinterpret_cast<float*>(epi_smem);
   int* tok_req = reinterpret_cast<int*>(st + 32 * kStLd);
   int* tok_pos = tok_req + 32;
+  long long* tok_base = reinterpret_cast<long long*>(tok_pos + 32);
   uint64_t* bars = reinterpret_cast<uint64_t*>(epi_smem + a.epi_bytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * a.stages + 4);
   const uint32_t smem0 = smem_u32(smem);
@@ -437,6 +439,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (a.out.op != OP_KV || et >= 32) return;
         const int m = m_base + et;
         int req = -1, pos = 0;
+        long long base = 0;
         if (m < a.M) {
           const int nrow = a.out.row0 + m;
           int lo = 0, hi = a.out.batch - 1;
@@ -448,14 +451,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             set_error(a.err, DFLASH_DEV_ROWS);
           } else {
             pos = a.out.start_pos[lo] + (nrow - a.out.cu_rows[lo]);
-            if (pos < 0 || pos >= a.out.cap || pos >= a.out.max_pos)
+            const KvPages& pg = a.out.pages;
+            if (pg.table != nullptr && !pg.req_ok[lo]) {
+              // the page check reported the request: it writes nothing
+            } else if (pos < 0 || pos >= a.out.cap || pos >= a.out.max_pos) {
               set_error(a.err, DFLASH_DEV_CTX_CAP);
-            else
+            } else if (pg.table == nullptr) {
               req = lo;
+              base = (long long)lo * a.out.nkv * a.out.cap + pos;
+            } else {
+              req = lo;
+              const int page = pg.table[(long long)lo * pg.max_pages + pos / pg.page];
+              base = (long long)page * a.out.nkv * pg.page + pos % pg.page;
+            }
           }
         }
         tok_req[et] = req;
         tok_pos[et] = pos;
+        tok_base[et] = base;
       };
       if (EPI == EPI_PARTIAL && a.out.op == OP_PARTIAL) {
         // partials are read back right away by the reduction kernel: keep them in L2
@@ -484,7 +497,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int jj = 0; jj < 32; ++jj) st[jj * kStLd + row] = v[jj];
           token_maps(w.m0 + c * 32);
           epi_bar_sync();
-          apply_op(a.out, a.M, a.N, st, tok_req, tok_pos, w.m0 + c * 32, w.n0, et);
+          apply_op(a.out, a.M, a.N, st, tok_req, tok_pos, tok_base, w.m0 + c * 32, w.n0, et);
           epi_bar_sync();
         }
         release();
@@ -497,9 +510,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
               const int m = w.m0 + c * 32 + jj;
-              if (m < a.M)
-                a.out.dbg[(a.out.dbg_rows ? (int64_t)a.out.dbg_rows[m] : (int64_t)m) *
-                              a.out.dbg_ld + n] = v[jj];
+              if (m >= a.M) continue;
+              const int64_t d = a.out.dbg_rows ? (int64_t)a.out.dbg_rows[m] : (int64_t)m;
+              if (a.out.dbg_valid && !a.out.dbg_valid[d / a.out.B]) continue;
+              if (a.out.dbg_bf16)
+                static_cast<__nv_bfloat16*>(a.out.dbg)[d * a.out.dbg_ld + n] =
+                    __float2bfloat16_rn(v[jj]);
+              else
+                static_cast<float*>(a.out.dbg)[d * a.out.dbg_ld + n] = v[jj];
             }
           }
           // transpose through shared memory: lane jj then owns token column jj

@@ -71,6 +71,26 @@ struct LmStat {                // per (token row, 128-wide vocab tile)
 
 enum GemmEpi { EPI_PARTIAL = 0, EPI_LMHEAD = 1 };
 
+// Where injected K/V rows live.  table == nullptr: the contiguous cache
+// [L][batch][nkv][cap][hd].  Otherwise paged pools [L][n_pages][nkv][page][hd]
+// (prefix sharing): position p of request r is at page table[r * max_pages +
+// p / page], slot p % page; `page` is a multiple of 64 so that no 64-key
+// attention tile crosses a page.
+struct KvPages {
+  const int32_t* table = nullptr;
+  const int32_t* req_ok = nullptr;  // injection: 1 when every page a request's rows touch is mapped
+  int max_pages = 0, page = 0, n_pages = 0;
+};
+
+// Row (in units of hd elements) of (layer, request, position, head) in the K/V
+// store of `batch` requests and capacity `cap`, for a mapped position.
+__host__ __device__ inline int64_t kv_row(const KvPages& pg, int layer, int batch, int req,
+                                          int nkv, int head, int cap, int pos) {
+  if (pg.table == nullptr) return (((int64_t)layer * batch + req) * nkv + head) * cap + pos;
+  const int page = pg.table[(int64_t)req * pg.max_pages + pos / pg.page];
+  return (((int64_t)layer * pg.n_pages + page) * nkv + head) * pg.page + pos % pg.page;
+}
+
 // What the EPI_PARTIAL kernel does with the product Y[m][n] = sum_k X[m][k] W[n][k].
 // OP_PARTIAL writes each K split's share (fp32, for a reduction kernel); the
 // other ops need an unsplit GEMM and apply the step that follows the
@@ -93,9 +113,11 @@ struct GemmOut {
   int op = OP_PARTIAL;
   float* part = nullptr;          // OP_PARTIAL: [splits][M][N] fp32
   LmStat* stats = nullptr;        // EPI_LMHEAD: [M][ceil(N/128)]
-  float* dbg = nullptr;           // EPI_LMHEAD, optional: logits rows
+  void* dbg = nullptr;            // EPI_LMHEAD, optional: logits rows
   const int32_t* dbg_rows = nullptr;  // token row -> dbg row
   int64_t dbg_ld = 0;             // dbg row stride (elements)
+  int dbg_bf16 = 0;               // dbg rows stored as bf16 (else fp32)
+  const int32_t* dbg_valid = nullptr;  // optional: skip dbg row d when !dbg_valid[d / B]
   // fused ops
   float* f32 = nullptr;           // OP_STORE / OP_RESID: [M][N]
   __half* h1 = nullptr;
@@ -107,6 +129,8 @@ struct GemmOut {
   const int32_t* req_valid = nullptr;  // OP_QKV
   const int32_t* cu_rows = nullptr;    // OP_KV
   const int32_t* start_pos = nullptr;  // OP_KV
+  KvPages pages;                       // OP_KV: the K/V store (contiguous when no table)
+  int64_t kv_ls = 0, kv_hs = 0;        // OP_KV: rows between layers / between heads
   int B = 0, nq = 0, nkv = 0, hd = 0, I = 0;
   int row0 = 0, batch = 0, cap = 0, max_pos = 0;
 };
@@ -183,11 +207,16 @@ void launch_qkv_post(const float* part, int splits, int M, int B, const int32_t*
                      const float* sin_t, T* q, T* kb, T* vb, cudaStream_t s);
 template <typename T>
 void launch_swiglu(const float* part, int splits, int M, int I, T* act, cudaStream_t s);
+// cap: positions per request (max_pages * page when paged).
 template <typename T>
 void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int L, int nkv, int hd,
                        const int32_t* cu_rows, const int32_t* start_pos, int batch, int cap,
-                       const float* cos_t, const float* sin_t, int max_pos, T* kc, T* vc,
-                       int32_t* err, cudaStream_t s);
+                       const KvPages& pages, const float* cos_t, const float* sin_t, int max_pos,
+                       T* kc, T* vc, int32_t* err, cudaStream_t s);
+// One warp per request: req_ok[r] = 1 when every page holding positions
+// start_pos[r] .. start_pos[r] + rows - 1 is mapped, else 0 and DFLASH_DEV_PAGE.
+void launch_inject_page_check(const int32_t* cu_rows, const int32_t* start_pos, int batch,
+                              const KvPages& pages, int32_t* req_ok, int32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- attention
 constexpr int kAttnMaxRows = 64;  // B * (n_q / n_kv) query rows per (request, kv head)
@@ -199,28 +228,51 @@ constexpr int kAttnMaxRows = 64;  // B * (n_q / n_kv) query rows per (request, k
 // call), merges them into o [batch * B][nq][hd].  The cache is
 // [L][batch][nkv][cap][hd]; `layer` selects the layer.
 int launch_attn_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
-                   const __half* vc, int layer, int batch, int cap, const int32_t* ctx_len,
+                   const __half* vc, const KvPages& pages, int layer, int batch, int cap,
+                   const int32_t* ctx_len,
                    const int32_t* req_valid, int B, int nq, int nkv, int hd, int L, int chunk,
                    int n_chunks, float* part_o, float* part_ml, unsigned* cnt, __half* o,
                    int32_t* err, cudaStream_t s);
 
 // T: type of q, the block's k/v and the output o; TC: K/V cache type.
+// Paged K/V (pages.table set) is read by the tensor-core kernel only.
 template <typename T, typename TC>
 int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, const TC* vc,
-                           int layer, int L, int batch, int cap, const int32_t* ctx_len,
+                           const KvPages& pages, int layer, int L, int batch, int cap,
+                           const int32_t* ctx_len,
                            const int32_t* req_valid, int B, int nq, int nkv, int hd,
                            float* part_o, float* part_ml, int n_chunks, int chunk, T* o,
                            unsigned* cnt, int32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- draft bookkeeping
+// cap bounds ctx_len + B; with paged K/V every page below ctx_len must also be
+// mapped (else the request is invalid and DFLASH_DEV_PAGE is set).
 void launch_draft_init(const int32_t* anchor, const int32_t* ctx_len, int batch, int B, int V,
-                       int mask_id, int cap, int32_t* tokens, int32_t* zrow, int32_t* lm_rows,
-                       int32_t* cstep, int32_t* req_valid, int32_t* err, cudaStream_t s);
+                       int mask_id, int cap, const KvPages& pages, int32_t* tokens, int32_t* zrow,
+                       int32_t* lm_rows, int32_t* cstep, int32_t* req_valid, int32_t* err,
+                       cudaStream_t s);
 void launch_lm_reduce(const LmStat* stats, int n_vtiles, int rows, int32_t* tok, float* conf,
                       cudaStream_t s);
+// dbg (optional): logits rows copied to dbg[dbg_rows[q] * dbg_ld ...] as fp32, or
+// as bf16 when dbg_bf16; rows of requests with !dbg_valid[dbg_rows[q] / B] are
+// skipped when dbg_valid is given.
 void launch_lm_stats_from_logits(const float* logits, int rows, int V, LmStat* stats,
-                                 float* dbg, const int32_t* dbg_rows, int64_t dbg_ld,
-                                 cudaStream_t s);
+                                 void* dbg, const int32_t* dbg_rows, int64_t dbg_ld,
+                                 int dbg_bf16, const int32_t* dbg_valid, int B, cudaStream_t s);
+
+// ---------------------------------------------------------------- sampled drafting
+// Draw of every still-masked row at denoising step `step` from its logits row
+// q[lm_rows[row]] (fp32, or bf16 when q_bf16): Gumbel-max at temperature tau with
+// Philox4x64-10 stream 2 noise, and the untempered probability of the drawn
+// token.  part: [rows][chunks] partials; cnt: one zeroed counter per row.
+int sampled_draw_chunks(int rows, int V);
+size_t sampled_draw_part_bytes(int rows, int chunks);
+// Rows of requests with !req_valid[r] (req_valid nullable) read nothing and draw
+// token 0 with confidence 0.
+int launch_sampled_draw(const void* q, int q_bf16, const int32_t* lm_rows,
+                        const int32_t* req_valid, int rows, int B, int V, int step, float tau,
+                        uint64_t seed, uint64_t offset, int32_t* tok, float* conf, void* part,
+                        int chunks, unsigned* cnt, cudaStream_t s);
 void launch_commit(const int32_t* tok, const float* conf, int batch, int B, int rem, int k,
                    int step, int32_t* tokens, int32_t* zrow, int32_t* lm_rows, int32_t* cstep,
                    cudaStream_t s);

@@ -298,7 +298,7 @@ template <typename T>
 __global__ void kv_scatter_kernel(const float* __restrict__ part, int splits, int n_rows,
                                   int row0, int L, int nkv, int hd, const int32_t* __restrict__ cu_rows,
                                   const int32_t* __restrict__ start_pos, int batch, int cap,
-                                  const float* __restrict__ cos_t,
+                                  const KvPages pg, const float* __restrict__ cos_t,
                                   const float* __restrict__ sin_t, int max_pos,
                                   T* __restrict__ kc, T* __restrict__ vc, int32_t* err) {
   pdl_trigger();
@@ -321,6 +321,7 @@ __global__ void kv_scatter_kernel(const float* __restrict__ part, int splits, in
     return;
   }
   const int pos = start_pos[r] + (n - cu_rows[r]);
+  if (pg.table != nullptr && !pg.req_ok[r]) return;  // the page check reported it
   if (pos < 0 || pos >= cap || pos >= max_pos) {
     if (p == 0) set_error(err, DFLASH_DEV_CTX_CAP);
     return;
@@ -345,7 +346,7 @@ __global__ void kv_scatter_kernel(const float* __restrict__ part, int splits, in
     x1 = y1;
     x2 = y2;
   }
-  T* dst = (is_v ? vc : kc) + ((((size_t)l * batch + r) * nkv + head) * cap + pos) * hd;
+  T* dst = (is_v ? vc : kc) + (size_t)kv_row(pg, l, batch, r, nkv, head, cap, pos) * hd;
   store4<T>(dst + i, x1.x, x1.y, x1.z, x1.w);
   store4<T>(dst + i + half, x2.x, x2.y, x2.z, x2.w);
 }
@@ -353,14 +354,53 @@ __global__ void kv_scatter_kernel(const float* __restrict__ part, int splits, in
 template <typename T>
 void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int L, int nkv,
                        int hd, const int32_t* cu_rows, const int32_t* start_pos, int batch, int cap,
-                       const float* cos_t, const float* sin_t, int max_pos, T* kc, T* vc,
-                       int32_t* err, cudaStream_t s) {
+                       const KvPages& pages, const float* cos_t, const float* sin_t, int max_pos,
+                       T* kc, T* vc, int32_t* err, cudaStream_t s) {
   if (n_rows <= 0) return;
   const int pairs = L * 2 * nkv * hd / 2;
   dim3 grid((pairs / 4 + 255) / 256, n_rows);
   TimedScope ts(s, TC_ROW);
   launch_pdl(kv_scatter_kernel<T>, dim3(grid), dim3(256), 0, s, 1, part, splits, n_rows, row0, L,
-      nkv, hd, cu_rows, start_pos, batch, cap, cos_t, sin_t, max_pos, kc, vc, err);
+      nkv, hd, cu_rows, start_pos, batch, cap, pages, cos_t, sin_t, max_pos, kc, vc, err);
+}
+
+// One warp per request: the pages holding its rows' positions must all be
+// mapped (an entry in [0, n_pages) inside the request's table row); a request
+// with an unmapped one writes nothing and reports DFLASH_DEV_PAGE.
+__global__ void inject_page_check_kernel(const int32_t* __restrict__ cu_rows,
+                                         const int32_t* __restrict__ start_pos, int batch,
+                                         const KvPages pg, int32_t* __restrict__ req_ok,
+                                         int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= batch) return;
+  const int n = cu_rows[r + 1] - cu_rows[r];
+  const int st = start_pos[r];
+  bool bad = false;
+  if (n > 0 && st >= 0) {
+    const int p0 = st / pg.page;
+    const long long last = ((long long)st + n - 1) / pg.page;
+    for (long long k = p0 + lane; k <= last; k += 32) {
+      const int e = k < pg.max_pages ? pg.table[(long long)r * pg.max_pages + k] : -1;
+      bad |= e < 0 || e >= pg.n_pages;
+    }
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0) {
+    req_ok[r] = bad ? 0 : 1;
+    if (bad) set_error(err, DFLASH_DEV_PAGE);
+  }
+}
+
+void launch_inject_page_check(const int32_t* cu_rows, const int32_t* start_pos, int batch,
+                              const KvPages& pages, int32_t* req_ok, int32_t* err,
+                              cudaStream_t s) {
+  TimedScope ts(s, TC_ROW);
+  const int wpb = 4;
+  launch_pdl(inject_page_check_kernel, dim3((batch + wpb - 1) / wpb), dim3(32 * wpb), 0, s, 1,
+             cu_rows, start_pos, batch, pages, req_ok, err);
 }
 
 // T: activation type (GEMM operand); TC: K/V cache type; TE: embedding type.
@@ -375,8 +415,9 @@ void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int 
   template void launch_swiglu<T>(const float*, int, int, int, T*, cudaStream_t);
 #define DFLASH_INST_C(TC)                                                                        \
   template void launch_kv_scatter<TC>(const float*, int, int, int, int, int, int,                \
-                                      const int32_t*, const int32_t*, int, int, const float*,    \
-                                      const float*, int, TC*, TC*, int32_t*, cudaStream_t);
+                                      const int32_t*, const int32_t*, int, int, const KvPages&,  \
+                                      const float*, const float*, int, TC*, TC*, int32_t*,       \
+                                      cudaStream_t);
 
 DFLASH_INST_A(float)
 DFLASH_INST_A(__half)

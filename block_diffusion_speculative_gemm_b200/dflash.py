@@ -21,7 +21,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "dflash.h")
 HEADERS = [HEADER, os.path.join(os.path.dirname(_HERE), "include", "dflash_debug.h")]
 
 OK, EINVAL, EUNSUPPORTED, ECUDA, ENOMEM, EWORKSPACE, ESCRATCH = 0, -1, -2, -3, -4, -5, -6
-DEV_CTX_CAP, DEV_OUT_CAP, DEV_TOKEN_RANGE, DEV_TIMEOUT, DEV_ROWS = 1, 2, 4, 8, 16
+DEV_CTX_CAP, DEV_OUT_CAP, DEV_TOKEN_RANGE, DEV_TIMEOUT, DEV_ROWS, DEV_PAGE = 1, 2, 4, 8, 16, 32
 F32, BF16, F16 = 0, 1, 2
 TIMING_CLASSES = ("gemm", "attention", "row", "verify", "lm_head")
 
@@ -75,6 +75,13 @@ def lib() -> ctypes.CDLL:
                                        sz, vp]
         L.dflash_draft_block.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp,
                                          sz, vp]
+        L.dflash_inject_kv_paged.argtypes = [vp, ctypes.POINTER(vp), vp, vp, i32, i32, vp, vp,
+                                             i32, i32, vp, i32, vp, sz, vp]
+        L.dflash_draft_block_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, i32, i32, i32,
+                                               i32, vp, vp, vp, vp, sz, vp]
+        L.dflash_draft_block_sampled.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                                 ctypes.c_float, ctypes.c_uint64,
+                                                 ctypes.c_uint64, vp, vp, vp, i32, vp, sz, vp]
         L.dflash_verify.argtypes = [vp, i32, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp, sz,
                                     vp]
         L.dflash_get_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
@@ -268,6 +275,96 @@ def draft_block(model: Model, anchor: torch.Tensor, ctx_len: torch.Tensor, k_cac
         model.handle, _ptr(anchor), _ptr(ctx_len), _ptr(k_cache), _ptr(v_cache), k_cache.shape[3],
         batch, B, n_steps, _ptr(draft_tokens), _ptr(commit_step), _ptr(logits_dbg), _ptr(ws),
         ws.numel(), _stream(stream)))
+
+
+def _need_pages(model: Model, k_pool, v_pool, page_table, batch):
+    s = model.shape
+    _need(k_pool, "k_pool", model.cache_dtype)
+    _need(v_pool, "v_pool", model.cache_dtype, k_pool.shape)
+    if k_pool.dim() != 5 or k_pool.shape[0] != s.L or k_pool.shape[2] != s.nkv or \
+            k_pool.shape[4] != s.hd:
+        raise ValueError("k_pool must be [L, n_pages, n_kv, page_size, head_dim]")
+    _need(page_table, "page_table", torch.int32)
+    if page_table.dim() != 2 or page_table.shape[0] != batch:
+        raise ValueError("page_table must be [batch, max_pages]")
+    return k_pool.shape[1], k_pool.shape[3], page_table.shape[1]
+
+
+def inject_kv_paged(model: Model, taps: Sequence[torch.Tensor], cu_rows: torch.Tensor,
+                    start_pos: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                    page_table: torch.Tensor, ws: torch.Tensor, stream=None):
+    """Injection through a page table into K/V page pools (prefix sharing); see
+    dflash_inject_kv_paged in include/dflash.h."""
+    s = model.shape
+    batch = start_pos.numel()
+    n_rows = taps[0].shape[0]
+    if len(taps) != s.n_tap:
+        raise ValueError(f"expected {s.n_tap} taps")
+    for i, t in enumerate(taps):
+        _need(t, f"taps[{i}]", model.tdtype, (n_rows, s.H_t))
+    _need(cu_rows, "cu_rows", torch.int32, (batch + 1,))
+    _need(start_pos, "start_pos", torch.int32)
+    n_pages, page, max_pages = _need_pages(model, k_pool, v_pool, page_table, batch)
+    _need(ws, "ws", torch.uint8)
+    arr = (ctypes.c_void_p * s.n_tap)(*[t.data_ptr() for t in taps])
+    _check("dflash_inject_kv_paged", lib().dflash_inject_kv_paged(
+        model.handle, arr, _ptr(cu_rows), _ptr(start_pos), batch, n_rows, _ptr(k_pool),
+        _ptr(v_pool), n_pages, page, _ptr(page_table), max_pages, _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def draft_block_paged(model: Model, anchor: torch.Tensor, ctx_len: torch.Tensor,
+                      k_pool: torch.Tensor, v_pool: torch.Tensor, page_table: torch.Tensor, B: int,
+                      n_steps: int, draft_tokens: torch.Tensor, ws: torch.Tensor,
+                      commit_step: Optional[torch.Tensor] = None,
+                      logits_dbg: Optional[torch.Tensor] = None, stream=None):
+    """Greedy drafting over paged K/V; see dflash_draft_block_paged in include/dflash.h."""
+    s = model.shape
+    batch = anchor.numel()
+    _need(anchor, "anchor", torch.int32)
+    _need(ctx_len, "ctx_len", torch.int32, (batch,))
+    n_pages, page, max_pages = _need_pages(model, k_pool, v_pool, page_table, batch)
+    _need(draft_tokens, "draft_tokens", torch.int32, (batch, B))
+    if commit_step is not None:
+        _need(commit_step, "commit_step", torch.int32, (batch, B))
+    if logits_dbg is not None:
+        _need(logits_dbg, "logits_dbg", torch.float32, (n_steps, batch, B, s.V))
+    _need(ws, "ws", torch.uint8)
+    _check("dflash_draft_block_paged", lib().dflash_draft_block_paged(
+        model.handle, _ptr(anchor), _ptr(ctx_len), _ptr(k_pool), _ptr(v_pool), n_pages, page,
+        _ptr(page_table), max_pages, batch, B, n_steps, _ptr(draft_tokens), _ptr(commit_step),
+        _ptr(logits_dbg), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def draft_block_sampled(model: Model, anchor: torch.Tensor, ctx_len: torch.Tensor,
+                        k_cache: torch.Tensor, v_cache: torch.Tensor, B: int, n_steps: int,
+                        temperature: float, seed: int, offset: int, draft_tokens: torch.Tensor,
+                        draft_logits: torch.Tensor, ws: torch.Tensor,
+                        commit_step: Optional[torch.Tensor] = None, stream=None):
+    """Sampled (temperature) drafting; ``draft_logits`` (float32 or bfloat16
+    [batch, B, V]) receives each position's committing-step logits, the q rows of
+    sampled verify.  See dflash_draft_block_sampled in include/dflash.h."""
+    s = model.shape
+    batch = anchor.numel()
+    _need(anchor, "anchor", torch.int32)
+    _need(ctx_len, "ctx_len", torch.int32, (batch,))
+    _need(k_cache, "k_cache", model.cache_dtype)
+    _need(v_cache, "v_cache", model.cache_dtype, k_cache.shape)
+    if k_cache.dim() != 5 or tuple(k_cache.shape[:3]) != (s.L, batch, s.nkv) or k_cache.shape[4] != s.hd:
+        raise ValueError("k_cache must be [L, batch, n_kv, cap, head_dim]")
+    _need(draft_tokens, "draft_tokens", torch.int32, (batch, B))
+    if commit_step is not None:
+        _need(commit_step, "commit_step", torch.int32, (batch, B))
+    dt = {torch.bfloat16: BF16, torch.float32: F32}.get(draft_logits.dtype)
+    if dt is None:
+        raise TypeError("draft_logits must be bfloat16 or float32")
+    _need(draft_logits, "draft_logits", None, (batch, B, s.V))
+    _need(ws, "ws", torch.uint8)
+    _check("dflash_draft_block_sampled", lib().dflash_draft_block_sampled(
+        model.handle, _ptr(anchor), _ptr(ctx_len), _ptr(k_cache), _ptr(v_cache), k_cache.shape[3],
+        batch, B, n_steps, float(temperature), int(seed) & (2**64 - 1), int(offset) & (2**64 - 1),
+        _ptr(draft_tokens), _ptr(commit_step), _ptr(draft_logits), dt, _ptr(ws), ws.numel(),
+        _stream(stream)))
 
 
 def verify(target_logits: torch.Tensor, draft_tokens: torch.Tensor, out_tokens: torch.Tensor,

@@ -19,6 +19,9 @@
  *                       decide_acceptance(logits, draft_block), read greedily.
  *   dflash_verify_sampled  the same step under temperature sampling
  *                       (speculative sampling; see its declaration).
+ *   dflash_draft_block_sampled  drafting under temperature sampling.
+ *   dflash_inject_kv_paged, dflash_draft_block_paged  the same calls over a
+ *                       paged K/V store with prefix sharing.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -68,6 +71,7 @@ extern "C" {
 #define DFLASH_DEV_TOKEN_RANGE 4  /* token id outside [0, V) */
 #define DFLASH_DEV_TIMEOUT     8  /* a bounded device wait expired */
 #define DFLASH_DEV_ROWS        16 /* cu_rows not monotone or not ending at n_rows */
+#define DFLASH_DEV_PAGE        32 /* a position's page-table entry is unmapped (paged K/V) */
 
 /* ---- element types ---------------------------------------------------- */
 #define DFLASH_F32  0
@@ -188,6 +192,70 @@ int dflash_draft_block(const dflash_model* m, const int32_t* anchor, const int32
                        const void* k_cache, const void* v_cache, int cache_cap, int batch, int B,
                        int n_steps, int32_t* draft_tokens, int32_t* commit_step, float* logits_dbg,
                        void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Paged K/V with prefix sharing.  "DFlash: Block Diffusion for Flash Speculative
+ * Decoding", §2 KV 注入: the injected K/V is cached for reuse and supports prefix
+ * sharing.  An injected row depends only on the target hidden state at its
+ * position and on the position, so requests whose contexts share a prefix can
+ * share the pages that hold it.  The pages give no layout; this one is:
+ *   k_pool, v_pool  device fp16 [n_layers][n_pages][n_kv][page_size][head_dim]
+ *                   (DFLASH_BF16 models only), 16-byte aligned; K after RoPE.
+ *   page_table      device int32 [batch][max_pages]: position p of request r is
+ *                   at page page_table[r][p / page_size], slot p % page_size.
+ *                   An entry of -1, or any id outside [0, n_pages), is unmapped.
+ *   page_size       a multiple of 64 (no 64-key attention tile crosses a page).
+ * Requests may map the same page; the caller makes sure that no two requests of
+ * one injection call write the same (page, slot).
+ * dflash_inject_kv_paged: as dflash_inject_kv, writing through the table.  A
+ * request whose rows touch an unmapped page writes none of its rows and sets
+ * DFLASH_DEV_PAGE; rows past page_size * max_pages set DFLASH_DEV_CTX_CAP.
+ * dflash_draft_block_paged: as dflash_draft_block, reading the context through
+ * the table.  A request with an unmapped page below ctx_len, or with
+ * ctx_len > page_size * max_pages, writes nothing and sets DFLASH_DEV_PAGE or
+ * DFLASH_DEV_CTX_CAP.  Workspaces: dflash_workspace_size with the call's batch.
+ * L * n_pages * n_kv * page_size must stay below 2^31 (DFLASH_EUNSUPPORTED).
+ */
+int dflash_inject_kv_paged(const dflash_model* m, const void* const* taps, const int32_t* cu_rows,
+                           const int32_t* start_pos, int batch, int n_rows, void* k_pool,
+                           void* v_pool, int n_pages, int page_size, const int32_t* page_table,
+                           int max_pages, void* ws, size_t ws_bytes, void* stream);
+int dflash_draft_block_paged(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_len,
+                             const void* k_pool, const void* v_pool, int n_pages, int page_size,
+                             const int32_t* page_table, int max_pages, int batch, int B,
+                             int n_steps, int32_t* draft_tokens, int32_t* commit_step,
+                             float* logits_dbg, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Sampled (temperature) drafting.  "DFlash + Spec V2 深度解析", §2.3 块扩散 gives
+ * the greedy steps; "DFlash: Block Diffusion for Flash Speculative Decoding",
+ * §消融实验结论, says drafting holds up under high-temperature sampling; the
+ * pages give no sampling rule.  The rule taken is the sampled counterpart of
+ * the greedy one.  At step t every still-masked position j of request r draws
+ *   x_j = argmax_v (Y_jv / temperature - log(-log U'_v))   (ties to the lower id)
+ * from its LM-head logits Y_j, with U'_v = ((w >> 11) + 1/2) 2^-53 and w the
+ * 64-bit word n % 4 of Philox4x64-10 (Salmon et al., SC 2011) under key
+ * (seed, 0) at counter (offset, r, 2, n / 4), n = (t B + j) V + v.  Its
+ * confidence is the untempered probability softmax(Y_j)(x_j).  The
+ * ceil(remaining / (n_steps - t)) most confident positions (ties to the lower
+ * position) commit their drawn tokens.
+ *   draft_logits  device [batch, B, V] out, of draft_logits_dtype (DFLASH_F32 or
+ *                 DFLASH_BF16), 16-byte aligned: row j holds the logits of the step
+ *                 that committed position j, the draft distribution q_j that
+ *                 dflash_verify_sampled takes (row 0 is not written).  The draw
+ *                 reads the stored row, so each token is drawn from exactly the
+ *                 row the caller receives.
+ *   temperature   in [1e-4, 1e4]; equal (seed, offset) repeat the call's draws.
+ * Other arguments, errors and limits as dflash_draft_block; batch * B <= 32768
+ * (DFLASH_EUNSUPPORTED beyond).  A request that sets a device error bit writes
+ * none of its draft_tokens, commit_step or draft_logits.
+ */
+int dflash_draft_block_sampled(const dflash_model* m, const int32_t* anchor,
+                               const int32_t* ctx_len, const void* k_cache, const void* v_cache,
+                               int cache_cap, int batch, int B, int n_steps, float temperature,
+                               uint64_t seed, uint64_t offset, int32_t* draft_tokens,
+                               int32_t* commit_step, void* draft_logits, int draft_logits_dtype,
+                               void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Greedy verify.

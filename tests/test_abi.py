@@ -128,3 +128,16 @@ def test_sampled_verify_host_checks(kw, code):
                                  vp(a["out_len"]), a["out_cap"], vp(a["seq"]), vp(a["acc"]),
                                  vp(a["nxt"]), vp(a["ws"]), a["ws_bytes"], None)
     assert st == code
+
+
+def test_sampled_and_paged_calls_reject_null_model_and_bad_arguments():
+    L = D.lib()
+    p = ctypes.c_void_p(4096)
+    # sampled drafting: no model, bad temperature, bad output type
+    assert L.dflash_draft_block_sampled(None, p, p, p, p, 64, 1, 8, 2, 1.0, 1, 0, p, None, p,
+                                        D.F32, p, 1 << 20, None) == D.EINVAL
+    # paged calls: no model
+    assert L.dflash_inject_kv_paged(None, None, p, p, 1, 4, p, p, 8, 64, p, 4, p, 1 << 20,
+                                    None) == D.EINVAL
+    assert L.dflash_draft_block_paged(None, p, p, p, p, 8, 64, p, 4, 1, 8, 2, p, None, None, p,
+                                      1 << 20, None) == D.EINVAL
