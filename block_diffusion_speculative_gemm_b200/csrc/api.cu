@@ -13,6 +13,9 @@
 
 using namespace dflash;
 
+static_assert(sizeof(LmStat) == sizeof(dflash_lm_stat), "shard record layout");
+static_assert(sizeof(ArgPart) == sizeof(dflash_row_argmax), "verify shard record layout");
+
 // ============================================================== timing
 namespace dflash {
 namespace timing_detail {
@@ -102,6 +105,7 @@ struct LayerPack {
 struct dflash_model {
   dflash_config cfg;
   int device = 0;
+  int vocab_lo = 0, vocab_hi = 0;  // LM-head rows held: [vocab_lo, vocab_hi) of the vocabulary
   size_t esz = 2;
   void* emb = nullptr;
   void* W_fc = nullptr;
@@ -366,15 +370,23 @@ extern "C" const char* dflash_status_str(int st) {
   }
 }
 
-extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weights* w,
-                                   dflash_model** out) {
+namespace {
+
+int model_create(const dflash_config* cfg, const dflash_weights* w, int vocab_lo, int vocab_hi,
+                 dflash_model** out) {
   if (!cfg || !w || !out || !w->layers) return DFLASH_EINVAL;
   *out = nullptr;
   if (!config_ok(*cfg)) return DFLASH_EINVAL;
   if (!config_supported(*cfg)) return DFLASH_EUNSUPPORTED;
+  if (vocab_lo < 0 || vocab_hi > cfg->vocab || vocab_hi <= vocab_lo) return DFLASH_EINVAL;
+  const bool shard = vocab_lo != 0 || vocab_hi != cfg->vocab;
+  if (shard && cfg->dtype != DFLASH_BF16) return DFLASH_EUNSUPPORTED;
   const dflash_config& c = *cfg;
   dflash_model* m = new dflash_model();
   m->cfg = c;
+  m->vocab_lo = vocab_lo;
+  m->vocab_hi = vocab_hi;
+  const size_t Vs = (size_t)(vocab_hi - vocab_lo);  // LM-head rows held
   cudaGetDevice(&m->device);
   m->esz = c.dtype == DFLASH_BF16 ? 2 : 4;
   const size_t e = m->esz;
@@ -386,14 +398,15 @@ extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weight
   };
   m->emb = dmalloc(m, e * V * d);
   m->W_fc = dmalloc(m, e * d * c.n_tap * c.H_t);
-  m->W_lm = dmalloc(m, e * V * d);
+  m->W_lm = dmalloc(m, e * Vs * d);
   m->W_kv = dmalloc(m, e * c.n_layers * 2 * nkv * hd * d);
   if (!m->emb || !m->W_fc || !m->W_lm || !m->W_kv) return fail(DFLASH_ENOMEM);
   // embedding and fc stay in the model dtype (their inputs are exact in it);
   // every other GEMM weight goes through pack_weights
   if (!copy_rows(m->emb, w->emb, e * V * d) ||
       !copy_rows(m->W_fc, w->W_fc, e * d * c.n_tap * c.H_t) ||
-      !pack_weights(m, m->W_lm, w->W_lm, V * d))
+      !w->W_lm ||
+      !pack_weights(m, m->W_lm, static_cast<const uint8_t*>(w->W_lm) + e * vocab_lo * d, Vs * d))
     return fail(DFLASH_EINVAL);
   m->g_ctx = gain_copy(m, w->g_ctx);
   m->g_final = gain_copy(m, w->g_final);
@@ -447,7 +460,7 @@ extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weight
     const int H = DFLASH_F16;
     bool ok = encode_weight_map(m->mfc, m->W_fc, c.d, c.n_tap * c.H_t, DFLASH_BF16) &&
               encode_weight_map(m->mkv, m->W_kv, c.n_layers * 2 * kvrows, c.d, H) &&
-              encode_weight_map(m->mlm, m->W_lm, c.vocab, c.d, H);
+              encode_weight_map(m->mlm, m->W_lm, (int)Vs, c.d, H);
     for (int l = 0; l < c.n_layers && ok; ++l) {
       LayerPack& P = m->layers[l];
       ok = encode_weight_map(P.mqkv, P.Wqkv, qkv_out(c), c.d, H) &&
@@ -468,7 +481,7 @@ extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weight
     };
     ok = tile_into(m->mfc, m->W_fc, c.d, c.n_tap * c.H_t) &&
          tile_into(m->mkv, m->W_kv, c.n_layers * 2 * kvrows, c.d) &&
-         tile_into(m->mlm, m->W_lm, c.vocab, c.d);
+         tile_into(m->mlm, m->W_lm, (int)Vs, c.d);
     for (int l = 0; l < c.n_layers && ok; ++l) {
       LayerPack& P = m->layers[l];
       ok = tile_into(P.mqkv, P.Wqkv, qkv_out(c), c.d) &&
@@ -492,6 +505,22 @@ extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weight
     return fail(DFLASH_ECUDA);
   *out = m;
   return DFLASH_OK;
+}
+
+bool whole_vocab(const dflash_model* m) {
+  return m->vocab_lo == 0 && m->vocab_hi == m->cfg.vocab;
+}
+
+}  // namespace
+
+extern "C" int dflash_model_create(const dflash_config* cfg, const dflash_weights* w,
+                                   dflash_model** out) {
+  return model_create(cfg, w, 0, cfg ? cfg->vocab : 0, out);
+}
+
+extern "C" int dflash_model_create_shard(const dflash_config* cfg, const dflash_weights* w,
+                                         int vocab_lo, int vocab_hi, dflash_model** out) {
+  return model_create(cfg, w, vocab_lo, vocab_hi, out);
 }
 
 extern "C" int dflash_model_destroy(dflash_model* m) {
@@ -701,13 +730,36 @@ struct SampleArgs {
 
 // T: activation / GEMM operand type; TC: K/V cache type; TE: embedding type.
 // samp == nullptr: greedy drafting (argmax, max-probability confidence).
+// Which parts of a draft one call runs.  The whole draft (dflash_draft_block)
+// runs them all; a vocabulary-parallel draft runs them one at a time so that the
+// per-row LM-head statistics of every vocabulary shard can be exchanged between
+// the forward and the commit of each step.
+struct DraftPhase {
+  bool init = true;                // block initialisation (and the request checks)
+  bool forward = true;             // embedding, layers and LM head of the steps run
+  bool commit = true;              // token choice and commit of the steps run
+  bool finish = true;              // copy-out of the draft tokens and commit steps
+  int t0 = 0, t1 = 1 << 30;        // the steps run: [t0, min(t1, n_steps))
+  LmStat* shard_stats = nullptr;   // forward only: per-row statistics of this shard (out)
+  const LmStat* gathered = nullptr;  // commit: [world][rows] statistics of every shard
+  int world = 0;
+};
+
+// Masked positions per request before step t of an n_steps draft of block B.
+int masked_before(int B, int n_steps, int t) {
+  int rem = B - 1;
+  for (int u = 0; u < t && u < n_steps; ++u) rem -= (rem + (n_steps - u) - 1) / (n_steps - u);
+  return rem;
+}
+
 // pg.table set: the context is read from paged pools, cap = positions per
 // request (the RoPE bound on ctx_len + B).
 template <typename T, typename TC, typename TE>
 int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_len,
                const void* k_cache, const void* v_cache, int cap, const KvPages& pg, int batch,
                int B, int n_steps, int32_t* draft_tokens, int32_t* commit_step, float* logits_dbg,
-               const SampleArgs* samp, void* ws, cudaStream_t s) {
+               const SampleArgs* samp, void* ws, cudaStream_t s,
+               const DraftPhase& ph = DraftPhase()) {
   const dflash_config& c = m->cfg;
   const DraftLayout L = draft_layout(c, batch, B);
   const int M = batch * B;
@@ -734,7 +786,8 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
   LmStat* stats = at<LmStat>(ws, L.stats);
   const TC* kc = static_cast<const TC*>(k_cache);
   const TC* vc = static_cast<const TC*>(v_cache);
-  const int n_vt = (c.vocab + kTileN - 1) / kTileN;
+  // LM-head vocabulary tiles this model holds (all of them unless it is a shard)
+  const int n_vt = (m->vocab_hi - m->vocab_lo + kTileN - 1) / kTileN;
   const bool bf16 = c.dtype == DFLASH_BF16;
 
   // split-KV chunk: a multiple of the attention tile (64 keys) sized for
@@ -749,8 +802,9 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
     chunk = g_attn_chunk;
   const int n_chunks = (cap + B + chunk - 1) / chunk;
 
-  launch_draft_init(anchor, ctx_len, batch, B, c.vocab, c.mask_id, cap, pg, tokens, zrow, lm_rows,
-                    cstep, valid, err, s);
+  if (ph.init)
+    launch_draft_init(anchor, ctx_len, batch, B, c.vocab, c.mask_id, cap, pg, tokens, zrow,
+                      lm_rows, cstep, valid, err, s);
   auto gemm = [&](const WeightMap& W, const void* wptr, int N, int K, const T* X, float* out,
                   size_t cap_elems, int* splits_out) -> int {
     if (bf16) {
@@ -767,10 +821,12 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
     return DFLASH_OK;
   };
 
-  int rem = B - 1;
+  int rem = masked_before(B, n_steps, ph.t0);
   int st = DFLASH_OK;
-  for (int t = 0; t < n_steps; ++t) {
+  for (int t = ph.t0; t < std::min(ph.t1, n_steps); ++t) {
     const int k = (rem + (n_steps - t) - 1) / (n_steps - t);
+    const int rows = batch * rem;
+    if (!ph.forward) goto choose;
     launch_embed_norm<TE, T>(tokens, static_cast<const TE*>(m->emb), m->layers[0].g_in, x, h, M, c.d,
                          c.eps, s);
     for (int l = 0; l < c.n_layers; ++l) {
@@ -841,7 +897,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
     // drafting writes every masked row's logits into the caller's draft-logits
     // rows (a position's row is last written at the step that commits it) and
     // draws from them; greedy drafting reduces the tile statistics.
-    const int rows = batch * rem;
+    {
     void* dbg = logits_dbg ? logits_dbg + (size_t)t * M * c.vocab : nullptr;
     int dbg_bf16 = 0;
     const int32_t* dbg_valid = nullptr;
@@ -853,6 +909,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
     if (bf16) {
       GemmOut go;
       go.stats = stats;
+      go.vocab_offset = m->vocab_lo;
       go.dbg = dbg;
       go.dbg_rows = lm_rows;
       go.dbg_ld = c.vocab;
@@ -869,19 +926,30 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
       launch_lm_stats_from_logits(logits, rows, c.vocab, stats, dbg, lm_rows, c.vocab, dbg_bf16,
                                   dbg_valid, B, s);
     }
-    if (samp) {
+    if (ph.shard_stats) {
+      // this shard's per-row (max, id, sum): the caller exchanges them
+      launch_lm_reduce(stats, n_vt, rows, n_vt, 1, nullptr, nullptr, ph.shard_stats, s);
+    } else if (samp) {
       if ((st = launch_sampled_draw(samp->q, samp->q_bf16, lm_rows, valid, rows, B, c.vocab, t,
                                     samp->tau, samp->seed, samp->offset, lm_tok, lm_conf,
                                     at<void>(ws, L.draw), sampled_draw_chunks(rows, c.vocab),
                                     attn_cnt, s)))
         return st;
-    } else {
-      launch_lm_reduce(stats, n_vt, rows, lm_tok, lm_conf, s);
+    } else if (ph.commit) {
+      launch_lm_reduce(stats, n_vt, rows, n_vt, 1, lm_tok, lm_conf, nullptr, s);
     }
-    launch_commit(lm_tok, lm_conf, batch, B, rem, k, t, tokens, zrow, lm_rows, cstep, s);
+    }
+  choose:
+    if (ph.commit) {
+      // every shard's statistics, shards in vocabulary order: the argmax over the
+      // whole vocabulary and its max-probability
+      if (ph.gathered)
+        launch_lm_reduce(ph.gathered, ph.world, rows, 1, rows, lm_tok, lm_conf, nullptr, s);
+      launch_commit(lm_tok, lm_conf, batch, B, rem, k, t, tokens, zrow, lm_rows, cstep, s);
+    }
     rem -= k;
   }
-  launch_draft_finish(tokens, cstep, valid, batch, B, draft_tokens, commit_step, s);
+  if (ph.finish) launch_draft_finish(tokens, cstep, valid, batch, B, draft_tokens, commit_step, s);
   return cuda_status();
 }
 
@@ -900,6 +968,7 @@ extern "C" int dflash_draft_block(const dflash_model* m, const int32_t* anchor,
   if (!aligned16(k_cache) || !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(ws) & 255))
     return DFLASH_EINVAL;
   if (cache_cap > c.max_pos) return DFLASH_EINVAL;
+  if (!whole_vocab(m)) return DFLASH_EUNSUPPORTED;  // a shard drafts through the step calls
   if (B * (c.n_q / c.n_kv) > kAttnRows) return DFLASH_EUNSUPPORTED;
   if ((size_t)batch * B > 65535) return DFLASH_EUNSUPPORTED;
   if ((size_t)batch * c.n_kv * 4 > kHeader - kCntOff) return DFLASH_EUNSUPPORTED;
@@ -929,6 +998,7 @@ extern "C" int dflash_draft_block_paged(const dflash_model* m, const int32_t* an
   if (reinterpret_cast<uintptr_t>(ws) & 255) return DFLASH_EINVAL;
   int st = check_pages(m, k_pool, v_pool, n_pages, page_size, page_table, max_pages);
   if (st) return st;
+  if (!whole_vocab(m)) return DFLASH_EUNSUPPORTED;
   if (B * (c.n_q / c.n_kv) > kAttnRows) return DFLASH_EUNSUPPORTED;
   if ((size_t)batch * B > 65535) return DFLASH_EUNSUPPORTED;
   if ((size_t)batch * c.n_kv * 4 > kHeader - kCntOff) return DFLASH_EUNSUPPORTED;
@@ -965,6 +1035,7 @@ extern "C" int dflash_draft_block_sampled(const dflash_model* m, const int32_t* 
       (reinterpret_cast<uintptr_t>(ws) & 255))
     return DFLASH_EINVAL;
   if (cache_cap > c.max_pos) return DFLASH_EINVAL;
+  if (!whole_vocab(m)) return DFLASH_EUNSUPPORTED;
   if (B * (c.n_q / c.n_kv) > kAttnRows) return DFLASH_EUNSUPPORTED;
   // one completion counter per masked row of the draw
   if ((size_t)batch * B * 4 > kHeader - kCntOff) return DFLASH_EUNSUPPORTED;
@@ -980,6 +1051,105 @@ extern "C" int dflash_draft_block_sampled(const dflash_model* m, const int32_t* 
   return draft_impl<float, float, float>(m, anchor, ctx_len, k_cache, v_cache, cache_cap,
                                          KvPages{}, batch, B, n_steps, draft_tokens, commit_step,
                                          nullptr, &sa, ws, s);
+}
+
+// ============================================================== vocabulary-parallel draft
+namespace {
+
+// Shared host checks of the draft step calls (contiguous K/V, bf16 models).
+int check_steps(const dflash_model* m, int batch, int B, int n_steps, int step, void* ws,
+                size_t ws_bytes) {
+  if (!m || batch < 1 || B < 2 || B > 16 || n_steps < 1 || n_steps > B - 1) return DFLASH_EINVAL;
+  if (step < 0 || step >= n_steps || !ws || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return DFLASH_EINVAL;
+  const dflash_config& c = m->cfg;
+  if (c.dtype != DFLASH_BF16) return DFLASH_EUNSUPPORTED;
+  if (B * (c.n_q / c.n_kv) > kAttnRows) return DFLASH_EUNSUPPORTED;
+  if ((size_t)batch * B > 65535) return DFLASH_EUNSUPPORTED;
+  if ((size_t)batch * c.n_kv * 4 > kHeader - kCntOff) return DFLASH_EUNSUPPORTED;
+  if (ws_bytes < draft_layout(c, batch, B).end) return DFLASH_EWORKSPACE;
+  return DFLASH_OK;
+}
+
+int run_phase(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_len,
+              const void* k_cache, const void* v_cache, int cap, int batch, int B, int n_steps,
+              int32_t* draft_tokens, int32_t* commit_step, void* ws, void* stream,
+              const DraftPhase& ph) {
+  return draft_impl<__half, __half, __nv_bfloat16>(m, anchor, ctx_len, k_cache, v_cache, cap,
+                                                   KvPages{}, batch, B, n_steps, draft_tokens,
+                                                   commit_step, nullptr, nullptr, ws,
+                                                   (cudaStream_t)stream, ph);
+}
+
+}  // namespace
+
+extern "C" int dflash_draft_rows(int batch, int B, int n_steps, int step) {
+  if (batch < 1 || B < 2 || n_steps < 1 || n_steps > B - 1 || step < 0 || step >= n_steps)
+    return DFLASH_EINVAL;
+  return batch * masked_before(B, n_steps, step);
+}
+
+extern "C" int dflash_draft_begin(const dflash_model* m, const int32_t* anchor,
+                                  const int32_t* ctx_len, int cache_cap, int batch, int B,
+                                  int n_steps, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_steps(m, batch, B, n_steps, 0, ws, ws_bytes);
+  if (st) return st;
+  if (!anchor || !ctx_len || cache_cap < 1 || cache_cap > m->cfg.max_pos) return DFLASH_EINVAL;
+  DraftPhase ph;
+  ph.forward = ph.commit = ph.finish = false;
+  ph.t1 = 0;
+  return run_phase(m, anchor, ctx_len, nullptr, nullptr, cache_cap, batch, B, n_steps, nullptr,
+                   nullptr, ws, stream, ph);
+}
+
+extern "C" int dflash_draft_forward_shard(const dflash_model* m, const int32_t* ctx_len,
+                                          const void* k_cache, const void* v_cache,
+                                          int cache_cap, int batch, int B, int n_steps, int step,
+                                          void* shard_stats, void* ws, size_t ws_bytes,
+                                          void* stream) {
+  int st = check_steps(m, batch, B, n_steps, step, ws, ws_bytes);
+  if (st) return st;
+  if (!ctx_len || !k_cache || !v_cache || !shard_stats || cache_cap < 1 ||
+      cache_cap > m->cfg.max_pos)
+    return DFLASH_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(shard_stats)) return DFLASH_EINVAL;
+  DraftPhase ph;
+  ph.init = ph.commit = ph.finish = false;
+  ph.t0 = step;
+  ph.t1 = step + 1;
+  ph.shard_stats = static_cast<LmStat*>(shard_stats);
+  return run_phase(m, nullptr, ctx_len, k_cache, v_cache, cache_cap, batch, B, n_steps, nullptr,
+                   nullptr, ws, stream, ph);
+}
+
+extern "C" int dflash_draft_commit_shards(const dflash_model* m, const void* gathered, int world,
+                                          int batch, int B, int n_steps, int step, void* ws,
+                                          size_t ws_bytes, void* stream) {
+  int st = check_steps(m, batch, B, n_steps, step, ws, ws_bytes);
+  if (st) return st;
+  if (!gathered || world < 1 || !aligned16(gathered)) return DFLASH_EINVAL;
+  DraftPhase ph;
+  ph.init = ph.forward = ph.finish = false;
+  ph.t0 = step;
+  ph.t1 = step + 1;
+  ph.gathered = static_cast<const LmStat*>(gathered);
+  ph.world = world;
+  // cap only sizes the attention chunks, which this phase does not launch
+  return run_phase(m, nullptr, nullptr, nullptr, nullptr, m->cfg.max_pos, batch, B, n_steps,
+                   nullptr, nullptr, ws, stream, ph);
+}
+
+extern "C" int dflash_draft_end(const dflash_model* m, int batch, int B, int n_steps,
+                                int32_t* draft_tokens, int32_t* commit_step, void* ws,
+                                size_t ws_bytes, void* stream) {
+  int st = check_steps(m, batch, B, n_steps, 0, ws, ws_bytes);
+  if (st) return st;
+  if (!draft_tokens) return DFLASH_EINVAL;
+  DraftPhase ph;
+  ph.init = ph.forward = ph.commit = false;
+  ph.t1 = 0;
+  return run_phase(m, nullptr, nullptr, nullptr, nullptr, m->cfg.max_pos, batch, B, n_steps,
+                   draft_tokens, commit_step, ws, stream, ph);
 }
 
 // ============================================================== verify
@@ -1002,6 +1172,41 @@ extern "C" int dflash_verify(const void* target_logits, int logits_dtype,
                        out_len, out_cap, seq_lens, accept_len, next_anchor,
                        at<void>(ws, kHeader), chunks, at<unsigned>(ws, kCntOff), err_word(ws),
                        (cudaStream_t)stream);
+}
+
+// ============================================================== vocabulary-parallel verify
+extern "C" int dflash_verify_shard(const void* logits_shard, int logits_dtype, int batch, int B,
+                                   int Vs, int vocab_offset, void* row_argmax, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  if (batch < 0 || B < 2 || B > 32 || Vs < 1 || vocab_offset < 0) return DFLASH_EINVAL;
+  if (logits_dtype != DFLASH_BF16 && logits_dtype != DFLASH_F32) return DFLASH_EINVAL;
+  if ((int64_t)vocab_offset + Vs > 0x7fffffffLL) return DFLASH_EINVAL;
+  if (batch == 0) return DFLASH_OK;
+  if (!logits_shard || !row_argmax || !ws) return DFLASH_EINVAL;
+  if (!aligned16(logits_shard) || (reinterpret_cast<uintptr_t>(ws) & 255)) return DFLASH_EINVAL;
+  if ((int64_t)batch * B > 65535) return DFLASH_EUNSUPPORTED;
+  if (ws_bytes < verify_bytes(batch, B, Vs)) return DFLASH_EWORKSPACE;
+  const int chunks = verify_chunks(batch * B, Vs);
+  return launch_verify_shard(logits_shard, logits_dtype, batch, B, Vs, vocab_offset,
+                             static_cast<ArgPart*>(row_argmax), at<void>(ws, kHeader), chunks,
+                             at<unsigned>(ws, kCntOff), (cudaStream_t)stream);
+}
+
+extern "C" int dflash_verify_merge(const void* gathered, int world, const int32_t* draft_tokens,
+                                   int batch, int B, int V, int32_t* out_tokens, int32_t* out_len,
+                                   int out_cap, int32_t* seq_lens, int32_t* accept_len,
+                                   int32_t* next_anchor, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  if (batch < 0 || B < 2 || B > 32 || V < 1 || out_cap < 1 || world < 1) return DFLASH_EINVAL;
+  if (batch == 0) return DFLASH_OK;
+  if (!gathered || !draft_tokens || !out_tokens || !out_len || !seq_lens || !accept_len ||
+      !next_anchor || !ws)
+    return DFLASH_EINVAL;
+  if (!aligned16(gathered) || (reinterpret_cast<uintptr_t>(ws) & 255)) return DFLASH_EINVAL;
+  if (ws_bytes < kHeader) return DFLASH_EWORKSPACE;
+  return launch_verify_merge(static_cast<const ArgPart*>(gathered), world, draft_tokens, batch, B,
+                             V, out_tokens, out_len, out_cap, seq_lens, accept_len, next_anchor,
+                             err_word(ws), (cudaStream_t)stream);
 }
 
 // ============================================================== sampled verify

@@ -87,17 +87,21 @@ __device__ __forceinline__ void stat_merge(float& mx, int& id, float& se, float 
 }
 
 __global__ void lm_reduce_kernel(const LmStat* __restrict__ stats, int n_vtiles,
-                                 int32_t* __restrict__ tok, float* __restrict__ conf) {
+                                 int64_t row_stride, int64_t tile_stride,
+                                 int32_t* __restrict__ tok, float* __restrict__ conf,
+                                 LmStat* __restrict__ out_stat) {
   pdl_trigger();
   pdl_wait();
   __shared__ float s_m[32], s_s[32];
   __shared__ int s_i[32];
   const int q = blockIdx.x;
-  const LmStat* st = stats + (size_t)q * n_vtiles;
+  const LmStat* st = stats + (int64_t)q * row_stride;
   float mx = -INFINITY, se = 0.f;
   int id = 0x7fffffff;
   for (int t = threadIdx.x; t < n_vtiles; t += blockDim.x) {
-    const LmStat v = st[t];
+    const LmStat v = st[(int64_t)t * tile_stride];
+    if (v.max == -INFINITY) continue;  // an empty tile (a shard with no columns)
+    if (mx == -INFINITY) { mx = v.max; id = v.idx; se = v.sumexp; continue; }
     stat_merge(mx, id, se, v.max, v.idx, v.sumexp);
   }
   // tree merge inside the warp, then across warps
@@ -121,16 +125,19 @@ __global__ void lm_reduce_kernel(const LmStat* __restrict__ stats, int n_vtiles,
       if (M == -INFINITY) { M = s_m[k]; I = s_i[k]; S = s_s[k]; continue; }
       stat_merge(M, I, S, s_m[k], s_i[k], s_s[k]);
     }
-    tok[q] = I;
-    conf[q] = 1.f / S;
+    if (tok) tok[q] = I;
+    if (conf) conf[q] = 1.f / S;
+    if (out_stat) out_stat[q] = LmStat{M, I, S, 0.f};
   }
 }
 
-void launch_lm_reduce(const LmStat* stats, int n_vtiles, int rows, int32_t* tok, float* conf,
+void launch_lm_reduce(const LmStat* stats, int n_tiles, int rows, int64_t row_stride,
+                      int64_t tile_stride, int32_t* tok, float* conf, LmStat* out_stat,
                       cudaStream_t s) {
   if (rows <= 0) return;
   TimedScope ts(s, TC_ROW);
-  launch_pdl(lm_reduce_kernel, dim3(rows), dim3(256), 0, s, 1, stats, n_vtiles, tok, conf);
+  launch_pdl(lm_reduce_kernel, dim3(rows), dim3(256), 0, s, 1, stats, n_tiles, row_stride,
+             tile_stride, tok, conf, out_stat);
 }
 
 // fp32 model type: tile statistics from a full logits matrix [rows, V].

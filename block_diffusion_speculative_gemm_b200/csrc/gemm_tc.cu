@@ -537,7 +537,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           LmStat st;
           st.max = mx;
-          st.idx = w.n0 + q * 32 + bi;
+          st.idx = a.out.vocab_offset + w.n0 + q * 32 + bi;
           st.sumexp = se;
           st.pad = 0.f;
           lm_part[q * kMaxBN + c * 32 + lane] = st;

@@ -113,6 +113,7 @@ struct GemmOut {
   int op = OP_PARTIAL;
   float* part = nullptr;          // OP_PARTIAL: [splits][M][N] fp32
   LmStat* stats = nullptr;        // EPI_LMHEAD: [M][ceil(N/128)]
+  int vocab_offset = 0;           // EPI_LMHEAD: global id of weight row 0 (a vocabulary shard)
   void* dbg = nullptr;            // EPI_LMHEAD, optional: logits rows
   const int32_t* dbg_rows = nullptr;  // token row -> dbg row
   int64_t dbg_ld = 0;             // dbg row stride (elements)
@@ -251,7 +252,11 @@ void launch_draft_init(const int32_t* anchor, const int32_t* ctx_len, int batch,
                        int mask_id, int cap, const KvPages& pages, int32_t* tokens, int32_t* zrow,
                        int32_t* lm_rows, int32_t* cstep, int32_t* req_valid, int32_t* err,
                        cudaStream_t s);
-void launch_lm_reduce(const LmStat* stats, int n_vtiles, int rows, int32_t* tok, float* conf,
+// Per row q: merges the n_tiles statistics stats[q * row_stride + t * tile_stride]
+// (t ascending) into the row's argmax token and max-probability confidence,
+// and, when out_stat is given, the merged (max, id, sum) itself.
+void launch_lm_reduce(const LmStat* stats, int n_tiles, int rows, int64_t row_stride,
+                      int64_t tile_stride, int32_t* tok, float* conf, LmStat* out_stat,
                       cudaStream_t s);
 // dbg (optional): logits rows copied to dbg[dbg_rows[q] * dbg_ld ...] as fp32, or
 // as bf16 when dbg_bf16; rows of requests with !dbg_valid[dbg_rows[q] / B] are
@@ -286,6 +291,20 @@ int launch_verify(const void* logits, int dtype, const int32_t* draft, int batch
                   int32_t* accept_len, int32_t* next_anchor, void* part, int chunks,
                   unsigned* cnt, int32_t* err, cudaStream_t s);
 int verify_chunks(int rows, int V);
+// Vocabulary shard of verify: per row, the (largest logit, lowest global id)
+// over the shard's columns (global id = vocab_offset + column).
+struct ArgPart {
+  float v;
+  int32_t i;
+};
+int launch_verify_shard(const void* logits, int dtype, int batch, int B, int Vs, int vocab_offset,
+                        ArgPart* out, void* part, int chunks, unsigned* cnt, cudaStream_t s);
+// Accept step from per-shard row argmaxes parts[w * batch * B + row], w < world
+// (shards in ascending vocabulary order).
+int launch_verify_merge(const ArgPart* parts, int world, const int32_t* draft, int batch, int B,
+                        int V, int32_t* out_tokens, int32_t* out_len, int out_cap,
+                        int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
+                        int32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- sampled verify
 // Scratch bytes of one sampled-verify call (placed after the workspace header).

@@ -19,11 +19,6 @@ namespace dflash {
 constexpr int kVerifyThreads = 256;
 constexpr int kVerifyUnroll = 4;
 
-struct ArgPart {
-  float v;
-  int32_t i;
-};
-
 template <typename T>
 __device__ __forceinline__ void scan16(const uint4& u, int base, float& best, int& bi) {
   constexpr int W = 16 / sizeof(T);
@@ -35,20 +30,31 @@ __device__ __forceinline__ void scan16(const uint4& u, int base, float& best, in
   }
 }
 
-// Accept step of request r from its B x chunks partials (one warp).
-__device__ void verify_accept(const ArgPart* part, int chunks, int r, const int32_t* draft, int B,
-                              int V, int32_t* out_tokens, int32_t* out_len, int out_cap,
+// Argmax of row `row` from its partials part[row * row_stride + c * chunk_stride],
+// c < chunks (ascending columns), written by other CTAs or kernels: read from L2.
+__device__ __forceinline__ void merge_row(const ArgPart* part, int64_t row_stride,
+                                          int64_t chunk_stride, int chunks, int row,
+                                          float& best, int& bi) {
+  const ArgPart* p = part + (int64_t)row * row_stride;
+  best = __ldcg(&p[0].v);
+  bi = __ldcg(&p[0].i);
+  for (int c = 1; c < chunks; ++c)
+    argmax_merge(best, bi, __ldcg(&p[c * chunk_stride].v), __ldcg(&p[c * chunk_stride].i));
+}
+
+// Accept step of request r from its B rows' partials (one warp; see merge_row).
+__device__ void verify_accept(const ArgPart* part, int64_t row_stride, int64_t chunk_stride,
+                              int chunks, int r, const int32_t* draft, int B, int V,
+                              int32_t* out_tokens, int32_t* out_len, int out_cap,
                               int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
                               int32_t* err) {
   const int lane = threadIdx.x & 31;
   int g = 0;
   int d = 0;
   if (lane < B) {
-    // written by other CTAs of this grid: read from L2
-    const ArgPart* p = part + (size_t)(r * B + lane) * chunks;
-    float best = __ldcg(&p[0].v);
-    int bi = __ldcg(&p[0].i);
-    for (int c = 1; c < chunks; ++c) argmax_merge(best, bi, __ldcg(&p[c].v), __ldcg(&p[c].i));
+    float best;
+    int bi;
+    merge_row(part, row_stride, chunk_stride, chunks, r * B + lane, best, bi);
     g = bi;
     d = draft[(size_t)r * B + lane];
   }
@@ -83,7 +89,7 @@ __global__ void __launch_bounds__(kVerifyThreads)
                   ArgPart* __restrict__ part, unsigned* __restrict__ cnt,
                   const int32_t* __restrict__ draft, int B, int32_t* out_tokens, int32_t* out_len,
                   int out_cap, int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
-                  int32_t* err) {
+                  int32_t* err, ArgPart* shard_out, int vocab_offset) {
   pdl_trigger();
   pdl_wait();
   __shared__ float s_v[kVerifyThreads / 32];
@@ -137,8 +143,18 @@ __global__ void __launch_bounds__(kVerifyThreads)
   __syncthreads();
   if (!s_last || threadIdx.x >= 32) return;
   __threadfence();  // every partial of request r counted before this CTA's reads
-  verify_accept(part, chunks, r, draft, B, V, out_tokens, out_len, out_cap, seq_lens, accept_len,
-                next_anchor, err);
+  if (shard_out != nullptr) {
+    // a vocabulary shard: publish each row's argmax with its global id
+    if (lane < B) {
+      float best;
+      int bi;
+      merge_row(part, chunks, 1, chunks, r * B + lane, best, bi);
+      shard_out[r * B + lane] = ArgPart{best, bi + vocab_offset};
+    }
+  } else {
+    verify_accept(part, chunks, 1, chunks, r, draft, B, V, out_tokens, out_len, out_cap,
+                  seq_lens, accept_len, next_anchor, err);
+  }
   if (lane == 0) cnt[r] = 0;  // ready for the next call
 }
 
@@ -167,13 +183,70 @@ int launch_verify(const void* logits, int dtype, const int32_t* draft, int batch
     const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(logits);
     auto k = vec ? verify_kernel<__nv_bfloat16, true> : verify_kernel<__nv_bfloat16, false>;
     e = launch_pdl(k, grid, block, 0, s, 1, x, V, chunk, chunks, part, cnt, draft, B, out_tokens,
-                   out_len, out_cap, seq_lens, accept_len, next_anchor, err);
+                   out_len, out_cap, seq_lens, accept_len, next_anchor, err, (ArgPart*)nullptr, 0);
   } else {
     const float* x = static_cast<const float*>(logits);
     auto k = vec ? verify_kernel<float, true> : verify_kernel<float, false>;
     e = launch_pdl(k, grid, block, 0, s, 1, x, V, chunk, chunks, part, cnt, draft, B, out_tokens,
-                   out_len, out_cap, seq_lens, accept_len, next_anchor, err);
+                   out_len, out_cap, seq_lens, accept_len, next_anchor, err, (ArgPart*)nullptr, 0);
   }
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
+}
+
+int launch_verify_shard(const void* logits, int dtype, int batch, int B, int Vs, int vocab_offset,
+                        ArgPart* out, void* part_v, int chunks, unsigned* cnt, cudaStream_t s) {
+  const int rows = batch * B;
+  ArgPart* part = reinterpret_cast<ArgPart*>(part_v);
+  int chunk = (Vs + chunks - 1) / chunks;
+  chunk = (chunk + 63) / 64 * 64;
+  const int esz = dtype == DFLASH_BF16 ? 2 : 4;
+  const bool vec = ((size_t)Vs * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(logits) % 16) == 0;
+  const dim3 grid(chunks, rows), block(kVerifyThreads);
+  TimedScope ts(s, TC_VERIFY);
+  cudaError_t e;
+  if (dtype == DFLASH_BF16) {
+    const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(logits);
+    auto k = vec ? verify_kernel<__nv_bfloat16, true> : verify_kernel<__nv_bfloat16, false>;
+    e = launch_pdl(k, grid, block, 0, s, 1, x, Vs, chunk, chunks, part, cnt,
+                   (const int32_t*)nullptr, B, (int32_t*)nullptr, (int32_t*)nullptr, 0,
+                   (int32_t*)nullptr, (int32_t*)nullptr, (int32_t*)nullptr, (int32_t*)nullptr, out,
+                   vocab_offset);
+  } else {
+    const float* x = static_cast<const float*>(logits);
+    auto k = vec ? verify_kernel<float, true> : verify_kernel<float, false>;
+    e = launch_pdl(k, grid, block, 0, s, 1, x, Vs, chunk, chunks, part, cnt,
+                   (const int32_t*)nullptr, B, (int32_t*)nullptr, (int32_t*)nullptr, 0,
+                   (int32_t*)nullptr, (int32_t*)nullptr, (int32_t*)nullptr, (int32_t*)nullptr, out,
+                   vocab_offset);
+  }
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
+}
+
+// One warp per request: row i's argmax merged over the shards in order, then the
+// accept step.
+__global__ void verify_merge_kernel(const ArgPart* __restrict__ parts, int world, int batch,
+                                    const int32_t* __restrict__ draft, int B, int V,
+                                    int32_t* out_tokens, int32_t* out_len, int out_cap,
+                                    int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
+                                    int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= batch) return;
+  verify_accept(parts, 1, (int64_t)batch * B, world, r, draft, B, V, out_tokens, out_len, out_cap,
+                seq_lens, accept_len, next_anchor, err);
+}
+
+int launch_verify_merge(const ArgPart* parts, int world, const int32_t* draft, int batch, int B,
+                        int V, int32_t* out_tokens, int32_t* out_len, int out_cap,
+                        int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
+                        int32_t* err, cudaStream_t s) {
+  TimedScope ts(s, TC_VERIFY);
+  const int wpb = 4;
+  const cudaError_t e =
+      launch_pdl(verify_merge_kernel, dim3((batch + wpb - 1) / wpb), dim3(32 * wpb), 0, s, 1,
+                 parts, world, batch, draft, B, V, out_tokens, out_len, out_cap, seq_lens,
+                 accept_len, next_anchor, err);
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 

@@ -75,6 +75,17 @@ def lib() -> ctypes.CDLL:
                                        sz, vp]
         L.dflash_draft_block.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp,
                                          sz, vp]
+        L.dflash_model_create_shard.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Weights),
+                                                i32, i32, ctypes.POINTER(vp)]
+        L.dflash_draft_rows.argtypes = [i32, i32, i32, i32]
+        L.dflash_draft_begin.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, sz, vp]
+        L.dflash_draft_forward_shard.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp,
+                                                 sz, vp]
+        L.dflash_draft_commit_shards.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp, sz, vp]
+        L.dflash_draft_end.argtypes = [vp, i32, i32, i32, vp, vp, vp, sz, vp]
+        L.dflash_verify_shard.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, sz, vp]
+        L.dflash_verify_merge.argtypes = [vp, i32, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp,
+                                          sz, vp]
         L.dflash_inject_kv_paged.argtypes = [vp, ctypes.POINTER(vp), vp, vp, i32, i32, vp, vp,
                                              i32, i32, vp, i32, vp, sz, vp]
         L.dflash_draft_block_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, i32, i32, i32,
@@ -169,7 +180,7 @@ class Model:
     g_final, W_lm, layers[l] with g_in, Wq, Wk, Wv, Wo, g_post, Wg, Wu, Wd).
     """
 
-    def __init__(self, shape, weights: Dict, max_pos: int):
+    def __init__(self, shape, weights: Dict, max_pos: int, vocab_range=None):
         self.shape = shape
         self.dtype = BF16 if shape.dtype == "bf16" else F32
         self.tdtype = _TORCH_DT[self.dtype]
@@ -194,8 +205,15 @@ class Model:
                     g_ctx=p(weights["g_ctx"], "g_ctx"), g_final=p(weights["g_final"], "g_final"),
                     W_lm=p(weights["W_lm"], "W_lm"), layers=layers)
         handle = ctypes.c_void_p()
-        _check("dflash_model_create", lib().dflash_model_create(ctypes.byref(cfg), ctypes.byref(w),
-                                                                ctypes.byref(handle)))
+        if vocab_range is None:
+            _check("dflash_model_create", lib().dflash_model_create(
+                ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(handle)))
+            self.vocab_range = (0, shape.V)
+        else:
+            lo, hi = (int(v) for v in vocab_range)
+            _check("dflash_model_create_shard", lib().dflash_model_create_shard(
+                ctypes.byref(cfg), ctypes.byref(w), lo, hi, ctypes.byref(handle)))
+            self.vocab_range = (lo, hi)
         self.handle = handle
         self.max_pos = int(max_pos)
 
@@ -365,6 +383,116 @@ def draft_block_sampled(model: Model, anchor: torch.Tensor, ctx_len: torch.Tenso
         batch, B, n_steps, float(temperature), int(seed) & (2**64 - 1), int(offset) & (2**64 - 1),
         _ptr(draft_tokens), _ptr(commit_step), _ptr(draft_logits), dt, _ptr(ws), ws.numel(),
         _stream(stream)))
+
+
+def draft_rows(batch: int, B: int, n_steps: int, step: int) -> int:
+    """Masked rows of the batch at a denoising step (the rows of its shard records)."""
+    n = int(lib().dflash_draft_rows(batch, B, n_steps, step))
+    if n < 0:
+        raise DFlashError("dflash_draft_rows", n)
+    return n
+
+
+def _need_kv(model: Model, k_cache, v_cache, batch):
+    s = model.shape
+    _need(k_cache, "k_cache", model.cache_dtype)
+    _need(v_cache, "v_cache", model.cache_dtype, k_cache.shape)
+    if k_cache.dim() != 5 or tuple(k_cache.shape[:3]) != (s.L, batch, s.nkv) or k_cache.shape[4] != s.hd:
+        raise ValueError("k_cache must be [L, batch, n_kv, cap, head_dim]")
+
+
+def draft_begin(model: Model, anchor: torch.Tensor, ctx_len: torch.Tensor, cache_cap: int, B: int,
+                n_steps: int, ws: torch.Tensor, stream=None):
+    batch = anchor.numel()
+    _need(anchor, "anchor", torch.int32)
+    _need(ctx_len, "ctx_len", torch.int32, (batch,))
+    _need(ws, "ws", torch.uint8)
+    _check("dflash_draft_begin", lib().dflash_draft_begin(
+        model.handle, _ptr(anchor), _ptr(ctx_len), int(cache_cap), batch, B, n_steps, _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def draft_forward_shard(model: Model, ctx_len: torch.Tensor, k_cache: torch.Tensor,
+                        v_cache: torch.Tensor, B: int, n_steps: int, step: int,
+                        shard_stats: torch.Tensor, ws: torch.Tensor, stream=None):
+    """One step's forward; shard_stats (float32 [rows, 4]) receives this shard's
+    (max, id bits, sumexp, 0) record of every masked row."""
+    batch = ctx_len.numel()
+    _need(ctx_len, "ctx_len", torch.int32, (batch,))
+    _need_kv(model, k_cache, v_cache, batch)
+    _need(shard_stats, "shard_stats", torch.float32, (draft_rows(batch, B, n_steps, step), 4))
+    _need(ws, "ws", torch.uint8)
+    _check("dflash_draft_forward_shard", lib().dflash_draft_forward_shard(
+        model.handle, _ptr(ctx_len), _ptr(k_cache), _ptr(v_cache), k_cache.shape[3], batch, B,
+        n_steps, step, _ptr(shard_stats), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def draft_commit_shards(model: Model, gathered: torch.Tensor, batch: int, B: int, n_steps: int,
+                        step: int, ws: torch.Tensor, stream=None):
+    """Merges every shard's records (float32 [world, rows, 4], shards in vocabulary
+    order) and commits the step."""
+    rows = draft_rows(batch, B, n_steps, step)
+    _need(gathered, "gathered", torch.float32)
+    if gathered.dim() != 3 or tuple(gathered.shape[1:]) != (rows, 4):
+        raise ValueError(f"gathered must be [world, {rows}, 4]")
+    _need(ws, "ws", torch.uint8)
+    _check("dflash_draft_commit_shards", lib().dflash_draft_commit_shards(
+        model.handle, _ptr(gathered), gathered.shape[0], batch, B, n_steps, step, _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def draft_end(model: Model, B: int, n_steps: int, draft_tokens: torch.Tensor, ws: torch.Tensor,
+              commit_step: Optional[torch.Tensor] = None, stream=None):
+    batch = draft_tokens.shape[0]
+    _need(draft_tokens, "draft_tokens", torch.int32, (batch, B))
+    if commit_step is not None:
+        _need(commit_step, "commit_step", torch.int32, (batch, B))
+    _need(ws, "ws", torch.uint8)
+    _check("dflash_draft_end", lib().dflash_draft_end(
+        model.handle, batch, B, n_steps, _ptr(draft_tokens), _ptr(commit_step), _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def verify_shard(logits_shard: torch.Tensor, vocab_offset: int, row_argmax: torch.Tensor,
+                 ws: torch.Tensor, stream=None):
+    """Per row of this rank's target-logit columns [batch, B, Vs]: (largest value,
+    global id) into row_argmax (float32 [batch * B, 2], the id as int32 bits)."""
+    if logits_shard.dim() != 3:
+        raise ValueError("logits_shard must be [batch, B, Vs]")
+    batch, B, Vs = logits_shard.shape
+    dt = {torch.bfloat16: BF16, torch.float32: F32}.get(logits_shard.dtype)
+    if dt is None:
+        raise TypeError("logits_shard must be bfloat16 or float32")
+    _need(logits_shard, "logits_shard")
+    _need(row_argmax, "row_argmax", torch.float32, (batch * B, 2))
+    _need(ws, "ws", torch.uint8)
+    _check("dflash_verify_shard", lib().dflash_verify_shard(
+        _ptr(logits_shard), dt, batch, B, Vs, int(vocab_offset), _ptr(row_argmax), _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def verify_merge(gathered: torch.Tensor, draft_tokens: torch.Tensor, V: int,
+                 out_tokens: torch.Tensor, out_len: torch.Tensor, seq_lens: torch.Tensor,
+                 accept_len: torch.Tensor, next_anchor: torch.Tensor, ws: torch.Tensor,
+                 stream=None):
+    """Greedy verify from every shard's row argmaxes (float32 [world, batch * B, 2],
+    shards in vocabulary order)."""
+    batch, B = draft_tokens.shape
+    _need(gathered, "gathered", torch.float32)
+    if gathered.dim() != 3 or tuple(gathered.shape[1:]) != (batch * B, 2):
+        raise ValueError(f"gathered must be [world, {batch * B}, 2]")
+    _need(draft_tokens, "draft_tokens", torch.int32, (batch, B))
+    _need(out_tokens, "out_tokens", torch.int32)
+    if out_tokens.dim() != 2 or out_tokens.shape[0] != batch:
+        raise ValueError("out_tokens must be [batch, out_cap]")
+    for n, t in (("out_len", out_len), ("seq_lens", seq_lens), ("accept_len", accept_len),
+                 ("next_anchor", next_anchor)):
+        _need(t, n, torch.int32, (batch,))
+    _need(ws, "ws", torch.uint8)
+    _check("dflash_verify_merge", lib().dflash_verify_merge(
+        _ptr(gathered), gathered.shape[0], _ptr(draft_tokens), batch, B, int(V), _ptr(out_tokens),
+        _ptr(out_len), out_tokens.shape[1], _ptr(seq_lens), _ptr(accept_len), _ptr(next_anchor),
+        _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def verify(target_logits: torch.Tensor, draft_tokens: torch.Tensor, out_tokens: torch.Tensor,

@@ -22,6 +22,8 @@
  *   dflash_draft_block_sampled  drafting under temperature sampling.
  *   dflash_inject_kv_paged, dflash_draft_block_paged  the same calls over a
  *                       paged K/V store with prefix sharing.
+ *   dflash_draft_begin .. dflash_draft_end, dflash_verify_shard/_merge
+ *                       drafting and verify with the vocabulary split over GPUs.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -256,6 +258,82 @@ int dflash_draft_block_sampled(const dflash_model* m, const int32_t* anchor,
                                uint64_t seed, uint64_t offset, int32_t* draft_tokens,
                                int32_t* commit_step, void* draft_logits, int draft_logits_dtype,
                                void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Vocabulary-parallel LM head and verify across GPUs ("DFlash + Spec V2 深度解析",
+ * §3.3: the engine serves the target with tensor parallelism, --tp-size 8).
+ * Each of `world` ranks holds a contiguous shard [vocab_lo, vocab_hi) of the
+ * vocabulary, shards in rank order covering [0, V).  Per row, a shard reduces
+ * its part of the vocabulary to one 16-byte record; the ranks all-gather the
+ * records (the only exchange: 16 bytes per row per rank, e.g. an NCCL
+ * all-gather on the same stream) and every rank merges them, shards in order,
+ * to the same argmax (lowest global id on ties) and confidence.
+ */
+typedef struct {
+  float max;     /* largest logit of the row in the shard */
+  int32_t id;    /* its global vocabulary id (lowest on ties) */
+  float sumexp;  /* sum over the shard of exp(logit - max) */
+  float pad;
+} dflash_lm_stat;
+
+typedef struct {
+  float value;   /* largest target logit of the row in the shard */
+  int32_t id;    /* its global vocabulary id (lowest on ties) */
+} dflash_row_argmax;
+
+/* A model whose LM head holds only rows [vocab_lo, vocab_hi) of W_lm (w->W_lm
+ * still points at the whole [V, d] matrix; only the shard is copied).  Every
+ * other weight is whole.  DFLASH_BF16 models only.  Such a model drafts only
+ * through the step calls below (the one-call drafts return DFLASH_EUNSUPPORTED). */
+int dflash_model_create_shard(const dflash_config* cfg, const dflash_weights* w, int vocab_lo,
+                              int vocab_hi, dflash_model** out);
+
+/* Masked rows of every request at denoising step `step` (the rows of that
+ * step's records: request-major, positions ascending), or DFLASH_EINVAL. */
+int dflash_draft_rows(int batch, int B, int n_steps, int step);
+
+/* A greedy draft in steps, on every rank with the same inputs:
+ *   dflash_draft_begin          block initialisation and request checks;
+ *   for step = 0 .. n_steps-1:
+ *     dflash_draft_forward_shard  the step's forward; writes this shard's record
+ *                                 of every masked row to shard_stats (device,
+ *                                 dflash_draft_rows(...) records, 16-byte aligned);
+ *     (the caller all-gathers the records of every rank into `gathered`,
+ *      [world][rows] records, rank-major)
+ *     dflash_draft_commit_shards  merges them and commits the step;
+ *   dflash_draft_end            writes draft_tokens / commit_step as
+ *                               dflash_draft_block does.
+ * With world = 1 and a whole-vocabulary model the result equals
+ * dflash_draft_block.  Arguments and errors as dflash_draft_block; the steps of
+ * one draft share the workspace and must not interleave with other calls on it. */
+int dflash_draft_begin(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_len,
+                       int cache_cap, int batch, int B, int n_steps, void* ws, size_t ws_bytes,
+                       void* stream);
+int dflash_draft_forward_shard(const dflash_model* m, const int32_t* ctx_len, const void* k_cache,
+                               const void* v_cache, int cache_cap, int batch, int B, int n_steps,
+                               int step, void* shard_stats, void* ws, size_t ws_bytes,
+                               void* stream);
+int dflash_draft_commit_shards(const dflash_model* m, const void* gathered, int world, int batch,
+                               int B, int n_steps, int step, void* ws, size_t ws_bytes,
+                               void* stream);
+int dflash_draft_end(const dflash_model* m, int batch, int B, int n_steps, int32_t* draft_tokens,
+                     int32_t* commit_step, void* ws, size_t ws_bytes, void* stream);
+
+/* Verify across vocabulary shards.  dflash_verify_shard: logits_shard is
+ * [batch, B, Vs] (this rank's columns, global ids vocab_offset ..
+ * vocab_offset + Vs - 1), row_argmax receives batch * B dflash_row_argmax
+ * records; workspace dflash_verify_workspace_size(batch, B, Vs).
+ * dflash_verify_merge: gathered holds [world][batch * B] records (rank-major,
+ * 16-byte aligned); it takes g_i as the merged argmax and then does exactly
+ * what dflash_verify does (same outputs and device errors; workspace: the
+ * header, dflash_verify_workspace_size(0, B, V) bytes). */
+int dflash_verify_shard(const void* logits_shard, int logits_dtype, int batch, int B, int Vs,
+                        int vocab_offset, void* row_argmax, void* ws, size_t ws_bytes,
+                        void* stream);
+int dflash_verify_merge(const void* gathered, int world, const int32_t* draft_tokens, int batch,
+                        int B, int V, int32_t* out_tokens, int32_t* out_len, int out_cap,
+                        int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor, void* ws,
+                        size_t ws_bytes, void* stream);
 
 /*
  * Greedy verify.

@@ -10,3 +10,4 @@ from .dflash_oracle import __all__  # noqa: F401
 from . import sampled_verify  # noqa: F401
 from . import sampled_draft  # noqa: F401
 from . import paged_kv  # noqa: F401
+from . import vocab_parallel  # noqa: F401
