@@ -8,10 +8,21 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "internal.h"
 
 using namespace dflash;
+
+namespace {
+// One NVTX range per C-ABI call, named after the call: profilers show the
+// library's calls on the host timeline (no cost without a tool attached).
+struct NvtxCall {
+  explicit NvtxCall(const char* name) { nvtxRangePushA(name); }
+  ~NvtxCall() { nvtxRangePop(); }
+};
+}  // namespace
 
 static_assert(sizeof(LmStat) == sizeof(dflash_lm_stat), "shard record layout");
 static_assert(sizeof(ArgPart) == sizeof(dflash_row_argmax), "verify shard record layout");
@@ -106,6 +117,7 @@ struct dflash_model {
   dflash_config cfg;
   int device = 0;
   int vocab_lo = 0, vocab_hi = 0;  // LM-head rows held: [vocab_lo, vocab_hi) of the vocabulary
+  int32_t* range_flag = nullptr;     // set by the packing kernels: a weight overflowed fp16
   size_t esz = 2;
   void* emb = nullptr;
   void* W_fc = nullptr;
@@ -156,11 +168,17 @@ bool copy_rows(void* dst, const void* src, size_t bytes) {
   return src != nullptr && cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToDevice) == cudaSuccess;
 }
 
+// range: set to 1 when a weight does not fit fp16 (|w| >= 65520 rounds to inf).
 __global__ void bf16_to_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
-                                   size_t n) {
+                                   size_t n, int32_t* range) {
+  bool bad = false;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (size_t)gridDim.x * blockDim.x)
-    dst[i] = __float2half_rn(__bfloat162float(src[i]));
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float v = __bfloat162float(src[i]);
+    dst[i] = __float2half_rn(v);
+    bad |= narrow_bad<__half>(v);
+  }
+  if (bad) *range = 1;
 }
 
 // Copies `elems` weight elements into a prepacked buffer.  For the bf16 model
@@ -174,7 +192,7 @@ bool pack_weights(const dflash_model* m, void* dst, const void* src, size_t elem
   if (m->cfg.dtype != DFLASH_BF16) return copy_rows(dst, src, elems * sizeof(float));
   const unsigned blocks = (unsigned)std::min<size_t>((elems + 255) / 256, 148 * 32);
   bf16_to_f16_kernel<<<blocks, 256>>>(static_cast<const __nv_bfloat16*>(src),
-                                      static_cast<__half*>(dst), elems);
+                                      static_cast<__half*>(dst), elems, m->range_flag);
   return cudaGetLastError() == cudaSuccess;
 }
 
@@ -227,6 +245,17 @@ constexpr size_t kCntOff = 256;
 constexpr size_t kHeader = kCntOff + (size_t(128) << 10);
 constexpr int kMaxChunks = 64;
 int g_attn_chunk = 0;  // split-KV chunk override in keys (tests and tuning; 0 = rule)
+// GEMM schedules.  0 (default): the LM head streams K evenly over all workers
+// (stream-K; its tiles are mostly whole, so little is left to finish in the
+// kernel, and the last partial wave of 1187 vocabulary tiles disappears), the
+// projections and the injection take fixed K splits, whose partials the
+// following reduction kernels sum over hundreds of CTAs.  1: fixed splits
+// everywhere.  2: stream-K everywhere (each split tile finished by its last
+// piece inside the GEMM; measured 2x slower for the 256-token projections,
+// whose few tiles split 3-5 ways).
+int g_gemm_sched = 0;
+bool sk_projections() { return g_gemm_sched == 2; }
+bool sk_lm_head() { return g_gemm_sched != 1; }
 constexpr int kAttnRows = 64;
 constexpr int kInjectChunkRows = 16384;
 constexpr int kMaxSplits = 16;
@@ -235,12 +264,12 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct DraftLayout {
   size_t tokens, zrow, lm_rows, cstep, req_valid, lm_tok, lm_conf, x, h, q, kb, vb, o, act, part,
-      attn_o, attn_ml, stats, draw, logits, end;
+      sk, attn_o, attn_ml, stats, draw, logits, end;
   size_t part_elems;  // fp32 elements of split-K partials
 };
 
 struct InjectLayout {
-  size_t c, u, part, req_ok, end;
+  size_t c, u, part, sk, req_ok, end;
   size_t part_elems;
   int chunk_rows;
 };
@@ -277,6 +306,7 @@ DraftLayout draft_layout(const dflash_config& c, int batch, int B) {
   // split-K partials: room for 4 splits of the widest projection
   L.part_elems = 4 * M * (size_t)draft_part_cols(c);
   L.part = take(4 * L.part_elems);
+  L.sk = take(gemm_sk_slot_bytes((int)M));  // stream-K fixup shares
   const size_t arows = (size_t)batch * c.n_kv * kMaxChunks * kAttnRows;
   L.attn_o = take(4 * arows * c.head_dim);
   L.attn_ml = take(8 * arows);
@@ -302,10 +332,13 @@ InjectLayout inject_layout(const dflash_config& c, int max_rows, int batch = 0) 
   off = align256(off + esz * n * c.d);
   L.u = off;  // fc output before its RMSNorm (fp32)
   off = align256(off + 4 * n * c.d);
-  // small row counts may split K up to kMaxSplits ways
-  L.part_elems = (n <= 256 ? (size_t)kMaxSplits : 1) * n * ncol;
+  // row counts up to 256 may split K up to kMaxSplits ways: room for the
+  // largest of those, so a workspace sized for n rows also serves fewer rows
+  L.part_elems = std::max((size_t)kMaxSplits * std::min<size_t>(n, 256), n) * ncol;
   L.part = off;
   off = align256(off + 4 * L.part_elems);
+  L.sk = off;
+  off = align256(off + gemm_sk_slot_bytes(L.chunk_rows));
   L.req_ok = off;
   off = align256(off + 4 * (size_t)std::max(batch, 0));
   L.end = off;
@@ -320,6 +353,15 @@ size_t verify_bytes(int batch, int B, int V) {
 }
 
 int32_t* err_word(void* ws) { return static_cast<int32_t*>(ws); }
+
+// Stream-K scratch of a GEMM: the layout's share slots and the header's
+// completion counters (every kernel using them waits for its predecessor to
+// finish first and leaves them at zero).
+void use_stream_k(GemmOut& o, void* ws, size_t slots_off) {
+  o.sk_slots = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + slots_off);
+  o.sk_cnt = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + kCntOff);
+  o.sk_cnt_cap = (int)((kHeader - kCntOff) / sizeof(unsigned));
+}
 
 template <typename P>
 P* at(void* ws, size_t off) {
@@ -344,15 +386,19 @@ int splits_for(int M, int N, int K, size_t cap_elems) {
 // holding 64 gate rows, then the 64 up rows of the same features.
 template <typename Tin, typename Tout>
 __global__ void pack_gu_kernel(const Tin* __restrict__ wg, const Tin* __restrict__ wu,
-                               Tout* __restrict__ out, int I, int d) {
+                               Tout* __restrict__ out, int I, int d, int32_t* range) {
   const size_t total = (size_t)2 * I * d;
+  bool bad = false;
   for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (size_t)gridDim.x * blockDim.x) {
     const int n = (int)(idx / d), k = (int)(idx % d);
     const int blk = n >> 7, w = n & 127;
     const Tin* src = (w < 64 ? wg : wu) + ((size_t)(blk * 64 + (w & 63))) * d + k;
-    out[idx] = from_f<Tout>(to_f(*src));
+    const float v = to_f(*src);
+    out[idx] = from_f<Tout>(v);
+    bad |= narrow_bad<Tout>(v);
   }
+  if (bad) *range = 1;
 }
 
 }  // namespace
@@ -396,6 +442,9 @@ int model_create(const dflash_config* cfg, const dflash_weights* w, int vocab_lo
     delete m;
     return code;
   };
+  m->range_flag = static_cast<int32_t*>(dmalloc(m, sizeof(int32_t)));
+  if (!m->range_flag || cudaMemset(m->range_flag, 0, sizeof(int32_t)) != cudaSuccess)
+    return fail(DFLASH_ENOMEM);
   m->emb = dmalloc(m, e * V * d);
   m->W_fc = dmalloc(m, e * d * c.n_tap * c.H_t);
   m->W_lm = dmalloc(m, e * Vs * d);
@@ -436,12 +485,12 @@ int model_create(const dflash_config* cfg, const dflash_weights* w, int vocab_lo
       if (c.dtype == DFLASH_BF16)
         pack_gu_kernel<__nv_bfloat16, __half><<<blocks, 256>>>(
             static_cast<const __nv_bfloat16*>(lw.Wg), static_cast<const __nv_bfloat16*>(lw.Wu),
-            static_cast<__half*>((void*)gu), (int)I, (int)d);
+            static_cast<__half*>((void*)gu), (int)I, (int)d, m->range_flag);
       else
         pack_gu_kernel<float, float><<<blocks, 256>>>(static_cast<const float*>(lw.Wg),
                                                      static_cast<const float*>(lw.Wu),
                                                      static_cast<float*>((void*)gu), (int)I,
-                                                     (int)d);
+                                                     (int)d, m->range_flag);
     }
     P.g_in = gain_copy(m, lw.g_in);
     P.g_post = gain_copy(m, lw.g_post);
@@ -503,6 +552,11 @@ int model_create(const dflash_config* cfg, const dflash_weights* w, int vocab_lo
   }
   if (cudaDeviceSynchronize() != cudaSuccess || cudaGetLastError() != cudaSuccess)
     return fail(DFLASH_ECUDA);
+  // the bf16 model type multiplies in fp16: a weight past fp16's range is refused
+  int32_t range = 0;
+  if (cudaMemcpy(&range, m->range_flag, sizeof(range), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return fail(DFLASH_ECUDA);
+  if (range) return fail(DFLASH_EUNSUPPORTED);
   *out = m;
   return DFLASH_OK;
 }
@@ -596,8 +650,10 @@ int inject_impl(const dflash_model* m, const void* const* taps, const int32_t* c
     void* cbuf = at<void>(ws, L.c);
     int st;
     if (c.dtype == DFLASH_BF16) {
-      // u = concat(taps) W_fc^T, c = RMSNorm(u; g_ctx)
-      const int s1 = splits_for(n, c.d, c.n_tap * c.H_t, L.part_elems);
+      // u = concat(taps) W_fc^T, c = RMSNorm(u; g_ctx).  Stream-K: the GEMM
+      // finishes every tile itself and stores u; fixed splits leave partials
+      const bool skm = sk_projections();
+      const int s1 = skm ? 1 : splits_for(n, c.d, c.n_tap * c.H_t, L.part_elems);
       GemmOut o1;
       if (s1 == 1) {
         o1.op = OP_STORE;
@@ -605,12 +661,13 @@ int inject_impl(const dflash_model* m, const void* const* taps, const int32_t* c
       } else {
         o1.part = part;
       }
-      st = gemm_tc(m->mfc, seg, c.n_tap, c.H_t, c.H_t, n, s1, EPI_PARTIAL, o1, err, s);
+      if (skm) use_stream_k(o1, ws, L.sk);
+      st = gemm_tc(m->mfc, seg, c.n_tap, c.H_t, c.H_t, n, skm ? 0 : s1, EPI_PARTIAL, o1, err, s);
       if (st) return st;
       launch_ctx_norm<__half>(s1 == 1 ? o1.f32 : part, s1, n, c.d, m->g_ctx,
-                              static_cast<__half*>(cbuf), c.eps, s);
+                              static_cast<__half*>(cbuf), c.eps, err, s);
       // every layer's K (RoPE) and V into the cache
-      const int s2 = splits_for(n, kvN, c.d, L.part_elems);
+      const int s2 = skm ? 1 : splits_for(n, kvN, c.d, L.part_elems);
       const void* cseg[1] = {cbuf};
       GemmOut o2;
       if (s2 == 1) {
@@ -633,7 +690,8 @@ int inject_impl(const dflash_model* m, const void* const* taps, const int32_t* c
       } else {
         o2.part = part;
       }
-      st = gemm_tc(m->mkv, cseg, 1, c.d, c.d, n, s2, EPI_PARTIAL, o2, err, s);
+      if (skm) use_stream_k(o2, ws, L.sk);
+      st = gemm_tc(m->mkv, cseg, 1, c.d, c.d, n, skm ? 0 : s2, EPI_PARTIAL, o2, err, s);
       if (st) return st;
       if (s2 > 1)
         launch_kv_scatter<__half>(part, s2, n, r0, c.n_layers, c.n_kv, c.head_dim, cu_rows,
@@ -645,7 +703,7 @@ int inject_impl(const dflash_model* m, const void* const* taps, const int32_t* c
       for (int t = 0; t < c.n_tap; ++t) fseg[t] = static_cast<const float*>(seg[t]);
       gemm_simt_f32(static_cast<const float*>(m->W_fc), c.d, c.n_tap * c.H_t, fseg, c.n_tap,
                     c.H_t, n, part, s);
-      launch_ctx_norm<float>(part, 1, n, c.d, m->g_ctx, static_cast<float*>(cbuf), c.eps, s);
+      launch_ctx_norm<float>(part, 1, n, c.d, m->g_ctx, static_cast<float*>(cbuf), c.eps, err, s);
       const float* cseg[1] = {static_cast<const float*>(cbuf)};
       gemm_simt_f32(static_cast<const float*>(m->W_kv), kvN, c.d, cseg, 1, c.d, n, part, s);
       launch_kv_scatter<float>(part, 1, n, r0, c.n_layers, c.n_kv, c.head_dim, cu_rows,
@@ -679,6 +737,7 @@ extern "C" int dflash_inject_kv(const dflash_model* m, const void* const* taps,
                                 const int32_t* cu_rows, const int32_t* start_pos, int batch,
                                 int n_rows, void* k_cache, void* v_cache, int cache_cap, void* ws,
                                 size_t ws_bytes, void* stream) {
+  NvtxCall nvtx_("dflash_inject_kv");
   if (!m || batch < 1 || n_rows < 0 || cache_cap < 1) return DFLASH_EINVAL;
   if (n_rows == 0) return DFLASH_OK;
   const dflash_config& c = m->cfg;
@@ -697,6 +756,7 @@ extern "C" int dflash_inject_kv_paged(const dflash_model* m, const void* const* 
                                       int batch, int n_rows, void* k_pool, void* v_pool,
                                       int n_pages, int page_size, const int32_t* page_table,
                                       int max_pages, void* ws, size_t ws_bytes, void* stream) {
+  NvtxCall nvtx_("dflash_inject_kv_paged");
   if (!m || batch < 1 || n_rows < 0) return DFLASH_EINVAL;
   if (n_rows == 0) return DFLASH_OK;
   const dflash_config& c = m->cfg;
@@ -828,7 +888,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
     const int rows = batch * rem;
     if (!ph.forward) goto choose;
     launch_embed_norm<TE, T>(tokens, static_cast<const TE*>(m->emb), m->layers[0].g_in, x, h, M, c.d,
-                         c.eps, s);
+                         c.eps, err, s);
     for (int l = 0; l < c.n_layers; ++l) {
       const LayerPack& P = m->layers[l];
       const float* g_next = l + 1 < c.n_layers ? m->layers[l + 1].g_in : m->g_final;
@@ -847,13 +907,17 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
         go.nkv = nkv;
         go.hd = hd;
         go.I = c.inter;
+        // stream-K (default): every GEMM applies its fused op itself;
+        // fixed splits: split GEMMs leave partials for the reduction kernels
         int sp = 1;
         auto run = [&](const WeightMap& W, int N, int K, const void* X, int op) {
-          sp = splits_for(M, N, K, L.part_elems);
+          const bool skm = sk_projections();
+          sp = skm ? 1 : splits_for(M, N, K, L.part_elems);
           GemmOut g2 = go;
           g2.op = sp == 1 ? op : OP_PARTIAL;
+          if (skm) use_stream_k(g2, ws, L.sk);
           const void* seg[1] = {X};
-          return gemm_tc(W, seg, 1, K, K, M, sp, EPI_PARTIAL, g2, err, s);
+          return gemm_tc(W, seg, 1, K, K, M, skm ? 0 : sp, EPI_PARTIAL, g2, err, s);
         };
         go.h1 = reinterpret_cast<__half*>(q);
         go.h2 = reinterpret_cast<__half*>(kb);
@@ -861,7 +925,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
         if ((st = run(P.mqkv, qkv_out(c), c.d, h, OP_QKV))) return st;
         if (sp > 1)
           launch_qkv_post<T>(part, sp, M, B, ctx_len, valid, nq, nkv, hd, m->rope_cos,
-                             m->rope_sin, q, kb, vb, s);
+                             m->rope_sin, q, kb, vb, err, s);
         if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, pg, l, c.n_layers, batch, cap,
                                                 ctx_len, valid, B, nq, nkv, hd, attn_o, attn_ml,
                                                 n_chunks, chunk, o, attn_cnt, err, s)))
@@ -869,29 +933,29 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
         go.f32 = x;
         if ((st = run(P.mo, c.d, nq * hd, o, OP_RESID))) return st;
         launch_residual_norm<T>(sp > 1 ? part : nullptr, sp, M, c.d, x, P.g_post, h, nullptr,
-                                c.eps, s);
+                                c.eps, err, s);
         go.h1 = reinterpret_cast<__half*>(act);
         if ((st = run(P.mgu, 2 * c.inter, c.d, h, OP_SWIGLU))) return st;
-        if (sp > 1) launch_swiglu<T>(part, sp, M, c.inter, act, s);
+        if (sp > 1) launch_swiglu<T>(part, sp, M, c.inter, act, err, s);
         if ((st = run(P.md, c.d, c.inter, act, OP_RESID))) return st;
         launch_residual_norm<T>(sp > 1 ? part : nullptr, sp, M, c.d, x, g_next, h, next_rows,
-                                c.eps, s);
+                                c.eps, err, s);
         continue;
       }
       int sp = 1;
       if ((st = gemm(P.mqkv, P.Wqkv, qkv_out(c), c.d, h, part, L.part_elems, &sp))) return st;
       launch_qkv_post<T>(part, sp, M, B, ctx_len, valid, nq, nkv, hd, m->rope_cos, m->rope_sin,
-                         q, kb, vb, s);
+                         q, kb, vb, err, s);
       if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, pg, l, c.n_layers, batch, cap,
                                               ctx_len, valid, B, nq, nkv, hd, attn_o, attn_ml,
                                               n_chunks, chunk, o, attn_cnt, err, s)))
         return st;
       if ((st = gemm(P.mo, P.Wo, c.d, nq * hd, o, part, L.part_elems, &sp))) return st;
-      launch_residual_norm<T>(part, sp, M, c.d, x, P.g_post, h, nullptr, c.eps, s);
+      launch_residual_norm<T>(part, sp, M, c.d, x, P.g_post, h, nullptr, c.eps, err, s);
       if ((st = gemm(P.mgu, P.Wgu, 2 * c.inter, c.d, h, part, L.part_elems, &sp))) return st;
-      launch_swiglu<T>(part, sp, M, c.inter, act, s);
+      launch_swiglu<T>(part, sp, M, c.inter, act, err, s);
       if ((st = gemm(P.md, P.Wd, c.d, c.inter, act, part, L.part_elems, &sp))) return st;
-      launch_residual_norm<T>(part, sp, M, c.d, x, g_next, h, next_rows, c.eps, s);
+      launch_residual_norm<T>(part, sp, M, c.d, x, g_next, h, next_rows, c.eps, err, s);
     }
     // LM head over the still-masked rows (compact, request-major).  Sampled
     // drafting writes every masked row's logits into the caller's draft-logits
@@ -916,8 +980,11 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
       go.dbg_bf16 = dbg_bf16;
       go.dbg_valid = dbg_valid;
       go.B = B;
+      const bool skm = sk_lm_head();
+      if (skm) use_stream_k(go, ws, L.sk);
       const void* seg[1] = {h};
-      if ((st = gemm_tc(m->mlm, seg, 1, c.d, c.d, rows, 1, EPI_LMHEAD, go, err, s))) return st;
+      if ((st = gemm_tc(m->mlm, seg, 1, c.d, c.d, rows, skm ? 0 : 1, EPI_LMHEAD, go, err, s)))
+        return st;
     } else {
       float* logits = at<float>(ws, L.logits);
       const float* seg[1] = {reinterpret_cast<const float*>(h)};
@@ -945,7 +1012,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
       // whole vocabulary and its max-probability
       if (ph.gathered)
         launch_lm_reduce(ph.gathered, ph.world, rows, 1, rows, lm_tok, lm_conf, nullptr, s);
-      launch_commit(lm_tok, lm_conf, batch, B, rem, k, t, tokens, zrow, lm_rows, cstep, s);
+      launch_commit(lm_tok, lm_conf, batch, B, rem, k, t, tokens, zrow, lm_rows, cstep, err, s);
     }
     rem -= k;
   }
@@ -960,6 +1027,7 @@ extern "C" int dflash_draft_block(const dflash_model* m, const int32_t* anchor,
                                   int cache_cap, int batch, int B, int n_steps,
                                   int32_t* draft_tokens, int32_t* commit_step, float* logits_dbg,
                                   void* ws, size_t ws_bytes, void* stream) {
+  NvtxCall nvtx_("dflash_draft_block");
   if (!m || batch < 0 || B < 2 || B > 16 || n_steps < 1 || n_steps > B - 1 || cache_cap < 1)
     return DFLASH_EINVAL;
   if (batch == 0) return DFLASH_OK;
@@ -991,6 +1059,7 @@ extern "C" int dflash_draft_block_paged(const dflash_model* m, const int32_t* an
                                         int n_steps, int32_t* draft_tokens, int32_t* commit_step,
                                         float* logits_dbg, void* ws, size_t ws_bytes,
                                         void* stream) {
+  NvtxCall nvtx_("dflash_draft_block_paged");
   if (!m || batch < 0 || B < 2 || B > 16 || n_steps < 1 || n_steps > B - 1) return DFLASH_EINVAL;
   if (batch == 0) return DFLASH_OK;
   const dflash_config& c = m->cfg;
@@ -1023,6 +1092,7 @@ extern "C" int dflash_draft_block_sampled(const dflash_model* m, const int32_t* 
                                           int32_t* commit_step, void* draft_logits,
                                           int draft_logits_dtype, void* ws, size_t ws_bytes,
                                           void* stream) {
+  NvtxCall nvtx_("dflash_draft_block_sampled");
   if (!m || batch < 0 || B < 2 || B > 16 || n_steps < 1 || n_steps > B - 1 || cache_cap < 1)
     return DFLASH_EINVAL;
   if (!(temperature >= 1e-4f && temperature <= 1e4f)) return DFLASH_EINVAL;
@@ -1092,6 +1162,7 @@ extern "C" int dflash_draft_rows(int batch, int B, int n_steps, int step) {
 extern "C" int dflash_draft_begin(const dflash_model* m, const int32_t* anchor,
                                   const int32_t* ctx_len, int cache_cap, int batch, int B,
                                   int n_steps, void* ws, size_t ws_bytes, void* stream) {
+  NvtxCall nvtx_("dflash_draft_begin");
   int st = check_steps(m, batch, B, n_steps, 0, ws, ws_bytes);
   if (st) return st;
   if (!anchor || !ctx_len || cache_cap < 1 || cache_cap > m->cfg.max_pos) return DFLASH_EINVAL;
@@ -1107,6 +1178,7 @@ extern "C" int dflash_draft_forward_shard(const dflash_model* m, const int32_t* 
                                           int cache_cap, int batch, int B, int n_steps, int step,
                                           void* shard_stats, void* ws, size_t ws_bytes,
                                           void* stream) {
+  NvtxCall nvtx_("dflash_draft_forward_shard");
   int st = check_steps(m, batch, B, n_steps, step, ws, ws_bytes);
   if (st) return st;
   if (!ctx_len || !k_cache || !v_cache || !shard_stats || cache_cap < 1 ||
@@ -1125,6 +1197,7 @@ extern "C" int dflash_draft_forward_shard(const dflash_model* m, const int32_t* 
 extern "C" int dflash_draft_commit_shards(const dflash_model* m, const void* gathered, int world,
                                           int batch, int B, int n_steps, int step, void* ws,
                                           size_t ws_bytes, void* stream) {
+  NvtxCall nvtx_("dflash_draft_commit_shards");
   int st = check_steps(m, batch, B, n_steps, step, ws, ws_bytes);
   if (st) return st;
   if (!gathered || world < 1 || !aligned16(gathered)) return DFLASH_EINVAL;
@@ -1142,6 +1215,7 @@ extern "C" int dflash_draft_commit_shards(const dflash_model* m, const void* gat
 extern "C" int dflash_draft_end(const dflash_model* m, int batch, int B, int n_steps,
                                 int32_t* draft_tokens, int32_t* commit_step, void* ws,
                                 size_t ws_bytes, void* stream) {
+  NvtxCall nvtx_("dflash_draft_end");
   int st = check_steps(m, batch, B, n_steps, 0, ws, ws_bytes);
   if (st) return st;
   if (!draft_tokens) return DFLASH_EINVAL;
@@ -1158,6 +1232,7 @@ extern "C" int dflash_verify(const void* target_logits, int logits_dtype,
                              int32_t* out_tokens, int32_t* out_len, int out_cap, int32_t* seq_lens,
                              int32_t* accept_len, int32_t* next_anchor, void* ws, size_t ws_bytes,
                              void* stream) {
+  NvtxCall nvtx_("dflash_verify");
   if (batch < 0 || B < 2 || B > 32 || V < 1 || out_cap < 1) return DFLASH_EINVAL;
   if (logits_dtype != DFLASH_BF16 && logits_dtype != DFLASH_F32) return DFLASH_EINVAL;
   if (batch == 0) return DFLASH_OK;
@@ -1178,6 +1253,7 @@ extern "C" int dflash_verify(const void* target_logits, int logits_dtype,
 extern "C" int dflash_verify_shard(const void* logits_shard, int logits_dtype, int batch, int B,
                                    int Vs, int vocab_offset, void* row_argmax, void* ws,
                                    size_t ws_bytes, void* stream) {
+  NvtxCall nvtx_("dflash_verify_shard");
   if (batch < 0 || B < 2 || B > 32 || Vs < 1 || vocab_offset < 0) return DFLASH_EINVAL;
   if (logits_dtype != DFLASH_BF16 && logits_dtype != DFLASH_F32) return DFLASH_EINVAL;
   if ((int64_t)vocab_offset + Vs > 0x7fffffffLL) return DFLASH_EINVAL;
@@ -1197,6 +1273,7 @@ extern "C" int dflash_verify_merge(const void* gathered, int world, const int32_
                                    int out_cap, int32_t* seq_lens, int32_t* accept_len,
                                    int32_t* next_anchor, void* ws, size_t ws_bytes,
                                    void* stream) {
+  NvtxCall nvtx_("dflash_verify_merge");
   if (batch < 0 || B < 2 || B > 32 || V < 1 || out_cap < 1 || world < 1) return DFLASH_EINVAL;
   if (batch == 0) return DFLASH_OK;
   if (!gathered || !draft_tokens || !out_tokens || !out_len || !seq_lens || !accept_len ||
@@ -1223,6 +1300,7 @@ extern "C" int dflash_verify_sampled(const void* target_logits, const void* draf
                                      int out_cap, int32_t* seq_lens, int32_t* accept_len,
                                      int32_t* next_anchor, void* ws, size_t ws_bytes,
                                      void* stream) {
+  NvtxCall nvtx_("dflash_verify_sampled");
   if (batch < 0 || B < 2 || B > 32 || V < 1 || out_cap < 1) return DFLASH_EINVAL;
   if (logits_dtype != DFLASH_BF16 && logits_dtype != DFLASH_F32) return DFLASH_EINVAL;
   if (!(temperature >= 1e-4f && temperature <= 1e4f)) return DFLASH_EINVAL;
@@ -1283,6 +1361,33 @@ extern "C" int dflash_debug_gemm_tiled(const void* Wt, int N, int K, const void*
                  (cudaStream_t)stream);
 }
 
+extern "C" size_t dflash_debug_gemm_streamk_ws_bytes(int M) {
+  if (M < 1) return 0;
+  return kHeader + align256(gemm_sk_slot_bytes(M));
+}
+
+extern "C" int dflash_debug_gemm_streamk(const void* Wt, int N, int K, const void* X, int M,
+                                         int elem, float* out, void* ws, size_t ws_bytes,
+                                         void* stream) {
+  if (!Wt || !X || !out || !ws || N < 1 || K < 64 || K % 64 || M < 1) return DFLASH_EINVAL;
+  if (!aligned16(Wt) || !aligned16(X) || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return DFLASH_EINVAL;
+  if (elem != DFLASH_BF16 && elem != DFLASH_F16) return DFLASH_EINVAL;
+  if (ws_bytes < kHeader + gemm_sk_slot_bytes(M)) return DFLASH_EWORKSPACE;
+  WeightMap wm;
+  memset(&wm.map, 0, sizeof(wm.map));
+  wm.N = N;
+  wm.K = K;
+  wm.elem = elem;
+  if (!set_tiled_weights(wm, Wt)) return DFLASH_ECUDA;
+  GemmOut o;
+  o.op = OP_STORE;
+  o.f32 = out;
+  use_stream_k(o, ws, kHeader);
+  const void* seg[1] = {X};
+  return gemm_tc(wm, seg, 1, K, K, M, 0, EPI_PARTIAL, o, err_word(ws), (cudaStream_t)stream);
+}
+
 extern "C" size_t dflash_debug_tiled_bytes(int N, int K) {
   if (N < 1 || K < 64 || K % 64) return 0;
   return tiled_bytes(N, K);
@@ -1329,6 +1434,12 @@ extern "C" int dflash_debug_attn_chunk(int keys) {
 extern "C" int dflash_debug_split_weight(float w) {
   if (!(w >= 0.f && w <= 64.f)) return DFLASH_EINVAL;
   gemm_set_split_weight(w);
+  return DFLASH_OK;
+}
+
+extern "C" int dflash_debug_gemm_schedule(int sched) {
+  if (sched < 0 || sched > 2) return DFLASH_EINVAL;
+  g_gemm_sched = sched;
   return DFLASH_OK;
 }
 

@@ -222,7 +222,8 @@ template <int HD, int MT>
 __global__ void __launch_bounds__(kThreads)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __half* __restrict__ q, const __half* __restrict__ kb,
-                   const __half* __restrict__ vb, const KvPages pg, int layer, int batch, int cap,
+                   const __half* __restrict__ vb, const KvPages pg, long long kv_rows, int layer,
+                   int batch, int cap,
                    const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ req_valid,
                    int B, int nq, int nkv, int chunk, int n_chunks, float* __restrict__ part_o,
                    float* __restrict__ part_ml, unsigned* __restrict__ cnt,
@@ -286,8 +287,9 @@ __global__ void __launch_bounds__(kThreads)
     // the tile's first key position; a paged store finds its row through the
     // request's page table (a tile never crosses a page)
     const int p0 = k0 + t * kKeys;
-    const int y = pg.table == nullptr ? row_base + p0
-                                      : (int)kv_row(pg, layer, batch, r, nkv, g, cap, p0);
+    int y = pg.table == nullptr ? row_base + p0
+                                : (int)kv_row(pg, layer, batch, r, nkv, g, cap, p0);
+    if (!DFLASH_CHECK(y >= 0 && y < kv_rows, err)) y = 0;  // a tile inside the store
 #pragma unroll
     for (int h = 0; h < HALVES; ++h) {
       tma_load_2d(sK + h * kKeys * 128, &tmK, full(st), h * 64, y, policy_evict_first());
@@ -518,7 +520,7 @@ __global__ void __launch_bounds__(kThreads)
 
 template <int HD, int MT>
 int launch_cfg(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q, const __half* kb,
-               const __half* vb, const KvPages& pg, int layer, int batch, int cap,
+               const __half* vb, const KvPages& pg, long long kv_rows, int layer, int batch, int cap,
                const int32_t* ctx_len,
                const int32_t* req_valid, int B, int nq, int nkv, int chunk, int n_chunks,
                float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
@@ -530,7 +532,7 @@ int launch_cfg(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q, co
   dim3 grid(n_chunks, nkv, batch);
   const cudaError_t e =
       launch_pdl(attn_tc_kernel<HD, MT>, grid, dim3(kThreads), smem, s, 1, tk, tv, q, kb, vb, pg,
-                 layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, part_o,
+                 kv_rows, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, part_o,
                  part_ml, cnt, o, err);
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
@@ -550,12 +552,12 @@ int launch_hd(const __half* q, const __half* kb, const __half* vb, const __half*
     return DFLASH_ECUDA;
   const int R = B * (nq / nkv);
   if (R <= 16)
-    return launch_cfg<HD, 1>(tk, tv, q, kb, vb, pg, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
+    return launch_cfg<HD, 1>(tk, tv, q, kb, vb, pg, rows, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
                              chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
   if (R <= 32)
-    return launch_cfg<HD, 2>(tk, tv, q, kb, vb, pg, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
+    return launch_cfg<HD, 2>(tk, tv, q, kb, vb, pg, rows, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
                              chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
-  return launch_cfg<HD, 4>(tk, tv, q, kb, vb, pg, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
+  return launch_cfg<HD, 4>(tk, tv, q, kb, vb, pg, rows, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
                            chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
 }
 

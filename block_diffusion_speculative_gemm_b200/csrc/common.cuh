@@ -27,10 +27,30 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
   return __float2bfloat16_rn(v);
 }
 
+// True when v does not fit T: an fp16 store of a value that rounds past the
+// largest finite fp16 (|v| >= 65520) or of NaN.  fp32 and bf16 hold every
+// finite fp32 value of the path.
+template <typename T> __device__ __forceinline__ bool narrow_bad(float v) { return false; }
+template <> __device__ __forceinline__ bool narrow_bad<__half>(float v) {
+  return !(fabsf(v) < 65520.f);
+}
+
 // ---------------------------------------------------------------- errors
 __device__ __forceinline__ void set_error(int32_t* err, int bits) {
   if (err) atomicOr(err, bits);
 }
+
+// Bounds-checked build (-DDFLASH_CHECKED), the stand-in for a memory checker:
+// DFLASH_CHECK(cond, err) is true when cond holds; otherwise it sets
+// DFLASH_DEV_CHECK in err and is false, so that the access it guards is
+// skipped (never a trap).  In the normal build it is `true` and cond is not
+// evaluated.
+#ifdef DFLASH_CHECKED
+#define DFLASH_CHECK(cond, err) \
+  ((cond) ? true : (::dflash::set_error((err), DFLASH_DEV_CHECK), false))
+#else
+#define DFLASH_CHECK(cond, err) true
+#endif
 
 // ---------------------------------------------------------------- reductions
 __device__ __forceinline__ float warp_sum(float v) {

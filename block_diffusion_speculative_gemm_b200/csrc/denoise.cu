@@ -195,14 +195,15 @@ void launch_lm_stats_from_logits(const float* logits, int rows, int V, LmStat* s
 // own request's rows of zrow/tokens/cstep and its own compact range of lm_rows.
 __global__ void commit_kernel(const int32_t* __restrict__ tok, const float* __restrict__ conf,
                               int batch, int B, int rem, int k, int step, int32_t* tokens,
-                              int32_t* zrow, int32_t* lm_rows, int32_t* cstep) {
+                              int32_t* zrow, int32_t* lm_rows, int32_t* cstep, int32_t* err) {
   pdl_trigger();
   pdl_wait();
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= batch) return;
   const int m = r * B + lane;
-  const int q = lane < B ? zrow[m] : -1;
+  int q = lane < B ? zrow[m] : -1;
+  if (q >= 0 && !DFLASH_CHECK(q < batch * rem, err)) q = -1;
   const bool live = q >= 0;
   const float c = live ? conf[q] : -INFINITY;
   const int t = live ? tok[q] : 0;
@@ -235,11 +236,11 @@ __global__ void commit_kernel(const int32_t* __restrict__ tok, const float* __re
 
 void launch_commit(const int32_t* tok, const float* conf, int batch, int B, int rem, int k,
                    int step, int32_t* tokens, int32_t* zrow, int32_t* lm_rows, int32_t* cstep,
-                   cudaStream_t s) {
+                   int32_t* err, cudaStream_t s) {
   TimedScope ts(s, TC_ROW);
   const int wpb = 4;
   launch_pdl(commit_kernel, dim3((batch + wpb - 1) / wpb), dim3(32 * wpb), 0, s, 1, tok, conf,
-      batch, B, rem, k, step, tokens, zrow, lm_rows, cstep);
+      batch, B, rem, k, step, tokens, zrow, lm_rows, cstep, err);
 }
 
 __global__ void draft_finish_kernel(const int32_t* __restrict__ tokens,

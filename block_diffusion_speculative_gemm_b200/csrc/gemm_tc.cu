@@ -58,6 +58,12 @@ struct GemmArgs {
   int epi_bytes;      // shared bytes of the epilogue region
   uint32_t idesc;     // tcgen05 instruction descriptor (operand type, tile_rows x BN)
   const uint8_t* a_tiled;  // pre-tiled weights (bulk copies) or null (tensor map)
+  // stream-K schedule (sk = 1): workers (CTAs, or pairs) take equal shares of
+  // the sk_W = tiles * n_kb (tile, k-block) iterations, tiles in order; a tile
+  // split between workers is finished by whichever of its pieces arrives last
+  int sk;
+  int sk_P;
+  long long sk_W;
   GemmOut out;
   int32_t* err;
 };
@@ -75,29 +81,43 @@ constexpr int kLmSmem = 4 * kLmTr * 4 + 4 * kMaxBN * (int)sizeof(LmStat);
 // st[j * kStLd + r] = Y[m_base + j][n0 + r]; t = epilogue thread (0..127).
 // For OP_KV, tok_req/tok_pos hold each token's request and position (request
 // -1: skip) and tok_base the token's row in the K/V store at layer 0, head 0.
+// fp16 results that overflow set DFLASH_DEV_RANGE in err.
+//
+// Every op issues all of a chunk's global loads (the residual stream, the RoPE
+// table entries) before its first store: a load placed after a store the
+// compiler cannot prove disjoint would wait for it, and 32 tokens of
+// dependent round trips per chunk would stall the epilogue.
 __device__ __forceinline__ void apply_op(const GemmOut& o, int M, int N, const float* st,
                                          const int* tok_req, const int* tok_pos,
-                                         const long long* tok_base, int m_base, int n0, int t) {
+                                         const long long* tok_base, int m_base, int n0, int t,
+                                         int32_t* err) {
+  bool bad = false;
+  const int jn = min(32, M - m_base);  // tokens of this chunk
   switch (o.op) {
     case OP_STORE:
     case OP_RESID: {
       const int n = n0 + t;
       if (n >= N) break;
-      for (int j = 0; j < 32; ++j) {
-        const int m = m_base + j;
-        if (m >= M) break;
-        float* d = o.f32 + (size_t)m * N + n;
-        *d = (o.op == OP_RESID ? *d : 0.f) + st[j * kStLd + t];
-      }
+      float* base = o.f32 + (size_t)m_base * N + n;
+      float old[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        old[j] = (o.op == OP_RESID && j < jn) ? base[(size_t)j * N] : 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < jn) base[(size_t)j * N] = old[j] + st[j * kStLd + t];
     } break;
     case OP_SWIGLU: {
       const int p = t & 63, par = t >> 6;
       const int i = (n0 >> 1) + p;
-      for (int j = par; j < 32; j += 2) {
-        const int m = m_base + j;
-        if (m >= M) break;
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const int j = par + 2 * jj;
+        if (j >= jn) break;
         const float g = st[j * kStLd + p], u = st[j * kStLd + p + 64];
-        o.h1[(size_t)m * o.I + i] = __float2half_rn(g / (1.f + expf(-g)) * u);
+        const float y = g / (1.f + expf(-g)) * u;
+        o.h1[(size_t)(m_base + j) * o.I + i] = __float2half_rn(y);
+        bad |= narrow_bad<__half>(y);
       }
     } break;
     case OP_QKV: {
@@ -106,25 +126,32 @@ __device__ __forceinline__ void apply_op(const GemmOut& o, int M, int N, const f
       const int hl = p / half, i = p % half;
       const int ra = hl * hd + i;
       const int head = (n0 + hl * hd) / hd;
-      for (int j = par; j < 32; j += 2) {
-        const int m = m_base + j;
-        if (m >= M) break;
-        float x1 = st[j * kStLd + ra], x2 = st[j * kStLd + ra + half];
-        __half* dst;
-        if (head < o.nq + o.nkv) {
-          const int r = m / o.B;
-          const int pos = (o.req_valid[r] ? o.ctx_len[r] : 0) + m % o.B;
-          const float c = o.cos_t[(size_t)pos * half + i], sn = o.sin_t[(size_t)pos * half + i];
-          const float y1 = x1 * c - x2 * sn, y2 = x2 * c + x1 * sn;
-          x1 = y1;
-          x2 = y2;
-          dst = head < o.nq ? o.h1 + ((size_t)m * o.nq + head) * hd
-                            : o.h2 + ((size_t)m * o.nkv + head - o.nq) * hd;
-        } else {
-          dst = o.h3 + ((size_t)m * o.nkv + head - o.nq - o.nkv) * hd;
+      const bool rope = head < o.nq + o.nkv;
+      float cs[16], sn[16];
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const int j = par + 2 * jj;
+        cs[jj] = 1.f;
+        sn[jj] = 0.f;
+        if (rope && j < jn) {
+          const size_t e = (size_t)tok_pos[j] * half + i;
+          cs[jj] = o.cos_t[e];
+          sn[jj] = o.sin_t[e];
         }
-        dst[i] = __float2half_rn(x1);
-        dst[i + half] = __float2half_rn(x2);
+      }
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const int j = par + 2 * jj;
+        if (j >= jn) break;
+        const int m = m_base + j;
+        const float x1 = st[j * kStLd + ra], x2 = st[j * kStLd + ra + half];
+        const float y1 = x1 * cs[jj] - x2 * sn[jj], y2 = x2 * cs[jj] + x1 * sn[jj];
+        __half* dst = head < o.nq    ? o.h1 + ((size_t)m * o.nq + head) * hd
+                      : rope         ? o.h2 + ((size_t)m * o.nkv + head - o.nq) * hd
+                                     : o.h3 + ((size_t)m * o.nkv + head - o.nq - o.nkv) * hd;
+        dst[i] = __float2half_rn(y1);
+        dst[i + half] = __float2half_rn(y2);
+        bad |= narrow_bad<__half>(y1) || narrow_bad<__half>(y2);
       }
     } break;
     case OP_KV: {
@@ -137,28 +164,40 @@ __device__ __forceinline__ void apply_op(const GemmOut& o, int M, int N, const f
       const int layer = nl / per_layer, wl = nl % per_layer;
       const bool is_v = wl >= o.nkv * hd;
       const int head = (wl % (o.nkv * hd)) / hd;
-      for (int j = par; j < 32; j += 2) {
-        const int m = m_base + j;
-        if (m >= M) break;
-        const int req = tok_req[j];
-        if (req < 0) continue;
-        const int pos = tok_pos[j];
-        float x1 = st[j * kStLd + ra], x2 = st[j * kStLd + ra + half];
-        if (!is_v) {
-          const float c = o.cos_t[(size_t)pos * half + i], sn = o.sin_t[(size_t)pos * half + i];
-          const float y1 = x1 * c - x2 * sn, y2 = x2 * c + x1 * sn;
-          x1 = y1;
-          x2 = y2;
+      float cs[16], sn[16];
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const int j = par + 2 * jj;
+        cs[jj] = 1.f;
+        sn[jj] = 0.f;
+        if (!is_v && j < jn && tok_req[j] >= 0) {
+          const size_t e = (size_t)tok_pos[j] * half + i;
+          cs[jj] = o.cos_t[e];
+          sn[jj] = o.sin_t[e];
         }
-        __half* dst = (is_v ? o.h2 : o.h1) +
-                      (size_t)(layer * o.kv_ls + tok_base[j] + head * o.kv_hs) * hd;
-        dst[i] = __float2half_rn(x1);
-        dst[i + half] = __float2half_rn(x2);
+      }
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const int j = par + 2 * jj;
+        if (j >= jn) break;
+        if (tok_req[j] < 0) continue;
+        const float x1 = st[j * kStLd + ra], x2 = st[j * kStLd + ra + half];
+        const float y1 = x1 * cs[jj] - x2 * sn[jj], y2 = x2 * cs[jj] + x1 * sn[jj];
+        const long long drow = layer * o.kv_ls + tok_base[j] + head * o.kv_hs;
+        if (!DFLASH_CHECK(drow >= 0 && tok_base[j] + head * o.kv_hs < o.kv_ls &&
+                              layer < N / per_layer,
+                          err))
+          continue;
+        __half* dst = (is_v ? o.h2 : o.h1) + (size_t)drow * hd;
+        dst[i] = __float2half_rn(y1);
+        dst[i + half] = __float2half_rn(y2);
+        bad |= narrow_bad<__half>(y1) || narrow_bad<__half>(y2);
       }
     } break;
     default:
       break;
   }
+  if (bad) set_error(err, DFLASH_DEV_RANGE);
 }
 
 __host__ __device__ inline int tmem_cols_for(int bn) {
@@ -170,6 +209,34 @@ __host__ __device__ inline int tmem_cols_for(int bn) {
 struct Unit {
   int n0, m0, split, kb0, nk, tile;
 };
+
+// Stream-K: start of worker c's iteration range, and the worker whose range
+// holds iteration g (ranges are [c W / P, (c + 1) W / P), W >= P).
+__device__ __forceinline__ long long sk_g0(const GemmArgs& a, int c) {
+  return (long long)c * a.sk_W / a.sk_P;
+}
+__device__ __forceinline__ int sk_worker_of(const GemmArgs& a, long long g) {
+  return (int)(((g + 1) * a.sk_P + a.sk_W - 1) / a.sk_W) - 1;
+}
+// Fixup slot of worker c's piece of the tile starting at iteration tg: each
+// worker has at most two pieces that are not whole tiles, its first and last.
+__device__ __forceinline__ int sk_slot(const GemmArgs& a, int c, long long tg) {
+  return 2 * c + (sk_g0(a, c) >= tg ? 0 : 1);
+}
+
+// The work items of one worker in order: split units u = cid, cid + ncl, ...,
+// or the stream-K pieces of the worker's range.
+struct WorkIter {
+  long long g, g1;
+  int u;
+};
+__device__ __forceinline__ WorkIter work_begin(const GemmArgs& a, int cid) {
+  WorkIter it;
+  it.u = cid;
+  it.g = a.sk ? sk_g0(a, cid) : 0;
+  it.g1 = a.sk ? sk_g0(a, cid + 1) : 0;
+  return it;
+}
 
 // Unit u of the CTA with pair rank `rank` (0 outside pairs): its 128 weight
 // rows start at n0.
@@ -184,6 +251,27 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int rank) 
   w.kb0 = w.split * a.kb_per_split;
   w.nk = min(a.n_kb, w.kb0 + a.kb_per_split) - w.kb0;
   return w;
+}
+
+// Next work item of a worker; false when its work is done.
+__device__ __forceinline__ bool work_next(const GemmArgs& a, int ncl, int rank, WorkIter& it,
+                                          Unit& w) {
+  if (!a.sk) {
+    if (it.u >= a.units) return false;
+    w = decode_unit(a, it.u, rank);
+    it.u += ncl;
+    return true;
+  }
+  if (it.g >= it.g1) return false;
+  const int t = (int)(it.g / a.n_kb);
+  w.tile = t;
+  w.split = 0;
+  w.kb0 = (int)(it.g - (long long)t * a.n_kb);
+  w.nk = (int)min((long long)(a.n_kb - w.kb0), it.g1 - it.g);
+  w.m0 = (t / a.tiles_n) * a.BN;
+  w.n0 = (t % a.tiles_n) * a.tile_rows + rank * kTileN;
+  it.g += w.nk;
+  return true;
 }
 
 // Contiguous global -> shared bulk copy completing on an mbarrier.
@@ -244,6 +332,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   long long* tok_base = reinterpret_cast<long long*>(tok_pos + 32);
   uint64_t* bars = reinterpret_cast<uint64_t*>(epi_smem + a.epi_bytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * a.stages + 4);
+  volatile uint32_t* sk_flag = tmem_slot + 1;  // stream-K: this piece finishes its tile
   const uint32_t smem0 = smem_u32(smem);
   auto sA = [&](int s) { return smem0 + s * stage_bytes; };
   auto sB = [&](int s) { return smem0 + s * stage_bytes + kTileN * 128; };
@@ -299,7 +388,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // walk at its own offset so that the SMs do not all request the same
       // activation rows of L2 at the same moment)
       auto kx_of = [&](const Unit& w, int i) {
-        int ki = i + (int)((cid * 7u) % (unsigned)w.nk);
+        // stream-K pieces keep the natural order: the fixup sums pieces in order
+        int ki = i + (a.sk ? 0 : (int)((cid * 7u) % (unsigned)w.nk));
         if (ki >= w.nk) ki -= w.nk;
         return (w.kb0 + ki) * kTileK;
       };
@@ -332,18 +422,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // the first unit are requested before the predecessor kernel has
       // finished (their empty barriers are fresh), the activations after it.
       int pre = 0;
-      if (cid < a.units) {
-        const Unit w = decode_unit(a, cid, rank);
-        pre = min(a.stages, w.nk);
-        for (int i = 0; i < pre; ++i) {
-          expect(i);
-          load_w(i, w, kx_of(w, i));
+      {
+        WorkIter wi = work_begin(a, cid);
+        Unit w;
+        if (work_next(a, ncl, rank, wi, w)) {
+          pre = min(a.stages, w.nk);
+          for (int i = 0; i < pre; ++i) {
+            expect(i);
+            load_w(i, w, kx_of(w, i));
+          }
         }
       }
       pdl_wait();
       uint32_t it = 0;
-      for (int u = cid; u < a.units && ok; u += ncl) {
-        const Unit w = decode_unit(a, u, rank);
+      WorkIter wi = work_begin(a, cid);
+      Unit w;
+      while (ok && work_next(a, ncl, rank, wi, w)) {
         for (int i = 0; i < w.nk; ++i, ++it) {
           const int s = it % a.stages;
           const uint32_t ph = (it / a.stages) & 1;
@@ -365,8 +459,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0 && rank == 0) {
       uint32_t it = 0;
       int j = 0;
-      for (int u = cid; u < a.units && ok; u += ncl, ++j) {
-        const Unit w = decode_unit(a, u, 0);
+      WorkIter wi = work_begin(a, cid);
+      Unit w;
+      for (; ok && work_next(a, ncl, 0, wi, w); ++j) {
         const int b = j & 1;
         if (!mbar_wait(acc_empty(b), ((j >> 1) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
@@ -407,8 +502,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int nchunk = a.BN / 32;
     pdl_wait();  // the epilogue reads and writes other kernels' buffers
     int j = 0;
-    for (int u = cid; u < a.units; u += ncl, ++j) {
-      const Unit w = decode_unit(a, u, rank);
+    WorkIter wi = work_begin(a, cid);
+    Unit w;
+    for (; work_next(a, ncl, rank, wi, w); ++j) {
       const int b = j & 1;
       // the second half of a pair's last tile can lie past the weights
       const bool live = w.n0 < a.N;
@@ -434,9 +530,83 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         release();
         continue;
       }
-      // token -> (request, cache position) for OP_KV, one thread per token of the chunk
+      // Stream-K: a piece that is not a whole tile stores its share in its
+      // fixup slot ([token][128 rows] fp32) and counts itself on the tile's
+      // counter; the last piece to arrive sums every piece's share in worker
+      // order (its own from TMEM), so the result does not depend on the order
+      // of arrival, and applies the epilogue.  Nobody waits for anybody.
+      bool fix = false;
+      int c_lo = 0, c_hi = -1;
+      long long tg = 0;
+      auto slot_ptr = [&](int worker) {
+        return a.out.sk_slots +
+               ((size_t)sk_slot(a, worker, tg) * (PAIR ? 2 : 1) + rank) * kTileN * a.BN;
+      };
+      if (a.sk && !(w.kb0 == 0 && w.nk == a.n_kb)) {
+        tg = (long long)w.tile * a.n_kb;
+        c_lo = sk_worker_of(a, tg);
+        c_hi = sk_worker_of(a, tg + a.n_kb - 1);
+        float* my = slot_ptr(cid);
+        const uint64_t keep = policy_evict_last();
+        for (int c = 0; c < nchunk; ++c) {
+          if (w.m0 + c * 32 >= a.M) break;  // uniform across the CTA
+          float v[32];
+          tmem_ld32(tb + c * 32, v);
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) st_keep(my + (size_t)(c * 32 + jj) * kTileN + row, v[jj], keep);
+        }
+        __threadfence();  // this share is visible before the piece is counted
+        epi_bar_sync();
+        if (et == 0) {
+          unsigned* cnt = a.out.sk_cnt + (size_t)w.tile * 2 + rank;
+          const bool last = atomicAdd(cnt, 1u) == (unsigned)(c_hi - c_lo);
+          if (last) *cnt = 0;  // ready for the next launch
+          *sk_flag = last ? 1u : 0u;
+        }
+        epi_bar_sync();
+        if (*sk_flag == 0u) {
+          release();
+          continue;
+        }
+        __threadfence();  // every counted share is visible to the reads below
+        fix = true;
+      }
+      // the whole tile's value of chunk c: this piece's accumulator, or (fixup)
+      // the shares of every piece in worker order
+      auto load_chunk = [&](int c, float (&v)[32]) {
+        tmem_ld32(tb + c * 32, v);
+        if (!fix) return;
+        float acc[32];
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) acc[jj] = 0.f;
+        for (int cw = c_lo; cw <= c_hi; ++cw) {
+          if (cw == cid) {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) acc[jj] += v[jj];
+          } else {
+            const float* o = slot_ptr(cw) + (size_t)(c * 32) * kTileN + row;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) acc[jj] += __ldcg(o + (size_t)jj * kTileN);
+          }
+        }
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) v[jj] = acc[jj];
+      };
+      // token -> (request, cache position) for OP_KV, and the block position's
+      // RoPE position for OP_QKV; one thread per token of the chunk
       auto token_maps = [&](int m_base) {
-        if (a.out.op != OP_KV || et >= 32) return;
+        if (et >= 32) return;
+        if (a.out.op == OP_QKV) {
+          const int m = m_base + et;
+          int pos = 0;
+          if (m < a.M) {
+            const int r = m / a.out.B;
+            pos = (a.out.req_valid[r] ? a.out.ctx_len[r] : 0) + m % a.out.B;
+          }
+          tok_pos[et] = pos;
+          return;
+        }
+        if (a.out.op != OP_KV) return;
         const int m = m_base + et;
         int req = -1, pos = 0;
         long long base = 0;
@@ -488,16 +658,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         release();
       } else if (EPI == EPI_PARTIAL && a.splits == 1) {
-        // the whole K range is in TMEM: apply the op chunk by chunk
+        // the whole K range is in TMEM (or in the pieces' shares): apply the op
+        // chunk by chunk
         for (int c = 0; c < nchunk; ++c) {
           if (w.m0 + c * 32 >= a.M) break;
           float v[32];
-          tmem_ld32(tb + c * 32, v);
+          load_chunk(c, v);
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) st[jj * kStLd + row] = v[jj];
           token_maps(w.m0 + c * 32);
           epi_bar_sync();
-          apply_op(a.out, a.M, a.N, st, tok_req, tok_pos, tok_base, w.m0 + c * 32, w.n0, et);
+          apply_op(a.out, a.M, a.N, st, tok_req, tok_pos, tok_base, w.m0 + c * 32, w.n0, et,
+                   a.err);
           epi_bar_sync();
         }
         release();
@@ -505,7 +677,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         float* tr = lm_tr + q * kLmTr;
         for (int c = 0; c < nchunk; ++c) {
           float v[32];
-          tmem_ld32(tb + c * 32, v);
+          if (fix && w.m0 + c * 32 >= a.M) {  // no shares stored past the last token
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) v[jj] = 0.f;
+          } else {
+            load_chunk(c, v);
+          }
           if (a.out.dbg != nullptr && n < a.N) {
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
@@ -743,9 +920,15 @@ void tile_weights(const void* src, void* dst, int N, int K, cudaStream_t s) {
                                              static_cast<uint4*>(dst), N, K);
 }
 
+
 static int token_tile(int M) {
   if (M >= kMaxBN) return kMaxBN;
   return (M + 31) / 32 * 32;
+}
+
+size_t gemm_sk_slot_bytes(int M) {
+  // two shares per worker (its first and last pieces), 128 weight rows x the token tile each
+  return (size_t)2 * num_sms() * kTileN * token_tile(std::max(M, 1)) * sizeof(float);
 }
 
 int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, int ld_seg, int M,
@@ -753,6 +936,7 @@ int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, i
   if (M <= 0) return DFLASH_OK;
   if (n_seg < 1 || n_seg > kMaxSeg || seg_k % kTileK != 0 || W.K != n_seg * seg_k)
     return DFLASH_EINVAL;
+  const bool sk = splits == 0;
   const int BN = token_tile(M);
   const bool pair = W.tiled != nullptr && gemm_use_pair(M, W.N);
   const int bn_cta = pair ? BN / 2 : BN;
@@ -768,7 +952,7 @@ int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, i
   a.BN = BN;
   const int stage_bytes = kTileN * 128 + bn_cta * 128;
   a.n_kb = W.K / kTileK;
-  if (epi == EPI_LMHEAD) splits = 1;
+  if (epi == EPI_LMHEAD || sk) splits = 1;
   splits = gemm_effective_splits(W.K, splits);
   a.kb_per_split = (a.n_kb + splits - 1) / splits;
   a.tile_rows = pair ? 2 * kTileN : kTileN;
@@ -776,6 +960,17 @@ int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, i
   a.tiles_m = (M + BN - 1) / BN;
   a.units = a.tiles_n * a.tiles_m * splits;
   a.splits = splits;
+  a.sk = 0;
+  a.sk_P = 1;
+  a.sk_W = 1;
+  if (sk) {
+    const long long tiles = (long long)a.tiles_n * a.tiles_m;
+    if (!out.sk_slots || !out.sk_cnt || tiles * 2 > out.sk_cnt_cap) return DFLASH_EINVAL;
+    a.sk = 1;
+    a.sk_W = tiles * a.n_kb;
+    const int workers = pair ? num_sms() / 2 : num_sms();
+    a.sk_P = (int)std::min<long long>(workers, a.sk_W);
+  }
   // fused ops need the whole K range in one unit
   if (epi == EPI_PARTIAL && out.op != OP_PARTIAL && splits > 1) return DFLASH_EINVAL;
   a.n_vtiles = (W.N + kTileN - 1) / kTileN;
@@ -794,7 +989,7 @@ int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, i
   const int sms = num_sms();
   TimedScope ts(s, epi == EPI_LMHEAD ? TC_LMHEAD : TC_GEMM);
   if (!pair) {
-    const int grid = std::min(a.units, sms);
+    const int grid = sk ? a.sk_P : std::min(a.units, sms);
     auto k = epi == EPI_PARTIAL ? gemm_tc_kernel<EPI_PARTIAL, false>
                                 : gemm_tc_kernel<EPI_LMHEAD, false>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -805,8 +1000,8 @@ int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, i
   auto k =
       epi == EPI_PARTIAL ? gemm_tc_kernel<EPI_PARTIAL, true> : gemm_tc_kernel<EPI_LMHEAD, true>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  const cudaError_t e = launch_pdl(k, dim3(2 * std::min(a.units, sms / 2)), dim3(kGemmThreads),
-                                   smem, s, 2, W.tmap, maps, a);
+  const cudaError_t e = launch_pdl(k, dim3(2 * (sk ? a.sk_P : std::min(a.units, sms / 2))),
+                                   dim3(kGemmThreads), smem, s, 2, W.tmap, maps, a);
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 

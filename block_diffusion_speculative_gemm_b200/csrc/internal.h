@@ -131,6 +131,11 @@ struct GemmOut {
   const int32_t* cu_rows = nullptr;    // OP_KV
   const int32_t* start_pos = nullptr;  // OP_KV
   KvPages pages;                       // OP_KV: the K/V store (contiguous when no table)
+  // stream-K schedule (gemm_tc with splits == 0): fixup shares and per-tile
+  // counters (2 per tile, zero before and after the call)
+  float* sk_slots = nullptr;           // gemm_sk_slot_bytes(M) bytes
+  unsigned* sk_cnt = nullptr;
+  int sk_cnt_cap = 0;                  // counters available
   int64_t kv_ls = 0, kv_hs = 0;        // OP_KV: rows between layers / between heads
   int B = 0, nq = 0, nkv = 0, hd = 0, I = 0;
   int row0 = 0, batch = 0, cap = 0, max_pos = 0;
@@ -178,12 +183,18 @@ bool encode_2d(CUtensorMap* m, const void* ptr, int64_t rows, int cols, int ld, 
 
 // Y = X * W^T for X [M, K] of W's element type (given as n_seg K-segments of
 // seg_k columns, each [M, seg_k] with row stride ld_seg elements) and W [N, K].
+// splits >= 1: fixed K splits (OP_PARTIAL writes each split's share; a fused
+// op needs splits == 1).  splits == 0: stream-K, every worker the same number
+// of k-blocks, tiles split between workers finished in the kernel (any op,
+// and the LM-head epilogue), with out.sk_slots / out.sk_cnt as scratch.
 int gemm_tc(const WeightMap& W, const void* const* xseg, int n_seg, int seg_k, int ld_seg, int M,
             int splits, int epi, const GemmOut& out, int32_t* err, cudaStream_t s);
 
 // Number of K splits for an M x N x K weight-streaming GEMM; always a count
 // that gemm_tc uses unchanged (see gemm_effective_splits).
 int gemm_pick_splits(int M, int N, int K, int max_splits);
+// Fixup scratch of a stream-K GEMM of M token rows (an upper bound for any N, K).
+size_t gemm_sk_slot_bytes(int M);
 // The split count gemm_tc actually runs for a requested count: every split
 // gets ceil(k-blocks / splits) k-blocks, the last one possibly fewer.
 int gemm_effective_splits(int K, int splits);
@@ -193,21 +204,24 @@ void gemm_simt_f32(const float* W, int N, int K, const float* const* xseg, int n
                    int M, float* out, cudaStream_t s);
 
 // ---------------------------------------------------------------- row kernels
+// The row kernels that store fp16 set DFLASH_DEV_RANGE in err when a value
+// overflows fp16 (see narrow_bad).
 template <typename TE, typename T>
 void launch_embed_norm(const int32_t* tokens, const TE* emb, const float* g, float* x, T* h, int M,
-                       int d, float eps, cudaStream_t s);
+                       int d, float eps, int32_t* err, cudaStream_t s);
 template <typename T>
 void launch_residual_norm(const float* part, int splits, int M, int d, float* x, const float* g,
-                          T* h, const int32_t* out_row, float eps, cudaStream_t s);
+                          T* h, const int32_t* out_row, float eps, int32_t* err, cudaStream_t s);
 template <typename T>
 void launch_ctx_norm(const float* part, int splits, int n, int d, const float* g, T* c, float eps,
-                     cudaStream_t s);
+                     int32_t* err, cudaStream_t s);
 template <typename T>
 void launch_qkv_post(const float* part, int splits, int M, int B, const int32_t* ctx_len,
                      const int32_t* req_valid, int nq, int nkv, int hd, const float* cos_t,
-                     const float* sin_t, T* q, T* kb, T* vb, cudaStream_t s);
+                     const float* sin_t, T* q, T* kb, T* vb, int32_t* err, cudaStream_t s);
 template <typename T>
-void launch_swiglu(const float* part, int splits, int M, int I, T* act, cudaStream_t s);
+void launch_swiglu(const float* part, int splits, int M, int I, T* act, int32_t* err,
+                   cudaStream_t s);
 // cap: positions per request (max_pages * page when paged).
 template <typename T>
 void launch_kv_scatter(const float* part, int splits, int n_rows, int row0, int L, int nkv, int hd,
@@ -280,7 +294,7 @@ int launch_sampled_draw(const void* q, int q_bf16, const int32_t* lm_rows,
                         int chunks, unsigned* cnt, cudaStream_t s);
 void launch_commit(const int32_t* tok, const float* conf, int batch, int B, int rem, int k,
                    int step, int32_t* tokens, int32_t* zrow, int32_t* lm_rows, int32_t* cstep,
-                   cudaStream_t s);
+                   int32_t* err, cudaStream_t s);
 void launch_draft_finish(const int32_t* tokens, const int32_t* cstep, const int32_t* req_valid,
                          int batch, int B, int32_t* draft_out, int32_t* cstep_out,
                          cudaStream_t s);

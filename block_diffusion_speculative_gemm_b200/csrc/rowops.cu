@@ -46,24 +46,30 @@ __device__ __forceinline__ float4 sum_splits4(const float* part, int splits, siz
   return v;
 }
 
+// Stores four values; returns true when a value does not fit the element type
+// (an fp16 store of a value that rounds past the largest finite fp16, or NaN).
 template <typename T>
-__device__ __forceinline__ void store4(T* dst, float a, float b, float c, float d) {
+__device__ __forceinline__ bool store4(T* dst, float a, float b, float c, float d) {
   dst[0] = from_f<T>(a);
   dst[1] = from_f<T>(b);
   dst[2] = from_f<T>(c);
   dst[3] = from_f<T>(d);
+  return narrow_bad<T>(a) || narrow_bad<T>(b) || narrow_bad<T>(c) || narrow_bad<T>(d);
 }
 template <>
-__device__ __forceinline__ void store4<__half>(__half* dst, float a, float b, float c, float d) {
+__device__ __forceinline__ bool store4<__half>(__half* dst, float a, float b, float c, float d) {
   __half2 lo = __floats2half2_rn(a, b), hi = __floats2half2_rn(c, d);
   uint2 u;
   u.x = *reinterpret_cast<uint32_t*>(&lo);
   u.y = *reinterpret_cast<uint32_t*>(&hi);
   *reinterpret_cast<uint2*>(dst) = u;
+  return narrow_bad<__half>(a) || narrow_bad<__half>(b) || narrow_bad<__half>(c) ||
+         narrow_bad<__half>(d);
 }
 template <>
-__device__ __forceinline__ void store4<float>(float* dst, float a, float b, float c, float d) {
+__device__ __forceinline__ bool store4<float>(float* dst, float a, float b, float c, float d) {
   *reinterpret_cast<float4*>(dst) = make_float4(a, b, c, d);
+  return false;
 }
 
 // ---------------------------------------------------------------- embedding + RMSNorm
@@ -72,7 +78,7 @@ template <typename TE, typename T>
 __global__ void __launch_bounds__(kRowThreads)
     embed_norm_kernel(const int32_t* __restrict__ tokens, const TE* __restrict__ emb,
                       const float* __restrict__ g, float* __restrict__ x, T* __restrict__ h, int d,
-                      float eps) {
+                      float eps, int32_t* err) {
   pdl_trigger();
   pdl_wait();
   __shared__ float red[32];
@@ -88,23 +94,27 @@ __global__ void __launch_bounds__(kRowThreads)
     ss += v[i] * v[i];
   }
   const float inv = rsqrtf(block_sum(ss, red) / d + eps);
+  bool bad = false;
 #pragma unroll
   for (int i = 0; i < kMaxRowElems; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
     if (c < d) {
       x[(size_t)m * d + c] = v[i];
-      h[(size_t)m * d + c] = from_f<T>(v[i] * inv * g[c]);
+      const float y = v[i] * inv * g[c];
+      h[(size_t)m * d + c] = from_f<T>(y);
+      bad |= narrow_bad<T>(y);
     }
   }
+  if (bad) set_error(err, DFLASH_DEV_RANGE);
 }
 
 template <typename TE, typename T>
 void launch_embed_norm(const int32_t* tokens, const TE* emb, const float* g, float* x, T* h, int M,
-                       int d, float eps, cudaStream_t s) {
+                       int d, float eps, int32_t* err, cudaStream_t s) {
   if (M <= 0) return;
   TimedScope ts(s, TC_ROW);
   launch_pdl(embed_norm_kernel<TE, T>, dim3(M), dim3(kRowThreads), 0, s, 1, tokens, emb, g, x, h, d,
-      eps);
+      eps, err);
 }
 
 // ---------------------------------------------------------------- residual + RMSNorm
@@ -115,7 +125,7 @@ template <typename T>
 __global__ void __launch_bounds__(kRowThreads)
     residual_norm_kernel(const float* __restrict__ part, int splits, int M, int d,
                          float* __restrict__ x, const float* __restrict__ g, T* __restrict__ h,
-                         const int32_t* __restrict__ out_row, float eps) {
+                         const int32_t* __restrict__ out_row, float eps, int32_t* err) {
   pdl_trigger();
   pdl_wait();
   __shared__ float red[32];
@@ -146,24 +156,26 @@ __global__ void __launch_bounds__(kRowThreads)
   const float inv = rsqrtf(block_sum(ss, red) / d + eps);
   const int orow = out_row ? out_row[m] : m;
   if (orow < 0) return;
+  bool bad = false;
 #pragma unroll
   for (int i = 0; i < kV; ++i) {
     const int c = (threadIdx.x + i * kRowThreads) * 4;
     if (c < d) {
       const float4 gg = *reinterpret_cast<const float4*>(g + c);
-      store4<T>(h + (size_t)orow * d + c, v[i].x * inv * gg.x, v[i].y * inv * gg.y,
-                v[i].z * inv * gg.z, v[i].w * inv * gg.w);
+      bad |= store4<T>(h + (size_t)orow * d + c, v[i].x * inv * gg.x, v[i].y * inv * gg.y,
+                       v[i].z * inv * gg.z, v[i].w * inv * gg.w);
     }
   }
+  if (bad) set_error(err, DFLASH_DEV_RANGE);
 }
 
 template <typename T>
 void launch_residual_norm(const float* part, int splits, int M, int d, float* x, const float* g,
-                          T* h, const int32_t* out_row, float eps, cudaStream_t s) {
+                          T* h, const int32_t* out_row, float eps, int32_t* err, cudaStream_t s) {
   if (M <= 0) return;
   TimedScope ts(s, TC_ROW);
   launch_pdl(residual_norm_kernel<T>, dim3(M), dim3(kRowThreads), 0, s, 1, part, splits, M, d, x, g,
-      h, out_row, eps);
+      h, out_row, eps, err);
 }
 
 // ---------------------------------------------------------------- context-feature RMSNorm
@@ -171,7 +183,7 @@ void launch_residual_norm(const float* part, int splits, int M, int d, float* x,
 template <typename T>
 __global__ void __launch_bounds__(kRowThreads)
     ctx_norm_kernel(const float* __restrict__ part, int splits, int n_rows, int d,
-                    const float* __restrict__ g, T* __restrict__ c, float eps) {
+                    const float* __restrict__ g, T* __restrict__ c, float eps, int32_t* err) {
   pdl_trigger();
   pdl_wait();
   __shared__ float red[32];
@@ -188,23 +200,26 @@ __global__ void __launch_bounds__(kRowThreads)
     ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
   }
   const float inv = rsqrtf(block_sum(ss, red) / d + eps);
+  bool bad = false;
 #pragma unroll
   for (int i = 0; i < kV; ++i) {
     const int col = (threadIdx.x + i * kRowThreads) * 4;
     if (col < d) {
       const float4 gg = *reinterpret_cast<const float4*>(g + col);
-      store4<T>(c + (size_t)n * d + col, v[i].x * inv * gg.x, v[i].y * inv * gg.y,
-                v[i].z * inv * gg.z, v[i].w * inv * gg.w);
+      bad |= store4<T>(c + (size_t)n * d + col, v[i].x * inv * gg.x, v[i].y * inv * gg.y,
+                       v[i].z * inv * gg.z, v[i].w * inv * gg.w);
     }
   }
+  if (bad) set_error(err, DFLASH_DEV_RANGE);
 }
 
 template <typename T>
 void launch_ctx_norm(const float* part, int splits, int n, int d, const float* g, T* c, float eps,
-                     cudaStream_t s) {
+                     int32_t* err, cudaStream_t s) {
   if (n <= 0) return;
   TimedScope ts(s, TC_ROW);
-  launch_pdl(ctx_norm_kernel<T>, dim3(n), dim3(kRowThreads), 0, s, 1, part, splits, n, d, g, c, eps);
+  launch_pdl(ctx_norm_kernel<T>, dim3(n), dim3(kRowThreads), 0, s, 1, part, splits, n, d, g, c, eps,
+             err);
 }
 
 // ---------------------------------------------------------------- QKV epilogue
@@ -216,6 +231,7 @@ __global__ void qkv_post_kernel(const float* __restrict__ part, int splits, int 
                                 const int32_t* __restrict__ ctx_len,
                                 const int32_t* __restrict__ req_valid, int nq, int nkv, int hd,
                                 const float* __restrict__ cos_t, const float* __restrict__ sin_t,
+                                int32_t* err,
                                 T* __restrict__ q, T* __restrict__ kb, T* __restrict__ vb) {
   pdl_trigger();
   pdl_wait();
@@ -246,20 +262,21 @@ __global__ void qkv_post_kernel(const float* __restrict__ part, int splits, int 
   } else {
     dst = vb + ((size_t)m * nkv + head - nq - nkv) * hd;
   }
-  store4<T>(dst + i, x1.x, x1.y, x1.z, x1.w);
-  store4<T>(dst + i + half, x2.x, x2.y, x2.z, x2.w);
+  const bool bad = store4<T>(dst + i, x1.x, x1.y, x1.z, x1.w) |
+                   store4<T>(dst + i + half, x2.x, x2.y, x2.z, x2.w);
+  if (bad) set_error(err, DFLASH_DEV_RANGE);
 }
 
 template <typename T>
 void launch_qkv_post(const float* part, int splits, int M, int B, const int32_t* ctx_len,
                      const int32_t* req_valid, int nq, int nkv, int hd, const float* cos_t,
-                     const float* sin_t, T* q, T* kb, T* vb, cudaStream_t s) {
+                     const float* sin_t, T* q, T* kb, T* vb, int32_t* err, cudaStream_t s) {
   if (M <= 0) return;
   const int pairs = (nq + 2 * nkv) * hd / 2;
   dim3 grid((pairs / 4 + 255) / 256, M);
   TimedScope ts(s, TC_ROW);
   launch_pdl(qkv_post_kernel<T>, dim3(grid), dim3(256), 0, s, 1, part, splits, M, B, ctx_len,
-      req_valid, nq, nkv, hd, cos_t, sin_t, q, kb, vb);
+      req_valid, nq, nkv, hd, cos_t, sin_t, err, q, kb, vb);
 }
 
 // ---------------------------------------------------------------- SwiGLU
@@ -267,7 +284,7 @@ void launch_qkv_post(const float* part, int splits, int M, int B, const int32_t*
 // of the same features; act = silu(gate) * up.
 template <typename T>
 __global__ void swiglu_kernel(const float* __restrict__ part, int splits, int M, int I,
-                              T* __restrict__ act) {
+                              T* __restrict__ act, int32_t* err) {
   pdl_trigger();
   pdl_wait();
   const int m = blockIdx.y;
@@ -277,17 +294,19 @@ __global__ void swiglu_kernel(const float* __restrict__ part, int splits, int M,
   const size_t gc = (size_t)m * 2 * I + (size_t)(i >> 6) * 128 + (i & 63);
   const float4 g = sum_splits4(part, splits, stride, gc);
   const float4 u = sum_splits4(part, splits, stride, gc + 64);
-  store4<T>(act + (size_t)m * I + i, g.x / (1.f + expf(-g.x)) * u.x,
+  const bool bad = store4<T>(act + (size_t)m * I + i, g.x / (1.f + expf(-g.x)) * u.x,
             g.y / (1.f + expf(-g.y)) * u.y, g.z / (1.f + expf(-g.z)) * u.z,
             g.w / (1.f + expf(-g.w)) * u.w);
+  if (bad) set_error(err, DFLASH_DEV_RANGE);
 }
 
 template <typename T>
-void launch_swiglu(const float* part, int splits, int M, int I, T* act, cudaStream_t s) {
+void launch_swiglu(const float* part, int splits, int M, int I, T* act, int32_t* err,
+                   cudaStream_t s) {
   if (M <= 0) return;
   dim3 grid((I / 4 + 255) / 256, M);
   TimedScope ts(s, TC_ROW);
-  launch_pdl(swiglu_kernel<T>, dim3(grid), dim3(256), 0, s, 1, part, splits, M, I, act);
+  launch_pdl(swiglu_kernel<T>, dim3(grid), dim3(256), 0, s, 1, part, splits, M, I, act, err);
 }
 
 // ---------------------------------------------------------------- K/V cache scatter
@@ -346,9 +365,14 @@ __global__ void kv_scatter_kernel(const float* __restrict__ part, int splits, in
     x1 = y1;
     x2 = y2;
   }
-  T* dst = (is_v ? vc : kc) + (size_t)kv_row(pg, l, batch, r, nkv, head, cap, pos) * hd;
-  store4<T>(dst + i, x1.x, x1.y, x1.z, x1.w);
-  store4<T>(dst + i + half, x2.x, x2.y, x2.z, x2.w);
+  const long long drow = kv_row(pg, l, batch, r, nkv, head, cap, pos);
+  const long long rows = (long long)L * nkv * (pg.table ? (long long)pg.n_pages * pg.page
+                                                        : (long long)batch * cap);
+  if (!DFLASH_CHECK(drow >= 0 && drow < rows, err)) return;
+  T* dst = (is_v ? vc : kc) + (size_t)drow * hd;
+  const bool bad = store4<T>(dst + i, x1.x, x1.y, x1.z, x1.w) |
+                   store4<T>(dst + i + half, x2.x, x2.y, x2.z, x2.w);
+  if (bad) set_error(err, DFLASH_DEV_RANGE);
 }
 
 template <typename T>
@@ -406,13 +430,13 @@ void launch_inject_page_check(const int32_t* cu_rows, const int32_t* start_pos, 
 // T: activation type (GEMM operand); TC: K/V cache type; TE: embedding type.
 #define DFLASH_INST_A(T)                                                                         \
   template void launch_residual_norm<T>(const float*, int, int, int, float*, const float*, T*,   \
-                                        const int32_t*, float, cudaStream_t);                    \
+                                        const int32_t*, float, int32_t*, cudaStream_t);          \
   template void launch_ctx_norm<T>(const float*, int, int, int, const float*, T*, float,         \
-                                   cudaStream_t);                                                \
+                                   int32_t*, cudaStream_t);                                      \
   template void launch_qkv_post<T>(const float*, int, int, int, const int32_t*, const int32_t*,  \
                                    int, int, int, const float*, const float*, T*, T*, T*,        \
-                                   cudaStream_t);                                                \
-  template void launch_swiglu<T>(const float*, int, int, int, T*, cudaStream_t);
+                                   int32_t*, cudaStream_t);                                      \
+  template void launch_swiglu<T>(const float*, int, int, int, T*, int32_t*, cudaStream_t);
 #define DFLASH_INST_C(TC)                                                                        \
   template void launch_kv_scatter<TC>(const float*, int, int, int, int, int, int,                \
                                       const int32_t*, const int32_t*, int, int, const KvPages&,  \
@@ -424,9 +448,9 @@ DFLASH_INST_A(__half)
 DFLASH_INST_C(float)
 DFLASH_INST_C(__half)
 template void launch_embed_norm<float, float>(const int32_t*, const float*, const float*, float*,
-                                              float*, int, int, float, cudaStream_t);
+                                              float*, int, int, float, int32_t*, cudaStream_t);
 template void launch_embed_norm<__nv_bfloat16, __half>(const int32_t*, const __nv_bfloat16*,
                                                        const float*, float*, __half*, int, int,
-                                                       float, cudaStream_t);
+                                                       float, int32_t*, cudaStream_t);
 
 }  // namespace dflash

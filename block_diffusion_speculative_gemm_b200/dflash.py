@@ -21,7 +21,8 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "dflash.h")
 HEADERS = [HEADER, os.path.join(os.path.dirname(_HERE), "include", "dflash_debug.h")]
 
 OK, EINVAL, EUNSUPPORTED, ECUDA, ENOMEM, EWORKSPACE, ESCRATCH = 0, -1, -2, -3, -4, -5, -6
-DEV_CTX_CAP, DEV_OUT_CAP, DEV_TOKEN_RANGE, DEV_TIMEOUT, DEV_ROWS, DEV_PAGE = 1, 2, 4, 8, 16, 32
+DEV_CTX_CAP, DEV_OUT_CAP, DEV_TOKEN_RANGE, DEV_TIMEOUT, DEV_ROWS, DEV_PAGE, DEV_RANGE = (
+    1, 2, 4, 8, 16, 32, 64)
 F32, BF16, F16 = 0, 1, 2
 TIMING_CLASSES = ("gemm", "attention", "row", "verify", "lm_head")
 
@@ -118,6 +119,10 @@ def lib() -> ctypes.CDLL:
         L.dflash_debug_tile_weights.argtypes = [vp, vp, i32, i32, vp]
         L.dflash_debug_lmhead_tiled.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp, vp, vp]
         L.dflash_debug_gemm_mode.argtypes = [i32]
+        L.dflash_debug_gemm_schedule.argtypes = [i32]
+        L.dflash_debug_gemm_streamk_ws_bytes.argtypes = [i32]
+        L.dflash_debug_gemm_streamk_ws_bytes.restype = sz
+        L.dflash_debug_gemm_streamk.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp, sz, vp]
         L.dflash_debug_attn_chunk.argtypes = [i32]
         L.dflash_debug_pick_splits.argtypes = [i32, i32, i32]
         L.dflash_debug_wait_timeout.argtypes = [vp, vp]
@@ -676,6 +681,29 @@ def debug_attn_chunk(keys: int) -> None:
     """Process-wide split-KV chunk (keys, multiple of 64) of the draft attention;
     0 restores the library's rule (tests and tuning only)."""
     _check("dflash_debug_attn_chunk", lib().dflash_debug_attn_chunk(int(keys)))
+
+
+def debug_gemm_streamk(W: torch.Tensor, X: torch.Tensor, stream=None):
+    """(X @ W^T as float32 [M, N] through the stream-K schedule, the workspace's
+    error bits); W and X both bf16 or both fp16."""
+    _need(W, "W")
+    _need(X, "X", W.dtype)
+    N, K = W.shape
+    M = X.shape[0]
+    Wt = debug_tile_weights(W, stream)
+    out = torch.full((M, N), float("nan"), dtype=torch.float32, device=W.device)
+    ws = new_workspace(lib().dflash_debug_gemm_streamk_ws_bytes(M), W.device, stream)
+    _check("dflash_debug_gemm_streamk", lib().dflash_debug_gemm_streamk(
+        _ptr(Wt), N, K, _ptr(X), M, _ELEM[W.dtype], _ptr(out), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return out, get_error(ws, stream)
+
+
+def debug_gemm_schedule(sched: int) -> None:
+    """Process-wide schedule of the draft and injection GEMMs: 0 the library's
+    default (stream-K LM head, fixed-split projections), 1 fixed K splits
+    everywhere, 2 stream-K everywhere (tests and tuning)."""
+    _check("dflash_debug_gemm_schedule", lib().dflash_debug_gemm_schedule(int(sched)))
 
 
 def debug_gemm_mode(mode: int) -> None:

@@ -74,6 +74,8 @@ extern "C" {
 #define DFLASH_DEV_TIMEOUT     8  /* a bounded device wait expired */
 #define DFLASH_DEV_ROWS        16 /* cu_rows not monotone or not ending at n_rows */
 #define DFLASH_DEV_PAGE        32 /* a position's page-table entry is unmapped (paged K/V) */
+#define DFLASH_DEV_RANGE       64 /* an fp16 activation or cache entry overflowed (bf16 models) */
+#define DFLASH_DEV_CHECK      128 /* bounds-checked build only: an index failed its check */
 
 /* ---- element types ---------------------------------------------------- */
 #define DFLASH_F32  0

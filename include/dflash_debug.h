@@ -55,6 +55,29 @@ int dflash_debug_lmhead_tiled(const void* W_tiled, int N, int K, const void* X, 
  * DFLASH_EINVAL for any other value.  Not thread-safe; tests only. */
 int dflash_debug_gemm_mode(int mode);
 
+/* Y = X W^T through the stream-K schedule of the tcgen05 GEMM, stored as fp32
+ * out [M, N] (the fused-store epilogue after the in-kernel fixup of split
+ * tiles).  Wt is the pre-tiled image (dflash_debug_tile_weights), X [M, K] of
+ * the same 16-bit type; ws a zero-filled, 256-byte aligned workspace of at least
+ * dflash_debug_gemm_streamk_ws_bytes(M) bytes (its header holds the error word
+ * and the tile counters).  The launch mode (single CTAs or CTA pairs) follows
+ * dflash_debug_gemm_mode. */
+size_t dflash_debug_gemm_streamk_ws_bytes(int M);
+int dflash_debug_gemm_streamk(const void* Wt, int N, int K, const void* X, int M, int elem,
+                              float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Schedule of the draft and injection GEMMs for every later call,
+ * process-wide.  Stream-K: every CTA (or CTA pair) streams the same number of
+ * k-blocks; a tile split between workers is finished inside the GEMM by its
+ * last piece, which then applies the following elementwise step in its
+ * epilogue.  Fixed splits: K split a fixed number of ways, the partials summed
+ * by separate reduction kernels.  0 (default): stream-K for the LM head,
+ * fixed splits for the projections and the injection; 1: fixed splits
+ * everywhere; 2: stream-K everywhere.  All compute the same products (up to
+ * fp32 summation order).  DFLASH_EINVAL for any other value.  Not
+ * thread-safe; tests and tuning only. */
+int dflash_debug_gemm_schedule(int sched);
+
 /* Failure-detection check: launches one thread that waits, with the
  * library's bounded pipeline wait, on an mbarrier phase nothing completes.
  * After the wait limit (1 s) the kernel sets DFLASH_DEV_TIMEOUT in the error

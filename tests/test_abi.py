@@ -141,3 +141,11 @@ def test_sampled_and_paged_calls_reject_null_model_and_bad_arguments():
                                     None) == D.EINVAL
     assert L.dflash_draft_block_paged(None, p, p, p, p, 8, 64, p, 4, 1, 8, 2, p, None, None, p,
                                       1 << 20, None) == D.EINVAL
+
+
+def test_bounds_checked_build_exports_the_same_symbols():
+    from block_diffusion_speculative_gemm_b200 import build as Bld
+
+    lib = ctypes.CDLL(Bld.build(checked=True))
+    for n in D.header_symbols():
+        assert hasattr(lib, n), n

@@ -13,7 +13,7 @@ import torch
 import oracle as O
 import synth
 from synth.configs import shrink
-from tests.gpu_common import DraftReport, built, check_draft_request, oracle_caches_from
+from tests.gpu_common import DraftReport, built, check_draft_request, oracle_caches_from, record
 from block_diffusion_speculative_gemm_b200 import dflash as D
 
 pytestmark = pytest.mark.gpu
@@ -145,3 +145,33 @@ def test_draft_full_size_sampled_requests(name, requests):
     assert (out[:, 1:] >= 0).all() and (out[:, 1:] < cfg.V).all()
     assert (res["cst"][:, 1:] >= 0).all() and (res["cst"][:, 1:] < cfg.steps).all()
     print(name, _check(b, cfg, res, cfg.steps, requests, test=f"draft_full_size[{name}]"))
+
+
+def test_draft_gemm_schedules_agree():
+    """The GEMM schedules (the default: stream-K LM head and fixed-split
+    projections; fixed splits everywhere; stream-K everywhere, every split tile
+    finished inside the GEMM with the fused epilogues) compute the same products
+    up to fp32 summation order: every draft passes the oracle's rules, and their
+    logits agree far inside the tolerance."""
+    base = synth.get_config("qwen3_8b_bs32")
+    cfg = shrink(base, L=2, V=4096, batch=5, ctx=("uniform", 30, 700), I=1024, d=1024,
+                 H_t=512).replace(name="small8b_B8")
+    b = built(cfg)
+    runs = []
+    try:
+        for sched in (0, 1, 2):
+            D.debug_gemm_schedule(sched)
+            runs.append(_run_draft(b, cfg))
+    finally:
+        D.debug_gemm_schedule(0)
+    for res in runs:
+        assert res["err"] == 0
+        _check(b, cfg, res, cfg.steps, range(cfg.batch))
+    la = runs[0]["lg"]
+    for other in runs[1:]:
+        lb = other["lg"]
+        both = ~(torch.isnan(la) | torch.isnan(lb))
+        scale = la[both].abs().max().item()
+        diff = (la[both] - lb[both]).abs().max().item()
+        record("draft_gemm_schedules", max_rel_diff=diff / scale)
+        assert diff <= 2e-3 * scale

@@ -85,3 +85,33 @@ def test_lmhead_epilogue_stats(N, K, M, dtype, mode):
         assert torch.equal(idx[:, t], first.long())
         se = torch.exp(blk - mx[:, None]).sum(1)
         assert torch.allclose(st[:, t, 2], se, rtol=1e-5)
+
+
+@pytest.mark.parametrize("N,K,M", [
+    (128, 64, 16),          # one tile, one k-block: fewer iterations than workers
+    (6144, 4096, 256),      # QKV projection: ~20 k-blocks per worker, tiles split 3-4 ways
+    (4096, 4096, 256),      # output projection
+    (24576, 4096, 256),     # SwiGLU gate/up
+    (4096, 12288, 256),     # down projection
+    (1000, 512, 133),       # ragged weight and token rows
+    (4096, 20480, 154),     # injection fc over five taps
+    (640, 320, 1100),       # several token tiles, the last ragged
+    (130, 128, 48),         # the last weight tile has 2 live rows
+    (151936 // 8, 512, 224),  # an LM-head-like width
+])
+@pytest.mark.parametrize("mode", ["single", "pair"])
+def test_stream_k_gemm_matches_float64(N, K, M, mode):
+    """Stream-K: every worker streams the same number of k-blocks; split tiles
+    are finished inside the kernel by their last piece, summing the pieces in
+    worker order.  The product must be the fp64 product, and two runs must be
+    bit-identical (the sum order does not depend on which piece arrives last)."""
+    D.debug_gemm_mode(MODES[mode][1])
+    W, X = _inputs(N, K, M, N + 3 * K + M, torch.float16)
+    Wd, Xd = W.cuda(), X.cuda()
+    out, err = D.debug_gemm_streamk(Wd, Xd)
+    again, err2 = D.debug_gemm_streamk(Wd, Xd)
+    assert err == 0 and err2 == 0
+    ref = X.double() @ W.double().T
+    scale = ref.abs().max().item()
+    assert (out.double().cpu() - ref).abs().max().item() <= 2e-5 * scale + 1e-6
+    assert torch.equal(out, again)
