@@ -255,6 +255,12 @@ int g_attn_chunk = 0;  // split-KV chunk override in keys (tests and tuning; 0 =
 // whose few tiles split 3-5 ways).
 int g_gemm_sched = 0;
 bool sk_projections() { return g_gemm_sched == 2; }
+// Draft attention schedule: 0 (default) the split-KV grid of fixed key chunks;
+// 1 persistent (every CTA the same number of key tiles, one TMA ring across
+// (request, head) segments), which measured 15% slower at the 8B batch of 32
+// (0.92-0.95 against 0.79-0.80 ms per draft): the SMs' idle time is not what
+// bounds this kernel, its latency-bound mma.sync chains at ~9 warps per SM are.
+int g_attn_sched = 0;
 bool sk_lm_head() { return g_gemm_sched != 1; }
 constexpr int kAttnRows = 64;
 constexpr int kInjectChunkRows = 16384;
@@ -264,7 +270,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct DraftLayout {
   size_t tokens, zrow, lm_rows, cstep, req_valid, lm_tok, lm_conf, x, h, q, kb, vb, o, act, part,
-      sk, attn_o, attn_ml, stats, draw, logits, end;
+      sk, attn_o, attn_ml, seg, stats, draw, logits, end;
   size_t part_elems;  // fp32 elements of split-K partials
 };
 
@@ -307,9 +313,13 @@ DraftLayout draft_layout(const dflash_config& c, int batch, int B) {
   L.part_elems = 4 * M * (size_t)draft_part_cols(c);
   L.part = take(4 * L.part_elems);
   L.sk = take(gemm_sk_slot_bytes((int)M));  // stream-K fixup shares
-  const size_t arows = (size_t)batch * c.n_kv * kMaxChunks * kAttnRows;
+  // attention partials: the split-KV grid's [batch][nkv][chunk][64 rows], or
+  // the persistent schedule's (2 * SMs + batch * nkv) slots of 64 rows
+  const size_t arows = std::max((size_t)batch * c.n_kv * kMaxChunks * kAttnRows,
+                                ((size_t)2 * num_sms() + (size_t)batch * c.n_kv) * kAttnRows);
   L.attn_o = take(4 * arows * c.head_dim);
   L.attn_ml = take(8 * arows);
+  L.seg = take(4 * ((size_t)batch * c.n_kv + 1));  // persistent schedule: segment prefix
   L.stats = take(sizeof(LmStat) * M * n_vt);
   // sampled drafting's draw partials: rows x chunks never exceeds M + 600 (the
   // chunk count falls as the row count grows)
@@ -849,6 +859,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
   // LM-head vocabulary tiles this model holds (all of them unless it is a shard)
   const int n_vt = (m->vocab_hi - m->vocab_lo + kTileN - 1) / kTileN;
   const bool bf16 = c.dtype == DFLASH_BF16;
+  int32_t* seg_start = bf16 && g_attn_sched == 1 ? at<int32_t>(ws, L.seg) : nullptr;
 
   // split-KV chunk: a multiple of the attention tile (64 keys) sized for
   // about four CTAs per SM over the whole (request, kv head, chunk) grid, at
@@ -887,6 +898,9 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
     const int k = (rem + (n_steps - t) - 1) / (n_steps - t);
     const int rows = batch * rem;
     if (!ph.forward) goto choose;
+    if (bf16 && g_attn_sched == 1 &&
+        (st = launch_attn_plan(ctx_len, valid, batch, nkv, seg_start, s)))
+      return st;
     launch_embed_norm<TE, T>(tokens, static_cast<const TE*>(m->emb), m->layers[0].g_in, x, h, M, c.d,
                          c.eps, err, s);
     for (int l = 0; l < c.n_layers; ++l) {
@@ -928,7 +942,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
                              m->rope_sin, q, kb, vb, err, s);
         if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, pg, l, c.n_layers, batch, cap,
                                                 ctx_len, valid, B, nq, nkv, hd, attn_o, attn_ml,
-                                                n_chunks, chunk, o, attn_cnt, err, s)))
+                                                n_chunks, chunk, seg_start, o, attn_cnt, err, s)))
           return st;
         go.f32 = x;
         if ((st = run(P.mo, c.d, nq * hd, o, OP_RESID))) return st;
@@ -948,7 +962,7 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
                          q, kb, vb, err, s);
       if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, pg, l, c.n_layers, batch, cap,
                                               ctx_len, valid, B, nq, nkv, hd, attn_o, attn_ml,
-                                              n_chunks, chunk, o, attn_cnt, err, s)))
+                                              n_chunks, chunk, nullptr, o, attn_cnt, err, s)))
         return st;
       if ((st = gemm(P.mo, P.Wo, c.d, nq * hd, o, part, L.part_elems, &sp))) return st;
       launch_residual_norm<T>(part, sp, M, c.d, x, P.g_post, h, nullptr, c.eps, err, s);
@@ -1434,6 +1448,12 @@ extern "C" int dflash_debug_attn_chunk(int keys) {
 extern "C" int dflash_debug_split_weight(float w) {
   if (!(w >= 0.f && w <= 64.f)) return DFLASH_EINVAL;
   gemm_set_split_weight(w);
+  return DFLASH_OK;
+}
+
+extern "C" int dflash_debug_attn_schedule(int sched) {
+  if (sched < 0 || sched > 1) return DFLASH_EINVAL;
+  g_attn_sched = sched;
   return DFLASH_OK;
 }
 

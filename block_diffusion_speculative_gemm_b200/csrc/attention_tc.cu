@@ -518,6 +518,383 @@ __global__ void __launch_bounds__(kThreads)
   if (tid == 0) cnt[r * nkv + g] = 0;  // ready for the next launch
 }
 
+// ---------------------------------------------------------------- persistent schedule
+// Segment s = r * nkv + g (request r, kv head g) holds units 0 .. n_s - 1: its
+// ceil(T_r / 64) context tiles, then one unit for the block's own keys.
+// seg_start[s] = units before segment s, seg_start[S] = W.  CTA c of the P
+// CTAs with work takes units [c W / P, (c + 1) W / P): every CTA streams the
+// same number of tiles through one TMA ring that runs on across segments, and
+// sets up once.  A piece (the units of one segment inside one CTA's range)
+// publishes one (m, l, O) partial per warp; the piece that counts itself last
+// on the segment's counter merges every piece's partials, CTAs in order, into
+// the output rows and sets the counter back to zero.
+
+// One CTA of 1024 threads: exclusive scan of the segments' unit counts.
+__global__ void __launch_bounds__(1024)
+    attn_plan_kernel(const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ req_valid,
+                     int batch, int nkv, int32_t* __restrict__ seg_start) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  const int S = batch * nkv;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < S; base += blockDim.x) {
+    const int s = base + threadIdx.x;
+    int n = 0;
+    if (s < S) {
+      const int r = s / nkv;
+      const int T = req_valid[r] ? ctx_len[r] : 0;
+      n = (T + kKeys - 1) / kKeys + 1;
+    }
+    int x = n;  // inclusive scan inside the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[w] = x;
+    __syncthreads();
+    if (w == 0) {
+      int t = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
+      }
+      warp_tot[lane] = t;  // inclusive over warps
+    }
+    __syncthreads();
+    const int excl = carry + (w > 0 ? warp_tot[w - 1] : 0) + x - n;
+    if (s < S) seg_start[s] = excl;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = excl + n;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) seg_start[S] = carry;
+}
+
+// named barrier 1 among the 128 threads of the compute warps
+__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int HD, int MT>
+__global__ void __launch_bounds__(kThreads, 2)
+    attn_tc_persistent(const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __half* __restrict__ q,
+                       const __half* __restrict__ kb, const __half* __restrict__ vb,
+                       const KvPages pg, long long kv_rows, int layer, int batch, int cap,
+                       const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ req_valid,
+                       int B, int nq, int nkv, const int32_t* __restrict__ seg_start,
+                       float* __restrict__ part_o, float* __restrict__ part_ml,
+                       unsigned* __restrict__ cnt, __half* __restrict__ out, int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
+  using LY = Layout<HD, MT>;
+  using WP = Warp<HD, MT>;
+  constexpr int kStages = LY::kStages;
+  constexpr int NT = WP::NT, KS = WP::KS, KG = WP::KG, KPW = WP::KPW;
+  constexpr int HALVES = HD / 64;
+  constexpr int kRows = MT * 16;           // rows of one warp partial
+  constexpr int kAcc = (kRows * HD / 4 + 127) / 128;  // float4 outputs per thread in a merge
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t s_q = s_base + kStages * LY::kStage;
+  float* scratch = reinterpret_cast<float*>(smem + kStages * LY::kStage);  // the query area
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * LY::kStage + LY::kQ);
+  auto full = [&](int st) { return smem_u32(bars + st); };
+  auto empty = [&](int st) { return smem_u32(bars + kStages + st); };
+  __shared__ int s_last;
+
+  const int S = batch * nkv;
+  const long long W = seg_start[S];
+  const int P = (int)min((long long)gridDim.x, W);
+  const int c = blockIdx.x;
+  if (c >= P) return;  // the whole CTA, before any barrier is initialised
+  const long long g0 = (long long)c * W / P, g1 = (long long)(c + 1) * W / P;
+  const int G = nq / nkv;
+  const int R = B * G;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int mt = warp % MT, kg = warp / MT;
+
+  if (tid == 0) {
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(full(st), 1);
+      mbar_init(empty(st), kComputeWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();  // the last block-wide barrier: the producer warp runs on alone
+
+  // segment of unit gq: the last s with seg_start[s] <= gq
+  auto seg_of = [&](long long gq) {
+    int lo = 0, hi = S - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (seg_start[mid] <= gq) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
+  auto ctx_of = [&](int r) { return req_valid[r] ? ctx_len[r] : 0; };
+
+  if (warp == kComputeWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      int it = 0;
+      for (long long gq = g0; gq < g1 && ok;) {
+        const int sg = seg_of(gq);
+        const long long st0 = seg_start[sg], en = seg_start[sg + 1];
+        const int a = (int)(gq - st0), b = (int)(min(en, g1) - st0);
+        const int r = sg / nkv, gh = sg % nkv;
+        const int nctx = (ctx_of(r) + kKeys - 1) / kKeys;
+        const int row_base = pg.table == nullptr ? ((layer * batch + r) * nkv + gh) * cap : 0;
+        for (int t = a; t < min(b, nctx); ++t, ++it) {
+          const int stg = it % kStages;
+          if (it >= kStages && !mbar_wait(empty(stg), ((it / kStages) + 1) & 1)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sK = s_base + stg * LY::kStage, sV = sK + LY::kTile;
+          mbar_arrive_expect_tx(full(stg), 2 * LY::kTile);
+          const int p0 = t * kKeys;
+          int y = pg.table == nullptr ? row_base + p0
+                                      : (int)kv_row(pg, layer, batch, r, nkv, gh, cap, p0);
+          if (!DFLASH_CHECK(y >= 0 && y < kv_rows, err)) y = 0;
+#pragma unroll
+          for (int h = 0; h < HALVES; ++h) {
+            tma_load_2d(sK + h * kKeys * 128, &tmK, full(stg), h * 64, y, policy_evict_first());
+            tma_load_2d(sV + h * kKeys * 128, &tmV, full(stg), h * 64, y, policy_evict_first());
+          }
+        }
+        gq = st0 + b;
+      }
+      if (!ok) set_error(err, DFLASH_DEV_TIMEOUT);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- compute warps
+  const float sl2 = rsqrtf((float)HD) * 1.4426950408889634f;  // log2(e) / sqrt(hd)
+  const int mi = lane >> 3, li = lane & 7;
+  const LdsmOff lo = ldsm_offsets(lane);
+  bool ok = true;
+  int it = 0;
+  for (long long gq = g0; gq < g1;) {
+    const int sg = seg_of(gq);
+    const long long st0 = seg_start[sg], en = seg_start[sg + 1];
+    const int a = (int)(gq - st0), b = (int)(min(en, g1) - st0);
+    const int r = sg / nkv, gh = sg % nkv;
+    const int Tc = ctx_of(r);
+    const int nctx = (Tc + kKeys - 1) / kKeys;
+    const bool has_blk = b == (int)(en - st0);  // the segment's last unit: the block's keys
+
+    // query rows of this (request, kv head): row i = (position i / G, head gh*G + i % G)
+    for (int idx = tid; idx < kRows * (HD / 8); idx += 128) {
+      const int row = idx / (HD / 8), ch = idx % (HD / 8);
+      const void* src = q;
+      int bytes = 0;
+      if (row < R) {
+        src = q + ((size_t)(r * B + row / G) * nq + gh * G + row % G) * HD + ch * 8;
+        bytes = 16;
+      }
+      cp_async16(s_q + toff(LY::kQRows, row, ch), src, bytes);
+    }
+    cp_async_commit();
+    cp_async_wait_all();
+    compute_bar();
+    uint32_t qa[KS][4];
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int row = mt * 16 + (mi & 1) * 8 + li;
+      ldsm_x4(s_q + toff(LY::kQRows, row, ks * 2 + (mi >> 1)), qa[ks][0], qa[ks][1], qa[ks][2],
+              qa[ks][3]);
+    }
+    compute_bar();  // the query area now takes the block tile
+    if (has_blk) {
+      for (int idx = tid; idx < 2 * kBlkKeys * (HD / 8); idx += 128) {
+        const int mat = idx / (kBlkKeys * (HD / 8));
+        const int rem = idx % (kBlkKeys * (HD / 8));
+        const int row = rem / (HD / 8), ch = rem % (HD / 8);
+        const void* src = kb;
+        int bytes = 0;
+        if (row < B) {
+          src = (mat ? vb : kb) + ((size_t)(r * B + row) * nkv + gh) * HD + ch * 8;
+          bytes = 16;
+        }
+        cp_async16(s_q + mat * (kBlkKeys * HD * 2) + toff(kBlkKeys, row, ch), src, bytes);
+      }
+      cp_async_commit();
+    }
+
+    float o[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    for (int t = a; t < min(b, nctx); ++t, ++it) {
+      const int stg = it % kStages;
+      if (!mbar_wait(full(stg), (it / kStages) & 1)) ok = false;
+      const int nvalid = min(kKeys, Tc - t * kKeys);
+      const uint32_t sK = s_base + stg * LY::kStage, sV = sK + LY::kTile;
+      const int kbeg = kg * KPW;
+      if (nvalid < kbeg + KPW) {
+        // rows past the context hold other positions: zero this warp's V rows
+        // there so that masked keys contribute exactly nothing
+        uint8_t* v = smem + stg * LY::kStage + LY::kTile;
+        const int z0 = max(nvalid, kbeg);
+        for (int idx = lane; idx < (kbeg + KPW - z0) * (HD / 8); idx += 32) {
+          const int row = z0 + idx / (HD / 8), ch = idx % (HD / 8);
+          *reinterpret_cast<uint4*>(v + toff(kKeys, row, ch)) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async();  // before the stage goes back to the TMA
+        __syncwarp();
+      }
+      attend<HD, KPW>(sK, sV, kKeys, kbeg, nvalid, qa, o, m0, m1, l0, l1, sl2, lo, lane);
+      __syncwarp();
+      if (lane == 0)
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty(stg)) : "memory");
+    }
+    if (has_blk) {
+      cp_async_wait_all();
+      compute_bar();
+      if (kg == 0)
+        attend<HD, kBlkKeys>(s_q, s_q + kBlkKeys * HD * 2, kBlkKeys, 0, B, qa, o, m0, m1, l0, l1,
+                             sl2, lo, lane);
+    }
+
+    // this warp's partial: slot (c + sg) * KG + kg, rows of its row tile
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    {
+      const float ln2 = 0.6931471805599453f;  // partial maxima in natural-log units
+      const size_t pbase = ((size_t)(c + sg) * KG + kg) * kRows;
+      const int tq = lane & 3;
+      const int row0 = mt * 16 + (lane >> 2), row1 = row0 + 8;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const int col = n * 8 + 2 * tq;
+        if (row0 < R)
+          *reinterpret_cast<float2*>(part_o + (pbase + row0) * HD + col) =
+              make_float2(o[n][0], o[n][1]);
+        if (row1 < R)
+          *reinterpret_cast<float2*>(part_o + (pbase + row1) * HD + col) =
+              make_float2(o[n][2], o[n][3]);
+      }
+      if (tq == 0) {
+        if (row0 < R)
+          *reinterpret_cast<float2*>(part_ml + (pbase + row0) * 2) = make_float2(m0 * ln2, l0);
+        if (row1 < R)
+          *reinterpret_cast<float2*>(part_ml + (pbase + row1) * 2) = make_float2(m1 * ln2, l1);
+      }
+    }
+    __threadfence();  // this piece's partials are visible before it is counted
+    compute_bar();
+    // pieces of this segment: the CTAs whose ranges meet it
+    const int c_lo = (int)(((st0 + 1) * P + W - 1) / W) - 1;
+    const int c_hi = (int)((en * P + W - 1) / W) - 1;
+    if (tid == 0) {
+      const bool last = atomicAdd(&cnt[sg], 1u) == (unsigned)(c_hi - c_lo);
+      if (last) cnt[sg] = 0;  // ready for the next launch
+      s_last = last ? 1 : 0;
+    }
+    compute_bar();
+    if (s_last) {
+      __threadfence();  // every counted partial is visible to the reads below
+      // merge: weights exp(m - M) / L per (partial, row), CTAs in order
+      const int NP = (c_hi - c_lo + 1) * KG;
+      auto slot_of = [&](int e) { return (size_t)(c_lo + e / KG + sg) * KG + e % KG; };
+      float* sM = scratch;
+      float* sIL = scratch + kRows;
+      float* sw = scratch + 2 * kRows;
+      const int CH = (LY::kQ / 4 - 2 * kRows) / kRows;  // partials per weight chunk
+      if (tid < R) {
+        float M = -INFINITY, L = 0.f;
+        for (int e = 0; e < NP; ++e) {
+          const float2 ml =
+              __ldcg(reinterpret_cast<const float2*>(part_ml + (slot_of(e) * kRows + tid) * 2));
+          if (ml.x == -INFINITY) continue;
+          if (ml.x > M) {
+            L = (M == -INFINITY ? 0.f : L * expf(M - ml.x)) + ml.y;
+            M = ml.x;
+          } else {
+            L += ml.y * expf(ml.x - M);
+          }
+        }
+        sM[tid] = M;
+        sIL[tid] = L > 0.f ? 1.f / L : 0.f;
+      }
+      compute_bar();
+      float4 acc[kAcc];
+#pragma unroll
+      for (int k = 0; k < kAcc; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int e0 = 0; e0 < NP; e0 += CH) {
+        const int ne = min(CH, NP - e0);
+        for (int idx = tid; idx < ne * kRows; idx += 128) {
+          const int e = e0 + idx / kRows, row = idx % kRows;
+          float wgt = 0.f;
+          if (row < R) {
+            const float mm = __ldcg(part_ml + (slot_of(e) * kRows + row) * 2);
+            wgt = mm == -INFINITY ? 0.f : expf(mm - sM[row]) * sIL[row];
+          }
+          sw[idx] = wgt;
+        }
+        compute_bar();
+#pragma unroll
+        for (int k = 0; k < kAcc; ++k) {
+          const int i4 = tid + k * 128;
+          if (i4 >= R * HD / 4) break;
+          const int row = (i4 * 4) / HD, col = (i4 * 4) % HD;
+          for (int e = e0; e < e0 + ne; ++e) {
+            const float wgt = sw[(e - e0) * kRows + row];
+            const float4 v =
+                __ldcg(reinterpret_cast<const float4*>(part_o + (slot_of(e) * kRows + row) * HD + col));
+            acc[k].x += wgt * v.x;
+            acc[k].y += wgt * v.y;
+            acc[k].z += wgt * v.z;
+            acc[k].w += wgt * v.w;
+          }
+        }
+        compute_bar();
+      }
+#pragma unroll
+      for (int k = 0; k < kAcc; ++k) {
+        const int i4 = tid + k * 128;
+        if (i4 >= R * HD / 4) break;
+        const int row = (i4 * 4) / HD, col = (i4 * 4) % HD;
+        __half* dst = out + ((size_t)(r * B + row / G) * nq + gh * G + row % G) * HD + col;
+        *reinterpret_cast<__half2*>(dst) = __floats2half2_rn(acc[k].x, acc[k].y);
+        *reinterpret_cast<__half2*>(dst + 2) = __floats2half2_rn(acc[k].z, acc[k].w);
+      }
+    }
+    compute_bar();  // the query area is free for the next piece
+    gq = st0 + b;
+  }
+  if (!ok) set_error(err, DFLASH_DEV_TIMEOUT);
+}
+
+template <int HD, int MT>
+int launch_persistent(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q,
+                      const __half* kb, const __half* vb, const KvPages& pg, long long kv_rows,
+                      int layer, int batch, int cap, const int32_t* ctx_len,
+                      const int32_t* req_valid, int B, int nq, int nkv, const int32_t* seg_start,
+                      float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
+                      cudaStream_t s) {
+  const int smem = Layout<HD, MT>::kSmem;
+  if (cudaFuncSetAttribute(attn_tc_persistent<HD, MT>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return DFLASH_ECUDA;
+  const cudaError_t e = launch_pdl(attn_tc_persistent<HD, MT>, dim3(2 * num_sms()),
+                                   dim3(kThreads), smem, s, 1, tk, tv, q, kb, vb, pg, kv_rows,
+                                   layer, batch, cap, ctx_len, req_valid, B, nq, nkv, seg_start,
+                                   part_o, part_ml, cnt, o, err);
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
+}
+
 template <int HD, int MT>
 int launch_cfg(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q, const __half* kb,
                const __half* vb, const KvPages& pg, long long kv_rows, int layer, int batch, int cap,
@@ -540,10 +917,9 @@ int launch_cfg(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q, co
 template <int HD>
 int launch_hd(const __half* q, const __half* kb, const __half* vb, const __half* kc,
               const __half* vc, const KvPages& pg, int layer, int batch, int cap,
-              const int32_t* ctx_len,
-              const int32_t* req_valid, int B, int nq, int nkv, int L, int chunk, int n_chunks,
-              float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
-              cudaStream_t s) {
+              const int32_t* ctx_len, const int32_t* req_valid, int B, int nq, int nkv, int L,
+              int chunk, int n_chunks, const int32_t* seg_start, float* part_o, float* part_ml,
+              unsigned* cnt, __half* o, int32_t* err, cudaStream_t s) {
   CUtensorMap tk, tv;
   const int64_t rows = pg.table == nullptr ? (int64_t)L * batch * nkv * cap
                                            : (int64_t)L * pg.n_pages * nkv * pg.page;
@@ -551,6 +927,19 @@ int launch_hd(const __half* q, const __half* kb, const __half* vb, const __half*
       !encode_2d(&tv, vc, rows, HD, HD, kKeys, DFLASH_F16))
     return DFLASH_ECUDA;
   const int R = B * (nq / nkv);
+  if (seg_start != nullptr) {
+    if (R <= 16)
+      return launch_persistent<HD, 1>(tk, tv, q, kb, vb, pg, rows, layer, batch, cap, ctx_len,
+                                      req_valid, B, nq, nkv, seg_start, part_o, part_ml, cnt, o,
+                                      err, s);
+    if (R <= 32)
+      return launch_persistent<HD, 2>(tk, tv, q, kb, vb, pg, rows, layer, batch, cap, ctx_len,
+                                      req_valid, B, nq, nkv, seg_start, part_o, part_ml, cnt, o,
+                                      err, s);
+    return launch_persistent<HD, 4>(tk, tv, q, kb, vb, pg, rows, layer, batch, cap, ctx_len,
+                                    req_valid, B, nq, nkv, seg_start, part_o, part_ml, cnt, o, err,
+                                    s);
+  }
   if (R <= 16)
     return launch_cfg<HD, 1>(tk, tv, q, kb, vb, pg, rows, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
                              chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
@@ -563,14 +952,22 @@ int launch_hd(const __half* q, const __half* kb, const __half* vb, const __half*
 
 }  // namespace
 
+int launch_attn_plan(const int32_t* ctx_len, const int32_t* req_valid, int batch, int nkv,
+                     int32_t* seg_start, cudaStream_t s) {
+  TimedScope ts(s, TC_ATTN);
+  const cudaError_t e = launch_pdl(attn_plan_kernel, dim3(1), dim3(1024), 0, s, 1, ctx_len,
+                                   req_valid, batch, nkv, seg_start);
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
+}
+
 int launch_attn_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
                    const __half* vc, const KvPages& pg, int layer, int batch, int cap,
                    const int32_t* ctx_len,
                    const int32_t* req_valid, int B, int nq, int nkv, int hd, int L, int chunk,
-                   int n_chunks, float* part_o, float* part_ml, unsigned* cnt, __half* o,
-                   int32_t* err, cudaStream_t s) {
-  if (B * (nq / nkv) > kAttnMaxRows || chunk % kKeys != 0 || B > kBlkKeys ||
-      n_chunks > kMaxChunksTc)
+                   int n_chunks, const int32_t* seg_start, float* part_o, float* part_ml,
+                   unsigned* cnt, __half* o, int32_t* err, cudaStream_t s) {
+  if (B * (nq / nkv) > kAttnMaxRows || B > kBlkKeys) return DFLASH_EUNSUPPORTED;
+  if (seg_start == nullptr && (chunk % kKeys != 0 || n_chunks > kMaxChunksTc))
     return DFLASH_EUNSUPPORTED;
   if (pg.table == nullptr && (int64_t)L * batch * nkv * cap > 0x7fffffffLL)
     return DFLASH_EUNSUPPORTED;
@@ -580,10 +977,10 @@ int launch_attn_tc(const __half* q, const __half* kb, const __half* vb, const __
   TimedScope ts(s, TC_ATTN);
   if (hd == 128)
     return launch_hd<128>(q, kb, vb, kc, vc, pg, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, L,
-                          chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
+                          chunk, n_chunks, seg_start, part_o, part_ml, cnt, o, err, s);
   if (hd == 64)
     return launch_hd<64>(q, kb, vb, kc, vc, pg, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, L,
-                         chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
+                         chunk, n_chunks, seg_start, part_o, part_ml, cnt, o, err, s);
   return DFLASH_EUNSUPPORTED;
 }
 

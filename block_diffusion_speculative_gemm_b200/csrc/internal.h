@@ -242,22 +242,29 @@ constexpr int kAttnMaxRows = 64;  // B * (n_q / n_kv) query rows per (request, k
 // kv head), found with cnt[request * nkv + head] (zero before and after the
 // call), merges them into o [batch * B][nq][hd].  The cache is
 // [L][batch][nkv][cap][hd]; `layer` selects the layer.
+// Persistent schedule: seg_start (from launch_attn_plan, once per forward)
+// non-null; partials part_o [(2 * SMs + batch * nkv) * 64][hd] and part_ml
+// [...][2]; cnt one zeroed counter per (request, kv head).  seg_start null: the
+// split-KV grid of `chunk`-key chunks.
+int launch_attn_plan(const int32_t* ctx_len, const int32_t* req_valid, int batch, int nkv,
+                     int32_t* seg_start, cudaStream_t s);
 int launch_attn_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
                    const __half* vc, const KvPages& pages, int layer, int batch, int cap,
-                   const int32_t* ctx_len,
-                   const int32_t* req_valid, int B, int nq, int nkv, int hd, int L, int chunk,
-                   int n_chunks, float* part_o, float* part_ml, unsigned* cnt, __half* o,
-                   int32_t* err, cudaStream_t s);
+                   const int32_t* ctx_len, const int32_t* req_valid, int B, int nq, int nkv,
+                   int hd, int L, int chunk, int n_chunks, const int32_t* seg_start,
+                   float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
+                   cudaStream_t s);
 
 // T: type of q, the block's k/v and the output o; TC: K/V cache type.
-// Paged K/V (pages.table set) is read by the tensor-core kernel only.
+// Paged K/V (pages.table set) and the persistent schedule (seg_start set) are
+// the tensor-core kernel's only.
 template <typename T, typename TC>
 int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, const TC* vc,
                            const KvPages& pages, int layer, int L, int batch, int cap,
-                           const int32_t* ctx_len,
-                           const int32_t* req_valid, int B, int nq, int nkv, int hd,
-                           float* part_o, float* part_ml, int n_chunks, int chunk, T* o,
-                           unsigned* cnt, int32_t* err, cudaStream_t s);
+                           const int32_t* ctx_len, const int32_t* req_valid, int B, int nq,
+                           int nkv, int hd, float* part_o, float* part_ml, int n_chunks, int chunk,
+                           const int32_t* seg_start, T* o, unsigned* cnt, int32_t* err,
+                           cudaStream_t s);
 
 // ---------------------------------------------------------------- draft bookkeeping
 // cap bounds ctx_len + B; with paged K/V every page below ctx_len must also be

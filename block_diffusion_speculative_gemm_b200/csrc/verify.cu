@@ -91,7 +91,6 @@ __global__ void __launch_bounds__(kVerifyThreads)
                   int out_cap, int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
                   int32_t* err, ArgPart* shard_out, int vocab_offset) {
   pdl_trigger();
-  pdl_wait();
   __shared__ float s_v[kVerifyThreads / 32];
   __shared__ int s_i[kVerifyThreads / 32];
   __shared__ int s_last;
@@ -99,6 +98,23 @@ __global__ void __launch_bounds__(kVerifyThreads)
   const int v0 = c * chunk;
   const int v1 = min(V, v0 + chunk);
   const T* x = logits + (size_t)row * V;
+  if (VEC && (threadIdx.x & 31) == 0 && v1 > v0) {
+    // The logits are an input no kernel of the cycle writes: while the
+    // predecessor drains, each warp asks L2 for its share of the chunk.  L2 is
+    // the point of coherence, so a line prefetched early is never read stale.
+    const int nw = kVerifyThreads / 32, w = threadIdx.x >> 5;
+    const size_t bytes = (size_t)(v1 - v0) * sizeof(T);       // a multiple of 16
+    const size_t per = (bytes / nw + 15) / 16 * 16;
+    const size_t b0 = (size_t)w * per;
+    if (b0 < bytes) {
+      const uint32_t n = (uint32_t)min(per, bytes - b0);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                       reinterpret_cast<const uint8_t*>(x + v0) + b0),
+                   "r"(n)
+                   : "memory");
+    }
+  }
+  pdl_wait();
   float best = -INFINITY;
   int bi = 0x7fffffff;
   if (VEC) {

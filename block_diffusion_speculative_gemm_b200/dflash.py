@@ -120,6 +120,7 @@ def lib() -> ctypes.CDLL:
         L.dflash_debug_lmhead_tiled.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp, vp, vp]
         L.dflash_debug_gemm_mode.argtypes = [i32]
         L.dflash_debug_gemm_schedule.argtypes = [i32]
+        L.dflash_debug_attn_schedule.argtypes = [i32]
         L.dflash_debug_gemm_streamk_ws_bytes.argtypes = [i32]
         L.dflash_debug_gemm_streamk_ws_bytes.restype = sz
         L.dflash_debug_gemm_streamk.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp, sz, vp]
@@ -675,6 +676,12 @@ def debug_lmhead(W: torch.Tensor, X: torch.Tensor, err_ws: torch.Tensor, want_lo
             _ptr(W), N, K, _ptr(X), M, elem, _ptr(stats), _ptr(logits), _ptr(err_ws),
             _stream(stream)))
     return stats, logits
+
+
+def debug_attn_schedule(sched: int) -> None:
+    """Process-wide draft attention schedule: 0 the split-KV grid of fixed
+    chunks (default), 1 persistent (tests and tuning)."""
+    _check("dflash_debug_attn_schedule", lib().dflash_debug_attn_schedule(int(sched)))
 
 
 def debug_attn_chunk(keys: int) -> None:

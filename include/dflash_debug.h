@@ -95,6 +95,15 @@ int dflash_debug_pick_splits(int M, int N, int K);
  * thread-safe; tests and tuning only. */
 int dflash_debug_split_weight(float w);
 
+/* Schedule of the draft attention (bf16 models) for every later call,
+ * process-wide: 0 (default) the split-KV grid of fixed key chunks
+ * (dflash_debug_attn_chunk); 1 persistent, two CTAs per SM each streaming the
+ * same number of 64-key tiles over the (request, kv head) segments, segments
+ * split between CTAs merged by their last piece.  Both give the same result up
+ * to fp32 summation order.  DFLASH_EINVAL for any other value.  Not
+ * thread-safe; tests and tuning only. */
+int dflash_debug_attn_schedule(int sched);
+
 /* Split-KV chunk of the draft attention, in keys, for every later
  * dflash_draft_block call, process-wide: 0 = the library's rule (at least 512
  * keys, at most 64 chunks per request), else a multiple of 64 that is used

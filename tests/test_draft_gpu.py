@@ -107,7 +107,7 @@ def test_draft_attention_chunk_sizes(chunk):
                  H_t=512).replace(name="chunk8b")
     b = built(cfg)
     ctx = torch.tensor([0, 63, 64, 900], dtype=torch.int32)
-    D.debug_attn_chunk(chunk)
+    D.debug_attn_chunk(chunk)  # the split-KV grid (the default schedule)
     try:
         res = _run_draft(b, cfg, ctx=ctx)
     finally:
@@ -175,3 +175,33 @@ def test_draft_gemm_schedules_agree():
         diff = (la[both] - lb[both]).abs().max().item()
         record("draft_gemm_schedules", max_rel_diff=diff / scale)
         assert diff <= 2e-3 * scale
+
+
+@pytest.mark.parametrize("name,ctx", [
+    ("edge", (0, 1, 63, 64, 65, 600)),   # empty, one key, tile edges, a long one
+    ("uniform", None),
+])
+def test_draft_attention_schedules_agree(name, ctx):
+    """The persistent attention (every CTA the same number of key tiles across
+    (request, head) segments, segments split between CTAs merged by their last
+    piece) and the split-KV grid give the oracle's draft; their logits agree far
+    inside the tolerance."""
+    base = synth.get_config("qwen3_8b_bs32")
+    cfg = shrink(base, L=2, V=2048, batch=6, ctx=("uniform", 1, 700), I=512, d=512,
+                 H_t=512).replace(name="attn_sched8b")
+    b = built(cfg)
+    ctx_t = None if ctx is None else torch.tensor(ctx, dtype=torch.int32)
+    runs = []
+    try:
+        for sched in (1, 0):
+            D.debug_attn_schedule(sched)
+            runs.append(_run_draft(b, cfg, ctx=ctx_t))
+    finally:
+        D.debug_attn_schedule(0)
+    for res in runs:
+        assert res["err"] == 0
+        _check(b, cfg, res, cfg.steps, range(cfg.batch), test=f"draft_attention_schedules[{name}]")
+    la, lb = runs[0]["lg"], runs[1]["lg"]
+    both = ~(torch.isnan(la) | torch.isnan(lb))
+    scale = la[both].abs().max().item()
+    assert (la[both] - lb[both]).abs().max().item() <= 2e-3 * scale
