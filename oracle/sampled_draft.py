@@ -43,9 +43,10 @@ from typing import Optional
 import numpy as np
 
 from .dflash_oracle import Weights64, commit_count, draft_hidden, select_commits
-from .sampled_verify import gumbel_argmax, log_softmax, philox_words, uniform_open
+from .sampled_verify import (gumbel_argmax, log_softmax, neg_log_uniform_open, philox_words,
+                             uniform_open)
 
-__all__ = ["STREAM_DRAFT", "draft_draw_uniforms", "sampled_draft_block"]
+__all__ = ["STREAM_DRAFT", "draft_draw_uniforms", "draft_draw_exponentials", "sampled_draft_block"]
 
 STREAM_DRAFT = 2
 
@@ -55,6 +56,14 @@ def draft_draw_uniforms(seed: int, offset: int, request: int, step: int, pos: in
     """U'_v, v < V, of position `pos` at denoising step `step` (stream 2)."""
     n0 = (step * B + pos) * V
     return uniform_open(philox_words(seed, offset, request, STREAM_DRAFT, n0 + np.arange(V)))
+
+
+def draft_draw_exponentials(seed: int, offset: int, request: int, step: int, pos: int, B: int,
+                            V: int) -> np.ndarray:
+    """-ln U'_v, v < V, of the same draws, exact (neg_log_uniform_open)."""
+    n0 = (step * B + pos) * V
+    return neg_log_uniform_open(philox_words(seed, offset, request, STREAM_DRAFT,
+                                             n0 + np.arange(V)))
 
 
 def sampled_draft_block(anchor: int, T: int, caches, W: Weights64, cfg, tau: float, seed: int,
@@ -79,7 +88,7 @@ def sampled_draft_block(anchor: int, T: int, caches, W: Weights64, cfg, tau: flo
         lp1 = log_softmax(Y, 1.0)
         draws, confs = [], []
         for i, j in enumerate(masked):
-            x, _ = gumbel_argmax(lp[i], draft_draw_uniforms(seed, offset, request, t, j, B, V))
+            x, _ = gumbel_argmax(lp[i], draft_draw_exponentials(seed, offset, request, t, j, B, V))
             draws.append(x)
             confs.append(float(np.exp(lp1[i, x])))
         k = commit_count(len(masked), steps - t)

@@ -55,6 +55,8 @@ __all__ = [
     "STREAM_DRAW",
     "accept_uniforms",
     "draw_uniforms",
+    "draw_exponentials",
+    "neg_log_uniform_open",
     "log_softmax",
     "gumbel_argmax",
     "residual_log_weights",
@@ -132,6 +134,21 @@ def uniform_open(w) -> np.ndarray:
     return ((np.asarray(w, dtype=np.uint64) >> np.uint64(11)).astype(np.float64) + 0.5) * 2.0 ** -53
 
 
+def neg_log_uniform_open(w) -> np.ndarray:
+    """E = -ln U' for U' = ((w >> 11) + 1/2) * 2^-53, the exponential variate of a
+    Gumbel draw, without rounding U' first.  Below 1/2, U' = (k + 1/2) 2^-53 is
+    exact in float64 and E = -log U'.  From 1/2 up, U' needs 54 bits, but
+    1 - U' = (2^53 - 1 - k + 1/2) 2^-53 is exact and E = -log1p(-(1 - U')).
+    (Rounding U' to float64 would drop its last bit there and turn the top word
+    into U' = 1, E = 0.)"""
+    k = np.asarray(w, dtype=np.uint64) >> np.uint64(11)
+    lo = k < np.uint64(1 << 52)
+    u = (k.astype(np.float64) + 0.5) * 2.0 ** -53
+    m = ((np.uint64((1 << 53) - 1) - k).astype(np.float64) + 0.5) * 2.0 ** -53
+    with np.errstate(divide="ignore"):
+        return np.where(lo, -np.log(u), -np.log1p(-m))
+
+
 def accept_uniforms(seed: int, offset: int, request: int, n: int) -> np.ndarray:
     """U_0 .. U_{n-1} of a request (stream 0)."""
     return uniform_closed_open(philox_words(seed, offset, request, STREAM_ACCEPT, np.arange(n)))
@@ -142,6 +159,11 @@ def draw_uniforms(seed: int, offset: int, request: int, V: int) -> np.ndarray:
     return uniform_open(philox_words(seed, offset, request, STREAM_DRAW, np.arange(V)))
 
 
+def draw_exponentials(seed: int, offset: int, request: int, V: int) -> np.ndarray:
+    """-ln U'_0 .. -ln U'_{V-1} of a request (stream 1), exact (neg_log_uniform_open)."""
+    return neg_log_uniform_open(philox_words(seed, offset, request, STREAM_DRAW, np.arange(V)))
+
+
 def log_softmax(z, tau: float) -> np.ndarray:
     """log softmax(z / tau) over the last axis, in float64."""
     s = np.asarray(z, dtype=np.float64) / float(tau)
@@ -149,10 +171,11 @@ def log_softmax(z, tau: float) -> np.ndarray:
     return s - m - np.log(np.sum(np.exp(s - m), axis=-1, keepdims=True))
 
 
-def gumbel_argmax(logw: np.ndarray, u_open: np.ndarray):
-    """Gumbel-max draw: argmax_v (logw_v - log(-log U'_v)) over entries with a finite
-    log-weight, ties to the lowest index.  Returns (index, the score array)."""
-    score = np.where(np.isfinite(logw), logw - np.log(-np.log(u_open)), -np.inf)
+def gumbel_argmax(logw: np.ndarray, e: np.ndarray):
+    """Gumbel-max draw: argmax_v (logw_v - log E_v), E_v = -ln U'_v (so -log E_v is
+    the Gumbel variate), over entries with a finite log-weight, ties to the lowest
+    index.  Returns (index, the score array)."""
+    score = np.where(np.isfinite(logw), logw - np.log(e), -np.inf)
     return int(np.argmax(score)), score
 
 
@@ -195,7 +218,7 @@ def sampled_verify_request(Z, Y, draft, tau: float, seed: int, offset: int, requ
     logw = residual_log_weights(lp[a], lq[a + 1]) if a < B - 1 else lp[B - 1]
     if not np.any(np.isfinite(logw)):
         logw = lp[a]  # p == q to the last bit: the residual is empty, draw from p
-    tok, score = gumbel_argmax(logw, draw_uniforms(seed, offset, request, V))
+    tok, score = gumbel_argmax(logw, draw_exponentials(seed, offset, request, V))
     return {"a": a, "emitted": d[1:a + 1] + [tok], "token": tok, "log_rho": log_rho,
             "log_u": log_u, "score": score, "logw": logw}
 

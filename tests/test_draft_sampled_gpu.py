@@ -52,8 +52,7 @@ class SampledReport(DraftReport):
 
 
 def _gumbel(r, t, p, B, V):
-    u = SD.draft_draw_uniforms(SEED, OFFSET, r, t, p, B, V)
-    return -np.log(-np.log(u))
+    return -np.log(SD.draft_draw_exponentials(SEED, OFFSET, r, t, p, B, V))
 
 
 def check_sampled_request(b, r, anchor, T, caches, tokens_gpu, cstep_gpu, q_gpu, steps, tau,

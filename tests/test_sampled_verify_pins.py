@@ -15,6 +15,8 @@ Each check rests on something other than the oracle's own formulas:
 * the sure-accept and sure-reject cases, and the output bookkeeping.
 """
 
+from decimal import Decimal, localcontext
+
 import numpy as np
 import pytest
 import scipy.stats
@@ -70,10 +72,34 @@ def test_uniform_maps_end_points():
     assert SV.uniform_closed_open(np.uint64(0)) == 0.0
     assert SV.uniform_closed_open(np.uint64(M64)) == 1.0 - 2.0 ** -53
     assert SV.uniform_open(np.uint64(0)) == 2.0 ** -54
-    assert SV.uniform_open(np.uint64(M64)) == 1.0 - 2.0 ** -54
+    # the top word's U' = 1 - 2^-54 is not a float64; its exponential variate
+    # -ln U' is still exact and positive
+    assert SV.neg_log_uniform_open(np.uint64(M64)) == pytest.approx(2.0 ** -54, rel=1e-15)
+    assert SV.neg_log_uniform_open(np.uint64(0)) == pytest.approx(54 * np.log(2.0), rel=1e-15)
     # 53 significant bits: the low 11 bits of the word never matter
     assert SV.uniform_closed_open(np.uint64(2047)) == 0.0
     assert SV.uniform_closed_open(np.uint64(2048)) == 2.0 ** -53
+
+
+def _neg_log_decimal(k: int) -> Decimal:
+    """-ln(((k + 1/2) 2^-53)) in 50-digit decimal arithmetic."""
+    with localcontext() as ctx:
+        ctx.prec = 50
+        u = (Decimal(k) + Decimal("0.5")) / (Decimal(2) ** 53)
+        return -u.ln()
+
+
+def test_neg_log_uniform_open_matches_decimal():
+    # random words over both halves, the words at the switch between the two
+    # formulas and the ends, against an independent 50-digit evaluation
+    rng = np.random.default_rng(11)
+    ks = [int(x) for x in rng.integers(0, 1 << 53, size=200, dtype=np.uint64)]
+    ks += [0, 1, (1 << 52) - 1, 1 << 52, (1 << 52) + 1, (1 << 53) - 2, (1 << 53) - 1,
+           (1 << 53) - 1000, 1 << 40]
+    got = SV.neg_log_uniform_open(np.array(ks, dtype=np.uint64) << np.uint64(11))
+    for k, g in zip(ks, got):
+        want = float(_neg_log_decimal(k))
+        assert g == pytest.approx(want, rel=4e-16), k
 
 
 def test_streams_and_requests_are_distinct():
@@ -162,7 +188,7 @@ def test_bonus_draw_is_distributed_as_last_target_row():
 
 def test_gumbel_argmax_frequencies():
     p = np.array([0.5, 0.25, 0.125, 0.125])
-    toks = [SV.gumbel_argmax(np.log(p), SV.draw_uniforms(3, 0, r, 4))[0] for r in range(8000)]
+    toks = [SV.gumbel_argmax(np.log(p), SV.draw_exponentials(3, 0, r, 4))[0] for r in range(8000)]
     assert _chi2_pvalue(np.array(toks), p) > 1e-4
 
 

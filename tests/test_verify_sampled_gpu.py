@@ -62,7 +62,7 @@ def _draw_at(lp, lq, a, B, seed, offset, r, V):
     logw = SV.residual_log_weights(lp[a], lq[a + 1]) if a < B - 1 else lp[B - 1]
     if not np.any(np.isfinite(logw)):
         logw = lp[a]
-    return SV.gumbel_argmax(logw, SV.draw_uniforms(seed, offset, r, V))
+    return SV.gumbel_argmax(logw, SV.draw_exponentials(seed, offset, r, V))
 
 
 def _check(Z, Y, d, tau, seed, offset, out0, ol0, seq0, res, stats):
