@@ -320,6 +320,23 @@ def run_dflash(args, rank, world, local_rank):
         d1.record(stream)
         torch.cuda.synchronize()
     draft_ms = d0.elapsed_time(d1) / n_draft
+    # sampled drafting (temperature 1) over the same caches: the same forwards, the
+    # committing-step logits rows written for sampled verify, and a Gumbel-max draw
+    # over the vocabulary of every masked row in place of the LM-head argmax
+    q_rows = torch.empty((b, B, V), dtype=torch.bfloat16, device=dev)
+    draft_s = torch.zeros_like(draft)
+    for k in range(3):
+        D.draft_block_sampled(model, anchors_d, ctx_d, kc, vc, B, cfg.steps, 1.0, 0x5EED, k,
+                              draft_s, q_rows, ws)
+    torch.cuda.synchronize()
+    d0.record(stream)
+    for k in range(n_draft):
+        D.draft_block_sampled(model, anchors_d, ctx_d, kc, vc, B, cfg.steps, 1.0, 0x5EED, 3 + k,
+                              draft_s, q_rows, ws)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    sampled_ms = d0.elapsed_time(d1) / n_draft
+    del q_rows
     err = D.get_error(ws)
     if err:
         raise RuntimeError(f"device error word {err}")
@@ -398,6 +415,10 @@ def run_dflash(args, rank, world, local_rank):
                         "block_tok_s": round(b * world * B / (draft_ms / 1e3), 1),
                         "drafted_tok_s": round(b * world * (B - 1) / (draft_ms / 1e3), 1),
                         "clocks": dclk.summary()},
+        # dflash_draft_block_sampled at temperature 1, same loop
+        "draft_block_sampled": {"ms": round(sampled_ms, 4),
+                                "block_tok_s": round(b * world * B / (sampled_ms / 1e3), 1),
+                                "over_greedy": round(sampled_ms / draft_ms, 4)},
         "prefill_inject": prefill_report(cfg, n_p, prefill_ms, peaks),
         "clocks": clocks,
     }
@@ -813,6 +834,14 @@ def sampled_verify_report():
     ms_s = timed(sampled)
     ms_g = timed(greedy)
     assert D.get_error(ws) == 0
+
+    # context only (not on the path): PyTorch's row argmax over the same target
+    # logits, the library reduction that reads the same bytes as greedy verify
+    def torch_argmax(k):
+        Z, _, _ = sets[k % 2]
+        torch.argmax(Z.view(b * B, V), dim=-1)
+
+    ms_t = timed(torch_argmax)
     bytes_s = b * (2 * B - 1) * V * 2
     bytes_g = b * B * V * 2
     print(json.dumps({
@@ -822,6 +851,8 @@ def sampled_verify_report():
         "sampled_frac_hbm": round(bytes_s / ms_s / 1e6 / hbm, 4),
         "greedy_us": round(ms_g * 1e3, 2),
         "greedy_frac_hbm": round(bytes_g / ms_g / 1e6 / hbm, 4),
+        "torch_argmax_us": round(ms_t * 1e3, 2),
+        "torch_argmax_frac_hbm": round(bytes_g / ms_t / 1e6 / hbm, 4),
         "rows_per_s_sampled": round(b * B / (ms_s / 1e3), 1),
         "hbm_peak_GBps": hbm, "peak_source": peaks["source"]}), flush=True)
 

@@ -1434,6 +1434,12 @@ extern "C" int dflash_debug_wait_timeout(void* err_ws, void* stream) {
   return cuda_status();
 }
 
+extern "C" int dflash_debug_sample_math(const uint64_t* w, const float* d, int n, float* g2,
+                                        float* l2, void* stream) {
+  if (n < 0 || (n > 0 && (!w || !d || !g2 || !l2))) return DFLASH_EINVAL;
+  return launch_sample_math(w, d, n, g2, l2, (cudaStream_t)stream);
+}
+
 extern "C" int dflash_debug_pick_splits(int M, int N, int K) {
   if (M < 1 || N < 1 || K < 64 || K % 64) return DFLASH_EINVAL;
   return gemm_pick_splits(M, N, K, kMaxSplits);

@@ -35,6 +35,15 @@ template <> __device__ __forceinline__ bool narrow_bad<__half>(float v) {
   return !(fabsf(v) < 65520.f);
 }
 
+// 2^x from the hardware approximation (PTX ex2.approx.ftz.f32: relative error
+// about 2^-22, results below 2^-126 flushed to zero).  For sums of softmax
+// terms, where neither matters at fp32 accuracy.
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------- errors
 __device__ __forceinline__ void set_error(int32_t* err, int bits) {
   if (err) atomicOr(err, bits);

@@ -330,6 +330,8 @@ int launch_verify_merge(const ArgPart* parts, int world, const int32_t* draft, i
 // ---------------------------------------------------------------- sampled verify
 // Scratch bytes of one sampled-verify call (placed after the workspace header).
 size_t sampled_verify_bytes(int batch, int B, int V);
+int launch_sample_math(const uint64_t* w, const float* d, int n, float* g2, float* l2,
+                       cudaStream_t s);
 int launch_sampled_verify(const void* target, const void* drafted, int dtype, const int32_t* draft,
                           int batch, int B, int V, float tau, uint64_t seed, uint64_t offset,
                           int32_t* out_tokens, int32_t* out_len, int out_cap, int32_t* seq_lens,

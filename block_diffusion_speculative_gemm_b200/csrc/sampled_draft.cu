@@ -86,7 +86,7 @@ __device__ __forceinline__ void load4(const T* p, bool vec, float (&x)[4], int n
 }
 
 template <typename T, bool VEC>
-__global__ void __launch_bounds__(kSdThreads)
+__global__ void __launch_bounds__(kSdThreads, 4)
     sd_draw_kernel(const T* __restrict__ q, const int32_t* __restrict__ lm_rows,
                    const int32_t* __restrict__ req_valid, int B, int V, int step, float inv_tau,
                    int chunk, int chunks, SdPart* __restrict__ part, unsigned* __restrict__ cnt,
@@ -104,6 +104,7 @@ __global__ void __launch_bounds__(kSdThreads)
   if (req_valid == nullptr || req_valid[r]) {
     const T* y = q + (size_t)pos * V;
     const uint64_t n0 = ((uint64_t)step * B + j) * (uint64_t)V;
+    const float c2 = inv_tau * kLog2e;
     const int v0 = c * chunk, v1 = min(V, v0 + chunk);  // chunk is a multiple of 4
     // groups of 4 consecutive entries; their draws n0 + vb .. n0 + vb + 3 lie in
     // one Philox block when n0 % 4 == 0, else in two.  Each thread visits its
@@ -113,23 +114,30 @@ __global__ void __launch_bounds__(kSdThreads)
       float x[4];
       load4<T>(y + vb, VEC, x, n);
       const uint64_t na = n0 + (uint64_t)vb;
-      const int sh = (int)(na & 3u);
-      uint64_t wa[4], wb[4];
+      // VEC launches have V % 4 == 0, so n0 % 4 == 0 and every group is one block
+      const int sh = VEC ? 0 : (int)(na & 3u);
+      uint64_t wa[4], wb[4] = {0, 0, 0, 0};
       philox_block(seed, offset, r, kSdStream, na >> 2, wa);
-      if (sh != 0) philox_block(seed, offset, r, kSdStream, (na >> 2) + 1, wb);
+      if (!VEC && sh != 0) philox_block(seed, offset, r, kSdStream, (na >> 2) + 1, wb);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         if (k >= n) break;
-        const int wi = sh + k;
-        const uint64_t w = wi < 4 ? wa[wi] : wb[wi - 4];
+        // word sh + k of the two blocks, chosen by selects (a register index)
+        uint64_t w = wa[k];
+        if (!VEC) {
+          const uint64_t c1 = k < 3 ? wa[k + 1] : wb[k - 3];
+          const uint64_t c2w = k < 2 ? wa[k + 2] : wb[k - 2];
+          const uint64_t c3 = k < 1 ? wa[k + 3] : wb[k - 1];
+          w = sh == 1 ? c1 : sh == 2 ? c2w : sh == 3 ? c3 : w;
+        }
         const float t2 = x[k] * kLog2e;
         if (t2 > m) {
           s = (m == -INFINITY) ? 1.f : s * exp2f(m - t2) + 1.f;
           m = t2;
         } else {
-          s += exp2f(t2 - m);
+          s += ex2_ftz(t2 - m);
         }
-        const float sc = x[k] * inv_tau + gumbel_of(w);
+        const float sc = fmaf(x[k], c2, gumbel2_of(w));  // (Y / tau + G) log2 e
         if (sc > gs) {
           gs = sc;
           gi = vb + k;
@@ -205,25 +213,40 @@ int launch_sampled_draw(const void* q, int q_bf16, const int32_t* lm_rows,
                         uint64_t seed, uint64_t offset, int32_t* tok, float* conf, void* part,
                         int chunks, unsigned* cnt, cudaStream_t s) {
   if (rows <= 0) return DFLASH_OK;
-  int chunk = (V + chunks - 1) / chunks;
-  chunk = (chunk + 63) / 64 * 64;
   const int esz = q_bf16 ? 2 : 4;
   const bool vec = V % 4 == 0 && (reinterpret_cast<uintptr_t>(q) % (4 * esz)) == 0;
-  const dim3 grid(chunks, rows), block(kSdThreads);
   const float inv_tau = 1.f / tau;
   SdPart* p = static_cast<SdPart*>(part);
+  // `chunks` is what the partials were sized for; a launch takes no more
+  // chunks than fill the kernel's resident slots once
+  static int slots[2][2] = {};  // [bf16][vec]
+  auto fit = [&](auto kernel) {
+    int& sl = slots[q_bf16 ? 1 : 0][vec ? 1 : 0];
+    if (sl == 0) {
+      int per_sm = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kSdThreads, 0) !=
+              cudaSuccess || per_sm < 1)
+        per_sm = 1;
+      sl = per_sm * num_sms();
+    }
+    const int c = sl / rows;
+    return c < 1 ? 1 : (c < chunks ? c : chunks);
+  };
   TimedScope ts(s, TC_ROW);
   cudaError_t e;
+  auto go = [&](auto kernel, auto x) {
+    const int c = fit(kernel);
+    int chunk = (V + c - 1) / c;
+    chunk = (chunk + 63) / 64 * 64;
+    return launch_pdl(kernel, dim3(c, rows), dim3(kSdThreads), 0, s, 1, x, lm_rows, req_valid, B,
+                      V, step, inv_tau, chunk, c, p, cnt, tok, conf, seed, offset);
+  };
   if (q_bf16) {
     const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(q);
-    auto k = vec ? sd_draw_kernel<__nv_bfloat16, true> : sd_draw_kernel<__nv_bfloat16, false>;
-    e = launch_pdl(k, grid, block, 0, s, 1, x, lm_rows, req_valid, B, V, step, inv_tau, chunk,
-                   chunks, p, cnt, tok, conf, seed, offset);
+    e = go(vec ? sd_draw_kernel<__nv_bfloat16, true> : sd_draw_kernel<__nv_bfloat16, false>, x);
   } else {
     const float* x = static_cast<const float*>(q);
-    auto k = vec ? sd_draw_kernel<float, true> : sd_draw_kernel<float, false>;
-    e = launch_pdl(k, grid, block, 0, s, 1, x, lm_rows, req_valid, B, V, step, inv_tau, chunk,
-                   chunks, p, cnt, tok, conf, seed, offset);
+    e = go(vec ? sd_draw_kernel<float, true> : sd_draw_kernel<float, false>, x);
   }
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }

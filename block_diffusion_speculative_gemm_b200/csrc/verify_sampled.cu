@@ -55,9 +55,9 @@ struct SvPart {  // per (tensor row, chunk): max and sum of 2^(x c - max), c = l
 
 struct SvRec {  // per request, written by the stats kernel for the draw kernel
   int a, mode;
-  float mt, lst;  // target row a: max and log of the sum, natural units (x / tau)
-  float md, lsd;  // draft row a+1 (residual mode)
-  int pad[2];
+  float offp;  // target row a: log2 p_a(v) = z_v c + offp, c = log2 e / tau
+  float offq;  // draft row a+1 (residual mode): log2 q_{a+1}(v) = y_v c + offq
+  int pad[4];
 };
 
 struct SvDraw {  // per (request, chunk): best residual and best target-only draw
@@ -96,13 +96,13 @@ __device__ __forceinline__ void stat_add16(const uint4& u, float c, float& m, fl
   }
   if (m == -INFINITY) return;  // nothing finite yet: every x is -inf
 #pragma unroll
-  for (int k = 0; k < W; ++k) s += exp2f(x[k] - m);
+  for (int k = 0; k < W; ++k) s += ex2_ftz(x[k] - m);
 }
 
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kSvThreads)
     sv_stats_kernel(const T* __restrict__ target, const T* __restrict__ drafted, int rows, int B,
-                    int V, float c2, float inv_tau, int chunk, int chunks, SvPart* __restrict__ part,
+                    int V, float c2, int chunk, int chunks, SvPart* __restrict__ part,
                     unsigned* __restrict__ cnt, const int32_t* __restrict__ draft,
                     const int32_t* __restrict__ out_len, int out_cap, uint64_t seed,
                     uint64_t offset, SvRec* __restrict__ rec, int32_t* err) {
@@ -123,12 +123,12 @@ __global__ void __launch_bounds__(kSvThreads)
       const int nvec = max(0, v1 - v0) / W;
       const uint4* p = reinterpret_cast<const uint4*>(x + v0);
       int t = threadIdx.x;
-      for (; t + 3 * kSvThreads < nvec; t += 4 * kSvThreads) {
-        uint4 u[4];
+      for (; t + 7 * kSvThreads < nvec; t += 8 * kSvThreads) {  // 128 bytes in flight
+        uint4 u[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) u[j] = __ldcs(p + t + j * kSvThreads);
+        for (int j = 0; j < 8; ++j) u[j] = __ldcs(p + t + j * kSvThreads);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) stat_add16<T>(u[j], c2, m, s);
+        for (int j = 0; j < 8; ++j) stat_add16<T>(u[j], c2, m, s);
       }
       for (; t < nvec; t += kSvThreads) stat_add16<T>(__ldcs(p + t), c2, m, s);
       for (int v = v0 + nvec * W + threadIdx.x; v < v1; v += kSvThreads)
@@ -209,11 +209,9 @@ __global__ void __launch_bounds__(kSvThreads)
     SvRec q;
     q.a = a;
     q.mode = mode;
-    q.mt = st.m * kLn2;
-    q.lst = logf(st.s);
-    q.md = md_next * kLn2;
-    q.lsd = mode == SV_RESIDUAL ? logf(sd_next) : 0.f;
-    q.pad[0] = q.pad[1] = 0;
+    q.offp = -(st.m + log2f(st.s));
+    q.offq = mode == SV_RESIDUAL ? -(md_next + log2f(sd_next)) : 0.f;
+    q.pad[0] = q.pad[1] = q.pad[2] = q.pad[3] = 0;
     rec[r] = q;
   }
   if (lane == 0) cnt[r] = 0;  // ready for the draw kernel and the next call
@@ -248,9 +246,9 @@ __device__ __forceinline__ void load4(const T* p, bool vec, float (&x)[4], int n
 }
 
 template <typename T, bool VEC>
-__global__ void __launch_bounds__(kSvThreads)
+__global__ void __launch_bounds__(kSvThreads, 4)
     sv_draw_kernel(const T* __restrict__ target, const T* __restrict__ drafted, int B, int V,
-                   float inv_tau, int chunk, int chunks, const SvRec* __restrict__ rec,
+                   float c2, int chunk, int chunks, const SvRec* __restrict__ rec,
                    SvDraw* __restrict__ part, unsigned* __restrict__ cnt,
                    const int32_t* __restrict__ draft, int32_t* out_tokens, int32_t* out_len,
                    int out_cap, int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
@@ -261,12 +259,15 @@ __global__ void __launch_bounds__(kSvThreads)
   __shared__ int s_last;
   const int r = blockIdx.y, c = blockIdx.x;
   const SvRec q = rec[r];
+  // scores in log2 units: log2 w_v + G_v log2 e, the natural-unit score times
+  // log2 e, so the argmax is the same
   float sr = -INFINITY, sp = -INFINITY;
   int ir = 0x7fffffff, ip = 0x7fffffff;
   if (q.mode != SV_SKIP) {
     const bool residual = q.mode == SV_RESIDUAL;
     const T* zr = target + ((size_t)r * B + q.a) * V;
     const T* yr = residual ? drafted + ((size_t)r * B + q.a + 1) * V : zr;  // draft row a+1
+    const float dq = q.offq - q.offp;  // log2 q - log2 p = (y - z) c + dq
     const int v0 = c * chunk, v1 = min(V, v0 + chunk);  // chunk is a multiple of 4
     // groups of 4 consecutive entries share one Philox block; each thread
     // visits its groups in increasing order, so '>' keeps the lowest index
@@ -280,14 +281,14 @@ __global__ void __launch_bounds__(kSvThreads)
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         if (k >= n) break;
-        const float gum = gumbel_of(wds[k]);
-        const float lp = z[k] * inv_tau - q.mt - q.lst;
+        const float gum = gumbel2_of(wds[k]);
+        const float lp = fmaf(z[k], c2, q.offp);
         const float scp = lp + gum;
         if (scp > sp) { sp = scp; ip = vb + k; }
         if (residual) {
-          const float lq = yv[k] * inv_tau - q.md - q.lsd;
-          if (lp > lq) {
-            const float scr = lp + logf(-expm1f(lq - lp)) + gum;
+          const float d = fmaf(yv[k] - z[k], c2, dq);
+          if (d < 0.f) {
+            const float scr = lp + log2_one_minus_exp2(d) + gum;
             if (scr > sr) { sr = scr; ir = vb + k; }
           }
         }
@@ -344,11 +345,31 @@ __global__ void __launch_bounds__(kSvThreads)
   if (lane == 0) cnt[r] = 0;
 }
 
-int sv_chunks(int rows, int V, int min_chunk) {
-  int target = (4 * 148 + rows - 1) / rows;
+// Chunks per row.  The workspace is sized for the most a B200 can hold at
+// once (8 CTAs of 256 threads on each of 148 SMs); a launch takes as many
+// chunks as fill the resident slots of its kernel once (`slots`, from the
+// occupancy calculator), so that no CTA starts in a second wave.
+int sv_chunks_max(int rows, int V, int min_chunk) {
+  int target = (8 * 148 + rows - 1) / rows;
   int max_c = (V + min_chunk - 1) / min_chunk;
   int c = target < max_c ? target : max_c;
   return c < 1 ? 1 : c;
+}
+
+int sv_chunks(int rows, int V, int min_chunk, int slots) {
+  int c = slots / rows;
+  const int cap = sv_chunks_max(rows, V, min_chunk);
+  if (c > cap) c = cap;
+  return c < 1 ? 1 : c;
+}
+
+template <typename K>
+int resident_slots(K kernel) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kSvThreads, 0) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  return per_sm * num_sms();
 }
 
 int chunk_len(int V, int chunks) {
@@ -356,10 +377,25 @@ int chunk_len(int V, int chunks) {
   return (chunk + 63) / 64 * 64;
 }
 
+__global__ void sample_math_kernel(const uint64_t* __restrict__ w, const float* __restrict__ d,
+                                   int n, float* __restrict__ g2, float* __restrict__ l2) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  g2[i] = gumbel2_of(w[i]);
+  l2[i] = log2_one_minus_exp2(d[i]);
+}
+
 }  // namespace
 
+int launch_sample_math(const uint64_t* w, const float* d, int n, float* g2, float* l2,
+                       cudaStream_t s) {
+  if (n <= 0) return DFLASH_OK;
+  sample_math_kernel<<<(n + 255) / 256, 256, 0, s>>>(w, d, n, g2, l2);
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
+}
+
 size_t sampled_verify_bytes(int batch, int B, int V) {
-  const int c1 = sv_chunks(2 * batch * B, V, 4096), c2 = sv_chunks(batch, V, 2048);
+  const int c1 = sv_chunks_max(2 * batch * B, V, 4096), c2 = sv_chunks_max(batch, V, 2048);
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   return al((size_t)2 * batch * B * c1 * sizeof(SvPart)) + al((size_t)batch * sizeof(SvRec)) +
          al((size_t)batch * c2 * sizeof(SvDraw));
@@ -371,30 +407,36 @@ int launch_sampled_verify(const void* target, const void* drafted, int dtype, co
                           int32_t* accept_len, int32_t* next_anchor, void* scratch,
                           unsigned* cnt, int32_t* err, cudaStream_t s) {
   const int rows = batch * B;
-  const int c1 = sv_chunks(2 * rows, V, 4096), c2 = sv_chunks(batch, V, 2048);
-  const int k1 = chunk_len(V, c1), k2 = chunk_len(V, c2);
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   uint8_t* base = static_cast<uint8_t*>(scratch);
   SvPart* part1 = reinterpret_cast<SvPart*>(base);
-  SvRec* rec = reinterpret_cast<SvRec*>(base + al((size_t)2 * rows * c1 * sizeof(SvPart)));
+  SvRec* rec = reinterpret_cast<SvRec*>(
+      base + al((size_t)2 * rows * sv_chunks_max(2 * rows, V, 4096) * sizeof(SvPart)));
   SvDraw* part2 = reinterpret_cast<SvDraw*>(reinterpret_cast<uint8_t*>(rec) +
                                             al((size_t)batch * sizeof(SvRec)));
   const int esz = dtype == DFLASH_BF16 ? 2 : 4;
   const bool vec = ((size_t)V * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(target) % 16) == 0 &&
                    (reinterpret_cast<uintptr_t>(drafted) % 16) == 0;
-  const float inv_tau = 1.f / tau, c2f = kLog2e / tau;
+  const float c2f = kLog2e / tau;
   TimedScope ts(s, TC_VERIFY);
   cudaError_t e;
-  const dim3 g1(c1, 2 * rows), g2(c2, batch), blk(kSvThreads);
+  const dim3 blk(kSvThreads);
   if (dtype == DFLASH_BF16) {
     const __nv_bfloat16* zt = static_cast<const __nv_bfloat16*>(target);
     const __nv_bfloat16* yd = static_cast<const __nv_bfloat16*>(drafted);
     auto ka = vec ? sv_stats_kernel<__nv_bfloat16, true> : sv_stats_kernel<__nv_bfloat16, false>;
     auto kb = vec ? sv_draw_kernel<__nv_bfloat16, true> : sv_draw_kernel<__nv_bfloat16, false>;
-    e = launch_pdl(ka, g1, blk, 0, s, 1, zt, yd, rows, B, V, c2f, inv_tau, k1, c1, part1, cnt,
+    static int slots[2][2] = {};  // [vec][kernel]
+    if (slots[vec][0] == 0) slots[vec][0] = resident_slots(ka);
+    if (slots[vec][1] == 0) slots[vec][1] = resident_slots(kb);
+    const int c1 = sv_chunks(2 * rows, V, 4096, slots[vec][0]);
+    const int c2 = sv_chunks(batch, V, 2048, slots[vec][1]);
+    const int k1 = chunk_len(V, c1), k2 = chunk_len(V, c2);
+    const dim3 g1(c1, 2 * rows), g2(c2, batch);
+    e = launch_pdl(ka, g1, blk, 0, s, 1, zt, yd, rows, B, V, c2f, k1, c1, part1, cnt,
                    draft, (const int32_t*)out_len, out_cap, seed, offset, rec, err);
     if (e == cudaSuccess)
-      e = launch_pdl(kb, g2, blk, 0, s, 1, zt, yd, B, V, inv_tau, k2, c2, (const SvRec*)rec, part2,
+      e = launch_pdl(kb, g2, blk, 0, s, 1, zt, yd, B, V, c2f, k2, c2, (const SvRec*)rec, part2,
                      cnt, draft, out_tokens, out_len, out_cap, seq_lens, accept_len, next_anchor,
                      seed, offset);
   } else {
@@ -402,10 +444,17 @@ int launch_sampled_verify(const void* target, const void* drafted, int dtype, co
     const float* yd = static_cast<const float*>(drafted);
     auto ka = vec ? sv_stats_kernel<float, true> : sv_stats_kernel<float, false>;
     auto kb = vec ? sv_draw_kernel<float, true> : sv_draw_kernel<float, false>;
-    e = launch_pdl(ka, g1, blk, 0, s, 1, zt, yd, rows, B, V, c2f, inv_tau, k1, c1, part1, cnt,
+    static int slots[2][2] = {};  // [vec][kernel]
+    if (slots[vec][0] == 0) slots[vec][0] = resident_slots(ka);
+    if (slots[vec][1] == 0) slots[vec][1] = resident_slots(kb);
+    const int c1 = sv_chunks(2 * rows, V, 4096, slots[vec][0]);
+    const int c2 = sv_chunks(batch, V, 2048, slots[vec][1]);
+    const int k1 = chunk_len(V, c1), k2 = chunk_len(V, c2);
+    const dim3 g1(c1, 2 * rows), g2(c2, batch);
+    e = launch_pdl(ka, g1, blk, 0, s, 1, zt, yd, rows, B, V, c2f, k1, c1, part1, cnt,
                    draft, (const int32_t*)out_len, out_cap, seed, offset, rec, err);
     if (e == cudaSuccess)
-      e = launch_pdl(kb, g2, blk, 0, s, 1, zt, yd, B, V, inv_tau, k2, c2, (const SvRec*)rec, part2,
+      e = launch_pdl(kb, g2, blk, 0, s, 1, zt, yd, B, V, c2f, k2, c2, (const SvRec*)rec, part2,
                      cnt, draft, out_tokens, out_len, out_cap, seq_lens, accept_len, next_anchor,
                      seed, offset);
   }

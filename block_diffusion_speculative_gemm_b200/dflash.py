@@ -128,6 +128,7 @@ def lib() -> ctypes.CDLL:
         L.dflash_debug_pick_splits.argtypes = [i32, i32, i32]
         L.dflash_debug_wait_timeout.argtypes = [vp, vp]
         L.dflash_debug_split_weight.argtypes = [ctypes.c_float]
+        L.dflash_debug_sample_math.argtypes = [vp, vp, i32, vp, vp, vp]
         _lib = L
     return _lib
 
@@ -682,6 +683,20 @@ def debug_attn_schedule(sched: int) -> None:
     """Process-wide draft attention schedule: 0 the split-KV grid of fixed
     chunks (default), 1 persistent (tests and tuning)."""
     _check("dflash_debug_attn_schedule", lib().dflash_debug_attn_schedule(int(sched)))
+
+
+def debug_sample_math(w: torch.Tensor, d: torch.Tensor):
+    """Per-entry sampling arithmetic of the draw kernels (tests): returns
+    (g2, l2), the log2-unit Gumbel variate of each Philox word in `w`
+    (int64 holding the uint64 bits) and log2(1 - 2^d) for each d < 0."""
+    assert w.is_cuda and d.is_cuda and w.dtype == torch.int64 and d.dtype == torch.float32
+    assert w.is_contiguous() and d.is_contiguous() and w.numel() == d.numel()
+    n = w.numel()
+    g2 = torch.empty(n, dtype=torch.float32, device=w.device)
+    l2 = torch.empty_like(g2)
+    _check("dflash_debug_sample_math",
+           lib().dflash_debug_sample_math(_ptr(w), _ptr(d), n, _ptr(g2), _ptr(l2), _stream(None)))
+    return g2, l2
 
 
 def debug_attn_chunk(keys: int) -> None:

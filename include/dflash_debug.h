@@ -111,6 +111,16 @@ int dflash_debug_attn_schedule(int sched);
  * value or one that is not a multiple of 64.  Not thread-safe; tests only. */
 int dflash_debug_attn_chunk(int keys);
 
+/* The per-entry sampling arithmetic of the draw kernels, element by element,
+ * for accuracy tests.  For i < n: g2[i] = the Gumbel variate of Philox output
+ * word w[i] in log2 units, -log2(-ln U') with U' = ((w[i] >> 11) + 1/2) 2^-53;
+ * l2[i] = log2(1 - 2^d[i]) for d[i] < 0 (the log2 residual weight of a draw
+ * from max(0, p - q) relative to p, with d = log2 q - log2 p).  w, d, g2, l2
+ * are device arrays of n entries; the call is asynchronous on `stream`.
+ * DFLASH_EINVAL for n < 0 or a null array when n > 0. */
+int dflash_debug_sample_math(const uint64_t* w, const float* d, int n, float* g2, float* l2,
+                             void* stream);
+
 #ifdef __cplusplus
 }
 #endif
