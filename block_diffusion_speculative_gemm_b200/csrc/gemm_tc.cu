@@ -683,25 +683,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else {
             load_chunk(c, v);
           }
-          if (a.out.dbg != nullptr && n < a.N) {
-#pragma unroll
-            for (int jj = 0; jj < 32; ++jj) {
-              const int m = w.m0 + c * 32 + jj;
-              if (m >= a.M) continue;
-              const int64_t d = a.out.dbg_rows ? (int64_t)a.out.dbg_rows[m] : (int64_t)m;
-              if (a.out.dbg_valid && !a.out.dbg_valid[d / a.out.B]) continue;
-              if (a.out.dbg_bf16)
-                static_cast<__nv_bfloat16*>(a.out.dbg)[d * a.out.dbg_ld + n] =
-                    __float2bfloat16_rn(v[jj]);
-              else
-                static_cast<float*>(a.out.dbg)[d * a.out.dbg_ld + n] = v[jj];
-            }
-          }
           // transpose through shared memory: lane jj then owns token column jj
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) tr[jj * 33 + lane] = (n < a.N) ? v[jj] : -INFINITY;
           __syncwarp();
           const float* col = tr + lane * 33;
+          if (a.out.dbg != nullptr) {
+            // the logits rows: this lane's token, 32 consecutive vocabulary
+            // entries (64 or 128 contiguous bytes), one row lookup per lane
+            const int m = w.m0 + c * 32 + lane;
+            const int n0 = w.n0 + q * 32;
+            if (m < a.M) {
+              const int64_t d = a.out.dbg_rows ? (int64_t)a.out.dbg_rows[m] : (int64_t)m;
+              if (!a.out.dbg_valid || a.out.dbg_valid[d / a.out.B]) {
+                const int nv = min(32, a.N - n0);
+                if (a.out.dbg_bf16) {
+                  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.out.dbg) + d * a.out.dbg_ld + n0;
+                  if (nv == 32 && (reinterpret_cast<uintptr_t>(o) & 15) == 0) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                      uint4 u;
+                      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+                      for (int k = 0; k < 4; ++k)
+                        h[k] = __floats2bfloat162_rn(col[i + 2 * k], col[i + 2 * k + 1]);
+                      *reinterpret_cast<uint4*>(o + i) = u;
+                    }
+                  } else {
+                    for (int i = 0; i < nv; ++i) o[i] = __float2bfloat16_rn(col[i]);
+                  }
+                } else {
+                  float* o = static_cast<float*>(a.out.dbg) + d * a.out.dbg_ld + n0;
+                  if (nv == 32 && (reinterpret_cast<uintptr_t>(o) & 15) == 0) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                      *reinterpret_cast<float4*>(o + i) =
+                          make_float4(col[i], col[i + 1], col[i + 2], col[i + 3]);
+                  } else {
+                    for (int i = 0; i < nv; ++i) o[i] = col[i];
+                  }
+                }
+              }
+            }
+          }
           float mx = col[0];
           int bi = 0;
 #pragma unroll 8

@@ -83,11 +83,14 @@ __device__ void verify_accept(const ArgPart* part, int64_t row_stride, int64_t c
   }
 }
 
+// logits and draft are plain pointers: the L2 prefetch runs before the
+// dependency wait, and a const __restrict__ pointer would let the compiler
+// move a load of another kernel's output above that wait.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kVerifyThreads)
-    verify_kernel(const T* __restrict__ logits, int V, int chunk, int chunks,
-                  ArgPart* __restrict__ part, unsigned* __restrict__ cnt,
-                  const int32_t* __restrict__ draft, int B, int32_t* out_tokens, int32_t* out_len,
+    verify_kernel(const T* logits, int V, int chunk, int chunks, ArgPart* __restrict__ part,
+                  unsigned* __restrict__ cnt, const int32_t* draft, int B, int32_t* out_tokens,
+                  int32_t* out_len,
                   int out_cap, int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
                   int32_t* err, ArgPart* shard_out, int vocab_offset) {
   pdl_trigger();

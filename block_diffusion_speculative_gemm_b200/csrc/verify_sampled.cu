@@ -21,18 +21,21 @@
 // U_i (n = i), stream 1 gives U'_v (n = v).  A word w gives
 // U = (w >> 11) 2^-53 in [0, 1) and U' = ((w >> 11) + 1/2) 2^-53 in (0, 1).
 //
-// Two bandwidth-bound kernels chained by programmatic dependent launch:
+// Two kernels chained by programmatic dependent launch:
 //   sv_stats_kernel  one CTA per (row chunk, row) of the target and the draft
-//                    logits: (max, sum of 2^(x log2e / tau - max)) per chunk.
-//                    The last CTA of a request merges its rows (one warp,
-//                    lane i = row i), takes the accept decisions in the log
-//                    domain and records the accept length and the normalisers
-//                    of the row(s) the draw needs.
-//   sv_draw_kernel   one CTA per (vocabulary chunk, request) reads target row a
-//                    (and draft row a+1) once more, forms the Gumbel-perturbed
-//                    log-weights and keeps the best; the last CTA of a request
-//                    merges the chunks in order, writes d_1..d_a and the drawn
-//                    token behind out_len and advances the lengths.
+//                    logits, as many chunks as fill the resident slots once:
+//                    (max, sum of 2^(x log2e / tau - max)) per chunk, eight
+//                    16-byte loads in flight per thread.  The last CTA of a
+//                    request merges its rows (one warp, lane i = row i), takes
+//                    the accept decisions in the log domain and records the
+//                    accept length and the normalisers of the row(s) the draw
+//                    needs.
+//   sv_draw_kernel   one CTA per (vocabulary chunk, request), four per SM over
+//                    the batch, reads target row a (and draft row a+1) once
+//                    more, adds the Gumbel terms, keeps the best perturbed
+//                    log-weight; the last CTA of a request merges the chunks in
+//                    order, writes d_1..d_a and the drawn token behind out_len
+//                    and advances the lengths.
 // Counters count arrivals per request and are set back to zero by the CTA
 // that completes them, so the workspace stays reusable.
 #include "common.cuh"
@@ -79,64 +82,55 @@ __device__ __forceinline__ void stat_merge(float& m, float& s, float m2, float s
   m = M;
 }
 
+// The 16 bytes of u as floats: bf16 pairs widen by a shift / mask of each word.
 template <typename T>
-__device__ __forceinline__ void stat_add16(const uint4& u, float c, float& m, float& s) {
-  constexpr int W = 16 / sizeof(T);
-  const T* e = reinterpret_cast<const T*>(&u);
-  float x[W];
-  float mb = -INFINITY;
+__device__ __forceinline__ void unpack16(const uint4& u, float (&x)[16 / sizeof(T)]) {
+  if constexpr (sizeof(T) == 2) {
+    const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-  for (int k = 0; k < W; ++k) {
-    x[k] = to_f(e[k]) * c;
-    mb = fmaxf(mb, x[k]);
+    for (int k = 0; k < 4; ++k) {
+      x[2 * k] = __uint_as_float(wd[k] << 16);
+      x[2 * k + 1] = __uint_as_float(wd[k] & 0xffff0000u);
+    }
+  } else {
+    x[0] = __uint_as_float(u.x);
+    x[1] = __uint_as_float(u.y);
+    x[2] = __uint_as_float(u.z);
+    x[3] = __uint_as_float(u.w);
   }
+}
+
+// Adds the 16 bytes of u to the running (m, s0 + s1): the maximum is taken
+// on the raw values (c > 0 keeps the order) and the exponents are
+// fused multiply-adds x c - m; two partial sums halve the add chain.
+template <typename T>
+__device__ __forceinline__ void stat_add16_lean(const uint4& u, float c, float& m, float& s0,
+                                                float& s1) {
+  constexpr int W = 16 / sizeof(T);
+  float x[W];
+  unpack16<T>(u, x);
+  float mb = x[0];
+#pragma unroll
+  for (int k = 1; k < W; ++k) mb = fmaxf(mb, x[k]);
+  mb *= c;
   if (mb > m) {
-    s = (m == -INFINITY) ? 0.f : s * exp2f(m - mb);
+    const float sc = ex2_ftz(m - mb);  // 0 while m is -inf
+    s0 *= sc;
+    s1 *= sc;
     m = mb;
   }
   if (m == -INFINITY) return;  // nothing finite yet: every x is -inf
+  const float nm = -m;
 #pragma unroll
-  for (int k = 0; k < W; ++k) s += ex2_ftz(x[k] - m);
+  for (int k = 0; k < W; k += 2) {
+    s0 += ex2_ftz(fmaf(x[k], c, nm));
+    s1 += ex2_ftz(fmaf(x[k + 1], c, nm));
+  }
 }
 
-template <typename T, bool VEC>
-__global__ void __launch_bounds__(kSvThreads)
-    sv_stats_kernel(const T* __restrict__ target, const T* __restrict__ drafted, int rows, int B,
-                    int V, float c2, int chunk, int chunks, SvPart* __restrict__ part,
-                    unsigned* __restrict__ cnt, const int32_t* __restrict__ draft,
-                    const int32_t* __restrict__ out_len, int out_cap, uint64_t seed,
-                    uint64_t offset, SvRec* __restrict__ rec, int32_t* err) {
-  pdl_trigger();
-  pdl_wait();
-  __shared__ float s_m[kSvThreads / 32], s_s[kSvThreads / 32];
-  __shared__ int s_last;
-  const int y = blockIdx.y, c = blockIdx.x;
-  const bool is_draft = y >= rows;
-  const int row = is_draft ? y - rows : y;  // r * B + i
-  const int r = row / B;
-  float m = -INFINITY, s = 0.f;
-  if (!(is_draft && row % B == 0)) {  // draft row 0 (the anchor) has no distribution
-    const T* x = (is_draft ? drafted : target) + (size_t)row * V;
-    const int v0 = c * chunk, v1 = min(V, v0 + chunk);
-    if (VEC) {
-      constexpr int W = 16 / sizeof(T);
-      const int nvec = max(0, v1 - v0) / W;
-      const uint4* p = reinterpret_cast<const uint4*>(x + v0);
-      int t = threadIdx.x;
-      for (; t + 7 * kSvThreads < nvec; t += 8 * kSvThreads) {  // 128 bytes in flight
-        uint4 u[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) u[j] = __ldcs(p + t + j * kSvThreads);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) stat_add16<T>(u[j], c2, m, s);
-      }
-      for (; t < nvec; t += kSvThreads) stat_add16<T>(__ldcs(p + t), c2, m, s);
-      for (int v = v0 + nvec * W + threadIdx.x; v < v1; v += kSvThreads)
-        stat_merge(m, s, to_f(x[v]) * c2, 1.f);
-    } else {
-      for (int v = v0 + threadIdx.x; v < v1; v += kSvThreads) stat_merge(m, s, to_f(x[v]) * c2, 1.f);
-    }
-  }
+// (m, s) of the whole CTA, in warp order, returned to thread 0.  Every thread
+// of the CTA calls it; it ends with the CTA synchronised.
+__device__ __forceinline__ SvPart block_stat(float m, float s, float* s_m, float* s_s) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
@@ -149,30 +143,29 @@ __global__ void __launch_bounds__(kSvThreads)
     s_s[w] = s;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    m = s_m[0];
-    s = s_s[0];
-    for (int k = 1; k < kSvThreads / 32; ++k) stat_merge(m, s, s_m[k], s_s[k]);
-    part[(size_t)y * chunks + c] = SvPart{m, s};
-    __threadfence();  // the partial is visible before this CTA is counted
-    s_last = atomicAdd(&cnt[r], 1u) == (unsigned)(2 * B * chunks - 1);
-  }
-  __syncthreads();
-  if (!s_last || threadIdx.x >= 32) return;
-  __threadfence();  // every partial of request r counted before the reads below
+  SvPart r{s_m[0], s_s[0]};
+  if (threadIdx.x == 0)
+    for (int k = 1; k < kSvThreads / 32; ++k) stat_merge(r.m, r.s, s_m[k], s_s[k]);
+  __syncthreads();  // s_m / s_s free for the next call
+  return r;
+}
 
-  // ---- accept decisions of request r: lane i = block row i
-  auto merged = [&](int yy) {
-    const SvPart* p = part + (size_t)yy * chunks;
-    float mm = __ldcg(&p[0].m), ss = __ldcg(&p[0].s);
-    for (int k = 1; k < chunks; ++k) stat_merge(mm, ss, __ldcg(&p[k].m), __ldcg(&p[k].s));
-    return SvPart{mm, ss};
-  };
+// The accept decisions of request r, by one warp (lane i = block row i).
+// stat(y) returns the merged statistics of tensor row y: target row y for
+// y < rows, draft row y - rows otherwise.  Writes rec[r] and sets cnt[r] back
+// to zero for the draw kernel.
+template <typename T, typename StatFn>
+__device__ void sv_accept(int r, const T* __restrict__ target, const T* __restrict__ drafted,
+                          int rows, int B, int V, float c2, const int32_t* __restrict__ draft,
+                          const int32_t* __restrict__ out_len, int out_cap, uint64_t seed,
+                          uint64_t offset, SvRec* __restrict__ rec, unsigned* __restrict__ cnt,
+                          int32_t* err, StatFn stat) {
+  const int lane = threadIdx.x & 31;
   SvPart st{-INFINITY, 0.f}, sd{-INFINITY, 0.f};
   int d = 0;
   if (lane < B) {
-    st = merged(r * B + lane);
-    if (lane > 0) sd = merged(rows + r * B + lane);
+    st = stat(r * B + lane);
+    if (lane > 0) sd = stat(rows + r * B + lane);
     d = draft[(size_t)r * B + lane];
   }
   const unsigned bad = __ballot_sync(0xffffffffu, lane < B && (d < 0 || d >= V));
@@ -217,6 +210,73 @@ __global__ void __launch_bounds__(kSvThreads)
   if (lane == 0) cnt[r] = 0;  // ready for the draw kernel and the next call
 }
 
+// One thread's share of the n 16-byte units at p (units t, t + 256, ...),
+// eight loads in flight at a time.
+template <typename T>
+__device__ __forceinline__ void stat_units(const uint4* p, int n, float c, float& m, float& s) {
+  constexpr int D = 8;
+  float s0 = 0.f, s1 = 0.f;
+  m = -INFINITY;
+  int t = threadIdx.x;
+  for (; t + (D - 1) * kSvThreads < n; t += D * kSvThreads) {
+    uint4 u[D];
+#pragma unroll
+    for (int j = 0; j < D; ++j) u[j] = __ldcs(p + t + j * kSvThreads);
+#pragma unroll
+    for (int j = 0; j < D; ++j) stat_add16_lean<T>(u[j], c, m, s0, s1);
+  }
+  for (; t < n; t += kSvThreads) stat_add16_lean<T>(__ldcs(p + t), c, m, s0, s1);
+  s = s0 + s1;
+}
+
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kSvThreads)
+    sv_stats_kernel(const T* __restrict__ target, const T* __restrict__ drafted, int rows, int B,
+                    int V, float c2, int chunk, int chunks, SvPart* __restrict__ part,
+                    unsigned* __restrict__ cnt, const int32_t* __restrict__ draft,
+                    const int32_t* __restrict__ out_len, int out_cap, uint64_t seed,
+                    uint64_t offset, SvRec* __restrict__ rec, int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float s_m[kSvThreads / 32], s_s[kSvThreads / 32];
+  __shared__ int s_last;
+  const int y = blockIdx.y, c = blockIdx.x;
+  const bool is_draft = y >= rows;
+  const int row = is_draft ? y - rows : y;  // r * B + i
+  const int r = row / B;
+  float m = -INFINITY, s = 0.f;
+  if (!(is_draft && row % B == 0)) {  // draft row 0 (the anchor) has no distribution
+    const T* x = (is_draft ? drafted : target) + (size_t)row * V;
+    const int v0 = c * chunk, v1 = min(V, v0 + chunk);
+    if (VEC) {
+      constexpr int W = 16 / sizeof(T);
+      const int nvec = max(0, v1 - v0) / W;  // v0 is a multiple of 64: 16-byte aligned
+      stat_units<T>(reinterpret_cast<const uint4*>(x + v0), nvec, c2, m, s);
+      for (int v = v0 + nvec * W + threadIdx.x; v < v1; v += kSvThreads)
+        stat_merge(m, s, to_f(x[v]) * c2, 1.f);
+    } else {
+      for (int v = v0 + threadIdx.x; v < v1; v += kSvThreads) stat_merge(m, s, to_f(x[v]) * c2, 1.f);
+    }
+  }
+  const SvPart b = block_stat(m, s, s_m, s_s);
+  if (threadIdx.x == 0) {
+    part[(size_t)y * chunks + c] = b;
+    __threadfence();  // the partial is visible before this CTA is counted
+    s_last = atomicAdd(&cnt[r], 1u) == (unsigned)(2 * B * chunks - 1);
+  }
+  __syncthreads();
+  if (!s_last || threadIdx.x >= 32) return;
+  __threadfence();  // every partial of request r counted before the reads below
+  auto merged = [&](int yy) {
+    const SvPart* p = part + (size_t)yy * chunks;
+    float mm = __ldcg(&p[0].m), ss = __ldcg(&p[0].s);
+    for (int k = 1; k < chunks; ++k) stat_merge(mm, ss, __ldcg(&p[k].m), __ldcg(&p[k].s));
+    return SvPart{mm, ss};
+  };
+  sv_accept<T>(r, target, drafted, rows, B, V, c2, draft, out_len, out_cap, seed, offset, rec, cnt,
+               err, merged);
+}
+
 __device__ __forceinline__ void draw_merge(float& s, int& i, float s2, int i2) {
   if (s2 > s || (s2 == s && i2 < i)) {
     s = s2;
@@ -245,18 +305,19 @@ __device__ __forceinline__ void load4(const T* p, bool vec, float (&x)[4], int n
   for (int k = 0; k < 4; ++k) x[k] = k < n ? to_f(p[k]) : 0.f;
 }
 
+// The inputs another kernel writes (the logits, the draft tokens and the
+// stats pass's records) are read through plain pointers.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kSvThreads, 4)
-    sv_draw_kernel(const T* __restrict__ target, const T* __restrict__ drafted, int B, int V,
-                   float c2, int chunk, int chunks, const SvRec* __restrict__ rec,
-                   SvDraw* __restrict__ part, unsigned* __restrict__ cnt,
-                   const int32_t* __restrict__ draft, int32_t* out_tokens, int32_t* out_len,
-                   int out_cap, int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor,
-                   uint64_t seed, uint64_t offset) {
-  pdl_trigger();
-  pdl_wait();
+    sv_draw_kernel(const T* target, const T* drafted, int B, int V, float c2, int chunk,
+                   int chunks, const SvRec* rec, SvDraw* part, unsigned* cnt,
+                   const int32_t* draft, int32_t* out_tokens, int32_t* out_len, int out_cap,
+                   int32_t* seq_lens, int32_t* accept_len, int32_t* next_anchor, uint64_t seed,
+                   uint64_t offset) {
   __shared__ SvDraw s_d[kSvThreads / 32];
   __shared__ int s_last;
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.y, c = blockIdx.x;
   const SvRec q = rec[r];
   // scores in log2 units: log2 w_v + G_v log2 e, the natural-unit score times
@@ -268,27 +329,28 @@ __global__ void __launch_bounds__(kSvThreads, 4)
     const T* zr = target + ((size_t)r * B + q.a) * V;
     const T* yr = residual ? drafted + ((size_t)r * B + q.a + 1) * V : zr;  // draft row a+1
     const float dq = q.offq - q.offp;  // log2 q - log2 p = (y - z) c + dq
-    const int v0 = c * chunk, v1 = min(V, v0 + chunk);  // chunk is a multiple of 4
-    // groups of 4 consecutive entries share one Philox block; each thread
-    // visits its groups in increasing order, so '>' keeps the lowest index
+    const int v0 = c * chunk, v1 = min(V, v0 + chunk);  // chunk is a multiple of 64
+    // groups of 4 consecutive entries; each thread visits its groups in
+    // increasing order, so '>' keeps the lowest index
     for (int g = v0 / 4 + threadIdx.x; g * 4 < v1; g += kSvThreads) {
       const int vb = g * 4, n = min(4, v1 - vb);
-      float z[4], yv[4];
+      float z[4], yv[4], gum[4];
       load4<T>(zr + vb, VEC, z, n);
       if (residual) load4<T>(yr + vb, VEC, yv, n);
       uint64_t wds[4];
       philox_block(seed, offset, r, 1, (uint64_t)g, wds);
 #pragma unroll
+      for (int k = 0; k < 4; ++k) gum[k] = gumbel2_of(wds[k]);
+#pragma unroll
       for (int k = 0; k < 4; ++k) {
         if (k >= n) break;
-        const float gum = gumbel2_of(wds[k]);
         const float lp = fmaf(z[k], c2, q.offp);
-        const float scp = lp + gum;
+        const float scp = lp + gum[k];
         if (scp > sp) { sp = scp; ip = vb + k; }
         if (residual) {
           const float d = fmaf(yv[k] - z[k], c2, dq);
           if (d < 0.f) {
-            const float scr = lp + log2_one_minus_exp2(d) + gum;
+            const float scr = lp + log2_one_minus_exp2(d) + gum[k];
             if (scr > sr) { sr = scr; ir = vb + k; }
           }
         }
@@ -345,10 +407,11 @@ __global__ void __launch_bounds__(kSvThreads, 4)
   if (lane == 0) cnt[r] = 0;
 }
 
-// Chunks per row.  The workspace is sized for the most a B200 can hold at
-// once (8 CTAs of 256 threads on each of 148 SMs); a launch takes as many
-// chunks as fill the resident slots of its kernel once (`slots`, from the
-// occupancy calculator), so that no CTA starts in a second wave.
+// Chunks per row of the gridded stats pass (rows that are not 16-byte
+// aligned).  The workspace is sized for the most a B200 can hold at once
+// (8 CTAs of 256 threads on each of 148 SMs); a launch takes as many chunks as
+// fill the resident slots of its kernel once (`slots`), so that no CTA starts
+// in a second wave.
 int sv_chunks_max(int rows, int V, int min_chunk) {
   int target = (8 * 148 + rows - 1) / rows;
   int max_c = (V + min_chunk - 1) / min_chunk;
@@ -364,9 +427,10 @@ int sv_chunks(int rows, int V, int min_chunk, int slots) {
 }
 
 template <typename K>
-int resident_slots(K kernel) {
+int resident_slots(K kernel, size_t smem = 0) {
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kSvThreads, 0) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kSvThreads, smem) !=
+          cudaSuccess ||
       per_sm < 1)
     per_sm = 1;
   return per_sm * num_sms();
@@ -375,6 +439,16 @@ int resident_slots(K kernel) {
 int chunk_len(int V, int chunks) {
   int chunk = (V + chunks - 1) / chunks;
   return (chunk + 63) / 64 * 64;
+}
+
+// Draw chunks per request: four CTAs per SM over the batch, chunks of at
+// least 2048 entries (at most ceil(V / 2048) chunks, the workspace bound).
+int sv_draw_chunks_max(int V) { return (V + 2047) / 2048; }
+
+int sv_draw_chunks(int batch, int V) {
+  int q = 4 * num_sms() / (batch > 0 ? batch : 1);
+  if (q > sv_draw_chunks_max(V)) q = sv_draw_chunks_max(V);
+  return q < 1 ? 1 : q;
 }
 
 __global__ void sample_math_kernel(const uint64_t* __restrict__ w, const float* __restrict__ d,
@@ -394,12 +468,27 @@ int launch_sample_math(const uint64_t* w, const float* d, int n, float* g2, floa
   return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 
-size_t sampled_verify_bytes(int batch, int B, int V) {
-  const int c1 = sv_chunks_max(2 * batch * B, V, 4096), c2 = sv_chunks_max(batch, V, 2048);
+namespace {
+
+struct SvLayout {
+  size_t part1, rec, part2, total;
+};
+
+SvLayout sv_layout(int batch, int B, int V) {
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
-  return al((size_t)2 * batch * B * c1 * sizeof(SvPart)) + al((size_t)batch * sizeof(SvRec)) +
-         al((size_t)batch * c2 * sizeof(SvDraw));
+  const int rows = batch * B;
+  const size_t p1 = (size_t)2 * rows * sv_chunks_max(2 * rows, V, 4096);
+  SvLayout L;
+  L.part1 = 0;
+  L.rec = al(p1 * sizeof(SvPart));
+  L.part2 = L.rec + al((size_t)batch * sizeof(SvRec));
+  L.total = L.part2 + al((size_t)batch * sv_draw_chunks_max(V) * sizeof(SvDraw));
+  return L;
 }
+
+}  // namespace
+
+size_t sampled_verify_bytes(int batch, int B, int V) { return sv_layout(batch, B, V).total; }
 
 int launch_sampled_verify(const void* target, const void* drafted, int dtype, const int32_t* draft,
                           int batch, int B, int V, float tau, uint64_t seed, uint64_t offset,
@@ -407,57 +496,35 @@ int launch_sampled_verify(const void* target, const void* drafted, int dtype, co
                           int32_t* accept_len, int32_t* next_anchor, void* scratch,
                           unsigned* cnt, int32_t* err, cudaStream_t s) {
   const int rows = batch * B;
-  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const SvLayout L = sv_layout(batch, B, V);
   uint8_t* base = static_cast<uint8_t*>(scratch);
-  SvPart* part1 = reinterpret_cast<SvPart*>(base);
-  SvRec* rec = reinterpret_cast<SvRec*>(
-      base + al((size_t)2 * rows * sv_chunks_max(2 * rows, V, 4096) * sizeof(SvPart)));
-  SvDraw* part2 = reinterpret_cast<SvDraw*>(reinterpret_cast<uint8_t*>(rec) +
-                                            al((size_t)batch * sizeof(SvRec)));
+  SvPart* part1 = reinterpret_cast<SvPart*>(base + L.part1);
+  SvRec* rec = reinterpret_cast<SvRec*>(base + L.rec);
+  SvDraw* part2 = reinterpret_cast<SvDraw*>(base + L.part2);
   const int esz = dtype == DFLASH_BF16 ? 2 : 4;
   const bool vec = ((size_t)V * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(target) % 16) == 0 &&
                    (reinterpret_cast<uintptr_t>(drafted) % 16) == 0;
   const float c2f = kLog2e / tau;
+  const int q = sv_draw_chunks(batch, V), kq = chunk_len(V, q);
   TimedScope ts(s, TC_VERIFY);
-  cudaError_t e;
-  const dim3 blk(kSvThreads);
-  if (dtype == DFLASH_BF16) {
-    const __nv_bfloat16* zt = static_cast<const __nv_bfloat16*>(target);
-    const __nv_bfloat16* yd = static_cast<const __nv_bfloat16*>(drafted);
-    auto ka = vec ? sv_stats_kernel<__nv_bfloat16, true> : sv_stats_kernel<__nv_bfloat16, false>;
-    auto kb = vec ? sv_draw_kernel<__nv_bfloat16, true> : sv_draw_kernel<__nv_bfloat16, false>;
-    static int slots[2][2] = {};  // [vec][kernel]
-    if (slots[vec][0] == 0) slots[vec][0] = resident_slots(ka);
-    if (slots[vec][1] == 0) slots[vec][1] = resident_slots(kb);
-    const int c1 = sv_chunks(2 * rows, V, 4096, slots[vec][0]);
-    const int c2 = sv_chunks(batch, V, 2048, slots[vec][1]);
-    const int k1 = chunk_len(V, c1), k2 = chunk_len(V, c2);
-    const dim3 g1(c1, 2 * rows), g2(c2, batch);
-    e = launch_pdl(ka, g1, blk, 0, s, 1, zt, yd, rows, B, V, c2f, k1, c1, part1, cnt,
-                   draft, (const int32_t*)out_len, out_cap, seed, offset, rec, err);
-    if (e == cudaSuccess)
-      e = launch_pdl(kb, g2, blk, 0, s, 1, zt, yd, B, V, c2f, k2, c2, (const SvRec*)rec, part2,
-                     cnt, draft, out_tokens, out_len, out_cap, seq_lens, accept_len, next_anchor,
-                     seed, offset);
-  } else {
-    const float* zt = static_cast<const float*>(target);
-    const float* yd = static_cast<const float*>(drafted);
-    auto ka = vec ? sv_stats_kernel<float, true> : sv_stats_kernel<float, false>;
-    auto kb = vec ? sv_draw_kernel<float, true> : sv_draw_kernel<float, false>;
-    static int slots[2][2] = {};  // [vec][kernel]
-    if (slots[vec][0] == 0) slots[vec][0] = resident_slots(ka);
-    if (slots[vec][1] == 0) slots[vec][1] = resident_slots(kb);
-    const int c1 = sv_chunks(2 * rows, V, 4096, slots[vec][0]);
-    const int c2 = sv_chunks(batch, V, 2048, slots[vec][1]);
-    const int k1 = chunk_len(V, c1), k2 = chunk_len(V, c2);
-    const dim3 g1(c1, 2 * rows), g2(c2, batch);
-    e = launch_pdl(ka, g1, blk, 0, s, 1, zt, yd, rows, B, V, c2f, k1, c1, part1, cnt,
-                   draft, (const int32_t*)out_len, out_cap, seed, offset, rec, err);
-    if (e == cudaSuccess)
-      e = launch_pdl(kb, g2, blk, 0, s, 1, zt, yd, B, V, c2f, k2, c2, (const SvRec*)rec, part2,
-                     cnt, draft, out_tokens, out_len, out_cap, seq_lens, accept_len, next_anchor,
-                     seed, offset);
-  }
+  auto run = [&](auto tag) -> cudaError_t {
+    using T = decltype(tag);
+    const T* zt = static_cast<const T*>(target);
+    const T* yd = static_cast<const T*>(drafted);
+    auto ka = vec ? sv_stats_kernel<T, true> : sv_stats_kernel<T, false>;
+    static int slots[2] = {0, 0};  // [vec]
+    if (slots[vec] == 0) slots[vec] = resident_slots(ka);
+    const int c1 = sv_chunks(2 * rows, V, 4096, slots[vec]);
+    const cudaError_t e = launch_pdl(ka, dim3(c1, 2 * rows), dim3(kSvThreads), 0, s, 1, zt, yd,
+                                     rows, B, V, c2f, chunk_len(V, c1), c1, part1, cnt, draft,
+                                     (const int32_t*)out_len, out_cap, seed, offset, rec, err);
+    if (e != cudaSuccess) return e;
+    auto kb = vec ? sv_draw_kernel<T, true> : sv_draw_kernel<T, false>;
+    return launch_pdl(kb, dim3(q, batch), dim3(kSvThreads), 0, s, 1, zt, yd, B, V, c2f, kq, q,
+                      (const SvRec*)rec, part2, cnt, draft, out_tokens, out_len, out_cap,
+                      seq_lens, accept_len, next_anchor, seed, offset);
+  };
+  const cudaError_t e = dtype == DFLASH_BF16 ? run(__nv_bfloat16{}) : run(float{});
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 

@@ -113,6 +113,7 @@ def _case(b, B, V, label, dtype="bf16", plant=("geometric", 4.0)):
     (3, 16, 4099, "f32"),
     (64, 2, 3000, "bf16"),
     (2, 32, 777, "bf16"),      # a full warp of rows
+    (300, 4, 2048, "bf16"),    # balanced stats CTAs span several rows and requests
 ])
 @pytest.mark.parametrize("tau", [0.3, 1.0, 2.5])
 def test_sampled_verify_matches_oracle(b, B, V, dtype, tau):
