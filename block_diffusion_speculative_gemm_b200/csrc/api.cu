@@ -1458,8 +1458,9 @@ extern "C" int dflash_debug_split_weight(float w) {
 }
 
 extern "C" int dflash_debug_attn_schedule(int sched) {
-  if (sched < 0 || sched > 1) return DFLASH_EINVAL;
-  g_attn_sched = sched;
+  if (sched < 0 || sched > 2) return DFLASH_EINVAL;
+  g_attn_sched = sched == 1 ? 1 : 0;
+  g_attn_umma = sched == 2 ? 1 : 0;
   return DFLASH_OK;
 }
 

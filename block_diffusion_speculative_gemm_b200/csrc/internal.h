@@ -248,6 +248,19 @@ constexpr int kAttnMaxRows = 64;  // B * (n_q / n_kv) query rows per (request, k
 // split-KV grid of `chunk`-key chunks.
 int launch_attn_plan(const int32_t* ctx_len, const int32_t* req_valid, int batch, int nkv,
                      int32_t* seg_start, cudaStream_t s);
+// The tcgen05 attention kernel (head dim 128, at most 32 query rows per kv
+// head, contiguous K/V, the grid schedule): used by launch_attn_tc while
+// g_attn_umma is set (dflash_debug_attn_schedule(2)); tk/tv are tensor maps of
+// kUmmaKeys-row boxes.
+// DFLASH_EUNSUPPORTED outside its shapes.
+extern int g_attn_umma;
+constexpr int kUmmaKeys = 48;  // keys per context tile of the tcgen05 kernel (TMA box rows)
+int launch_attn_umma(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q,
+                     const __half* kb, const __half* vb, const KvPages& pg, long long kv_rows,
+                     int layer, int batch, int cap, const int32_t* ctx_len,
+                     const int32_t* req_valid, int B, int nq, int nkv, int chunk, int n_chunks,
+                     float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
+                     cudaStream_t s);
 int launch_attn_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
                    const __half* vc, const KvPages& pages, int layer, int batch, int cap,
                    const int32_t* ctx_len, const int32_t* req_valid, int B, int nq, int nkv,

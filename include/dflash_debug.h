@@ -97,11 +97,14 @@ int dflash_debug_split_weight(float w);
 
 /* Schedule of the draft attention (bf16 models) for every later call,
  * process-wide: 0 (default) the split-KV grid of fixed key chunks
- * (dflash_debug_attn_chunk); 1 persistent, two CTAs per SM each streaming the
- * same number of 64-key tiles over the (request, kv head) segments, segments
- * split between CTAs merged by their last piece.  Both give the same result up
- * to fp32 summation order.  DFLASH_EINVAL for any other value.  Not
- * thread-safe; tests and tuning only. */
+ * (dflash_debug_attn_chunk) on the mma.sync kernel; 1 persistent (mma.sync),
+ * two CTAs per SM each streaming the same number of 64-key tiles over the
+ * (request, kv head) segments, segments split between CTAs merged by their
+ * last piece; 2 the split-KV grid on the tcgen05 kernel where its shapes allow
+ * (head dim 128, at most 32 query rows per kv head, contiguous K/V; the
+ * mma.sync kernel elsewhere).  All give the same result up to fp32 summation
+ * order and the rounding of the probabilities to fp16.  DFLASH_EINVAL for any
+ * other value.  Not thread-safe; tests and tuning only. */
 int dflash_debug_attn_schedule(int sched);
 
 /* Split-KV chunk of the draft attention, in keys, for every later

@@ -182,10 +182,11 @@ def test_draft_gemm_schedules_agree():
     ("uniform", None),
 ])
 def test_draft_attention_schedules_agree(name, ctx):
-    """The persistent attention (every CTA the same number of key tiles across
-    (request, head) segments, segments split between CTAs merged by their last
-    piece) and the split-KV grid give the oracle's draft; their logits agree far
-    inside the tolerance."""
+    """The three attention schedules give the oracle's draft, and their logits
+    agree far inside the tolerance: the persistent mma.sync attention (every CTA
+    the same number of key tiles across (request, head) segments, segments split
+    between CTAs merged by their last piece), the split-KV grid on the mma.sync
+    kernel (the default) and the split-KV grid on the tcgen05 kernel."""
     base = synth.get_config("qwen3_8b_bs32")
     cfg = shrink(base, L=2, V=2048, batch=6, ctx=("uniform", 1, 700), I=512, d=512,
                  H_t=512).replace(name="attn_sched8b")
@@ -193,7 +194,7 @@ def test_draft_attention_schedules_agree(name, ctx):
     ctx_t = None if ctx is None else torch.tensor(ctx, dtype=torch.int32)
     runs = []
     try:
-        for sched in (1, 0):
+        for sched in (1, 0, 2):
             D.debug_attn_schedule(sched)
             runs.append(_run_draft(b, cfg, ctx=ctx_t))
     finally:
@@ -201,7 +202,15 @@ def test_draft_attention_schedules_agree(name, ctx):
     for res in runs:
         assert res["err"] == 0
         _check(b, cfg, res, cfg.steps, range(cfg.batch), test=f"draft_attention_schedules[{name}]")
-    la, lb = runs[0]["lg"], runs[1]["lg"]
-    both = ~(torch.isnan(la) | torch.isnan(lb))
-    scale = la[both].abs().max().item()
-    assert (la[both] - lb[both]).abs().max().item() <= 2e-3 * scale
+    # the first denoising step depends on no commit decision; later steps are
+    # compared where both schedules committed the same tokens (each run's
+    # near-tie choices are checked against the oracle's rules above)
+    for other in runs[1:]:
+        same = torch.equal(runs[0]["out"], other["out"]) and torch.equal(runs[0]["cst"],
+                                                                            other["cst"])
+        la, lb = runs[0]["lg"], other["lg"]
+        if not same:
+            la, lb = la[:1], lb[:1]
+        both = ~(torch.isnan(la) | torch.isnan(lb))
+        scale = la[both].abs().max().item()
+        assert (la[both] - lb[both]).abs().max().item() <= 2e-3 * scale
