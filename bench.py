@@ -216,6 +216,8 @@ def run_dflash(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    if args.attn_schedule:
+        D.debug_attn_schedule(args.attn_schedule)
     cfg = synth.get_config(WORKLOAD)
     if args.layers:
         # profiling variant: the same per-layer shapes with fewer layers (smaller footprint)
@@ -394,6 +396,8 @@ def run_dflash(args, rank, world, local_rank):
         "config": {"workload": cfg.name, "model": f"Qwen3-8B-shaped DFlash draft ({cfg.L} layers)",
                    "global_batch": b * world, "block": B, "denoise_steps": cfg.steps,
                    "ctx": "uniform[512,4096]", "inject_rows": n_s, "parallelism": f"dp{world}",
+                   "attention": ["split-KV grid, mma.sync", "persistent, mma.sync",
+                                 "split-KV grid, tcgen05"][args.attn_schedule],
                    "l2": "no flush: every step streams ~7.4 GB of weights and K/V (> 126 MB L2)"},
         "roofline": roof,
         "tensor_peak": {"TFLOPs": tc_peak, "kind": tc_kind,
@@ -873,6 +877,9 @@ def main():
                     help="cycles launched call by call versus replayed from a CUDA graph")
     ap.add_argument("--sampled-verify-report", action="store_true",
                     help="sampled (temperature) verify against its HBM roofline")
+    ap.add_argument("--attn-schedule", type=int, default=0,
+                    help="tuning only: draft attention schedule (0 default grid, 1 persistent, "
+                         "2 grid on the tcgen05 kernel)")
     args = ap.parse_args()
     if args.gemm_report:
         gemm_report()
