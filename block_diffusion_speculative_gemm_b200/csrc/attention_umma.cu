@@ -10,7 +10,8 @@
 //   softmax     warp 0, one thread per query row: reads its S row from TMEM,
 //               keeps a reference max (log2 units) and the sum, rescales its
 //               O row in TMEM when some row's max grew by more than 2^8, and
-//               writes P (fp16) to shared memory.
+//               writes P (fp16) into one of two shared-memory buffers, so it
+//               waits for the O += P V two tiles back, not the last one.
 //   O += P V    UMMA M = 128, N = 128 (head dim), K = 48 keys; V is the
 //               MN-major B operand (its rows are keys, head dim contiguous).
 // Warp 1 issues the MMAs (S of tile t + 1 before O += P V of tile t), warp 2
@@ -37,10 +38,13 @@ constexpr int kUThreads = 128;
 constexpr int kUTile = kUKeys * kHD * 2;         // K or V of one tile (12 KB)
 constexpr int kUStage = 2 * kUTile;
 constexpr int kURegion = 32 * 1024;              // Q, P and the block tile
-constexpr int kUSmem = kUStages * kUStage + kURegion + 1024;  // + alignment slack
-// region offsets: Q rows 0-31 of column half 0, P rows 0-31, block K and V
-// (16 rows x two column halves each), Q rows 0-31 of column half 1
-constexpr int kOffQ0 = 0, kOffP = 4096, kOffBK = 8192, kOffBV = 12288, kOffQ1 = 16384;
+constexpr int kUSmem = kURegion + kUStages * kUStage + 1024;  // + alignment slack
+// region offsets (the region comes first, so the unused rows of the last
+// buffers run over the stages, inside the allocation): Q rows 0-31 of column
+// half 0, P buffer 0 rows 0-31, block K and V (16 rows x two column halves
+// each), Q rows 0-31 of column half 1, P buffer 1 rows 0-31
+constexpr int kOffQ0 = 0, kOffP0 = 4096, kOffBK = 8192, kOffBV = 12288, kOffQ1 = 16384,
+              kOffP1 = 20480;
 constexpr uint32_t kColS = 0;    // two S buffers, 64 columns apart
 constexpr uint32_t kColO = 128;  // O: 128 columns
 constexpr uint32_t kTmemCols = 256;
@@ -102,7 +106,7 @@ __global__ void __launch_bounds__(kUThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bars[2 * kUStages + 4 + 3];
+  __shared__ __align__(8) uint64_t bars[2 * kUStages + 4 + 4];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -122,16 +126,17 @@ __global__ void __launch_bounds__(kUThreads, 2)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   const uint32_t s_base = smem_u32(smem);
-  const uint32_t s_reg = s_base + kUStages * kUStage;
-  auto sK = [&](int st) { return s_base + st * kUStage; };
-  auto sV = [&](int st) { return s_base + st * kUStage + kUTile; };
+  const uint32_t s_reg = s_base;
+  auto sK = [&](int st) { return s_base + kURegion + st * kUStage; };
+  auto sV = [&](int st) { return s_base + kURegion + st * kUStage + kUTile; };
+  auto pbuf = [&](int t) { return (uint32_t)((t & 1) ? kOffP1 : kOffP0); };
   auto full = [&](int st) { return smem_u32(&bars[st]); };
   auto empty = [&](int st) { return smem_u32(&bars[kUStages + st]); };
   auto s_full = [&](int b) { return smem_u32(&bars[2 * kUStages + b]); };
   auto s_free = [&](int b) { return smem_u32(&bars[2 * kUStages + 2 + b]); };
   const uint32_t p_full = smem_u32(&bars[2 * kUStages + 4]);
-  const uint32_t p_free = smem_u32(&bars[2 * kUStages + 5]);
-  const uint32_t o_done = smem_u32(&bars[2 * kUStages + 6]);
+  auto p_free = [&](int b) { return smem_u32(&bars[2 * kUStages + 5 + b]); };  // per P buffer
+  const uint32_t o_done = smem_u32(&bars[2 * kUStages + 7]);
 
   if (tid == 0) {
     for (int st = 0; st < kUStages; ++st) {
@@ -143,7 +148,8 @@ __global__ void __launch_bounds__(kUThreads, 2)
       mbar_init(s_free(b), 1);
     }
     mbar_init(p_full, 1);
-    mbar_init(p_free, 1);
+    mbar_init(p_free(0), 1);
+    mbar_init(p_free(1), 1);
     mbar_init(o_done, 1);
     fence_barrier_init();
     s_abort = 0;
@@ -239,11 +245,11 @@ __global__ void __launch_bounds__(kUThreads, 2)
           const uint64_t bdesc = blk ? desc_mn_sw128(s_reg + kOffBV, kUBlk * 128)
                                      : desc_mn_sw128(sV(t % kUStages) + kk * 16 * 128,
                                                      kUKeys * 128);
-          umma_f16(tmem + kColO, smem_desc_sw128(s_reg + kOffP + kk * 32), bdesc, id_o,
+          umma_f16(tmem + kColO, smem_desc_sw128(s_reg + pbuf(t) + kk * 32), bdesc, id_o,
                    (t > 0 || kk > 0) ? 1u : 0u);
         }
         if (!blk) umma_commit(empty(t % kUStages));
-        umma_commit(p_free);
+        umma_commit(p_free(t & 1));
       };
       for (int t = 0; t < ntot && ok; ++t) {
         const bool blk = t == nt;
@@ -328,25 +334,32 @@ __global__ void __launch_bounds__(kUThreads, 2)
         const __half2 h = __floats2half2_rn(e0, e1);
         pw[k] = *reinterpret_cast<const uint32_t*>(&h);
       }
-      // O and the P buffer are free once the previous tile's O += P V is done
-      if (t >= 1) {
-        if (!__all_sync(0xffffffffu, wait(p_free, (t - 1) & 1))) { ok = false; break; }
-        tc_fence_after();
-        if (move) {
-          const float cf = (m == -INFINITY || mn == -INFINITY) ? 1.f : exp2f(m - mn);
-#pragma unroll 1
-          for (int cc = 0; cc < kHD; cc += 32) {
-            float v[32];
-            tmem_ld32(lane_addr + kColO + cc, v);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= cf;
-            tmem_st32(lane_addr + kColO + cc, v);
-          }
-          l *= cf;
+      // P buffer t & 1 is free once O += P V of tile t - 2 is done; O may be
+      // rescaled only once O += P V of tile t - 1 is done
+      if (t >= 2 &&
+          !__all_sync(0xffffffffu, wait(p_free(t & 1), ((t / 2) - 1) & 1))) {
+        ok = false;
+        break;
+      }
+      if (t >= 1 && move) {
+        if (!__all_sync(0xffffffffu, wait(p_free((t - 1) & 1), ((t - 1) / 2) & 1))) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        const float cf = (m == -INFINITY || mn == -INFINITY) ? 1.f : exp2f(m - mn);
+#pragma unroll 1
+        for (int cc = 0; cc < kHD; cc += 32) {
+          float v[32];
+          tmem_ld32(lane_addr + kColO + cc, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= cf;
+          tmem_st32(lane_addr + kColO + cc, v);
+        }
+        l *= cf;
       }
       // this row of the P tile (keys as K), 16 bytes per 8 keys
-      uint8_t* prow = smem + kUStages * kUStage + kOffP;
+      uint8_t* prow = smem + pbuf(t);
 #pragma unroll
       for (int ch = 0; ch < kUKeys / 8; ++ch) {
         if (ch * 8 >= nk) break;
@@ -358,7 +371,7 @@ __global__ void __launch_bounds__(kUThreads, 2)
       if (!blk && nvalid < kUKeys) {
         // rows past the context hold other cache positions: zero them in V so
         // that masked keys contribute exactly nothing
-        uint8_t* v = smem + (t % kUStages) * kUStage + kUTile;
+        uint8_t* v = smem + kURegion + (t % kUStages) * kUStage + kUTile;
         for (int idx = lane; idx < (kUKeys - nvalid) * (kHD / 8); idx += 32) {
           const int row = nvalid + idx / (kHD / 8), ch = idx % (kHD / 8);
           *reinterpret_cast<uint4*>(v + (ch >> 3) * (kUKeys * 128) + swz(row, ch)) =
@@ -399,7 +412,8 @@ __global__ void __launch_bounds__(kUThreads, 2)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
-  attn_chunk_combine<kHD, kUThreads>(reinterpret_cast<float*>(smem), r, g, R, B, G, nq, nkv, Tc,
+  attn_chunk_combine<kHD, kUThreads>(reinterpret_cast<float*>(smem + kURegion), r, g, R, B, G, nq,
+                                     nkv, Tc,
                                      chunk, n_chunks, part_o, part_ml, cnt, out);
 }
 
