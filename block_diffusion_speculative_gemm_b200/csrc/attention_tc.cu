@@ -880,12 +880,7 @@ int launch_hd(const __half* q, const __half* kb, const __half* vb, const __half*
                                     s);
   }
   if (HD == 128 && R <= 32 && B <= 16 && pg.table == nullptr && g_attn_umma) {
-    // the tcgen05 kernel streams 48-key tiles
-    CUtensorMap tk48, tv48;
-    if (!encode_2d(&tk48, kc, rows, HD, HD, kUmmaKeys, DFLASH_F16) ||
-        !encode_2d(&tv48, vc, rows, HD, HD, kUmmaKeys, DFLASH_F16))
-      return DFLASH_ECUDA;
-    return launch_attn_umma(tk48, tv48, q, kb, vb, pg, rows, layer, batch, cap, ctx_len,
+    return launch_attn_umma(tk, tv, q, kb, vb, pg, rows, layer, batch, cap, ctx_len,
                             req_valid, B, nq, nkv, chunk, n_chunks, part_o, part_ml, cnt, o, err,
                             s);
   }

@@ -54,36 +54,52 @@ __device__ void attn_chunk_combine(float* scratch, int r, int g, int R, int B, i
     for (int cc = 0; cc < nvc; ++cc) sml[(cc * kAttnMaxRows + row) * 2] *= inv;
   }
   __syncthreads();
-  for (int i4 = tid; i4 < R * HD / 4; i4 += kThreads) {
-    const int row = (i4 * 4) / HD, col = (i4 * 4) % HD;
-    const float4* src = reinterpret_cast<const float4*>(part_o + (base + row) * HD + col);
-    const size_t cstride = (size_t)kAttnMaxRows * HD / 4;  // float4s from chunk to chunk
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int cc = 0;
-    for (; cc + 4 <= nvc; cc += 4) {  // four chunk loads in flight, summed in chunk order
-      float4 v[4];
+  // output float4 i4 = (row, col): row = 4 i4 / HD; chunk cc's partial of it
+  // sits cc * kAttnMaxRows * HD / 4 float4s after chunk 0's.  Each thread
+  // keeps kU outputs and two chunks of loads in flight, so the merge waits
+  // for about nvc / 2 memory round trips; chunks are summed in order.
+  constexpr int kU = 8;
+  const int total = R * HD / 4;
+  const size_t cstride = (size_t)kAttnMaxRows * HD / 4;
+  const float4* src0 = reinterpret_cast<const float4*>(part_o + base * HD);
+  for (int i0 = tid; i0 < total; i0 += kThreads * kU) {
+    float4 acc[kU];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = __ldcg(src + (size_t)(cc + u) * cstride);
+    for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int cc = 0; cc < nvc; cc += 2) {
+      float4 v[kU][2];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float w = sml[((cc + u) * kAttnMaxRows + row) * 2];
-        acc.x += w * v[u].x;
-        acc.y += w * v[u].y;
-        acc.z += w * v[u].z;
-        acc.w += w * v[u].w;
+      for (int u = 0; u < kU; ++u) {
+        const int i4 = i0 + u * kThreads;
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          v[u][k] = (i4 < total && cc + k < nvc) ? __ldcg(src0 + (size_t)(cc + k) * cstride + i4)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int row = ((i0 + u * kThreads) * 4) / HD;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          if (i0 + u * kThreads < total && cc + k < nvc) {
+            const float w = sml[((cc + k) * kAttnMaxRows + row) * 2];
+            acc[u].x += w * v[u][k].x;
+            acc[u].y += w * v[u][k].y;
+            acc[u].z += w * v[u][k].z;
+            acc[u].w += w * v[u][k].w;
+          }
+        }
       }
     }
-    for (; cc < nvc; ++cc) {
-      const float4 v = __ldcg(src + (size_t)cc * cstride);
-      const float w = sml[(cc * kAttnMaxRows + row) * 2];
-      acc.x += w * v.x;
-      acc.y += w * v.y;
-      acc.z += w * v.z;
-      acc.w += w * v.w;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i4 = i0 + u * kThreads;
+      if (i4 >= total) break;
+      const int row = (i4 * 4) / HD, col = (i4 * 4) % HD;
+      __half* dst = out + ((size_t)(r * B + row / G) * nq + g * G + row % G) * HD + col;
+      *reinterpret_cast<__half2*>(dst) = __floats2half2_rn(acc[u].x, acc[u].y);
+      *reinterpret_cast<__half2*>(dst + 2) = __floats2half2_rn(acc[u].z, acc[u].w);
     }
-    __half* dst = out + ((size_t)(r * B + row / G) * nq + g * G + row % G) * HD + col;
-    *reinterpret_cast<__half2*>(dst) = __floats2half2_rn(acc.x, acc.y);
-    *reinterpret_cast<__half2*>(dst + 2) = __floats2half2_rn(acc.z, acc.w);
   }
   if (tid == 0) cnt[r * nkv + g] = 0;  // ready for the next launch
 }

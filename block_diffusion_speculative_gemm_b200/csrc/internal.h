@@ -251,10 +251,9 @@ int launch_attn_plan(const int32_t* ctx_len, const int32_t* req_valid, int batch
 // The tcgen05 attention kernel (head dim 128, at most 32 query rows per kv
 // head, contiguous K/V, the grid schedule): used by launch_attn_tc while
 // g_attn_umma is set (dflash_debug_attn_schedule(2)); tk/tv are tensor maps of
-// kUmmaKeys-row boxes.
-// DFLASH_EUNSUPPORTED outside its shapes.
+// 64-row, 64-column boxes (the mma.sync kernel's).  DFLASH_EUNSUPPORTED
+// outside its shapes (and for a chunk that is not a multiple of 64 keys).
 extern int g_attn_umma;
-constexpr int kUmmaKeys = 48;  // keys per context tile of the tcgen05 kernel (TMA box rows)
 int launch_attn_umma(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q,
                      const __half* kb, const __half* vb, const KvPages& pg, long long kv_rows,
                      int layer, int batch, int cap, const int32_t* ctx_len,
