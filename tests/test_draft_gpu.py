@@ -98,23 +98,27 @@ def test_draft_context_lengths_edge_cases():
     print(_check(b, cfg, res, cfg.steps, range(cfg.batch), test="draft_context_edge_cases"))
 
 
+@pytest.mark.parametrize("sched", [0, 2])
 @pytest.mark.parametrize("chunk", [64, 192, 4096])
-def test_draft_attention_chunk_sizes(chunk):
+def test_draft_attention_chunk_sizes(chunk, sched):
     """The same requests with the split-KV chunk forced from one tile per chunk to one
-    chunk per request: every split and the chunk combine give the oracle's result."""
+    chunk per request: every split and the chunk combine give the oracle's result, on
+    the mma.sync kernel (schedule 0) and on the tcgen05 kernel (schedule 2)."""
     base = synth.get_config("qwen3_8b_bs32")
     cfg = shrink(base, L=1, V=2048, batch=4, ctx=("uniform", 1, 900), I=512, d=512,
                  H_t=512).replace(name="chunk8b")
     b = built(cfg)
     ctx = torch.tensor([0, 63, 64, 900], dtype=torch.int32)
-    D.debug_attn_chunk(chunk)  # the split-KV grid (the default schedule)
+    D.debug_attn_chunk(chunk)  # the split-KV grid
+    D.debug_attn_schedule(sched)
     try:
         res = _run_draft(b, cfg, ctx=ctx)
     finally:
         D.debug_attn_chunk(0)
+        D.debug_attn_schedule(0)
     assert res["err"] == 0
-    print(chunk, _check(b, cfg, res, cfg.steps, range(cfg.batch),
-                        test=f"draft_attention_chunk[{chunk}]"))
+    print(chunk, sched, _check(b, cfg, res, cfg.steps, range(cfg.batch),
+                               test=f"draft_attention_chunk[{chunk}-{sched}]"))
 
 
 def test_draft_rejects_bad_requests_without_writing():
@@ -145,6 +149,37 @@ def test_draft_full_size_sampled_requests(name, requests):
     assert (out[:, 1:] >= 0).all() and (out[:, 1:] < cfg.V).all()
     assert (res["cst"][:, 1:] >= 0).all() and (res["cst"][:, 1:] < cfg.steps).all()
     print(name, _check(b, cfg, res, cfg.steps, requests, test=f"draft_full_size[{name}]"))
+
+
+@pytest.mark.parametrize("name,requests", [
+    ("qwen3_8b_bs32", [5]),
+    ("qwen3_8b_ctx32k", [1]),   # 43 split-KV chunks per request: a long chunk merge
+])
+def test_draft_full_size_tcgen05_attention(name, requests):
+    """At full size the split-KV grid on the tcgen05 kernel gives a draft that
+    passes the oracle's rules on the sampled requests, and logits that agree with
+    the default mma.sync kernel far inside the tolerance (every denoising step
+    where both committed the same tokens, else the first)."""
+    cfg = synth.get_config(name)
+    b = built(cfg)
+    base = _run_draft(b, cfg)
+    try:
+        D.debug_attn_schedule(2)
+        umma = _run_draft(b, cfg)
+    finally:
+        D.debug_attn_schedule(0)
+    assert base["err"] == 0 and umma["err"] == 0
+    _check(b, cfg, umma, cfg.steps, requests, test=f"draft_full_size_tcgen05_attention[{name}]")
+    same = torch.equal(base["out"], umma["out"]) and torch.equal(base["cst"], umma["cst"])
+    la, lb = base["lg"], umma["lg"]
+    if not same:
+        la, lb = la[:1], lb[:1]
+    both = ~(torch.isnan(la) | torch.isnan(lb))
+    scale = la[both].abs().max().item()
+    diff = (la[both] - lb[both]).abs().max().item()
+    record("draft_full_size_tcgen05_attention", max_rel_diff=diff / scale, configs=1,
+           configs_same_commits=int(same))
+    assert diff <= 2e-3 * scale
 
 
 def test_draft_gemm_schedules_agree():
