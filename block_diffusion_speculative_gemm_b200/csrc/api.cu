@@ -270,7 +270,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct DraftLayout {
   size_t tokens, zrow, lm_rows, cstep, req_valid, lm_tok, lm_conf, x, h, q, kb, vb, o, act, part,
-      sk, attn_o, attn_ml, seg, stats, draw, logits, end;
+      sk, attn_o, attn_ml, seg, attn_chunk, stats, draw, logits, end;
   size_t part_elems;  // fp32 elements of split-K partials
 };
 
@@ -320,6 +320,8 @@ DraftLayout draft_layout(const dflash_config& c, int batch, int B) {
   L.attn_o = take(4 * arows * c.head_dim);
   L.attn_ml = take(8 * arows);
   L.seg = take(4 * ((size_t)batch * c.n_kv + 1));  // persistent schedule: segment prefix
+  // split-KV grid: the plan made on the device for a forward ({chunk, items, item...})
+  L.attn_chunk = take(4 * (4 + 2 * (size_t)batch * c.n_kv * kMaxChunks));
   L.stats = take(sizeof(LmStat) * M * n_vt);
   // sampled drafting's draw partials: rows x chunks never exceeds M + 600 (the
   // chunk count falls as the row count grows)
@@ -862,16 +864,26 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
   int32_t* seg_start = bf16 && g_attn_sched == 1 ? at<int32_t>(ws, L.seg) : nullptr;
 
   // split-KV chunk: a multiple of the attention tile (64 keys) sized for
-  // about four CTAs per SM over the whole (request, kv head, chunk) grid, at
-  // most 768 keys (each chunk's partial is merged by the last CTA of its
-  // request and head) and at most kMaxChunks chunks per request
-  int chunk = (int)std::min<int64_t>(768, (int64_t)(cap + B) * batch * c.n_kv / (4 * num_sms()));
+  // about four CTAs per SM over the whole (request, kv head, chunk) grid as if
+  // every request were at capacity, and at most kMaxChunks chunks per request.
+  // Unless a chunk is forced, a planning kernel then picks each forward's
+  // chunk (at least this one, so the grid's n_chunks columns cover it) from the
+  // actual context lengths, and grid columns past a request's last chunk exit.
+  // Without the planner (fp32 models, the persistent schedule) the chunk stays
+  // at most 768 keys: each chunk's partial is merged by the last CTA of its
+  // request and head.
+  const bool forced = g_attn_chunk > 0 && (cap + B + g_attn_chunk - 1) / g_attn_chunk <= kMaxChunks;
+  const bool planned = bf16 && g_attn_sched == 0 && !forced && c.n_kv <= 255;
+  int chunk = (int)std::min<int64_t>(planned ? INT32_MAX : 768,
+                                     (int64_t)(cap + B) * batch * c.n_kv / (4 * num_sms()));
   chunk = std::max(64, (chunk + 63) / 64 * 64);
   chunk = std::max(chunk, (cap + B + kMaxChunks - 1) / kMaxChunks);
   chunk = (chunk + 63) / 64 * 64;
-  if (g_attn_chunk > 0 && (cap + B + g_attn_chunk - 1) / g_attn_chunk <= kMaxChunks)
-    chunk = g_attn_chunk;
+  if (forced) chunk = g_attn_chunk;
   const int n_chunks = (cap + B + chunk - 1) / chunk;
+  int32_t* plan_dev = planned ? at<int32_t>(ws, L.attn_chunk) : nullptr;
+  const int attn_slots =
+      plan_dev ? attn_grid_slots(hd, B * (nq / nkv), B, pg.table != nullptr) : 0;
 
   if (ph.init)
     launch_draft_init(anchor, ctx_len, batch, B, c.vocab, c.mask_id, cap, pg, tokens, zrow,
@@ -903,6 +915,11 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
       return st;
     launch_embed_norm<TE, T>(tokens, static_cast<const TE*>(m->emb), m->layers[0].g_in, x, h, M, c.d,
                          c.eps, err, s);
+    // planned right before the first QKV GEMM, whose weight prefetch (issued
+    // before its dependency wait) covers the planning kernel
+    if (plan_dev && (st = launch_attn_chunk_plan(ctx_len, valid, batch, B, nkv, chunk, plan_dev,
+                                                  attn_slots, s)))
+      return st;
     for (int l = 0; l < c.n_layers; ++l) {
       const LayerPack& P = m->layers[l];
       const float* g_next = l + 1 < c.n_layers ? m->layers[l + 1].g_in : m->g_final;
@@ -942,7 +959,8 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
                              m->rope_sin, q, kb, vb, err, s);
         if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, pg, l, c.n_layers, batch, cap,
                                                 ctx_len, valid, B, nq, nkv, hd, attn_o, attn_ml,
-                                                n_chunks, chunk, seg_start, o, attn_cnt, err, s)))
+                                                n_chunks, chunk, plan_dev, seg_start, o, attn_cnt,
+                                                err, s)))
           return st;
         go.f32 = x;
         if ((st = run(P.mo, c.d, nq * hd, o, OP_RESID))) return st;
@@ -962,7 +980,8 @@ int draft_impl(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_
                          q, kb, vb, err, s);
       if ((st = launch_block_attention<T, TC>(q, kb, vb, kc, vc, pg, l, c.n_layers, batch, cap,
                                               ctx_len, valid, B, nq, nkv, hd, attn_o, attn_ml,
-                                              n_chunks, chunk, nullptr, o, attn_cnt, err, s)))
+                                              n_chunks, chunk, nullptr, nullptr, o, attn_cnt, err,
+                                              s)))
         return st;
       if ((st = gemm(P.mo, P.Wo, c.d, nq * hd, o, part, L.part_elems, &sp))) return st;
       launch_residual_norm<T>(part, sp, M, c.d, x, P.g_post, h, nullptr, c.eps, err, s);
@@ -1449,6 +1468,25 @@ extern "C" int dflash_debug_attn_chunk(int keys) {
   if (keys < 0 || keys % 64 != 0) return DFLASH_EINVAL;
   g_attn_chunk = keys;
   return DFLASH_OK;
+}
+
+extern "C" int dflash_debug_attn_plan(const int32_t* ctx_len, const int32_t* req_valid, int batch,
+                                      int B, int n_kv, int cap, int chunk_min, int slots,
+                                      int32_t* plan_out, long long plan_cap, void* stream) {
+  if (!ctx_len || !req_valid || !plan_out || batch <= 0 || B <= 0 || n_kv <= 0 || n_kv > 255 ||
+      slots <= 0 || cap < B || chunk_min <= 0 || chunk_min % 64 != 0 ||
+      (cap + chunk_min - 1) / chunk_min > 255)
+    return DFLASH_EINVAL;
+  if (plan_cap < 4 + 2LL * batch * n_kv * ((cap + chunk_min - 1) / chunk_min) ||
+      (reinterpret_cast<uintptr_t>(plan_out) & 7) != 0)
+    return DFLASH_EINVAL;
+  return launch_attn_chunk_plan(ctx_len, req_valid, batch, B, n_kv, chunk_min, plan_out, slots,
+                                (cudaStream_t)stream);
+}
+
+extern "C" int dflash_debug_attn_slots(int head_dim, int rows, int B) {
+  if (head_dim <= 0 || rows <= 0 || B <= 0) return DFLASH_EINVAL;
+  return attn_grid_slots(head_dim, rows, B, false);
 }
 
 extern "C" int dflash_debug_split_weight(float w) {

@@ -189,16 +189,18 @@ int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, c
                            const KvPages& pages, int layer, int L, int batch, int cap,
                            const int32_t* ctx_len, const int32_t* req_valid, int B, int nq,
                            int nkv, int hd, float* part_o, float* part_ml, int n_chunks, int chunk,
-                           const int32_t* seg_start, T* o, unsigned* cnt, int32_t* err,
-                           cudaStream_t s) {
+                           const int32_t* plan_dev, const int32_t* seg_start, T* o,
+                           unsigned* cnt, int32_t* err, cudaStream_t s) {
   if (B * (nq / nkv) > kMaxRows) return DFLASH_EUNSUPPORTED;
   dim3 grid(n_chunks, nkv, batch);
   if constexpr (std::is_same<T, __half>::value) {
     // the tensor-core kernel merges its chunks itself
     return launch_attn_tc(q, kb, vb, kc, vc, pages, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
-                          hd, L, chunk, n_chunks, seg_start, part_o, part_ml, cnt, o, err, s);
+                          hd, L, chunk, plan_dev, n_chunks, seg_start, part_o, part_ml, cnt, o,
+                          err, s);
   } else {
-    if (pages.table != nullptr || seg_start != nullptr) return DFLASH_EUNSUPPORTED;
+    if (pages.table != nullptr || seg_start != nullptr || plan_dev != nullptr)
+      return DFLASH_EUNSUPPORTED;
     {
       TimedScope ts(s, TC_ATTN);
       if (hd == 128) {
@@ -234,13 +236,14 @@ template int launch_block_attention<float, float>(const float*, const float*, co
                                                   const float*, const float*, const KvPages&, int,
                                                   int, int, int, const int32_t*, const int32_t*,
                                                   int, int, int, int, float*, float*, int, int,
-                                                  const int32_t*, float*, unsigned*, int32_t*,
-                                                  cudaStream_t);
+                                                  const int32_t*, const int32_t*, float*, unsigned*,
+                                                  int32_t*, cudaStream_t);
 template int launch_block_attention<__half, __half>(const __half*, const __half*, const __half*,
                                                     const __half*, const __half*, const KvPages&,
                                                     int, int, int, int, const int32_t*,
                                                     const int32_t*, int, int, int, int, float*,
-                                                    float*, int, int, const int32_t*, __half*,
-                                                    unsigned*, int32_t*, cudaStream_t);
+                                                    float*, int, int, const int32_t*,
+                                                    const int32_t*, __half*, unsigned*, int32_t*,
+                                                    cudaStream_t);
 
 }  // namespace dflash

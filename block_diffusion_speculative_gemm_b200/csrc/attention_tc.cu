@@ -16,6 +16,8 @@
 // back to zero -- merges the chunks into the output rows.
 //
 // Memory-bound: 4 * B * G flop per cache byte read, every cache byte read once.
+#include <algorithm>
+
 #include "attn_combine.cuh"
 #include "common.cuh"
 #include "internal.h"
@@ -228,11 +230,29 @@ __global__ void __launch_bounds__(kThreads)
                    const __half* __restrict__ vb, const KvPages pg, long long kv_rows, int layer,
                    int batch, int cap,
                    const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ req_valid,
-                   int B, int nq, int nkv, int chunk, int n_chunks, float* __restrict__ part_o,
-                   float* __restrict__ part_ml, unsigned* __restrict__ cnt,
-                   __half* __restrict__ out, int32_t* err) {
+                   int B, int nq, int nkv, int chunk_host, const int32_t* plan_dev, int n_chunks,
+                   float* __restrict__ part_o, float* __restrict__ part_ml,
+                   unsigned* __restrict__ cnt, __half* __restrict__ out, int32_t* err) {
   pdl_trigger();
   pdl_wait();
+  // A planned forward runs a 1-D grid over the planning kernel's work list
+  // ({chunk, items, -, -, then per item: request << 16 | kv head << 8 |
+  // chunk index and the request's context length}, in the 3-D grid's order);
+  // CTAs past the list exit.  Otherwise the grid is (chunk, kv head, request)
+  // with the host's chunk.
+  int c = blockIdx.x, g = blockIdx.y, r = blockIdx.z, chunk = chunk_host, Tc;
+  if (plan_dev != nullptr) {
+    const int n_items = plan_dev[1];
+    const int2 it = reinterpret_cast<const int2*>(plan_dev)[2 + blockIdx.x];
+    chunk = plan_dev[0];
+    if ((int)blockIdx.x >= n_items) return;
+    r = it.x >> 16;
+    g = (it.x >> 8) & 255;
+    c = it.x & 255;
+    Tc = it.y;
+  } else {
+    Tc = req_valid[r] ? ctx_len[r] : 0;
+  }
   using LY = Layout<HD, MT>;
   using WP = Warp<HD, MT>;
   constexpr int kStages = LY::kStages;
@@ -247,10 +267,8 @@ __global__ void __launch_bounds__(kThreads)
   auto full = [&](int st) { return smem_u32(bars + st); };
   auto empty = [&](int st) { return smem_u32(bars + kStages + st); };
 
-  const int c = blockIdx.x, g = blockIdx.y, r = blockIdx.z;
   const int G = nq / nkv;
   const int R = B * G;
-  const int Tc = req_valid[r] ? ctx_len[r] : 0;
   const int k0 = c * chunk;
   if (k0 >= Tc + B) return;
   const int k1 = min(Tc + B, k0 + chunk);
@@ -834,22 +852,118 @@ int launch_persistent(const CUtensorMap& tk, const CUtensorMap& tv, const __half
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 
+// Chunk of the split-KV grid for one forward, from the actual context
+// lengths.  The estimate follows how the grid behaves on B200: every CTA pays
+// a fixed cost (set-up, the partial's write and fence: about kPlanFixed 64-key
+// tiles' worth), CTAs run in waves over the resident slots, and the chunks of
+// a request are merged by its last CTA (about kPlanMerge tiles per chunk).
+// With L the mean keys of a request (context plus block), candidate q cuts L
+// into q chunks, scaled by kPlanScale so that requests a little longer than
+// the mean still take one chunk, rounded up to 64 keys and at least
+// chunk_min.  One thread per candidate q = 1..64; ties go to the larger chunk.
+// It then writes the forward's work list (see attn_tc_kernel).
+constexpr float kPlanFixed = 8.f;
+constexpr float kPlanMerge = 0.5f;
+constexpr float kPlanScale = 1.06f;
+constexpr int kPlanThreads = 64;
+
+__global__ void __launch_bounds__(kPlanThreads)
+    attn_chunk_plan_kernel(const int32_t* ctx_len, const int32_t* req_valid, int batch, int B,
+                           int nkv, int chunk_min, int slots, int32_t* plan) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float s_sum[kPlanThreads / 32];
+  __shared__ float s_est[kPlanThreads];
+  __shared__ int s_chunk[kPlanThreads];
+  __shared__ int s_tot[kPlanThreads / 32];
+  __shared__ int s_carry;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  auto keys = [&](int r) { return (req_valid[r] ? ctx_len[r] : 0) + B; };  // context + block
+  float acc = 0.f;
+  for (int r = threadIdx.x; r < batch; r += kPlanThreads) acc += (float)keys(r);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) s_sum[w] = acc;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int i = 0; i < kPlanThreads / 32; ++i) tot += s_sum[i];
+  const float L = fmaxf(tot / (float)max(batch, 1), 1.f);
+  const int q = threadIdx.x + 1;
+  int C = (int)ceilf(kPlanScale * L / (float)q);
+  C = max(chunk_min, (C + kKeys - 1) / kKeys * kKeys);
+  const float qe = ceilf(L / (float)C);  // chunks of a mean request
+  const float waves = ceilf((float)batch * (float)nkv * qe / (float)max(slots, 1));
+  s_est[threadIdx.x] = waves * ((float)((C + kKeys - 1) / kKeys) + kPlanFixed) + kPlanMerge * qe;
+  s_chunk[threadIdx.x] = C;
+  if (threadIdx.x == 0) s_carry = 0;
+  __syncthreads();
+  int best = 0;
+  for (int i = 1; i < kPlanThreads; ++i)
+    if (s_est[i] < s_est[best]) best = i;
+  const int chunk = s_chunk[best];
+  // the work list: every request's kv heads and chunks, in the order of the
+  // (chunk, kv head, request) grid, request-major
+  for (int base = 0; base < batch; base += kPlanThreads) {
+    const int r = base + threadIdx.x;
+    const int qr = r < batch ? (keys(r) + chunk - 1) / chunk : 0;
+    const int n = nkv * qr;
+    int x = n;  // inclusive scan inside the warp, then across the two warps
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_tot[w] = x;
+    __syncthreads();
+    const int start = s_carry + (w > 0 ? s_tot[0] : 0) + x - n;
+    const int Tr = r < batch && req_valid[r] ? ctx_len[r] : 0;
+    int2* items = reinterpret_cast<int2*>(plan) + 2;
+    for (int j = 0; j < n; ++j) items[start + j] = make_int2((r << 16) | ((j / qr) << 8) | (j % qr), Tr);
+    __syncthreads();
+    if (threadIdx.x == kPlanThreads - 1) s_carry = start + n;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    plan[0] = chunk;
+    plan[1] = s_carry;
+  }
+}
+
+// Resident CTAs per SM of the split-KV grid kernel.
+template <int HD, int MT>
+int grid_ctas_per_sm() {
+  static int n = -1;
+  if (n < 0) {
+    const int smem = Layout<HD, MT>::kSmem;
+    int v = 0;
+    if (cudaFuncSetAttribute(attn_tc_kernel<HD, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, attn_tc_kernel<HD, MT>, kThreads,
+                                                      smem) != cudaSuccess)
+      v = 1;
+    n = std::max(1, v);
+  }
+  return n;
+}
+
 template <int HD, int MT>
 int launch_cfg(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q, const __half* kb,
                const __half* vb, const KvPages& pg, long long kv_rows, int layer, int batch, int cap,
                const int32_t* ctx_len,
-               const int32_t* req_valid, int B, int nq, int nkv, int chunk, int n_chunks,
-               float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
-               cudaStream_t s) {
+               const int32_t* req_valid, int B, int nq, int nkv, int chunk,
+               const int32_t* plan_dev, int n_chunks, float* part_o, float* part_ml,
+               unsigned* cnt, __half* o, int32_t* err, cudaStream_t s) {
   const int smem = Layout<HD, MT>::kSmem;
   if (cudaFuncSetAttribute(attn_tc_kernel<HD, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess)
     return DFLASH_ECUDA;
-  dim3 grid(n_chunks, nkv, batch);
+  // a planned forward runs a 1-D grid sized for the smallest chunk the plan may pick
+  const dim3 grid = plan_dev != nullptr ? dim3(n_chunks * nkv * batch) : dim3(n_chunks, nkv, batch);
   const cudaError_t e =
       launch_pdl(attn_tc_kernel<HD, MT>, grid, dim3(kThreads), smem, s, 1, tk, tv, q, kb, vb, pg,
-                 kv_rows, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks, part_o,
-                 part_ml, cnt, o, err);
+                 kv_rows, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, plan_dev,
+                 n_chunks, part_o, part_ml, cnt, o, err);
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 
@@ -857,7 +971,8 @@ template <int HD>
 int launch_hd(const __half* q, const __half* kb, const __half* vb, const __half* kc,
               const __half* vc, const KvPages& pg, int layer, int batch, int cap,
               const int32_t* ctx_len, const int32_t* req_valid, int B, int nq, int nkv, int L,
-              int chunk, int n_chunks, const int32_t* seg_start, float* part_o, float* part_ml,
+              int chunk, const int32_t* plan_dev, int n_chunks, const int32_t* seg_start,
+              float* part_o, float* part_ml,
               unsigned* cnt, __half* o, int32_t* err, cudaStream_t s) {
   CUtensorMap tk, tv;
   const int64_t rows = pg.table == nullptr ? (int64_t)L * batch * nkv * cap
@@ -881,17 +996,17 @@ int launch_hd(const __half* q, const __half* kb, const __half* vb, const __half*
   }
   if (HD == 128 && R <= 32 && B <= 16 && pg.table == nullptr && g_attn_umma) {
     return launch_attn_umma(tk, tv, q, kb, vb, pg, rows, layer, batch, cap, ctx_len,
-                            req_valid, B, nq, nkv, chunk, n_chunks, part_o, part_ml, cnt, o, err,
-                            s);
+                            req_valid, B, nq, nkv, chunk, plan_dev, n_chunks, part_o, part_ml, cnt,
+                            o, err, s);
   }
   if (R <= 16)
     return launch_cfg<HD, 1>(tk, tv, q, kb, vb, pg, rows, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
-                             chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
+                             chunk, plan_dev, n_chunks, part_o, part_ml, cnt, o, err, s);
   if (R <= 32)
     return launch_cfg<HD, 2>(tk, tv, q, kb, vb, pg, rows, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
-                             chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
+                             chunk, plan_dev, n_chunks, part_o, part_ml, cnt, o, err, s);
   return launch_cfg<HD, 4>(tk, tv, q, kb, vb, pg, rows, layer, batch, cap, ctx_len, req_valid, B, nq, nkv,
-                           chunk, n_chunks, part_o, part_ml, cnt, o, err, s);
+                           chunk, plan_dev, n_chunks, part_o, part_ml, cnt, o, err, s);
 }
 
 }  // namespace
@@ -904,11 +1019,35 @@ int launch_attn_plan(const int32_t* ctx_len, const int32_t* req_valid, int batch
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 
+int launch_attn_chunk_plan(const int32_t* ctx_len, const int32_t* req_valid, int batch, int B,
+                           int nkv, int chunk_min, int32_t* chunk_out, int slots,
+                           cudaStream_t s) {
+  if (chunk_min <= 0 || chunk_min % kKeys != 0) return DFLASH_EINVAL;
+  TimedScope ts(s, TC_ATTN);
+  const cudaError_t e = launch_pdl(attn_chunk_plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, 1,
+                                   ctx_len, req_valid, batch, B, nkv, chunk_min, slots, chunk_out);
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
+}
+
+int attn_grid_slots(int hd, int R, int B, bool paged) {
+  int per = 1;
+  if (hd == 128 && R <= 32 && B <= 16 && !paged && g_attn_umma)
+    per = attn_umma_ctas_per_sm();
+  else if (hd == 128)
+    per = R <= 16 ? grid_ctas_per_sm<128, 1>()
+                  : (R <= 32 ? grid_ctas_per_sm<128, 2>() : grid_ctas_per_sm<128, 4>());
+  else if (hd == 64)
+    per = R <= 16 ? grid_ctas_per_sm<64, 1>()
+                  : (R <= 32 ? grid_ctas_per_sm<64, 2>() : grid_ctas_per_sm<64, 4>());
+  return per * num_sms();
+}
+
 int launch_attn_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
                    const __half* vc, const KvPages& pg, int layer, int batch, int cap,
                    const int32_t* ctx_len,
                    const int32_t* req_valid, int B, int nq, int nkv, int hd, int L, int chunk,
-                   int n_chunks, const int32_t* seg_start, float* part_o, float* part_ml,
+                   const int32_t* plan_dev, int n_chunks, const int32_t* seg_start,
+                   float* part_o, float* part_ml,
                    unsigned* cnt, __half* o, int32_t* err, cudaStream_t s) {
   if (B * (nq / nkv) > kAttnMaxRows || B > kBlkKeys) return DFLASH_EUNSUPPORTED;
   if (seg_start == nullptr && (chunk % kKeys != 0 || n_chunks > kMaxChunksTc))
@@ -921,10 +1060,10 @@ int launch_attn_tc(const __half* q, const __half* kb, const __half* vb, const __
   TimedScope ts(s, TC_ATTN);
   if (hd == 128)
     return launch_hd<128>(q, kb, vb, kc, vc, pg, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, L,
-                          chunk, n_chunks, seg_start, part_o, part_ml, cnt, o, err, s);
+                          chunk, plan_dev, n_chunks, seg_start, part_o, part_ml, cnt, o, err, s);
   if (hd == 64)
     return launch_hd<64>(q, kb, vb, kc, vc, pg, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, L,
-                         chunk, n_chunks, seg_start, part_o, part_ml, cnt, o, err, s);
+                         chunk, plan_dev, n_chunks, seg_start, part_o, part_ml, cnt, o, err, s);
   return DFLASH_EUNSUPPORTED;
 }
 

@@ -132,11 +132,29 @@ __global__ void __launch_bounds__(kUThreads, 2)
                      const __grid_constant__ CUtensorMap tmV, const __half* q, const __half* kb,
                      const __half* vb, const KvPages pg, long long kv_rows, int layer, int batch,
                      int cap, const int32_t* ctx_len, const int32_t* req_valid, int B, int nq,
-                     int nkv, int chunk, int n_chunks, float* __restrict__ part_o,
-                     float* __restrict__ part_ml, unsigned* __restrict__ cnt,
-                     __half* __restrict__ out, int32_t* err) {
+                     int nkv, int chunk_host, const int32_t* plan_dev, int n_chunks,
+                     float* __restrict__ part_o, float* __restrict__ part_ml,
+                     unsigned* __restrict__ cnt, __half* __restrict__ out, int32_t* err) {
   pdl_trigger();
   pdl_wait();
+  // A planned forward runs a 1-D grid over the planning kernel's work list
+  // ({chunk, items, -, -, then per item: request << 16 | kv head << 8 |
+  // chunk index and the request's context length}, in the 3-D grid's order);
+  // CTAs past the list exit.  Otherwise the grid is (chunk, kv head, request)
+  // with the host's chunk.
+  int c = blockIdx.x, g = blockIdx.y, r = blockIdx.z, chunk = chunk_host, Tc;
+  if (plan_dev != nullptr) {
+    const int n_items = plan_dev[1];
+    const int2 it = reinterpret_cast<const int2*>(plan_dev)[2 + blockIdx.x];
+    chunk = plan_dev[0];
+    if ((int)blockIdx.x >= n_items) return;
+    r = it.x >> 16;
+    g = (it.x >> 8) & 255;
+    c = it.x & 255;
+    Tc = it.y;
+  } else {
+    Tc = req_valid[r] ? ctx_len[r] : 0;
+  }
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -149,10 +167,8 @@ __global__ void __launch_bounds__(kUThreads, 2)
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
-  const int c = blockIdx.x, g = blockIdx.y, r = blockIdx.z;
   const int G = nq / nkv;
   const int R = B * G;
-  const int Tc = req_valid[r] ? ctx_len[r] : 0;
   const int k0 = c * chunk;
   if (k0 >= Tc + B) return;
   const int k1 = min(Tc + B, k0 + chunk);
@@ -493,23 +509,37 @@ __global__ void __launch_bounds__(kUThreads, 2)
 
 }  // namespace
 
+int attn_umma_ctas_per_sm() {
+  static int n = -1;
+  if (n < 0) {
+    int v = 0;
+    if (cudaFuncSetAttribute(attn_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kUSmem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, attn_umma_kernel, kUThreads, kUSmem) !=
+            cudaSuccess)
+      v = 1;
+    n = v > 0 ? v : 1;
+  }
+  return n;
+}
+
 int launch_attn_umma(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q,
                      const __half* kb, const __half* vb, const KvPages& pg, long long kv_rows,
                      int layer, int batch, int cap, const int32_t* ctx_len,
-                     const int32_t* req_valid, int B, int nq, int nkv, int chunk, int n_chunks,
-                     float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
-                     cudaStream_t s) {
+                     const int32_t* req_valid, int B, int nq, int nkv, int chunk,
+                     const int32_t* plan_dev, int n_chunks, float* part_o, float* part_ml,
+                     unsigned* cnt, __half* o, int32_t* err, cudaStream_t s) {
   if (B * (nq / nkv) > 32 || B > kUBlk || pg.table != nullptr || n_chunks > kAttnMaxChunks ||
       chunk % kUKeys != 0)
     return DFLASH_EUNSUPPORTED;
   if (cudaFuncSetAttribute(attn_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kUSmem) != cudaSuccess)
     return DFLASH_ECUDA;
-  const dim3 grid(n_chunks, nkv, batch);
+  const dim3 grid = plan_dev != nullptr ? dim3(n_chunks * nkv * batch) : dim3(n_chunks, nkv, batch);
   const cudaError_t e =
       launch_pdl(attn_umma_kernel, grid, dim3(kUThreads), kUSmem, s, 1, tk, tv, q, kb, vb, pg,
-                 kv_rows, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, n_chunks,
-                 part_o, part_ml, cnt, o, err);
+                 kv_rows, layer, batch, cap, ctx_len, req_valid, B, nq, nkv, chunk, plan_dev,
+                 n_chunks, part_o, part_ml, cnt, o, err);
   return e == cudaSuccess ? DFLASH_OK : DFLASH_ECUDA;
 }
 

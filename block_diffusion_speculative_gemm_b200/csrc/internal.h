@@ -248,24 +248,42 @@ constexpr int kAttnMaxRows = 64;  // B * (n_q / n_kv) query rows per (request, k
 // split-KV grid of `chunk`-key chunks.
 int launch_attn_plan(const int32_t* ctx_len, const int32_t* req_valid, int batch, int nkv,
                      int32_t* seg_start, cudaStream_t s);
+// Split-KV grid: the plan of every attention launch of one forward, made on
+// the device from the requests' actual context lengths.  plan receives {chunk,
+// n_items, -, -, items}: the chunk in keys, a multiple of 64 and at least
+// chunk_min (so a grid sized for chunk_min always covers the list), chosen to
+// minimise an estimate of the grid's time (waves of CTAs over `slots` resident
+// CTAs times the tiles plus a fixed cost of one chunk, plus the merge of a mean
+// request's chunks); plan[2..3] unused; then from int 4 one pair per (request,
+// kv head, chunk) with keys, {request << 16 | kv head << 8 | chunk index, the
+// request's context length (0 when it is not valid)}, request-major.  plan
+// holds 4 + 2 * batch * nkv * ceil((cap + B) / chunk_min) ints, 8-byte aligned.
+// slots: attn_grid_slots for the kernel the grid runs.
+int launch_attn_chunk_plan(const int32_t* ctx_len, const int32_t* req_valid, int batch, int B,
+                           int nkv, int chunk_min, int32_t* chunk_out, int slots,
+                           cudaStream_t s);
+// CTAs of the split-KV grid kernel (head dim hd, R = B * n_q / n_kv query rows
+// per kv head, contiguous or paged K/V) that are resident at once on the GPU.
+int attn_grid_slots(int hd, int R, int B, bool paged);
 // The tcgen05 attention kernel (head dim 128, at most 32 query rows per kv
 // head, contiguous K/V, the grid schedule): used by launch_attn_tc while
 // g_attn_umma is set (dflash_debug_attn_schedule(2)); tk/tv are tensor maps of
 // 64-row, 64-column boxes (the mma.sync kernel's).  DFLASH_EUNSUPPORTED
 // outside its shapes (and for a chunk that is not a multiple of 64 keys).
 extern int g_attn_umma;
+int attn_umma_ctas_per_sm();  // resident CTAs per SM of the tcgen05 attention kernel
 int launch_attn_umma(const CUtensorMap& tk, const CUtensorMap& tv, const __half* q,
                      const __half* kb, const __half* vb, const KvPages& pg, long long kv_rows,
                      int layer, int batch, int cap, const int32_t* ctx_len,
-                     const int32_t* req_valid, int B, int nq, int nkv, int chunk, int n_chunks,
-                     float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
-                     cudaStream_t s);
+                     const int32_t* req_valid, int B, int nq, int nkv, int chunk,
+                     const int32_t* plan_dev, int n_chunks, float* part_o, float* part_ml,
+                     unsigned* cnt, __half* o, int32_t* err, cudaStream_t s);
 int launch_attn_tc(const __half* q, const __half* kb, const __half* vb, const __half* kc,
                    const __half* vc, const KvPages& pages, int layer, int batch, int cap,
                    const int32_t* ctx_len, const int32_t* req_valid, int B, int nq, int nkv,
-                   int hd, int L, int chunk, int n_chunks, const int32_t* seg_start,
-                   float* part_o, float* part_ml, unsigned* cnt, __half* o, int32_t* err,
-                   cudaStream_t s);
+                   int hd, int L, int chunk, const int32_t* plan_dev, int n_chunks,
+                   const int32_t* seg_start, float* part_o, float* part_ml, unsigned* cnt,
+                   __half* o, int32_t* err, cudaStream_t s);
 
 // T: type of q, the block's k/v and the output o; TC: K/V cache type.
 // Paged K/V (pages.table set) and the persistent schedule (seg_start set) are
@@ -275,8 +293,8 @@ int launch_block_attention(const T* q, const T* kb, const T* vb, const TC* kc, c
                            const KvPages& pages, int layer, int L, int batch, int cap,
                            const int32_t* ctx_len, const int32_t* req_valid, int B, int nq,
                            int nkv, int hd, float* part_o, float* part_ml, int n_chunks, int chunk,
-                           const int32_t* seg_start, T* o, unsigned* cnt, int32_t* err,
-                           cudaStream_t s);
+                           const int32_t* plan_dev, const int32_t* seg_start, T* o,
+                           unsigned* cnt, int32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- draft bookkeeping
 // cap bounds ctx_len + B; with paged K/V every page below ctx_len must also be

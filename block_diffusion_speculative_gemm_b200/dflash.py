@@ -125,6 +125,9 @@ def lib() -> ctypes.CDLL:
         L.dflash_debug_gemm_streamk_ws_bytes.restype = sz
         L.dflash_debug_gemm_streamk.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp, sz, vp]
         L.dflash_debug_attn_chunk.argtypes = [i32]
+        L.dflash_debug_attn_plan.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp,
+                                             ctypes.c_longlong, vp]
+        L.dflash_debug_attn_slots.argtypes = [i32, i32, i32]
         L.dflash_debug_pick_splits.argtypes = [i32, i32, i32]
         L.dflash_debug_wait_timeout.argtypes = [vp, vp]
         L.dflash_debug_split_weight.argtypes = [ctypes.c_float]
@@ -704,6 +707,32 @@ def debug_attn_chunk(keys: int) -> None:
     """Process-wide split-KV chunk (keys, multiple of 64) of the draft attention;
     0 restores the library's rule (tests and tuning only)."""
     _check("dflash_debug_attn_chunk", lib().dflash_debug_attn_chunk(int(keys)))
+
+
+def debug_attn_plan(ctx_len: torch.Tensor, req_valid: torch.Tensor, B: int, n_kv: int, cap: int,
+                    chunk_min: int, slots: int):
+    """The draft attention planner on these context lengths (device int32
+    tensors), on the current stream (tests): returns (chunk, items) with items
+    the (request, kv head, chunk index, context length) of each CTA of the
+    attention grid, in launch order."""
+    n = 4 + 2 * int(ctx_len.numel()) * n_kv * ((cap + chunk_min - 1) // chunk_min)
+    out = torch.full((n,), -1, dtype=torch.int32, device=ctx_len.device)
+    _check("dflash_debug_attn_plan", lib().dflash_debug_attn_plan(
+        ctx_len.data_ptr(), req_valid.data_ptr(), int(ctx_len.numel()), int(B), int(n_kv),
+        int(cap), int(chunk_min), int(slots), out.data_ptr(), n,
+        torch.cuda.current_stream().cuda_stream))
+    h = out.cpu().tolist()
+    items = [(h[4 + 2 * i] >> 16, (h[4 + 2 * i] >> 8) & 255, h[4 + 2 * i] & 255, h[5 + 2 * i])
+             for i in range(h[1])]
+    return h[0], items
+
+
+def debug_attn_slots(head_dim: int, rows: int, B: int) -> int:
+    """Resident CTAs of the draft attention's split-KV grid kernel (tests)."""
+    r = lib().dflash_debug_attn_slots(int(head_dim), int(rows), int(B))
+    if r < 0:
+        raise RuntimeError(f"dflash_debug_attn_slots: {r}")
+    return r
 
 
 def debug_gemm_streamk(W: torch.Tensor, X: torch.Tensor, stream=None):

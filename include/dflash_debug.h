@@ -107,10 +107,31 @@ int dflash_debug_split_weight(float w);
  * other value.  Not thread-safe; tests and tuning only. */
 int dflash_debug_attn_schedule(int sched);
 
+/* The split-KV planner of the draft attention, run on its own.  For the device
+ * arrays ctx_len and req_valid (batch entries; ctx_len + B <= cap wherever
+ * req_valid is set) it writes to the device array plan_out (8-byte aligned,
+ * plan_cap ints, at least 4 + 2 * batch * n_kv * ceil(cap / chunk_min)) what a
+ * forward with block size B, n_kv kv heads, grid chunk chunk_min (a positive
+ * multiple of 64) and `slots` resident CTAs would use: {chunk, n_items, -, -},
+ * the chunk in keys (a multiple of 64, at least chunk_min), then one pair per
+ * (request, kv head, chunk) with keys, {request << 16 | kv head << 8 | chunk
+ * index, the request's context length or 0 where req_valid is 0},
+ * request-major.  Enqueued on `stream`; DFLASH_EINVAL for null pointers,
+ * non-positive sizes, more than 255 kv heads or chunks, a bad chunk_min or a
+ * short or misaligned plan_out.  dflash_debug_attn_slots returns the resident CTAs of the
+ * grid kernel the draft would run for head_dim and `rows` query rows per kv
+ * head (contiguous K/V), or DFLASH_EINVAL.  Tests only. */
+int dflash_debug_attn_plan(const int32_t* ctx_len, const int32_t* req_valid, int batch, int B,
+                           int n_kv, int cap, int chunk_min, int slots, int32_t* plan_out,
+                           long long plan_cap, void* stream);
+int dflash_debug_attn_slots(int head_dim, int rows, int B);
+
 /* Split-KV chunk of the draft attention, in keys, for every later
- * dflash_draft_block call, process-wide: 0 = the library's rule (at least 512
- * keys, at most 64 chunks per request), else a multiple of 64 that is used
- * whenever it gives at most 64 chunks.  Returns DFLASH_EINVAL for a negative
+ * dflash_draft_block call, process-wide: 0 = the library's rule (bf16 models
+ * on the default schedule: a planning kernel picks each forward's chunk from
+ * the actual context lengths, at least the grid chunk of at most 64 chunks per
+ * request), else a multiple of 64 that is used, unplanned, whenever it gives
+ * at most 64 chunks.  Returns DFLASH_EINVAL for a negative
  * value or one that is not a multiple of 64.  Not thread-safe; tests only. */
 int dflash_debug_attn_chunk(int keys);
 
