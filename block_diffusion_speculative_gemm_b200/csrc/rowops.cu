@@ -46,6 +46,23 @@ __device__ __forceinline__ float4 sum_splits4(const float* part, int splits, siz
   return v;
 }
 
+// Once a warp has consumed its split sums, the partials are dead: the GEMM
+// kept them in L2 (evict-last stores) for this read, and a dirty line left
+// there costs a DRAM write when it is evicted later.  The lane whose 16-byte
+// unit starts a 128-byte line drops that line of every split without writing
+// it back (the next GEMM rewrites every partial it leaves).  Called by every
+// lane after the warp's last use of the values; lines that are not 128-byte
+// aligned are left alone.
+__device__ __forceinline__ void discard_splits(const float* part, int splits, size_t stride,
+                                               size_t idx) {
+  if ((idx & 31) != 0) return;
+  for (int s = 0; s < splits; ++s) {
+    const float* line = part + idx + (size_t)s * stride;
+    if ((reinterpret_cast<uintptr_t>(line) & 127) == 0)
+      asm volatile("discard.global.L2 [%0], 128;" ::"l"(line) : "memory");
+  }
+}
+
 // Stores four values; returns true when a value does not fit the element type
 // (an fp16 store of a value that rounds past the largest finite fp16, or NaN).
 template <typename T>
@@ -153,7 +170,14 @@ __global__ void __launch_bounds__(kRowThreads)
     }
     ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
   }
-  const float inv = rsqrtf(block_sum(ss, red) / d + eps);
+  const float inv = rsqrtf(block_sum(ss, red) / d + eps);  // every sum consumed
+  if (part != nullptr) {
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+      const int c = (threadIdx.x + i * kRowThreads) * 4;
+      if (c < d) discard_splits(part, splits, stride, (size_t)m * d + c);
+    }
+  }
   const int orow = out_row ? out_row[m] : m;
   if (orow < 0) return;
   bool bad = false;
@@ -240,15 +264,18 @@ __global__ void qkv_post_kernel(const float* __restrict__ part, int splits, int 
   const int nh = nq + 2 * nkv;
   const int N = nh * hd;
   const int p4 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;  // first of 4 pairs
-  if (p4 >= nh * half) return;
-  const int head = p4 / half, i = p4 % half;
+  const bool live = p4 < nh * half;
+  const int head = (live ? p4 : 0) / half, i = (live ? p4 : 0) % half;
   const int r = m / B, j = m % B;
   const int pos = (req_valid[r] ? ctx_len[r] : 0) + j;
   const size_t stride = (size_t)M * N;
   const size_t c0 = (size_t)m * N + head * hd + i;
-  float4 x1 = sum_splits4(part, splits, stride, c0);
-  float4 x2 = sum_splits4(part, splits, stride, c0 + half);
-  T* dst;
+  float4 x1 = make_float4(0.f, 0.f, 0.f, 0.f), x2 = x1;
+  if (live) {
+    x1 = sum_splits4(part, splits, stride, c0);
+    x2 = sum_splits4(part, splits, stride, c0 + half);
+  }
+  T* dst = q;
   if (head < nq + nkv) {
     const float4 c = *reinterpret_cast<const float4*>(cos_t + (size_t)pos * half + i);
     const float4 sn = *reinterpret_cast<const float4*>(sin_t + (size_t)pos * half + i);
@@ -262,9 +289,16 @@ __global__ void qkv_post_kernel(const float* __restrict__ part, int splits, int 
   } else {
     dst = vb + ((size_t)m * nkv + head - nq - nkv) * hd;
   }
-  const bool bad = store4<T>(dst + i, x1.x, x1.y, x1.z, x1.w) |
-                   store4<T>(dst + i + half, x2.x, x2.y, x2.z, x2.w);
-  if (bad) set_error(err, DFLASH_DEV_RANGE);
+  if (live) {
+    const bool bad = store4<T>(dst + i, x1.x, x1.y, x1.z, x1.w) |
+                     store4<T>(dst + i + half, x2.x, x2.y, x2.z, x2.w);
+    if (bad) set_error(err, DFLASH_DEV_RANGE);
+  }
+  __syncwarp();  // every lane's stores used its loads
+  if (live) {
+    discard_splits(part, splits, stride, c0);
+    discard_splits(part, splits, stride, c0 + half);
+  }
 }
 
 template <typename T>
@@ -289,15 +323,22 @@ __global__ void swiglu_kernel(const float* __restrict__ part, int splits, int M,
   pdl_wait();
   const int m = blockIdx.y;
   const int i = (blockIdx.x * blockDim.x + threadIdx.x) * 4;  // 4 features in one 64-block
-  if (i >= I) return;
+  const bool live = i < I;
   const size_t stride = (size_t)M * 2 * I;
-  const size_t gc = (size_t)m * 2 * I + (size_t)(i >> 6) * 128 + (i & 63);
-  const float4 g = sum_splits4(part, splits, stride, gc);
-  const float4 u = sum_splits4(part, splits, stride, gc + 64);
-  const bool bad = store4<T>(act + (size_t)m * I + i, g.x / (1.f + expf(-g.x)) * u.x,
-            g.y / (1.f + expf(-g.y)) * u.y, g.z / (1.f + expf(-g.z)) * u.z,
-            g.w / (1.f + expf(-g.w)) * u.w);
-  if (bad) set_error(err, DFLASH_DEV_RANGE);
+  const size_t gc = (size_t)m * 2 * I + (size_t)((live ? i : 0) >> 6) * 128 + ((live ? i : 0) & 63);
+  if (live) {
+    const float4 g = sum_splits4(part, splits, stride, gc);
+    const float4 u = sum_splits4(part, splits, stride, gc + 64);
+    const bool bad = store4<T>(act + (size_t)m * I + i, g.x / (1.f + expf(-g.x)) * u.x,
+                               g.y / (1.f + expf(-g.y)) * u.y, g.z / (1.f + expf(-g.z)) * u.z,
+                               g.w / (1.f + expf(-g.w)) * u.w);
+    if (bad) set_error(err, DFLASH_DEV_RANGE);
+  }
+  __syncwarp();  // every lane's stores used its loads
+  if (live) {
+    discard_splits(part, splits, stride, gc);
+    discard_splits(part, splits, stride, gc + 64);
+  }
 }
 
 template <typename T>
