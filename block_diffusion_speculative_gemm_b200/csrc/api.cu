@@ -255,7 +255,8 @@ int g_attn_chunk = 0;  // split-KV chunk override in keys (tests and tuning; 0 =
 // whose few tiles split 3-5 ways).
 int g_gemm_sched = 0;
 bool sk_projections() { return g_gemm_sched == 2; }
-// Draft attention schedule: 0 (default) the split-KV grid of fixed key chunks;
+// Draft attention schedule: 0 (default) the split-KV grid, its chunk planned on
+// the device per forward;
 // 1 persistent (every CTA the same number of key tiles, one TMA ring across
 // (request, head) segments), which measured 15% slower at the 8B batch of 32
 // (0.92-0.95 against 0.79-0.80 ms per draft): the SMs' idle time is not what

@@ -683,9 +683,9 @@ def debug_lmhead(W: torch.Tensor, X: torch.Tensor, err_ws: torch.Tensor, want_lo
 
 
 def debug_attn_schedule(sched: int) -> None:
-    """Process-wide draft attention schedule: 0 the split-KV grid of fixed
-    chunks (default), 1 persistent, 2 the split-KV grid on the tcgen05 kernel
-    where it applies (tests and tuning)."""
+    """Process-wide draft attention schedule: 0 the split-KV grid with its
+    chunk planned on the device (default), 1 persistent, 2 the split-KV grid on
+    the tcgen05 kernel where it applies (tests and tuning)."""
     _check("dflash_debug_attn_schedule", lib().dflash_debug_attn_schedule(int(sched)))
 
 

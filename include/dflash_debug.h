@@ -96,8 +96,8 @@ int dflash_debug_pick_splits(int M, int N, int K);
 int dflash_debug_split_weight(float w);
 
 /* Schedule of the draft attention (bf16 models) for every later call,
- * process-wide: 0 (default) the split-KV grid of fixed key chunks
- * (dflash_debug_attn_chunk) on the mma.sync kernel; 1 persistent (mma.sync),
+ * process-wide: 0 (default) the split-KV grid on the mma.sync kernel, its key
+ * chunk planned on the device per forward (or forced by dflash_debug_attn_chunk); 1 persistent (mma.sync),
  * two CTAs per SM each streaming the same number of 64-key tiles over the
  * (request, kv head) segments, segments split between CTAs merged by their
  * last piece; 2 the split-KV grid on the tcgen05 kernel where its shapes allow
