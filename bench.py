@@ -396,8 +396,10 @@ def run_dflash(args, rank, world, local_rank):
         "config": {"workload": cfg.name, "model": f"Qwen3-8B-shaped DFlash draft ({cfg.L} layers)",
                    "global_batch": b * world, "block": B, "denoise_steps": cfg.steps,
                    "ctx": "uniform[512,4096]", "inject_rows": n_s, "parallelism": f"dp{world}",
-                   "attention": ["split-KV grid, mma.sync", "persistent, mma.sync",
-                                 "split-KV grid, tcgen05"][args.attn_schedule],
+                   "attention": ["split-KV grid (chunk planned per forward), mma.sync",
+                                 "persistent, mma.sync",
+                                 "split-KV grid (chunk planned per forward), tcgen05"][
+                                     args.attn_schedule],
                    "l2": "no flush: every step streams ~7.4 GB of weights and K/V (> 126 MB L2)"},
         "roofline": roof,
         "tensor_peak": {"TFLOPs": tc_peak, "kind": tc_kind,
