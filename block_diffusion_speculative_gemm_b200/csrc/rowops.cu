@@ -407,7 +407,7 @@ __global__ void kv_scatter_kernel(const float* __restrict__ part, int splits, in
     x2 = y2;
   }
   const long long drow = kv_row(pg, l, batch, r, nkv, head, cap, pos);
-  const long long rows = (long long)L * nkv * (pg.table ? (long long)pg.n_pages * pg.page
+  [[maybe_unused]] const long long rows = (long long)L * nkv * (pg.table ? (long long)pg.n_pages * pg.page
                                                         : (long long)batch * cap);
   if (!DFLASH_CHECK(drow >= 0 && drow < rows, err)) return;
   T* dst = (is_v ? vc : kc) + (size_t)drow * hd;
