@@ -933,8 +933,7 @@ __global__ void __launch_bounds__(kPlanThreads)
 // Resident CTAs per SM of the split-KV grid kernel.
 template <int HD, int MT>
 int grid_ctas_per_sm() {
-  static int n = -1;
-  if (n < 0) {
+  static const int n = [] {  // thread-safe one-time initialisation
     const int smem = Layout<HD, MT>::kSmem;
     int v = 0;
     if (cudaFuncSetAttribute(attn_tc_kernel<HD, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -942,8 +941,8 @@ int grid_ctas_per_sm() {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, attn_tc_kernel<HD, MT>, kThreads,
                                                       smem) != cudaSuccess)
       v = 1;
-    n = std::max(1, v);
-  }
+    return std::max(1, v);
+  }();
   return n;
 }
 

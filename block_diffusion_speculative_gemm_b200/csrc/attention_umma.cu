@@ -510,16 +510,15 @@ __global__ void __launch_bounds__(kUThreads, 2)
 }  // namespace
 
 int attn_umma_ctas_per_sm() {
-  static int n = -1;
-  if (n < 0) {
+  static const int n = [] {  // thread-safe one-time initialisation
     int v = 0;
     if (cudaFuncSetAttribute(attn_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kUSmem) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, attn_umma_kernel, kUThreads, kUSmem) !=
             cudaSuccess)
       v = 1;
-    n = v > 0 ? v : 1;
-  }
+    return v > 0 ? v : 1;
+  }();
   return n;
 }
 
