@@ -191,6 +191,11 @@ int dflash_inject_kv(const dflash_model* m, const void* const* taps, const int32
  * token (ties to the lower token id).  B in [2, 16], n_steps in [1, B-1].
  * A request with ctx_len + B > cache_cap or an anchor outside [0, V) sets a
  * device error bit and writes nothing.
+ * The same inputs give the same bits on every call.  The attention splits each
+ * request's context into chunks sized from the whole batch's context lengths
+ * (planned on the device for bf16 models), so a request's logits can change at
+ * fp32 rounding level, and a near-tie token can flip, when the other requests
+ * of its batch change.
  */
 int dflash_draft_block(const dflash_model* m, const int32_t* anchor, const int32_t* ctx_len,
                        const void* k_cache, const void* v_cache, int cache_cap, int batch, int B,
