@@ -49,3 +49,26 @@ def test_test_hooks_reject_out_of_range_values(L):
     assert L.dflash_debug_gemm_mode(0) == 0
     assert L.dflash_debug_split_weight(ctypes.c_float(-1.0)) == D.EINVAL
     assert L.dflash_debug_split_weight(ctypes.c_float(4.0)) == 0
+
+
+def test_attention_plan_hook_validates_before_enqueueing(L):
+    # every rejection happens on the host, before anything touches the (fake)
+    # device pointers: a null pointer, sizes, a chunk that is not a positive
+    # multiple of 64, more than 255 chunks or kv heads, a short or misaligned plan
+    p = 4096  # never dereferenced on these paths
+    bad = [
+        (0, p, 4, 8, 8, 4096, 1024, 296, p, 4096),       # null ctx_len
+        (p, p, 0, 8, 8, 4096, 1024, 296, p, 4096),       # empty batch
+        (p, p, 4, 8, 256, 4096, 1024, 296, p, 4096),     # more than 255 kv heads
+        (p, p, 4, 8, 8, 4096, 1000, 296, p, 4096),       # chunk_min not a multiple of 64
+        (p, p, 4, 8, 8, 4096, 1024, 0, p, 4096),         # no resident slots
+        (p, p, 4, 8, 8, 32768, 64, 296, p, 1 << 20),     # 512 chunks a request
+        (p, p, 4, 8, 8, 4096, 1024, 296, p, 4 + 2 * 4 * 8 * 4 - 1),  # plan one int short
+        (p, p, 4, 8, 8, 4096, 1024, 296, p + 4, 4096),   # plan not 8-byte aligned
+        (p, p, 4, 8, 8, 4, 64, 296, p, 4096),            # cap below the block
+    ]
+    for ctx, valid, batch, B, nkv, cap, cmin, slots, out, n in bad:
+        assert L.dflash_debug_attn_plan(ctx, valid, batch, B, nkv, cap, cmin, slots, out, n,
+                                        None) == D.EINVAL
+    assert L.dflash_debug_attn_slots(0, 32, 8) == D.EINVAL
+    assert L.dflash_debug_attn_slots(128, 32, 0) == D.EINVAL
